@@ -1,0 +1,201 @@
+/*
+ * moe.h - C ABI of libmoe.so: the single-GPU forward pass of a sparsely-gated
+ * Mixture-of-Experts layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer (Shazeer et al., "Outrageously Large Neural Networks: The Sparsely-Gated
+ * Mixture-of-Experts Layer", section "Methode"): y = sum_i G(x)_i E_i(x), where the
+ * experts E_i are feed-forward sub-networks and G is a sparse gate that is zero for all
+ * but k experts, so only k experts run per token.  The forward pass has five steps:
+ *
+ *   moe_route      router product x.W_g fused with the gate (softmax top-k, or noisy
+ *                  top-k) -> chosen experts and their gate values per token
+ *   moe_permute    per-expert histogram, scan, capacity truncation and a stable counting
+ *                  sort of the token->expert assignments; gathers the kept token rows
+ *   moe_expert_ffn per-expert FFN on the kept rows only (grouped GEMM, tensor cores)
+ *   moe_combine    gate-weighted sum of each token's expert outputs (un-permute)
+ *   moe_forward    all of the above on one stream
+ *
+ * Conventions for every call
+ *  - All pointers are DEVICE pointers unless stated, owned by the caller, and must
+ *    stay valid until the work queued on `stream` has finished.  The library never
+ *    allocates, frees or synchronises, except moe_get_error (which synchronises).
+ *  - Work is queued asynchronously on `stream` (NULL = the legacy default stream) on
+ *    the current CUDA device.  A call returns once its kernels are queued.
+ *  - Arguments are validated on the host before any launch; a bad argument returns
+ *    MOE_ERR_INVALID_ARG or MOE_ERR_UNSUPPORTED and queues nothing.  A failed launch
+ *    returns MOE_ERR_CUDA.  Problems only visible on the device (an expert index out of
+ *    range, inconsistent offsets, an expired bounded wait) set bits of the device error
+ *    word held in the workspace; read and clear them with moe_get_error.
+ *  - Layouts are row-major and contiguous.  Weight matrices are stored K-major (one row
+ *    per output feature, contiguous along the contraction): the pages write x.W_g with
+ *    W_g as [d_model, E]; w_gate here is its transpose [E, d_model].
+ *  - Index tensors are int32.  Assignment a = t*k + j is token t's j-th choice.
+ *  - Floating-point tensors of the layer (x, weights, x_perm, h, y_perm, y) are in
+ *    cfg->dtype; gates, noise, logit_bias, importance and load are always fp32.
+ *  - T == 0 is valid: nothing is launched, the per-expert outputs that are given
+ *    (counts, offsets, importance, load) are zero-filled on `stream`, and per-token
+ *    pointers may be NULL.
+ *  - The workspace `ws` is a device buffer of at least moe_workspace_size() bytes (or
+ *    moe_forward_workspace_size() for moe_forward), 256-byte aligned, zero-filled once
+ *    by the caller before first use (it holds the sticky device error word).  Calls that
+ *    share one workspace must be ordered on one stream.
+ *
+ * Supported shapes: bf16 needs d_model and d_ff multiples of 64 and E <= 256; fp32
+ * needs d_model and d_ff multiples of 4; all need 1 <= k <= min(E, 8), d_model % 8 == 0
+ * and T*k < 2^31.  Outside these the call returns MOE_ERR_UNSUPPORTED.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t); NULL selects the legacy default stream. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, bad size or enum, misaligned pointer */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid but outside the supported shapes/dtypes */
+  MOE_ERR_CUDA = 3,         /* a CUDA runtime/driver call or kernel launch failed */
+  MOE_ERR_DEVICE = 4        /* moe_get_error found device error bits set */
+} moe_status;
+
+/* Bits of the device error word (see moe_get_error). */
+enum {
+  MOE_DEVERR_EXPERT_INDEX = 1, /* a topk_idx entry outside [0, E): treated as dropped */
+  MOE_DEVERR_OFFSETS = 2,      /* offsets not non-decreasing in [0, T*k]: FFN skipped */
+  MOE_DEVERR_SLOT = 4,         /* a slot_pos entry outside [-1, T*k): treated as dropped */
+  MOE_DEVERR_TIMEOUT = 8       /* a bounded wait inside a pipelined kernel expired */
+};
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Gating rule.
+ * MOE_GATE_SOFTMAX_TOPK: scores l = x.W_g (+ logit_bias); the k largest are chosen.
+ *   renorm = 1: gates = Softmax(KeepTopK(l, k)) (Shazeer et al., "Noisy Top-K Gating",
+ *               without noise); renorm = 0: each chosen expert's gate is its probability
+ *               under the softmax over all E experts (the Switch Transformer top-1 rule).
+ * MOE_GATE_NOISY_TOPK: H = x.W_g (+ logit_bias) + noise * Softplus(x.W_noise), the k
+ *   largest of H are chosen and gates = Softmax(KeepTopK(H, k)) (Shazeer et al.,
+ *   "Noisy Top-K Gating"; renorm is ignored).  `noise` holds the StandardNormal() draws.
+ * Ties go to the lowest expert index; chosen experts are listed largest score first. */
+typedef enum { MOE_GATE_SOFTMAX_TOPK = 0, MOE_GATE_NOISY_TOPK = 1 } moe_gating;
+
+/* Expert activation: ReLU, or GELU in its exact form 0.5 z (1 + erf(z / sqrt 2)). */
+typedef enum { MOE_ACT_RELU = 0, MOE_ACT_GELU = 1 } moe_act;
+
+typedef struct {
+  int64_t T;              /* tokens */
+  int32_t d_model;        /* model width d */
+  int32_t d_ff;           /* expert hidden width f */
+  int32_t E;              /* experts */
+  int32_t k;              /* experts per token */
+  int32_t gating;         /* moe_gating */
+  int32_t renorm;         /* see moe_gating */
+  float capacity_factor;  /* > 0: capacity C = ceil(cf*T*k/E) per expert; <= 0: none */
+  int32_t act;            /* moe_act */
+  int32_t dtype;          /* moe_dtype of the layer tensors */
+} moe_config;
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(moe_status s);
+
+/* Capacity C = ceil(cf * T * k / E), computed exactly from the fp32 value of cf
+ * (capacity factors as in the setups table of the "moe paper models" page), or -1 when
+ * cfg->capacity_factor <= 0 (no limit).  Returns -2 for an invalid cfg. */
+int64_t moe_capacity(const moe_config* cfg);
+
+/* Bytes of workspace the step calls (moe_route ... moe_combine) need; 0 for an invalid
+ * or unsupported cfg. */
+size_t moe_workspace_size(const moe_config* cfg);
+
+/* Bytes of workspace moe_forward needs: the step workspace plus the intermediates
+ * (offsets, slot_pos, perm_src, x_perm, h, y_perm) it keeps there. */
+size_t moe_forward_workspace_size(const moe_config* cfg);
+
+/* Router product and gate [Shazeer et al., "Noisy Top-K Gating"; Switch Transformer,
+ * switch_routing].
+ *  x          [T, d_model] dtype
+ *  w_gate     [E, d_model] dtype (W_g transposed)
+ *  w_noise    [E, d_model] dtype, required for noisy gating, else ignored (may be NULL)
+ *  noise      [T, E] fp32 StandardNormal draws, required for noisy gating
+ *  logit_bias [E] fp32 added to the clean logits, or NULL
+ *  topk_idx   [T, k] int32 out: chosen experts, largest score first
+ *  topk_gate  [T, k] fp32 out: their gates
+ *  importance [E] fp32 out or NULL: Importance(X) = sum_t G(x_t) ("Load-Balancing-Losses")
+ *  load       [E] fp32 out or NULL: Load(X)_i = sum_t P(x_t, i) with
+ *             P(x,i) = Phi(((x.W_g)_i - kth_excluding(H,k,i)) / Softplus((x.W_noise)_i));
+ *             noisy gating with k < E only
+ *  near_tie   [T] uint8 out or NULL: 1 where the k-th and (k+1)-th scores differ by at
+ *             most 1e-4 (there two top-k choices are both correct up to rounding)
+ * The scores are accumulated in fp32 (bf16 inputs: exact bf16 products, fp32 sums). */
+moe_status moe_route(const moe_config* cfg, const void* x, const void* w_gate,
+                     const void* w_noise, const float* noise, const float* logit_bias,
+                     int32_t* topk_idx, float* topk_gate, float* importance, float* load,
+                     uint8_t* near_tie, void* ws, moe_stream_t stream);
+
+/* Capacity truncation and stable permutation by expert [Switch Transformer,
+ * switch_routing: dispatch is a gather of each expert's tokens].
+ *  topk_idx [T, k] int32 in
+ *  x        [T, d_model] dtype in
+ *  counts   [E] int32 out: assignments per expert before the capacity drop
+ *  offsets  [E+1] int32 out: expert e's kept rows are x_perm[offsets[e] : offsets[e+1]]
+ *  perm_src [T*k] int32 out: perm_src[s] = assignment a held by permuted row s
+ *           (entries at s >= offsets[E] are left untouched)
+ *  slot_pos [T*k] int32 out: permuted row of assignment a, or -1 if dropped
+ *  x_perm   [T*k, d_model] dtype out: x_perm[s] = x[perm_src[s] / k]
+ * Within an expert rows keep ascending a; the first C are kept (C = moe_capacity). */
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* x,
+                       int32_t* counts, int32_t* offsets, int32_t* perm_src,
+                       int32_t* slot_pos, void* x_perm, void* ws, moe_stream_t stream);
+
+/* Per-expert FFN on the kept rows [Shazeer et al.: experts are feed-forward networks;
+ * computation is skipped where G(x)_i = 0]:
+ *   h[s] = act(x_perm[s] . W1_e^T),  y_perm[s] = h[s] . W2_e^T  for offsets[e] <= s < offsets[e+1]
+ *  x_perm  [T*k, d_model] dtype in (rows >= offsets[E] are never read into outputs)
+ *  offsets [E+1] int32 in (as written by moe_permute; any non-decreasing values in
+ *          [0, T*k] are accepted)
+ *  w1      [E, d_ff, d_model] dtype,  w2 [E, d_model, d_ff] dtype
+ *  h       [T*k, d_ff] dtype out (hidden activations; rows < offsets[E] written)
+ *  y_perm  [T*k, d_model] dtype out (rows < offsets[E] written)
+ * bf16: tcgen05 tensor cores with fp32 accumulation; h and y_perm are rounded to bf16. */
+moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
+                          const void* w1, const void* w2, void* h, void* y_perm, void* ws,
+                          moe_stream_t stream);
+
+/* Gate-weighted combine [Shazeer et al., "Methode": y = sum_i G(x)_i E_i(x)]:
+ *   y[t] = sum_j topk_gate[t, j] * y_perm[slot_pos[t*k + j]]   (dropped slots add 0)
+ *  y_perm [T*k, d_model] dtype, slot_pos [T*k] int32, topk_gate [T, k] fp32 in
+ *  y      [T, d_model] dtype out; fp32 accumulation, one rounding to dtype. */
+moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* slot_pos,
+                       const float* topk_gate, void* y, void* ws, moe_stream_t stream);
+
+/* The whole layer forward on one stream: moe_route, moe_permute, moe_expert_ffn,
+ * moe_combine.  Inputs as in the step calls; y [T, d_model] dtype out.  topk_idx,
+ * topk_gate (both [T, k]) and counts ([E]) are outputs the caller must provide;
+ * importance, load and near_tie may be NULL.  The intermediates live in `ws`
+ * (moe_forward_workspace_size bytes). */
+moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_gate,
+                       const void* w_noise, const float* noise, const float* logit_bias,
+                       const void* w1, const void* w2, void* y, int32_t* topk_idx,
+                       float* topk_gate, int32_t* counts, float* importance, float* load,
+                       uint8_t* near_tie, void* ws, moe_stream_t stream);
+
+/* Synchronises `stream`, then reads the device error word in `ws` into *device_error
+ * (may be NULL) and clears it.  Returns MOE_OK if no bit was set, MOE_ERR_DEVICE if
+ * some were, MOE_ERR_CUDA if the synchronisation or copy failed. */
+moe_status moe_get_error(void* ws, moe_stream_t stream, int32_t* device_error);
+
+/* Number of kernels the most recent successful call on this host thread queued. */
+int32_t moe_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

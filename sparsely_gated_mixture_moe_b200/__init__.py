@@ -1,0 +1,190 @@
+"""Python binding of libmoe: the sparsely-gated Mixture-of-Experts layer forward on B200.
+
+A thin ctypes layer over the C ABI in include/moe.h.  Every step of the layer runs in
+the library's CUDA kernels; this module only marshals arguments (device pointers of
+torch tensors, the stream handle, the config struct) and turns status codes into
+exceptions.  There is no CPU fallback: importing fails loudly when libmoe.so has not
+been built, and every call requires CUDA tensors.
+
+    python -m sparsely_gated_mixture_moe_b200.build_lib      # build libmoe.so in-tree
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from .config import (ACT, DTYPE, GATING, MoEConfig, MoEError, STATUS, make_config)
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            "libmoe.so is not built (expected at %s); build it with "
+            "`python -m sparsely_gated_mixture_moe_b200.build_lib`" % _LIB_PATH)
+    lib = ctypes.CDLL(_LIB_PATH)
+    P = ctypes.c_void_p
+    C = ctypes.POINTER(MoEConfig)
+    sig = {
+        "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "moe_capacity": (ctypes.c_int64, [C]),
+        "moe_workspace_size": (ctypes.c_size_t, [C]),
+        "moe_forward_workspace_size": (ctypes.c_size_t, [C]),
+        "moe_route": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P, P]),
+        "moe_permute": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P]),
+        "moe_expert_ffn": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
+        "moe_combine": (ctypes.c_int, [C, P, P, P, P, P, P]),
+        "moe_forward": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]),
+        "moe_get_error": (ctypes.c_int, [P, P, ctypes.POINTER(ctypes.c_int32)]),
+        "moe_last_launch_count": (ctypes.c_int32, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+LIB_PATH = _LIB_PATH
+
+
+def _ptr(t: Optional[torch.Tensor], what: str):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % what)
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor (libmoe has no CPU path)" % what)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % what)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise MoEError(status, "%s: %s" % (what, lib.moe_status_string(status).decode()))
+
+
+def moe_capacity(cfg: MoEConfig) -> int:
+    """C = ceil(cf*T*k/E) computed by the library (-1: no limit)."""
+    return int(lib.moe_capacity(ctypes.byref(cfg)))
+
+
+def moe_workspace_size(cfg: MoEConfig) -> int:
+    return int(lib.moe_workspace_size(ctypes.byref(cfg)))
+
+
+def moe_forward_workspace_size(cfg: MoEConfig) -> int:
+    return int(lib.moe_forward_workspace_size(ctypes.byref(cfg)))
+
+
+def workspace(cfg: MoEConfig, device="cuda", forward: bool = False) -> torch.Tensor:
+    """A zero-filled device workspace of the size the library asks for."""
+    n = moe_forward_workspace_size(cfg) if forward else moe_workspace_size(cfg)
+    if n == 0:
+        raise MoEError(2, "config is invalid or unsupported")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def moe_route(cfg, x, w_gate, topk_idx, topk_gate, ws, w_noise=None, noise=None,
+              logit_bias=None, importance=None, load=None, near_tie=None, stream=None):
+    _check(lib.moe_route(ctypes.byref(cfg), _ptr(x, "x"), _ptr(w_gate, "w_gate"),
+                         _ptr(w_noise, "w_noise"), _ptr(noise, "noise"),
+                         _ptr(logit_bias, "logit_bias"), _ptr(topk_idx, "topk_idx"),
+                         _ptr(topk_gate, "topk_gate"), _ptr(importance, "importance"),
+                         _ptr(load, "load"), _ptr(near_tie, "near_tie"), _ptr(ws, "ws"),
+                         _stream(stream)), "moe_route")
+
+
+def moe_permute(cfg, topk_idx, x, counts, offsets, perm_src, slot_pos, x_perm, ws, stream=None):
+    _check(lib.moe_permute(ctypes.byref(cfg), _ptr(topk_idx, "topk_idx"), _ptr(x, "x"),
+                           _ptr(counts, "counts"), _ptr(offsets, "offsets"),
+                           _ptr(perm_src, "perm_src"), _ptr(slot_pos, "slot_pos"),
+                           _ptr(x_perm, "x_perm"), _ptr(ws, "ws"), _stream(stream)),
+           "moe_permute")
+
+
+def moe_expert_ffn(cfg, x_perm, offsets, w1, w2, h, y_perm, ws, stream=None):
+    _check(lib.moe_expert_ffn(ctypes.byref(cfg), _ptr(x_perm, "x_perm"), _ptr(offsets, "offsets"),
+                              _ptr(w1, "w1"), _ptr(w2, "w2"), _ptr(h, "h"),
+                              _ptr(y_perm, "y_perm"), _ptr(ws, "ws"), _stream(stream)),
+           "moe_expert_ffn")
+
+
+def moe_combine(cfg, y_perm, slot_pos, topk_gate, y, ws, stream=None):
+    _check(lib.moe_combine(ctypes.byref(cfg), _ptr(y_perm, "y_perm"), _ptr(slot_pos, "slot_pos"),
+                           _ptr(topk_gate, "topk_gate"), _ptr(y, "y"), _ptr(ws, "ws"),
+                           _stream(stream)), "moe_combine")
+
+
+def moe_forward(cfg, x, w_gate, w1, w2, y, topk_idx, topk_gate, counts, ws, w_noise=None,
+                noise=None, logit_bias=None, importance=None, load=None, near_tie=None,
+                stream=None):
+    _check(lib.moe_forward(ctypes.byref(cfg), _ptr(x, "x"), _ptr(w_gate, "w_gate"),
+                           _ptr(w_noise, "w_noise"), _ptr(noise, "noise"),
+                           _ptr(logit_bias, "logit_bias"), _ptr(w1, "w1"), _ptr(w2, "w2"),
+                           _ptr(y, "y"), _ptr(topk_idx, "topk_idx"), _ptr(topk_gate, "topk_gate"),
+                           _ptr(counts, "counts"), _ptr(importance, "importance"),
+                           _ptr(load, "load"), _ptr(near_tie, "near_tie"), _ptr(ws, "ws"),
+                           _stream(stream)), "moe_forward")
+
+
+def moe_get_error(ws: torch.Tensor, stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error word."""
+    v = ctypes.c_int32(0)
+    st = lib.moe_get_error(_ptr(ws, "ws"), _stream(stream), ctypes.byref(v))
+    if st not in (0, 4):
+        _check(st, "moe_get_error")
+    return int(v.value)
+
+
+def last_launch_count() -> int:
+    """Kernels queued by the most recent successful call on this thread."""
+    return int(lib.moe_last_launch_count())
+
+
+class MoELayer:
+    """Owns the device buffers of one layer configuration and runs its forward pass.
+
+    weights: dict with w_gate [E,d], w1 [E,f,d], w2 [E,d,f] (and w_noise [E,d] for noisy
+    gating, logit_bias [E] fp32 if used), CUDA tensors in the config's dtype.
+    """
+
+    def __init__(self, cfg: MoEConfig, weights: dict, device="cuda"):
+        self.cfg = cfg
+        self.w = weights
+        T, k, E, d = cfg.T, cfg.k, cfg.E, cfg.d_model
+        dt = torch.float32 if cfg.dtype == DTYPE["f32"] else torch.bfloat16
+        self.y = torch.empty(T, d, dtype=dt, device=device)
+        self.topk_idx = torch.empty(T, k, dtype=torch.int32, device=device)
+        self.topk_gate = torch.empty(T, k, dtype=torch.float32, device=device)
+        self.counts = torch.empty(E, dtype=torch.int32, device=device)
+        noisy = cfg.gating == GATING["noisy_topk"]
+        self.importance = torch.empty(E, dtype=torch.float32, device=device) if noisy else None
+        self.load = torch.empty(E, dtype=torch.float32, device=device) if noisy and k < E else None
+        self.near_tie = torch.empty(T, dtype=torch.uint8, device=device)
+        self.ws = workspace(cfg, device, forward=True)
+
+    def forward(self, x: torch.Tensor, noise: Optional[torch.Tensor] = None, stream=None):
+        w = self.w
+        moe_forward(self.cfg, x, w["w_gate"], w["w1"], w["w2"], self.y, self.topk_idx,
+                    self.topk_gate, self.counts, self.ws, w_noise=w.get("w_noise"), noise=noise,
+                    logit_bias=w.get("logit_bias"), importance=self.importance, load=self.load,
+                    near_tie=self.near_tie, stream=stream)
+        return self.y
+
+
+__all__ = ["ACT", "DTYPE", "GATING", "MoEConfig", "MoEError", "MoELayer", "STATUS", "lib",
+           "make_config", "moe_capacity", "moe_combine", "moe_expert_ffn", "moe_forward",
+           "moe_forward_workspace_size", "moe_get_error", "moe_permute", "moe_route",
+           "moe_workspace_size", "workspace", "last_launch_count"]

@@ -1,0 +1,106 @@
+// Gate-weighted combine (un-permute): y[t] = sum_j G_{t,j} * y_perm[slot_pos[t*k + j]].
+//
+// The layer output of Shazeer et al. ("Methode"): y = sum_i G(x)_i E_i(x), with only the
+// k chosen experts contributing and a dropped assignment (slot_pos = -1) adding nothing.
+// One warp per token; each lane handles 16-byte vectors of the row (8 bf16 or 4 fp32),
+// gathers the k expert rows, accumulates in fp32 and rounds once to the output dtype.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+template <typename T>
+struct Vec;
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ static void load(const void* p, float (&v)[4]) {
+    const float4 u = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+  }
+  __device__ static void store(void* p, const float (&v)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void load(const void* p, float (&v)[8]) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
+      const float2 f = __bfloat1622float2(b);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  }
+  __device__ static void store(void* p, const float (&v)[8]) {
+    *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+  }
+};
+
+constexpr int kCombineWarps = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(kCombineWarps * 32)
+    combine_kernel(const T* __restrict__ y_perm, const int32_t* __restrict__ slot_pos,
+                   const float* __restrict__ gate, T* __restrict__ y, int64_t T_, int k, int d,
+                   int* err) {
+  constexpr int V = Vec<T>::N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kCombineWarps + warp;
+  if (t >= T_) return;
+  const int64_t nrows = T_ * k;
+  int slot[8];
+  float g[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    slot[j] = -1;
+    g[j] = 0.0f;
+    if (j < k) {
+      const int s = slot_pos[t * k + j];
+      if (s >= 0 && s < nrows) {
+        slot[j] = s;
+        g[j] = gate[t * k + j];
+      } else if (s != -1 && lane == 0) {
+        set_error(err, kErrSlot);
+      }
+    }
+  }
+  const int nv = d / V;
+  for (int v = lane; v < nv; v += 32) {
+    float acc[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[i] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (slot[j] >= 0) {
+        float r[V];
+        Vec<T>::load(y_perm + static_cast<int64_t>(slot[j]) * d + v * V, r);
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] = fmaf(g[j], r[i], acc[i]);
+      }
+    }
+    Vec<T>::store(y + t * d + v * V, acc);
+  }
+}
+
+cudaError_t launch_combine(const CombineProblem& p, const LaunchCtx& c) {
+  const int64_t blocks = (p.T + kCombineWarps - 1) / kCombineWarps;
+  if (blocks == 0) return cudaSuccess;
+  if (p.dtype == MOE_BF16)
+    combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), kCombineWarps * 32, 0, c.stream>>>(
+        static_cast<const __nv_bfloat16*>(p.y_perm), p.slot_pos, p.gate,
+        static_cast<__nv_bfloat16*>(p.y), p.T, p.k, p.d, c.err);
+  else
+    combine_kernel<float><<<static_cast<unsigned>(blocks), kCombineWarps * 32, 0, c.stream>>>(
+        static_cast<const float*>(p.y_perm), p.slot_pos, p.gate, static_cast<float*>(p.y), p.T,
+        p.k, p.d, c.err);
+  ++*c.launches;
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,340 @@
+// Per-expert FFN on the kept rows as a grouped GEMM on the 5th-generation tensor cores.
+//
+//   up:   h[s]      = act(x_perm[s] . W1_e^T)     [rows of e] x [d_ff, d_model]^T
+//   down: y_perm[s] = h[s] . W2_e^T               [rows of e] x [d_model, d_ff]^T
+//
+// Experts are the feed-forward sub-networks of the sparsely-gated MoE layer (Shazeer et
+// al., "Schlüsselbegriffe"); each runs only on the rows routed to it ("Methode": no
+// computation where G(x)_i = 0).  Expert e owns permuted rows [offsets[e], offsets[e+1]).
+//
+// Kernel design (one CTA per SM, persistent):
+//   warp 0      TMA producer: A tile [128 x 64] and B tile [BN x 64] per k-block into a
+//               4-stage ring of 128-byte-swizzled shared-memory buffers.
+//   warp 1      TMEM owner and MMA issuer: one thread issues tcgen05.mma (M=128, N=BN,
+//               K=16) into one of two TMEM accumulators (2 x 256 fp32 columns), and
+//               tcgen05.commit releases smem stages and hands finished accumulators on.
+//   warps 2-9   epilogue: tcgen05.ld of the accumulator (each warp reads its 32-lane
+//               quarter, half of the columns), activation, bf16 rounding, stores of the
+//               rows that belong to the expert (a ragged tail is masked).
+// Tiles are (expert, n-tile, m-tile) with m innermost, so CTAs running at the same time
+// share weight tiles through L2 and each expert's weights stream from HBM about once.
+// Rows past an expert's end that a 128-row tile reads belong to the next expert or lie
+// past the buffer (TMA fills those with zeros); they only feed masked output rows.
+// No cross-CTA waits; every mbarrier wait is bounded and an expired wait sets
+// kErrTimeout, drains this CTA's in-flight copies and MMAs and frees TMEM.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace gg {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + EPI_WARPS * 32;
+constexpr int A_BYTES = BM * BK * 2;        // 16 KB
+constexpr int B_BYTES_MAX = 256 * BK * 2;   // 32 KB
+constexpr int MAX_GROUPS = 1024;
+constexpr int TMEM_COLS = 512;              // two accumulators of up to 256 columns
+constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_BYTES + B_BYTES_MAX) +
+                           256 /*barriers, flags*/ + 4 * (MAX_GROUPS + 1 + 40);
+
+struct Args {
+  const int32_t* offsets;
+  int E;
+  int N;         // output columns (d_ff for up, d_model for down)
+  int K;         // contraction (d_model for up, d_ff for down)
+  int bn;        // N tile: 256, 128 or 64 (divides N)
+  int n_tiles;   // N / bn
+  int64_t rows_cap;
+  __nv_bfloat16* out;
+  int act;       // 0 none, 1 ReLU, 2 GELU
+  int* err;
+};
+
+struct Tile {
+  int e, mt, nt, row0, valid;
+};
+
+__device__ __forceinline__ Tile decode_tile(int L, const int* tp, const Args& a) {
+  // expert: the largest e with tp[e] * n_tiles <= L
+  int lo = 0, hi = a.E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tp[mid] * a.n_tiles <= L) lo = mid; else hi = mid - 1;
+  }
+  Tile t;
+  t.e = lo;
+  const int mte = tp[lo + 1] - tp[lo];
+  const int local = L - tp[lo] * a.n_tiles;
+  t.nt = local / mte;
+  t.mt = local - t.nt * mte;
+  const int r0 = __ldg(a.offsets + lo), r1 = __ldg(a.offsets + lo + 1);
+  t.row0 = r0 + t.mt * BM;
+  t.valid = min(BM, r1 - t.row0);
+  return t;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
+                           const __grid_constant__ CUtensorMap tmB, const Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES_MAX);
+  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
+  const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
+  const uint32_t drain = smem_u32(bars + 2 * STAGES + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* scratch = reinterpret_cast<int*>(smem + STAGES * (A_BYTES + B_BYTES_MAX) + 256);
+  int* tp = scratch + 40;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  const bool ok = block_tile_prefix(a.offsets, a.E, a.rows_cap, BM, tp, scratch);
+  if (!ok && threadIdx.x == 0) set_error(a.err, kErrOffsets);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int total = ok ? tp[a.E] * a.n_tiles : 0;
+  const int kblocks = a.K / BK;
+  const uint32_t b_bytes = static_cast<uint32_t>(a.bn) * BK * 2;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_par = 0;
+      bool aborted = false;
+      for (int L = blockIdx.x; L < total && !aborted; L += gridDim.x) {
+        const Tile t = decode_tile(L, tp, a);
+        const int brow = t.e * a.N + t.nt * a.bn;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, s_abort)) {
+            aborted = true;
+            break;
+          }
+          mbar_arrive_expect_tx(full0 + 8 * stage, A_BYTES + b_bytes);
+          tma_load_2d(smem_u32(sA + stage * A_BYTES), &tmA, full0 + 8 * stage, kb * BK, t.row0);
+          tma_load_2d(smem_u32(sB + stage * B_BYTES_MAX), &tmB, full0 + 8 * stage, kb * BK, brow);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (aborted) {
+        set_error(a.err, kErrTimeout);
+        *s_abort = 1;
+        // let every copy this thread started land before the CTA releases its smem
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s)) mbar_wait(full0 + 8 * s, (armed_par >> s) & 1, nullptr, kDrainLimitNs);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      const uint32_t idesc = idesc_bf16_f32(BM, a.bn);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool aborted = false;
+      for (int L = blockIdx.x; L < total && !aborted; L += gridDim.x) {
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1, s_abort)) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, s_abort)) {
+            aborted = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * B_BYTES_MAX);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_bf16(d_tmem, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32), idesc,
+                        (kb | kk) != 0 ? 1u : 0u);
+          tc_commit(empty0 + 8 * stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (aborted) break;
+        tc_commit(tfull0 + 8 * acc);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      if (aborted) {
+        set_error(a.err, kErrTimeout);
+        *s_abort = 1;
+        tc_commit(drain);  // wait for the MMAs already issued before TMEM is freed
+        mbar_wait(drain, 0, nullptr, kDrainLimitNs);
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;                // TMEM lane quarter this warp may read
+    const int half = (warp - 2) >> 2;      // which half of the tile's columns
+    const int cols = a.bn >> 1;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x) {
+      const Tile t = decode_tile(L, tp, a);
+      if (!mbar_wait(tfull0 + 8 * acc, acc_phase, s_abort)) {
+        if (lane == 0) set_error(a.err, kErrTimeout);
+        *s_abort = 1;
+        break;
+      }
+      tc_fence_after();
+      const int r = q * 32 + lane;
+      const bool row_ok = r < t.valid;
+      __nv_bfloat16* orow =
+          a.out + static_cast<int64_t>(t.row0 + r) * a.N + t.nt * a.bn + half * cols;
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256 + half * cols;
+      for (int c = 0; c < cols; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tbase + c, v);
+        tmem_ld_wait();
+        if (row_ok) {
+          uint32_t packed[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            packed[j] = pack_bf16x2(apply_act(__uint_as_float(v[2 * j]), a.act),
+                                    apply_act(__uint_as_float(v[2 * j + 1]), a.act));
+          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
+                                packed[4 * j + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+}  // namespace gg
+
+// ------------------------------------------------------------------- host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows) {
+  auto encode = get_encode_fn();
+  if (encode == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static int pick_bn(int N) {
+  if (N % 256 == 0) return 256;
+  if (N % 128 == 0) return 128;
+  return 64;
+}
+
+static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void* B, int E, int N,
+                              void* out, const int32_t* offsets, int act, const LaunchCtx& c) {
+  const int bn = pick_bn(N);
+  CUtensorMap tmA, tmB;
+  if (!make_tmap_bf16(&tmA, A, static_cast<uint64_t>(rows_cap), K, gg::BM)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16(&tmB, B, static_cast<uint64_t>(E) * N, K, bn)) return cudaErrorInvalidValue;
+  gg::Args a;
+  a.offsets = offsets;
+  a.E = E;
+  a.N = N;
+  a.K = K;
+  a.bn = bn;
+  a.n_tiles = N / bn;
+  a.rows_cap = rows_cap;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.act = act;
+  a.err = c.err;
+  // upper bound of the tile count: sum_e ceil(n_e / BM) <= rows_cap / BM + E
+  const int64_t max_tiles = (rows_cap / gg::BM + E) * static_cast<int64_t>(a.n_tiles);
+  const int grid = static_cast<int>(max_tiles < c.num_sms ? max_tiles : c.num_sms);
+  if (grid <= 0) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(gg::grouped_gemm_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, gg::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  gg::grouped_gemm_tc_kernel<<<grid, gg::THREADS, gg::SMEM_BYTES, c.stream>>>(tmA, tmB, a);
+  ++*c.launches;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c) {
+  if (p.E > gg::MAX_GROUPS) return cudaErrorInvalidValue;
+  cudaError_t e = launch_one(p.x_perm, p.rows_cap, p.d, p.w1, p.E, p.f, p.h, p.offsets, p.act, c);
+  if (e != cudaSuccess) return e;
+  return launch_one(p.h, p.rows_cap, p.f, p.w2, p.E, p.d, p.y_perm, p.offsets, 0, c);
+}
+
+}  // namespace moe

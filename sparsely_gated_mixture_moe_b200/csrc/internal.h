@@ -1,0 +1,100 @@
+// Host-side launchers shared by the translation units of libmoe.  Each launcher queues
+// its kernels on `stream`, adds the number of launches to *launches and returns the
+// CUDA error of the last launch (cudaSuccess on success).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+struct LaunchCtx {
+  cudaStream_t stream;
+  int num_sms;
+  int* err;       // device error word
+  int* launches;  // host counter
+};
+
+// ---- route -----------------------------------------------------------------------
+struct RouteProblem {
+  int64_t T;
+  int d, E, k;
+  int noisy, renorm;
+  const void* x;
+  const void* w_gate;
+  const void* w_noise;
+  const float* noise;
+  const float* bias;
+  int32_t* topk_idx;
+  float* topk_gate;
+  uint8_t* near_tie;
+  float* importance;  // may be null
+  float* load;        // may be null
+  float* partials;    // workspace: [route_blocks][2][E]
+  float* logits_ws;   // fp32 path only: [T][E]
+  float* nz_ws;       // fp32 path only: [T][E]
+};
+int route_blocks(int64_t T);
+cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c);
+cudaError_t launch_route_f32(const RouteProblem& p, const LaunchCtx& c);
+
+// ---- permute ---------------------------------------------------------------------
+constexpr int kPermChunk = 2048;  // assignments per permute block
+struct PermuteProblem {
+  int64_t n;  // T*k assignments
+  int k, E, d, esize;
+  int64_t C;  // capacity, < 0: none
+  const int32_t* topk_idx;
+  const void* x;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm_src;
+  int32_t* slot_pos;
+  void* x_perm;
+  int32_t* blk;  // workspace [nblk][E]
+};
+int64_t permute_blocks(int64_t n);
+cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c);
+
+// ---- expert FFN ------------------------------------------------------------------
+struct FfnProblem {
+  int64_t rows_cap;  // T*k
+  int d, f, E, act;  // act: 1 ReLU, 2 GELU
+  const void* x_perm;
+  const int32_t* offsets;
+  const void* w1;
+  const void* w2;
+  void* h;
+  void* y_perm;
+};
+cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c);
+cudaError_t launch_ffn_f32(const FfnProblem& p, const LaunchCtx& c);
+
+// fp32 SIMT grouped product out[r, n] = act(sum_k A[r, k] B_g[n, k]) for the rows r of
+// each group g (offsets, or a single group of `rows` rows when offsets is null).
+cudaError_t launch_sgemm_grouped(const float* A, const float* B, float* out,
+                                 const int32_t* offsets, int groups, int64_t rows_cap, int N,
+                                 int K, int act, const LaunchCtx& c);
+
+// ---- combine ---------------------------------------------------------------------
+struct CombineProblem {
+  int64_t T;
+  int k, d, dtype;
+  const void* y_perm;
+  const int32_t* slot_pos;
+  const float* gate;
+  void* y;
+};
+cudaError_t launch_combine(const CombineProblem& p, const LaunchCtx& c);
+
+// ---- tensor maps -----------------------------------------------------------------
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix with a box of
+// [box_rows, 64 columns] and 128-byte swizzling; out-of-range elements read as zero.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows);
+
+}  // namespace moe

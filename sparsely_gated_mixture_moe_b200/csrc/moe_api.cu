@@ -1,0 +1,374 @@
+// C ABI of libmoe (declared in include/moe.h): host-side argument validation, the
+// workspace layout, and the launch sequence of each step and of the fused forward.
+#include <string.h>
+
+#include "internal.h"
+#include "moe.h"
+
+namespace moe {
+namespace {
+
+thread_local int32_t g_last_launches = 0;
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int esize(const moe_config* c) { return c->dtype == MOE_BF16 ? 2 : 4; }
+
+// Structural validity of the config (MOE_ERR_INVALID_ARG) and supported shapes
+// (MOE_ERR_UNSUPPORTED).
+moe_status check_config(const moe_config* c) {
+  if (c == nullptr) return MOE_ERR_INVALID_ARG;
+  if (c->T < 0 || c->d_model <= 0 || c->d_ff <= 0 || c->E <= 0 || c->k <= 0 || c->k > c->E)
+    return MOE_ERR_INVALID_ARG;
+  if (c->gating != MOE_GATE_SOFTMAX_TOPK && c->gating != MOE_GATE_NOISY_TOPK) return MOE_ERR_INVALID_ARG;
+  if (c->act != MOE_ACT_RELU && c->act != MOE_ACT_GELU) return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (!(c->capacity_factor == c->capacity_factor)) return MOE_ERR_INVALID_ARG;  // NaN
+  if (c->k > 8) return MOE_ERR_UNSUPPORTED;
+  if (c->T * static_cast<int64_t>(c->k) >= (int64_t{1} << 31)) return MOE_ERR_UNSUPPORTED;
+  if (c->T * static_cast<int64_t>(c->E) >= (int64_t{1} << 31)) return MOE_ERR_UNSUPPORTED;
+  if (c->d_model % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (c->dtype == MOE_BF16) {
+    if (c->d_model % 64 != 0 || c->d_ff % 64 != 0 || c->E > 256) return MOE_ERR_UNSUPPORTED;
+  } else {
+    if (c->d_ff % 4 != 0 || c->E > 1024) return MOE_ERR_UNSUPPORTED;
+  }
+  return MOE_OK;
+}
+
+struct Layout {
+  size_t err, blk, partials, logits, nz, steps;                  // step workspace
+  size_t offsets, slot_pos, perm_src, x_perm, h, y_perm, forward;  // + forward intermediates
+};
+
+Layout layout(const moe_config* c) {
+  Layout L;
+  const int64_t n = c->T * c->k;
+  size_t o = 0;
+  L.err = o;
+  o = align_up(o + 16);
+  L.blk = o;
+  o = align_up(o + static_cast<size_t>(permute_blocks(n)) * c->E * 4);
+  L.partials = o;
+  o = align_up(o + static_cast<size_t>(route_blocks(c->T)) * 2 * c->E * 4);
+  L.logits = o;
+  L.nz = o;
+  if (c->dtype == MOE_F32) {
+    o = align_up(o + static_cast<size_t>(c->T) * c->E * 4);
+    L.nz = o;
+    if (c->gating == MOE_GATE_NOISY_TOPK) o = align_up(o + static_cast<size_t>(c->T) * c->E * 4);
+  }
+  L.steps = o;
+  L.offsets = o;
+  o = align_up(o + static_cast<size_t>(c->E + 1) * 4);
+  L.slot_pos = o;
+  o = align_up(o + static_cast<size_t>(n) * 4);
+  L.perm_src = o;
+  o = align_up(o + static_cast<size_t>(n) * 4);
+  L.x_perm = o;
+  o = align_up(o + static_cast<size_t>(n) * c->d_model * esize(c));
+  L.h = o;
+  o = align_up(o + static_cast<size_t>(n) * c->d_ff * esize(c));
+  L.y_perm = o;
+  o = align_up(o + static_cast<size_t>(n) * c->d_model * esize(c));
+  L.forward = o;
+  return L;
+}
+
+int64_t capacity_of(const moe_config* c) {
+  const float cf = c->capacity_factor;
+  if (!(cf > 0.0f)) return -1;
+  // exact ceil(cf * T * k / E) with cf = m * 2^ex, m a 24-bit integer
+  int ex = 0;
+  const double fr = frexp(static_cast<double>(cf), &ex);  // cf = fr * 2^ex, fr in [0.5, 1)
+  const uint64_t m = static_cast<uint64_t>(ldexp(fr, 24));  // exact for a float
+  ex -= 24;                                                 // cf = m * 2^ex
+  unsigned __int128 num = static_cast<unsigned __int128>(m) * static_cast<uint64_t>(c->T) *
+                          static_cast<uint64_t>(c->k);
+  unsigned __int128 den = static_cast<unsigned __int128>(c->E);
+  if (ex >= 0) {
+    if (ex > 60) return INT64_MAX;
+    num <<= ex;
+  } else {
+    if (-ex > 60) den <<= 60; else den <<= -ex;
+  }
+  const unsigned __int128 q = (num + den - 1) / den;
+  return q > static_cast<unsigned __int128>(INT64_MAX) ? INT64_MAX : static_cast<int64_t>(q);
+}
+
+struct Ctx {
+  LaunchCtx lc;
+  int launches = 0;
+  bool ok = false;
+  Ctx(void* ws, moe_stream_t stream) {
+    lc.stream = reinterpret_cast<cudaStream_t>(stream);
+    lc.err = reinterpret_cast<int*>(ws);
+    lc.launches = &launches;
+    int dev = 0;
+    ok = cudaGetDevice(&dev) == cudaSuccess &&
+         cudaDeviceGetAttribute(&lc.num_sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess;
+  }
+  moe_status finish(cudaError_t e) {
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    g_last_launches = launches;
+    return MOE_OK;
+  }
+};
+
+moe_status do_route(const moe_config* cfg, const Layout& L, const void* x, const void* w_gate,
+                    const void* w_noise, const float* noise, const float* logit_bias,
+                    int32_t* topk_idx, float* topk_gate, float* importance, float* load,
+                    uint8_t* near_tie, void* ws, Ctx& ctx) {
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  RouteProblem p;
+  p.T = cfg->T;
+  p.d = cfg->d_model;
+  p.E = cfg->E;
+  p.k = cfg->k;
+  p.noisy = cfg->gating == MOE_GATE_NOISY_TOPK;
+  p.renorm = cfg->renorm != 0;
+  p.x = x;
+  p.w_gate = w_gate;
+  p.w_noise = w_noise;
+  p.noise = noise;
+  p.bias = logit_bias;
+  p.topk_idx = topk_idx;
+  p.topk_gate = topk_gate;
+  p.near_tie = near_tie;
+  p.importance = importance;
+  p.load = load;
+  p.partials = reinterpret_cast<float*>(w + L.partials);
+  p.logits_ws = reinterpret_cast<float*>(w + L.logits);
+  p.nz_ws = reinterpret_cast<float*>(w + L.nz);
+  cudaError_t e = cfg->dtype == MOE_BF16 ? launch_route_bf16(p, ctx.lc) : launch_route_f32(p, ctx.lc);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status check_route_args(const moe_config* cfg, const void* x, const void* w_gate,
+                            const void* w_noise, const float* noise, const int32_t* topk_idx,
+                            const float* topk_gate, const float* load, const void* ws) {
+  if (!x || !w_gate || !topk_idx || !topk_gate || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  const bool noisy = cfg->gating == MOE_GATE_NOISY_TOPK;
+  if (noisy && (!w_noise || !noise || !aligned16(w_noise))) return MOE_ERR_INVALID_ARG;
+  if (load && !(noisy && cfg->k < cfg->E)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status do_permute(const moe_config* cfg, const Layout& L, const int32_t* topk_idx,
+                      const void* x, int32_t* counts, int32_t* offsets, int32_t* perm_src,
+                      int32_t* slot_pos, void* x_perm, void* ws, Ctx& ctx) {
+  PermuteProblem p;
+  p.n = cfg->T * cfg->k;
+  p.k = cfg->k;
+  p.E = cfg->E;
+  p.d = cfg->d_model;
+  p.esize = esize(cfg);
+  p.C = capacity_of(cfg);
+  p.topk_idx = topk_idx;
+  p.x = x;
+  p.counts = counts;
+  p.offsets = offsets;
+  p.perm_src = perm_src;
+  p.slot_pos = slot_pos;
+  p.x_perm = x_perm;
+  p.blk = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + L.blk);
+  return launch_permute(p, ctx.lc) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status do_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets, const void* w1,
+                  const void* w2, void* h, void* y_perm, Ctx& ctx) {
+  FfnProblem p;
+  p.rows_cap = cfg->T * cfg->k;
+  p.d = cfg->d_model;
+  p.f = cfg->d_ff;
+  p.E = cfg->E;
+  p.act = cfg->act == MOE_ACT_GELU ? 2 : 1;
+  p.x_perm = x_perm;
+  p.offsets = offsets;
+  p.w1 = w1;
+  p.w2 = w2;
+  p.h = h;
+  p.y_perm = y_perm;
+  cudaError_t e = cfg->dtype == MOE_BF16 ? launch_ffn_bf16(p, ctx.lc) : launch_ffn_f32(p, ctx.lc);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status do_combine(const moe_config* cfg, const void* y_perm, const int32_t* slot_pos,
+                      const float* gate, void* y, Ctx& ctx) {
+  CombineProblem p;
+  p.T = cfg->T;
+  p.k = cfg->k;
+  p.d = cfg->d_model;
+  p.dtype = cfg->dtype;
+  p.y_perm = y_perm;
+  p.slot_pos = slot_pos;
+  p.gate = gate;
+  p.y = y;
+  return launch_combine(p, ctx.lc) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// T == 0: nothing to route; zero the per-expert outputs that are defined anyway.
+moe_status empty_batch(const moe_config* cfg, int32_t* counts, int32_t* offsets, float* importance,
+                       float* load, moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t E = static_cast<size_t>(cfg->E);
+  if (counts && cudaMemsetAsync(counts, 0, E * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (offsets && cudaMemsetAsync(offsets, 0, (E + 1) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (importance && cudaMemsetAsync(importance, 0, E * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (load && cudaMemsetAsync(load, 0, E * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+  g_last_launches = 0;
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE: return "device error bits set";
+  }
+  return "unknown status";
+}
+
+int64_t moe_capacity(const moe_config* cfg) {
+  if (check_config(cfg) == MOE_ERR_INVALID_ARG) return -2;
+  return capacity_of(cfg);
+}
+
+size_t moe_workspace_size(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return layout(cfg).steps;
+}
+
+size_t moe_forward_workspace_size(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return layout(cfg).forward;
+}
+
+moe_status moe_route(const moe_config* cfg, const void* x, const void* w_gate, const void* w_noise,
+                     const float* noise, const float* logit_bias, int32_t* topk_idx,
+                     float* topk_gate, float* importance, float* load, uint8_t* near_tie, void* ws,
+                     moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return empty_batch(cfg, nullptr, nullptr, importance, load, stream);
+  st = check_route_args(cfg, x, w_gate, w_noise, noise, topk_idx, topk_gate, load, ws);
+  if (st != MOE_OK) return st;
+  Ctx ctx(ws, stream);
+  if (!ctx.ok) return MOE_ERR_CUDA;
+  st = do_route(cfg, layout(cfg), x, w_gate, w_noise, noise, logit_bias, topk_idx, topk_gate,
+                importance, load, near_tie, ws, ctx);
+  return st == MOE_OK ? ctx.finish(cudaSuccess) : st;
+}
+
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* x,
+                       int32_t* counts, int32_t* offsets, int32_t* perm_src, int32_t* slot_pos,
+                       void* x_perm, void* ws, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+  if (cfg->T == 0) return empty_batch(cfg, counts, offsets, nullptr, nullptr, stream);
+  if (!topk_idx || !x || !perm_src || !slot_pos || !x_perm || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_perm) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  Ctx ctx(ws, stream);
+  if (!ctx.ok) return MOE_ERR_CUDA;
+  st = do_permute(cfg, layout(cfg), topk_idx, x, counts, offsets, perm_src, slot_pos, x_perm, ws, ctx);
+  return st == MOE_OK ? ctx.finish(cudaSuccess) : st;
+}
+
+moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
+                          const void* w1, const void* w2, void* h, void* y_perm, void* ws,
+                          moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) {
+    g_last_launches = 0;
+    return MOE_OK;
+  }
+  if (!x_perm || !offsets || !w1 || !w2 || !h || !y_perm || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_perm) || !aligned16(w1) || !aligned16(w2) || !aligned16(h) ||
+      !aligned16(y_perm) || !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  Ctx ctx(ws, stream);
+  if (!ctx.ok) return MOE_ERR_CUDA;
+  st = do_ffn(cfg, x_perm, offsets, w1, w2, h, y_perm, ctx);
+  return st == MOE_OK ? ctx.finish(cudaSuccess) : st;
+}
+
+moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* slot_pos,
+                       const float* topk_gate, void* y, void* ws, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) {
+    g_last_launches = 0;
+    return MOE_OK;
+  }
+  if (!y_perm || !slot_pos || !topk_gate || !y || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_perm) || !aligned16(y) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  Ctx ctx(ws, stream);
+  if (!ctx.ok) return MOE_ERR_CUDA;
+  st = do_combine(cfg, y_perm, slot_pos, topk_gate, y, ctx);
+  return st == MOE_OK ? ctx.finish(cudaSuccess) : st;
+}
+
+moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const void* w_noise,
+                       const float* noise, const float* logit_bias, const void* w1, const void* w2,
+                       void* y, int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                       float* importance, float* load, uint8_t* near_tie, void* ws,
+                       moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts) return MOE_ERR_INVALID_ARG;
+  if (cfg->T == 0) return empty_batch(cfg, counts, nullptr, importance, load, stream);
+  st = check_route_args(cfg, x, w_gate, w_noise, noise, topk_idx, topk_gate, load, ws);
+  if (st != MOE_OK) return st;
+  if (!w1 || !w2 || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w1) || !aligned16(w2) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  Ctx ctx(ws, stream);
+  if (!ctx.ok) return MOE_ERR_CUDA;
+  const Layout L = layout(cfg);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
+  int32_t* slot_pos = reinterpret_cast<int32_t*>(w + L.slot_pos);
+  int32_t* perm_src = reinterpret_cast<int32_t*>(w + L.perm_src);
+  void* x_perm = w + L.x_perm;
+  void* h = w + L.h;
+  void* y_perm = w + L.y_perm;
+  st = do_route(cfg, L, x, w_gate, w_noise, noise, logit_bias, topk_idx, topk_gate, importance, load,
+                near_tie, ws, ctx);
+  if (st != MOE_OK) return st;
+  st = do_permute(cfg, L, topk_idx, x, counts, offsets, perm_src, slot_pos, x_perm, ws, ctx);
+  if (st != MOE_OK) return st;
+  st = do_ffn(cfg, x_perm, offsets, w1, w2, h, y_perm, ctx);
+  if (st != MOE_OK) return st;
+  st = do_combine(cfg, y_perm, slot_pos, topk_gate, y, ctx);
+  if (st != MOE_OK) return st;
+  return ctx.finish(cudaSuccess);
+}
+
+moe_status moe_get_error(void* ws, moe_stream_t stream, int32_t* device_error) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(&v, ws, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v != 0 && cudaMemset(ws, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
+  if (device_error) *device_error = v;
+  return v == 0 ? MOE_OK : MOE_ERR_DEVICE;
+}
+
+int32_t moe_last_launch_count(void) { return g_last_launches; }
+
+}  // extern "C"

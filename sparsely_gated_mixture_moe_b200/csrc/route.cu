@@ -1,0 +1,469 @@
+// Router product fused with the gate.
+//
+// Scores (Shazeer et al., "Noisy Top-K Gating"; Switch Transformer, switch_routing):
+//   softmax gating: l = x.W_g (+ bias); choose the k largest l;
+//                   renorm: G = Softmax(KeepTopK(l, k)); else gate = softmax(l)[chosen]
+//   noisy gating:   H = l + n * Softplus(x.W_noise); choose the k largest H;
+//                   G = Softmax(KeepTopK(H, k))
+// Ties go to the lowest expert index (columns are scanned in ascending order and a new
+// value displaces a kept one only when strictly larger).  For noisy gating the kernel
+// also forms, per block of 128 tokens, the partial sums of Importance = sum_t G(x_t) and
+// Load_i = sum_t Phi((l_i - kth_excluding(H, k, i)) / Softplus((x.W_noise)_i))
+// ("Load-Balancing-Losses"); a second kernel adds the partials in a fixed order, so
+// results are bit-reproducible (no floating-point atomics).
+//
+// bf16: one CTA per 128 tokens.  Warp 0 streams x tiles [128 x 64] and W_g (and
+// W_noise) tiles [E_pad x 64] with TMA into a shared-memory ring; one thread of warp 1
+// issues tcgen05.mma (M=128, N=E_pad) into TMEM; then each of the 4 warps reads its 32
+// token rows back from TMEM (one token per thread, 32 experts per tcgen05.ld) and runs
+// the gate in registers.  The logits never touch HBM.
+// fp32: the logits come from the SIMT product into the workspace and the same gate code
+// reads them back (one token per thread).
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+constexpr int kMaxK = 8;
+constexpr int kRouteBM = 128;
+
+int route_blocks(int64_t T) { return static_cast<int>((T + kRouteBM - 1) / kRouteBM); }
+
+struct GateArgs {
+  int64_t T;
+  int E, k, noisy, renorm;
+  const float* noise;
+  const float* bias;
+  int32_t* topk_idx;
+  float* topk_gate;
+  uint8_t* near_tie;
+  float* partials;  // [gridDim.x][2][E] or null
+};
+
+__device__ __forceinline__ float softplus_f(float z) {
+  return fmaxf(z, 0.0f) + log1pf(expf(-fabsf(z)));
+}
+
+// Runs the gate for the token of this thread.  `fetch(c, l, z)` must fill l[0..31] with
+// the raw clean logits x.W_g of experts c..c+31 and z[0..31] with x.W_noise (noisy
+// only); it is called by all 32 lanes of the warp together, for c = 0, 32, ...
+// `red` is shared memory of at least nwarps * 32 * 33 * 2 + 2 * nwarps * E floats when
+// partials are requested; every thread of the block must call this function.
+template <class Fetch>
+__device__ __forceinline__ void gate_token(const Fetch& fetch, int64_t t, const GateArgs& g,
+                                           float* red) {
+  const bool valid = t < g.T;
+  const int E = g.E, k = g.k;
+  float val[kMaxK + 1];
+  int ids[kMaxK + 1];
+#pragma unroll
+  for (int s = 0; s <= kMaxK; ++s) {
+    val[s] = -INFINITY;
+    ids[s] = -1;
+  }
+  float m = -INFINITY, ssum = 0.0f;  // running softmax over all experts (renorm == 0)
+  const float* noise_row = (g.noisy && valid) ? g.noise + t * E : nullptr;
+
+  for (int c = 0; c < E; c += 32) {
+    float l[32], z[32];
+    fetch(c, l, z);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int e = c + j;
+      if (e < E) {
+        float s = l[j] + (g.bias ? __ldg(g.bias + e) : 0.0f);
+        if (!g.noisy && !g.renorm) {
+          const float mn = fmaxf(m, s);
+          ssum = ssum * expf(m - mn) + expf(s - mn);
+          m = mn;
+        }
+        if (g.noisy) s += (noise_row ? __ldg(noise_row + e) : 0.0f) * softplus_f(z[j]);
+        // insert into the descending list of the k+1 largest; strict '>' keeps the
+        // lower index first among equal values
+        float cv = s;
+        int ci = e;
+#pragma unroll
+        for (int q = 0; q <= kMaxK; ++q) {
+          if (q <= k && cv > val[q]) {
+            const float tv = val[q];
+            const int ti = ids[q];
+            val[q] = cv;
+            ids[q] = ci;
+            cv = tv;
+            ci = ti;
+          }
+        }
+      }
+    }
+  }
+
+  float gate[kMaxK];
+  if (g.noisy || g.renorm) {
+    float den = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      gate[j] = (j < k) ? expf(val[j] - val[0]) : 0.0f;
+      den += gate[j];
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) gate[j] /= den;
+  } else {
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) gate[j] = (j < k) ? expf(val[j] - m) / ssum : 0.0f;
+  }
+  float kth = -INFINITY, kth1 = -INFINITY;  // k-th and (k+1)-th largest scores
+#pragma unroll
+  for (int j = 0; j <= kMaxK; ++j) {
+    if (j == k - 1) kth = val[j];
+    if (j == k) kth1 = val[j];
+  }
+  if (valid) {
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (j < k) {
+        g.topk_idx[t * k + j] = ids[j];
+        g.topk_gate[t * k + j] = gate[j];
+      }
+    if (g.near_tie) g.near_tie[t] = (k < E && (kth - kth1) <= 1e-4f) ? 1 : 0;
+  }
+
+  if (g.partials == nullptr) return;
+  // ---- Importance and Load partial sums over this block's tokens
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  float* tr_imp = red + warp * (32 * 33 * 2);
+  float* tr_load = tr_imp + 32 * 33;
+  float* wsum = red + nwarps * (32 * 33 * 2);  // [nwarps][2][E]
+  for (int c = 0; c < E; c += 32) {
+    float l[32], z[32];
+    fetch(c, l, z);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int e = c + j;
+      float gi = 0.0f, pi = 0.0f;
+      if (valid && e < E) {
+        if (g.noisy && k < E) {
+          // recomputed exactly as in the first pass, so H >= kth means "among the top k"
+          const float li = l[j] + (g.bias ? __ldg(g.bias + e) : 0.0f);
+          const float sp = softplus_f(z[j]);
+          const float H = li + __ldg(noise_row + e) * sp;
+          const float ex = (H >= kth) ? kth1 : kth;  // kth_excluding(H, k, e)
+          pi = 0.5f * erfcf(-((li - ex) / sp) * 0.70710678118654752f);
+        }
+#pragma unroll
+        for (int q = 0; q < kMaxK; ++q)
+          if (q < k && ids[q] == e) gi = gate[q];
+      }
+      tr_imp[lane * 33 + j] = gi;
+      tr_load[lane * 33 + j] = pi;
+    }
+    __syncwarp();
+    float si = 0.0f, sl = 0.0f;
+    for (int r = 0; r < 32; ++r) {
+      si += tr_imp[r * 33 + lane];
+      sl += tr_load[r * 33 + lane];
+    }
+    if (c + lane < E) {
+      wsum[(warp * 2 + 0) * E + c + lane] = si;
+      wsum[(warp * 2 + 1) * E + c + lane] = sl;
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float si = 0.0f, sl = 0.0f;
+    for (int w = 0; w < nwarps; ++w) {
+      si += wsum[(w * 2 + 0) * E + e];
+      sl += wsum[(w * 2 + 1) * E + e];
+    }
+    g.partials[(static_cast<int64_t>(blockIdx.x) * 2 + 0) * E + e] = si;
+    g.partials[(static_cast<int64_t>(blockIdx.x) * 2 + 1) * E + e] = sl;
+  }
+}
+
+// ------------------------------------------------------------------ bf16 router
+
+namespace rt {
+constexpr int THREADS = 128;
+constexpr int BK = 64;
+constexpr int A_BYTES = kRouteBM * BK * 2;  // 16 KB
+}  // namespace rt
+
+struct RouteTcArgs {
+  GateArgs g;
+  int e_pad;      // E rounded up to a multiple of 16 (the MMA N)
+  int acc_cols;   // TMEM columns per accumulator (power of two >= 32, >= e_pad)
+  int kblocks;    // d / 64
+  int nb;         // 1, or 2 with W_noise
+  int stages;
+  int bar_off;    // byte offset of the barriers in shared memory
+  int* err;
+};
+
+__global__ void __launch_bounds__(rt::THREADS, 1)
+    route_tc_kernel(const __grid_constant__ CUtensorMap tmX,
+                    const __grid_constant__ CUtensorMap tmG,
+                    const __grid_constant__ CUtensorMap tmN, const RouteTcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int b_bytes = a.e_pad * rt::BK * 2;
+  const int stage_bytes = rt::A_BYTES + a.nb * b_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.bar_off);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + a.stages);
+  const uint32_t done = smem_u32(bars + 2 * a.stages);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * a.stages + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ncols = static_cast<uint32_t>(a.nb * a.acc_cols);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(done, 1);
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int t0 = blockIdx.x * kRouteBM;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmX);
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_par = 0;
+      bool aborted = false;
+      for (int kb = 0; kb < a.kblocks; ++kb) {
+        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, s_abort)) {
+          aborted = true;
+          break;
+        }
+        uint8_t* st = smem + stage * stage_bytes;
+        const uint32_t fb = full0 + 8 * stage;
+        mbar_arrive_expect_tx(fb, static_cast<uint32_t>(stage_bytes));
+        tma_load_2d(smem_u32(st), &tmX, fb, kb * rt::BK, t0);
+        tma_load_2d(smem_u32(st + rt::A_BYTES), &tmG, fb, kb * rt::BK, 0);
+        if (a.nb == 2) tma_load_2d(smem_u32(st + rt::A_BYTES + b_bytes), &tmN, fb, kb * rt::BK, 0);
+        armed |= 1u << stage;
+        armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == a.stages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (aborted) {
+        set_error(a.err, kErrTimeout);
+        *s_abort = 1;
+        for (int s = 0; s < a.stages; ++s)
+          if (armed & (1u << s)) mbar_wait(full0 + 8 * s, (armed_par >> s) & 1, nullptr, kDrainLimitNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kRouteBM, a.e_pad);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool aborted = false;
+      for (int kb = 0; kb < a.kblocks; ++kb) {
+        if (!mbar_wait(full0 + 8 * stage, phase, s_abort)) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + stage * stage_bytes);
+#pragma unroll
+        for (int kk = 0; kk < rt::BK / 16; ++kk) {
+          const uint64_t ad = sdesc_k128(st + kk * 32);
+          const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+          tc_mma_bf16(tmem_base, ad, sdesc_k128(st + rt::A_BYTES + kk * 32), idesc, acc);
+          if (a.nb == 2)
+            tc_mma_bf16(tmem_base + a.acc_cols, ad,
+                        sdesc_k128(st + rt::A_BYTES + b_bytes + kk * 32), idesc, acc);
+        }
+        tc_commit(empty0 + 8 * stage);
+        if (++stage == a.stages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (aborted) {
+        set_error(a.err, kErrTimeout);
+        *s_abort = 1;
+      }
+      tc_commit(done);  // arrives once every MMA issued above has finished
+      if (aborted) mbar_wait(done, 0, nullptr, kDrainLimitNs);
+    }
+    __syncwarp();
+  }
+  if (!mbar_wait(done, 0, s_abort)) *s_abort = 1;
+  __syncthreads();
+  const bool ok = (*s_abort == 0);
+  tc_fence_after();
+  if (ok) {
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    auto fetch = [&](int c, float (&l)[32], float (&z)[32]) {
+      uint32_t v[32];
+      tmem_ld32(tmem_base + lane_base + c, v);
+      if (a.nb == 2) {
+        uint32_t w[32];
+        tmem_ld32(tmem_base + lane_base + a.acc_cols + c, w);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) z[j] = __uint_as_float(w[j]);
+      } else {
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) z[j] = 0.0f;
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) l[j] = __uint_as_float(v[j]);
+    };
+    // the stage buffers are idle once `done` has fired: reuse them for the reduction
+    gate_token(fetch, static_cast<int64_t>(t0) + threadIdx.x, a.g, reinterpret_cast<float*>(smem));
+  } else if (threadIdx.x == 0) {
+    set_error(a.err, kErrTimeout);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, ncols);
+}
+
+// ------------------------------------------------------------------ fp32 router
+
+// One token per thread; the logits were written to the workspace by the SIMT product.
+__global__ void __launch_bounds__(128)
+    gate_f32_kernel(const float* __restrict__ logits, const float* __restrict__ nz, GateArgs g) {
+  extern __shared__ float red[];
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const bool valid = t < g.T;
+  const int E = g.E;
+  auto fetch = [&](int c, float (&l)[32], float (&z)[32]) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const bool in = valid && (c + j < E);
+      l[j] = in ? logits[t * E + c + j] : 0.0f;
+      z[j] = (in && nz != nullptr) ? nz[t * E + c + j] : 0.0f;
+    }
+  };
+  gate_token(fetch, t, g, red);
+}
+
+__global__ void finalize_importance_load_kernel(const float* __restrict__ partials, int nblocks,
+                                                int E, float* importance, float* load) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= E) return;
+  float si = 0.0f, sl = 0.0f;
+  for (int b = 0; b < nblocks; ++b) {
+    si += partials[(static_cast<int64_t>(b) * 2 + 0) * E + e];
+    sl += partials[(static_cast<int64_t>(b) * 2 + 1) * E + e];
+  }
+  if (importance) importance[e] = si;
+  if (load) load[e] = sl;
+}
+
+// ------------------------------------------------------------------ launchers
+
+static GateArgs gate_args(const RouteProblem& p) {
+  GateArgs g;
+  g.T = p.T;
+  g.E = p.E;
+  g.k = p.k;
+  g.noisy = p.noisy;
+  g.renorm = p.renorm;
+  g.noise = p.noise;
+  g.bias = p.bias;
+  g.topk_idx = p.topk_idx;
+  g.topk_gate = p.topk_gate;
+  g.near_tie = p.near_tie;
+  g.partials = (p.importance || p.load) ? p.partials : nullptr;
+  return g;
+}
+
+static size_t reduction_smem(int E, int nwarps) {
+  return static_cast<size_t>(nwarps) * (32 * 33 * 2) * 4 + static_cast<size_t>(2) * nwarps * E * 4;
+}
+
+static cudaError_t launch_finalize(const RouteProblem& p, int nblocks, const LaunchCtx& c) {
+  if (!(p.importance || p.load)) return cudaSuccess;
+  finalize_importance_load_kernel<<<(p.E + 127) / 128, 128, 0, c.stream>>>(
+      p.partials, nblocks, p.E, p.importance, p.load);
+  ++*c.launches;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
+  RouteTcArgs a;
+  a.g = gate_args(p);
+  a.e_pad = (p.E + 15) / 16 * 16;
+  a.acc_cols = 32;
+  while (a.acc_cols < a.e_pad) a.acc_cols <<= 1;
+  a.kblocks = p.d / rt::BK;
+  a.nb = p.noisy ? 2 : 1;
+  const int stage_bytes = rt::A_BYTES + a.nb * a.e_pad * rt::BK * 2;
+  int stages = (160 * 1024) / stage_bytes;
+  if (stages > 8) stages = 8;
+  if (stages > a.kblocks) stages = a.kblocks;
+  if (stages < 2) stages = 2;
+  a.stages = stages;
+  int region = stages * stage_bytes;
+  const int red = static_cast<int>(reduction_smem(p.E, rt::THREADS / 32));
+  if (region < red) region = red;
+  a.bar_off = (region + 127) / 128 * 128;
+  a.err = c.err;
+  const int smem = 1024 + a.bar_off + 8 * (2 * stages + 1) + 16;
+
+  CUtensorMap tmX, tmG, tmN;
+  if (!make_tmap_bf16(&tmX, p.x, static_cast<uint64_t>(p.T), p.d, kRouteBM)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16(&tmG, p.w_gate, static_cast<uint64_t>(p.E), p.d, a.e_pad)) return cudaErrorInvalidValue;
+  if (p.noisy) {
+    if (!make_tmap_bf16(&tmN, p.w_noise, static_cast<uint64_t>(p.E), p.d, a.e_pad)) return cudaErrorInvalidValue;
+  } else {
+    tmN = tmG;
+  }
+  cudaError_t e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int nblocks = route_blocks(p.T);
+  route_tc_kernel<<<nblocks, rt::THREADS, smem, c.stream>>>(tmX, tmG, tmN, a);
+  ++*c.launches;
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_finalize(p, nblocks, c);
+}
+
+cudaError_t launch_route_f32(const RouteProblem& p, const LaunchCtx& c) {
+  cudaError_t e = launch_sgemm_grouped(static_cast<const float*>(p.x), static_cast<const float*>(p.w_gate),
+                                       p.logits_ws, nullptr, 1, p.T, p.E, p.d, 0, c);
+  if (e != cudaSuccess) return e;
+  if (p.noisy) {
+    e = launch_sgemm_grouped(static_cast<const float*>(p.x), static_cast<const float*>(p.w_noise),
+                             p.nz_ws, nullptr, 1, p.T, p.E, p.d, 0, c);
+    if (e != cudaSuccess) return e;
+  }
+  GateArgs g = gate_args(p);
+  const size_t smem = g.partials ? reduction_smem(p.E, 4) : 0;
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(gate_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  const int nblocks = route_blocks(p.T);
+  gate_f32_kernel<<<nblocks, 128, smem, c.stream>>>(p.logits_ws, p.noisy ? p.nz_ws : nullptr, g);
+  ++*c.launches;
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_finalize(p, nblocks, c);
+}
+
+}  // namespace moe

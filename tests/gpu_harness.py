@@ -1,0 +1,214 @@
+"""Helpers of the GPU parity tests: run the library's steps on a workload and compare
+each against the CPU oracle on the same inputs.
+
+Step-wise parity feeds every oracle step the GPU's own upstream outputs (its expert
+choices, its permuted rows), so a near tie in the router cannot cascade into later
+steps; the end-to-end check follows the GPU's choice only at near ties (where the two
+choices are both correct up to rounding) and the oracle's everywhere else.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import sparsely_gated_mixture_moe_b200 as moe
+from oracle import moe_oracle as orc
+import workloads
+
+# max-abs error / RMS of the oracle output (bf16 and fp32 layer tensors)
+TOL = {"f32": 1e-5, "bf16": 2e-2}
+# absolute tolerance on fp32 gate values (fp32 softmax of fp32-accumulated scores)
+GATE_ATOL = 2e-5
+NEAR_TIE = 1e-4
+
+
+def rel_err(got, want) -> float:
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    if want.size == 0:
+        return 0.0
+    rms = float(np.sqrt(np.mean(want ** 2)))
+    if rms == 0.0:
+        return float(np.max(np.abs(got - want)))
+    return float(np.max(np.abs(got - want))) / rms
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu").double().numpy()
+
+
+def config_of(w: workloads.Workload) -> moe.MoEConfig:
+    return moe.make_config(w.T, w.d_model, w.d_ff, w.E, w.k, gating=w.gating, renorm=w.renorm,
+                           capacity_factor=w.capacity_factor, act=w.act, dtype=w.dtype)
+
+
+def to_device(inp):
+    return {k: v.cuda() for k, v in inp.items()}
+
+
+def run_steps(w, dev, cfg=None):
+    """The four step calls on one stream; returns every output on the CPU."""
+    cfg = cfg or config_of(w)
+    T, k, E, d, f = w.T, w.k, w.E, w.d_model, w.d_ff
+    dt = w.torch_dtype
+    cu = "cuda"
+    o = {
+        "topk_idx": torch.full((T, k), -7, dtype=torch.int32, device=cu),
+        "topk_gate": torch.full((T, k), float("nan"), dtype=torch.float32, device=cu),
+        "near_tie": torch.full((T,), 9, dtype=torch.uint8, device=cu),
+        "counts": torch.full((E,), -7, dtype=torch.int32, device=cu),
+        "offsets": torch.full((E + 1,), -7, dtype=torch.int32, device=cu),
+        "perm_src": torch.full((max(T * k, 1),), -7, dtype=torch.int32, device=cu),
+        "slot_pos": torch.full((max(T * k, 1),), -7, dtype=torch.int32, device=cu),
+        "x_perm": torch.zeros(max(T * k, 1), d, dtype=dt, device=cu),
+        "h": torch.zeros(max(T * k, 1), f, dtype=dt, device=cu),
+        "y_perm": torch.zeros(max(T * k, 1), d, dtype=dt, device=cu),
+        "y": torch.full((T, d), float("nan"), dtype=dt, device=cu),
+    }
+    noisy = w.gating == "noisy_topk"
+    o["importance"] = torch.full((E,), float("nan"), device=cu)
+    o["load"] = torch.full((E,), float("nan"), device=cu) if noisy and k < E else None
+    ws = moe.workspace(cfg, cu)
+    moe.moe_route(cfg, dev["x"], dev["w_gate"], o["topk_idx"], o["topk_gate"], ws,
+                  w_noise=dev.get("w_noise"), noise=dev.get("noise"),
+                  logit_bias=dev.get("logit_bias"), importance=o["importance"], load=o["load"],
+                  near_tie=o["near_tie"])
+    moe.moe_permute(cfg, o["topk_idx"], dev["x"], o["counts"], o["offsets"], o["perm_src"],
+                    o["slot_pos"], o["x_perm"], ws)
+    moe.moe_expert_ffn(cfg, o["x_perm"], o["offsets"], dev["w1"], dev["w2"], o["h"], o["y_perm"], ws)
+    moe.moe_combine(cfg, o["y_perm"], o["slot_pos"], o["topk_gate"], o["y"], ws)
+    err = moe.moe_get_error(ws)
+    out = {kk: (v.cpu() if v is not None else None) for kk, v in o.items()}
+    out["device_error"] = err
+    return out
+
+
+def run_forward(w, dev, cfg=None):
+    cfg = cfg or config_of(w)
+    layer = moe.MoELayer(cfg, {kk: v for kk, v in dev.items() if kk not in ("x", "noise")})
+    y = layer.forward(dev["x"], noise=dev.get("noise"))
+    err = moe.moe_get_error(layer.ws)
+    return {"y": y.cpu(), "topk_idx": layer.topk_idx.cpu(), "topk_gate": layer.topk_gate.cpu(),
+            "counts": layer.counts.cpu(), "device_error": err,
+            "importance": None if layer.importance is None else layer.importance.cpu(),
+            "load": None if layer.load is None else layer.load.cpu()}
+
+
+def reconcile_choice(w, r, idx_gpu):
+    """The oracle's expert choice, except at near ties where the GPU's choice is taken
+    after checking it is a correct one (its scores within the near-tie margin of the
+    oracle's k-th score).  Returns (idx, n_near_tie, n_differ)."""
+    idx_o = r["idx"]
+    near = r["gap"] <= NEAR_TIE
+    differ = ~np.all(idx_gpu == idx_o, axis=1)
+    bad = differ & ~near
+    assert not bad.any(), "expert choice differs on %d non-near-tie tokens, e.g. %s" % (
+        int(bad.sum()), np.nonzero(bad)[0][:5])
+    idx = idx_o.copy()
+    if differ.any():
+        s = -np.sort(-r["scores"], axis=1)
+        kth = s[:, w.k - 1]
+        rows = np.nonzero(differ)[0]
+        chosen = np.take_along_axis(r["scores"][rows], idx_gpu[rows], axis=1)
+        assert np.all(chosen >= kth[rows, None] - NEAR_TIE)
+        assert all(len(set(v)) == w.k for v in idx_gpu[rows].tolist())
+        idx[rows] = idx_gpu[rows]
+    return idx, int(near.sum()), int(differ.sum())
+
+
+def check_route(w, inp, g, report):
+    r = orc.route(inp, w)
+    idx_g = g["topk_idx"].long().numpy()
+    assert idx_g.min() >= 0 and idx_g.max() < w.E
+    idx, n_near, n_diff = reconcile_choice(w, r, idx_g)
+    renorm = True if w.gating == "noisy_topk" else w.renorm
+    gates_o = orc.gate_values(r["scores"], idx, renorm)
+    gerr = float(np.max(np.abs(g["topk_gate"].double().numpy() - gates_o))) if w.T else 0.0
+    assert gerr <= GATE_ATOL, gerr
+    nt = g["near_tie"].numpy().astype(bool)
+    # the GPU's near-tie flag agrees with the oracle's gap away from the threshold
+    assert not np.any(nt & (r["gap"] > 2 * NEAR_TIE))
+    assert not np.any(~nt & (r["gap"] < 0.5 * NEAR_TIE))
+    report.update(near_ties=n_near, choice_differs=n_diff, gate_abs_err=gerr)
+    if g.get("importance") is not None:
+        G = orc.dense_gates(w.T, w.E, idx, gates_o)
+        imp = orc.importance(G)
+        ierr = rel_err(g["importance"].double().numpy(), imp)
+        assert ierr <= 1e-4, ierr
+        report["importance_err"] = ierr
+    if g.get("load") is not None:
+        lerr = rel_err(g["load"].double().numpy(), r["load"])
+        assert lerr <= 1e-4, lerr
+        report["load_err"] = lerr
+    return idx, gates_o
+
+
+def check_permute(w, inp, g, report):
+    idx_g = g["topk_idx"].long().numpy()
+    C = orc.capacity(w.capacity_factor, w.T, w.k, w.E)
+    counts, offsets, perm_src, slot_pos = orc.dispatch(idx_g, w.E, C)
+    n = int(offsets[-1])
+    assert g["counts"].tolist() == counts.tolist()
+    assert g["offsets"].tolist() == offsets.tolist()
+    assert g["slot_pos"][: w.T * w.k].tolist() == slot_pos.tolist()
+    assert g["perm_src"][:n].tolist() == perm_src.tolist()
+    # x_perm rows are byte copies of the token rows
+    assert torch.equal(g["x_perm"][:n], inp["x"][torch.from_numpy(perm_src // w.k)])
+    report.update(kept=n, dropped=w.T * w.k - n, capacity=C)
+    return n
+
+
+def check_ffn(w, inp, g, n, report, rows=None):
+    """y_perm (and h) of the GPU against the oracle's experts on the GPU's own x_perm."""
+    off = g["offsets"].numpy()
+    tol = TOL[w.dtype]
+    if rows is None:
+        h_o, y_o = orc.expert_ffn(f64(g["x_perm"][:n]), off, inp["w1"], inp["w2"], w.act)
+        eh = rel_err(f64(g["h"][:n]), h_o)
+        ey = rel_err(f64(g["y_perm"][:n]), y_o)
+    else:
+        e_of = np.searchsorted(off, rows, side="right") - 1
+        hs, ys = [], []
+        for s, e in zip(rows, e_of):
+            h1, y1 = orc.expert(f64(g["x_perm"][s:s + 1]), inp["w1"][e], inp["w2"][e], w.act)
+            hs.append(h1[0])
+            ys.append(y1[0])
+        eh = rel_err(f64(g["h"][rows]), np.array(hs))
+        ey = rel_err(f64(g["y_perm"][rows]), np.array(ys))
+    assert eh <= tol, eh
+    assert ey <= tol, ey
+    report.update(h_err=eh, y_perm_err=ey)
+
+
+def check_combine(w, g, report, rows=None):
+    sp = g["slot_pos"][: w.T * w.k].numpy()
+    gates = g["topk_gate"].double().numpy()
+    if rows is None:
+        y_o = orc.combine(f64(g["y_perm"]), sp, gates, w.T, w.k)
+        e = rel_err(f64(g["y"]), y_o)
+    else:
+        sub_sp = sp.reshape(w.T, w.k)[rows]
+        yp = f64(g["y_perm"])
+        y_o = np.zeros((len(rows), w.d_model))
+        for n_, (t, s_row) in enumerate(zip(rows, sub_sp)):
+            for j, s in enumerate(s_row):
+                if s >= 0:
+                    y_o[n_] += gates[t, j] * yp[s]
+        e = rel_err(f64(g["y"][rows]), y_o)
+    assert e <= TOL[w.dtype], e
+    report["combine_err"] = e
+
+
+def check_end_to_end(w, inp, g, idx, gates, report, rows=None):
+    tol = TOL[w.dtype]
+    if rows is None:
+        rows = list(range(w.T))
+    y_o, r = orc.moe_forward_rows(inp, w, rows, idx=idx, gates=gates)
+    e = rel_err(f64(g["y"][rows]), y_o)
+    assert e <= tol, e
+    # fully dropped tokens output exactly zero
+    sp = r["slot_pos"].reshape(w.T, w.k)
+    dropped = [i for i, t in enumerate(rows) if np.all(sp[t] < 0)]
+    if dropped:
+        assert torch.all(g["y"][[rows[i] for i in dropped]] == 0)
+    report.update(y_err=e, fully_dropped_checked=len(dropped))

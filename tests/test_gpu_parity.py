@@ -1,0 +1,160 @@
+"""Parity of the CUDA path with the CPU oracle, element by element, on seeded inputs.
+
+Small cases (the oracle finishes in seconds) cover every workload's shape family at a
+reduced token count, several 128-row tiles with ragged tails, each N-tile width of the
+grouped GEMM, capacity stress, and the degenerate cases (one expert, k = E, one token,
+no tokens, T not a multiple of the tile).  The full-size cases run the exact workloads
+the benchmark times and compare sampled outputs plus everything that is cheap to check
+everywhere (choices, gates, the permutation, counts)."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from workloads import Workload
+from tests import gpu_harness as H
+
+pytestmark = pytest.mark.gpu
+
+W = workloads.WORKLOADS
+SMALL = {
+    "tiny": W["tiny"],
+    "switch_T2048": W["switch"].scaled(T=2048),
+    "noisy_T1024": W["noisy"].scaled(T=1024),
+    "gshard_T1024": W["gshard"].scaled(T=1024),
+    "zipf_T2048": W["zipf"].scaled(T=2048),
+    "multitile_T4096": Workload("mt", T=4096, d_model=256, d_ff=512, E=16, k=2, act="gelu"),
+    "bn128_T1000": Workload("b128", T=1000, d_model=384, d_ff=640, E=12, k=3, act="relu"),
+    "bn64_T777": Workload("b64", T=777, d_model=448, d_ff=192, E=5, k=2, act="gelu"),
+    "cap0.25": Workload("c25", T=1024, d_model=128, d_ff=256, E=8, k=2, capacity_factor=0.25),
+    "cap0.5_switch": Workload("c50", T=1024, d_model=128, d_ff=256, E=8, k=1, renorm=False,
+                              capacity_factor=0.5, act="gelu"),
+    "cap1.0": Workload("c100", T=1024, d_model=128, d_ff=256, E=8, k=2, capacity_factor=1.0),
+    "noisy_small_E": Workload("nz", T=600, d_model=128, d_ff=128, E=12, k=3, gating="noisy_topk"),
+    "f32_noisy": Workload("f32n", T=300, d_model=64, d_ff=96, E=10, k=3, gating="noisy_topk",
+                          dtype="f32"),
+    "f32_switch_cap": Workload("f32s", T=257, d_model=32, d_ff=64, E=6, k=1, renorm=False,
+                               capacity_factor=0.75, act="gelu", dtype="f32"),
+    "one_expert": Workload("e1", T=300, d_model=128, d_ff=128, E=1, k=1),
+    "k_equals_E": Workload("kE", T=200, d_model=64, d_ff=128, E=4, k=4, act="gelu"),
+    "one_token": Workload("t1", T=1, d_model=64, d_ff=64, E=8, k=2),
+    "E8_bf16_pad": Workload("e8", T=500, d_model=64, d_ff=64, E=8, k=2),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_steps_and_forward_small(name):
+    w = SMALL[name]
+    inp = workloads.make_inputs(w)
+    dev = H.to_device(inp)
+    g = H.run_steps(w, dev)
+    assert g["device_error"] == 0
+    rep = {}
+    idx, gates = H.check_route(w, inp, g, rep)
+    n = H.check_permute(w, inp, g, rep)
+    H.check_ffn(w, inp, g, n, rep)
+    H.check_combine(w, g, rep)
+    H.check_end_to_end(w, inp, g, idx, gates, rep)
+    f = H.run_forward(w, dev)
+    assert f["device_error"] == 0
+    # the fused call runs the same kernels: identical results
+    assert torch.equal(f["topk_idx"], g["topk_idx"])
+    assert torch.equal(f["counts"], g["counts"])
+    assert torch.equal(f["y"].view(torch.int16) if w.dtype == "bf16" else f["y"], 
+                       g["y"].view(torch.int16) if w.dtype == "bf16" else g["y"])
+    print(name, rep)
+
+
+def test_empty_batch():
+    w = Workload("t0", T=0, d_model=64, d_ff=64, E=4, k=2, gating="noisy_topk")
+    inp = workloads.make_inputs(w)
+    dev = H.to_device(inp)
+    g = H.run_steps(w, dev)
+    assert g["device_error"] == 0
+    assert g["counts"].tolist() == [0] * 4
+    assert g["offsets"].tolist() == [0] * 5
+    assert g["importance"].tolist() == [0.0] * 4 and g["load"].tolist() == [0.0] * 4
+
+
+def test_deterministic_repeat():
+    w = SMALL["noisy_T1024"]
+    dev = H.to_device(workloads.make_inputs(w))
+    a, b = H.run_steps(w, dev), H.run_steps(w, dev)
+    for key in ("topk_idx", "topk_gate", "counts", "slot_pos", "y", "importance", "load"):
+        assert torch.equal(a[key], b[key]), key
+
+
+def test_bad_expert_index_sets_error_and_drops():
+    """An out-of-range index fed to moe_permute is reported through the device error
+    word and treated as dropped; nothing else changes."""
+    import sparsely_gated_mixture_moe_b200 as moe
+    w = Workload("bad", T=64, d_model=64, d_ff=64, E=4, k=2)
+    cfg = H.config_of(w)
+    inp = workloads.make_inputs(w)
+    x = inp["x"].cuda()
+    idx = torch.tensor([[0, 1]] * 64, dtype=torch.int32)
+    idx[5, 1] = 7
+    idx[9, 0] = -3
+    ws = moe.workspace(cfg)
+    counts = torch.empty(4, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(5, dtype=torch.int32, device="cuda")
+    perm_src = torch.empty(128, dtype=torch.int32, device="cuda")
+    slot_pos = torch.empty(128, dtype=torch.int32, device="cuda")
+    x_perm = torch.empty(128, 64, dtype=torch.bfloat16, device="cuda")
+    moe.moe_permute(cfg, idx.cuda(), x, counts, offsets, perm_src, slot_pos, x_perm, ws)
+    err = moe.moe_get_error(ws)
+    assert err == 1
+    assert moe.moe_get_error(ws) == 0  # cleared by the read
+    sp = slot_pos.cpu().numpy()
+    assert sp[5 * 2 + 1] == -1 and sp[9 * 2 + 0] == -1
+    assert counts.cpu().tolist() == [63, 63, 0, 0]
+
+
+def test_bad_offsets_set_error():
+    """Offsets that are not non-decreasing make moe_expert_ffn skip its work and report
+    MOE_DEVERR_OFFSETS instead of reading or writing out of range."""
+    import sparsely_gated_mixture_moe_b200 as moe
+    w = Workload("off", T=64, d_model=64, d_ff=64, E=4, k=1)
+    cfg = H.config_of(w)
+    inp = H.to_device(workloads.make_inputs(w))
+    ws = moe.workspace(cfg)
+    offsets = torch.tensor([0, 30, 10, 50, 64], dtype=torch.int32, device="cuda")
+    h = torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda")
+    moe.moe_expert_ffn(cfg, inp["x"], offsets, inp["w1"], inp["w2"], h, y, ws)
+    assert moe.moe_get_error(ws) & 2
+    offsets = torch.tensor([0, 10, 20, 30, 65], dtype=torch.int32, device="cuda")  # past T*k
+    moe.moe_expert_ffn(cfg, inp["x"], offsets, inp["w1"], inp["w2"], h, y, ws)
+    assert moe.moe_get_error(ws) & 2
+
+
+FULL = ["switch", "noisy", "gshard", "zipf"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(name):
+    """The benchmark's workloads at full size, in the launch configuration the benchmark
+    times.  Choices, gates, importance/load and the whole permutation are checked on
+    every token; expert outputs and layer outputs on a sample of rows (including each
+    expert's first and last kept row)."""
+    w = W[name]
+    inp = workloads.make_inputs(w)
+    dev = H.to_device(inp)
+    g = H.run_steps(w, dev)
+    assert g["device_error"] == 0
+    rep = {}
+    idx, gates = H.check_route(w, inp, g, rep)
+    n = H.check_permute(w, inp, g, rep)
+    rng = np.random.default_rng(0)
+    off = g["offsets"].numpy()
+    edge = [int(off[e]) for e in range(w.E) if off[e + 1] > off[e]][:16] + \
+           [int(off[e + 1]) - 1 for e in range(w.E) if off[e + 1] > off[e]][:16]
+    rows = sorted(set(edge) | set(rng.choice(n, size=min(n, 48), replace=False).tolist()))
+    H.check_ffn(w, inp, g, n, rep, rows=rows)
+    toks = sorted(set(rng.choice(w.T, size=48, replace=False).tolist()) | {0, w.T - 1})
+    H.check_combine(w, g, rep, rows=toks)
+    H.check_end_to_end(w, inp, g, idx, gates, rep, rows=toks)
+    f = H.run_forward(w, dev)
+    assert f["device_error"] == 0
+    assert torch.equal(f["y"].view(torch.int16), g["y"].view(torch.int16))
+    print(name, rep)
