@@ -1,0 +1,455 @@
+"""Benchmark of the sparsely-gated MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload switch] [--impl reference]
+
+One step is one pass of the whole layer (route, permute, expert FFN, combine) over one
+batch of synthetic tokens.  Default workload: the Switch-style top-1 layer (T=16384,
+d_model=768, d_ff=3072, E=128, capacity factor 1.25, GELU, bf16).  Under torchrun every
+rank runs an independent replica on its own GPU (the layer forward has no exchange step
+on one device), the step time is the max over ranks, and the value is the tokens of all
+ranks per second.
+
+Timing: W untimed warm-up steps; then K steps, each preceded (outside its events) by a
+write of a 256 MB buffer that flushes the 126 MB L2; CUDA events on the launching stream
+bracket each step and each step call.  The dominant kernel is the tcgen05 grouped GEMM
+(two launches per step: up- and down-projection); its roofline uses the algorithmic
+bytes/FLOPs of those two launches over the event time of the expert-FFN call.
+
+--impl reference times the CPU oracle on this machine's host cores instead (a bounded
+sample of the same workload per step) and prints the same JSON line with impl=reference.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "MoE layer fwd tokens/s; expert GEMM TFLOP/s and % of B200 bf16 / HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+GEMM_SOURCES = ["sparsely_gated_mixture_moe_b200/csrc/grouped_gemm_tc.cu",
+                "sparsely_gated_mixture_moe_b200/csrc/common.cuh"]
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def dist_env():
+    """(rank, local_rank, world) from the torchrun environment, or (0, 0, 1)."""
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank scalar over the process group (identity without one)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def gemm_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the grouped GEMM from the committed ncu summary, or None
+    when there is none for this workload or the kernel source changed since."""
+    p = os.path.join(ROOT, "profiles", "grouped_gemm_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    sha = gemm_source_sha()
+    for line in open(p):
+        f = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
+        if f.get("workload") == workload and f.get("src_sha") == sha and "bytes_per_launch" in f:
+            return float(f["bytes_per_launch"])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        rows = []
+        for l in getattr(self, "lines", []):
+            p = [x.strip() for x in l.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                rows.append((float(p[1]), float(p[2]), p[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v == "Active"})
+        top = max(r[0] for r in rows)
+        loaded = [r[0] for r in rows if r[0] >= 0.5 * top] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def algorithmic(w: workloads.Workload, n_kept: int, counts_kept):
+    """Algorithmic FLOPs and bytes of each step (kept assignments only, no padding).
+
+    FFN FLOPs 4*N*d*f (two products).  FFN bytes: the weights of the experts that got
+    rows, x_perm (dtype) read, y_perm (fp32) written.  Route bytes: x, the gating
+    weights, noise, and the chosen indices and gates.  Permute: x rows read, x_perm
+    rows written, indices.  Combine: y_perm rows read, gates and slots, y written."""
+    es = 2 if w.dtype == "bf16" else 4
+    T, d, f, E, k = w.T, w.d_model, w.d_ff, w.E, w.k
+    active = int(sum(1 for c in counts_kept if c > 0))
+    ffn_flops = 4.0 * n_kept * d * f
+    ffn_bytes = active * 2.0 * d * f * es + n_kept * d * es + n_kept * d * 4.0
+    noisy = w.gating == "noisy_topk"
+    route_bytes = T * d * es + E * d * es * (2 if noisy else 1) + (T * E * 4 if noisy else 0) + T * k * 8
+    permute_bytes = n_kept * d * es * 2 + T * k * 4 * 3
+    combine_bytes = n_kept * d * 4.0 + T * k * 8 + T * d * 4.0
+    return {"ffn_flops": ffn_flops, "ffn_bytes": ffn_bytes, "route_bytes": route_bytes,
+            "permute_bytes": permute_bytes, "combine_bytes": combine_bytes}
+
+
+# ------------------------------------------------------------------------ CPU oracle arm
+
+def oracle_sample(w, inp, n_tokens):
+    """The oracle's forward over a contiguous sample of n_tokens tokens (routing and
+    capacity computed over that sample).  Returns seconds."""
+    from oracle import moe_oracle as orc
+    sub = {k: (v[:n_tokens] if k in ("x", "noise") else v) for k, v in inp.items()}
+    ws = w.scaled(T=n_tokens)
+    t0 = time.perf_counter()
+    orc.moe_forward(sub, ws)
+    return time.perf_counter() - t0
+
+
+def cpu_cores():
+    n = len(os.sched_getaffinity(0))
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        blas = n
+    return n, blas
+
+
+def sample_size(w, inp, seconds):
+    """Tokens of the workload the oracle forwards in about `seconds` (>= 16)."""
+    n0 = min(w.T, 256)
+    dt = oracle_sample(w, inp, n0)
+    return int(max(16, min(w.T, n0 * seconds / max(dt, 1e-4))))
+
+
+def cpu_baseline(w, inp, budget_s=15.0):
+    """Time the oracle as it stands on a token sample sized to about budget_s."""
+    n = sample_size(w, inp, budget_s)
+    dt = oracle_sample(w, inp, n)
+    cores, blas = cpu_cores()
+    return {"value": n / dt, "unit": "tokens/s", "cores": blas, "kind": "oracle",
+            "sample": "%d of the workload's %d tokens, one forward pass (NumPy fp64; %d host "
+                      "cores visible, %d BLAS threads)" % (n, w.T, cores, blas)}
+
+
+def run_reference(args, w):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    inp = workloads.make_inputs(w)
+    per_step = max(0.05, 120.0 / (args.steps + args.warmup))
+    n = sample_size(w, inp, per_step)
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, n)
+    times = [oracle_sample(w, inp, n) for _ in range(args.steps)]
+    per_tok = sum(times) / (len(times) * n)
+    value = 1.0 / per_tok
+    cores, blas = cpu_cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_tok * w.T * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_json(w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas, "kind": "oracle",
+                         "sample": "each step: %d of the workload's %d tokens, one forward pass "
+                                   "(ms_per_step scaled to all tokens)" % (n, w.T)},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_json(w):
+    c = {"workload": "%s: T=%d d_model=%d d_ff=%d E=%d k=%d gating=%s%s cf=%s act=%s %s" % (
+        w.name, w.T, w.d_model, w.d_ff, w.E, w.k, w.gating,
+        "" if w.gating == "noisy_topk" else ("(renorm)" if w.renorm else "(full-softmax gate)"),
+        w.capacity_factor, w.act, w.dtype),
+        "T": w.T, "d_model": w.d_model, "d_ff": w.d_ff, "E": w.E, "k": w.k,
+        "capacity_factor": w.capacity_factor, "hidden_split": w.hidden_split,
+        "l2": "flushed before every timed step (256 MB write)",
+        "parallelism": "replicas"}
+    return c
+
+
+# ------------------------------------------------------------------------------ GPU arm
+
+def run_gpu(args, w):
+    import torch.distributed as dist
+    import sparsely_gated_mixture_moe_b200 as moe
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+
+    inp = workloads.make_inputs(w)
+    d = {k: v.to(dev) for k, v in inp.items()}
+    cfg = moe.make_config(w.T, w.d_model, w.d_ff, w.E, w.k, gating=w.gating, renorm=w.renorm,
+                          capacity_factor=w.capacity_factor, act=w.act, dtype=w.dtype,
+                          hidden_split=w.hidden_split)
+    T, k, E, dm, f = w.T, w.k, w.E, w.d_model, w.d_ff
+    planes = 2 if (w.hidden_split and w.dtype == "bf16") else 1
+    o = dict(
+        idx=torch.empty(T, k, dtype=torch.int32, device=dev),
+        gate=torch.empty(T, k, dtype=torch.float32, device=dev),
+        near=torch.empty(T, dtype=torch.uint8, device=dev),
+        counts=torch.empty(E, dtype=torch.int32, device=dev),
+        offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+        perm_src=torch.empty(T * k, dtype=torch.int32, device=dev),
+        slot_pos=torch.empty(T * k, dtype=torch.int32, device=dev),
+        x_perm=torch.empty(T * k, dm, dtype=w.torch_dtype, device=dev),
+        h=torch.empty(planes * T * k, f, dtype=w.torch_dtype, device=dev),
+        y_perm=torch.empty(T * k, dm, dtype=torch.float32, device=dev),
+        y=torch.empty(T, dm, dtype=torch.float32, device=dev))
+    noisy = w.gating == "noisy_topk"
+    o["importance"] = torch.empty(E, dtype=torch.float32, device=dev) if noisy else None
+    o["load"] = torch.empty(E, dtype=torch.float32, device=dev) if noisy and k < E else None
+    ws = moe.workspace(cfg, dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    launches = [0]
+
+    def step(evs=None):
+        n = 0
+        if evs:
+            evs[0].record(stream)
+        moe.moe_route(cfg, d["x"], d["w_gate"], o["idx"], o["gate"], ws, w_noise=d.get("w_noise"),
+                      noise=d.get("noise"), logit_bias=d.get("logit_bias"),
+                      importance=o["importance"], load=o["load"], near_tie=o["near"])
+        n += moe.last_launch_count()
+        if evs:
+            evs[1].record(stream)
+        moe.moe_permute(cfg, o["idx"], d["x"], o["counts"], o["offsets"], o["perm_src"],
+                        o["slot_pos"], o["x_perm"], ws)
+        n += moe.last_launch_count()
+        if evs:
+            evs[2].record(stream)
+        moe.moe_expert_ffn(cfg, o["x_perm"], o["offsets"], d["w1"], d["w2"], o["h"], o["y_perm"], ws)
+        n += moe.last_launch_count()
+        if evs:
+            evs[3].record(stream)
+        moe.moe_combine(cfg, o["y_perm"], o["slot_pos"], o["gate"], o["y"], ws)
+        n += moe.last_launch_count()
+        if evs:
+            evs[4].record(stream)
+        launches[0] += n
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize(dev)
+    err = moe.moe_get_error(ws)
+    if err:
+        raise RuntimeError("device error word %d after warm-up" % err)
+    offs = o["offsets"].cpu().tolist()
+    kept = [offs[e + 1] - offs[e] for e in range(E)]
+    n_kept = offs[-1]
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    launches[0] = 0
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            step(evs[i])
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)]
+                    for i in range(args.steps)])  # ms: route, permute, ffn, combine
+    step_ms = float(np.mean(per.sum(axis=1)))
+    step_ms_max = max_over_ranks(step_ms, dev)
+    err = moe.moe_get_error(ws)
+    if err:
+        raise RuntimeError("device error word %d after the timed steps" % err)
+
+    # ---- end to end through the fused public call, host buffers in pinned memory
+    layer = moe.MoELayer(cfg, {kk: v for kk, v in d.items() if kk not in ("x", "noise")}, device=dev)
+    x_host = inp["x"].pin_memory()
+    noise_host = inp["noise"].pin_memory() if noisy else None
+    y_host = torch.empty(T, dm, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(d["x"])
+    noise_dev = torch.empty_like(d["noise"]) if noisy else None
+    h2d = x_host.numel() * x_host.element_size() + (noise_host.numel() * 4 if noisy else 0)
+    d2h = y_host.numel() * 4
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        if noisy:
+            noise_dev.copy_(noise_host, non_blocking=True)
+        layer.forward(x_dev, noise=noise_dev)
+        y_host.copy_(layer.y, non_blocking=True)
+
+    for _ in range(max(3, args.warmup // 4)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e_steps = max(3, min(args.steps, 200))
+    e2e_ms = []
+    for i in range(e2e_steps):
+        flush.fill_(float(i))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    e2e_mean = max_over_ranks(float(np.mean(e2e_ms)), dev)
+    if not torch.equal(y_host, layer.y.cpu()):
+        raise RuntimeError("end-to-end output mismatch between host copy and device result")
+
+    peaks, peak_src = load_peaks()
+    alg = algorithmic(w, n_kept, kept)
+    ffn_ms = float(np.mean(per[:, 2]))
+    gemm_launch_s = ffn_ms * 1e-3 / 2.0
+    ffn_tflops = alg["ffn_flops"] / (ffn_ms * 1e-3) / 1e12
+    ffn_gbs = alg["ffn_bytes"] / (ffn_ms * 1e-3) / 1e9
+    ai = alg["ffn_flops"] / alg["ffn_bytes"]
+    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    traffic = recorded_traffic(w.name)
+    if ai < ridge:
+        roof = {"bound": "hbm", "achieved": ffn_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ffn_gbs / peaks["hbm_gbs"]}
+    else:
+        roof = {"bound": "tensor", "achieved": ffn_tflops, "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": ffn_tflops / peaks["bf16_tflops_sustained"]}
+    roof.update({"traffic": traffic, "kernel": "grouped_gemm_tc_kernel (2 launches/step)",
+                 "algorithmic_per_launch": {"flops": alg["ffn_flops"] / 2,
+                                            "bytes": alg["ffn_bytes"] / 2},
+                 "launch_ms": gemm_launch_s * 1e3, "peak_source": "%s (MEASURED_PEAKS.json)" % peak_src
+                 if peak_src == "measured" else "fallback"})
+
+    value = T * world / (step_ms_max * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded; random-init weights)", "config": config_json(w),
+        "roofline": roof,
+        "expert_gemm": {"tflops": ffn_tflops, "frac_of_bf16_peak": ffn_tflops / peaks["bf16_tflops"],
+                        "gbs": ffn_gbs, "frac_of_hbm": ffn_gbs / peaks["hbm_gbs"],
+                        "arith_intensity": ai},
+        "steps_ms": {"route": float(np.mean(per[:, 0])), "permute": float(np.mean(per[:, 1])),
+                     "expert_ffn": ffn_ms, "combine": float(np.mean(per[:, 3]))},
+        "step_gbs": {"route": alg["route_bytes"] / (np.mean(per[:, 0]) * 1e-3) / 1e9,
+                     "permute": alg["permute_bytes"] / (np.mean(per[:, 1]) * 1e-3) / 1e9,
+                     "combine": alg["combine_bytes"] / (np.mean(per[:, 3]) * 1e-3) / 1e9},
+        "kept_rows": n_kept,
+        "e2e": {"value": T * world / (e2e_mean * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_mean,
+                "call": "MoELayer.forward (moe_forward) with pinned host x/noise in, y out"},
+        "gpu_launches": launches[0],
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inp)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="switch", choices=list(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = workloads.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

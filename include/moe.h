@@ -30,8 +30,9 @@
  *    per output feature, contiguous along the contraction): the pages write x.W_g with
  *    W_g as [d_model, E]; w_gate here is its transpose [E, d_model].
  *  - Index tensors are int32.  Assignment a = t*k + j is token t's j-th choice.
- *  - Floating-point tensors of the layer (x, weights, x_perm, h, y_perm, y) are in
- *    cfg->dtype; gates, noise, logit_bias, importance and load are always fp32.
+ *  - x, the weights, x_perm and h are in cfg->dtype; the expert outputs y_perm, the
+ *    layer output y, gates, noise, logit_bias, importance and load are always fp32 (the
+ *    products accumulate in fp32 and are not rounded to bf16 on the way out).
  *  - T == 0 is valid: nothing is launched, the per-expert outputs that are given
  *    (counts, offsets, importance, load) are zero-filled on `stream`, and per-token
  *    pointers may be NULL.
@@ -99,7 +100,11 @@ typedef struct {
   int32_t renorm;         /* see moe_gating */
   float capacity_factor;  /* > 0: capacity C = ceil(cf*T*k/E) per expert; <= 0: none */
   int32_t act;            /* moe_act */
-  int32_t dtype;          /* moe_dtype of the layer tensors */
+  int32_t dtype;          /* moe_dtype of x, the weights, x_perm and h */
+  int32_t hidden_split;   /* bf16 only, 0 or 1: 1 carries the hidden activations h as two
+                             bf16 planes, hi = bf16(v) and lo = bf16(v - hi), and the
+                             down-projection accumulates both (about 16 significant bits
+                             instead of 8, for twice the down-projection MMA work) */
 } moe_config;
 
 /* Human-readable name of a status code (static string). */
@@ -161,22 +166,24 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
  *  offsets [E+1] int32 in (as written by moe_permute; any non-decreasing values in
  *          [0, T*k] are accepted)
  *  w1      [E, d_ff, d_model] dtype,  w2 [E, d_model, d_ff] dtype
- *  h       [T*k, d_ff] dtype out (hidden activations; rows < offsets[E] written)
- *  y_perm  [T*k, d_model] dtype out (rows < offsets[E] written)
- * bf16: tcgen05 tensor cores with fp32 accumulation; h and y_perm are rounded to bf16. */
+ *  h       [P*T*k, d_ff] dtype out (hidden activations; P = 2 when cfg->hidden_split,
+ *          with the remainder plane starting at row T*k; rows < offsets[E] written)
+ *  y_perm  [T*k, d_model] fp32 out (rows < offsets[E] written)
+ * bf16: tcgen05 tensor cores with fp32 accumulation; h is rounded to bf16 (plus its
+ * bf16 remainder in split mode).  fp32: FP32 FMA throughout. */
 moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
                           const void* w1, const void* w2, void* h, void* y_perm, void* ws,
                           moe_stream_t stream);
 
 /* Gate-weighted combine [Shazeer et al., "Methode": y = sum_i G(x)_i E_i(x)]:
  *   y[t] = sum_j topk_gate[t, j] * y_perm[slot_pos[t*k + j]]   (dropped slots add 0)
- *  y_perm [T*k, d_model] dtype, slot_pos [T*k] int32, topk_gate [T, k] fp32 in
- *  y      [T, d_model] dtype out; fp32 accumulation, one rounding to dtype. */
+ *  y_perm [T*k, d_model] fp32, slot_pos [T*k] int32, topk_gate [T, k] fp32 in
+ *  y      [T, d_model] fp32 out; accumulated in the order j = 0 .. k-1. */
 moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* slot_pos,
                        const float* topk_gate, void* y, void* ws, moe_stream_t stream);
 
 /* The whole layer forward on one stream: moe_route, moe_permute, moe_expert_ffn,
- * moe_combine.  Inputs as in the step calls; y [T, d_model] dtype out.  topk_idx,
+ * moe_combine.  Inputs as in the step calls; y [T, d_model] fp32 out.  topk_idx,
  * topk_gate (both [T, k]) and counts ([E]) are outputs the caller must provide;
  * importance, load and near_tie may be NULL.  The intermediates live in `ws`
  * (moe_forward_workspace_size bytes). */

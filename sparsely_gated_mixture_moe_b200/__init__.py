@@ -157,15 +157,15 @@ class MoELayer:
     """Owns the device buffers of one layer configuration and runs its forward pass.
 
     weights: dict with w_gate [E,d], w1 [E,f,d], w2 [E,d,f] (and w_noise [E,d] for noisy
-    gating, logit_bias [E] fp32 if used), CUDA tensors in the config's dtype.
+    gating, logit_bias [E] fp32 if used), CUDA tensors in the config's dtype.  The layer
+    output y [T, d] is fp32.
     """
 
     def __init__(self, cfg: MoEConfig, weights: dict, device="cuda"):
         self.cfg = cfg
         self.w = weights
         T, k, E, d = cfg.T, cfg.k, cfg.E, cfg.d_model
-        dt = torch.float32 if cfg.dtype == DTYPE["f32"] else torch.bfloat16
-        self.y = torch.empty(T, d, dtype=dt, device=device)
+        self.y = torch.empty(T, d, dtype=torch.float32, device=device)
         self.topk_idx = torch.empty(T, k, dtype=torch.int32, device=device)
         self.topk_gate = torch.empty(T, k, dtype=torch.float32, device=device)
         self.counts = torch.empty(E, dtype=torch.int32, device=device)

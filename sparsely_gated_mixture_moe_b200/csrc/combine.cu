@@ -2,8 +2,9 @@
 //
 // The layer output of Shazeer et al. ("Methode"): y = sum_i G(x)_i E_i(x), with only the
 // k chosen experts contributing and a dropped assignment (slot_pos = -1) adding nothing.
-// One warp per token; each lane handles 16-byte vectors of the row (8 bf16 or 4 fp32),
-// gathers the k expert rows, accumulates in fp32 and rounds once to the output dtype.
+// y_perm and y are fp32 for both layer dtypes (the expert outputs leave the tensor cores
+// as fp32 accumulators).  One warp per token; each lane handles 16-byte vectors of the
+// row, gathers the k expert rows and accumulates in fp32 in the order j = 0 .. k-1.
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,26 +23,6 @@ struct Vec<float> {
     *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
   }
 };
-template <>
-struct Vec<__nv_bfloat16> {
-  static constexpr int N = 8;
-  __device__ static void load(const void* p, float (&v)[8]) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
-      const float2 f = __bfloat1622float2(b);
-      v[2 * i] = f.x;
-      v[2 * i + 1] = f.y;
-    }
-  }
-  __device__ static void store(void* p, const float (&v)[8]) {
-    *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-  }
-};
-
 constexpr int kCombineWarps = 8;
 
 template <typename T>
@@ -91,14 +72,9 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
 cudaError_t launch_combine(const CombineProblem& p, const LaunchCtx& c) {
   const int64_t blocks = (p.T + kCombineWarps - 1) / kCombineWarps;
   if (blocks == 0) return cudaSuccess;
-  if (p.dtype == MOE_BF16)
-    combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), kCombineWarps * 32, 0, c.stream>>>(
-        static_cast<const __nv_bfloat16*>(p.y_perm), p.slot_pos, p.gate,
-        static_cast<__nv_bfloat16*>(p.y), p.T, p.k, p.d, c.err);
-  else
-    combine_kernel<float><<<static_cast<unsigned>(blocks), kCombineWarps * 32, 0, c.stream>>>(
-        static_cast<const float*>(p.y_perm), p.slot_pos, p.gate, static_cast<float*>(p.y), p.T,
-        p.k, p.d, c.err);
+  combine_kernel<float><<<static_cast<unsigned>(blocks), kCombineWarps * 32, 0, c.stream>>>(
+      static_cast<const float*>(p.y_perm), p.slot_pos, p.gate, static_cast<float*>(p.y), p.T,
+      p.k, p.d, c.err);
   ++*c.launches;
   return cudaGetLastError();
 }

@@ -3,13 +3,19 @@
 //   up:   h[s]      = act(x_perm[s] . W1_e^T)     [rows of e] x [d_ff, d_model]^T
 //   down: y_perm[s] = h[s] . W2_e^T               [rows of e] x [d_model, d_ff]^T
 //
+// h is bf16 (the operand type of the second product).  In split mode the up-projection
+// also stores the rounding remainder lo = bf16(v - hi) as a second plane and the
+// down-projection accumulates hi.W2^T + lo.W2^T in the same TMEM accumulator (two MMAs
+// per k-step sharing the W2 tile), so h carries about 16 significant bits.  y_perm is
+// fp32.
+//
 // Experts are the feed-forward sub-networks of the sparsely-gated MoE layer (Shazeer et
 // al., "Schlüsselbegriffe"); each runs only on the rows routed to it ("Methode": no
 // computation where G(x)_i = 0).  Expert e owns permuted rows [offsets[e], offsets[e+1]).
 //
 // Kernel design (one CTA per SM, persistent):
-//   warp 0      TMA producer: A tile [128 x 64] and B tile [BN x 64] per k-block into a
-//               4-stage ring of 128-byte-swizzled shared-memory buffers.
+//   warp 0      TMA producer: A tile(s) [128 x 64] and B tile [BN x 64] per k-block into
+//               a 4-stage (3 with two A planes) ring of 128-byte-swizzled buffers.
 //   warp 1      TMEM owner and MMA issuer: one thread issues tcgen05.mma (M=128, N=BN,
 //               K=16) into one of two TMEM accumulators (2 x 256 fp32 columns), and
 //               tcgen05.commit releases smem stages and hands finished accumulators on.
@@ -34,15 +40,21 @@ namespace gg {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int STAGES = 4;
+constexpr int MAX_STAGES = 4;
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + EPI_WARPS * 32;
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
 constexpr int B_BYTES_MAX = 256 * BK * 2;   // 32 KB
 constexpr int MAX_GROUPS = 1024;
 constexpr int TMEM_COLS = 512;              // two accumulators of up to 256 columns
-constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_BYTES + B_BYTES_MAX) +
-                           256 /*barriers, flags*/ + 4 * (MAX_GROUPS + 1 + 40);
+constexpr int RING_BYTES = 196608;           // 4 x (16 + 32) KB, or 3 x (2 x 16 + 32) KB
+constexpr int SMEM_BYTES = 1024 /*align slack*/ + RING_BYTES + 256 /*barriers, flags*/ +
+                           4 * (MAX_GROUPS + 1 + 40);
+
+// Epilogue output modes.
+constexpr int OUT_BF16 = 0;        // act, bf16
+constexpr int OUT_BF16_SPLIT = 1;  // act, bf16 hi plane + bf16 remainder plane
+constexpr int OUT_F32 = 2;         // fp32
 
 struct Args {
   const int32_t* offsets;
@@ -52,8 +64,11 @@ struct Args {
   int bn;        // N tile: 256, 128 or 64 (divides N)
   int n_tiles;   // N / bn
   int64_t rows_cap;
-  __nv_bfloat16* out;
+  void* out;
   int act;       // 0 none, 1 ReLU, 2 GELU
+  int out_mode;  // OUT_*
+  int n_a;       // A planes: 1, or 2 (hi and lo rows at row and rows_cap + row)
+  int stages;
   int* err;
 };
 
@@ -86,18 +101,20 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES_MAX);
-  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+  // stage s: A plane(s) at ring + s * stage_bytes, then the B tile
+  const int STAGES = a.stages;
+  const int stage_bytes = a.n_a * A_BYTES + B_BYTES_MAX;
+  uint8_t* ring = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RING_BYTES);
+  // bars: full[MAX_STAGES], empty[MAX_STAGES], tfull[2], tempty[2], drain
   const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = smem_u32(bars + STAGES);
-  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
-  const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
-  const uint32_t drain = smem_u32(bars + 2 * STAGES + 4);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  const uint32_t empty0 = smem_u32(bars + MAX_STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * MAX_STAGES);
+  const uint32_t tempty0 = smem_u32(bars + 2 * MAX_STAGES + 2);
+  const uint32_t drain = smem_u32(bars + 2 * MAX_STAGES + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * MAX_STAGES + 5);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  int* scratch = reinterpret_cast<int*>(smem + STAGES * (A_BYTES + B_BYTES_MAX) + 256);
+  int* scratch = reinterpret_cast<int*>(smem + RING_BYTES + 256);
   int* tp = scratch + 40;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -132,6 +149,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int total = ok ? tp[a.E] * a.n_tiles : 0;
   const int kblocks = a.K / BK;
   const uint32_t b_bytes = static_cast<uint32_t>(a.bn) * BK * 2;
+  const int plane_rows = static_cast<int>(a.rows_cap);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -147,9 +165,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             aborted = true;
             break;
           }
-          mbar_arrive_expect_tx(full0 + 8 * stage, A_BYTES + b_bytes);
-          tma_load_2d(smem_u32(sA + stage * A_BYTES), &tmA, full0 + 8 * stage, kb * BK, t.row0);
-          tma_load_2d(smem_u32(sB + stage * B_BYTES_MAX), &tmB, full0 + 8 * stage, kb * BK, brow);
+          uint8_t* st = ring + stage * stage_bytes;
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, a.n_a * A_BYTES + b_bytes);
+          tma_load_2d(smem_u32(st), &tmA, fb, kb * BK, t.row0);
+          if (a.n_a == 2) tma_load_2d(smem_u32(st + A_BYTES), &tmA, fb, kb * BK, t.row0 + plane_rows);
+          tma_load_2d(smem_u32(st + a.n_a * A_BYTES), &tmB, fb, kb * BK, brow);
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -186,12 +207,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
-          const uint32_t b0 = smem_u32(sB + stage * B_BYTES_MAX);
+          const uint32_t a0 = smem_u32(ring + stage * stage_bytes);
+          const uint32_t b0 = a0 + a.n_a * A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            tc_mma_bf16(d_tmem, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32), idesc,
-                        (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t bd = sdesc_k128(b0 + kk * 32);
+            tc_mma_bf16(d_tmem, sdesc_k128(a0 + kk * 32), bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            if (a.n_a == 2) tc_mma_bf16(d_tmem, sdesc_k128(a0 + A_BYTES + kk * 32), bd, idesc, 1u);
+          }
           tc_commit(empty0 + 8 * stage);
           if (++stage == STAGES) {
             stage = 0;
@@ -227,8 +250,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const int r = q * 32 + lane;
       const bool row_ok = r < t.valid;
-      __nv_bfloat16* orow =
-          a.out + static_cast<int64_t>(t.row0 + r) * a.N + t.nt * a.bn + half * cols;
+      const int64_t oidx = static_cast<int64_t>(t.row0 + r) * a.N + t.nt * a.bn + half * cols;
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256 + half * cols;
       for (int c = 0; c < cols; c += 32) {
@@ -236,16 +258,37 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld32(tbase + c, v);
         tmem_ld_wait();
         if (row_ok) {
-          uint32_t packed[16];
+          if (a.out_mode == OUT_F32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + oidx + c);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            packed[j] = pack_bf16x2(apply_act(__uint_as_float(v[2 * j]), a.act),
-                                    apply_act(__uint_as_float(v[2 * j + 1]), a.act));
-          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+            for (int j = 0; j < 8; ++j)
+              dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                   __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+          } else {
+            float f[32];
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
-                                packed[4 * j + 3]);
+            for (int j = 0; j < 32; ++j) f[j] = apply_act(__uint_as_float(v[j]), a.act);
+            uint32_t hi[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) hi[j] = pack_bf16x2(f[2 * j], f[2 * j + 1]);
+            __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + oidx + c;
+            uint4* dst = reinterpret_cast<uint4*>(ob);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
+            if (a.out_mode == OUT_BF16_SPLIT) {
+              uint32_t lo[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const float2 h2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi[j]));
+                lo[j] = pack_bf16x2(f[2 * j] - h2.x, f[2 * j + 1] - h2.y);
+              }
+              uint4* dlo = reinterpret_cast<uint4*>(ob + a.rows_cap * a.N);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                dlo[j] = make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
+            }
+          }
         }
       }
       tc_fence_before();
@@ -301,11 +344,13 @@ static int pick_bn(int N) {
   return 64;
 }
 
-static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void* B, int E, int N,
-                              void* out, const int32_t* offsets, int act, const LaunchCtx& c) {
+static cudaError_t launch_one(const void* A, int n_a, int64_t rows_cap, int K, const void* B, int E,
+                              int N, void* out, int out_mode, const int32_t* offsets, int act,
+                              const LaunchCtx& c) {
   const int bn = pick_bn(N);
   CUtensorMap tmA, tmB;
-  if (!make_tmap_bf16(&tmA, A, static_cast<uint64_t>(rows_cap), K, gg::BM)) return cudaErrorInvalidValue;
+  // with two A planes the map spans both: lo rows sit rows_cap rows below hi rows
+  if (!make_tmap_bf16(&tmA, A, static_cast<uint64_t>(rows_cap) * n_a, K, gg::BM)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16(&tmB, B, static_cast<uint64_t>(E) * N, K, bn)) return cudaErrorInvalidValue;
   gg::Args a;
   a.offsets = offsets;
@@ -315,8 +360,11 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
   a.bn = bn;
   a.n_tiles = N / bn;
   a.rows_cap = rows_cap;
-  a.out = static_cast<__nv_bfloat16*>(out);
+  a.out = out;
   a.act = act;
+  a.out_mode = out_mode;
+  a.n_a = n_a;
+  a.stages = gg::RING_BYTES / (n_a * gg::A_BYTES + gg::B_BYTES_MAX);
   a.err = c.err;
   // upper bound of the tile count: sum_e ceil(n_e / BM) <= rows_cap / BM + E
   const int64_t max_tiles = (rows_cap / gg::BM + E) * static_cast<int64_t>(a.n_tiles);
@@ -332,9 +380,11 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
 
 cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c) {
   if (p.E > gg::MAX_GROUPS) return cudaErrorInvalidValue;
-  cudaError_t e = launch_one(p.x_perm, p.rows_cap, p.d, p.w1, p.E, p.f, p.h, p.offsets, p.act, c);
+  const int planes = p.hidden_split ? 2 : 1;
+  cudaError_t e = launch_one(p.x_perm, 1, p.rows_cap, p.d, p.w1, p.E, p.f, p.h,
+                             p.hidden_split ? gg::OUT_BF16_SPLIT : gg::OUT_BF16, p.offsets, p.act, c);
   if (e != cudaSuccess) return e;
-  return launch_one(p.h, p.rows_cap, p.f, p.w2, p.E, p.d, p.y_perm, p.offsets, 0, c);
+  return launch_one(p.h, planes, p.rows_cap, p.f, p.w2, p.E, p.d, p.y_perm, gg::OUT_F32, p.offsets, 0, c);
 }
 
 }  // namespace moe

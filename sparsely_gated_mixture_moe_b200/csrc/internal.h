@@ -64,6 +64,7 @@ cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c);
 struct FfnProblem {
   int64_t rows_cap;  // T*k
   int d, f, E, act;  // act: 1 ReLU, 2 GELU
+  int hidden_split;  // bf16 path: h carried as a hi plane plus a remainder plane
   const void* x_perm;
   const int32_t* offsets;
   const void* w1;
@@ -83,7 +84,7 @@ cudaError_t launch_sgemm_grouped(const float* A, const float* B, float* out,
 // ---- combine ---------------------------------------------------------------------
 struct CombineProblem {
   int64_t T;
-  int k, d, dtype;
+  int k, d;
   const void* y_perm;
   const int32_t* slot_pos;
   const float* gate;

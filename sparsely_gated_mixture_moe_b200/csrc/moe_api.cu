@@ -16,6 +16,7 @@ size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int esize(const moe_config* c) { return c->dtype == MOE_BF16 ? 2 : 4; }
+int hidden_planes(const moe_config* c) { return (c->dtype == MOE_BF16 && c->hidden_split) ? 2 : 1; }
 
 // Structural validity of the config (MOE_ERR_INVALID_ARG) and supported shapes
 // (MOE_ERR_UNSUPPORTED).
@@ -27,6 +28,7 @@ moe_status check_config(const moe_config* c) {
   if (c->act != MOE_ACT_RELU && c->act != MOE_ACT_GELU) return MOE_ERR_INVALID_ARG;
   if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (!(c->capacity_factor == c->capacity_factor)) return MOE_ERR_INVALID_ARG;  // NaN
+  if (c->hidden_split != 0 && c->hidden_split != 1) return MOE_ERR_INVALID_ARG;
   if (c->k > 8) return MOE_ERR_UNSUPPORTED;
   if (c->T * static_cast<int64_t>(c->k) >= (int64_t{1} << 31)) return MOE_ERR_UNSUPPORTED;
   if (c->T * static_cast<int64_t>(c->E) >= (int64_t{1} << 31)) return MOE_ERR_UNSUPPORTED;
@@ -71,9 +73,9 @@ Layout layout(const moe_config* c) {
   L.x_perm = o;
   o = align_up(o + static_cast<size_t>(n) * c->d_model * esize(c));
   L.h = o;
-  o = align_up(o + static_cast<size_t>(n) * c->d_ff * esize(c));
+  o = align_up(o + static_cast<size_t>(n) * c->d_ff * esize(c) * hidden_planes(c));
   L.y_perm = o;
-  o = align_up(o + static_cast<size_t>(n) * c->d_model * esize(c));
+  o = align_up(o + static_cast<size_t>(n) * c->d_model * 4);
   L.forward = o;
   return L;
 }
@@ -187,6 +189,7 @@ moe_status do_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offs
   p.f = cfg->d_ff;
   p.E = cfg->E;
   p.act = cfg->act == MOE_ACT_GELU ? 2 : 1;
+  p.hidden_split = hidden_planes(cfg) == 2;
   p.x_perm = x_perm;
   p.offsets = offsets;
   p.w1 = w1;
@@ -203,7 +206,6 @@ moe_status do_combine(const moe_config* cfg, const void* y_perm, const int32_t* 
   p.T = cfg->T;
   p.k = cfg->k;
   p.d = cfg->d_model;
-  p.dtype = cfg->dtype;
   p.y_perm = y_perm;
   p.slot_pos = slot_pos;
   p.gate = gate;

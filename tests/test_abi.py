@@ -30,10 +30,11 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_config_struct_layout():
-    # int64 T, six int32, float, two int32 -> 48 bytes with 8-byte alignment
+    # int64 T, six int32, float, three int32 -> 48 bytes with 8-byte alignment
     assert ctypes.sizeof(moe.MoEConfig) == 48
     assert moe.MoEConfig.capacity_factor.offset == 32
     assert moe.MoEConfig.dtype.offset == 40
+    assert moe.MoEConfig.hidden_split.offset == 44
 
 
 def test_status_strings():
@@ -88,6 +89,9 @@ def test_route_validation():
     assert _route(bad) == 1
     bad = _cfg()
     bad.T = -1
+    assert _route(bad) == 1
+    bad = _cfg()
+    bad.hidden_split = 2
     assert _route(bad) == 1
     assert moe.lib.moe_route(None, FAKE, FAKE, None, None, None, FAKE, FAKE, None, None, None,
                              FAKE, None) == 1

@@ -39,6 +39,8 @@ SMALL = {
     "k_equals_E": Workload("kE", T=200, d_model=64, d_ff=128, E=4, k=4, act="gelu"),
     "one_token": Workload("t1", T=1, d_model=64, d_ff=64, E=8, k=2),
     "E8_bf16_pad": Workload("e8", T=500, d_model=64, d_ff=64, E=8, k=2),
+    "split_multitile": Workload("sp", T=3000, d_model=192, d_ff=384, E=6, k=2, act="gelu",
+                                hidden_split=True, capacity_factor=0.9),
 }
 
 
@@ -60,8 +62,7 @@ def test_steps_and_forward_small(name):
     # the fused call runs the same kernels: identical results
     assert torch.equal(f["topk_idx"], g["topk_idx"])
     assert torch.equal(f["counts"], g["counts"])
-    assert torch.equal(f["y"].view(torch.int16) if w.dtype == "bf16" else f["y"], 
-                       g["y"].view(torch.int16) if w.dtype == "bf16" else g["y"])
+    assert torch.equal(f["y"], g["y"])
     print(name, rep)
 
 
@@ -156,5 +157,5 @@ def test_full_size_sampled(name):
     H.check_end_to_end(w, inp, g, idx, gates, rep, rows=toks)
     f = H.run_forward(w, dev)
     assert f["device_error"] == 0
-    assert torch.equal(f["y"].view(torch.int16), g["y"].view(torch.int16))
+    assert torch.equal(f["y"], g["y"])
     print(name, rep)
