@@ -244,7 +244,7 @@ def config_json(w):
         "" if w.gating == "noisy_topk" else ("(renorm)" if w.renorm else "(full-softmax gate)"),
         w.capacity_factor, w.act, w.dtype),
         "T": w.T, "d_model": w.d_model, "d_ff": w.d_ff, "E": w.E, "k": w.k,
-        "capacity_factor": w.capacity_factor, "hidden_split": w.hidden_split,
+        "capacity_factor": w.capacity_factor, "hidden_f16": w.hidden_f16,
         "l2": "flushed before every timed step (256 MB write)",
         "parallelism": "replicas"}
     return c
@@ -267,9 +267,9 @@ def run_gpu(args, w):
     d = {k: v.to(dev) for k, v in inp.items()}
     cfg = moe.make_config(w.T, w.d_model, w.d_ff, w.E, w.k, gating=w.gating, renorm=w.renorm,
                           capacity_factor=w.capacity_factor, act=w.act, dtype=w.dtype,
-                          hidden_split=w.hidden_split)
+                          hidden_f16=w.hidden_f16)
+    d = moe.prepare_weights(cfg, d)     # fp16 w2 for fp16 hidden activations (exact re-encoding)
     T, k, E, dm, f = w.T, w.k, w.E, w.d_model, w.d_ff
-    planes = 2 if (w.hidden_split and w.dtype == "bf16") else 1
     o = dict(
         idx=torch.empty(T, k, dtype=torch.int32, device=dev),
         gate=torch.empty(T, k, dtype=torch.float32, device=dev),
@@ -279,7 +279,7 @@ def run_gpu(args, w):
         perm_src=torch.empty(T * k, dtype=torch.int32, device=dev),
         slot_pos=torch.empty(T * k, dtype=torch.int32, device=dev),
         x_perm=torch.empty(T * k, dm, dtype=w.torch_dtype, device=dev),
-        h=torch.empty(planes * T * k, f, dtype=w.torch_dtype, device=dev),
+        h=torch.empty(T * k, f, dtype=torch.float16 if w.hidden_f16 else w.torch_dtype, device=dev),
         y_perm=torch.empty(T * k, dm, dtype=torch.float32, device=dev),
         y=torch.empty(T, dm, dtype=torch.float32, device=dev))
     noisy = w.gating == "noisy_topk"

@@ -101,10 +101,11 @@ typedef struct {
   float capacity_factor;  /* > 0: capacity C = ceil(cf*T*k/E) per expert; <= 0: none */
   int32_t act;            /* moe_act */
   int32_t dtype;          /* moe_dtype of x, the weights, x_perm and h */
-  int32_t hidden_split;   /* bf16 only, 0 or 1: 1 carries the hidden activations h as two
-                             bf16 planes, hi = bf16(v) and lo = bf16(v - hi), and the
-                             down-projection accumulates both (about 16 significant bits
-                             instead of 8, for twice the down-projection MMA work) */
+  int32_t hidden_f16;     /* bf16 only, 0 or 1: 1 stores the hidden activations h in fp16
+                             (11 significant bits instead of 8) and takes w2 in fp16, since
+                             both operands of one tensor-core product share a type; a bf16
+                             w2 converts to fp16 exactly wherever |w| >= 2^-17 (see
+                             moe_bf16_to_f16).  Needs |h| < 65504. */
 } moe_config;
 
 /* Human-readable name of a status code (static string). */
@@ -166,11 +167,11 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
  *  offsets [E+1] int32 in (as written by moe_permute; any non-decreasing values in
  *          [0, T*k] are accepted)
  *  w1      [E, d_ff, d_model] dtype,  w2 [E, d_model, d_ff] dtype
- *  h       [P*T*k, d_ff] dtype out (hidden activations; P = 2 when cfg->hidden_split,
- *          with the remainder plane starting at row T*k; rows < offsets[E] written)
+ *  h       [T*k, d_ff] out (hidden activations; rows < offsets[E] written): dtype, or
+ *          fp16 when cfg->hidden_f16
  *  y_perm  [T*k, d_model] fp32 out (rows < offsets[E] written)
- * bf16: tcgen05 tensor cores with fp32 accumulation; h is rounded to bf16 (plus its
- * bf16 remainder in split mode).  fp32: FP32 FMA throughout. */
+ * w2 is fp16 when cfg->hidden_f16, else dtype.  bf16: tcgen05 tensor cores with fp32
+ * accumulation; h is rounded once to its storage type.  fp32: FP32 FMA throughout. */
 moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
                           const void* w1, const void* w2, void* h, void* y_perm, void* ws,
                           moe_stream_t stream);
@@ -197,6 +198,17 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_gate,
  * (may be NULL) and clears it.  Returns MOE_OK if no bit was set, MOE_ERR_DEVICE if
  * some were, MOE_ERR_CUDA if the synchronisation or copy failed. */
 moe_status moe_get_error(void* ws, moe_stream_t stream, int32_t* device_error);
+
+/* Re-encodes n bf16 values as fp16 (round to nearest even), e.g. w2 for
+ * cfg->hidden_f16.  fp16's 11 significant bits hold every bf16 value of magnitude in
+ * [2^-17, 65504] exactly; smaller magnitudes round to fp16's subnormal grid (absolute
+ * error <= 2^-25) and larger ones to +-inf.
+ *  src        [n] bf16 device in;  dst [n] fp16 device out (may not alias src)
+ *  n_inexact  device int32 or NULL: incremented by the number of values not converted
+ *             exactly
+ * Weight preparation, run once before the forward passes that use it. */
+moe_status moe_bf16_to_f16(const void* src, void* dst, int64_t n, int32_t* n_inexact,
+                           moe_stream_t stream);
 
 /* Number of kernels the most recent successful call on this host thread queued. */
 int32_t moe_last_launch_count(void);

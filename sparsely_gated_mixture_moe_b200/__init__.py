@@ -6,7 +6,7 @@ torch tensors, the stream handle, the config struct) and turns status codes into
 exceptions.  There is no CPU fallback: importing fails loudly when libmoe.so has not
 been built, and every call requires CUDA tensors.
 
-    python -m sparsely_gated_mixture_moe_b200.build_lib      # build libmoe.so in-tree
+    python sparsely_gated_mixture_moe_b200/build_lib.py      # build libmoe.so in-tree
 """
 from __future__ import annotations
 
@@ -25,7 +25,7 @@ def _load():
     if not os.path.exists(_LIB_PATH):
         raise ImportError(
             "libmoe.so is not built (expected at %s); build it with "
-            "`python -m sparsely_gated_mixture_moe_b200.build_lib`" % _LIB_PATH)
+            "`python sparsely_gated_mixture_moe_b200/build_lib.py`" % _LIB_PATH)
     lib = ctypes.CDLL(_LIB_PATH)
     P = ctypes.c_void_p
     C = ctypes.POINTER(MoEConfig)
@@ -41,6 +41,7 @@ def _load():
         "moe_forward": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]),
         "moe_get_error": (ctypes.c_int, [P, P, ctypes.POINTER(ctypes.c_int32)]),
         "moe_last_launch_count": (ctypes.c_int32, []),
+        "moe_bf16_to_f16": (ctypes.c_int, [P, P, ctypes.c_int64, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -148,6 +149,26 @@ def moe_get_error(ws: torch.Tensor, stream=None) -> int:
     return int(v.value)
 
 
+def moe_bf16_to_f16(src: torch.Tensor, dst: torch.Tensor, n_inexact=None, stream=None):
+    """Re-encode a bf16 CUDA tensor as fp16 into `dst` (same shape); `n_inexact` (an int32
+    CUDA tensor of one element, or None) is incremented by the values not kept exactly."""
+    if src.dtype != torch.bfloat16 or dst.dtype != torch.float16 or src.shape != dst.shape:
+        raise ValueError("moe_bf16_to_f16 needs a bf16 source and an fp16 destination of one shape")
+    _check(lib.moe_bf16_to_f16(_ptr(src, "src"), _ptr(dst, "dst"), src.numel(),
+                               _ptr(n_inexact, "n_inexact"), _stream(stream)), "moe_bf16_to_f16")
+
+
+def prepare_weights(cfg: MoEConfig, weights: dict, stream=None) -> dict:
+    """Weights as the forward pass takes them: with cfg.hidden_f16, w2 re-encoded to fp16
+    by the library (the other tensors are passed through)."""
+    out = dict(weights)
+    if cfg.hidden_f16 and cfg.dtype == DTYPE["bf16"] and weights["w2"].dtype == torch.bfloat16:
+        w2 = torch.empty(weights["w2"].shape, dtype=torch.float16, device=weights["w2"].device)
+        moe_bf16_to_f16(weights["w2"], w2, stream=stream)
+        out["w2"] = w2
+    return out
+
+
 def last_launch_count() -> int:
     """Kernels queued by the most recent successful call on this thread."""
     return int(lib.moe_last_launch_count())
@@ -163,7 +184,7 @@ class MoELayer:
 
     def __init__(self, cfg: MoEConfig, weights: dict, device="cuda"):
         self.cfg = cfg
-        self.w = weights
+        self.w = prepare_weights(cfg, weights)
         T, k, E, d = cfg.T, cfg.k, cfg.E, cfg.d_model
         self.y = torch.empty(T, d, dtype=torch.float32, device=device)
         self.topk_idx = torch.empty(T, k, dtype=torch.int32, device=device)
@@ -187,4 +208,5 @@ class MoELayer:
 __all__ = ["ACT", "DTYPE", "GATING", "MoEConfig", "MoEError", "MoELayer", "STATUS", "lib",
            "make_config", "moe_capacity", "moe_combine", "moe_expert_ffn", "moe_forward",
            "moe_forward_workspace_size", "moe_get_error", "moe_permute", "moe_route",
-           "moe_workspace_size", "workspace", "last_launch_count"]
+           "moe_workspace_size", "workspace", "last_launch_count", "moe_bf16_to_f16",
+           "prepare_weights"]

@@ -1,6 +1,8 @@
 """Build libmoe.so (the CUDA kernels and the C ABI) in-tree for sm_100a with nvcc.
 
-    python -m sparsely_gated_mixture_moe_b200.build_lib [--verbose-ptxas]
+    python sparsely_gated_mixture_moe_b200/build_lib.py [--verbose-ptxas]
+
+(run it as a script: importing the package loads the library it builds)
 
 Objects go to _build/ at the repository root; the shared library lands next to this
 file, where the Python binding loads it from.

@@ -29,14 +29,14 @@ class MoEConfig(ctypes.Structure):
         ("capacity_factor", ctypes.c_float),
         ("act", ctypes.c_int32),
         ("dtype", ctypes.c_int32),
-        ("hidden_split", ctypes.c_int32),
+        ("hidden_f16", ctypes.c_int32),
     ]
 
 
 def make_config(T, d_model, d_ff, E, k, gating="softmax_topk", renorm=True,
-                capacity_factor=None, act="relu", dtype="bf16", hidden_split=False) -> MoEConfig:
+                capacity_factor=None, act="relu", dtype="bf16", hidden_f16=False) -> MoEConfig:
     """Build a MoEConfig from plain values (capacity_factor None = no limit)."""
     return MoEConfig(T=T, d_model=d_model, d_ff=d_ff, E=E, k=k, gating=GATING[gating],
                      renorm=1 if renorm else 0,
                      capacity_factor=0.0 if capacity_factor is None else float(capacity_factor),
-                     act=ACT[act], dtype=DTYPE[dtype], hidden_split=1 if hidden_split else 0)
+                     act=ACT[act], dtype=DTYPE[dtype], hidden_f16=1 if hidden_f16 else 0)

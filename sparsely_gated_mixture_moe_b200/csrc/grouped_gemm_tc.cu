@@ -3,25 +3,24 @@
 //   up:   h[s]      = act(x_perm[s] . W1_e^T)     [rows of e] x [d_ff, d_model]^T
 //   down: y_perm[s] = h[s] . W2_e^T               [rows of e] x [d_model, d_ff]^T
 //
-// h is bf16 (the operand type of the second product).  In split mode the up-projection
-// also stores the rounding remainder lo = bf16(v - hi) as a second plane and the
-// down-projection accumulates hi.W2^T + lo.W2^T in the same TMEM accumulator (two MMAs
-// per k-step sharing the W2 tile), so h carries about 16 significant bits.  y_perm is
-// fp32.
+// h is stored in the operand type of the second product: bf16, or fp16 when W2 is given
+// in fp16 (11 instead of 8 significant bits for h; A and B of one MMA always share a
+// type).  y_perm is fp32.
 //
 // Experts are the feed-forward sub-networks of the sparsely-gated MoE layer (Shazeer et
 // al., "Schlüsselbegriffe"); each runs only on the rows routed to it ("Methode": no
 // computation where G(x)_i = 0).  Expert e owns permuted rows [offsets[e], offsets[e+1]).
 //
 // Kernel design (one CTA per SM, persistent):
-//   warp 0      TMA producer: A tile(s) [128 x 64] and B tile [BN x 64] per k-block into
-//               a 4-stage (3 with two A planes) ring of 128-byte-swizzled buffers.
+//   warp 0      TMA producer: A tile [128 x 64] and B tile [BN x 64] per k-block into a
+//               4-stage ring of 128-byte-swizzled shared-memory buffers.
 //   warp 1      TMEM owner and MMA issuer: one thread issues tcgen05.mma (M=128, N=BN,
 //               K=16) into one of two TMEM accumulators (2 x 256 fp32 columns), and
 //               tcgen05.commit releases smem stages and hands finished accumulators on.
 //   warps 2-9   epilogue: tcgen05.ld of the accumulator (each warp reads its 32-lane
-//               quarter, half of the columns), activation, bf16 rounding, stores of the
-//               rows that belong to the expert (a ragged tail is masked).
+//               quarter, half of the columns), activation, rounding to bf16/fp16 (or fp32
+//               as is), stores of the rows that belong to the expert (a ragged tail is
+//               masked).
 // Tiles are (expert, n-tile, m-tile) with m innermost, so CTAs running at the same time
 // share weight tiles through L2 and each expert's weights stream from HBM about once.
 // Rows past an expert's end that a 128-row tile reads belong to the next expert or lie
@@ -40,21 +39,22 @@ namespace gg {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int MAX_STAGES = 4;
+constexpr int STAGES = 4;
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 64 + EPI_WARPS * 32;
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
 constexpr int B_BYTES_MAX = 256 * BK * 2;   // 32 KB
 constexpr int MAX_GROUPS = 1024;
 constexpr int TMEM_COLS = 512;              // two accumulators of up to 256 columns
-constexpr int RING_BYTES = 196608;           // 4 x (16 + 32) KB, or 3 x (2 x 16 + 32) KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES_MAX;
+constexpr int RING_BYTES = STAGES * STAGE_BYTES;  // 192 KB
 constexpr int SMEM_BYTES = 1024 /*align slack*/ + RING_BYTES + 256 /*barriers, flags*/ +
                            4 * (MAX_GROUPS + 1 + 40);
 
 // Epilogue output modes.
-constexpr int OUT_BF16 = 0;        // act, bf16
-constexpr int OUT_BF16_SPLIT = 1;  // act, bf16 hi plane + bf16 remainder plane
-constexpr int OUT_F32 = 2;         // fp32
+constexpr int OUT_BF16 = 0;  // act, bf16
+constexpr int OUT_F16 = 1;   // act, fp16
+constexpr int OUT_F32 = 2;   // fp32
 
 struct Args {
   const int32_t* offsets;
@@ -67,8 +67,7 @@ struct Args {
   void* out;
   int act;       // 0 none, 1 ReLU, 2 GELU
   int out_mode;  // OUT_*
-  int n_a;       // A planes: 1, or 2 (hi and lo rows at row and rows_cap + row)
-  int stages;
+  int ab_f16;    // operand type of A and B: 1 fp16, 0 bf16
   int* err;
 };
 
@@ -101,18 +100,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  // stage s: A plane(s) at ring + s * stage_bytes, then the B tile
-  const int STAGES = a.stages;
-  const int stage_bytes = a.n_a * A_BYTES + B_BYTES_MAX;
+  // stage s: A tile at ring + s * STAGE_BYTES, then the B tile
   uint8_t* ring = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RING_BYTES);
-  // bars: full[MAX_STAGES], empty[MAX_STAGES], tfull[2], tempty[2], drain
+  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
   const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = smem_u32(bars + MAX_STAGES);
-  const uint32_t tfull0 = smem_u32(bars + 2 * MAX_STAGES);
-  const uint32_t tempty0 = smem_u32(bars + 2 * MAX_STAGES + 2);
-  const uint32_t drain = smem_u32(bars + 2 * MAX_STAGES + 4);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * MAX_STAGES + 5);
+  const uint32_t empty0 = smem_u32(bars + STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
+  const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
+  const uint32_t drain = smem_u32(bars + 2 * STAGES + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* scratch = reinterpret_cast<int*>(smem + RING_BYTES + 256);
   int* tp = scratch + 40;
@@ -149,7 +146,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int total = ok ? tp[a.E] * a.n_tiles : 0;
   const int kblocks = a.K / BK;
   const uint32_t b_bytes = static_cast<uint32_t>(a.bn) * BK * 2;
-  const int plane_rows = static_cast<int>(a.rows_cap);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -165,12 +161,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             aborted = true;
             break;
           }
-          uint8_t* st = ring + stage * stage_bytes;
+          uint8_t* st = ring + stage * STAGE_BYTES;
           const uint32_t fb = full0 + 8 * stage;
-          mbar_arrive_expect_tx(fb, a.n_a * A_BYTES + b_bytes);
+          mbar_arrive_expect_tx(fb, A_BYTES + b_bytes);
           tma_load_2d(smem_u32(st), &tmA, fb, kb * BK, t.row0);
-          if (a.n_a == 2) tma_load_2d(smem_u32(st + A_BYTES), &tmA, fb, kb * BK, t.row0 + plane_rows);
-          tma_load_2d(smem_u32(st + a.n_a * A_BYTES), &tmB, fb, kb * BK, brow);
+          tma_load_2d(smem_u32(st + A_BYTES), &tmB, fb, kb * BK, brow);
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -190,7 +185,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_bf16_f32(BM, a.bn);
+      const uint32_t idesc = idesc_f32acc(BM, a.bn, a.ab_f16 ? kFmtF16 : kFmtBF16);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool aborted = false;
@@ -207,14 +202,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(ring + stage * stage_bytes);
-          const uint32_t b0 = a0 + a.n_a * A_BYTES;
+          const uint32_t a0 = smem_u32(ring + stage * STAGE_BYTES);
+          const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t bd = sdesc_k128(b0 + kk * 32);
-            tc_mma_bf16(d_tmem, sdesc_k128(a0 + kk * 32), bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-            if (a.n_a == 2) tc_mma_bf16(d_tmem, sdesc_k128(a0 + A_BYTES + kk * 32), bd, idesc, 1u);
-          }
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_f16kind(d_tmem, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32), idesc,
+                           (kb | kk) != 0 ? 1u : 0u);
           tc_commit(empty0 + 8 * stage);
           if (++stage == STAGES) {
             stage = 0;
@@ -265,29 +258,22 @@ __global__ void __launch_bounds__(THREADS, 1)
               dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                                    __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
           } else {
-            float f[32];
+            uint32_t pk[16];
+            if (a.out_mode == OUT_F16) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) f[j] = apply_act(__uint_as_float(v[j]), a.act);
-            uint32_t hi[16];
+              for (int j = 0; j < 16; ++j)
+                pk[j] = pack_f16x2(apply_act(__uint_as_float(v[2 * j]), a.act),
+                                   apply_act(__uint_as_float(v[2 * j + 1]), a.act));
+            } else {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) hi[j] = pack_bf16x2(f[2 * j], f[2 * j + 1]);
-            __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + oidx + c;
-            uint4* dst = reinterpret_cast<uint4*>(ob);
+              for (int j = 0; j < 16; ++j)
+                pk[j] = pack_bf16x2(apply_act(__uint_as_float(v[2 * j]), a.act),
+                                    apply_act(__uint_as_float(v[2 * j + 1]), a.act));
+            }
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + oidx + c);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
-            if (a.out_mode == OUT_BF16_SPLIT) {
-              uint32_t lo[16];
-#pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const float2 h2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi[j]));
-                lo[j] = pack_bf16x2(f[2 * j] - h2.x, f[2 * j + 1] - h2.y);
-              }
-              uint4* dlo = reinterpret_cast<uint4*>(ob + a.rows_cap * a.N);
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                dlo[j] = make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
-            }
+              dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
           }
         }
       }
@@ -323,15 +309,16 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                    uint32_t box_rows) {
+bool make_tmap_2b(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows, int f16) {
   auto encode = get_encode_fn();
   if (encode == nullptr) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+  CUresult r = encode(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                      2, const_cast<void*>(base), dims,
                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -344,14 +331,13 @@ static int pick_bn(int N) {
   return 64;
 }
 
-static cudaError_t launch_one(const void* A, int n_a, int64_t rows_cap, int K, const void* B, int E,
-                              int N, void* out, int out_mode, const int32_t* offsets, int act,
+static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void* B, int E, int N,
+                              int ab_f16, void* out, int out_mode, const int32_t* offsets, int act,
                               const LaunchCtx& c) {
   const int bn = pick_bn(N);
   CUtensorMap tmA, tmB;
-  // with two A planes the map spans both: lo rows sit rows_cap rows below hi rows
-  if (!make_tmap_bf16(&tmA, A, static_cast<uint64_t>(rows_cap) * n_a, K, gg::BM)) return cudaErrorInvalidValue;
-  if (!make_tmap_bf16(&tmB, B, static_cast<uint64_t>(E) * N, K, bn)) return cudaErrorInvalidValue;
+  if (!make_tmap_2b(&tmA, A, static_cast<uint64_t>(rows_cap), K, gg::BM, ab_f16)) return cudaErrorInvalidValue;
+  if (!make_tmap_2b(&tmB, B, static_cast<uint64_t>(E) * N, K, bn, ab_f16)) return cudaErrorInvalidValue;
   gg::Args a;
   a.offsets = offsets;
   a.E = E;
@@ -363,8 +349,7 @@ static cudaError_t launch_one(const void* A, int n_a, int64_t rows_cap, int K, c
   a.out = out;
   a.act = act;
   a.out_mode = out_mode;
-  a.n_a = n_a;
-  a.stages = gg::RING_BYTES / (n_a * gg::A_BYTES + gg::B_BYTES_MAX);
+  a.ab_f16 = ab_f16;
   a.err = c.err;
   // upper bound of the tile count: sum_e ceil(n_e / BM) <= rows_cap / BM + E
   const int64_t max_tiles = (rows_cap / gg::BM + E) * static_cast<int64_t>(a.n_tiles);
@@ -380,11 +365,11 @@ static cudaError_t launch_one(const void* A, int n_a, int64_t rows_cap, int K, c
 
 cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c) {
   if (p.E > gg::MAX_GROUPS) return cudaErrorInvalidValue;
-  const int planes = p.hidden_split ? 2 : 1;
-  cudaError_t e = launch_one(p.x_perm, 1, p.rows_cap, p.d, p.w1, p.E, p.f, p.h,
-                             p.hidden_split ? gg::OUT_BF16_SPLIT : gg::OUT_BF16, p.offsets, p.act, c);
+  const int hf = p.hidden_f16 ? 1 : 0;
+  cudaError_t e = launch_one(p.x_perm, p.rows_cap, p.d, p.w1, p.E, p.f, 0, p.h,
+                             hf ? gg::OUT_F16 : gg::OUT_BF16, p.offsets, p.act, c);
   if (e != cudaSuccess) return e;
-  return launch_one(p.h, planes, p.rows_cap, p.f, p.w2, p.E, p.d, p.y_perm, gg::OUT_F32, p.offsets, 0, c);
+  return launch_one(p.h, p.rows_cap, p.f, p.w2, p.E, p.d, hf, p.y_perm, gg::OUT_F32, p.offsets, 0, c);
 }
 
 }  // namespace moe

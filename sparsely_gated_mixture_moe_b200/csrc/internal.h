@@ -64,7 +64,7 @@ cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c);
 struct FfnProblem {
   int64_t rows_cap;  // T*k
   int d, f, E, act;  // act: 1 ReLU, 2 GELU
-  int hidden_split;  // bf16 path: h carried as a hi plane plus a remainder plane
+  int hidden_f16;    // bf16 path: h stored in fp16 and w2 given in fp16
   const void* x_perm;
   const int32_t* offsets;
   const void* w1;
@@ -92,10 +92,19 @@ struct CombineProblem {
 };
 cudaError_t launch_combine(const CombineProblem& p, const LaunchCtx& c);
 
+// ---- weight preparation ----------------------------------------------------------
+cudaError_t launch_bf16_to_f16(const void* src, void* dst, int64_t n, int32_t* n_inexact,
+                               const LaunchCtx& c);
+
 // ---- tensor maps -----------------------------------------------------------------
-// 2-D bf16 tensor map over a row-major [rows, cols] matrix with a box of
-// [box_rows, 64 columns] and 128-byte swizzling; out-of-range elements read as zero.
-bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                    uint32_t box_rows);
+// 2-D tensor map of 2-byte elements (bf16, or fp16 when f16 != 0) over a row-major
+// [rows, cols] matrix with a box of [box_rows, 64 columns] and 128-byte swizzling;
+// out-of-range elements read as zero.
+bool make_tmap_2b(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows, int f16);
+inline bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                           uint32_t box_rows) {
+  return make_tmap_2b(map, base, rows, cols, box_rows, 0);
+}
 
 }  // namespace moe

@@ -16,7 +16,7 @@ size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int esize(const moe_config* c) { return c->dtype == MOE_BF16 ? 2 : 4; }
-int hidden_planes(const moe_config* c) { return (c->dtype == MOE_BF16 && c->hidden_split) ? 2 : 1; }
+
 
 // Structural validity of the config (MOE_ERR_INVALID_ARG) and supported shapes
 // (MOE_ERR_UNSUPPORTED).
@@ -28,7 +28,7 @@ moe_status check_config(const moe_config* c) {
   if (c->act != MOE_ACT_RELU && c->act != MOE_ACT_GELU) return MOE_ERR_INVALID_ARG;
   if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (!(c->capacity_factor == c->capacity_factor)) return MOE_ERR_INVALID_ARG;  // NaN
-  if (c->hidden_split != 0 && c->hidden_split != 1) return MOE_ERR_INVALID_ARG;
+  if (c->hidden_f16 != 0 && c->hidden_f16 != 1) return MOE_ERR_INVALID_ARG;
   if (c->k > 8) return MOE_ERR_UNSUPPORTED;
   if (c->T * static_cast<int64_t>(c->k) >= (int64_t{1} << 31)) return MOE_ERR_UNSUPPORTED;
   if (c->T * static_cast<int64_t>(c->E) >= (int64_t{1} << 31)) return MOE_ERR_UNSUPPORTED;
@@ -73,7 +73,7 @@ Layout layout(const moe_config* c) {
   L.x_perm = o;
   o = align_up(o + static_cast<size_t>(n) * c->d_model * esize(c));
   L.h = o;
-  o = align_up(o + static_cast<size_t>(n) * c->d_ff * esize(c) * hidden_planes(c));
+  o = align_up(o + static_cast<size_t>(n) * c->d_ff * esize(c));
   L.y_perm = o;
   o = align_up(o + static_cast<size_t>(n) * c->d_model * 4);
   L.forward = o;
@@ -189,7 +189,7 @@ moe_status do_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offs
   p.f = cfg->d_ff;
   p.E = cfg->E;
   p.act = cfg->act == MOE_ACT_GELU ? 2 : 1;
-  p.hidden_split = hidden_planes(cfg) == 2;
+  p.hidden_f16 = cfg->dtype == MOE_BF16 && cfg->hidden_f16;
   p.x_perm = x_perm;
   p.offsets = offsets;
   p.w1 = w1;
@@ -369,6 +369,18 @@ moe_status moe_get_error(void* ws, moe_stream_t stream, int32_t* device_error) {
   if (v != 0 && cudaMemset(ws, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
   if (device_error) *device_error = v;
   return v == 0 ? MOE_OK : MOE_ERR_DEVICE;
+}
+
+moe_status moe_bf16_to_f16(const void* src, void* dst, int64_t n, int32_t* n_inexact,
+                           moe_stream_t stream) {
+  if (n < 0 || (n > 0 && (!src || !dst))) return MOE_ERR_INVALID_ARG;
+  if (n == 0) {
+    g_last_launches = 0;
+    return MOE_OK;
+  }
+  Ctx ctx(nullptr, stream);
+  if (!ctx.ok) return MOE_ERR_CUDA;
+  return ctx.finish(launch_bf16_to_f16(src, dst, n, n_inexact, ctx.lc));
 }
 
 int32_t moe_last_launch_count(void) { return g_last_launches; }

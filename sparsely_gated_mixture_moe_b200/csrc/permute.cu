@@ -6,15 +6,17 @@
 // only the first C assignments of an expert are kept (capacity factor, "moe paper models"
 // Table 2), the rest are dropped (slot_pos = -1).
 //
-// Three kernels, no atomics on global memory and no cross-block waits:
+// Four kernels, no atomics on global memory and no cross-block waits:
 //   count    block b counts its chunk of 2048 assignments per expert (shared-memory
 //            histogram) -> blk[b][e]
 //   scan     one block: per expert an exclusive scan over the chunks (blk[b][e] becomes
 //            the number of earlier assignments of e), counts[e], kept[e] = min(count, C),
 //            and offsets = exclusive scan of kept
-//   scatter  block b ranks its chunk stably (warp match + per-warp prefix), writes
-//            slot_pos / perm_src and copies the kept token rows into x_perm with 16-byte
-//            vector loads and stores
+//   scatter  block b ranks its chunk stably (warp match + per-warp prefix) and writes
+//            slot_pos / perm_src
+//   gather   x_perm[s] = x[perm_src[s] / k] for every kept row s < offsets[E]: one warp
+//            per row, 16-byte vectors, a grid of several blocks per SM so that enough
+//            loads are in flight to stream at HBM rate
 #include "common.cuh"
 #include "internal.h"
 
@@ -79,30 +81,10 @@ __global__ void __launch_bounds__(pm::SCAN_THREADS)
   if (threadIdx.x == 0) offsets[E] = carry;
 }
 
-template <int VEC_BYTES>
-__device__ __forceinline__ void copy_row(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst,
-                                         int row_bytes, int lane) {
-  const int nv = row_bytes / 16;
-  const uint4* s = reinterpret_cast<const uint4*>(src);
-  uint4* d = reinterpret_cast<uint4*>(dst);
-  int v = lane;
-  for (; v + 96 < nv; v += 128) {
-    const uint4 a0 = __ldg(s + v), a1 = __ldg(s + v + 32), a2 = __ldg(s + v + 64),
-                a3 = __ldg(s + v + 96);
-    d[v] = a0;
-    d[v + 32] = a1;
-    d[v + 64] = a2;
-    d[v + 96] = a3;
-  }
-  for (; v < nv; v += 32) d[v] = __ldg(s + v);
-}
-
 __global__ void __launch_bounds__(pm::THREADS)
     perm_scatter_kernel(const int32_t* __restrict__ idx, int64_t n, int k, int E, int64_t C,
                         const int32_t* __restrict__ blk, const int32_t* __restrict__ offsets,
-                        int32_t* __restrict__ perm_src, int32_t* __restrict__ slot_pos,
-                        const uint8_t* __restrict__ x, uint8_t* __restrict__ x_perm,
-                        int row_bytes) {
+                        int32_t* __restrict__ perm_src, int32_t* __restrict__ slot_pos) {
   extern __shared__ int wbase[];  // [WARPS][E]: running rank base of each warp per expert
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t lt_mask = (1u << lane) - 1u;
@@ -147,16 +129,34 @@ __global__ void __launch_bounds__(pm::THREADS)
       slot_pos[a] = slot;
       if (slot >= 0) perm_src[slot] = static_cast<int32_t>(a);
     }
-    // copy the kept rows of this round, one row per warp step
-    uint32_t kept = __ballot_sync(0xffffffffu, slot >= 0);
-    while (kept) {
-      const int src_lane = __ffs(kept) - 1;
-      kept &= kept - 1;
-      const int s = __shfl_sync(0xffffffffu, slot, src_lane);
-      const int64_t t = (base + r * 32 + src_lane) / k;
-      copy_row<16>(x + t * row_bytes, x_perm + static_cast<int64_t>(s) * row_bytes, row_bytes, lane);
-    }
     __syncwarp();
+  }
+}
+
+constexpr int kGatherWarps = 8;
+
+__global__ void __launch_bounds__(kGatherWarps * 32)
+    perm_gather_kernel(const int32_t* __restrict__ perm_src, const int32_t* __restrict__ offsets,
+                       int E, int k, const uint8_t* __restrict__ x, uint8_t* __restrict__ x_perm,
+                       int row_bytes) {
+  const int lane = threadIdx.x & 31;
+  const int n_kept = __ldg(offsets + E);
+  const int nv = row_bytes >> 4;
+  const int warps = gridDim.x * kGatherWarps;
+  for (int s = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); s < n_kept; s += warps) {
+    const int64_t t = __ldg(perm_src + s) / k;
+    const uint4* src = reinterpret_cast<const uint4*>(x + t * row_bytes);
+    uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(s) * row_bytes);
+    int v = lane;
+    for (; v + 96 < nv; v += 128) {
+      const uint4 a0 = __ldg(src + v), a1 = __ldg(src + v + 32), a2 = __ldg(src + v + 64),
+                  a3 = __ldg(src + v + 96);
+      dst[v] = a0;
+      dst[v + 32] = a1;
+      dst[v + 64] = a2;
+      dst[v + 96] = a3;
+    }
+    for (; v < nv; v += 32) dst[v] = __ldg(src + v);
   }
 }
 
@@ -181,8 +181,17 @@ cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c) {
     if (e != cudaSuccess) return e;
   }
   perm_scatter_kernel<<<static_cast<unsigned>(nblk), pm::THREADS, wsmem, c.stream>>>(
-      p.topk_idx, p.n, p.k, p.E, p.C, p.blk, p.offsets, p.perm_src, p.slot_pos,
-      static_cast<const uint8_t*>(p.x), static_cast<uint8_t*>(p.x_perm), p.d * p.esize);
+      p.topk_idx, p.n, p.k, p.E, p.C, p.blk, p.offsets, p.perm_src, p.slot_pos);
+  ++*c.launches;
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // enough warps for every row when the grid allows, capped at 16 blocks per SM
+  int64_t gblocks = (p.n + kGatherWarps - 1) / kGatherWarps;
+  const int64_t cap = static_cast<int64_t>(c.num_sms) * 16;
+  if (gblocks > cap) gblocks = cap;
+  perm_gather_kernel<<<static_cast<unsigned>(gblocks), kGatherWarps * 32, 0, c.stream>>>(
+      p.perm_src, p.offsets, p.E, p.k, static_cast<const uint8_t*>(p.x),
+      static_cast<uint8_t*>(p.x_perm), p.d * p.esize);
   ++*c.launches;
   return cudaGetLastError();
 }

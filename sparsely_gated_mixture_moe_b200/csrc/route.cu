@@ -44,137 +44,221 @@ __device__ __forceinline__ float softplus_f(float z) {
   return fmaxf(z, 0.0f) + log1pf(expf(-fabsf(z)));
 }
 
-// Runs the gate for the token of this thread.  `fetch(c, l, z)` must fill l[0..31] with
-// the raw clean logits x.W_g of experts c..c+31 and z[0..31] with x.W_noise (noisy
-// only); it is called by all 32 lanes of the warp together, for c = 0, 32, ...
-// `red` is shared memory of at least nwarps * 32 * 33 * 2 + 2 * nwarps * E floats when
-// partials are requested; every thread of the block must call this function.
-template <class Fetch>
-__device__ __forceinline__ void gate_token(const Fetch& fetch, int64_t t, const GateArgs& g,
-                                           float* red) {
+// Descending list of the KM+1 largest (score, expert) pairs seen; a pair ranks higher
+// when its score is larger, or equal with a lower expert index.  Insertion order does
+// not matter, so partial lists over disjoint expert sets merge exactly.
+template <int KM>
+struct TopList {
+  float v[KM + 1];
+  int i[KM + 1];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int s = 0; s <= KM; ++s) {
+      v[s] = -INFINITY;
+      i[s] = 0x7fffffff;
+    }
+  }
+  // keeps the first k+1 slots (k <= KM)
+  __device__ __forceinline__ void insert(float cv, int ci, int k) {
+#pragma unroll
+    for (int q = 0; q <= KM; ++q) {
+      if (q <= k && (cv > v[q] || (cv == v[q] && ci < i[q]))) {
+        const float tv = v[q];
+        const int ti = i[q];
+        v[q] = cv;
+        i[q] = ci;
+        cv = tv;
+        ci = ti;
+      }
+    }
+  }
+};
+
+// Shared-memory bytes gate_tile needs for a block of 128*G threads.
+__host__ __device__ constexpr int gate_smem_bytes(int KM, int G, int E) {
+  return G * 128 * (KM + 1) * 8     // partial lists (scores, experts)
+         + G * 128 * 8              // partial softmax (max, sum)
+         + 128 * (2 * KM + 2) * 4   // final experts, gates, k-th and (k+1)-th score
+         + 4 * G * 32 * 33 * 4      // per-warp transpose for the reductions
+         + 4 * 2 * E * 4            // per-lane-quarter column sums
+         + 64;
+}
+
+// The gate for one tile of 128 tokens, computed by 128*G threads: thread (warp w, lane l)
+// owns token row r = 32*(w%4) + l and the expert columns c = 32*(w/4) + 32*G*i + j.
+// `fetch(c, l, z)` fills l[0..31] with the raw clean logits x.W_g of experts c..c+31 of
+// this thread's token and z[0..31] with x.W_noise (noisy gating); it is called by all 32
+// lanes of a warp together.  Every thread of the block must call gate_tile.
+template <int KM, int G, class Fetch>
+__device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const GateArgs& g,
+                                          uint8_t* smem) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = warp & 3, grp = warp >> 2;
+  const int row = q * 32 + lane;
+  const int64_t t = t0 + row;
   const bool valid = t < g.T;
   const int E = g.E, k = g.k;
-  float val[kMaxK + 1];
-  int ids[kMaxK + 1];
-#pragma unroll
-  for (int s = 0; s <= kMaxK; ++s) {
-    val[s] = -INFINITY;
-    ids[s] = -1;
-  }
-  float m = -INFINITY, ssum = 0.0f;  // running softmax over all experts (renorm == 0)
   const float* noise_row = (g.noisy && valid) ? g.noise + t * E : nullptr;
+  const bool full_softmax = !g.noisy && !g.renorm;
 
-  for (int c = 0; c < E; c += 32) {
+  float* pv = reinterpret_cast<float*>(smem);                    // [G][128][KM+1]
+  int* pi = reinterpret_cast<int*>(pv + G * 128 * (KM + 1));     // [G][128][KM+1]
+  float* pm = reinterpret_cast<float*>(pi + G * 128 * (KM + 1)); // [G][128]
+  float* ps = pm + G * 128;                                      // [G][128]
+  int* fid = reinterpret_cast<int*>(ps + G * 128);               // [128][KM]
+  float* fgate = reinterpret_cast<float*>(fid + 128 * KM);       // [128][KM]
+  float* fkth = fgate + 128 * KM;                                // [128][2]
+  float* tr = fkth + 128 * 2;                                    // [4G warps][32][33]
+  float* qsum = tr + 4 * G * 32 * 33;                            // [4][2][E]
+
+  // ---- pass 1: partial top-(k+1) and softmax statistics over this thread's experts
+  TopList<KM> top;
+  top.init();
+  float m = -INFINITY, ssum = 0.0f;
+  for (int c = grp * 32; c < E; c += 32 * G) {
     float l[32], z[32];
     fetch(c, l, z);
+    float sc[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const int e = c + j;
+      float s = -INFINITY;
       if (e < E) {
-        float s = l[j] + (g.bias ? __ldg(g.bias + e) : 0.0f);
-        if (!g.noisy && !g.renorm) {
-          const float mn = fmaxf(m, s);
-          ssum = ssum * expf(m - mn) + expf(s - mn);
-          m = mn;
-        }
+        s = l[j] + (g.bias ? __ldg(g.bias + e) : 0.0f);
         if (g.noisy) s += (noise_row ? __ldg(noise_row + e) : 0.0f) * softplus_f(z[j]);
-        // insert into the descending list of the k+1 largest; strict '>' keeps the
-        // lower index first among equal values
-        float cv = s;
-        int ci = e;
+      }
+      sc[j] = s;
+    }
+    if (full_softmax) {
+      float cm = -INFINITY;
 #pragma unroll
-        for (int q = 0; q <= kMaxK; ++q) {
-          if (q <= k && cv > val[q]) {
-            const float tv = val[q];
-            const int ti = ids[q];
-            val[q] = cv;
-            ids[q] = ci;
-            cv = tv;
-            ci = ti;
-          }
+      for (int j = 0; j < 32; ++j) cm = fmaxf(cm, sc[j]);
+      const float nm = fmaxf(m, cm);
+      float cs = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) cs += (c + j < E) ? expf(sc[j] - nm) : 0.0f;
+      ssum = (m == -INFINITY ? 0.0f : ssum * expf(m - nm)) + cs;
+      m = nm;
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (c + j < E) top.insert(sc[j], c + j, k);
+  }
+#pragma unroll
+  for (int s2 = 0; s2 <= KM; ++s2) {
+    pv[(grp * 128 + row) * (KM + 1) + s2] = top.v[s2];
+    pi[(grp * 128 + row) * (KM + 1) + s2] = top.i[s2];
+  }
+  pm[grp * 128 + row] = m;
+  ps[grp * 128 + row] = ssum;
+  __syncthreads();
+
+  // ---- merge the G partial results of each token (group 0) and write the outputs
+  if (grp == 0) {
+    for (int g2 = 1; g2 < G; ++g2) {
+#pragma unroll
+      for (int s2 = 0; s2 <= KM; ++s2)
+        if (s2 <= k)
+          top.insert(pv[(g2 * 128 + row) * (KM + 1) + s2], pi[(g2 * 128 + row) * (KM + 1) + s2], k);
+      const float m2 = pm[g2 * 128 + row], s2v = ps[g2 * 128 + row];
+      if (m2 != -INFINITY) {
+        const float nm = fmaxf(m, m2);
+        ssum = (m == -INFINITY ? 0.0f : ssum * expf(m - nm)) + s2v * expf(m2 - nm);
+        m = nm;
+      }
+    }
+    float gate[KM];
+    if (full_softmax) {
+#pragma unroll
+      for (int j = 0; j < KM; ++j) gate[j] = (j < k) ? expf(top.v[j] - m) / ssum : 0.0f;
+    } else {
+      float den = 0.0f;
+#pragma unroll
+      for (int j = 0; j < KM; ++j) {
+        gate[j] = (j < k) ? expf(top.v[j] - top.v[0]) : 0.0f;
+        den += gate[j];
+      }
+#pragma unroll
+      for (int j = 0; j < KM; ++j) gate[j] /= den;
+    }
+    float kth = -INFINITY, kth1 = -INFINITY;  // k-th and (k+1)-th largest scores
+#pragma unroll
+    for (int j = 0; j <= KM; ++j) {
+      if (j == k - 1) kth = top.v[j];
+      if (j == k) kth1 = top.v[j];
+    }
+    if (valid) {
+#pragma unroll
+      for (int j = 0; j < KM; ++j)
+        if (j < k) {
+          g.topk_idx[t * k + j] = top.i[j];
+          g.topk_gate[t * k + j] = gate[j];
         }
-      }
-    }
-  }
-
-  float gate[kMaxK];
-  if (g.noisy || g.renorm) {
-    float den = 0.0f;
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-      gate[j] = (j < k) ? expf(val[j] - val[0]) : 0.0f;
-      den += gate[j];
+      if (g.near_tie) g.near_tie[t] = (k < E && (kth - kth1) <= 1e-4f) ? 1 : 0;
     }
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) gate[j] /= den;
-  } else {
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j) gate[j] = (j < k) ? expf(val[j] - m) / ssum : 0.0f;
+    for (int j = 0; j < KM; ++j) {
+      fid[row * KM + j] = (j < k) ? top.i[j] : -1;
+      fgate[row * KM + j] = gate[j];
+    }
+    fkth[row * 2 + 0] = kth;
+    fkth[row * 2 + 1] = kth1;
   }
-  float kth = -INFINITY, kth1 = -INFINITY;  // k-th and (k+1)-th largest scores
-#pragma unroll
-  for (int j = 0; j <= kMaxK; ++j) {
-    if (j == k - 1) kth = val[j];
-    if (j == k) kth1 = val[j];
-  }
-  if (valid) {
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j)
-      if (j < k) {
-        g.topk_idx[t * k + j] = ids[j];
-        g.topk_gate[t * k + j] = gate[j];
-      }
-    if (g.near_tie) g.near_tie[t] = (k < E && (kth - kth1) <= 1e-4f) ? 1 : 0;
-  }
+  if (g.partials == nullptr) return;  // uniform across the block
+  __syncthreads();
 
-  if (g.partials == nullptr) return;
-  // ---- Importance and Load partial sums over this block's tokens
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nwarps = blockDim.x >> 5;
-  float* tr_imp = red + warp * (32 * 33 * 2);
-  float* tr_load = tr_imp + 32 * 33;
-  float* wsum = red + nwarps * (32 * 33 * 2);  // [nwarps][2][E]
-  for (int c = 0; c < E; c += 32) {
+  // ---- pass 2: Importance and Load partial sums over this tile's tokens
+  const float kth = fkth[row * 2 + 0], kth1 = fkth[row * 2 + 1];
+  int ids[KM];
+  float gts[KM];
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    ids[j] = fid[row * KM + j];
+    gts[j] = fgate[row * KM + j];
+  }
+  float* mytr = tr + warp * (32 * 33);
+  for (int c = grp * 32; c < E; c += 32 * G) {
     float l[32], z[32];
     fetch(c, l, z);
+    float gi[32], pl[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const int e = c + j;
-      float gi = 0.0f, pi = 0.0f;
+      gi[j] = 0.0f;
+      pl[j] = 0.0f;
       if (valid && e < E) {
         if (g.noisy && k < E) {
-          // recomputed exactly as in the first pass, so H >= kth means "among the top k"
+          // recomputed exactly as in pass 1, so H >= kth means "among the top k"
           const float li = l[j] + (g.bias ? __ldg(g.bias + e) : 0.0f);
           const float sp = softplus_f(z[j]);
           const float H = li + __ldg(noise_row + e) * sp;
           const float ex = (H >= kth) ? kth1 : kth;  // kth_excluding(H, k, e)
-          pi = 0.5f * erfcf(-((li - ex) / sp) * 0.70710678118654752f);
+          pl[j] = 0.5f * erfcf(-((li - ex) / sp) * 0.70710678118654752f);
         }
 #pragma unroll
-        for (int q = 0; q < kMaxK; ++q)
-          if (q < k && ids[q] == e) gi = gate[q];
+        for (int jj = 0; jj < KM; ++jj)
+          if (ids[jj] == e) gi[j] = gts[jj];
       }
-      tr_imp[lane * 33 + j] = gi;
-      tr_load[lane * 33 + j] = pi;
     }
-    __syncwarp();
-    float si = 0.0f, sl = 0.0f;
-    for (int r = 0; r < 32; ++r) {
-      si += tr_imp[r * 33 + lane];
-      sl += tr_load[r * 33 + lane];
+    // column sums over the warp's 32 tokens through a padded transpose
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) mytr[lane * 33 + j] = pass == 0 ? gi[j] : pl[j];
+      __syncwarp();
+      float acc = 0.0f;
+      for (int r = 0; r < 32; ++r) acc += mytr[r * 33 + lane];
+      if (c + lane < E) qsum[(q * 2 + pass) * E + c + lane] = acc;
+      __syncwarp();
     }
-    if (c + lane < E) {
-      wsum[(warp * 2 + 0) * E + c + lane] = si;
-      wsum[(warp * 2 + 1) * E + c + lane] = sl;
-    }
-    __syncwarp();
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     float si = 0.0f, sl = 0.0f;
-    for (int w = 0; w < nwarps; ++w) {
-      si += wsum[(w * 2 + 0) * E + e];
-      sl += wsum[(w * 2 + 1) * E + e];
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) {
+      si += qsum[(qq * 2 + 0) * E + e];
+      sl += qsum[(qq * 2 + 1) * E + e];
     }
     g.partials[(static_cast<int64_t>(blockIdx.x) * 2 + 0) * E + e] = si;
     g.partials[(static_cast<int64_t>(blockIdx.x) * 2 + 1) * E + e] = sl;
@@ -184,7 +268,9 @@ __device__ __forceinline__ void gate_token(const Fetch& fetch, int64_t t, const 
 // ------------------------------------------------------------------ bf16 router
 
 namespace rt {
-constexpr int THREADS = 128;
+// expert-column groups per token: 4 (16 warps), or 2 for k > 4 to leave registers for
+// the longer top-(k+1) lists
+constexpr int groups_for(int KM) { return KM > 4 ? 2 : 4; }
 constexpr int BK = 64;
 constexpr int A_BYTES = kRouteBM * BK * 2;  // 16 KB
 }  // namespace rt
@@ -200,7 +286,8 @@ struct RouteTcArgs {
   int* err;
 };
 
-__global__ void __launch_bounds__(rt::THREADS, 1)
+template <int KM, int G = rt::groups_for(KM)>
+__global__ void __launch_bounds__(128 * G, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     const __grid_constant__ CUtensorMap tmG,
                     const __grid_constant__ CUtensorMap tmN, const RouteTcArgs a) {
@@ -271,7 +358,7 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kRouteBM, a.e_pad);
+      const uint32_t idesc = idesc_f32acc(kRouteBM, a.e_pad, kFmtBF16);
       int stage = 0;
       uint32_t phase = 0;
       bool aborted = false;
@@ -286,10 +373,10 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
         for (int kk = 0; kk < rt::BK / 16; ++kk) {
           const uint64_t ad = sdesc_k128(st + kk * 32);
           const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
-          tc_mma_bf16(tmem_base, ad, sdesc_k128(st + rt::A_BYTES + kk * 32), idesc, acc);
+          tc_mma_f16kind(tmem_base, ad, sdesc_k128(st + rt::A_BYTES + kk * 32), idesc, acc);
           if (a.nb == 2)
-            tc_mma_bf16(tmem_base + a.acc_cols, ad,
-                        sdesc_k128(st + rt::A_BYTES + b_bytes + kk * 32), idesc, acc);
+            tc_mma_f16kind(tmem_base + a.acc_cols, ad,
+                           sdesc_k128(st + rt::A_BYTES + b_bytes + kk * 32), idesc, acc);
         }
         tc_commit(empty0 + 8 * stage);
         if (++stage == a.stages) {
@@ -311,7 +398,8 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
   const bool ok = (*s_abort == 0);
   tc_fence_after();
   if (ok) {
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    // warp w reads TMEM lanes 32*(w%4) .. +31: its token rows
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     auto fetch = [&](int c, float (&l)[32], float (&z)[32]) {
       uint32_t v[32];
       tmem_ld32(tmem_base + lane_base + c, v);
@@ -329,8 +417,8 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
 #pragma unroll
       for (int j = 0; j < 32; ++j) l[j] = __uint_as_float(v[j]);
     };
-    // the stage buffers are idle once `done` has fired: reuse them for the reduction
-    gate_token(fetch, static_cast<int64_t>(t0) + threadIdx.x, a.g, reinterpret_cast<float*>(smem));
+    // the stage buffers are idle once `done` has fired: reuse them for the gate
+    gate_tile<KM, G>(fetch, t0, a.g, smem);
   } else if (threadIdx.x == 0) {
     set_error(a.err, kErrTimeout);
   }
@@ -342,11 +430,14 @@ __global__ void __launch_bounds__(rt::THREADS, 1)
 
 // ------------------------------------------------------------------ fp32 router
 
-// One token per thread; the logits were written to the workspace by the SIMT product.
-__global__ void __launch_bounds__(128)
+// The logits were written to the workspace by the SIMT product; 128 threads, one token
+// row each, walk all expert columns (one column group).
+template <int KM>
+__global__ void __launch_bounds__(128, 1)
     gate_f32_kernel(const float* __restrict__ logits, const float* __restrict__ nz, GateArgs g) {
-  extern __shared__ float red[];
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  extern __shared__ __align__(16) uint8_t gsmem[];
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRouteBM;
+  const int64_t t = t0 + threadIdx.x;
   const bool valid = t < g.T;
   const int E = g.E;
   auto fetch = [&](int c, float (&l)[32], float (&z)[32]) {
@@ -357,7 +448,7 @@ __global__ void __launch_bounds__(128)
       z[j] = (in && nz != nullptr) ? nz[t * E + c + j] : 0.0f;
     }
   };
-  gate_token(fetch, t, g, red);
+  gate_tile<KM, 1>(fetch, t0, g, gsmem);
 }
 
 __global__ void finalize_importance_load_kernel(const float* __restrict__ partials, int nblocks,
@@ -391,14 +482,23 @@ static GateArgs gate_args(const RouteProblem& p) {
   return g;
 }
 
-static size_t reduction_smem(int E, int nwarps) {
-  return static_cast<size_t>(nwarps) * (32 * 33 * 2) * 4 + static_cast<size_t>(2) * nwarps * E * 4;
-}
+static int k_bucket(int k) { return k <= 1 ? 1 : k <= 2 ? 2 : k <= 4 ? 4 : 8; }
 
 static cudaError_t launch_finalize(const RouteProblem& p, int nblocks, const LaunchCtx& c) {
   if (!(p.importance || p.load)) return cudaSuccess;
   finalize_importance_load_kernel<<<(p.E + 127) / 128, 128, 0, c.stream>>>(
       p.partials, nblocks, p.E, p.importance, p.load);
+  ++*c.launches;
+  return cudaGetLastError();
+}
+
+template <int KM>
+static cudaError_t launch_route_tc(const CUtensorMap& tmX, const CUtensorMap& tmG,
+                                   const CUtensorMap& tmN, const RouteTcArgs& a, int smem,
+                                   int nblocks, const LaunchCtx& c) {
+  cudaError_t e = cudaFuncSetAttribute(route_tc_kernel<KM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  route_tc_kernel<KM><<<nblocks, 128 * rt::groups_for(KM), smem, c.stream>>>(tmX, tmG, tmN, a);
   ++*c.launches;
   return cudaGetLastError();
 }
@@ -417,8 +517,9 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   if (stages > a.kblocks) stages = a.kblocks;
   if (stages < 2) stages = 2;
   a.stages = stages;
+  const int km = k_bucket(p.k);
   int region = stages * stage_bytes;
-  const int red = static_cast<int>(reduction_smem(p.E, rt::THREADS / 32));
+  const int red = gate_smem_bytes(km, rt::groups_for(km), p.E);
   if (region < red) region = red;
   a.bar_off = (region + 127) / 128 * 128;
   a.err = c.err;
@@ -432,14 +533,29 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   } else {
     tmN = tmG;
   }
-  cudaError_t e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
   const int nblocks = route_blocks(p.T);
-  route_tc_kernel<<<nblocks, rt::THREADS, smem, c.stream>>>(tmX, tmG, tmN, a);
-  ++*c.launches;
-  e = cudaGetLastError();
+  cudaError_t e;
+  switch (km) {
+    case 1: e = launch_route_tc<1>(tmX, tmG, tmN, a, smem, nblocks, c); break;
+    case 2: e = launch_route_tc<2>(tmX, tmG, tmN, a, smem, nblocks, c); break;
+    case 4: e = launch_route_tc<4>(tmX, tmG, tmN, a, smem, nblocks, c); break;
+    default: e = launch_route_tc<8>(tmX, tmG, tmN, a, smem, nblocks, c); break;
+  }
   if (e != cudaSuccess) return e;
   return launch_finalize(p, nblocks, c);
+}
+
+template <int KM>
+static cudaError_t launch_gate_f32(const RouteProblem& p, const GateArgs& g, int nblocks,
+                                   const LaunchCtx& c) {
+  const int smem = gate_smem_bytes(KM, 1, p.E);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(gate_f32_kernel<KM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+  }
+  gate_f32_kernel<KM><<<nblocks, 128, smem, c.stream>>>(p.logits_ws, p.noisy ? p.nz_ws : nullptr, g);
+  ++*c.launches;
+  return cudaGetLastError();
 }
 
 cudaError_t launch_route_f32(const RouteProblem& p, const LaunchCtx& c) {
@@ -451,17 +567,14 @@ cudaError_t launch_route_f32(const RouteProblem& p, const LaunchCtx& c) {
                              p.nz_ws, nullptr, 1, p.T, p.E, p.d, 0, c);
     if (e != cudaSuccess) return e;
   }
-  GateArgs g = gate_args(p);
-  const size_t smem = g.partials ? reduction_smem(p.E, 4) : 0;
-  if (smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(gate_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-  }
+  const GateArgs g = gate_args(p);
   const int nblocks = route_blocks(p.T);
-  gate_f32_kernel<<<nblocks, 128, smem, c.stream>>>(p.logits_ws, p.noisy ? p.nz_ws : nullptr, g);
-  ++*c.launches;
-  e = cudaGetLastError();
+  switch (k_bucket(p.k)) {
+    case 1: e = launch_gate_f32<1>(p, g, nblocks, c); break;
+    case 2: e = launch_gate_f32<2>(p, g, nblocks, c); break;
+    case 4: e = launch_gate_f32<4>(p, g, nblocks, c); break;
+    default: e = launch_gate_f32<8>(p, g, nblocks, c); break;
+  }
   if (e != cudaSuccess) return e;
   return launch_finalize(p, nblocks, c);
 }

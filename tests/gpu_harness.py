@@ -41,11 +41,18 @@ def f64(t: torch.Tensor) -> np.ndarray:
 def config_of(w: workloads.Workload) -> moe.MoEConfig:
     return moe.make_config(w.T, w.d_model, w.d_ff, w.E, w.k, gating=w.gating, renorm=w.renorm,
                            capacity_factor=w.capacity_factor, act=w.act, dtype=w.dtype,
-                           hidden_split=w.hidden_split)
+                           hidden_f16=w.hidden_f16)
 
 
-def hidden_planes(w):
-    return 2 if (w.dtype == "bf16" and w.hidden_split) else 1
+def hidden_dtype(w):
+    if w.dtype == "f32":
+        return torch.float32
+    return torch.float16 if w.hidden_f16 else torch.bfloat16
+
+
+def to_device_prepared(w, inp, cfg=None):
+    """Inputs on the GPU, weights as the forward pass takes them (fp16 w2 with fp16 h)."""
+    return moe.prepare_weights(cfg or config_of(w), to_device(inp))
 
 
 def to_device(inp):
@@ -55,6 +62,7 @@ def to_device(inp):
 def run_steps(w, dev, cfg=None):
     """The four step calls on one stream; returns every output on the CPU."""
     cfg = cfg or config_of(w)
+    dev = moe.prepare_weights(cfg, dev)
     T, k, E, d, f = w.T, w.k, w.E, w.d_model, w.d_ff
     dt = w.torch_dtype
     cu = "cuda"
@@ -67,7 +75,7 @@ def run_steps(w, dev, cfg=None):
         "perm_src": torch.full((max(T * k, 1),), -7, dtype=torch.int32, device=cu),
         "slot_pos": torch.full((max(T * k, 1),), -7, dtype=torch.int32, device=cu),
         "x_perm": torch.zeros(max(T * k, 1), d, dtype=dt, device=cu),
-        "h": torch.zeros(hidden_planes(w) * max(T * k, 1), f, dtype=dt, device=cu),
+        "h": torch.zeros(max(T * k, 1), f, dtype=hidden_dtype(w), device=cu),
         "y_perm": torch.zeros(max(T * k, 1), d, dtype=torch.float32, device=cu),
         "y": torch.full((T, d), float("nan"), dtype=torch.float32, device=cu),
     }
@@ -165,11 +173,7 @@ def check_permute(w, inp, g, report):
 
 
 def gpu_hidden(w, g, rows):
-    """The GPU's hidden activations as one value per element (hi + lo in split mode)."""
-    h = f64(g["h"][rows])
-    if hidden_planes(w) == 2:
-        h = h + f64(g["h"][np.asarray(rows) + w.T * w.k])
-    return h
+    return f64(g["h"][rows])
 
 
 def check_ffn(w, inp, g, n, report, rows=None):
@@ -177,7 +181,7 @@ def check_ffn(w, inp, g, n, report, rows=None):
 
     h is an intermediate stored in bf16 (or as a bf16 pair): each element must be the
     oracle's value up to that storage's rounding, |dh| <= u |h| + 1e-4 rms(h), with
-    u = 2^-8 for one bf16 and 2^-15 for the pair (fp32 path: 1e-5 of rms)."""
+    u = 2^-8 for bf16 and 2^-11 for fp16 (fp32 path: 1e-5 of rms)."""
     off = g["offsets"].numpy()
     if rows is None:
         rows = list(range(n))
@@ -193,7 +197,7 @@ def check_ffn(w, inp, g, n, report, rows=None):
     h_g = gpu_hidden(w, g, rows)
     rms_h = float(np.sqrt(np.mean(h_o ** 2))) if h_o.size else 0.0
     if w.dtype == "bf16":
-        u = 2.0 ** -15 if hidden_planes(w) == 2 else BF16_U
+        u = 2.0 ** -11 if w.hidden_f16 else BF16_U
         bound = u * np.abs(h_o) + 1e-4 * rms_h
     else:
         bound = 1e-5 * rms_h + 1e-6 * np.abs(h_o)

@@ -34,7 +34,7 @@ def test_config_struct_layout():
     assert ctypes.sizeof(moe.MoEConfig) == 48
     assert moe.MoEConfig.capacity_factor.offset == 32
     assert moe.MoEConfig.dtype.offset == 40
-    assert moe.MoEConfig.hidden_split.offset == 44
+    assert moe.MoEConfig.hidden_f16.offset == 44
 
 
 def test_status_strings():
@@ -91,7 +91,7 @@ def test_route_validation():
     bad.T = -1
     assert _route(bad) == 1
     bad = _cfg()
-    bad.hidden_split = 2
+    bad.hidden_f16 = 2
     assert _route(bad) == 1
     assert moe.lib.moe_route(None, FAKE, FAKE, None, None, None, FAKE, FAKE, None, None, None,
                              FAKE, None) == 1

@@ -39,8 +39,8 @@ SMALL = {
     "k_equals_E": Workload("kE", T=200, d_model=64, d_ff=128, E=4, k=4, act="gelu"),
     "one_token": Workload("t1", T=1, d_model=64, d_ff=64, E=8, k=2),
     "E8_bf16_pad": Workload("e8", T=500, d_model=64, d_ff=64, E=8, k=2),
-    "split_multitile": Workload("sp", T=3000, d_model=192, d_ff=384, E=6, k=2, act="gelu",
-                                hidden_split=True, capacity_factor=0.9),
+    "f16_hidden_multitile": Workload("h16", T=3000, d_model=192, d_ff=384, E=6, k=2, act="gelu",
+                                     hidden_f16=True, capacity_factor=0.9),
 }
 
 
@@ -159,3 +159,23 @@ def test_full_size_sampled(name):
     assert f["device_error"] == 0
     assert torch.equal(f["y"], g["y"])
     print(name, rep)
+
+
+def test_bf16_to_f16_reencoding():
+    """The library's re-encoding equals a round-to-nearest-even conversion and is exact
+    for every value of magnitude >= 2^-17 (the count of inexact values is reported)."""
+    import sparsely_gated_mixture_moe_b200 as moe
+    w2 = workloads.make_inputs(W["switch"].scaled(T=16))["w2"]
+    special = torch.tensor([0.0, -0.0, 2.0 ** -17, 2.0 ** -18, 3.0 * 2.0 ** -20, 65504.0, 1e5,
+                            -1e-30, 1.0 + 2.0 ** -7], dtype=torch.bfloat16)
+    for src in (w2.reshape(-1), special):
+        ref = src.to(torch.float16)
+        inexact_cpu = int((ref.double() != src.double()).sum())
+        dst = torch.empty(src.shape, dtype=torch.float16, device="cuda")
+        cnt = torch.zeros(1, dtype=torch.int32, device="cuda")
+        moe.moe_bf16_to_f16(src.cuda(), dst, n_inexact=cnt)
+        assert torch.equal(dst.cpu().view(torch.int16), ref.view(torch.int16))
+        assert int(cnt.item()) == inexact_cpu
+        big = src.double().abs() >= 2.0 ** -17
+        fin = src.double().abs() <= 65504
+        assert torch.equal(ref.double()[big & fin], src.double()[big & fin])

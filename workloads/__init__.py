@@ -49,11 +49,11 @@ class Workload:
             under the softmax over all experts (Switch top-1 rule).
     capacity_factor: None = no limit; else C = ceil(cf * T * k / E) per expert.
     zipf_s: None, or the Zipf exponent of the per-expert logit bias.
-    hidden_split: carry the expert hidden activations as a bf16 pair (hi + remainder)
-            instead of one bf16 value.  The Switch workload needs it to keep the layer
-            output within max|err|/RMS <= 2e-2: its top-1 gates vary several-fold between
-            tokens, which stretches the max-to-RMS ratio of the error that a single bf16
-            rounding of h leaves.
+    hidden_f16: store the expert hidden activations in fp16 (11 significant bits)
+            instead of bf16 (8), with W2 re-encoded to fp16 for the second product.  The
+            Switch workload needs it to keep the layer output within max|err|/RMS <= 2e-2:
+            its top-1 gates vary several-fold between tokens, which stretches the
+            max-to-RMS ratio of the error that a bf16 rounding of h leaves.
     """
 
     name: str
@@ -68,7 +68,7 @@ class Workload:
     act: str = "relu"
     dtype: str = "bf16"
     zipf_s: Optional[float] = None
-    hidden_split: bool = False
+    hidden_f16: bool = False
     seed: int = 0
 
     def scaled(self, **kw) -> "Workload":
@@ -90,7 +90,7 @@ WORKLOADS: Dict[str, Workload] = {
                      renorm=True, capacity_factor=None, act="relu", dtype="f32"),
     "switch": Workload("switch", T=16384, d_model=768, d_ff=3072, E=128, k=1,
                        gating="softmax_topk", renorm=False, capacity_factor=1.25,
-                       act="gelu", dtype="bf16", hidden_split=True),
+                       act="gelu", dtype="bf16", hidden_f16=True),
     "noisy": Workload("noisy", T=8192, d_model=512, d_ff=1024, E=256, k=4,
                       gating="noisy_topk", renorm=True, capacity_factor=None,
                       act="relu", dtype="bf16"),
