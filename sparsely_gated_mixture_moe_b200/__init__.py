@@ -42,6 +42,7 @@ def _load():
         "moe_get_error": (ctypes.c_int, [P, P, ctypes.POINTER(ctypes.c_int32)]),
         "moe_last_launch_count": (ctypes.c_int32, []),
         "moe_bf16_to_f16": (ctypes.c_int, [P, P, ctypes.c_int64, P, P]),
+        "moe_permute_noalloc": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -113,6 +114,17 @@ def moe_permute(cfg, topk_idx, x, counts, offsets, perm_src, slot_pos, x_perm, w
                            _ptr(perm_src, "perm_src"), _ptr(slot_pos, "slot_pos"),
                            _ptr(x_perm, "x_perm"), _ptr(ws, "ws"), _stream(stream)),
            "moe_permute")
+
+
+def moe_permute_noalloc(cfg, topk_idx, x, counts, offsets, perm_src, slot_pos, x_perm,
+                        stream=None):
+    """moe_permute with the library's fixed device scratch instead of a workspace (for
+    callers that cannot allocate); see include/moe.h for its size limit and sharing."""
+    _check(lib.moe_permute_noalloc(ctypes.byref(cfg), _ptr(topk_idx, "topk_idx"), _ptr(x, "x"),
+                                   _ptr(counts, "counts"), _ptr(offsets, "offsets"),
+                                   _ptr(perm_src, "perm_src"), _ptr(slot_pos, "slot_pos"),
+                                   _ptr(x_perm, "x_perm"), _stream(stream)),
+           "moe_permute_noalloc")
 
 
 def moe_expert_ffn(cfg, x_perm, offsets, w1, w2, h, y_perm, ws, stream=None):
@@ -209,4 +221,4 @@ __all__ = ["ACT", "DTYPE", "GATING", "MoEConfig", "MoEError", "MoELayer", "STATU
            "make_config", "moe_capacity", "moe_combine", "moe_expert_ffn", "moe_forward",
            "moe_forward_workspace_size", "moe_get_error", "moe_permute", "moe_route",
            "moe_workspace_size", "workspace", "last_launch_count", "moe_bf16_to_f16",
-           "prepare_weights"]
+           "prepare_weights", "moe_permute_noalloc"]

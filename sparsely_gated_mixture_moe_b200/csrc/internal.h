@@ -96,6 +96,11 @@ cudaError_t launch_combine(const CombineProblem& p, const LaunchCtx& c);
 cudaError_t launch_bf16_to_f16(const void* src, void* dst, int64_t n, int32_t* n_inexact,
                                const LaunchCtx& c);
 
+// ---- host helpers shared by the entry points (moe_api.cu) ------------------------
+moe_status check_config_host(const moe_config* cfg);  // MOE_OK / INVALID_ARG / UNSUPPORTED
+int64_t capacity_host(const moe_config* cfg);         // C, or -1 for no limit
+void set_last_launch_count(int32_t n);
+
 // ---- tensor maps -----------------------------------------------------------------
 // 2-D tensor map of 2-byte elements (bf16, or fp16 when f16 != 0) over a row-major
 // [rows, cols] matrix with a box of [box_rows, 64 columns] and 128-byte swizzling;

@@ -227,6 +227,11 @@ moe_status empty_batch(const moe_config* cfg, int32_t* counts, int32_t* offsets,
 }
 
 }  // namespace
+
+moe_status check_config_host(const moe_config* cfg) { return check_config(cfg); }
+int64_t capacity_host(const moe_config* cfg) { return capacity_of(cfg); }
+void set_last_launch_count(int32_t n) { g_last_launches = n; }
+
 }  // namespace moe
 
 using namespace moe;

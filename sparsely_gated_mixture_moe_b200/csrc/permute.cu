@@ -17,6 +17,8 @@
 //   gather   x_perm[s] = x[perm_src[s] / k] for every kept row s < offsets[E]: one warp
 //            per row, 16-byte vectors, a grid of several blocks per SM so that enough
 //            loads are in flight to stream at HBM rate
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -197,3 +199,91 @@ cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c) {
 }
 
 }  // namespace moe
+
+// ------------------------------------------------------------------------------------
+// moe_permute without a caller-provided workspace, for callers that cannot allocate
+// device memory.  Its per-chunk, per-expert counts live in a fixed array in the
+// library's own device memory instead of in `ws`.
+
+namespace moe {
+
+// Every device that loads libmoe holds this array until the process exits.
+static __device__ __align__(256) int32_t g_permute_scratch[MOE_NOALLOC_SCRATCH_BYTES / 4];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_permute_scratch on the current device.  In host code the name
+// g_permute_scratch is only a host-side stand-in, so the address is looked up once per
+// device, with that device current, and cached.
+cudaError_t scratch_address(int dev, void** out) {
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_permute_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_idx,
+                                          const void* x, int32_t* counts, int32_t* offsets,
+                                          int32_t* perm_src, int32_t* slot_pos, void* x_perm,
+                                          moe_stream_t stream) {
+  using namespace moe;
+  moe_status st = check_config_host(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cfg->T == 0) {
+    const size_t E = static_cast<size_t>(cfg->E);
+    if (cudaMemsetAsync(counts, 0, E * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(offsets, 0, (E + 1) * 4, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    set_last_launch_count(0);
+    return MOE_OK;
+  }
+  if (!topk_idx || !x || !perm_src || !slot_pos || !x_perm) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(x_perm) & 15u))
+    return MOE_ERR_INVALID_ARG;
+  const int64_t n = cfg->T * cfg->k;
+  // the scratch holds one int32 per (2048-assignment chunk, expert)
+  if (permute_blocks(n) * cfg->E * 4 > static_cast<int64_t>(MOE_NOALLOC_SCRATCH_BYTES))
+    return MOE_ERR_UNSUPPORTED;
+  int dev = 0;
+  LaunchCtx c;
+  int launches = 0;
+  void* scratch = nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&c.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      scratch_address(dev, &scratch) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  c.stream = s;
+  c.err = nullptr;  // no error word: out-of-range expert indices are dropped unreported
+  c.launches = &launches;
+  PermuteProblem p;
+  p.n = n;
+  p.k = cfg->k;
+  p.E = cfg->E;
+  p.d = cfg->d_model;
+  p.esize = cfg->dtype == MOE_BF16 ? 2 : 4;
+  p.C = capacity_host(cfg);
+  p.topk_idx = topk_idx;
+  p.x = x;
+  p.counts = counts;
+  p.offsets = offsets;
+  p.perm_src = perm_src;
+  p.slot_pos = slot_pos;
+  p.x_perm = x_perm;
+  p.blk = static_cast<int32_t*>(scratch);  // fully rewritten by the count kernel each call
+  if (launch_permute(p, c) != cudaSuccess) return MOE_ERR_CUDA;
+  set_last_launch_count(launches);
+  return MOE_OK;
+}
