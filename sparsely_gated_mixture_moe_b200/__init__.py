@@ -43,6 +43,7 @@ def _load():
         "moe_last_launch_count": (ctypes.c_int32, []),
         "moe_bf16_to_f16": (ctypes.c_int, [P, P, ctypes.c_int64, P, P]),
         "moe_permute_noalloc": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
+        "moe_erf_check": (ctypes.c_int, [P, P, P, ctypes.c_int64, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -17,10 +17,12 @@
 //   warp 1      TMEM owner and MMA issuer: one thread issues tcgen05.mma (M=128, N=BN,
 //               K=16) into one of two TMEM accumulators (2 x 256 fp32 columns), and
 //               tcgen05.commit releases smem stages and hands finished accumulators on.
-//   warps 2-9   epilogue: tcgen05.ld of the accumulator (each warp reads its 32-lane
-//               quarter, half of the columns), activation, rounding to bf16/fp16 (or fp32
-//               as is), stores of the rows that belong to the expert (a ragged tail is
-//               masked).
+//   warps 2-13  epilogue: tcgen05.ld of the accumulator (each warp reads its 32-lane
+//               quarter and every third 32-column chunk), activation, rounding to
+//               bf16/fp16 (or fp32 as is), stores of the rows that belong to the expert
+//               (a ragged tail is masked).  Three warps per lane quarter keep a ragged
+//               tile, whose rows all sit in the first quarters, from serialising on few
+//               warps.
 // Tiles are (expert, n-tile, m-tile) with m innermost, so CTAs running at the same time
 // share weight tiles through L2 and each expert's weights stream from HBM about once.
 // Rows past an expert's end that a 128-row tile reads belong to the next expert or lie
@@ -40,7 +42,8 @@ namespace gg {
 constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int STAGES = 4;
-constexpr int EPI_WARPS = 8;
+constexpr int EPI_WARPS = 12;  // 3 per TMEM lane quarter (more would cap registers below need)
+constexpr int EPI_SUBS = EPI_WARPS / 4;
 constexpr int THREADS = 64 + EPI_WARPS * 32;
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
 constexpr int B_BYTES_MAX = 256 * BK * 2;   // 32 KB
@@ -92,6 +95,61 @@ __device__ __forceinline__ Tile decode_tile(int L, const int* tp, const Args& a)
   t.row0 = r0 + t.mt * BM;
   t.valid = min(BM, r1 - t.row0);
   return t;
+}
+
+// erf by Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
+// erf(x) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-x^2), t = 1 / (1 + p x),
+// x >= 0, |error| <= 1.5e-7 (odd extension for x < 0).  About a third of the
+// instructions of a full-accuracy erf; the activations it feeds are rounded to 16 bits.
+__device__ __forceinline__ float erf_as7126(float x) {
+  const float ax = fabsf(x);
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, ax, 1.0f));
+  float poly = fmaf(1.061405429f, t, -1.453152027f);
+  poly = fmaf(poly, t, 1.421413741f);
+  poly = fmaf(poly, t, -0.284496736f);
+  poly = fmaf(poly, t, 0.254829592f);
+  poly *= t;
+  const float y = 1.0f - poly * __expf(-ax * ax);
+  return copysignf(y, x);
+}
+
+template <int ACT>
+__device__ __forceinline__ float epi_act(float z) {
+  if (ACT == 1) return fmaxf(z, 0.0f);
+  if (ACT == 2) return 0.5f * z * (1.0f + erf_as7126(z * 0.70710678118654752f));
+  return z;
+}
+
+// One warp's share of a finished accumulator: its 32 rows (one per lane), the 32-column
+// chunks sub*32 + 32*EPI_SUBS*i of the tile; rows outside the expert are not stored.
+template <int MODE, int ACT>
+__device__ __forceinline__ void epilogue_rows(const Args& a, uint32_t tbase, int64_t oidx, int sub,
+                                              bool row_ok) {
+  for (int c = sub * 32; c < a.bn; c += 32 * EPI_SUBS) {
+    uint32_t v[32];
+    tmem_ld32(tbase + c, v);
+    tmem_ld_wait();
+    if (!row_ok) continue;
+    if (MODE == OUT_F32) {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + oidx + c);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                             __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+    } else {
+      uint32_t pk[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float x0 = epi_act<ACT>(__uint_as_float(v[2 * j]));
+        const float x1 = epi_act<ACT>(__uint_as_float(v[2 * j + 1]));
+        pk[j] = MODE == OUT_F16 ? pack_f16x2(x0, x1) : pack_bf16x2(x0, x1);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + oidx + c);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -228,9 +286,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    const int q = warp & 3;                // TMEM lane quarter this warp may read
-    const int half = (warp - 2) >> 2;      // which half of the tile's columns
-    const int cols = a.bn >> 1;
+    const int q = warp & 3;               // TMEM lane quarter this warp may read
+    const int sub = (warp - 2) >> 2;      // which 32-column chunks: sub*32 + 96*i
+    const int mode = a.out_mode * 3 + a.act;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x) {
@@ -243,38 +301,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const int r = q * 32 + lane;
       const bool row_ok = r < t.valid;
-      const int64_t oidx = static_cast<int64_t>(t.row0 + r) * a.N + t.nt * a.bn + half * cols;
-      const uint32_t tbase =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256 + half * cols;
-      for (int c = 0; c < cols; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(tbase + c, v);
-        tmem_ld_wait();
-        if (row_ok) {
-          if (a.out_mode == OUT_F32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + oidx + c);
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                   __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-          } else {
-            uint32_t pk[16];
-            if (a.out_mode == OUT_F16) {
-#pragma unroll
-              for (int j = 0; j < 16; ++j)
-                pk[j] = pack_f16x2(apply_act(__uint_as_float(v[2 * j]), a.act),
-                                   apply_act(__uint_as_float(v[2 * j + 1]), a.act));
-            } else {
-#pragma unroll
-              for (int j = 0; j < 16; ++j)
-                pk[j] = pack_bf16x2(apply_act(__uint_as_float(v[2 * j]), a.act),
-                                    apply_act(__uint_as_float(v[2 * j + 1]), a.act));
-            }
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + oidx + c);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-          }
+      const int64_t oidx = static_cast<int64_t>(t.row0 + r) * a.N + t.nt * a.bn;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256;
+      // a warp none of whose rows belong to the expert skips the tile
+      if (__any_sync(0xffffffffu, row_ok)) {
+        switch (mode) {
+          case OUT_BF16 * 3 + 1: epilogue_rows<OUT_BF16, 1>(a, tbase, oidx, sub, row_ok); break;
+          case OUT_BF16 * 3 + 2: epilogue_rows<OUT_BF16, 2>(a, tbase, oidx, sub, row_ok); break;
+          case OUT_F16 * 3 + 1: epilogue_rows<OUT_F16, 1>(a, tbase, oidx, sub, row_ok); break;
+          case OUT_F16 * 3 + 2: epilogue_rows<OUT_F16, 2>(a, tbase, oidx, sub, row_ok); break;
+          default: epilogue_rows<OUT_F32, 0>(a, tbase, oidx, sub, row_ok); break;
         }
       }
       tc_fence_before();
@@ -373,3 +409,28 @@ cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c) {
 }
 
 }  // namespace moe
+
+// ------------------------------------------------------------- erf self-check
+
+namespace moe {
+__global__ void erf_check_kernel(const float* __restrict__ x, float* __restrict__ fast,
+                                 float* __restrict__ ref, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    fast[i] = gg::erf_as7126(x[i]);
+    ref[i] = erff(x[i]);
+  }
+}
+}  // namespace moe
+
+extern "C" moe_status moe_erf_check(const float* x, float* fast, float* ref, int64_t n,
+                                    moe_stream_t stream) {
+  if (n < 0 || (n > 0 && (!x || !fast || !ref))) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  moe::erf_check_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                          reinterpret_cast<cudaStream_t>(stream)>>>(x, fast, ref, n);
+  moe::set_last_launch_count(1);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}

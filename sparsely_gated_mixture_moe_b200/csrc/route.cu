@@ -79,16 +79,19 @@ __host__ __device__ constexpr int gate_smem_bytes(int KM, int G, int E) {
   return G * 128 * (KM + 1) * 8     // partial lists (scores, experts)
          + G * 128 * 8              // partial softmax (max, sum)
          + 128 * (2 * KM + 2) * 4   // final experts, gates, k-th and (k+1)-th score
-         + 4 * G * 32 * 33 * 4      // per-warp transpose for the reductions
+         + 4 * G * 2 * 32 * 33 * 4  // per-warp transposes (two quantities) for the reductions
          + 4 * 2 * E * 4            // per-lane-quarter column sums
          + 64;
 }
 
 // The gate for one tile of 128 tokens, computed by 128*G threads: thread (warp w, lane l)
 // owns token row r = 32*(w%4) + l and the expert columns c = 32*(w/4) + 32*G*i + j.
-// `fetch(c, l, z)` fills l[0..31] with the raw clean logits x.W_g of experts c..c+31 of
-// this thread's token and z[0..31] with x.W_noise (noisy gating); it is called by all 32
-// lanes of a warp together.  Every thread of the block must call gate_tile.
+// `fetch(c, l, z)` fills l[0..7] with the raw clean logits x.W_g of experts c..c+7 of
+// this thread's token (c a multiple of 8) and z[0..7] with x.W_noise (noisy gating); it
+// is called by all 32 lanes of a warp together.  The loops step 8 experts at a time and
+// are not unrolled: each block runs this code once, so a short instruction stream (few
+// instruction-cache misses) matters more than unrolling.  Every thread of the block must
+// call gate_tile.
 template <int KM, int G, class Fetch>
 __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const GateArgs& g,
                                           uint8_t* smem) {
@@ -99,7 +102,9 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
   const bool valid = t < g.T;
   const int E = g.E, k = g.k;
   const float* noise_row = (g.noisy && valid) ? g.noise + t * E : nullptr;
-  const bool full_softmax = !g.noisy && !g.renorm;
+  const float* bias = g.bias;
+  const bool noisy = g.noisy != 0;
+  const bool full_softmax = !noisy && !g.renorm;
 
   float* pv = reinterpret_cast<float*>(smem);                    // [G][128][KM+1]
   int* pi = reinterpret_cast<int*>(pv + G * 128 * (KM + 1));     // [G][128][KM+1]
@@ -108,41 +113,43 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
   int* fid = reinterpret_cast<int*>(ps + G * 128);               // [128][KM]
   float* fgate = reinterpret_cast<float*>(fid + 128 * KM);       // [128][KM]
   float* fkth = fgate + 128 * KM;                                // [128][2]
-  float* tr = fkth + 128 * 2;                                    // [4G warps][32][33]
-  float* qsum = tr + 4 * G * 32 * 33;                            // [4][2][E]
+  float* tr = fkth + 128 * 2;                                    // [4G warps][2][32][33]
+  float* qsum = tr + 4 * G * 2 * 32 * 33;                        // [4][2][E]
 
   // ---- pass 1: partial top-(k+1) and softmax statistics over this thread's experts
   TopList<KM> top;
   top.init();
   float m = -INFINITY, ssum = 0.0f;
-  for (int c = grp * 32; c < E; c += 32 * G) {
-    float l[32], z[32];
-    fetch(c, l, z);
-    float sc[32];
+  for (int c0 = grp * 32; c0 < E; c0 += 32 * G) {
+#pragma unroll 1
+    for (int c = c0; c < c0 + 32 && c < E; c += 8) {
+      float l[8], z[8], sc[8];
+      fetch(c, l, z);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int e = c + j;
-      float s = -INFINITY;
-      if (e < E) {
-        s = l[j] + (g.bias ? __ldg(g.bias + e) : 0.0f);
-        if (g.noisy) s += (noise_row ? __ldg(noise_row + e) : 0.0f) * softplus_f(z[j]);
+      for (int j = 0; j < 8; ++j) {
+        const int e = c + j;
+        float s = -INFINITY;
+        if (e < E) {
+          s = l[j] + (bias ? __ldg(bias + e) : 0.0f);
+          if (noisy) s += (noise_row ? __ldg(noise_row + e) : 0.0f) * softplus_f(z[j]);
+        }
+        sc[j] = s;
       }
-      sc[j] = s;
+      if (full_softmax) {
+        float cm = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) cm = fmaxf(cm, sc[j]);
+        const float nm = fmaxf(m, cm);
+        float cs = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) cs += (c + j < E) ? __expf(sc[j] - nm) : 0.0f;
+        ssum = (m == -INFINITY ? 0.0f : ssum * __expf(m - nm)) + cs;
+        m = nm;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (c + j < E) top.insert(sc[j], c + j, k);
     }
-    if (full_softmax) {
-      float cm = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) cm = fmaxf(cm, sc[j]);
-      const float nm = fmaxf(m, cm);
-      float cs = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) cs += (c + j < E) ? expf(sc[j] - nm) : 0.0f;
-      ssum = (m == -INFINITY ? 0.0f : ssum * expf(m - nm)) + cs;
-      m = nm;
-    }
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (c + j < E) top.insert(sc[j], c + j, k);
   }
 #pragma unroll
   for (int s2 = 0; s2 <= KM; ++s2) {
@@ -155,6 +162,7 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
 
   // ---- merge the G partial results of each token (group 0) and write the outputs
   if (grp == 0) {
+#pragma unroll 1
     for (int g2 = 1; g2 < G; ++g2) {
 #pragma unroll
       for (int s2 = 0; s2 <= KM; ++s2)
@@ -209,48 +217,56 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
 
   // ---- pass 2: Importance and Load partial sums over this tile's tokens
   const float kth = fkth[row * 2 + 0], kth1 = fkth[row * 2 + 1];
-  int ids[KM];
-  float gts[KM];
+  float* mytr = tr + warp * (2 * 32 * 33);
+  for (int c0 = grp * 32; c0 < E; c0 += 32 * G) {
+#pragma unroll 1
+    for (int c = c0; c < c0 + 32; c += 8) {
+      float gi[8], pl[8];
 #pragma unroll
-  for (int j = 0; j < KM; ++j) {
-    ids[j] = fid[row * KM + j];
-    gts[j] = fgate[row * KM + j];
-  }
-  float* mytr = tr + warp * (32 * 33);
-  for (int c = grp * 32; c < E; c += 32 * G) {
-    float l[32], z[32];
-    fetch(c, l, z);
-    float gi[32], pl[32];
+      for (int j = 0; j < 8; ++j) {
+        gi[j] = 0.0f;
+        pl[j] = 0.0f;
+      }
+      if (c < E) {
+        float l[8], z[8];
+        fetch(c, l, z);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int e = c + j;
-      gi[j] = 0.0f;
-      pl[j] = 0.0f;
-      if (valid && e < E) {
-        if (g.noisy && k < E) {
-          // recomputed exactly as in pass 1, so H >= kth means "among the top k"
-          const float li = l[j] + (g.bias ? __ldg(g.bias + e) : 0.0f);
-          const float sp = softplus_f(z[j]);
-          const float H = li + __ldg(noise_row + e) * sp;
-          const float ex = (H >= kth) ? kth1 : kth;  // kth_excluding(H, k, e)
-          pl[j] = 0.5f * erfcf(-((li - ex) / sp) * 0.70710678118654752f);
+        for (int j = 0; j < 8; ++j) {
+          const int e = c + j;
+          if (valid && e < E) {
+            if (noisy && k < E) {
+              // recomputed exactly as in pass 1, so H >= kth means "among the top k"
+              const float li = l[j] + (bias ? __ldg(bias + e) : 0.0f);
+              const float sp = softplus_f(z[j]);
+              const float H = li + __ldg(noise_row + e) * sp;
+              const float ex = (H >= kth) ? kth1 : kth;  // kth_excluding(H, k, e)
+              pl[j] = 0.5f * erfcf(-((li - ex) / sp) * 0.70710678118654752f);
+            }
+#pragma unroll 1
+            for (int jj = 0; jj < k; ++jj)
+              if (fid[row * KM + jj] == e) gi[j] = fgate[row * KM + jj];
+          }
         }
+      }
 #pragma unroll
-        for (int jj = 0; jj < KM; ++jj)
-          if (ids[jj] == e) gi[j] = gts[jj];
+      for (int j = 0; j < 8; ++j) {
+        mytr[lane * 33 + (c - c0) + j] = gi[j];
+        mytr[32 * 33 + lane * 33 + (c - c0) + j] = pl[j];
       }
     }
-    // column sums over the warp's 32 tokens through a padded transpose
-#pragma unroll
-    for (int pass = 0; pass < 2; ++pass) {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) mytr[lane * 33 + j] = pass == 0 ? gi[j] : pl[j];
-      __syncwarp();
-      float acc = 0.0f;
-      for (int r = 0; r < 32; ++r) acc += mytr[r * 33 + lane];
-      if (c + lane < E) qsum[(q * 2 + pass) * E + c + lane] = acc;
-      __syncwarp();
+    // column sums over the warp's 32 tokens through the padded transpose
+    __syncwarp();
+    float si = 0.0f, sl = 0.0f;
+#pragma unroll 4
+    for (int r = 0; r < 32; ++r) {
+      si += mytr[r * 33 + lane];
+      sl += mytr[32 * 33 + r * 33 + lane];
     }
+    if (c0 + lane < E) {
+      qsum[(q * 2 + 0) * E + c0 + lane] = si;
+      qsum[(q * 2 + 1) * E + c0 + lane] = sl;
+    }
+    __syncwarp();
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -400,22 +416,22 @@ __global__ void __launch_bounds__(128 * G, 1)
   if (ok) {
     // warp w reads TMEM lanes 32*(w%4) .. +31: its token rows
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    auto fetch = [&](int c, float (&l)[32], float (&z)[32]) {
-      uint32_t v[32];
-      tmem_ld32(tmem_base + lane_base + c, v);
+    auto fetch = [&](int c, float (&l)[8], float (&z)[8]) {
+      uint32_t v[8];
+      tmem_ld8(tmem_base + lane_base + c, v);
       if (a.nb == 2) {
-        uint32_t w[32];
-        tmem_ld32(tmem_base + lane_base + a.acc_cols + c, w);
+        uint32_t w[8];
+        tmem_ld8(tmem_base + lane_base + a.acc_cols + c, w);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) z[j] = __uint_as_float(w[j]);
+        for (int j = 0; j < 8; ++j) z[j] = __uint_as_float(w[j]);
       } else {
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) z[j] = 0.0f;
+        for (int j = 0; j < 8; ++j) z[j] = 0.0f;
       }
 #pragma unroll
-      for (int j = 0; j < 32; ++j) l[j] = __uint_as_float(v[j]);
+      for (int j = 0; j < 8; ++j) l[j] = __uint_as_float(v[j]);
     };
     // the stage buffers are idle once `done` has fired: reuse them for the gate
     gate_tile<KM, G>(fetch, t0, a.g, smem);
@@ -440,9 +456,9 @@ __global__ void __launch_bounds__(128, 1)
   const int64_t t = t0 + threadIdx.x;
   const bool valid = t < g.T;
   const int E = g.E;
-  auto fetch = [&](int c, float (&l)[32], float (&z)[32]) {
+  auto fetch = [&](int c, float (&l)[8], float (&z)[8]) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < 8; ++j) {
       const bool in = valid && (c + j < E);
       l[j] = in ? logits[t * E + c + j] : 0.0f;
       z[j] = (in && nz != nullptr) ? nz[t * E + c + j] : 0.0f;

@@ -179,3 +179,19 @@ def test_bf16_to_f16_reencoding():
         big = src.double().abs() >= 2.0 ** -17
         fin = src.double().abs() <= 65504
         assert torch.equal(ref.double()[big & fin], src.double()[big & fin])
+
+
+def test_fast_erf_matches_cuda_erff():
+    """The GELU epilogue's erf (Abramowitz & Stegun 7.1.26) stays within its published
+    error bound of CUDA's erff, plus float rounding."""
+    import ctypes
+    import sparsely_gated_mixture_moe_b200 as moe
+    x = torch.cat([torch.linspace(-12, 12, 2_000_001), torch.tensor(
+        [0.0, -0.0, 1e-30, -1e-30, float("inf"), float("-inf"), 3.4e38, -3.4e38])]).cuda()
+    fast, ref = torch.empty_like(x), torch.empty_like(x)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    assert moe.lib.moe_erf_check(p(x), p(fast), p(ref), x.numel(), None) == 0
+    torch.cuda.synchronize()
+    d = (fast - ref).abs()
+    assert float(d.max()) <= 2.5e-7, float(d.max())
+    assert fast[-4].item() == 1.0 and fast[-3].item() == -1.0
