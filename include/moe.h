@@ -87,7 +87,10 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * Ties go to the lowest expert index; chosen experts are listed largest score first. */
 typedef enum { MOE_GATE_SOFTMAX_TOPK = 0, MOE_GATE_NOISY_TOPK = 1 } moe_gating;
 
-/* Expert activation: ReLU, or GELU in its exact form 0.5 z (1 + erf(z / sqrt 2)). */
+/* Expert activation: ReLU, or GELU in its erf form 0.5 z (1 + erf(z / sqrt 2)) (not the
+ * tanh approximation).  The bf16 tensor-core path evaluates erf by Abramowitz & Stegun
+ * formula 7.1.26 (|error| <= 1.5e-7, far below the 16-bit rounding of h that follows);
+ * the fp32 path uses CUDA's erff. */
 typedef enum { MOE_ACT_RELU = 0, MOE_ACT_GELU = 1 } moe_act;
 
 typedef struct {
