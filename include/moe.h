@@ -241,7 +241,8 @@ moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_idx, c
                                int32_t* slot_pos, void* x_perm, moe_stream_t stream);
 
 /* Diagnostic: evaluates, for n fp32 inputs x, the erf approximation the GELU epilogue of
- * the tensor-core FFN uses (Abramowitz & Stegun formula 7.1.26, |error| <= 1.5e-7) into
+ * the tensor-core FFN uses (Abramowitz & Stegun formula 7.1.26, |error| <= 1.5e-7; with its fast fp32 evaluation
+ * within 1e-6 of erff) into
  * fast[] and CUDA's erff into ref[], so a test can bound their difference.  No
  * counterpart on the pages (they do not fix the GELU form).  All pointers device. */
 moe_status moe_erf_check(const float* x, float* fast, float* ref, int64_t n,
