@@ -214,24 +214,25 @@ moe_status moe_bf16_to_f16(const void* src, void* dst, int64_t n, int32_t* n_ine
                            moe_stream_t stream);
 
 /* moe_permute for callers that cannot allocate device memory.  It takes no workspace:
- * its scratch (one int32 per 2048-assignment chunk and expert) is a fixed array of
- * MOE_NOALLOC_SCRATCH_BYTES inside libmoe's own device memory, which every GPU that
- * loads the library holds until the process exits.  The pages have no counterpart; this
- * is plumbing for hosts that own all device memory or forbid allocation where they call
- * us: plugins running inside another runtime's memory arena, code on a latency path where
- * cudaMalloc's implicit synchronisation and possible failure are not acceptable, and
- * callbacks in which CUDA allocation calls are not allowed.
+ * its scratch (a 256-byte counter block, then one int32 per 256-assignment chunk and
+ * expert) is a fixed array of MOE_NOALLOC_SCRATCH_BYTES inside libmoe's own device
+ * memory, which every GPU that loads the library holds until the process exits.  The
+ * pages have no counterpart; this is plumbing for hosts that own all device memory or
+ * forbid allocation where they call us: plugins running inside another runtime's memory
+ * arena, code on a latency path where cudaMalloc's implicit synchronisation and possible
+ * failure are not acceptable, and callbacks in which CUDA allocation calls are not
+ * allowed.
  *  Arguments, outputs and results are those of moe_permute, bit for bit.
- *  Sizes: ceil(T*k / 2048) * E * 4 must not exceed MOE_NOALLOC_SCRATCH_BYTES (for E = 128
- *  that is T*k up to 4,194,304); larger problems return MOE_ERR_UNSUPPORTED and queue
- *  nothing.
+ *  Sizes: 256 + ceil(T*k / 256) * E * 4 must not exceed MOE_NOALLOC_SCRATCH_BYTES (for
+ *  E = 128 that is T*k up to 524,032); larger problems return MOE_ERR_UNSUPPORTED and
+ *  queue nothing.
  *  Set-up: the first call on a device, with that device current, looks up the array's
  *  device address (cudaGetSymbolAddress) and caches it; make that first call before any
  *  stream capture.
- *  Sharing: every call uses the same array, which keeps the previous call's contents
- *  (each call rewrites all it reads, so nothing needs clearing); calls whose work
- *  overlaps on the GPU (other streams, other host threads) race on it and must be
- *  serialised by the caller.
+ *  Sharing: every call uses the same array, which keeps the previous call's contents;
+ *  each call clears the counter that must start at zero (cudaMemsetAsync on `stream`) and
+ *  rewrites everything else it reads.  Calls whose work overlaps on the GPU (other
+ *  streams, other host threads) race on the array and must be serialised by the caller.
  *  Errors: there is no device error word: an out-of-range expert index is treated as
  *  dropped without a report.  Never calls cudaMalloc, cudaFree or any allocating
  *  routine. */

@@ -52,7 +52,31 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
     }
   }
   const int nv = d / V;
-  for (int v = lane; v < nv; v += 32) {
+  // four vectors per lane per step so that several loads per slot are in flight
+  int v = lane;
+  for (; v + 96 < nv; v += 128) {
+    float acc[4][V];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[u][i] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (slot[j] >= 0) {
+        const T* src = y_perm + static_cast<int64_t>(slot[j]) * d + v * V;
+        float r[4][V];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) Vec<T>::load(src + u * 32 * V, r[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int i = 0; i < V; ++i) acc[u][i] = fmaf(g[j], r[u][i], acc[u][i]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) Vec<T>::store(y + t * d + (v + u * 32) * V, acc[u]);
+  }
+  for (; v < nv; v += 32) {
     float acc[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = 0.0f;

@@ -43,7 +43,7 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c);
 cudaError_t launch_route_f32(const RouteProblem& p, const LaunchCtx& c);
 
 // ---- permute ---------------------------------------------------------------------
-constexpr int kPermChunk = 2048;  // assignments per permute block
+constexpr int kPermChunk = 256;  // assignments per permute block (one per thread)
 struct PermuteProblem {
   int64_t n;  // T*k assignments
   int k, E, d, esize;
@@ -55,7 +55,8 @@ struct PermuteProblem {
   int32_t* perm_src;
   int32_t* slot_pos;
   void* x_perm;
-  int32_t* blk;  // workspace [nblk][E]
+  int32_t* blk;     // workspace [nblk][E]
+  int32_t* ticket;  // workspace counter, zero between calls
 };
 int64_t permute_blocks(int64_t n);
 cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c);

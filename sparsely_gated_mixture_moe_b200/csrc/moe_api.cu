@@ -178,6 +178,7 @@ moe_status do_permute(const moe_config* cfg, const Layout& L, const int32_t* top
   p.slot_pos = slot_pos;
   p.x_perm = x_perm;
   p.blk = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + L.blk);
+  p.ticket = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + L.err + 8);
   return launch_permute(p, ctx.lc) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -6,17 +6,17 @@
 // only the first C assignments of an expert are kept (capacity factor, "moe paper models"
 // Table 2), the rest are dropped (slot_pos = -1).
 //
-// Four kernels, no atomics on global memory and no cross-block waits:
-//   count    block b counts its chunk of 2048 assignments per expert (shared-memory
-//            histogram) -> blk[b][e]
-//   scan     one block: per expert an exclusive scan over the chunks (blk[b][e] becomes
-//            the number of earlier assignments of e), counts[e], kept[e] = min(count, C),
-//            and offsets = exclusive scan of kept
-//   scatter  block b ranks its chunk stably (warp match + per-warp prefix) and writes
-//            slot_pos / perm_src
-//   gather   x_perm[s] = x[perm_src[s] / k] for every kept row s < offsets[E]: one warp
-//            per row, 16-byte vectors, a grid of several blocks per SM so that enough
-//            loads are in flight to stream at HBM rate
+// Three kernels, no cross-block waits:
+//   count+scan  block b counts its chunk of 256 assignments per expert (shared-memory
+//               histogram) into blk[b][e]; the last block to finish (a ticket counter)
+//               turns blk into per-chunk rank bases with a segmented scan over the chunks,
+//               writes counts[e], kept[e] = min(count, C) and offsets (exclusive scan of
+//               kept), and resets the ticket
+//   scatter     block b ranks its chunk stably (warp match + per-warp prefix) and writes
+//               slot_pos / perm_src
+//   gather      x_perm[s] = x[perm_src[s] / k] for every kept row s < offsets[E]: one warp
+//               per row, 16-byte vectors, a grid of several blocks per SM so that enough
+//               loads are in flight to stream at HBM rate
 #include <mutex>
 
 #include "common.cuh"
@@ -26,112 +26,131 @@ namespace moe {
 namespace pm {
 constexpr int THREADS = 256;
 constexpr int WARPS = THREADS / 32;
-constexpr int PER_WARP = kPermChunk / WARPS;  // 256 assignments per warp, 8 rounds of 32
-constexpr int SCAN_THREADS = 1024;
+static_assert(kPermChunk == THREADS, "one assignment per thread per chunk");
 }  // namespace pm
 
 int64_t permute_blocks(int64_t n) { return (n + kPermChunk - 1) / kPermChunk; }
 
-__global__ void __launch_bounds__(pm::THREADS)
-    perm_count_kernel(const int32_t* __restrict__ idx, int64_t n, int E, int32_t* __restrict__ blk,
-                      int* err) {
-  extern __shared__ int hist[];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
-  __syncthreads();
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * kPermChunk;
-  for (int i = threadIdx.x; i < kPermChunk; i += blockDim.x) {
-    const int64_t a = base + i;
-    if (a >= n) break;
-    const int e = idx[a];
-    if (e < 0 || e >= E) {
-      set_error(err, kErrExpertIndex);
-      continue;
-    }
-    atomicAdd(&hist[e], 1);
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    blk[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
-}
+// Shared memory of perm_count_scan_kernel: hist[E] and, for the scan, seg[2][256] and
+// kept[E] ints.
+static size_t count_scan_smem(int E) { return (static_cast<size_t>(E) * 2 + 512 + 64) * 4; }
 
-__global__ void __launch_bounds__(pm::SCAN_THREADS)
-    perm_scan_kernel(int32_t* __restrict__ blk, int nblk, int E, int64_t C,
-                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
-  extern __shared__ int kept[];  // [E]
-  __shared__ int scratch[40];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = 0;
-    for (int b = 0; b < nblk; ++b) {
-      const int64_t i = static_cast<int64_t>(b) * E + e;
-      const int cnt = blk[i];
-      blk[i] = run;
-      run += cnt;
-    }
-    counts[e] = run;
-    kept[e] = (C >= 0 && run > C) ? static_cast<int>(C) : run;
+__global__ void __launch_bounds__(pm::THREADS)
+    perm_count_scan_kernel(const int32_t* __restrict__ idx, int64_t n, int E, int64_t C,
+                           int32_t* __restrict__ blk, int32_t* __restrict__ counts,
+                           int32_t* __restrict__ offsets, int32_t* ticket, int* err) {
+  extern __shared__ int sm[];
+  int* hist = sm;                 // [E]
+  int* seg = hist + E;            // [256] segment sums, then segment bases
+  int* kept = seg + 512;          // [E]
+  int* scratch = kept + E;        // [40]
+  __shared__ int s_last;
+  const int tid = threadIdx.x;
+  const int nblk = gridDim.x;
+  for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int64_t a = static_cast<int64_t>(blockIdx.x) * kPermChunk + tid;
+  if (a < n) {
+    const int e = idx[a];
+    if (e < 0 || e >= E) set_error(err, kErrExpertIndex);
+    else atomicAdd(&hist[e], 1);
   }
   __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) blk[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(ticket, 1) == nblk - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  // ---- last block: per expert, exclusive scan of blk[.][e] over the chunks.  With
+  // E < 256 several threads share an expert, each owning a contiguous run of chunks.
+  int tpe = 1;
+  while (tpe * 2 * E <= pm::THREADS) tpe *= 2;
+  const int len = (nblk + tpe - 1) / tpe;
+  for (int e0 = 0; e0 < E; e0 += pm::THREADS / tpe) {
+    const int e = e0 + tid % (pm::THREADS / tpe);
+    const int part = tid / (pm::THREADS / tpe);
+    const bool act = (tid % (pm::THREADS / tpe)) < (pm::THREADS / tpe) && e < E && part < tpe;
+    const int b0 = part * len, b1 = min(nblk, b0 + len);
+    int sum = 0;
+    if (act)
+      for (int b = b0; b < b1; ++b) sum += __ldcg(blk + static_cast<int64_t>(b) * E + e);
+    if (act) seg[part * (pm::THREADS / tpe) + (e - e0)] = sum;
+    __syncthreads();
+    if (act && part == 0) {
+      int run = 0;
+      for (int q = 0; q < tpe; ++q) {
+        const int v = seg[q * (pm::THREADS / tpe) + (e - e0)];
+        seg[256 + q * (pm::THREADS / tpe) + (e - e0)] = run;
+        run += v;
+      }
+      counts[e] = run;
+      kept[e] = (C >= 0 && run > C) ? static_cast<int>(C) : run;
+    }
+    __syncthreads();
+    if (act) {
+      int run = seg[256 + part * (pm::THREADS / tpe) + (e - e0)];
+      for (int b = b0; b < b1; ++b) {
+        const int64_t i = static_cast<int64_t>(b) * E + e;
+        const int c = __ldcg(blk + i);
+        blk[i] = run;
+        run += c;
+      }
+    }
+    __syncthreads();
+  }
   int carry = 0;
   for (int base = 0; base < E; base += blockDim.x) {
-    const int e = base + threadIdx.x;
+    const int e = base + tid;
     const int v = e < E ? kept[e] : 0;
     int tot;
     const int incl = block_incl_scan(v, scratch, &tot);
     if (e < E) offsets[e] = carry + incl - v;
     carry += tot;
   }
-  if (threadIdx.x == 0) offsets[E] = carry;
+  if (tid == 0) {
+    offsets[E] = carry;
+    *ticket = 0;  // ready for the next call
+  }
 }
 
 __global__ void __launch_bounds__(pm::THREADS)
-    perm_scatter_kernel(const int32_t* __restrict__ idx, int64_t n, int k, int E, int64_t C,
+    perm_scatter_kernel(const int32_t* __restrict__ idx, int64_t n, int E, int64_t C,
                         const int32_t* __restrict__ blk, const int32_t* __restrict__ offsets,
                         int32_t* __restrict__ perm_src, int32_t* __restrict__ slot_pos) {
-  extern __shared__ int wbase[];  // [WARPS][E]: running rank base of each warp per expert
+  extern __shared__ int wbase[];  // [WARPS][E]: rank base of each warp per expert
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * kPermChunk + warp * pm::PER_WARP;
+  const int64_t a = static_cast<int64_t>(blockIdx.x) * kPermChunk + threadIdx.x;
 
   for (int i = threadIdx.x; i < pm::WARPS * E; i += blockDim.x) wbase[i] = 0;
   __syncthreads();
-  // per-warp histogram of this warp's 256 assignments
-  for (int r = 0; r < pm::PER_WARP / 32; ++r) {
-    const int64_t a = base + r * 32 + lane;
-    int e = (a < n) ? idx[a] : -1;
-    if (e < 0 || e >= E) e = -1;
-    const uint32_t peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && (peers & lt_mask) == 0) wbase[warp * E + e] += __popc(peers);
-    __syncwarp();
-  }
+  int e = (a < n) ? idx[a] : -1;
+  if (e < 0 || e >= E) e = -1;
+  const uint32_t peers = __match_any_sync(0xffffffffu, e);
+  if (e >= 0 && (peers & lt_mask) == 0) wbase[warp * E + e] = __popc(peers);
   __syncthreads();
-  // exclusive scan over the warps, offset by the chunk's rank base from the scan kernel
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = blk[static_cast<int64_t>(blockIdx.x) * E + e];
+  // exclusive scan over the warps, offset by the chunk's rank base from the scan
+  for (int x = threadIdx.x; x < E; x += blockDim.x) {
+    int run = blk[static_cast<int64_t>(blockIdx.x) * E + x];
     for (int w = 0; w < pm::WARPS; ++w) {
-      const int c = wbase[w * E + e];
-      wbase[w * E + e] = run;
+      const int c = wbase[w * E + x];
+      wbase[w * E + x] = run;
       run += c;
     }
   }
   __syncthreads();
-  // ranks in assignment order: warp-major, then round, then lane
-  for (int r = 0; r < pm::PER_WARP / 32; ++r) {
-    const int64_t a = base + r * 32 + lane;
-    int e = (a < n) ? idx[a] : -1;
-    if (e < 0 || e >= E) e = -1;
-    const uint32_t peers = __match_any_sync(0xffffffffu, e);
-    int slot = -1;
-    if (e >= 0) {
-      const int rank = wbase[warp * E + e] + __popc(peers & lt_mask);
-      if (C < 0 || rank < C) slot = offsets[e] + rank;
-    }
-    __syncwarp();
-    if (e >= 0 && (peers & lt_mask) == 0) wbase[warp * E + e] += __popc(peers);
-    if (a < n) {
-      slot_pos[a] = slot;
-      if (slot >= 0) perm_src[slot] = static_cast<int32_t>(a);
-    }
-    __syncwarp();
+  // ranks in assignment order: warp, then lane
+  int slot = -1;
+  if (e >= 0) {
+    const int rank = wbase[warp * E + e] + __popc(peers & lt_mask);
+    if (C < 0 || rank < C) slot = offsets[e] + rank;
+  }
+  if (a < n) {
+    slot_pos[a] = slot;
+    if (slot >= 0) perm_src[slot] = static_cast<int32_t>(a);
   }
 }
 
@@ -165,14 +184,15 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
 cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c) {
   const int64_t nblk = permute_blocks(p.n);
   if (nblk == 0) return cudaSuccess;
-  const size_t hist_smem = static_cast<size_t>(p.E) * 4;
-  perm_count_kernel<<<static_cast<unsigned>(nblk), pm::THREADS, hist_smem, c.stream>>>(
-      p.topk_idx, p.n, p.E, p.blk, c.err);
-  ++*c.launches;
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  perm_scan_kernel<<<1, pm::SCAN_THREADS, hist_smem, c.stream>>>(p.blk, static_cast<int>(nblk), p.E,
-                                                                 p.C, p.counts, p.offsets);
+  cudaError_t e = cudaSuccess;
+  const size_t cs_smem = count_scan_smem(p.E);
+  if (cs_smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(perm_count_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(cs_smem));
+    if (e != cudaSuccess) return e;
+  }
+  perm_count_scan_kernel<<<static_cast<unsigned>(nblk), pm::THREADS, cs_smem, c.stream>>>(
+      p.topk_idx, p.n, p.E, p.C, p.blk, p.counts, p.offsets, p.ticket, c.err);
   ++*c.launches;
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -183,7 +203,7 @@ cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c) {
     if (e != cudaSuccess) return e;
   }
   perm_scatter_kernel<<<static_cast<unsigned>(nblk), pm::THREADS, wsmem, c.stream>>>(
-      p.topk_idx, p.n, p.k, p.E, p.C, p.blk, p.offsets, p.perm_src, p.slot_pos);
+      p.topk_idx, p.n, p.E, p.C, p.blk, p.offsets, p.perm_src, p.slot_pos);
   ++*c.launches;
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -254,8 +274,8 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
   if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(x_perm) & 15u))
     return MOE_ERR_INVALID_ARG;
   const int64_t n = cfg->T * cfg->k;
-  // the scratch holds one int32 per (2048-assignment chunk, expert)
-  if (permute_blocks(n) * cfg->E * 4 > static_cast<int64_t>(MOE_NOALLOC_SCRATCH_BYTES))
+  // the scratch holds a 256-byte counter block, then one int32 per (chunk, expert)
+  if (256 + permute_blocks(n) * cfg->E * 4 > static_cast<int64_t>(MOE_NOALLOC_SCRATCH_BYTES))
     return MOE_ERR_UNSUPPORTED;
   int dev = 0;
   LaunchCtx c;
@@ -282,7 +302,11 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
   p.perm_src = perm_src;
   p.slot_pos = slot_pos;
   p.x_perm = x_perm;
-  p.blk = static_cast<int32_t*>(scratch);  // fully rewritten by the count kernel each call
+  // the ticket must start at zero: clear it (a call cut short could have left it set);
+  // the per-chunk counts are fully rewritten by the count kernel each call
+  p.ticket = static_cast<int32_t*>(scratch);
+  p.blk = static_cast<int32_t*>(scratch) + 64;
+  if (cudaMemsetAsync(p.ticket, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
   if (launch_permute(p, c) != cudaSuccess) return MOE_ERR_CUDA;
   set_last_launch_count(launches);
   return MOE_OK;

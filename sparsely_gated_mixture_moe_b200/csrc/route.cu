@@ -102,6 +102,19 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
   const bool valid = t < g.T;
   const int E = g.E, k = g.k;
   const float* noise_row = (g.noisy && valid) ? g.noise + t * E : nullptr;
+  // 8 noise draws per step, as two 16-byte loads when the rows keep 16-byte alignment
+  const bool noise_vec = g.noisy && (E % 4 == 0) && ((reinterpret_cast<uintptr_t>(g.noise) & 15u) == 0);
+  auto load_noise8 = [&](int c, float (&nz)[8]) {
+    if (noise_row != nullptr && noise_vec && c + 8 <= E) {
+      const float4 u0 = __ldg(reinterpret_cast<const float4*>(noise_row + c));
+      const float4 u1 = __ldg(reinterpret_cast<const float4*>(noise_row + c + 4));
+      nz[0] = u0.x; nz[1] = u0.y; nz[2] = u0.z; nz[3] = u0.w;
+      nz[4] = u1.x; nz[5] = u1.y; nz[6] = u1.z; nz[7] = u1.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) nz[j] = (noise_row != nullptr && c + j < E) ? __ldg(noise_row + c + j) : 0.0f;
+    }
+  };
   const float* bias = g.bias;
   const bool noisy = g.noisy != 0;
   const bool full_softmax = !noisy && !g.renorm;
@@ -123,15 +136,16 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
   for (int c0 = grp * 32; c0 < E; c0 += 32 * G) {
 #pragma unroll 1
     for (int c = c0; c < c0 + 32 && c < E; c += 8) {
-      float l[8], z[8], sc[8];
+      float l[8], z[8], sc[8], nz[8];
       fetch(c, l, z);
+      if (noisy) load_noise8(c, nz);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int e = c + j;
         float s = -INFINITY;
         if (e < E) {
           s = l[j] + (bias ? __ldg(bias + e) : 0.0f);
-          if (noisy) s += (noise_row ? __ldg(noise_row + e) : 0.0f) * softplus_f(z[j]);
+          if (noisy) s += nz[j] * softplus_f(z[j]);
         }
         sc[j] = s;
       }
@@ -189,11 +203,14 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
 #pragma unroll
       for (int j = 0; j < KM; ++j) gate[j] /= den;
     }
-    float kth = -INFINITY, kth1 = -INFINITY;  // k-th and (k+1)-th largest scores
+    // k-th and (k+1)-th largest scores.  The list is sorted, so they are the minimum of
+    // the first k entries and the maximum of the rest; written as predicated min/max (a
+    // select on j == k would become an indexed load and push the list to local memory).
+    float kth = INFINITY, kth1 = -INFINITY;
 #pragma unroll
     for (int j = 0; j <= KM; ++j) {
-      if (j == k - 1) kth = top.v[j];
-      if (j == k) kth1 = top.v[j];
+      if (j < k) kth = fminf(kth, top.v[j]);
+      else kth1 = fmaxf(kth1, top.v[j]);
     }
     if (valid) {
 #pragma unroll
@@ -228,8 +245,9 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
         pl[j] = 0.0f;
       }
       if (c < E) {
-        float l[8], z[8];
+        float l[8], z[8], nz[8];
         fetch(c, l, z);
+        if (noisy) load_noise8(c, nz);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int e = c + j;
@@ -238,7 +256,7 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
               // recomputed exactly as in pass 1, so H >= kth means "among the top k"
               const float li = l[j] + (bias ? __ldg(bias + e) : 0.0f);
               const float sp = softplus_f(z[j]);
-              const float H = li + __ldg(noise_row + e) * sp;
+              const float H = li + nz[j] * sp;
               const float ex = (H >= kth) ? kth1 : kth;  // kth_excluding(H, k, e)
               pl[j] = 0.5f * erfcf(-((li - ex) / sp) * 0.70710678118654752f);
             }
