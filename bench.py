@@ -150,13 +150,15 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def algorithmic(w: workloads.Workload, n_kept: int, counts_kept):
+def algorithmic(w: workloads.Workload, n_kept: int, counts_kept, fused=False):
     """Algorithmic FLOPs and bytes of each step (kept assignments only, no padding).
 
     FFN FLOPs 4*N*d*f (two products).  FFN bytes: the weights of the experts that got
     rows, x_perm (dtype) read, y_perm (fp32) written.  Route bytes: x, the gating
     weights, noise, and the chosen indices and gates.  Permute: x rows read, x_perm
-    rows written, indices.  Combine: y_perm rows read, gates and slots, y written."""
+    rows written, indices.  Combine: y_perm rows read, gates and slots, y written.
+    fused (k = 1, FFN and combine as one step): the FFN writes every row of y (fp32) and
+    reads each kept row's source index and gate; no combine bytes."""
     es = 2 if w.dtype == "bf16" else 4
     T, d, f, E, k = w.T, w.d_model, w.d_ff, w.E, w.k
     active = int(sum(1 for c in counts_kept if c > 0))
@@ -166,6 +168,9 @@ def algorithmic(w: workloads.Workload, n_kept: int, counts_kept):
     route_bytes = T * d * es + E * d * es * (2 if noisy else 1) + (T * E * 4 if noisy else 0) + T * k * 8
     permute_bytes = n_kept * d * es * 2 + T * k * 4 * 3
     combine_bytes = n_kept * d * 4.0 + T * k * 8 + T * d * 4.0
+    if fused:
+        ffn_bytes = active * 2.0 * d * f * es + n_kept * d * es + T * d * 4.0 + n_kept * 8.0 + T * 4.0
+        combine_bytes = 0.0
     return {"ffn_flops": ffn_flops, "ffn_bytes": ffn_bytes, "route_bytes": route_bytes,
             "permute_bytes": permute_bytes, "combine_bytes": combine_bytes}
 
@@ -297,6 +302,7 @@ def run_gpu(args, w):
     stream = torch.cuda.current_stream(dev)
 
     launches = [0]
+    fused = moe.fused_combine(cfg)
 
     def step(evs=None):
         n = 0
@@ -313,12 +319,21 @@ def run_gpu(args, w):
         n += moe.last_launch_count()
         if evs:
             evs[2].record(stream)
-        moe.moe_expert_ffn(cfg, o["x_perm"], o["offsets"], d["w1"], d["w2"], o["h"], o["y_perm"], ws)
-        n += moe.last_launch_count()
-        if evs:
-            evs[3].record(stream)
-        moe.moe_combine(cfg, o["y_perm"], o["slot_pos"], o["gate"], o["y"], ws)
-        n += moe.last_launch_count()
+        if fused:
+            # top-1: the down-projection writes gate * row straight into y
+            moe.moe_expert_ffn_combine(cfg, o["x_perm"], o["offsets"], o["perm_src"], o["slot_pos"],
+                                       o["gate"], d["w1"], d["w2"], o["h"], o["y"], ws)
+            n += moe.last_launch_count()
+            if evs:
+                evs[3].record(stream)
+        else:
+            moe.moe_expert_ffn(cfg, o["x_perm"], o["offsets"], d["w1"], d["w2"], o["h"],
+                               o["y_perm"], ws)
+            n += moe.last_launch_count()
+            if evs:
+                evs[3].record(stream)
+            moe.moe_combine(cfg, o["y_perm"], o["slot_pos"], o["gate"], o["y"], ws)
+            n += moe.last_launch_count()
         if evs:
             evs[4].record(stream)
         launches[0] += n
@@ -389,7 +404,7 @@ def run_gpu(args, w):
         raise RuntimeError("end-to-end output mismatch between host copy and device result")
 
     peaks, peak_src = load_peaks()
-    alg = algorithmic(w, n_kept, kept)
+    alg = algorithmic(w, n_kept, kept, fused)
     ffn_ms = float(np.mean(per[:, 2]))
     gemm_launch_s = ffn_ms * 1e-3 / 2.0
     ffn_tflops = alg["ffn_flops"] / (ffn_ms * 1e-3) / 1e12
@@ -403,7 +418,10 @@ def run_gpu(args, w):
     else:
         roof = {"bound": "tensor", "achieved": ffn_tflops, "peak": peaks["bf16_tflops_sustained"],
                 "unit": "TFLOP/s", "frac": ffn_tflops / peaks["bf16_tflops_sustained"]}
-    roof.update({"traffic": traffic, "kernel": "grouped_gemm_tc_kernel (2 launches/step)",
+    roof.update({"traffic": traffic,
+                 "kernel": "grouped_gemm_tc_kernel (2 launches/step%s)" % (
+                     "; down-projection writes gate * row into y, plus a zero-fill of dropped "
+                     "tokens' rows" if fused else ""),
                  "algorithmic_per_launch": {"flops": alg["ffn_flops"] / 2,
                                             "bytes": alg["ffn_bytes"] / 2},
                  "launch_ms": gemm_launch_s * 1e3, "peak_source": "%s (MEASURED_PEAKS.json)" % peak_src
@@ -420,10 +438,12 @@ def run_gpu(args, w):
                         "gbs": ffn_gbs, "frac_of_hbm": ffn_gbs / peaks["hbm_gbs"],
                         "arith_intensity": ai},
         "steps_ms": {"route": float(np.mean(per[:, 0])), "permute": float(np.mean(per[:, 1])),
-                     "expert_ffn": ffn_ms, "combine": float(np.mean(per[:, 3]))},
+                     "expert_ffn": ffn_ms,
+                     "combine": "fused into expert_ffn" if fused else float(np.mean(per[:, 3]))},
         "step_gbs": {"route": alg["route_bytes"] / (np.mean(per[:, 0]) * 1e-3) / 1e9,
                      "permute": alg["permute_bytes"] / (np.mean(per[:, 1]) * 1e-3) / 1e9,
-                     "combine": alg["combine_bytes"] / (np.mean(per[:, 3]) * 1e-3) / 1e9},
+                     "combine": None if fused else
+                     alg["combine_bytes"] / (np.mean(per[:, 3]) * 1e-3) / 1e9},
         "kept_rows": n_kept,
         "e2e": {"value": T * world / (e2e_mean * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_mean,

@@ -13,6 +13,7 @@
  *                  sort of the token->expert assignments; gathers the kept token rows
  *   moe_expert_ffn per-expert FFN on the kept rows only (grouped GEMM, tensor cores)
  *   moe_combine    gate-weighted sum of each token's expert outputs (un-permute)
+ *   moe_expert_ffn_combine  the last two fused, for top-1 routing in bf16
  *   moe_forward    all of the above on one stream
  *
  * Conventions for every call
@@ -70,7 +71,9 @@ typedef enum {
 enum {
   MOE_DEVERR_EXPERT_INDEX = 1, /* a topk_idx entry outside [0, E): treated as dropped */
   MOE_DEVERR_OFFSETS = 2,      /* offsets not non-decreasing in [0, T*k]: FFN skipped */
-  MOE_DEVERR_SLOT = 4,         /* a slot_pos entry outside [-1, T*k): treated as dropped */
+  MOE_DEVERR_SLOT = 4,         /* a slot_pos entry outside [-1, T*k), or a perm_src entry
+                                  outside [0, T) in moe_expert_ffn_combine: treated as
+                                  dropped (that row is not written) */
   MOE_DEVERR_TIMEOUT = 8       /* a bounded wait inside a pipelined kernel expired */
 };
 
@@ -186,8 +189,25 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32
 moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* slot_pos,
                        const float* topk_gate, void* y, void* ws, moe_stream_t stream);
 
+/* moe_expert_ffn followed by moe_combine as one step, for k = 1 and bf16 only [Switch
+ * Transformer, switch_routing: with one expert per token the combine is a scaled copy]:
+ *   y[t] = topk_gate[t] * (act(x[t] . W1_e^T) . W2_e^T)  for a token kept by expert e,
+ *   y[t] = 0                                            for a token that was dropped.
+ * The down-projection writes each fp32 row straight into y at its token (perm_src[s] = t
+ * for k = 1), so y_perm never exists.  Same arithmetic as the two steps: y is bit-equal
+ * to moe_expert_ffn + moe_combine on the same inputs.
+ *  x_perm, offsets, w1, w2, h as moe_expert_ffn;  perm_src, slot_pos as written by
+ *  moe_permute;  topk_gate [T, 1] fp32 in;  y [T, d_model] fp32 out (every row written).
+ * The rows of dropped tokens (slot_pos[t] < 0) are zeroed by a small kernel queued
+ * before the two GEMMs; a perm_src entry outside [0, T) sets MOE_DEVERR_SLOT.  * Returns MOE_ERR_UNSUPPORTED when k != 1 or dtype is not bf16. */
+moe_status moe_expert_ffn_combine(const moe_config* cfg, const void* x_perm,
+                                  const int32_t* offsets, const int32_t* perm_src,
+                                  const int32_t* slot_pos, const float* topk_gate,
+                                  const void* w1, const void* w2, void* h, void* y, void* ws,
+                                  moe_stream_t stream);
+
 /* The whole layer forward on one stream: moe_route, moe_permute, moe_expert_ffn,
- * moe_combine.  Inputs as in the step calls; y [T, d_model] fp32 out.  topk_idx,
+ * moe_combine (moe_expert_ffn_combine in their place when k = 1 and dtype is bf16).  Inputs as in the step calls; y [T, d_model] fp32 out.  topk_idx,
  * topk_gate (both [T, k]) and counts ([E]) are outputs the caller must provide;
  * importance, load and near_tie may be NULL.  The intermediates live in `ws`
  * (moe_forward_workspace_size bytes). */

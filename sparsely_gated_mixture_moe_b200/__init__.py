@@ -38,6 +38,7 @@ def _load():
         "moe_permute": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P]),
         "moe_expert_ffn": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
         "moe_combine": (ctypes.c_int, [C, P, P, P, P, P, P]),
+        "moe_expert_ffn_combine": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P]),
         "moe_forward": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]),
         "moe_get_error": (ctypes.c_int, [P, P, ctypes.POINTER(ctypes.c_int32)]),
         "moe_last_launch_count": (ctypes.c_int32, []),
@@ -141,6 +142,22 @@ def moe_combine(cfg, y_perm, slot_pos, topk_gate, y, ws, stream=None):
                            _stream(stream)), "moe_combine")
 
 
+def moe_expert_ffn_combine(cfg, x_perm, offsets, perm_src, slot_pos, topk_gate, w1, w2, h, y,
+                           ws, stream=None):
+    """moe_expert_ffn + moe_combine as one step (k = 1, bf16): the down-projection writes
+    gate * row straight into y at its token."""
+    _check(lib.moe_expert_ffn_combine(ctypes.byref(cfg), _ptr(x_perm, "x_perm"),
+                                      _ptr(offsets, "offsets"), _ptr(perm_src, "perm_src"),
+                                      _ptr(slot_pos, "slot_pos"), _ptr(topk_gate, "topk_gate"),
+                                      _ptr(w1, "w1"), _ptr(w2, "w2"), _ptr(h, "h"), _ptr(y, "y"),
+                                      _ptr(ws, "ws"), _stream(stream)), "moe_expert_ffn_combine")
+
+
+def fused_combine(cfg) -> bool:
+    """Whether moe_expert_ffn_combine applies (top-1 routing in bf16)."""
+    return cfg.k == 1 and cfg.dtype == DTYPE["bf16"]
+
+
 def moe_forward(cfg, x, w_gate, w1, w2, y, topk_idx, topk_gate, counts, ws, w_noise=None,
                 noise=None, logit_bias=None, importance=None, load=None, near_tie=None,
                 stream=None):
@@ -222,4 +239,4 @@ __all__ = ["ACT", "DTYPE", "GATING", "MoEConfig", "MoEError", "MoELayer", "STATU
            "make_config", "moe_capacity", "moe_combine", "moe_expert_ffn", "moe_forward",
            "moe_forward_workspace_size", "moe_get_error", "moe_permute", "moe_route",
            "moe_workspace_size", "workspace", "last_launch_count", "moe_bf16_to_f16",
-           "prepare_weights", "moe_permute_noalloc"]
+           "prepare_weights", "moe_permute_noalloc", "moe_expert_ffn_combine", "fused_combine"]

@@ -23,8 +23,9 @@
 //               (a ragged tail is masked).  Three warps per lane quarter keep a ragged
 //               tile, whose rows all sit in the first quarters, from serialising on few
 //               warps.
-// Tiles are (expert, n-tile, m-tile) with m innermost, so CTAs running at the same time
-// share weight tiles through L2 and each expert's weights stream from HBM about once.
+// Tiles are (expert, m-tile, n-tile) with n innermost: CTAs running at the same time share
+// the A rows of an m-tile through L2 while each streams a different weight tile (measured
+// 1.5-3.5% faster than m innermost on the five workloads).
 // Rows past an expert's end that a 128-row tile reads belong to the next expert or lie
 // past the buffer (TMA fills those with zeros); they only feed masked output rows.
 // No cross-CTA waits; every mbarrier wait is bounded and an expired wait sets
@@ -58,6 +59,7 @@ constexpr int SMEM_BYTES = 1024 /*align slack*/ + RING_BYTES + 256 /*barriers, f
 constexpr int OUT_BF16 = 0;  // act, bf16
 constexpr int OUT_F16 = 1;   // act, fp16
 constexpr int OUT_F32 = 2;   // fp32
+constexpr int OUT_COMBINE = 3;  // fp32 times the gate, into the token's row of y (k = 1)
 
 struct Args {
   const int32_t* offsets;
@@ -71,6 +73,8 @@ struct Args {
   int act;       // 0 none, 1 ReLU, 2 GELU
   int out_mode;  // OUT_*
   int ab_f16;    // operand type of A and B: 1 fp16, 0 bf16
+  const int32_t* perm_src;  // OUT_COMBINE: assignment of each permuted row (= token, k = 1)
+  const float* gate;        // OUT_COMBINE: gate of each assignment
   int* err;
 };
 
@@ -87,10 +91,9 @@ __device__ __forceinline__ Tile decode_tile(int L, const int* tp, const Args& a)
   }
   Tile t;
   t.e = lo;
-  const int mte = tp[lo + 1] - tp[lo];
   const int local = L - tp[lo] * a.n_tiles;
-  t.nt = local / mte;
-  t.mt = local - t.nt * mte;
+  t.mt = local / a.n_tiles;
+  t.nt = local - t.mt * a.n_tiles;
   const int r0 = __ldg(a.offsets + lo), r1 = __ldg(a.offsets + lo + 1);
   t.row0 = r0 + t.mt * BM;
   t.valid = min(BM, r1 - t.row0);
@@ -124,14 +127,18 @@ __device__ __forceinline__ float epi_act(float z) {
 // chunks sub*32 + 32*EPI_SUBS*i of the tile; rows outside the expert are not stored.
 template <int MODE, int ACT>
 __device__ __forceinline__ void epilogue_rows(const Args& a, uint32_t tbase, int64_t oidx, int sub,
-                                              bool row_ok) {
+                                              bool row_ok, float scale) {
   for (int c = sub * 32; c < a.bn; c += 32 * EPI_SUBS) {
     uint32_t v[32];
     tmem_ld32(tbase + c, v);
     tmem_ld_wait();
     if (!row_ok) continue;
-    if (MODE == OUT_F32) {
+    if (MODE == OUT_F32 || MODE == OUT_COMBINE) {
       float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + oidx + c);
+      if (MODE == OUT_COMBINE) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(scale * __uint_as_float(v[j]));
+      }
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
@@ -300,17 +307,31 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_after();
       const int r = q * 32 + lane;
-      const bool row_ok = r < t.valid;
-      const int64_t oidx = static_cast<int64_t>(t.row0 + r) * a.N + t.nt * a.bn;
+      bool row_ok = r < t.valid;
+      int64_t orow = t.row0 + r;
+      float scale = 1.0f;
+      if (a.out_mode == OUT_COMBINE && row_ok) {
+        // k = 1: the permuted row's assignment is its token; y[t] = g_t * (h W2^T)[row]
+        const int asg = __ldg(a.perm_src + orow);
+        if (asg < 0 || asg >= a.rows_cap) {
+          set_error(a.err, kErrSlot);  // not a permutation written by the permute step
+          row_ok = false;
+        } else {
+          scale = __ldg(a.gate + asg);
+          orow = asg;
+        }
+      }
+      const int64_t oidx = orow * a.N + t.nt * a.bn;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256;
       // a warp none of whose rows belong to the expert skips the tile
       if (__any_sync(0xffffffffu, row_ok)) {
         switch (mode) {
-          case OUT_BF16 * 3 + 1: epilogue_rows<OUT_BF16, 1>(a, tbase, oidx, sub, row_ok); break;
-          case OUT_BF16 * 3 + 2: epilogue_rows<OUT_BF16, 2>(a, tbase, oidx, sub, row_ok); break;
-          case OUT_F16 * 3 + 1: epilogue_rows<OUT_F16, 1>(a, tbase, oidx, sub, row_ok); break;
-          case OUT_F16 * 3 + 2: epilogue_rows<OUT_F16, 2>(a, tbase, oidx, sub, row_ok); break;
-          default: epilogue_rows<OUT_F32, 0>(a, tbase, oidx, sub, row_ok); break;
+          case OUT_BF16 * 3 + 1: epilogue_rows<OUT_BF16, 1>(a, tbase, oidx, sub, row_ok, scale); break;
+          case OUT_BF16 * 3 + 2: epilogue_rows<OUT_BF16, 2>(a, tbase, oidx, sub, row_ok, scale); break;
+          case OUT_F16 * 3 + 1: epilogue_rows<OUT_F16, 1>(a, tbase, oidx, sub, row_ok, scale); break;
+          case OUT_F16 * 3 + 2: epilogue_rows<OUT_F16, 2>(a, tbase, oidx, sub, row_ok, scale); break;
+          case OUT_COMBINE * 3 + 0: epilogue_rows<OUT_COMBINE, 0>(a, tbase, oidx, sub, row_ok, scale); break;
+          default: epilogue_rows<OUT_F32, 0>(a, tbase, oidx, sub, row_ok, scale); break;
         }
       }
       tc_fence_before();
@@ -369,7 +390,8 @@ static int pick_bn(int N) {
 
 static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void* B, int E, int N,
                               int ab_f16, void* out, int out_mode, const int32_t* offsets, int act,
-                              const LaunchCtx& c) {
+                              const LaunchCtx& c, const int32_t* perm_src = nullptr,
+                              const float* gate = nullptr) {
   const int bn = pick_bn(N);
   CUtensorMap tmA, tmB;
   if (!make_tmap_2b(&tmA, A, static_cast<uint64_t>(rows_cap), K, gg::BM, ab_f16)) return cudaErrorInvalidValue;
@@ -386,6 +408,8 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
   a.act = act;
   a.out_mode = out_mode;
   a.ab_f16 = ab_f16;
+  a.perm_src = perm_src;
+  a.gate = gate;
   a.err = c.err;
   // upper bound of the tile count: sum_e ceil(n_e / BM) <= rows_cap / BM + E
   const int64_t max_tiles = (rows_cap / gg::BM + E) * static_cast<int64_t>(a.n_tiles);
@@ -397,6 +421,33 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
   gg::grouped_gemm_tc_kernel<<<grid, gg::THREADS, gg::SMEM_BYTES, c.stream>>>(tmA, tmB, a);
   ++*c.launches;
   return cudaGetLastError();
+}
+
+// Rows of tokens whose only assignment was dropped (k = 1) get y = 0: the fused combine
+// writes only kept tokens.  One warp per token.
+__global__ void zero_dropped_kernel(const int32_t* __restrict__ slot_pos, int64_t T, float* __restrict__ y,
+                                    int d) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T || slot_pos[t] >= 0) return;
+  float4* row = reinterpret_cast<float4*>(y + t * d);
+  for (int v = threadIdx.x & 31; v < d / 4; v += 32) row[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+cudaError_t launch_ffn_combine_bf16(const FfnProblem& p, const int32_t* perm_src,
+                                    const int32_t* slot_pos, const float* gate, float* y,
+                                    const LaunchCtx& c) {
+  if (p.E > gg::MAX_GROUPS) return cudaErrorInvalidValue;
+  const int64_t T = p.rows_cap;  // k = 1: one assignment per token
+  zero_dropped_kernel<<<static_cast<unsigned>((T + 7) / 8), 256, 0, c.stream>>>(slot_pos, T, y, p.d);
+  ++*c.launches;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int hf = p.hidden_f16 ? 1 : 0;
+  e = launch_one(p.x_perm, p.rows_cap, p.d, p.w1, p.E, p.f, 0, p.h, hf ? gg::OUT_F16 : gg::OUT_BF16,
+                 p.offsets, p.act, c);
+  if (e != cudaSuccess) return e;
+  return launch_one(p.h, p.rows_cap, p.f, p.w2, p.E, p.d, hf, y, gg::OUT_COMBINE, p.offsets, 0, c,
+                    perm_src, gate);
 }
 
 cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c) {

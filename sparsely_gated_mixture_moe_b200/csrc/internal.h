@@ -75,6 +75,11 @@ struct FfnProblem {
 };
 cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c);
 cudaError_t launch_ffn_f32(const FfnProblem& p, const LaunchCtx& c);
+// k = 1, bf16: expert FFN whose down-projection writes y[t] = gate[t] * row directly (and
+// zeroes the rows of dropped tokens) instead of y_perm.
+cudaError_t launch_ffn_combine_bf16(const FfnProblem& p, const int32_t* perm_src,
+                                    const int32_t* slot_pos, const float* gate, float* y,
+                                    const LaunchCtx& c);
 
 // fp32 SIMT grouped product out[r, n] = act(sum_k A[r, k] B_g[n, k]) for the rows r of
 // each group g (offsets, or a single group of `rows` rows when offsets is null).

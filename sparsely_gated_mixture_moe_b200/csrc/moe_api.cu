@@ -214,6 +214,28 @@ moe_status do_combine(const moe_config* cfg, const void* y_perm, const int32_t* 
   return launch_combine(p, ctx.lc) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+moe_status do_ffn_combine(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
+                          const int32_t* perm_src, const int32_t* slot_pos, const float* gate,
+                          const void* w1, const void* w2, void* h, void* y, Ctx& ctx) {
+  FfnProblem p;
+  p.rows_cap = cfg->T;  // k = 1
+  p.d = cfg->d_model;
+  p.f = cfg->d_ff;
+  p.E = cfg->E;
+  p.act = cfg->act == MOE_ACT_GELU ? 2 : 1;
+  p.hidden_f16 = cfg->hidden_f16;
+  p.x_perm = x_perm;
+  p.offsets = offsets;
+  p.w1 = w1;
+  p.w2 = w2;
+  p.h = h;
+  p.y_perm = nullptr;
+  cudaError_t e = launch_ffn_combine_bf16(p, perm_src, slot_pos, gate, static_cast<float*>(y), ctx.lc);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+bool fused_combine(const moe_config* cfg) { return cfg->k == 1 && cfg->dtype == MOE_BF16; }
+
 // T == 0: nothing to route; zero the per-expert outputs that are defined anyway.
 moe_status empty_batch(const moe_config* cfg, int32_t* counts, int32_t* offsets, float* importance,
                        float* load, moe_stream_t stream) {
@@ -331,6 +353,29 @@ moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t*
   return st == MOE_OK ? ctx.finish(cudaSuccess) : st;
 }
 
+moe_status moe_expert_ffn_combine(const moe_config* cfg, const void* x_perm,
+                                  const int32_t* offsets, const int32_t* perm_src,
+                                  const int32_t* slot_pos, const float* topk_gate,
+                                  const void* w1, const void* w2, void* h, void* y, void* ws,
+                                  moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!fused_combine(cfg)) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T == 0) {
+    g_last_launches = 0;
+    return MOE_OK;
+  }
+  if (!x_perm || !offsets || !perm_src || !slot_pos || !topk_gate || !w1 || !w2 || !h || !y || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_perm) || !aligned16(w1) || !aligned16(w2) || !aligned16(h) || !aligned16(y) ||
+      !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  Ctx ctx(ws, stream);
+  if (!ctx.ok) return MOE_ERR_CUDA;
+  st = do_ffn_combine(cfg, x_perm, offsets, perm_src, slot_pos, topk_gate, w1, w2, h, y, ctx);
+  return st == MOE_OK ? ctx.finish(cudaSuccess) : st;
+}
+
 moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const void* w_noise,
                        const float* noise, const float* logit_bias, const void* w1, const void* w2,
                        void* y, int32_t* topk_idx, float* topk_gate, int32_t* counts,
@@ -359,6 +404,11 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_gate,
   if (st != MOE_OK) return st;
   st = do_permute(cfg, L, topk_idx, x, counts, offsets, perm_src, slot_pos, x_perm, ws, ctx);
   if (st != MOE_OK) return st;
+  if (fused_combine(cfg)) {
+    st = do_ffn_combine(cfg, x_perm, offsets, perm_src, slot_pos, topk_gate, w1, w2, h, y, ctx);
+    if (st != MOE_OK) return st;
+    return ctx.finish(cudaSuccess);
+  }
   st = do_ffn(cfg, x_perm, offsets, w1, w2, h, y_perm, ctx);
   if (st != MOE_OK) return st;
   st = do_combine(cfg, y_perm, slot_pos, topk_gate, y, ctx);

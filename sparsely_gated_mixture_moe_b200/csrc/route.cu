@@ -5,20 +5,27 @@
 //                   renorm: G = Softmax(KeepTopK(l, k)); else gate = softmax(l)[chosen]
 //   noisy gating:   H = l + n * Softplus(x.W_noise); choose the k largest H;
 //                   G = Softmax(KeepTopK(H, k))
-// Ties go to the lowest expert index (columns are scanned in ascending order and a new
-// value displaces a kept one only when strictly larger).  For noisy gating the kernel
-// also forms, per block of 128 tokens, the partial sums of Importance = sum_t G(x_t) and
+// Ties go to the lowest expert index (the running top list ranks equal scores by
+// expert index, so lists built over disjoint expert sets merge exactly).  For noisy
+// gating the kernel also forms, per block of 128 tokens, the partial sums of
+// Importance = sum_t G(x_t) and
 // Load_i = sum_t Phi((l_i - kth_excluding(H, k, i)) / Softplus((x.W_noise)_i))
 // ("Load-Balancing-Losses"); a second kernel adds the partials in a fixed order, so
 // results are bit-reproducible (no floating-point atomics).
 //
-// bf16: one CTA per 128 tokens.  Warp 0 streams x tiles [128 x 64] and W_g (and
-// W_noise) tiles [E_pad x 64] with TMA into a shared-memory ring; one thread of warp 1
-// issues tcgen05.mma (M=128, N=E_pad) into TMEM; then each of the 4 warps reads its 32
-// token rows back from TMEM (one token per thread, 32 experts per tcgen05.ld) and runs
-// the gate in registers.  The logits never touch HBM.
+// bf16: one CTA per 128 tokens, with G groups of 4 warps (G = 4, or 2 when k > 4).  Warp
+// 0 streams x tiles [128 x 64] and W_g (and W_noise) tiles [E_pad x 64] with TMA into a
+// shared-memory ring; one thread of warp 1 issues tcgen05.mma (M=128, N=E_pad) into
+// TMEM.  Then every thread owns one token row of its warp's TMEM lane quarter and a
+// disjoint set of expert columns (32-column slices, group g taking slices g, g+G, ...),
+// read 8 at a time with tcgen05.ld.  Pass 1 keeps a running top-(k+1) list and the
+// maximum in registers; a group of 8 scores whose maximum is below the current
+// (k+1)-th score skips the insertion (the common case once the list fills).  With the
+// Switch gate (softmax over all experts) a second sweep adds exp(score - max).  Group 0
+// merges the G partial lists and sums through shared memory and writes the outputs.
+// The logits never touch HBM.
 // fp32: the logits come from the SIMT product into the workspace and the same gate code
-// reads them back (one token per thread).
+// reads them back (one token per thread, G = 1).
 #include "common.cuh"
 #include "internal.h"
 
@@ -129,40 +136,56 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
   float* tr = fkth + 128 * 2;                                    // [4G warps][2][32][33]
   float* qsum = tr + 4 * G * 2 * 32 * 33;                        // [4][2][E]
 
-  // ---- pass 1: partial top-(k+1) and softmax statistics over this thread's experts
+  // ---- pass 1: partial top-(k+1) and maximum over this thread's experts
+  auto scores8 = [&](int c, float (&sc)[8]) {
+    float l[8], z[8], nz[8];
+    fetch(c, l, z);
+    if (noisy) load_noise8(c, nz);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = c + j;
+      float s = -INFINITY;
+      if (e < E) {
+        s = l[j] + (bias ? __ldg(bias + e) : 0.0f);
+        if (noisy) s += nz[j] * softplus_f(z[j]);
+      }
+      sc[j] = s;
+    }
+  };
   TopList<KM> top;
   top.init();
+  float thr = -INFINITY;  // the current (k+1)-th score: values below it cannot enter the list
   float m = -INFINITY, ssum = 0.0f;
   for (int c0 = grp * 32; c0 < E; c0 += 32 * G) {
 #pragma unroll 1
     for (int c = c0; c < c0 + 32 && c < E; c += 8) {
-      float l[8], z[8], sc[8], nz[8];
-      fetch(c, l, z);
-      if (noisy) load_noise8(c, nz);
+      float sc[8];
+      scores8(c, sc);
+      float gm = fmaxf(fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])),
+                       fmaxf(fmaxf(sc[4], sc[5]), fmaxf(sc[6], sc[7])));
+      m = fmaxf(m, gm);
+      if (gm >= thr) {  // rare after the first few groups
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int e = c + j;
-        float s = -INFINITY;
-        if (e < E) {
-          s = l[j] + (bias ? __ldg(bias + e) : 0.0f);
-          if (noisy) s += nz[j] * softplus_f(z[j]);
-        }
-        sc[j] = s;
+        for (int j = 0; j < 8; ++j)
+          if (c + j < E && sc[j] >= thr) top.insert(sc[j], c + j, k);
+        // slots past k stay at -inf, so the maximum over slots >= k is slot k
+        thr = -INFINITY;
+#pragma unroll
+        for (int q2 = 0; q2 <= KM; ++q2)
+          if (q2 >= k) thr = fmaxf(thr, top.v[q2]);
       }
-      if (full_softmax) {
-        float cm = -INFINITY;
+    }
+  }
+  if (full_softmax) {
+    // sum of exp(score - max) over this thread's experts, independent terms
+    for (int c0 = grp * 32; c0 < E; c0 += 32 * G) {
+#pragma unroll 1
+      for (int c = c0; c < c0 + 32 && c < E; c += 8) {
+        float sc[8];
+        scores8(c, sc);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) cm = fmaxf(cm, sc[j]);
-        const float nm = fmaxf(m, cm);
-        float cs = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) cs += (c + j < E) ? __expf(sc[j] - nm) : 0.0f;
-        ssum = (m == -INFINITY ? 0.0f : ssum * __expf(m - nm)) + cs;
-        m = nm;
+        for (int j = 0; j < 8; ++j) ssum += (c + j < E) ? __expf(sc[j] - m) : 0.0f;
       }
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (c + j < E) top.insert(sc[j], c + j, k);
     }
   }
 #pragma unroll

@@ -91,6 +91,12 @@ def run_steps(w, dev, cfg=None):
                     o["slot_pos"], o["x_perm"], ws)
     moe.moe_expert_ffn(cfg, o["x_perm"], o["offsets"], dev["w1"], dev["w2"], o["h"], o["y_perm"], ws)
     moe.moe_combine(cfg, o["y_perm"], o["slot_pos"], o["topk_gate"], o["y"], ws)
+    if moe.fused_combine(cfg):
+        # the fused FFN + combine step on the same permuted rows, into its own y
+        o["y_fused"] = torch.full((T, d), float("nan"), dtype=torch.float32, device=cu)
+        h2 = torch.zeros_like(o["h"])
+        moe.moe_expert_ffn_combine(cfg, o["x_perm"], o["offsets"], o["perm_src"], o["slot_pos"],
+                                   o["topk_gate"], dev["w1"], dev["w2"], h2, o["y_fused"], ws)
     err = moe.moe_get_error(ws)
     out = {kk: (v.cpu() if v is not None else None) for kk, v in o.items()}
     out["device_error"] = err
@@ -227,6 +233,10 @@ def check_combine(w, g, report, rows=None):
     # fp32 in, fp32 accumulation, fp32 out on both paths
     assert e <= TOL["f32"], e
     report["combine_err"] = e
+    if "y_fused" in g:
+        # one fp32 product g * row on both paths (k = 1): equal value for value
+        assert torch.equal(g["y_fused"], g["y"]), float((g["y_fused"] - g["y"]).abs().max())
+        report["fused_combine"] = "equal"
 
 
 def check_end_to_end(w, inp, g, idx, gates, report, rows=None):

@@ -106,6 +106,13 @@ def test_other_steps_validation():
     assert moe.lib.moe_expert_ffn(c, P, P, P, P, FAKE_ODD, P, P, None) == 1
     assert moe.lib.moe_combine(c, P, None, P, P, P, None) == 1
     assert moe.lib.moe_combine(c, P, P, P, FAKE_ODD, P, None) == 1
+    # the fused FFN + combine step: k = 1 and bf16 only, then the usual argument checks
+    c1 = ctypes.byref(_cfg(k=1))
+    assert moe.lib.moe_expert_ffn_combine(c, P, P, P, P, P, P, P, P, P, P, None) == 2
+    assert moe.lib.moe_expert_ffn_combine(ctypes.byref(_cfg(k=1, dtype="f32")), P, P, P, P, P, P,
+                                          P, P, P, P, None) == 2
+    assert moe.lib.moe_expert_ffn_combine(c1, P, P, None, P, P, P, P, P, P, P, None) == 1
+    assert moe.lib.moe_expert_ffn_combine(c1, P, P, P, P, P, P, P, P, FAKE_ODD, P, None) == 1
     assert moe.lib.moe_forward(c, P, P, None, None, None, P, P, None, P, P, P, None, None, None,
                                P, None) == 1
     assert moe.lib.moe_get_error(None, None, None) == 1
