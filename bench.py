@@ -420,7 +420,7 @@ def run_gpu(args, w):
                 "unit": "TFLOP/s", "frac": ffn_tflops / peaks["bf16_tflops_sustained"]}
     roof.update({"traffic": traffic,
                  "kernel": "grouped_gemm_tc_kernel (2 launches/step%s)" % (
-                     "; down-projection writes gate * row into y, plus a zero-fill of dropped "
+                     "; the down-projection writes gate * row into y and zeroes dropped "
                      "tokens' rows" if fused else ""),
                  "algorithmic_per_launch": {"flops": alg["ffn_flops"] / 2,
                                             "bytes": alg["ffn_bytes"] / 2},

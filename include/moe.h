@@ -198,8 +198,9 @@ moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t*
  * to moe_expert_ffn + moe_combine on the same inputs.
  *  x_perm, offsets, w1, w2, h as moe_expert_ffn;  perm_src, slot_pos as written by
  *  moe_permute;  topk_gate [T, 1] fp32 in;  y [T, d_model] fp32 out (every row written).
- * The rows of dropped tokens (slot_pos[t] < 0) are zeroed by a small kernel queued
- * before the two GEMMs; a perm_src entry outside [0, T) sets MOE_DEVERR_SLOT.  * Returns MOE_ERR_UNSUPPORTED when k != 1 or dtype is not bf16. */
+ * The rows of dropped tokens (slot_pos[t] < 0) are zeroed by the down-projection's
+ * epilogue threads before its first tile; a perm_src entry outside [0, T) sets
+ * MOE_DEVERR_SLOT.  * Returns MOE_ERR_UNSUPPORTED when k != 1 or dtype is not bf16. */
 moe_status moe_expert_ffn_combine(const moe_config* cfg, const void* x_perm,
                                   const int32_t* offsets, const int32_t* perm_src,
                                   const int32_t* slot_pos, const float* topk_gate,

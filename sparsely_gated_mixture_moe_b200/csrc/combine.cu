@@ -33,6 +33,8 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
   constexpr int V = Vec<T>::N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kCombineWarps + warp;
+  grid_dep_wait();
+  grid_dep_launch();
   if (t >= T_) return;
   const int64_t nrows = T_ * k;
   int slot[8];
@@ -96,11 +98,9 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
 cudaError_t launch_combine(const CombineProblem& p, const LaunchCtx& c) {
   const int64_t blocks = (p.T + kCombineWarps - 1) / kCombineWarps;
   if (blocks == 0) return cudaSuccess;
-  combine_kernel<float><<<static_cast<unsigned>(blocks), kCombineWarps * 32, 0, c.stream>>>(
-      static_cast<const float*>(p.y_perm), p.slot_pos, p.gate, static_cast<float*>(p.y), p.T,
-      p.k, p.d, c.err);
-  ++*c.launches;
-  return cudaGetLastError();
+  return launch_kernel(combine_kernel<float>, dim3(static_cast<unsigned>(blocks)),
+                       dim3(kCombineWarps * 32), 0, c, static_cast<const float*>(p.y_perm),
+                       p.slot_pos, p.gate, static_cast<float*>(p.y), p.T, p.k, p.d, c.err);
 }
 
 }  // namespace moe

@@ -21,6 +21,15 @@ constexpr int kErrTimeout = 8;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
 constexpr unsigned long long kDrainLimitNs = 100000000ull;  // 0.1 s for teardown drains
 
+// Programmatic dependent launch.  grid_dep_wait: block until the kernel that precedes this
+// one on the stream has completed and its memory operations are visible (returns at once
+// when the launch did not allow an early start).  grid_dep_launch: let the next kernel on
+// the stream be scheduled now; it still waits in its own grid_dep_wait.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void set_error(int* err, int bits) {
   if (err != nullptr) atomicOr(err, bits);
 }

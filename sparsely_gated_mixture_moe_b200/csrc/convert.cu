@@ -7,6 +7,8 @@ namespace moe {
 
 __global__ void bf16_to_f16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst,
                                    int64_t n, int32_t* n_inexact) {
+  grid_dep_wait();
+  grid_dep_launch();
   int inexact = 0;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -27,10 +29,9 @@ cudaError_t launch_bf16_to_f16(const void* src, void* dst, int64_t n, int32_t* n
   int64_t blocks = (n + 255) / 256;
   const int64_t cap = static_cast<int64_t>(c.num_sms) * 16;
   if (blocks > cap) blocks = cap;
-  bf16_to_f16_kernel<<<static_cast<unsigned>(blocks), 256, 0, c.stream>>>(
-      static_cast<const __nv_bfloat16*>(src), static_cast<__half*>(dst), n, n_inexact);
-  ++*c.launches;
-  return cudaGetLastError();
+  return launch_kernel(bf16_to_f16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, c,
+                       static_cast<const __nv_bfloat16*>(src), static_cast<__half*>(dst), n,
+                       n_inexact);
 }
 
 }  // namespace moe

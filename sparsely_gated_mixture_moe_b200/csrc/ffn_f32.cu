@@ -20,6 +20,8 @@ __global__ void __launch_bounds__(sg::THREADS)
   __shared__ int tp[sg::MAX_GROUPS + 1];
   __shared__ int scratch[40];
   const int tid = threadIdx.x;
+  grid_dep_wait();
+  grid_dep_launch();
 
   int g = 0;
   int64_t row0, row_end;
@@ -94,10 +96,8 @@ cudaError_t launch_sgemm_grouped(const float* A, const float* B, float* out,
   const int64_t mt = offsets ? rows_cap / sg::BM + groups : (rows_cap + sg::BM - 1) / sg::BM;
   if (mt <= 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>(mt), static_cast<unsigned>((N + sg::BN - 1) / sg::BN));
-  sgemm_grouped_kernel<<<grid, sg::THREADS, 0, c.stream>>>(A, B, out, offsets, groups, rows_cap,
-                                                           N, K, act, c.err);
-  ++*c.launches;
-  return cudaGetLastError();
+  return launch_kernel(sgemm_grouped_kernel, grid, dim3(sg::THREADS), 0, c, A, B, out, offsets,
+                       groups, rows_cap, N, K, act, c.err);
 }
 
 cudaError_t launch_ffn_f32(const FfnProblem& p, const LaunchCtx& c) {

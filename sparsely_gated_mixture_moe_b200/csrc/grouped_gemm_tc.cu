@@ -75,6 +75,7 @@ struct Args {
   int ab_f16;    // operand type of A and B: 1 fp16, 0 bf16
   const int32_t* perm_src;  // OUT_COMBINE: assignment of each permuted row (= token, k = 1)
   const float* gate;        // OUT_COMBINE: gate of each assignment
+  const int32_t* slot_pos;  // OUT_COMBINE: permuted row of each token, < 0 when dropped
   int* err;
 };
 
@@ -202,6 +203,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
     tmem_relinquish();
   }
+  grid_dep_wait();  // offsets and A come from the previous kernels on the stream
+  grid_dep_launch();
   const bool ok = block_tile_prefix(a.offsets, a.E, a.rows_cap, BM, tp, scratch);
   if (!ok && threadIdx.x == 0) set_error(a.err, kErrOffsets);
   tc_fence_before();
@@ -296,6 +299,23 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int q = warp & 3;               // TMEM lane quarter this warp may read
     const int sub = (warp - 2) >> 2;      // which 32-column chunks: sub*32 + 96*i
     const int mode = a.out_mode * 3 + a.act;
+    if (a.out_mode == OUT_COMBINE) {
+      // y = 0 for tokens whose only assignment was dropped (no tile writes them); done
+      // while the first tile's operands stream in
+      const int ew = warp - 2;
+      const int64_t stride = static_cast<int64_t>(gridDim.x) * EPI_WARPS * 32;
+      for (int64_t b = (static_cast<int64_t>(blockIdx.x) * EPI_WARPS + ew) * 32; b < a.rows_cap;
+           b += stride) {
+        const bool drop = b + lane < a.rows_cap && __ldg(a.slot_pos + b + lane) < 0;
+        uint32_t m = __ballot_sync(0xffffffffu, drop);
+        while (m) {
+          const int j = __ffs(m) - 1;
+          m &= m - 1;
+          float4* row = reinterpret_cast<float4*>(static_cast<float*>(a.out) + (b + j) * a.N);
+          for (int v = lane; v < a.N / 4; v += 32) row[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+    }
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x) {
@@ -391,7 +411,7 @@ static int pick_bn(int N) {
 static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void* B, int E, int N,
                               int ab_f16, void* out, int out_mode, const int32_t* offsets, int act,
                               const LaunchCtx& c, const int32_t* perm_src = nullptr,
-                              const float* gate = nullptr) {
+                              const float* gate = nullptr, const int32_t* slot_pos = nullptr) {
   const int bn = pick_bn(N);
   CUtensorMap tmA, tmB;
   if (!make_tmap_2b(&tmA, A, static_cast<uint64_t>(rows_cap), K, gg::BM, ab_f16)) return cudaErrorInvalidValue;
@@ -410,6 +430,7 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
   a.ab_f16 = ab_f16;
   a.perm_src = perm_src;
   a.gate = gate;
+  a.slot_pos = slot_pos;
   a.err = c.err;
   // upper bound of the tile count: sum_e ceil(n_e / BM) <= rows_cap / BM + E
   const int64_t max_tiles = (rows_cap / gg::BM + E) * static_cast<int64_t>(a.n_tiles);
@@ -418,36 +439,20 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
   cudaError_t e = cudaFuncSetAttribute(gg::grouped_gemm_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, gg::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  gg::grouped_gemm_tc_kernel<<<grid, gg::THREADS, gg::SMEM_BYTES, c.stream>>>(tmA, tmB, a);
-  ++*c.launches;
-  return cudaGetLastError();
-}
-
-// Rows of tokens whose only assignment was dropped (k = 1) get y = 0: the fused combine
-// writes only kept tokens.  One warp per token.
-__global__ void zero_dropped_kernel(const int32_t* __restrict__ slot_pos, int64_t T, float* __restrict__ y,
-                                    int d) {
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T || slot_pos[t] >= 0) return;
-  float4* row = reinterpret_cast<float4*>(y + t * d);
-  for (int v = threadIdx.x & 31; v < d / 4; v += 32) row[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+  return launch_kernel(gg::grouped_gemm_tc_kernel, dim3(grid), dim3(gg::THREADS), gg::SMEM_BYTES, c,
+                       tmA, tmB, a);
 }
 
 cudaError_t launch_ffn_combine_bf16(const FfnProblem& p, const int32_t* perm_src,
                                     const int32_t* slot_pos, const float* gate, float* y,
                                     const LaunchCtx& c) {
   if (p.E > gg::MAX_GROUPS) return cudaErrorInvalidValue;
-  const int64_t T = p.rows_cap;  // k = 1: one assignment per token
-  zero_dropped_kernel<<<static_cast<unsigned>((T + 7) / 8), 256, 0, c.stream>>>(slot_pos, T, y, p.d);
-  ++*c.launches;
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   const int hf = p.hidden_f16 ? 1 : 0;
-  e = launch_one(p.x_perm, p.rows_cap, p.d, p.w1, p.E, p.f, 0, p.h, hf ? gg::OUT_F16 : gg::OUT_BF16,
+  cudaError_t e = launch_one(p.x_perm, p.rows_cap, p.d, p.w1, p.E, p.f, 0, p.h, hf ? gg::OUT_F16 : gg::OUT_BF16,
                  p.offsets, p.act, c);
   if (e != cudaSuccess) return e;
   return launch_one(p.h, p.rows_cap, p.f, p.w2, p.E, p.d, hf, y, gg::OUT_COMBINE, p.offsets, 0, c,
-                    perm_src, gate);
+                    perm_src, gate, slot_pos);
 }
 
 cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c) {

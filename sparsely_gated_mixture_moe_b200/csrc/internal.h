@@ -19,6 +19,29 @@ struct LaunchCtx {
   int* launches;  // host counter
 };
 
+// Every kernel of the library is launched with programmatic stream serialisation: the
+// launch may start while the previous kernel on the stream is still running, and the
+// kernel's grid_dep_wait() (at its top, before any global-memory access) blocks until
+// that kernel has completed and its writes are visible.  Only the prologue (barrier
+// init, TMEM allocation, descriptor prefetch) overlaps the previous kernel's tail.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          const LaunchCtx& c, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = c.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  ++*c.launches;
+  return e;
+}
+
 // ---- route -----------------------------------------------------------------------
 struct RouteProblem {
   int64_t T;
@@ -57,6 +80,8 @@ struct PermuteProblem {
   void* x_perm;
   int32_t* blk;     // workspace [nblk][E]
   int32_t* ticket;  // workspace counter, zero between calls
+  int32_t* sync;    // two workspace counters, zero between calls, for the one-launch
+                    // path (null: always use the three-kernel path)
 };
 int64_t permute_blocks(int64_t n);
 cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c);
@@ -75,8 +100,8 @@ struct FfnProblem {
 };
 cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c);
 cudaError_t launch_ffn_f32(const FfnProblem& p, const LaunchCtx& c);
-// k = 1, bf16: expert FFN whose down-projection writes y[t] = gate[t] * row directly (and
-// zeroes the rows of dropped tokens) instead of y_perm.
+// k = 1, bf16: expert FFN whose down-projection writes y[t] = gate[t] * row directly (its
+// epilogue also zeroes the rows of dropped tokens) instead of y_perm.
 cudaError_t launch_ffn_combine_bf16(const FfnProblem& p, const int32_t* perm_src,
                                     const int32_t* slot_pos, const float* gate, float* y,
                                     const LaunchCtx& c);

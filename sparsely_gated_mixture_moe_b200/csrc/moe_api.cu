@@ -179,6 +179,7 @@ moe_status do_permute(const moe_config* cfg, const Layout& L, const int32_t* top
   p.x_perm = x_perm;
   p.blk = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + L.blk);
   p.ticket = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + L.err + 8);
+  p.sync = p.ticket;  // words 2 and 3 of the error block, zero between calls
   return launch_permute(p, ctx.lc) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

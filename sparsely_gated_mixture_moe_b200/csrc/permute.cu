@@ -6,7 +6,8 @@
 // only the first C assignments of an expert are kept (capacity factor, "moe paper models"
 // Table 2), the rest are dropped (slot_pos = -1).
 //
-// Three kernels, no cross-block waits:
+// One launch when every block of its grid can be resident at once (perm_fused_kernel,
+// below), else three kernels with no cross-block waits:
 //   count+scan  block b counts its chunk of 256 assignments per expert (shared-memory
 //               histogram) into blk[b][e]; the last block to finish (a ticket counter)
 //               turns blk into per-chunk rank bases with a segmented scan over the chunks,
@@ -48,6 +49,8 @@ __global__ void __launch_bounds__(pm::THREADS)
   const int tid = threadIdx.x;
   const int nblk = gridDim.x;
   for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
+  grid_dep_wait();
+  grid_dep_launch();
   __syncthreads();
   const int64_t a = static_cast<int64_t>(blockIdx.x) * kPermChunk + tid;
   if (a < n) {
@@ -126,6 +129,8 @@ __global__ void __launch_bounds__(pm::THREADS)
   const int64_t a = static_cast<int64_t>(blockIdx.x) * kPermChunk + threadIdx.x;
 
   for (int i = threadIdx.x; i < pm::WARPS * E; i += blockDim.x) wbase[i] = 0;
+  grid_dep_wait();
+  grid_dep_launch();
   __syncthreads();
   int e = (a < n) ? idx[a] : -1;
   if (e < 0 || e >= E) e = -1;
@@ -161,6 +166,8 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
                        int E, int k, const uint8_t* __restrict__ x, uint8_t* __restrict__ x_perm,
                        int row_bytes) {
   const int lane = threadIdx.x & 31;
+  grid_dep_wait();
+  grid_dep_launch();
   const int n_kept = __ldg(offsets + E);
   const int nv = row_bytes >> 4;
   const int warps = gridDim.x * kGatherWarps;
@@ -181,20 +188,268 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
   }
 }
 
+// ------------------------------------------------------------------ one-launch path
+//
+// The same counting sort in one launch.  Blocks of 1024 threads; block c < nchunks owns
+// assignments [1024c, 1024c + 1024).
+//   phase 1  each owner block ranks its chunk stably (warp match + per-warp prefix, kept
+//            in registers and shared memory) and writes its per-expert counts to
+//            blk[e][c]
+//   barrier
+//   phase 2  each owner block sums column e of blk below its chunk (its rank base) and
+//            over all chunks (the expert's count), scans min(count, C) over the experts
+//            into offsets (block 0 writes counts and offsets), and writes slot_pos and
+//            perm_src for its chunk.  Every owner block redoes these small sums itself,
+//            so no second scan pass or flag is needed
+//   barrier
+//   phase 3  all blocks copy the kept rows x[perm_src[s] / k] -> x_perm[s]
+// The grid never exceeds what the occupancy query says fits on the GPU at once, so every
+// block reaches each barrier; the waits are bounded all the same (1 s, then the timeout
+// bit and an early exit).  The barrier counter and an exit counter live in the workspace
+// and are reset by the last block to leave.
+namespace pf {
+constexpr int THREADS = 1024;
+constexpr int WARPS = THREADS / 32;
+constexpr int CHUNK = THREADS;
+}  // namespace pf
+
+static size_t fused_smem(int E) {
+  return (static_cast<size_t>(pf::WARPS) * E + 3 * static_cast<size_t>(E) + 2 * pf::THREADS + 64) * 4;
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Barrier over all blocks of the grid (all resident).  Arrivals accumulate in *ctr over
+// the launch; a barrier is complete once *ctr reaches `target`.  Gives up after the wait
+// limit: sets the timeout bit and *s_abort.  Every thread must call it.
+__device__ bool grid_barrier(int* ctr, int target, int* err, volatile int* s_abort) {
+  __syncthreads();
+  if (threadIdx.x == 0 && *s_abort == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1);
+    const unsigned long long t0 = globaltimer_ns();
+    while (ld_acquire_gpu(ctr) < target) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        set_error(err, kErrTimeout);
+        *s_abort = 1;
+        break;
+      }
+      __nanosleep(100);
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  return *s_abort == 0;
+}
+
+__global__ void __launch_bounds__(pf::THREADS, 1)
+    perm_fused_kernel(const int32_t* __restrict__ idx, int64_t n, int E, int64_t C, int k,
+                      int nchunks, int32_t* blk, int32_t* __restrict__ counts, int32_t* offsets,
+                      int32_t* perm_src, int32_t* __restrict__ slot_pos,
+                      const uint8_t* __restrict__ x, uint8_t* __restrict__ x_perm, int row_bytes,
+                      int32_t* sync, int* err) {
+  extern __shared__ int fsm[];
+  int* wbase = fsm;                     // [WARPS][E]: per-warp rank bases
+  int* s_pre = wbase + pf::WARPS * E;   // [E]: rank base of this chunk
+  int* s_tot = s_pre + E;               // [E]: assignments per expert
+  int* s_off = s_tot + E;               // [E]: offsets
+  int* segp = s_off + E;                // [THREADS]
+  int* segt = segp + pf::THREADS;       // [THREADS]
+  int* scratch = segt + pf::THREADS;    // [64]
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  if (tid == 0) s_abort = 0;
+  for (int i = tid; i < pf::WARPS * E; i += pf::THREADS) wbase[i] = 0;
+  grid_dep_wait();
+  grid_dep_launch();
+  __syncthreads();
+
+  // ---- phase 1: stable ranks within the chunk, chunk counts to blk[e][c]
+  const int c = blockIdx.x;
+  const bool owner = c < nchunks;  // uniform across the block
+  const int64_t a = static_cast<int64_t>(c) * pf::CHUNK + tid;
+  int e = -1;
+  uint32_t peers = 0;
+  if (owner) {
+    if (a < n) {
+      e = idx[a];
+      if (e < 0 || e >= E) {
+        set_error(err, kErrExpertIndex);
+        e = -1;
+      }
+    }
+    peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && (peers & lt_mask) == 0) wbase[warp * E + e] = __popc(peers);
+  }
+  __syncthreads();
+  if (owner) {
+    for (int xe = tid; xe < E; xe += pf::THREADS) {
+      int run = 0;
+      for (int w = 0; w < pf::WARPS; ++w) {
+        const int v = wbase[w * E + xe];
+        wbase[w * E + xe] = run;
+        run += v;
+      }
+      blk[static_cast<int64_t>(xe) * nchunks + c] = run;
+    }
+  }
+  const int G = static_cast<int>(gridDim.x);
+  bool ok = grid_barrier(sync, G, err, &s_abort);
+
+  // ---- phase 2: rank bases, counts, offsets; slot_pos and perm_src of this chunk
+  if (ok && owner) {
+    int tpe = 1;  // threads per expert, each summing a run of chunks
+    while (tpe * 2 * E <= pf::THREADS) tpe *= 2;
+    const int epr = pf::THREADS / tpe;  // experts per round
+    const int len = (nchunks + tpe - 1) / tpe;
+    for (int e0 = 0; e0 < E; e0 += epr) {
+      const int el = tid % epr, part = tid / epr, xe = e0 + el;
+      int pre = 0, tot = 0;
+      if (xe < E) {
+        const int b0 = part * len, b1 = min(nchunks, b0 + len);
+        const int32_t* col = blk + static_cast<int64_t>(xe) * nchunks;
+        for (int b = b0; b < b1; ++b) {
+          const int v = __ldcg(col + b);
+          tot += v;
+          pre += (b < c) ? v : 0;
+        }
+      }
+      segp[tid] = pre;
+      segt[tid] = tot;
+      __syncthreads();
+      if (part == 0 && xe < E) {
+        int P = 0, S = 0;
+        for (int q = 0; q < tpe; ++q) {
+          P += segp[q * epr + el];
+          S += segt[q * epr + el];
+        }
+        s_pre[xe] = P;
+        s_tot[xe] = S;
+      }
+      __syncthreads();
+    }
+    int carry = 0;
+    for (int base = 0; base < E; base += pf::THREADS) {
+      const int xe = base + tid;
+      const int tot = xe < E ? s_tot[xe] : 0;
+      const int kv = (C >= 0 && tot > C) ? static_cast<int>(C) : tot;
+      int sum;
+      const int incl = block_incl_scan(kv, scratch, &sum);
+      if (xe < E) {
+        s_off[xe] = carry + incl - kv;
+        if (c == 0) {
+          counts[xe] = tot;
+          offsets[xe] = carry + incl - kv;
+        }
+      }
+      carry += sum;
+    }
+    if (c == 0 && tid == 0) offsets[E] = carry;
+    __syncthreads();
+    if (a < n) {
+      int slot = -1;
+      if (e >= 0) {
+        const int rank = s_pre[e] + wbase[warp * E + e] + __popc(peers & lt_mask);
+        if (C < 0 || rank < C) slot = s_off[e] + rank;
+      }
+      slot_pos[a] = slot;
+      if (slot >= 0) perm_src[slot] = static_cast<int32_t>(a);
+    }
+  }
+  ok = ok && grid_barrier(sync, 2 * G, err, &s_abort);
+
+  // ---- phase 3: x_perm[s] = x[perm_src[s] / k], two rows per warp in flight
+  if (ok) {
+    const int n_kept = __ldcg(offsets + E);
+    const int nv = row_bytes >> 4;
+    const int stride = G * pf::WARPS;
+    for (int s = blockIdx.x * pf::WARPS + warp; s < n_kept; s += 2 * stride) {
+      const int s2 = s + stride;
+      const bool two = s2 < n_kept;
+      const int64_t t1 = __ldcg(perm_src + s) / k;
+      const int64_t t2 = two ? __ldcg(perm_src + s2) / k : t1;
+      const uint4* src1 = reinterpret_cast<const uint4*>(x + t1 * row_bytes);
+      const uint4* src2 = reinterpret_cast<const uint4*>(x + t2 * row_bytes);
+      uint4* dst1 = reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(s) * row_bytes);
+      uint4* dst2 = reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(two ? s2 : s) * row_bytes);
+      int v = lane;
+      for (; v + 32 < nv; v += 64) {
+        const uint4 a0 = __ldg(src1 + v), a1 = __ldg(src1 + v + 32);
+        const uint4 b0 = __ldg(src2 + v), b1 = __ldg(src2 + v + 32);
+        dst1[v] = a0;
+        dst1[v + 32] = a1;
+        if (two) {
+          dst2[v] = b0;
+          dst2[v + 32] = b1;
+        }
+      }
+      for (; v < nv; v += 32) {
+        const uint4 a0 = __ldg(src1 + v), b0 = __ldg(src2 + v);
+        dst1[v] = a0;
+        if (two) dst2[v] = b0;
+      }
+    }
+  }
+
+  // ---- the last block to leave resets both counters for the next call
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(sync + 1, 1) == G - 1) {
+      atomicExch(sync, 0);
+      atomicExch(sync + 1, 0);
+    }
+  }
+}
+
+// Grid for the one-launch path, or 0 when its blocks would not all fit at once.
+static int fused_grid(const PermuteProblem& p, const LaunchCtx& c, size_t smem) {
+  if (p.sync == nullptr) return 0;
+  const int64_t nchunks = (p.n + pf::CHUNK - 1) / pf::CHUNK;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(perm_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return 0;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, perm_fused_kernel, pf::THREADS,
+                                                    smem) != cudaSuccess)
+    return 0;
+  const int64_t cap = static_cast<int64_t>(per_sm) * c.num_sms;
+  if (nchunks > cap) return 0;
+  // enough warps to keep about four rows each in the gather, at least one block per chunk
+  int64_t g = (p.n + 4 * pf::WARPS - 1) / (4 * pf::WARPS);
+  if (g > cap) g = cap;
+  if (g < nchunks) g = nchunks;
+  return static_cast<int>(g);
+}
+
 cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c) {
   const int64_t nblk = permute_blocks(p.n);
   if (nblk == 0) return cudaSuccess;
   cudaError_t e = cudaSuccess;
+  const size_t f_smem = fused_smem(p.E);
+  const int fg = fused_grid(p, c, f_smem);
+  if (fg > 0) {
+    const int nchunks = static_cast<int>((p.n + pf::CHUNK - 1) / pf::CHUNK);
+    return launch_kernel(perm_fused_kernel, dim3(fg), dim3(pf::THREADS), f_smem, c, p.topk_idx,
+                         p.n, p.E, p.C, p.k, nchunks, p.blk, p.counts, p.offsets, p.perm_src,
+                         p.slot_pos, static_cast<const uint8_t*>(p.x),
+                         static_cast<uint8_t*>(p.x_perm), p.d * p.esize, p.sync, c.err);
+  }
   const size_t cs_smem = count_scan_smem(p.E);
   if (cs_smem > 48 * 1024) {
     e = cudaFuncSetAttribute(perm_count_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(cs_smem));
     if (e != cudaSuccess) return e;
   }
-  perm_count_scan_kernel<<<static_cast<unsigned>(nblk), pm::THREADS, cs_smem, c.stream>>>(
-      p.topk_idx, p.n, p.E, p.C, p.blk, p.counts, p.offsets, p.ticket, c.err);
-  ++*c.launches;
-  e = cudaGetLastError();
+  e = launch_kernel(perm_count_scan_kernel, dim3(static_cast<unsigned>(nblk)), dim3(pm::THREADS),
+                    cs_smem, c, p.topk_idx, p.n, p.E, p.C, p.blk, p.counts, p.offsets, p.ticket,
+                    c.err);
   if (e != cudaSuccess) return e;
   const size_t wsmem = static_cast<size_t>(pm::WARPS) * p.E * 4;
   if (wsmem > 48 * 1024) {
@@ -202,20 +457,19 @@ cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c) {
                              static_cast<int>(wsmem));
     if (e != cudaSuccess) return e;
   }
-  perm_scatter_kernel<<<static_cast<unsigned>(nblk), pm::THREADS, wsmem, c.stream>>>(
-      p.topk_idx, p.n, p.E, p.C, p.blk, p.offsets, p.perm_src, p.slot_pos);
-  ++*c.launches;
-  e = cudaGetLastError();
+  e = launch_kernel(perm_scatter_kernel, dim3(static_cast<unsigned>(nblk)), dim3(pm::THREADS),
+                    wsmem, c, p.topk_idx, p.n, p.E, p.C, static_cast<const int32_t*>(p.blk),
+                    static_cast<const int32_t*>(p.offsets), p.perm_src, p.slot_pos);
   if (e != cudaSuccess) return e;
   // enough warps for every row when the grid allows, capped at 16 blocks per SM
   int64_t gblocks = (p.n + kGatherWarps - 1) / kGatherWarps;
   const int64_t cap = static_cast<int64_t>(c.num_sms) * 16;
   if (gblocks > cap) gblocks = cap;
-  perm_gather_kernel<<<static_cast<unsigned>(gblocks), kGatherWarps * 32, 0, c.stream>>>(
-      p.perm_src, p.offsets, p.E, p.k, static_cast<const uint8_t*>(p.x),
-      static_cast<uint8_t*>(p.x_perm), p.d * p.esize);
-  ++*c.launches;
-  return cudaGetLastError();
+  return launch_kernel(perm_gather_kernel, dim3(static_cast<unsigned>(gblocks)),
+                       dim3(kGatherWarps * 32), 0, c, static_cast<const int32_t*>(p.perm_src),
+                       static_cast<const int32_t*>(p.offsets), p.E, p.k,
+                       static_cast<const uint8_t*>(p.x), static_cast<uint8_t*>(p.x_perm),
+                       p.d * p.esize);
 }
 
 }  // namespace moe
@@ -306,6 +560,7 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
   // the per-chunk counts are fully rewritten by the count kernel each call
   p.ticket = static_cast<int32_t*>(scratch);
   p.blk = static_cast<int32_t*>(scratch) + 64;
+  p.sync = nullptr;  // always the three-kernel path here
   if (cudaMemsetAsync(p.ticket, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
   if (launch_permute(p, c) != cudaSuccess) return MOE_ERR_CUDA;
   set_last_launch_count(launches);

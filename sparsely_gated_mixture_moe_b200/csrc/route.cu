@@ -31,7 +31,6 @@
 
 namespace moe {
 
-constexpr int kMaxK = 8;
 constexpr int kRouteBM = 128;
 
 int route_blocks(int64_t T) { return static_cast<int>((T + kRouteBM - 1) / kRouteBM); }
@@ -47,8 +46,17 @@ struct GateArgs {
   float* partials;  // [gridDim.x][2][E] or null
 };
 
+// Softplus(z) = max(z, 0) + log(1 + e^-|z|), with the fast exponential and logarithm:
+// for u = e^-|z| < 1/64 log(1 + u) is its Taylor polynomial to u^4 (truncation below
+// 1/64^5 / 5 relative), else __logf(1 + u), whose absolute error on [1, 2] is below
+// 2^-21.  The result is within about 5e-7 of the exact value, far inside the margin at
+// which the top-k choice counts as a near tie (1e-4).
 __device__ __forceinline__ float softplus_f(float z) {
-  return fmaxf(z, 0.0f) + log1pf(expf(-fabsf(z)));
+  const float u = __expf(-fabsf(z));
+  const float l1p = (u < 0.015625f)
+                        ? u * (1.0f - u * (0.5f - u * (0.33333333f - u * 0.25f)))
+                        : __logf(1.0f + u);
+  return fmaxf(z, 0.0f) + l1p;
 }
 
 // Descending list of the KM+1 largest (score, expert) pairs seen; a pair ranks higher
@@ -257,6 +265,13 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
 
   // ---- pass 2: Importance and Load partial sums over this tile's tokens
   const float kth = fkth[row * 2 + 0], kth1 = fkth[row * 2 + 1];
+  int myid[KM];  // this token's chosen experts (-1 past k) and their gates
+  float myg[KM];
+#pragma unroll
+  for (int jj = 0; jj < KM; ++jj) {
+    myid[jj] = fid[row * KM + jj];
+    myg[jj] = fgate[row * KM + jj];
+  }
   float* mytr = tr + warp * (2 * 32 * 33);
   for (int c0 = grp * 32; c0 < E; c0 += 32 * G) {
 #pragma unroll 1
@@ -283,9 +298,9 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
               const float ex = (H >= kth) ? kth1 : kth;  // kth_excluding(H, k, e)
               pl[j] = 0.5f * erfcf(-((li - ex) / sp) * 0.70710678118654752f);
             }
-#pragma unroll 1
-            for (int jj = 0; jj < k; ++jj)
-              if (fid[row * KM + jj] == e) gi[j] = fgate[row * KM + jj];
+#pragma unroll
+            for (int jj = 0; jj < KM; ++jj)
+              if (myid[jj] == e) gi[j] = myg[jj];
           }
         }
       }
@@ -380,6 +395,8 @@ __global__ void __launch_bounds__(128 * G, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int t0 = blockIdx.x * kRouteBM;
+  grid_dep_wait();  // x and the outputs' previous readers belong to earlier kernels
+  grid_dep_launch();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -493,6 +510,8 @@ template <int KM>
 __global__ void __launch_bounds__(128, 1)
     gate_f32_kernel(const float* __restrict__ logits, const float* __restrict__ nz, GateArgs g) {
   extern __shared__ __align__(16) uint8_t gsmem[];
+  grid_dep_wait();
+  grid_dep_launch();
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRouteBM;
   const int64_t t = t0 + threadIdx.x;
   const bool valid = t < g.T;
@@ -511,6 +530,8 @@ __global__ void __launch_bounds__(128, 1)
 __global__ void finalize_importance_load_kernel(const float* __restrict__ partials, int nblocks,
                                                 int E, float* importance, float* load) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  grid_dep_wait();
+  grid_dep_launch();
   if (e >= E) return;
   float si = 0.0f, sl = 0.0f;
   for (int b = 0; b < nblocks; ++b) {
@@ -543,10 +564,8 @@ static int k_bucket(int k) { return k <= 1 ? 1 : k <= 2 ? 2 : k <= 4 ? 4 : 8; }
 
 static cudaError_t launch_finalize(const RouteProblem& p, int nblocks, const LaunchCtx& c) {
   if (!(p.importance || p.load)) return cudaSuccess;
-  finalize_importance_load_kernel<<<(p.E + 127) / 128, 128, 0, c.stream>>>(
-      p.partials, nblocks, p.E, p.importance, p.load);
-  ++*c.launches;
-  return cudaGetLastError();
+  return launch_kernel(finalize_importance_load_kernel, dim3((p.E + 127) / 128), dim3(128), 0, c,
+                       static_cast<const float*>(p.partials), nblocks, p.E, p.importance, p.load);
 }
 
 template <int KM>
@@ -555,9 +574,8 @@ static cudaError_t launch_route_tc(const CUtensorMap& tmX, const CUtensorMap& tm
                                    int nblocks, const LaunchCtx& c) {
   cudaError_t e = cudaFuncSetAttribute(route_tc_kernel<KM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  route_tc_kernel<KM><<<nblocks, 128 * rt::groups_for(KM), smem, c.stream>>>(tmX, tmG, tmN, a);
-  ++*c.launches;
-  return cudaGetLastError();
+  return launch_kernel(route_tc_kernel<KM>, dim3(nblocks), dim3(128 * rt::groups_for(KM)), smem, c,
+                       tmX, tmG, tmN, a);
 }
 
 cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
@@ -610,9 +628,9 @@ static cudaError_t launch_gate_f32(const RouteProblem& p, const GateArgs& g, int
     cudaError_t e = cudaFuncSetAttribute(gate_f32_kernel<KM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
   }
-  gate_f32_kernel<KM><<<nblocks, 128, smem, c.stream>>>(p.logits_ws, p.noisy ? p.nz_ws : nullptr, g);
-  ++*c.launches;
-  return cudaGetLastError();
+  return launch_kernel(gate_f32_kernel<KM>, dim3(nblocks), dim3(128), smem, c,
+                       static_cast<const float*>(p.logits_ws),
+                       static_cast<const float*>(p.noisy ? p.nz_ws : nullptr), g);
 }
 
 cudaError_t launch_route_f32(const RouteProblem& p, const LaunchCtx& c) {

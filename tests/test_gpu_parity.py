@@ -129,16 +129,20 @@ def test_bad_offsets_set_error():
     assert moe.moe_get_error(ws) & 2
 
 
-FULL = ["switch", "noisy", "gshard", "zipf"]
+FULL = {name: W[name] for name in ("switch", "noisy", "gshard", "zipf")}
+# More assignments (200,000) than one permutation launch can keep resident on a B200
+# (1024 per block, one block per SM): moe_permute takes its three-kernel path here.
+FULL["three_kernel_permute_T200k"] = Workload("t200k", T=200_000, d_model=64, d_ff=128, E=8, k=1,
+                                              renorm=False, capacity_factor=1.0, act="relu")
 
 
-@pytest.mark.parametrize("name", FULL)
+@pytest.mark.parametrize("name", list(FULL))
 def test_full_size_sampled(name):
     """The benchmark's workloads at full size, in the launch configuration the benchmark
     times.  Choices, gates, importance/load and the whole permutation are checked on
     every token; expert outputs and layer outputs on a sample of rows (including each
     expert's first and last kept row)."""
-    w = W[name]
+    w = FULL[name]
     inp = workloads.make_inputs(w)
     dev = H.to_device(inp)
     g = H.run_steps(w, dev)
@@ -197,3 +201,25 @@ def test_fast_erf_matches_cuda_erff():
     d = (fast - ref).abs()
     assert float(d.max()) <= 1e-6, float(d.max())
     assert fast[-4].item() == 1.0 and fast[-3].item() == -1.0
+
+
+@pytest.mark.parametrize("name,launches", [("switch", 1), ("three_kernel_permute_T200k", 3)])
+def test_permute_launch_path(name, launches):
+    """moe_permute runs as one launch (grid barriers between its phases) when every block
+    of that grid fits on the GPU at once, and as three kernels otherwise."""
+    import sparsely_gated_mixture_moe_b200 as moe
+    w = FULL[name]
+    cfg = H.config_of(w)
+    dev = H.to_device(workloads.make_inputs(w))
+    n = w.T * w.k
+    gen = torch.Generator().manual_seed(7)
+    idx = torch.randint(0, w.E, (w.T, w.k), generator=gen, dtype=torch.int32).cuda()
+    o = {key: torch.empty(size, dtype=torch.int32, device="cuda")
+         for key, size in (("counts", w.E), ("offsets", w.E + 1), ("perm_src", n), ("slot_pos", n))}
+    x_perm = torch.empty(n, w.d_model, dtype=w.torch_dtype, device="cuda")
+    ws = moe.workspace(cfg)
+    moe.moe_permute(cfg, idx, dev["x"], o["counts"], o["offsets"], o["perm_src"], o["slot_pos"],
+                    x_perm, ws)
+    assert moe.last_launch_count() == launches
+    assert moe.moe_get_error(ws) == 0
+    assert o["counts"].tolist() == torch.bincount(idx.view(-1).long(), minlength=w.E).tolist()
