@@ -89,30 +89,61 @@ struct TopList {
   }
 };
 
-// Shared-memory bytes gate_tile needs for a block of 128*G threads.
+// Shared-memory bytes gate_tile needs for 128*G gate threads.
 __host__ __device__ constexpr int gate_smem_bytes(int KM, int G, int E) {
   return G * 128 * (KM + 1) * 8     // partial lists (scores, experts)
          + G * 128 * 8              // partial softmax (max, sum)
          + 128 * (2 * KM + 2) * 4   // final experts, gates, k-th and (k+1)-th score
-         + 4 * G * 2 * 32 * 33 * 4  // per-warp transposes (two quantities) for the reductions
-         + 4 * 2 * E * 4            // per-lane-quarter column sums
+         + 4 * 2 * E * 4            // per-lane-quarter column sums (Importance, Load)
          + 64;
 }
 
-// The gate for one tile of 128 tokens, computed by 128*G threads: thread (warp w, lane l)
-// owns token row r = 32*(w%4) + l and the expert columns c = 32*(w/4) + 32*G*i + j.
+// Sum of v[j] over the 32 lanes of a warp for each of the 8 columns j, as a
+// reduce-scatter: each step halves the columns a lane keeps and adds its partner's
+// half; afterwards lane l holds the sum of column 4*(l&1) + 2*((l>>1)&1) + ((l>>2)&1)
+// (lanes 0..7 hold all eight).  The order of additions is fixed, so the sums are
+// reproducible.
+__device__ __forceinline__ float warp_colsum8(const float (&v)[8], int lane) {
+  const bool b0 = lane & 1, b1 = lane & 2, b2 = lane & 4;
+  float w4[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float send = b0 ? v[j] : v[j + 4];
+    const float keep = b0 ? v[j + 4] : v[j];
+    w4[j] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+  }
+  float w2[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const float send = b1 ? w4[j] : w4[j + 2];
+    const float keep = b1 ? w4[j + 2] : w4[j];
+    w2[j] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  float w1 = (b2 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? w2[0] : w2[1], 4);
+  w1 += __shfl_xor_sync(0xffffffffu, w1, 8);
+  w1 += __shfl_xor_sync(0xffffffffu, w1, 16);
+  return w1;
+}
+__device__ __forceinline__ int colsum8_column(int lane) {
+  return 4 * (lane & 1) + 2 * ((lane >> 1) & 1) + ((lane >> 2) & 1);
+}
+
+// The gate for one tile of 128 tokens (tokens 128*tile ...), computed by 128*G gate
+// threads: the thread in lane l of gate warp w owns token row r = 32*q + l, where q is
+// the TMEM lane quarter its warp may read, and the expert columns c = 32*grp + 32*G*i + j
+// of its column group grp = w / 4 (the four warps of a group cover the four quarters).
 // `fetch(c, l, z)` fills l[0..7] with the raw clean logits x.W_g of experts c..c+7 of
 // this thread's token (c a multiple of 8) and z[0..7] with x.W_noise (noisy gating); it
-// is called by all 32 lanes of a warp together.  The loops step 8 experts at a time and
-// are not unrolled: each block runs this code once, so a short instruction stream (few
-// instruction-cache misses) matters more than unrolling.  Every thread of the block must
-// call gate_tile.
-template <int KM, int G, class Fetch>
-__device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const GateArgs& g,
+// is called by all 32 lanes of a warp together.  `sync()` is a barrier over the 128*G
+// gate threads.  The loops step 8 experts at a time and are not unrolled, which keeps
+// the instruction stream short.
+template <int KM, int G, class Fetch, class Sync>
+__device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, int q, int grp,
+                                          int gtid, int64_t tile, const GateArgs& g,
                                           uint8_t* smem) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q = warp & 3, grp = warp >> 2;
+  const int lane = gtid & 31;
   const int row = q * 32 + lane;
+  const int64_t t0 = tile * kRouteBM;
   const int64_t t = t0 + row;
   const bool valid = t < g.T;
   const int E = g.E, k = g.k;
@@ -141,8 +172,7 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
   int* fid = reinterpret_cast<int*>(ps + G * 128);               // [128][KM]
   float* fgate = reinterpret_cast<float*>(fid + 128 * KM);       // [128][KM]
   float* fkth = fgate + 128 * KM;                                // [128][2]
-  float* tr = fkth + 128 * 2;                                    // [4G warps][2][32][33]
-  float* qsum = tr + 4 * G * 2 * 32 * 33;                        // [4][2][E]
+  float* qsum = fkth + 128 * 2;                                  // [4][2][E]
 
   // ---- pass 1: partial top-(k+1) and maximum over this thread's experts
   auto scores8 = [&](int c, float (&sc)[8]) {
@@ -172,7 +202,7 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
       float gm = fmaxf(fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])),
                        fmaxf(fmaxf(sc[4], sc[5]), fmaxf(sc[6], sc[7])));
       m = fmaxf(m, gm);
-      if (gm >= thr) {  // rare after the first few groups
+      if (gm >= thr) {
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           if (c + j < E && sc[j] >= thr) top.insert(sc[j], c + j, k);
@@ -203,7 +233,7 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
   }
   pm[grp * 128 + row] = m;
   ps[grp * 128 + row] = ssum;
-  __syncthreads();
+  sync();
 
   // ---- merge the G partial results of each token (group 0) and write the outputs
   if (grp == 0) {
@@ -260,8 +290,11 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
     fkth[row * 2 + 0] = kth;
     fkth[row * 2 + 1] = kth1;
   }
-  if (g.partials == nullptr) return;  // uniform across the block
-  __syncthreads();
+  if (g.partials == nullptr) {  // uniform across the gate threads
+    sync();                     // the lists are reused by the next tile
+    return;
+  }
+  sync();
 
   // ---- pass 2: Importance and Load partial sums over this tile's tokens
   const float kth = fkth[row * 2 + 0], kth1 = fkth[row * 2 + 1];
@@ -272,7 +305,6 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
     myid[jj] = fid[row * KM + jj];
     myg[jj] = fgate[row * KM + jj];
   }
-  float* mytr = tr + warp * (2 * 32 * 33);
   for (int c0 = grp * 32; c0 < E; c0 += 32 * G) {
 #pragma unroll 1
     for (int c = c0; c < c0 + 32; c += 8) {
@@ -304,47 +336,46 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, int64_t t0, const 
           }
         }
       }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        mytr[lane * 33 + (c - c0) + j] = gi[j];
-        mytr[32 * 33 + lane * 33 + (c - c0) + j] = pl[j];
+      // column sums over the warp's 32 tokens
+      const float si = warp_colsum8(gi, lane);
+      const float sl = warp_colsum8(pl, lane);
+      const int col = c + colsum8_column(lane);
+      if (lane < 8 && col < E) {
+        qsum[(q * 2 + 0) * E + col] = si;
+        qsum[(q * 2 + 1) * E + col] = sl;
       }
     }
-    // column sums over the warp's 32 tokens through the padded transpose
-    __syncwarp();
-    float si = 0.0f, sl = 0.0f;
-#pragma unroll 4
-    for (int r = 0; r < 32; ++r) {
-      si += mytr[r * 33 + lane];
-      sl += mytr[32 * 33 + r * 33 + lane];
-    }
-    if (c0 + lane < E) {
-      qsum[(q * 2 + 0) * E + c0 + lane] = si;
-      qsum[(q * 2 + 1) * E + c0 + lane] = sl;
-    }
-    __syncwarp();
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+  sync();
+  for (int e = gtid; e < E; e += 128 * G) {
     float si = 0.0f, sl = 0.0f;
 #pragma unroll
     for (int qq = 0; qq < 4; ++qq) {
       si += qsum[(qq * 2 + 0) * E + e];
       sl += qsum[(qq * 2 + 1) * E + e];
     }
-    g.partials[(static_cast<int64_t>(blockIdx.x) * 2 + 0) * E + e] = si;
-    g.partials[(static_cast<int64_t>(blockIdx.x) * 2 + 1) * E + e] = sl;
+    g.partials[(tile * 2 + 0) * E + e] = si;
+    g.partials[(tile * 2 + 1) * E + e] = sl;
   }
+  sync();  // qsum and the lists are reused by the next tile
 }
 
 // ------------------------------------------------------------------ bf16 router
+//
+// Persistent and warp-specialised.  Warp 0 streams the x tile and the gating weights of
+// each of the CTA's token tiles through a ring of shared-memory stages (TMA); warp 1
+// issues the MMAs of a tile into one of two TMEM accumulator buffers (one when the two
+// products of noisy gating fill TMEM); the 4*G gate warps read a finished buffer, run
+// the gate and hand the buffer back.  So one tile's gate overlaps the next tile's loads
+// and MMAs.
 
 namespace rt {
-// expert-column groups per token: 4 (16 warps), or 2 for k > 4 to leave registers for
-// the longer top-(k+1) lists
+// expert-column groups per token: 4 (16 gate warps), or 2 for k > 4 to leave registers
+// for the longer top-(k+1) lists
 constexpr int groups_for(int KM) { return KM > 4 ? 2 : 4; }
 constexpr int BK = 64;
 constexpr int A_BYTES = kRouteBM * BK * 2;  // 16 KB
+constexpr int GATE_WARP0 = 2;
 }  // namespace rt
 
 struct RouteTcArgs {
@@ -353,13 +384,20 @@ struct RouteTcArgs {
   int acc_cols;   // TMEM columns per accumulator (power of two >= 32, >= e_pad)
   int kblocks;    // d / 64
   int nb;         // 1, or 2 with W_noise
+  int nbuf;       // TMEM accumulator buffers: 2, or 1 when 2 * nb * acc_cols > 512
   int stages;
-  int bar_off;    // byte offset of the barriers in shared memory
+  int ntiles;     // ceil(T / 128)
+  int gate_off;   // byte offset of the gate scratch in shared memory
+  int bar_off;    // byte offset of the barriers
   int* err;
 };
 
+__device__ __forceinline__ void gate_bar_sync(int nthreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
 template <int KM, int G = rt::groups_for(KM)>
-__global__ void __launch_bounds__(128 * G, 1)
+__global__ void __launch_bounds__(64 + 128 * G, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     const __grid_constant__ CUtensorMap tmG,
                     const __grid_constant__ CUtensorMap tmN, const RouteTcArgs a) {
@@ -371,20 +409,35 @@ __global__ void __launch_bounds__(128 * G, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + a.bar_off);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = smem_u32(bars + a.stages);
-  const uint32_t done = smem_u32(bars + 2 * a.stages);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * a.stages + 1);
+  const uint32_t tfull0 = smem_u32(bars + 2 * a.stages);
+  const uint32_t tempty0 = smem_u32(bars + 2 * a.stages + 2);
+  const uint32_t drain = smem_u32(bars + 2 * a.stages + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * a.stages + 5);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* s_gate_fail = reinterpret_cast<volatile int*>(tmem_holder + 2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t ncols = static_cast<uint32_t>(a.nb * a.acc_cols);
+  const uint32_t buf_cols = static_cast<uint32_t>(a.nb * a.acc_cols);
+  const uint32_t ncols = buf_cols * static_cast<uint32_t>(a.nbuf);
+  constexpr int GATE_WARPS = 4 * G;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
-    mbar_init(done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, GATE_WARPS);
+    }
+    mbar_init(drain, 1);
     *s_abort = 0;
+    *s_gate_fail = 0;
     fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmG);
+    if (a.nb == 2) tma_prefetch_desc(&tmN);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), ncols);
@@ -394,107 +447,139 @@ __global__ void __launch_bounds__(128 * G, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int t0 = blockIdx.x * kRouteBM;
-  grid_dep_wait();  // x and the outputs' previous readers belong to earlier kernels
+  grid_dep_wait();  // x, and readers of the outputs, belong to earlier kernels
   grid_dep_launch();
 
   if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&tmX);
+      // ------------------------------------------------------------ TMA producer
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_par = 0;
       bool aborted = false;
-      for (int kb = 0; kb < a.kblocks; ++kb) {
-        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, s_abort)) {
-          aborted = true;
-          break;
-        }
-        uint8_t* st = smem + stage * stage_bytes;
-        const uint32_t fb = full0 + 8 * stage;
-        mbar_arrive_expect_tx(fb, static_cast<uint32_t>(stage_bytes));
-        tma_load_2d(smem_u32(st), &tmX, fb, kb * rt::BK, t0);
-        tma_load_2d(smem_u32(st + rt::A_BYTES), &tmG, fb, kb * rt::BK, 0);
-        if (a.nb == 2) tma_load_2d(smem_u32(st + rt::A_BYTES + b_bytes), &tmN, fb, kb * rt::BK, 0);
-        armed |= 1u << stage;
-        armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-        if (++stage == a.stages) {
-          stage = 0;
-          phase ^= 1;
+      for (int L = blockIdx.x; L < a.ntiles && !aborted; L += gridDim.x) {
+        for (int kb = 0; kb < a.kblocks; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, s_abort)) {
+            aborted = true;
+            break;
+          }
+          uint8_t* st = smem + stage * stage_bytes;
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, static_cast<uint32_t>(stage_bytes));
+          tma_load_2d(smem_u32(st), &tmX, fb, kb * rt::BK, L * kRouteBM);
+          tma_load_2d(smem_u32(st + rt::A_BYTES), &tmG, fb, kb * rt::BK, 0);
+          if (a.nb == 2) tma_load_2d(smem_u32(st + rt::A_BYTES + b_bytes), &tmN, fb, kb * rt::BK, 0);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == a.stages) {
+            stage = 0;
+            phase ^= 1;
+          }
         }
       }
       if (aborted) {
         set_error(a.err, kErrTimeout);
         *s_abort = 1;
+        // let every copy this thread started land before the CTA releases its smem
         for (int s = 0; s < a.stages; ++s)
           if (armed & (1u << s)) mbar_wait(full0 + 8 * s, (armed_par >> s) & 1, nullptr, kDrainLimitNs);
       }
     }
-    __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
       const uint32_t idesc = idesc_f32acc(kRouteBM, a.e_pad, kFmtBF16);
-      int stage = 0;
-      uint32_t phase = 0;
+      int stage = 0, buf = 0;
+      uint32_t phase = 0, buf_phase = 0;
       bool aborted = false;
-      for (int kb = 0; kb < a.kblocks; ++kb) {
-        if (!mbar_wait(full0 + 8 * stage, phase, s_abort)) {
+      for (int L = blockIdx.x; L < a.ntiles && !aborted; L += gridDim.x) {
+        if (!mbar_wait(tempty0 + 8 * buf, buf_phase ^ 1, s_abort)) {
           aborted = true;
           break;
         }
         tc_fence_after();
-        const uint32_t st = smem_u32(smem + stage * stage_bytes);
+        const uint32_t d0 = tmem_base + static_cast<uint32_t>(buf) * buf_cols;
+        for (int kb = 0; kb < a.kblocks; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, s_abort)) {
+            aborted = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + stage * stage_bytes);
 #pragma unroll
-        for (int kk = 0; kk < rt::BK / 16; ++kk) {
-          const uint64_t ad = sdesc_k128(st + kk * 32);
-          const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
-          tc_mma_f16kind(tmem_base, ad, sdesc_k128(st + rt::A_BYTES + kk * 32), idesc, acc);
-          if (a.nb == 2)
-            tc_mma_f16kind(tmem_base + a.acc_cols, ad,
-                           sdesc_k128(st + rt::A_BYTES + b_bytes + kk * 32), idesc, acc);
+          for (int kk = 0; kk < rt::BK / 16; ++kk) {
+            const uint64_t ad = sdesc_k128(st + kk * 32);
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            tc_mma_f16kind(d0, ad, sdesc_k128(st + rt::A_BYTES + kk * 32), idesc, acc);
+            if (a.nb == 2)
+              tc_mma_f16kind(d0 + a.acc_cols, ad,
+                             sdesc_k128(st + rt::A_BYTES + b_bytes + kk * 32), idesc, acc);
+          }
+          tc_commit(empty0 + 8 * stage);
+          if (++stage == a.stages) {
+            stage = 0;
+            phase ^= 1;
+          }
         }
-        tc_commit(empty0 + 8 * stage);
-        if (++stage == a.stages) {
-          stage = 0;
-          phase ^= 1;
+        if (aborted) break;
+        tc_commit(tfull0 + 8 * buf);
+        if (++buf == a.nbuf) {
+          buf = 0;
+          buf_phase ^= 1;
         }
       }
       if (aborted) {
         set_error(a.err, kErrTimeout);
         *s_abort = 1;
+        tc_commit(drain);  // wait for the MMAs already issued before TMEM is freed
+        mbar_wait(drain, 0, nullptr, kDrainLimitNs);
       }
-      tc_commit(done);  // arrives once every MMA issued above has finished
-      if (aborted) mbar_wait(done, 0, nullptr, kDrainLimitNs);
     }
-    __syncwarp();
-  }
-  if (!mbar_wait(done, 0, s_abort)) *s_abort = 1;
-  __syncthreads();
-  const bool ok = (*s_abort == 0);
-  tc_fence_after();
-  if (ok) {
-    // warp w reads TMEM lanes 32*(w%4) .. +31: its token rows
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    auto fetch = [&](int c, float (&l)[8], float (&z)[8]) {
-      uint32_t v[8];
-      tmem_ld8(tmem_base + lane_base + c, v);
-      if (a.nb == 2) {
-        uint32_t w[8];
-        tmem_ld8(tmem_base + lane_base + a.acc_cols + c, w);
-        tmem_ld_wait();
+  } else {
+    // -------------------------------------------------------------- gate warps
+    const int gw = warp - rt::GATE_WARP0;  // 0 .. 4G-1
+    const int q = warp & 3;                // TMEM lane quarter this warp may read
+    const int grp = gw >> 2;
+    const int gtid = gw * 32 + lane;
+    auto sync = [] { gate_bar_sync(128 * G); };
+    uint8_t* gsm = smem + a.gate_off;
+    int buf = 0;
+    uint32_t buf_phase = 0;
+    for (int L = blockIdx.x; L < a.ntiles; L += gridDim.x) {
+      // every gate warp waits; the decision to stop is taken together after a barrier,
+      // so that no gate warp is left at one of the gate's barriers
+      if (!mbar_wait(tfull0 + 8 * buf, buf_phase, s_abort)) *s_gate_fail = 1;
+      sync();
+      if (*s_gate_fail) break;
+      tc_fence_after();
+      const uint32_t lane_base = (static_cast<uint32_t>(q * 32) << 16) +
+                                 static_cast<uint32_t>(buf) * buf_cols;
+      auto fetch = [&](int c, float (&l)[8], float (&z)[8]) {
+        uint32_t v[8];
+        tmem_ld8(tmem_base + lane_base + c, v);
+        if (a.nb == 2) {
+          uint32_t w[8];
+          tmem_ld8(tmem_base + lane_base + a.acc_cols + c, w);
+          tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) z[j] = __uint_as_float(w[j]);
-      } else {
-        tmem_ld_wait();
+          for (int j = 0; j < 8; ++j) z[j] = __uint_as_float(w[j]);
+        } else {
+          tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) z[j] = 0.0f;
+          for (int j = 0; j < 8; ++j) z[j] = 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) l[j] = __uint_as_float(v[j]);
+      };
+      gate_tile<KM, G>(fetch, sync, q, grp, gtid, L, a.g, gsm);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * buf);
+      if (++buf == a.nbuf) {
+        buf = 0;
+        buf_phase ^= 1;
       }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) l[j] = __uint_as_float(v[j]);
-    };
-    // the stage buffers are idle once `done` has fired: reuse them for the gate
-    gate_tile<KM, G>(fetch, t0, a.g, smem);
-  } else if (threadIdx.x == 0) {
-    set_error(a.err, kErrTimeout);
+    }
+    if (*s_gate_fail && gtid == 0) set_error(a.err, kErrTimeout);
   }
   tc_fence_before();
   __syncthreads();
@@ -524,7 +609,9 @@ __global__ void __launch_bounds__(128, 1)
       z[j] = (in && nz != nullptr) ? nz[t * E + c + j] : 0.0f;
     }
   };
-  gate_tile<KM, 1>(fetch, t0, g, gsmem);
+  const int warp = threadIdx.x >> 5;
+  gate_tile<KM, 1>(fetch, [] { __syncthreads(); }, warp, 0, static_cast<int>(threadIdx.x),
+                   static_cast<int64_t>(blockIdx.x), g, gsmem);
 }
 
 __global__ void finalize_importance_load_kernel(const float* __restrict__ partials, int nblocks,
@@ -571,11 +658,11 @@ static cudaError_t launch_finalize(const RouteProblem& p, int nblocks, const Lau
 template <int KM>
 static cudaError_t launch_route_tc(const CUtensorMap& tmX, const CUtensorMap& tmG,
                                    const CUtensorMap& tmN, const RouteTcArgs& a, int smem,
-                                   int nblocks, const LaunchCtx& c) {
+                                   int grid, const LaunchCtx& c) {
   cudaError_t e = cudaFuncSetAttribute(route_tc_kernel<KM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  return launch_kernel(route_tc_kernel<KM>, dim3(nblocks), dim3(128 * rt::groups_for(KM)), smem, c,
-                       tmX, tmG, tmN, a);
+  return launch_kernel(route_tc_kernel<KM>, dim3(grid), dim3(64 + 128 * rt::groups_for(KM)), smem,
+                       c, tmX, tmG, tmN, a);
 }
 
 cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
@@ -586,19 +673,21 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   while (a.acc_cols < a.e_pad) a.acc_cols <<= 1;
   a.kblocks = p.d / rt::BK;
   a.nb = p.noisy ? 2 : 1;
-  const int stage_bytes = rt::A_BYTES + a.nb * a.e_pad * rt::BK * 2;
-  int stages = (160 * 1024) / stage_bytes;
-  if (stages > 8) stages = 8;
-  if (stages > a.kblocks) stages = a.kblocks;
-  if (stages < 2) stages = 2;
-  a.stages = stages;
+  a.nbuf = 2 * a.nb * a.acc_cols <= 512 ? 2 : 1;
+  a.ntiles = route_blocks(p.T);
   const int km = k_bucket(p.k);
-  int region = stages * stage_bytes;
-  const int red = gate_smem_bytes(km, rt::groups_for(km), p.E);
-  if (region < red) region = red;
-  a.bar_off = (region + 127) / 128 * 128;
+  const int scratch = gate_smem_bytes(km, rt::groups_for(km), p.E);
+  const int stage_bytes = rt::A_BYTES + a.nb * a.e_pad * rt::BK * 2;
+  // the ring takes what the gate scratch and the barriers leave of 227 KB
+  const int bar_bytes = 8 * (2 * 8 + 5) + 16;
+  int stages = (227 * 1024 - 1024 - (scratch + 127) / 128 * 128 - bar_bytes) / stage_bytes;
+  if (stages > 8) stages = 8;
+  if (stages < 2) return cudaErrorInvalidValue;  // not reached for E <= 256, d % 64 == 0
+  a.stages = stages;
+  a.gate_off = stages * stage_bytes;
+  a.bar_off = a.gate_off + (scratch + 127) / 128 * 128;
   a.err = c.err;
-  const int smem = 1024 + a.bar_off + 8 * (2 * stages + 1) + 16;
+  const int smem = 1024 + a.bar_off + 8 * (2 * stages + 5) + 16;
 
   CUtensorMap tmX, tmG, tmN;
   if (!make_tmap_bf16(&tmX, p.x, static_cast<uint64_t>(p.T), p.d, kRouteBM)) return cudaErrorInvalidValue;
@@ -608,16 +697,16 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   } else {
     tmN = tmG;
   }
-  const int nblocks = route_blocks(p.T);
+  const int grid = a.ntiles < c.num_sms ? a.ntiles : c.num_sms;
   cudaError_t e;
   switch (km) {
-    case 1: e = launch_route_tc<1>(tmX, tmG, tmN, a, smem, nblocks, c); break;
-    case 2: e = launch_route_tc<2>(tmX, tmG, tmN, a, smem, nblocks, c); break;
-    case 4: e = launch_route_tc<4>(tmX, tmG, tmN, a, smem, nblocks, c); break;
-    default: e = launch_route_tc<8>(tmX, tmG, tmN, a, smem, nblocks, c); break;
+    case 1: e = launch_route_tc<1>(tmX, tmG, tmN, a, smem, grid, c); break;
+    case 2: e = launch_route_tc<2>(tmX, tmG, tmN, a, smem, grid, c); break;
+    case 4: e = launch_route_tc<4>(tmX, tmG, tmN, a, smem, grid, c); break;
+    default: e = launch_route_tc<8>(tmX, tmG, tmN, a, smem, grid, c); break;
   }
   if (e != cudaSuccess) return e;
-  return launch_finalize(p, nblocks, c);
+  return launch_finalize(p, a.ntiles, c);
 }
 
 template <int KM>
