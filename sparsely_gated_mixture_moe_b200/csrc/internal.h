@@ -84,6 +84,7 @@ struct PermuteProblem {
                     // path (null: always use the three-kernel path)
 };
 int64_t permute_blocks(int64_t n);
+int64_t permute_count_chunks(int64_t n);
 cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c);
 
 // ---- expert FFN ------------------------------------------------------------------

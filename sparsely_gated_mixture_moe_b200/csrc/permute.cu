@@ -31,6 +31,9 @@ static_assert(kPermChunk == THREADS, "one assignment per thread per chunk");
 }  // namespace pm
 
 int64_t permute_blocks(int64_t n) { return (n + kPermChunk - 1) / kPermChunk; }
+// Chunks of the per-chunk count array the workspace must hold: the three-kernel path uses
+// ceil(n / 256) chunks of 256 assignments, the one-launch path at most ceil(n / 128).
+int64_t permute_count_chunks(int64_t n) { return (n + 127) / 128; }
 
 // Shared memory of perm_count_scan_kernel: hist[E] and, for the scan, seg[2][256] and
 // kept[E] ints.
@@ -190,31 +193,28 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
 
 // ------------------------------------------------------------------ one-launch path
 //
-// The same counting sort in one launch.  Blocks of 1024 threads; block c < nchunks owns
-// assignments [1024c, 1024c + 1024).
-//   phase 1  each owner block ranks its chunk stably (warp match + per-warp prefix, kept
-//            in registers and shared memory) and writes its per-expert counts to
-//            blk[e][c]
+// The same counting sort in one launch with one grid barrier.  The n assignments are
+// split into nchunks chunks of `chunk` (<= 1024, a multiple of 32) consecutive
+// assignments, one per block of 1024 threads; all blocks are resident at once (the grid
+// never exceeds what the occupancy query says fits).
+//   phase 1  the block ranks its chunk stably (warp match + per-warp prefix, kept in
+//            registers and shared memory) and writes its per-expert counts to blk[e][c]
 //   barrier
-//   phase 2  each owner block sums column e of blk below its chunk (its rank base) and
-//            over all chunks (the expert's count), scans min(count, C) over the experts
-//            into offsets (block 0 writes counts and offsets), and writes slot_pos and
-//            perm_src for its chunk.  Every owner block redoes these small sums itself,
-//            so no second scan pass or flag is needed
-//   barrier
-//   phase 3  all blocks copy the kept rows x[perm_src[s] / k] -> x_perm[s]
-// The grid never exceeds what the occupancy query says fits on the GPU at once, so every
-// block reaches each barrier; the waits are bounded all the same (1 s, then the timeout
-// bit and an early exit).  The barrier counter and an exit counter live in the workspace
-// and are reset by the last block to leave.
+//   phase 2  the block sums column e of blk below its chunk (its rank base) and over all
+//            chunks (the expert's count), scans min(count, C) into offsets (block 0
+//            writes counts and offsets), writes slot_pos and perm_src for its chunk, and
+//            copies its kept rows x[a / k] -> x_perm[slot] (16-byte vectors, two rows
+//            per warp in flight).  Every block redoes the small column sums itself, so
+//            no second scan pass or flag is needed.
+// The barrier is an arrival counter in the workspace with a bounded wait (1 s, then the
+// timeout bit and an early exit); the last block to leave resets it and the exit counter.
 namespace pf {
 constexpr int THREADS = 1024;
 constexpr int WARPS = THREADS / 32;
-constexpr int CHUNK = THREADS;
 }  // namespace pf
 
 static size_t fused_smem(int E) {
-  return (static_cast<size_t>(pf::WARPS) * E + 3 * static_cast<size_t>(E) + 2 * pf::THREADS + 64) * 4;
+  return (static_cast<size_t>(pf::WARPS) * E + 3 * static_cast<size_t>(E) + 3 * pf::THREADS + 64) * 4;
 }
 
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
@@ -224,8 +224,8 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
 }
 
 // Barrier over all blocks of the grid (all resident).  Arrivals accumulate in *ctr over
-// the launch; a barrier is complete once *ctr reaches `target`.  Gives up after the wait
-// limit: sets the timeout bit and *s_abort.  Every thread must call it.
+// the launch; the barrier is complete once *ctr reaches `target`.  Gives up after the
+// wait limit: sets the timeout bit and *s_abort.  Every thread must call it.
 __device__ bool grid_barrier(int* ctr, int target, int* err, volatile int* s_abort) {
   __syncthreads();
   if (threadIdx.x == 0 && *s_abort == 0) {
@@ -238,7 +238,7 @@ __device__ bool grid_barrier(int* ctr, int target, int* err, volatile int* s_abo
         *s_abort = 1;
         break;
       }
-      __nanosleep(100);
+      __nanosleep(64);
     }
     __threadfence();
   }
@@ -248,10 +248,10 @@ __device__ bool grid_barrier(int* ctr, int target, int* err, volatile int* s_abo
 
 __global__ void __launch_bounds__(pf::THREADS, 1)
     perm_fused_kernel(const int32_t* __restrict__ idx, int64_t n, int E, int64_t C, int k,
-                      int nchunks, int32_t* blk, int32_t* __restrict__ counts, int32_t* offsets,
-                      int32_t* perm_src, int32_t* __restrict__ slot_pos,
-                      const uint8_t* __restrict__ x, uint8_t* __restrict__ x_perm, int row_bytes,
-                      int32_t* sync, int* err) {
+                      int chunk, int nchunks, int32_t* blk, int32_t* __restrict__ counts,
+                      int32_t* __restrict__ offsets, int32_t* __restrict__ perm_src,
+                      int32_t* __restrict__ slot_pos, const uint8_t* __restrict__ x,
+                      uint8_t* __restrict__ x_perm, int row_bytes, int32_t* sync, int* err) {
   extern __shared__ int fsm[];
   int* wbase = fsm;                     // [WARPS][E]: per-warp rank bases
   int* s_pre = wbase + pf::WARPS * E;   // [E]: rank base of this chunk
@@ -259,24 +259,27 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
   int* s_off = s_tot + E;               // [E]: offsets
   int* segp = s_off + E;                // [THREADS]
   int* segt = segp + pf::THREADS;       // [THREADS]
-  int* scratch = segt + pf::THREADS;    // [64]
+  int* s_slot = segt + pf::THREADS;     // [THREADS]: slot of each assignment of the chunk
+  int* scratch = s_slot + pf::THREADS;  // [64]
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t lt_mask = (1u << lane) - 1u;
+  const int c = blockIdx.x;
+  const int64_t a0 = static_cast<int64_t>(c) * chunk;
+  const int cn = static_cast<int>(min(static_cast<int64_t>(chunk), n - a0));  // > 0
+  const int nw = (chunk + 31) >> 5;  // warps holding assignments
   if (tid == 0) s_abort = 0;
-  for (int i = tid; i < pf::WARPS * E; i += pf::THREADS) wbase[i] = 0;
+  for (int i = tid; i < nw * E; i += pf::THREADS) wbase[i] = 0;
   grid_dep_wait();
   grid_dep_launch();
   __syncthreads();
 
   // ---- phase 1: stable ranks within the chunk, chunk counts to blk[e][c]
-  const int c = blockIdx.x;
-  const bool owner = c < nchunks;  // uniform across the block
-  const int64_t a = static_cast<int64_t>(c) * pf::CHUNK + tid;
+  const int64_t a = a0 + tid;
   int e = -1;
   uint32_t peers = 0;
-  if (owner) {
-    if (a < n) {
+  if (warp < nw) {  // uniform across the warp
+    if (tid < cn) {
       e = idx[a];
       if (e < 0 || e >= E) {
         set_error(err, kErrExpertIndex);
@@ -287,22 +290,19 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     if (e >= 0 && (peers & lt_mask) == 0) wbase[warp * E + e] = __popc(peers);
   }
   __syncthreads();
-  if (owner) {
-    for (int xe = tid; xe < E; xe += pf::THREADS) {
-      int run = 0;
-      for (int w = 0; w < pf::WARPS; ++w) {
-        const int v = wbase[w * E + xe];
-        wbase[w * E + xe] = run;
-        run += v;
-      }
-      blk[static_cast<int64_t>(xe) * nchunks + c] = run;
+  for (int xe = tid; xe < E; xe += pf::THREADS) {
+    int run = 0;
+    for (int w = 0; w < nw; ++w) {
+      const int v = wbase[w * E + xe];
+      wbase[w * E + xe] = run;
+      run += v;
     }
+    blk[static_cast<int64_t>(xe) * nchunks + c] = run;
   }
-  const int G = static_cast<int>(gridDim.x);
-  bool ok = grid_barrier(sync, G, err, &s_abort);
+  const bool ok = grid_barrier(sync, nchunks, err, &s_abort);
 
-  // ---- phase 2: rank bases, counts, offsets; slot_pos and perm_src of this chunk
-  if (ok && owner) {
+  // ---- phase 2: rank bases, counts, offsets; slot_pos, perm_src and rows of this chunk
+  if (ok) {
     int tpe = 1;  // threads per expert, each summing a run of chunks
     while (tpe * 2 * E <= pf::THREADS) tpe *= 2;
     const int epr = pf::THREADS / tpe;  // experts per round
@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     }
     if (c == 0 && tid == 0) offsets[E] = carry;
     __syncthreads();
-    if (a < n) {
+    if (tid < cn) {
       int slot = -1;
       if (e >= 0) {
         const int rank = s_pre[e] + wbase[warp * E + e] + __popc(peers & lt_mask);
@@ -359,39 +359,38 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       }
       slot_pos[a] = slot;
       if (slot >= 0) perm_src[slot] = static_cast<int32_t>(a);
+      s_slot[tid] = slot;
     }
-  }
-  ok = ok && grid_barrier(sync, 2 * G, err, &s_abort);
-
-  // ---- phase 3: x_perm[s] = x[perm_src[s] / k], two rows per warp in flight
-  if (ok) {
-    const int n_kept = __ldcg(offsets + E);
+    __syncthreads();
+    // the chunk's kept rows, in assignment order; warp w takes assignments w, w + 32, ...
     const int nv = row_bytes >> 4;
-    const int stride = G * pf::WARPS;
-    for (int s = blockIdx.x * pf::WARPS + warp; s < n_kept; s += 2 * stride) {
-      const int s2 = s + stride;
-      const bool two = s2 < n_kept;
-      const int64_t t1 = __ldcg(perm_src + s) / k;
-      const int64_t t2 = two ? __ldcg(perm_src + s2) / k : t1;
+    for (int i = warp; i < cn; i += 2 * pf::WARPS) {
+      const int i2 = i + pf::WARPS;
+      const int sl1 = s_slot[i];
+      const int sl2 = i2 < cn ? s_slot[i2] : -1;
+      if (sl1 < 0 && sl2 < 0) continue;
+      const int64_t t1 = (a0 + i) / k, t2 = (a0 + i2) / k;
       const uint4* src1 = reinterpret_cast<const uint4*>(x + t1 * row_bytes);
-      const uint4* src2 = reinterpret_cast<const uint4*>(x + t2 * row_bytes);
-      uint4* dst1 = reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(s) * row_bytes);
-      uint4* dst2 = reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(two ? s2 : s) * row_bytes);
+      const uint4* src2 = reinterpret_cast<const uint4*>(x + (sl2 >= 0 ? t2 : t1) * row_bytes);
+      uint4* dst1 = reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(sl1 >= 0 ? sl1 : 0) * row_bytes);
+      uint4* dst2 = reinterpret_cast<uint4*>(x_perm + static_cast<int64_t>(sl2 >= 0 ? sl2 : 0) * row_bytes);
       int v = lane;
       for (; v + 32 < nv; v += 64) {
-        const uint4 a0 = __ldg(src1 + v), a1 = __ldg(src1 + v + 32);
-        const uint4 b0 = __ldg(src2 + v), b1 = __ldg(src2 + v + 32);
-        dst1[v] = a0;
-        dst1[v + 32] = a1;
-        if (two) {
-          dst2[v] = b0;
-          dst2[v + 32] = b1;
+        const uint4 p0 = __ldg(src1 + v), p1 = __ldg(src1 + v + 32);
+        const uint4 q0 = __ldg(src2 + v), q1 = __ldg(src2 + v + 32);
+        if (sl1 >= 0) {
+          dst1[v] = p0;
+          dst1[v + 32] = p1;
+        }
+        if (sl2 >= 0) {
+          dst2[v] = q0;
+          dst2[v + 32] = q1;
         }
       }
       for (; v < nv; v += 32) {
-        const uint4 a0 = __ldg(src1 + v), b0 = __ldg(src2 + v);
-        dst1[v] = a0;
-        if (two) dst2[v] = b0;
+        const uint4 p0 = __ldg(src1 + v), q0 = __ldg(src2 + v);
+        if (sl1 >= 0) dst1[v] = p0;
+        if (sl2 >= 0) dst2[v] = q0;
       }
     }
   }
@@ -400,17 +399,18 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
   __syncthreads();
   if (tid == 0) {
     __threadfence();
-    if (atomicAdd(sync + 1, 1) == G - 1) {
+    if (atomicAdd(sync + 1, 1) == nchunks - 1) {
       atomicExch(sync, 0);
       atomicExch(sync + 1, 0);
     }
   }
 }
 
-// Grid for the one-launch path, or 0 when its blocks would not all fit at once.
-static int fused_grid(const PermuteProblem& p, const LaunchCtx& c, size_t smem) {
+// Chunking for the one-launch path: returns the number of chunks (= blocks) and sets
+// *chunk, or returns 0 when the chunks would exceed 1024 assignments or the blocks would
+// not all fit on the GPU at once.
+static int fused_chunks(const PermuteProblem& p, const LaunchCtx& c, size_t smem, int* chunk) {
   if (p.sync == nullptr) return 0;
-  const int64_t nchunks = (p.n + pf::CHUNK - 1) / pf::CHUNK;
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(perm_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
@@ -420,12 +420,15 @@ static int fused_grid(const PermuteProblem& p, const LaunchCtx& c, size_t smem) 
                                                     smem) != cudaSuccess)
     return 0;
   const int64_t cap = static_cast<int64_t>(per_sm) * c.num_sms;
-  if (nchunks > cap) return 0;
-  // enough warps to keep about four rows each in the gather, at least one block per chunk
-  int64_t g = (p.n + 4 * pf::WARPS - 1) / (4 * pf::WARPS);
+  // at least 128 assignments per chunk, at most one chunk per resident block
+  int64_t g = (p.n + 127) / 128;
   if (g > cap) g = cap;
-  if (g < nchunks) g = nchunks;
-  return static_cast<int>(g);
+  if (g < 1) return 0;
+  int64_t ch = (p.n + g - 1) / g;
+  ch = (ch + 31) / 32 * 32;
+  if (ch > pf::THREADS) return 0;
+  *chunk = static_cast<int>(ch);
+  return static_cast<int>((p.n + ch - 1) / ch);
 }
 
 cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c) {
@@ -433,12 +436,12 @@ cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c) {
   if (nblk == 0) return cudaSuccess;
   cudaError_t e = cudaSuccess;
   const size_t f_smem = fused_smem(p.E);
-  const int fg = fused_grid(p, c, f_smem);
-  if (fg > 0) {
-    const int nchunks = static_cast<int>((p.n + pf::CHUNK - 1) / pf::CHUNK);
-    return launch_kernel(perm_fused_kernel, dim3(fg), dim3(pf::THREADS), f_smem, c, p.topk_idx,
-                         p.n, p.E, p.C, p.k, nchunks, p.blk, p.counts, p.offsets, p.perm_src,
-                         p.slot_pos, static_cast<const uint8_t*>(p.x),
+  int chunk = 0;
+  const int nchunks = fused_chunks(p, c, f_smem, &chunk);
+  if (nchunks > 0) {
+    return launch_kernel(perm_fused_kernel, dim3(nchunks), dim3(pf::THREADS), f_smem, c,
+                         p.topk_idx, p.n, p.E, p.C, p.k, chunk, nchunks, p.blk, p.counts,
+                         p.offsets, p.perm_src, p.slot_pos, static_cast<const uint8_t*>(p.x),
                          static_cast<uint8_t*>(p.x_perm), p.d * p.esize, p.sync, c.err);
   }
   const size_t cs_smem = count_scan_smem(p.E);
