@@ -101,22 +101,6 @@ __device__ __forceinline__ Tile decode_tile(int L, const int* tp, const Args& a)
   return t;
 }
 
-// erf by Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
-// erf(x) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-x^2), t = 1 / (1 + p x),
-// x >= 0, |error| <= 1.5e-7 (odd extension for x < 0).  About a third of the
-// instructions of a full-accuracy erf; the activations it feeds are rounded to 16 bits.
-__device__ __forceinline__ float erf_as7126(float x) {
-  const float ax = fabsf(x);
-  const float t = __fdividef(1.0f, fmaf(0.3275911f, ax, 1.0f));
-  float poly = fmaf(1.061405429f, t, -1.453152027f);
-  poly = fmaf(poly, t, 1.421413741f);
-  poly = fmaf(poly, t, -0.284496736f);
-  poly = fmaf(poly, t, 0.254829592f);
-  poly *= t;
-  const float y = 1.0f - poly * __expf(-ax * ax);
-  return copysignf(y, x);
-}
-
 template <int ACT>
 __device__ __forceinline__ float epi_act(float z) {
   if (ACT == 1) return fmaxf(z, 0.0f);
@@ -473,7 +457,7 @@ __global__ void erf_check_kernel(const float* __restrict__ x, float* __restrict_
                                  float* __restrict__ ref, int64_t n) {
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    fast[i] = gg::erf_as7126(x[i]);
+    fast[i] = erf_as7126(x[i]);
     ref[i] = erff(x[i]);
   }
 }

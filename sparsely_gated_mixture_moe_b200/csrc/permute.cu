@@ -32,8 +32,9 @@ static_assert(kPermChunk == THREADS, "one assignment per thread per chunk");
 
 int64_t permute_blocks(int64_t n) { return (n + kPermChunk - 1) / kPermChunk; }
 // Chunks of the per-chunk count array the workspace must hold: the three-kernel path uses
-// ceil(n / 256) chunks of 256 assignments, the one-launch path at most ceil(n / 128).
-int64_t permute_count_chunks(int64_t n) { return (n + 127) / 128; }
+// ceil(n / 256) chunks of 256 assignments, the one-launch path at most ceil(n / 128),
+// padded to a multiple of 4.
+int64_t permute_count_chunks(int64_t n) { return (n + 127) / 128 + 3; }
 
 // Shared memory of perm_count_scan_kernel: hist[E] and, for the scan, seg[2][256] and
 // kept[E] ints.
@@ -199,6 +200,8 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
 // never exceeds what the occupancy query says fits).
 //   phase 1  the block ranks its chunk stably (warp match + per-warp prefix, kept in
 //            registers and shared memory) and writes its per-expert counts to blk[e][c]
+//            (rows padded to a multiple of 4 chunks, the padding zeroed by block 0, so
+//            that phase 2 reads them as 16-byte vectors)
 //   barrier
 //   phase 2  the block sums column e of blk below its chunk (its rank base) and over all
 //            chunks (the expert's count), scans min(count, C) into offsets (block 0
@@ -290,6 +293,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     if (e >= 0 && (peers & lt_mask) == 0) wbase[warp * E + e] = __popc(peers);
   }
   __syncthreads();
+  const int ncs = (nchunks + 3) & ~3;  // padded row length of blk
   for (int xe = tid; xe < E; xe += pf::THREADS) {
     int run = 0;
     for (int w = 0; w < nw; ++w) {
@@ -297,26 +301,32 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       wbase[w * E + xe] = run;
       run += v;
     }
-    blk[static_cast<int64_t>(xe) * nchunks + c] = run;
+    blk[static_cast<int64_t>(xe) * ncs + c] = run;
+    if (c == 0)
+      for (int b = nchunks; b < ncs; ++b) blk[static_cast<int64_t>(xe) * ncs + b] = 0;
   }
   const bool ok = grid_barrier(sync, nchunks, err, &s_abort);
 
   // ---- phase 2: rank bases, counts, offsets; slot_pos, perm_src and rows of this chunk
   if (ok) {
-    int tpe = 1;  // threads per expert, each summing a run of chunks
+    int tpe = 1;  // threads per expert, each summing a run of 4-chunk vectors
     while (tpe * 2 * E <= pf::THREADS) tpe *= 2;
     const int epr = pf::THREADS / tpe;  // experts per round
-    const int len = (nchunks + tpe - 1) / tpe;
+    const int nq = ncs >> 2;
+    const int len = (nq + tpe - 1) / tpe;
     for (int e0 = 0; e0 < E; e0 += epr) {
       const int el = tid % epr, part = tid / epr, xe = e0 + el;
       int pre = 0, tot = 0;
       if (xe < E) {
-        const int b0 = part * len, b1 = min(nchunks, b0 + len);
-        const int32_t* col = blk + static_cast<int64_t>(xe) * nchunks;
-        for (int b = b0; b < b1; ++b) {
-          const int v = __ldcg(col + b);
-          tot += v;
-          pre += (b < c) ? v : 0;
+        const int q0 = part * len, q1 = min(nq, q0 + len);
+        const int4* col = reinterpret_cast<const int4*>(blk + static_cast<int64_t>(xe) * ncs);
+#pragma unroll 4
+        for (int qi = q0; qi < q1; ++qi) {
+          const int4 v = __ldcg(col + qi);
+          const int b = 4 * qi;
+          tot += v.x + v.y + v.z + v.w;
+          pre += (b < c ? v.x : 0) + (b + 1 < c ? v.y : 0) + (b + 2 < c ? v.z : 0) +
+                 (b + 3 < c ? v.w : 0);
         }
       }
       segp[tid] = pre;

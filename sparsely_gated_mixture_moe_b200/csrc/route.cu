@@ -73,7 +73,24 @@ struct TopList {
       i[s] = 0x7fffffff;
     }
   }
-  // keeps the first k+1 slots (k <= KM)
+  // Branch-free insertion of a score that arrives after every equal score already in the
+  // list (ascending expert order): it displaces the entries it strictly exceeds.  Every
+  // slot is computed from the old list, so the KM+1 updates are independent.
+  __device__ __forceinline__ void push(float cv, int ci) {
+#pragma unroll
+    for (int q = KM; q >= 1; --q) {
+      const bool up = cv > v[q - 1];
+      const bool here = cv > v[q];
+      const float nv = up ? v[q - 1] : (here ? cv : v[q]);
+      const int ni = up ? i[q - 1] : (here ? ci : i[q]);
+      v[q] = nv;
+      i[q] = ni;
+    }
+    const bool first = cv > v[0];
+    v[0] = first ? cv : v[0];
+    i[0] = first ? ci : i[0];
+  }
+  // keeps the first k+1 slots (k <= KM); equal scores rank by expert index
   __device__ __forceinline__ void insert(float cv, int ci, int k) {
 #pragma unroll
     for (int q = 0; q <= KM; ++q) {
@@ -95,7 +112,16 @@ __host__ __device__ constexpr int gate_smem_bytes(int KM, int G, int E) {
          + G * 128 * 8              // partial softmax (max, sum)
          + 128 * (2 * KM + 2) * 4   // final experts, gates, k-th and (k+1)-th score
          + 4 * 2 * E * 4            // per-lane-quarter column sums (Importance, Load)
+         + E * 4                    // logit bias (zeros when there is none)
          + 64;
+}
+
+// Bias of each expert's logit into shared memory (zeros without a bias), by `nthreads`
+// threads of which this is number `tid`; the caller synchronises before gate_tile.
+__device__ __forceinline__ void load_bias_smem(const GateArgs& g, uint8_t* smem, int KM, int G,
+                                               int tid, int nthreads) {
+  float* sbias = reinterpret_cast<float*>(smem + gate_smem_bytes(KM, G, g.E) - 64 - g.E * 4);
+  for (int e = tid; e < g.E; e += nthreads) sbias[e] = g.bias ? __ldg(g.bias + e) : 0.0f;
 }
 
 // Sum of v[j] over the 32 lanes of a warp for each of the 8 columns j, as a
@@ -130,14 +156,18 @@ __device__ __forceinline__ int colsum8_column(int lane) {
 
 // The gate for one tile of 128 tokens (tokens 128*tile ...), computed by 128*G gate
 // threads: the thread in lane l of gate warp w owns token row r = 32*q + l, where q is
-// the TMEM lane quarter its warp may read, and the expert columns c = 32*grp + 32*G*i + j
-// of its column group grp = w / 4 (the four warps of a group cover the four quarters).
-// `fetch(c, l, z)` fills l[0..7] with the raw clean logits x.W_g of experts c..c+7 of
-// this thread's token (c a multiple of 8) and z[0..7] with x.W_noise (noisy gating); it
-// is called by all 32 lanes of a warp together.  `sync()` is a barrier over the 128*G
-// gate threads.  The loops step 8 experts at a time and are not unrolled, which keeps
-// the instruction stream short.
-template <int KM, int G, class Fetch, class Sync>
+// the TMEM lane quarter its warp may read, and the expert columns c = W*grp + W*G*i + j
+// (0 <= j < W) of its column group grp = w / 4 (the four warps of a group cover the
+// four quarters).
+// `fetch(c, l, z)` fills l[0..W-1] with the raw clean logits x.W_g of experts c..c+W-1
+// of this thread's token (c a multiple of W) and z[0..W-1] with x.W_noise (noisy
+// gating); it is called by all 32 lanes of a warp together and waits once for its
+// loads.  `sync()` is a barrier over the 128*G gate threads.  Each W-column slice is
+// scored from registers: its maximum updates the running softmax (one rescale per
+// slice), and a group of 8 scores enters the top list by branch-free insertion unless
+// no lane of the warp has one above its current (k+1)-th score.  The logit bias has been loaded into shared memory
+// (load_bias_smem) by the caller.
+template <int KM, int G, int W, class Fetch, class Sync>
 __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, int q, int grp,
                                           int gtid, int64_t tile, const GateArgs& g,
                                           uint8_t* smem) {
@@ -161,7 +191,6 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
       for (int j = 0; j < 8; ++j) nz[j] = (noise_row != nullptr && c + j < E) ? __ldg(noise_row + c + j) : 0.0f;
     }
   };
-  const float* bias = g.bias;
   const bool noisy = g.noisy != 0;
   const bool full_softmax = !noisy && !g.renorm;
 
@@ -174,55 +203,69 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
   float* fkth = fgate + 128 * KM;                                // [128][2]
   float* qsum = fkth + 128 * 2;                                  // [4][2][E]
 
-  // ---- pass 1: partial top-(k+1) and maximum over this thread's experts
-  auto scores8 = [&](int c, float (&sc)[8]) {
-    float l[8], z[8], nz[8];
-    fetch(c, l, z);
-    if (noisy) load_noise8(c, nz);
+  const float* sbias = qsum + 4 * 2 * E;                       // [E]
+
+  // ---- pass 1: partial top-(k+1), maximum and softmax sum over this thread's experts
+  auto scores = [&](int cs, float (&sc)[W]) {
+    float l[W], z[W];
+    fetch(cs, l, z);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = c + j;
-      float s = -INFINITY;
-      if (e < E) {
-        s = l[j] + (bias ? __ldg(bias + e) : 0.0f);
-        if (noisy) s += nz[j] * softplus_f(z[j]);
+    for (int g8 = 0; g8 < W / 8; ++g8) {
+      float nz[8];
+      if (noisy) load_noise8(cs + 8 * g8, nz);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int jj = 8 * g8 + j, e = cs + jj;
+        float sv = -INFINITY;
+        if (e < E) {
+          sv = l[jj] + sbias[e];
+          if (noisy) sv += nz[j] * softplus_f(z[jj]);
+        }
+        sc[jj] = sv;
       }
-      sc[j] = s;
     }
   };
   TopList<KM> top;
   top.init();
   float thr = -INFINITY;  // the current (k+1)-th score: values below it cannot enter the list
   float m = -INFINITY, ssum = 0.0f;
-  for (int c0 = grp * 32; c0 < E; c0 += 32 * G) {
 #pragma unroll 1
-    for (int c = c0; c < c0 + 32 && c < E; c += 8) {
-      float sc[8];
-      scores8(c, sc);
-      float gm = fmaxf(fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])),
-                       fmaxf(fmaxf(sc[4], sc[5]), fmaxf(sc[6], sc[7])));
-      m = fmaxf(m, gm);
-      if (gm >= thr) {
+  for (int cs = grp * W; cs < E; cs += W * G) {
+    {
+      float sc[W];
+      scores(cs, sc);
+      float gm8[W / 8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (c + j < E && sc[j] >= thr) top.insert(sc[j], c + j, k);
-        // slots past k stay at -inf, so the maximum over slots >= k is slot k
-        thr = -INFINITY;
-#pragma unroll
-        for (int q2 = 0; q2 <= KM; ++q2)
-          if (q2 >= k) thr = fmaxf(thr, top.v[q2]);
+      for (int g8 = 0; g8 < W / 8; ++g8) {
+        const float* v8 = sc + 8 * g8;
+        gm8[g8] = fmaxf(fmaxf(fmaxf(v8[0], v8[1]), fmaxf(v8[2], v8[3])),
+                        fmaxf(fmaxf(v8[4], v8[5]), fmaxf(v8[6], v8[7])));
       }
-    }
-  }
-  if (full_softmax) {
-    // sum of exp(score - max) over this thread's experts, independent terms
-    for (int c0 = grp * 32; c0 < E; c0 += 32 * G) {
-#pragma unroll 1
-      for (int c = c0; c < c0 + 32 && c < E; c += 8) {
-        float sc[8];
-        scores8(c, sc);
+      float sm = gm8[0];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) ssum += (c + j < E) ? __expf(sc[j] - m) : 0.0f;
+      for (int g8 = 1; g8 < W / 8; ++g8) sm = fmaxf(sm, gm8[g8]);
+      if (full_softmax) {
+        const float nm = fmaxf(m, sm);
+        float add = 0.0f;
+#pragma unroll
+        for (int jj = 0; jj < W; ++jj) add += (cs + jj < E) ? __expf(sc[jj] - nm) : 0.0f;
+        ssum = ssum * __expf(m - nm) + add;  // exp(-inf) = 0 before the first slice
+        m = nm;
+      } else {
+        m = fmaxf(m, sm);
+      }
+#pragma unroll
+      for (int g8 = 0; g8 < W / 8; ++g8) {
+        // skipped by the whole warp when no lane has a score above its (k+1)-th
+        if (__any_sync(0xffffffffu, gm8[g8] > thr)) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) top.push(sc[8 * g8 + j], cs + 8 * g8 + j);
+          // the list is sorted, so the maximum over slots >= k is slot k
+          thr = -INFINITY;
+#pragma unroll
+          for (int q2 = 0; q2 <= KM; ++q2)
+            if (q2 >= k) thr = fmaxf(thr, top.v[q2]);
+        }
       }
     }
   }
@@ -305,44 +348,58 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
     myid[jj] = fid[row * KM + jj];
     myg[jj] = fgate[row * KM + jj];
   }
-  for (int c0 = grp * 32; c0 < E; c0 += 32 * G) {
 #pragma unroll 1
-    for (int c = c0; c < c0 + 32; c += 8) {
-      float gi[8], pl[8];
+  for (int cs = grp * W; cs < E; cs += W * G) {
+    {
+      float gi[W], pl[W];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        gi[j] = 0.0f;
-        pl[j] = 0.0f;
+      for (int jj = 0; jj < W; ++jj) {
+        gi[jj] = 0.0f;
+        pl[jj] = 0.0f;
       }
-      if (c < E) {
-        float l[8], z[8], nz[8];
-        fetch(c, l, z);
-        if (noisy) load_noise8(c, nz);
+      {
+        float l[W], z[W];
+        fetch(cs, l, z);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int e = c + j;
-          if (valid && e < E) {
-            if (noisy && k < E) {
-              // recomputed exactly as in pass 1, so H >= kth means "among the top k"
-              const float li = l[j] + (bias ? __ldg(bias + e) : 0.0f);
-              const float sp = softplus_f(z[j]);
-              const float H = li + nz[j] * sp;
-              const float ex = (H >= kth) ? kth1 : kth;  // kth_excluding(H, k, e)
-              pl[j] = 0.5f * erfcf(-((li - ex) / sp) * 0.70710678118654752f);
+        for (int g8 = 0; g8 < W / 8; ++g8) {
+          float nz[8];
+          if (noisy) load_noise8(cs + 8 * g8, nz);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int jj = 8 * g8 + j, e = cs + jj;
+            if (valid && e < E) {
+              if (noisy && k < E) {
+                // recomputed exactly as in pass 1, so H >= kth means "among the top k"
+                const float li = l[jj] + sbias[e];
+                const float sp = softplus_f(z[jj]);
+                const float H = li + nz[j] * sp;
+                const float ex = (H >= kth) ? kth1 : kth;  // kth_excluding(H, k, e)
+                // Phi((l_e - kth_excluding) / Softplus(z_e))
+                pl[jj] = 0.5f + 0.5f * erf_as7126(__fdividef(li - ex, sp) * 0.70710678118654752f);
+              }
+#pragma unroll
+              for (int q3 = 0; q3 < KM; ++q3)
+                if (myid[q3] == e) gi[jj] = myg[q3];
             }
-#pragma unroll
-            for (int jj = 0; jj < KM; ++jj)
-              if (myid[jj] == e) gi[j] = myg[jj];
           }
         }
       }
-      // column sums over the warp's 32 tokens
-      const float si = warp_colsum8(gi, lane);
-      const float sl = warp_colsum8(pl, lane);
-      const int col = c + colsum8_column(lane);
-      if (lane < 8 && col < E) {
-        qsum[(q * 2 + 0) * E + col] = si;
-        qsum[(q * 2 + 1) * E + col] = sl;
+      // column sums over the warp's 32 tokens, 8 columns at a time
+#pragma unroll
+      for (int g8 = 0; g8 < W / 8; ++g8) {
+        float a8[8], b8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          a8[j] = gi[8 * g8 + j];
+          b8[j] = pl[8 * g8 + j];
+        }
+        const float si = warp_colsum8(a8, lane);
+        const float sl = warp_colsum8(b8, lane);
+        const int col = cs + 8 * g8 + colsum8_column(lane);
+        if (lane < 8 && col < E) {
+          qsum[(q * 2 + 0) * E + col] = si;
+          qsum[(q * 2 + 1) * E + col] = sl;
+        }
       }
     }
   }
@@ -397,7 +454,7 @@ __device__ __forceinline__ void gate_bar_sync(int nthreads) {
 }
 
 template <int KM, int G = rt::groups_for(KM)>
-__global__ void __launch_bounds__(64 + 128 * G, 1)
+__global__ void __launch_bounds__(64 + 128 * G)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     const __grid_constant__ CUtensorMap tmG,
                     const __grid_constant__ CUtensorMap tmN, const RouteTcArgs a) {
@@ -542,6 +599,8 @@ __global__ void __launch_bounds__(64 + 128 * G, 1)
     const int gtid = gw * 32 + lane;
     auto sync = [] { gate_bar_sync(128 * G); };
     uint8_t* gsm = smem + a.gate_off;
+    load_bias_smem(a.g, gsm, KM, G, gtid, 128 * G);
+    sync();
     int buf = 0;
     uint32_t buf_phase = 0;
     for (int L = blockIdx.x; L < a.ntiles; L += gridDim.x) {
@@ -553,24 +612,33 @@ __global__ void __launch_bounds__(64 + 128 * G, 1)
       tc_fence_after();
       const uint32_t lane_base = (static_cast<uint32_t>(q * 32) << 16) +
                                  static_cast<uint32_t>(buf) * buf_cols;
-      auto fetch = [&](int c, float (&l)[8], float (&z)[8]) {
-        uint32_t v[8];
-        tmem_ld8(tmem_base + lane_base + c, v);
-        if (a.nb == 2) {
-          uint32_t w[8];
-          tmem_ld8(tmem_base + lane_base + a.acc_cols + c, w);
+      if (a.nb == 2) {
+        // noisy gating: 16 columns of x.W_g and of x.W_noise per wait
+        auto fetch = [&](int c, float (&l)[16], float (&z)[16]) {
+          uint32_t v[16], w[16];
+          tmem_ld16(tmem_base + lane_base + c, v);
+          tmem_ld16(tmem_base + lane_base + a.acc_cols + c, w);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 8; ++j) z[j] = __uint_as_float(w[j]);
-        } else {
+          for (int j = 0; j < 16; ++j) {
+            l[j] = __uint_as_float(v[j]);
+            z[j] = __uint_as_float(w[j]);
+          }
+        };
+        gate_tile<KM, G, 16>(fetch, sync, q, grp, gtid, L, a.g, gsm);
+      } else {
+        auto fetch = [&](int c, float (&l)[16], float (&z)[16]) {
+          uint32_t v[16];
+          tmem_ld16(tmem_base + lane_base + c, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 8; ++j) z[j] = 0.0f;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) l[j] = __uint_as_float(v[j]);
-      };
-      gate_tile<KM, G>(fetch, sync, q, grp, gtid, L, a.g, gsm);
+          for (int j = 0; j < 16; ++j) {
+            l[j] = __uint_as_float(v[j]);
+            z[j] = 0.0f;
+          }
+        };
+        gate_tile<KM, G, 16>(fetch, sync, q, grp, gtid, L, a.g, gsm);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * buf);
@@ -601,17 +669,19 @@ __global__ void __launch_bounds__(128, 1)
   const int64_t t = t0 + threadIdx.x;
   const bool valid = t < g.T;
   const int E = g.E;
-  auto fetch = [&](int c, float (&l)[8], float (&z)[8]) {
+  auto fetch = [&](int c, float (&l)[16], float (&z)[16]) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 16; ++j) {
       const bool in = valid && (c + j < E);
       l[j] = in ? logits[t * E + c + j] : 0.0f;
       z[j] = (in && nz != nullptr) ? nz[t * E + c + j] : 0.0f;
     }
   };
   const int warp = threadIdx.x >> 5;
-  gate_tile<KM, 1>(fetch, [] { __syncthreads(); }, warp, 0, static_cast<int>(threadIdx.x),
-                   static_cast<int64_t>(blockIdx.x), g, gsmem);
+  load_bias_smem(g, gsmem, KM, 1, static_cast<int>(threadIdx.x), 128);
+  __syncthreads();
+  gate_tile<KM, 1, 16>(fetch, [] { __syncthreads(); }, warp, 0, static_cast<int>(threadIdx.x),
+                       static_cast<int64_t>(blockIdx.x), g, gsmem);
 }
 
 __global__ void finalize_importance_load_kernel(const float* __restrict__ partials, int nblocks,
