@@ -33,7 +33,10 @@ namespace moe {
 
 constexpr int kRouteBM = 128;
 
-int route_blocks(int64_t T) { return static_cast<int>((T + kRouteBM - 1) / kRouteBM); }
+// Tiles of the router: 128 tokens, or 64 ("half tiles") when 128-token tiles would leave
+// most SMs idle.  The partial Importance/Load sums are kept per tile, so the workspace
+// is sized for 64-token tiles.
+int route_blocks(int64_t T) { return static_cast<int>((T + 63) / 64); }
 
 struct GateArgs {
   int64_t T;
@@ -169,11 +172,16 @@ __device__ __forceinline__ int colsum8_column(int lane) {
 // (load_bias_smem) by the caller.
 template <int KM, int G, int W, class Fetch, class Sync>
 __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, int q, int grp,
-                                          int gtid, int64_t tile, const GateArgs& g,
+                                          int gtid, int64_t tile, bool half, const GateArgs& g,
                                           uint8_t* smem) {
   const int lane = gtid & 31;
-  const int row = q * 32 + lane;
-  const int64_t t0 = tile * kRouteBM;
+  // half tiles: 64 tokens whose rows fill both halves of the MMA operand, so quarters q
+  // and q+2 hold the same tokens and split their experts (2G column groups)
+  const int ntok = half ? 64 : 128;
+  const int row = half ? (q & 1) * 32 + lane : q * 32 + lane;
+  const int CG = half ? 2 * G : G;
+  const int cgrp = half ? grp * 2 + (q >> 1) : grp;
+  const int64_t t0 = tile * ntok;
   const int64_t t = t0 + row;
   const bool valid = t < g.T;
   const int E = g.E, k = g.k;
@@ -230,7 +238,7 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
   float thr = -INFINITY;  // the current (k+1)-th score: values below it cannot enter the list
   float m = -INFINITY, ssum = 0.0f;
 #pragma unroll 1
-  for (int cs = grp * W; cs < E; cs += W * G) {
+  for (int cs = cgrp * W; cs < E; cs += W * CG) {
     {
       float sc[W];
       scores(cs, sc);
@@ -271,22 +279,22 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
   }
 #pragma unroll
   for (int s2 = 0; s2 <= KM; ++s2) {
-    pv[(grp * 128 + row) * (KM + 1) + s2] = top.v[s2];
-    pi[(grp * 128 + row) * (KM + 1) + s2] = top.i[s2];
+    pv[(cgrp * ntok + row) * (KM + 1) + s2] = top.v[s2];
+    pi[(cgrp * ntok + row) * (KM + 1) + s2] = top.i[s2];
   }
-  pm[grp * 128 + row] = m;
-  ps[grp * 128 + row] = ssum;
+  pm[cgrp * ntok + row] = m;
+  ps[cgrp * ntok + row] = ssum;
   sync();
 
   // ---- merge the G partial results of each token (group 0) and write the outputs
-  if (grp == 0) {
+  if (cgrp == 0) {
 #pragma unroll 1
-    for (int g2 = 1; g2 < G; ++g2) {
+    for (int g2 = 1; g2 < CG; ++g2) {
 #pragma unroll
       for (int s2 = 0; s2 <= KM; ++s2)
         if (s2 <= k)
-          top.insert(pv[(g2 * 128 + row) * (KM + 1) + s2], pi[(g2 * 128 + row) * (KM + 1) + s2], k);
-      const float m2 = pm[g2 * 128 + row], s2v = ps[g2 * 128 + row];
+          top.insert(pv[(g2 * ntok + row) * (KM + 1) + s2], pi[(g2 * ntok + row) * (KM + 1) + s2], k);
+      const float m2 = pm[g2 * ntok + row], s2v = ps[g2 * ntok + row];
       if (m2 != -INFINITY) {
         const float nm = fmaxf(m, m2);
         ssum = (m == -INFINITY ? 0.0f : ssum * expf(m - nm)) + s2v * expf(m2 - nm);
@@ -349,7 +357,7 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
     myg[jj] = fgate[row * KM + jj];
   }
 #pragma unroll 1
-  for (int cs = grp * W; cs < E; cs += W * G) {
+  for (int cs = cgrp * W; cs < E; cs += W * CG) {
     {
       float gi[W], pl[W];
 #pragma unroll
@@ -406,8 +414,9 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
   sync();
   for (int e = gtid; e < E; e += 128 * G) {
     float si = 0.0f, sl = 0.0f;
-#pragma unroll
-    for (int qq = 0; qq < 4; ++qq) {
+    // half tiles: column e was summed by the quarter pair of its column group only
+    const int q0 = half ? 2 * (((e / W) % CG) & 1) : 0, q1 = half ? q0 + 2 : 4;
+    for (int qq = q0; qq < q1; ++qq) {
       si += qsum[(qq * 2 + 0) * E + e];
       sl += qsum[(qq * 2 + 1) * E + e];
     }
@@ -443,7 +452,8 @@ struct RouteTcArgs {
   int nb;         // 1, or 2 with W_noise
   int nbuf;       // TMEM accumulator buffers: 2, or 1 when 2 * nb * acc_cols > 512
   int stages;
-  int ntiles;     // ceil(T / 128)
+  int half;       // 1: 64-token tiles, each loaded into both halves of the MMA operand
+  int ntiles;     // ceil(T / 128), or ceil(T / 64) with half tiles
   int gate_off;   // byte offset of the gate scratch in shared memory
   int bar_off;    // byte offset of the barriers
   int* err;
@@ -522,7 +532,12 @@ __global__ void __launch_bounds__(64 + 128 * G)
           uint8_t* st = smem + stage * stage_bytes;
           const uint32_t fb = full0 + 8 * stage;
           mbar_arrive_expect_tx(fb, static_cast<uint32_t>(stage_bytes));
-          tma_load_2d(smem_u32(st), &tmX, fb, kb * rt::BK, L * kRouteBM);
+          if (a.half) {  // the same 64 token rows into operand rows 0-63 and 64-127
+            tma_load_2d(smem_u32(st), &tmX, fb, kb * rt::BK, L * 64);
+            tma_load_2d(smem_u32(st + rt::A_BYTES / 2), &tmX, fb, kb * rt::BK, L * 64);
+          } else {
+            tma_load_2d(smem_u32(st), &tmX, fb, kb * rt::BK, L * kRouteBM);
+          }
           tma_load_2d(smem_u32(st + rt::A_BYTES), &tmG, fb, kb * rt::BK, 0);
           if (a.nb == 2) tma_load_2d(smem_u32(st + rt::A_BYTES + b_bytes), &tmN, fb, kb * rt::BK, 0);
           armed |= 1u << stage;
@@ -625,7 +640,7 @@ __global__ void __launch_bounds__(64 + 128 * G)
             z[j] = __uint_as_float(w[j]);
           }
         };
-        gate_tile<KM, G, 16>(fetch, sync, q, grp, gtid, L, a.g, gsm);
+        gate_tile<KM, G, 16>(fetch, sync, q, grp, gtid, L, a.half != 0, a.g, gsm);
       } else {
         auto fetch = [&](int c, float (&l)[16], float (&z)[16]) {
           uint32_t v[16];
@@ -637,7 +652,7 @@ __global__ void __launch_bounds__(64 + 128 * G)
             z[j] = 0.0f;
           }
         };
-        gate_tile<KM, G, 16>(fetch, sync, q, grp, gtid, L, a.g, gsm);
+        gate_tile<KM, G, 16>(fetch, sync, q, grp, gtid, L, a.half != 0, a.g, gsm);
       }
       tc_fence_before();
       __syncwarp();
@@ -681,7 +696,7 @@ __global__ void __launch_bounds__(128, 1)
   load_bias_smem(g, gsmem, KM, 1, static_cast<int>(threadIdx.x), 128);
   __syncthreads();
   gate_tile<KM, 1, 16>(fetch, [] { __syncthreads(); }, warp, 0, static_cast<int>(threadIdx.x),
-                       static_cast<int64_t>(blockIdx.x), g, gsmem);
+                       static_cast<int64_t>(blockIdx.x), false, g, gsmem);
 }
 
 __global__ void finalize_importance_load_kernel(const float* __restrict__ partials, int nblocks,
@@ -744,7 +759,10 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   a.kblocks = p.d / rt::BK;
   a.nb = p.noisy ? 2 : 1;
   a.nbuf = 2 * a.nb * a.acc_cols <= 512 ? 2 : 1;
-  a.ntiles = route_blocks(p.T);
+  // half tiles when 128-token tiles would fill at most half of the SMs
+  const int full_tiles = static_cast<int>((p.T + kRouteBM - 1) / kRouteBM);
+  a.half = 2 * full_tiles <= c.num_sms ? 1 : 0;
+  a.ntiles = a.half ? static_cast<int>((p.T + 63) / 64) : full_tiles;
   const int km = k_bucket(p.k);
   const int scratch = gate_smem_bytes(km, rt::groups_for(km), p.E);
   const int stage_bytes = rt::A_BYTES + a.nb * a.e_pad * rt::BK * 2;
@@ -760,7 +778,8 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   const int smem = 1024 + a.bar_off + 8 * (2 * stages + 5) + 16;
 
   CUtensorMap tmX, tmG, tmN;
-  if (!make_tmap_bf16(&tmX, p.x, static_cast<uint64_t>(p.T), p.d, kRouteBM)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16(&tmX, p.x, static_cast<uint64_t>(p.T), p.d, a.half ? 64 : kRouteBM))
+    return cudaErrorInvalidValue;
   if (!make_tmap_bf16(&tmG, p.w_gate, static_cast<uint64_t>(p.E), p.d, a.e_pad)) return cudaErrorInvalidValue;
   if (p.noisy) {
     if (!make_tmap_bf16(&tmN, p.w_noise, static_cast<uint64_t>(p.E), p.d, a.e_pad)) return cudaErrorInvalidValue;
@@ -802,7 +821,7 @@ cudaError_t launch_route_f32(const RouteProblem& p, const LaunchCtx& c) {
     if (e != cudaSuccess) return e;
   }
   const GateArgs g = gate_args(p);
-  const int nblocks = route_blocks(p.T);
+  const int nblocks = static_cast<int>((p.T + kRouteBM - 1) / kRouteBM);
   switch (k_bucket(p.k)) {
     case 1: e = launch_gate_f32<1>(p, g, nblocks, c); break;
     case 2: e = launch_gate_f32<2>(p, g, nblocks, c); break;
