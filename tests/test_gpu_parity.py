@@ -41,6 +41,8 @@ SMALL = {
     "E8_bf16_pad": Workload("e8", T=500, d_model=64, d_ff=64, E=8, k=2),
     "f16_hidden_multitile": Workload("h16", T=3000, d_model=192, d_ff=384, E=6, k=2, act="gelu",
                                      hidden_f16=True, capacity_factor=0.9),
+    # k = 8: the router's longest top lists (two column groups of gate warps)
+    "k8_E32": Workload("k8", T=1500, d_model=128, d_ff=128, E=32, k=8, act="relu"),
 }
 
 
@@ -134,6 +136,11 @@ FULL = {name: W[name] for name in ("switch", "noisy", "gshard", "zipf")}
 # (1024 per block, one block per SM): moe_permute takes its three-kernel path here.
 FULL["three_kernel_permute_T200k"] = Workload("t200k", T=200_000, d_model=64, d_ff=128, E=8, k=1,
                                               renorm=False, capacity_factor=1.0, act="relu")
+# Router on 128-token tiles with several tiles per CTA (more than 74 tiles): noisy gating
+# with its two products in one TMEM buffer, and k = 8 with two gate column groups.
+FULL["noisy_full_tiles_T20000"] = W["noisy"].scaled(T=20_000)
+FULL["k8_full_tiles_T12000"] = Workload("k8f", T=12_000, d_model=256, d_ff=256, E=64, k=8,
+                                        act="gelu", capacity_factor=1.5)
 
 
 @pytest.mark.parametrize("name", list(FULL))
