@@ -230,3 +230,31 @@ def test_permute_launch_path(name, launches):
     assert moe.last_launch_count() == launches
     assert moe.moe_get_error(ws) == 0
     assert o["counts"].tolist() == torch.bincount(idx.view(-1).long(), minlength=w.E).tolist()
+
+
+def test_forward_replays_from_a_cuda_graph():
+    """moe_forward captured into a CUDA graph (its kernels and their programmatic launch
+    edges) and replayed gives the eager result bit for bit, also after the input changes
+    in place."""
+    import sparsely_gated_mixture_moe_b200 as moe
+    w = W["switch"].scaled(T=2048)
+    cfg = H.config_of(w)
+    dev = H.to_device(workloads.make_inputs(w))
+    layer = moe.MoELayer(cfg, {kk: v for kk, v in dev.items() if kk not in ("x", "noise")})
+    x = dev["x"].clone()
+    y1 = layer.forward(x).clone()
+    x2 = workloads.make_inputs(w.scaled(T=2048, seed=5))["x"].cuda()
+    layer.forward(x2)
+    y2 = layer.y.clone()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+        layer.forward(x)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(layer.y, y1)
+    x.copy_(x2)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(layer.y, y2)
+    assert moe.moe_get_error(layer.ws) == 0
