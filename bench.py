@@ -371,13 +371,13 @@ def run_gpu(args, w):
         raise RuntimeError("device error word %d after the timed steps" % err)
 
     # ---- the same step replayed from a CUDA graph (informational): no host work and no
-    # phase events between the kernels, so every launch edge is programmatic
-    graph_info = None
+    # phase events between the kernels, so every launch edge is programmatic.  Every rank
+    # takes the same collective step whether or not its capture worked.
+    graph_err, g_local, n_graph = None, float("inf"), max(3, min(args.steps, 200))
     try:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             step()
-        n_graph = max(3, min(args.steps, 200))
         g_ms = []
         for i in range(n_graph + 3):
             flush_l2(i)
@@ -388,15 +388,19 @@ def run_gpu(args, w):
             b.synchronize()
             if i >= 3:
                 g_ms.append(a.elapsed_time(b))
-        g_mean = max_over_ranks(float(np.mean(g_ms)), dev)
-        graph_info = {"value": T * world / (g_mean * 1e-3), "unit": "tokens/s", "ms_per_step": g_mean,
-                      "steps": n_graph, "note": "one step (route, permute, expert FFN, combine) "
-                      "captured once and replayed; L2 flushed before each replay"}
         del graph
         if moe.moe_get_error(ws):
             raise RuntimeError("device error word set after the graph replays")
+        g_local = float(np.mean(g_ms))
     except RuntimeError as ex:
-        graph_info = {"unavailable": str(ex).splitlines()[0][:200]}
+        graph_err = str(ex).splitlines()[0][:200]
+    g_mean = max_over_ranks(g_local, dev)
+    if graph_err is not None or not np.isfinite(g_mean):
+        graph_info = {"unavailable": graph_err or "capture failed on another rank"}
+    else:
+        graph_info = {"value": T * world / (g_mean * 1e-3), "unit": "tokens/s", "ms_per_step": g_mean,
+                      "steps": n_graph, "note": "one step (route, permute, expert FFN, combine) "
+                      "captured once and replayed; L2 flushed before each replay"}
 
     # ---- end to end through the public layer call, host buffers in pinned memory.
     # Every step copies its x (and noise) in from pinned host memory and its y out.  The
