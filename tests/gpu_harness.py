@@ -185,7 +185,7 @@ def gpu_hidden(w, g, rows):
 def check_ffn(w, inp, g, n, report, rows=None):
     """y_perm and h of the GPU against the oracle's experts on the GPU's own x_perm.
 
-    h is an intermediate stored in bf16 (or as a bf16 pair): each element must be the
+    h is an intermediate stored in bf16 (or fp16): each element must be the
     oracle's value up to that storage's rounding, |dh| <= u |h| + 1e-4 rms(h), with
     u = 2^-8 for bf16 and 2^-11 for fp16 (fp32 path: 1e-5 of rms)."""
     off = g["offsets"].numpy()
