@@ -262,6 +262,15 @@ moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_idx, c
                                int32_t* counts, int32_t* offsets, int32_t* perm_src,
                                int32_t* slot_pos, void* x_perm, moe_stream_t stream);
 
+/* Diagnostic: runs the permutation's grid barrier on two blocks with a target that no
+ * block ever reaches, so every block's bounded wait expires: after about one second
+ * each block sets MOE_DEVERR_TIMEOUT in the workspace's error word and returns, and the
+ * last block out resets the barrier counters, as a permutation that lost a block
+ * would.  A test reads the error word (moe_get_error) and then runs a normal call on
+ * the same workspace.  ws: a workspace as for the step calls (at least 16 bytes).  No
+ * counterpart on the pages. */
+moe_status moe_wait_timeout_check(void* ws, moe_stream_t stream);
+
 /* Diagnostic: evaluates, for n fp32 inputs x, the erf approximation the GELU epilogue of
  * the tensor-core FFN uses (Abramowitz & Stegun formula 7.1.26, |error| <= 1.5e-7; with its fast fp32 evaluation
  * within 1e-6 of erff) into

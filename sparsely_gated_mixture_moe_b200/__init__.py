@@ -45,6 +45,7 @@ def _load():
         "moe_bf16_to_f16": (ctypes.c_int, [P, P, ctypes.c_int64, P, P]),
         "moe_permute_noalloc": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
         "moe_erf_check": (ctypes.c_int, [P, P, P, ctypes.c_int64, P]),
+        "moe_wait_timeout_check": (ctypes.c_int, [P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

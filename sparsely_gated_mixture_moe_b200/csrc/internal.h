@@ -86,6 +86,7 @@ struct PermuteProblem {
 int64_t permute_blocks(int64_t n);
 int64_t permute_count_chunks(int64_t n);
 cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c);
+cudaError_t launch_wait_timeout_check(int32_t* sync, int* err, const LaunchCtx& c);
 
 // ---- expert FFN ------------------------------------------------------------------
 struct FfnProblem {

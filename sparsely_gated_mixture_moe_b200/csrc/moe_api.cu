@@ -440,6 +440,15 @@ moe_status moe_bf16_to_f16(const void* src, void* dst, int64_t n, int32_t* n_ine
   return ctx.finish(launch_bf16_to_f16(src, dst, n, n_inexact, ctx.lc));
 }
 
+moe_status moe_wait_timeout_check(void* ws, moe_stream_t stream) {
+  if (!ws || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  Ctx ctx(ws, stream);
+  if (!ctx.ok) return MOE_ERR_CUDA;
+  // the barrier counters are words 2 and 3 of the error block, as for moe_permute
+  int32_t* sync = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + 8);
+  return ctx.finish(launch_wait_timeout_check(sync, ctx.lc.err, ctx.lc));
+}
+
 int32_t moe_last_launch_count(void) { return g_last_launches; }
 
 }  // extern "C"

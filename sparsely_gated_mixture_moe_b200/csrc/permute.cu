@@ -416,6 +416,30 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
   }
 }
 
+// The grid barrier with a target no block reaches (one more arrival than blocks): every
+// block's wait expires, sets the timeout bit and returns; the last block out resets the
+// counters.  Used by moe_wait_timeout_check.
+__global__ void barrier_timeout_check_kernel(int32_t* sync, int* err) {
+  __shared__ int s_abort;
+  grid_dep_wait();
+  grid_dep_launch();
+  if (threadIdx.x == 0) s_abort = 0;
+  __syncthreads();
+  grid_barrier(sync, static_cast<int>(gridDim.x) + 1, err, &s_abort);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(sync + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      atomicExch(sync, 0);
+      atomicExch(sync + 1, 0);
+    }
+  }
+}
+
+cudaError_t launch_wait_timeout_check(int32_t* sync, int* err, const LaunchCtx& c) {
+  return launch_kernel(barrier_timeout_check_kernel, dim3(2), dim3(32), 0, c, sync, err);
+}
+
 // Chunking for the one-launch path: returns the number of chunks (= blocks) and sets
 // *chunk, or returns 0 when the chunks would exceed 1024 assignments or the blocks would
 // not all fit on the GPU at once.

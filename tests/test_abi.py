@@ -116,6 +116,8 @@ def test_other_steps_validation():
     assert moe.lib.moe_forward(c, P, P, None, None, None, P, P, None, P, P, P, None, None, None,
                                P, None) == 1
     assert moe.lib.moe_get_error(None, None, None) == 1
+    assert moe.lib.moe_wait_timeout_check(None, None) == 1
+    assert moe.lib.moe_wait_timeout_check(FAKE_ODD, None) == 1
 
 
 def test_workspace_sizes():

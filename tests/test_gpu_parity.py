@@ -258,3 +258,37 @@ def test_forward_replays_from_a_cuda_graph():
     torch.cuda.synchronize()
     assert torch.equal(layer.y, y2)
     assert moe.moe_get_error(layer.ws) == 0
+
+
+def test_bounded_wait_expires_and_reports_timeout():
+    """A grid barrier that can never complete (failure detection without a fault): each
+    block's wait gives up after its limit, the timeout bit reaches the host through the
+    error word, and the same workspace then serves a normal permutation exactly (the
+    barrier counters were reset and the context is still usable)."""
+    import ctypes
+    import sparsely_gated_mixture_moe_b200 as moe
+    from oracle import moe_oracle as orc
+    w = W["switch"].scaled(T=4096)
+    cfg = H.config_of(w)
+    ws = moe.workspace(cfg)
+    assert moe.lib.moe_wait_timeout_check(ctypes.c_void_p(ws.data_ptr()), None) == 0
+    assert moe.moe_get_error(ws) == 8          # MOE_DEVERR_TIMEOUT, and cleared
+    assert moe.moe_get_error(ws) == 0
+    dev = H.to_device(workloads.make_inputs(w))
+    gen = torch.Generator().manual_seed(3)
+    idx = torch.randint(0, w.E, (w.T, w.k), generator=gen, dtype=torch.int32)
+    n = w.T * w.k
+    o = {key: torch.empty(size, dtype=torch.int32, device="cuda")
+         for key, size in (("counts", w.E), ("offsets", w.E + 1), ("perm_src", n), ("slot_pos", n))}
+    x_perm = torch.empty(n, w.d_model, dtype=w.torch_dtype, device="cuda")
+    moe.moe_permute(cfg, idx.cuda(), dev["x"], o["counts"], o["offsets"], o["perm_src"],
+                    o["slot_pos"], x_perm, ws)
+    assert moe.last_launch_count() == 1
+    assert moe.moe_get_error(ws) == 0
+    C = orc.capacity(w.capacity_factor, w.T, w.k, w.E)
+    counts, offsets, perm_src, slot_pos = orc.dispatch(idx.long().numpy(), w.E, C)
+    assert o["counts"].cpu().tolist() == counts.tolist()
+    assert o["offsets"].cpu().tolist() == offsets.tolist()
+    kept = int(offsets[-1])
+    assert o["perm_src"][:kept].cpu().tolist() == perm_src.tolist()
+    assert o["slot_pos"].cpu().tolist() == slot_pos.tolist()
