@@ -10,10 +10,16 @@ on one device), the step time is the max over ranks, and the value is the tokens
 ranks per second.
 
 Timing: W untimed warm-up steps; then K steps, each preceded (outside its events) by a
-write of a 256 MB buffer that flushes the 126 MB L2; CUDA events on the launching stream
-bracket each step and each step call.  The dominant kernel is the tcgen05 grouped GEMM
-(two launches per step: up- and down-projection); its roofline uses the algorithmic
-bytes/FLOPs of those two launches over the event time of the expert-FFN call.
+write and read-back of a 256 MB buffer that flushes the 126 MB L2; CUDA events on the
+launching stream bracket each step and each step call.  The dominant kernel is the
+tcgen05 grouped GEMM (two launches per step: up- and down-projection); its roofline uses
+the algorithmic bytes/FLOPs of those two launches over the event time of the expert-FFN
+call, and its DRAM traffic per launch comes from the committed ncu summary while the
+kernel sources match it.  Also reported: the same step captured into a CUDA graph and
+replayed (`graph`), and the end-to-end throughput through MoELayer.forward with every
+step's inputs copied in from pinned host memory and its output copied out, consecutive
+steps pipelined over H2D / compute / D2H streams (`e2e`, with the serial per-step
+latency beside it).
 
 --impl reference times the CPU oracle on this machine's host cores instead (a bounded
 sample of the same workload per step) and prints the same JSON line with impl=reference.

@@ -7,25 +7,27 @@
 //                   G = Softmax(KeepTopK(H, k))
 // Ties go to the lowest expert index (the running top list ranks equal scores by
 // expert index, so lists built over disjoint expert sets merge exactly).  For noisy
-// gating the kernel also forms, per block of 128 tokens, the partial sums of
-// Importance = sum_t G(x_t) and
+// gating (or when Importance is asked for) the kernel also forms, per token tile, the
+// partial sums of Importance = sum_t G(x_t) and
 // Load_i = sum_t Phi((l_i - kth_excluding(H, k, i)) / Softplus((x.W_noise)_i))
 // ("Load-Balancing-Losses"); a second kernel adds the partials in a fixed order, so
 // results are bit-reproducible (no floating-point atomics).
 //
-// bf16: one CTA per 128 tokens, with G groups of 4 warps (G = 4, or 2 when k > 4).  Warp
-// 0 streams x tiles [128 x 64] and W_g (and W_noise) tiles [E_pad x 64] with TMA into a
-// shared-memory ring; one thread of warp 1 issues tcgen05.mma (M=128, N=E_pad) into
-// TMEM.  Then every thread owns one token row of its warp's TMEM lane quarter and a
-// disjoint set of expert columns (32-column slices, group g taking slices g, g+G, ...),
-// read 8 at a time with tcgen05.ld.  Pass 1 keeps a running top-(k+1) list and the
-// maximum in registers; a group of 8 scores whose maximum is below the current
-// (k+1)-th score skips the insertion (the common case once the list fills).  With the
-// Switch gate (softmax over all experts) a second sweep adds exp(score - max).  Group 0
-// merges the G partial lists and sums through shared memory and writes the outputs.
-// The logits never touch HBM.
-// fp32: the logits come from the SIMT product into the workspace and the same gate code
-// reads them back (one token per thread, G = 1).
+// bf16 (route_tc_kernel): persistent over token tiles, warp-specialised.  Warp 0 streams
+// x tiles [128 x 64] and W_g (and W_noise) tiles [E_pad x 64] with TMA into a ring of
+// shared-memory stages; one thread of warp 1 issues tcgen05.mma (M=128, N=E_pad) into
+// one of two TMEM accumulator buffers (one when noisy gating's two products fill TMEM);
+// 4*G gate warps (G = 4, or 2 when k > 4) take a finished buffer, run gate_tile and hand
+// it back, so one tile's gate overlaps the next tile's loads.  Tiles are 128 tokens, or
+// 64 tokens loaded into both halves of the MMA operand when 128-token tiles would fill
+// at most half of the SMs.  In gate_tile each thread owns one token row of its warp's
+// TMEM lane quarter and 16-column slices of experts interleaved across the column
+// groups, read with one tcgen05.ld + wait per slice; it keeps a running top-(k+1) list
+// (branch-free insertion) and the running softmax in registers, then one column group
+// merges the partial lists through shared memory and writes the outputs.  The logits
+// never touch HBM.
+// fp32 (gate_f32_kernel): the logits come from the SIMT product into the workspace and
+// the same gate code reads them back (one token per thread, G = 1).
 #include "common.cuh"
 #include "internal.h"
 
