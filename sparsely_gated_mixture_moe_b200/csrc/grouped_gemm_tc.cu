@@ -420,8 +420,7 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
   const int64_t max_tiles = (rows_cap / gg::BM + E) * static_cast<int64_t>(a.n_tiles);
   const int grid = static_cast<int>(max_tiles < c.num_sms ? max_tiles : c.num_sms);
   if (grid <= 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(gg::grouped_gemm_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, gg::SMEM_BYTES);
+  cudaError_t e = ensure_smem_limit(gg::grouped_gemm_tc_kernel, gg::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   return launch_kernel(gg::grouped_gemm_tc_kernel, dim3(grid), dim3(gg::THREADS), gg::SMEM_BYTES, c,
                        tmA, tmB, a);

@@ -8,6 +8,10 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "moe.h"
 
 namespace moe {
@@ -18,6 +22,25 @@ struct LaunchCtx {
   int* err;       // device error word
   int* launches;  // host counter
 };
+
+// Raises a kernel's dynamic shared-memory limit to at least `bytes` on the current device,
+// calling cudaFuncSetAttribute only the first time a larger limit is needed there (the
+// attribute outlives the call; repeating it on every launch only costs host time).
+template <typename... KArgs>
+cudaError_t ensure_smem_limit(void (*kernel)(KArgs...), int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, int> limit;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(dev, reinterpret_cast<const void*>(kernel));
+  const auto it = limit.find(key);
+  if (it != limit.end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) limit[key] = bytes;
+  return e;
+}
 
 // Every kernel of the library is launched with programmatic stream serialisation: the
 // launch may start while the previous kernel on the stream is still running, and the

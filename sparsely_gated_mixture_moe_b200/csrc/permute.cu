@@ -446,8 +446,7 @@ cudaError_t launch_wait_timeout_check(int32_t* sync, int* err, const LaunchCtx& 
 static int fused_chunks(const PermuteProblem& p, const LaunchCtx& c, size_t smem, int* chunk) {
   if (p.sync == nullptr) return 0;
   if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(perm_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+      ensure_smem_limit(perm_fused_kernel, static_cast<int>(smem)) != cudaSuccess)
     return 0;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, perm_fused_kernel, pf::THREADS,
@@ -480,8 +479,7 @@ cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c) {
   }
   const size_t cs_smem = count_scan_smem(p.E);
   if (cs_smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(perm_count_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(cs_smem));
+    e = ensure_smem_limit(perm_count_scan_kernel, static_cast<int>(cs_smem));
     if (e != cudaSuccess) return e;
   }
   e = launch_kernel(perm_count_scan_kernel, dim3(static_cast<unsigned>(nblk)), dim3(pm::THREADS),
@@ -490,8 +488,7 @@ cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c) {
   if (e != cudaSuccess) return e;
   const size_t wsmem = static_cast<size_t>(pm::WARPS) * p.E * 4;
   if (wsmem > 48 * 1024) {
-    e = cudaFuncSetAttribute(perm_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(wsmem));
+    e = ensure_smem_limit(perm_scatter_kernel, static_cast<int>(wsmem));
     if (e != cudaSuccess) return e;
   }
   e = launch_kernel(perm_scatter_kernel, dim3(static_cast<unsigned>(nblk)), dim3(pm::THREADS),

@@ -746,7 +746,7 @@ template <int KM>
 static cudaError_t launch_route_tc(const CUtensorMap& tmX, const CUtensorMap& tmG,
                                    const CUtensorMap& tmN, const RouteTcArgs& a, int smem,
                                    int grid, const LaunchCtx& c) {
-  cudaError_t e = cudaFuncSetAttribute(route_tc_kernel<KM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = ensure_smem_limit(route_tc_kernel<KM>, smem);
   if (e != cudaSuccess) return e;
   return launch_kernel(route_tc_kernel<KM>, dim3(grid), dim3(64 + 128 * rt::groups_for(KM)), smem,
                        c, tmX, tmG, tmN, a);
@@ -805,7 +805,7 @@ static cudaError_t launch_gate_f32(const RouteProblem& p, const GateArgs& g, int
                                    const LaunchCtx& c) {
   const int smem = gate_smem_bytes(KM, 1, p.E);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(gate_f32_kernel<KM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = ensure_smem_limit(gate_f32_kernel<KM>, smem);
     if (e != cudaSuccess) return e;
   }
   return launch_kernel(gate_f32_kernel<KM>, dim3(nblocks), dim3(128), smem, c,
