@@ -10,7 +10,7 @@ Loss whose gradients are returned (dy is the gradient of the loss with respect t
 [SGMoE "Load-Balancing-Losses": the auxiliary losses are a scaling factor times the
 squared coefficient of variation of Importance and of Load].
 
-Readings where the pages are silent (each is also listed in the design doc):
+Readings where the pages are silent:
   * The top-k choice and the capacity drop are piecewise constant: no gradient flows
     through which experts are chosen or kept, only through the values.
   * The noise draws are inputs, not parameters.

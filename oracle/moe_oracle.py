@@ -17,7 +17,7 @@ Sources (pages by title, then section):
   [Setups] "moe paper models" page, Table 2 (TOP-K and capacity columns: capacity
            factors 1/1.5/2x, 1.25, 2).
 
-Readings where the pages are silent or garbled (each is also listed in the design doc):
+Readings where the pages are silent or garbled:
   * KeepTopK keeps v_i when v_i is among the k largest entries and sets the rest to -inf.
   * Ties in the top-k choice go to the lowest expert index.
   * The top-k decision is taken on the scores rounded to fp32 (the kernel's precision);
