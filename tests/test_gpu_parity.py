@@ -43,6 +43,11 @@ SMALL = {
                                      hidden_f16=True, capacity_factor=0.9),
     # k = 8: the router's longest top lists (two column groups of gate warps)
     "k8_E32": Workload("k8", T=1500, d_model=128, d_ff=128, E=32, k=8, act="relu"),
+    # the largest supported expert counts: fp32 E = 1024 (the one-launch permutation's
+    # biggest shared-memory footprint) and bf16 E = 256 with k = 8
+    "f32_E1024": Workload("e1024", T=2048, d_model=32, d_ff=32, E=1024, k=2, dtype="f32"),
+    "E256_k8": Workload("e256k8", T=1200, d_model=128, d_ff=128, E=256, k=8, act="gelu",
+                        capacity_factor=2.0),
 }
 
 
