@@ -48,6 +48,9 @@ SMALL = {
     "f32_E1024": Workload("e1024", T=2048, d_model=32, d_ff=32, E=1024, k=2, dtype="f32"),
     "E256_k8": Workload("e256k8", T=1200, d_model=128, d_ff=128, E=256, k=8, act="gelu",
                         capacity_factor=2.0),
+    # noisy gating with capacity drops (Importance still sums the gates before the drop)
+    "noisy_capacity": Workload("nzc", T=900, d_model=128, d_ff=128, E=16, k=2,
+                               gating="noisy_topk", capacity_factor=0.5),
 }
 
 
@@ -146,6 +149,9 @@ FULL["three_kernel_permute_T200k"] = Workload("t200k", T=200_000, d_model=64, d_
 FULL["noisy_full_tiles_T20000"] = W["noisy"].scaled(T=20_000)
 FULL["k8_full_tiles_T12000"] = Workload("k8f", T=12_000, d_model=256, d_ff=256, E=64, k=8,
                                         act="gelu", capacity_factor=1.5)
+# just past the half-tile threshold (75 tiles of 128 > 148 / 2): 128-token tiles with a
+# ragged last tile
+FULL["noisy_full_tiles_ragged_T9473"] = W["noisy"].scaled(T=9_473)
 
 
 @pytest.mark.parametrize("name", list(FULL))
