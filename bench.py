@@ -1,13 +1,15 @@
 """Benchmark of the sparsely-gated MoE layer forward on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload switch] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload zipf] [--impl reference]
 
 One step is one pass of the whole layer (route, permute, expert FFN, combine) over one
-batch of synthetic tokens.  Default workload: the Switch-style top-1 layer (T=16384,
-d_model=768, d_ff=3072, E=128, capacity factor 1.25, GELU, bf16).  Under torchrun every
-rank runs an independent replica on its own GPU (the layer forward has no exchange step
-on one device), the step time is the max over ranks, and the value is the tokens of all
-ranks per second.
+batch of synthetic tokens.  The headline workload (default) is the largest single-GPU
+one, the skewed dropless top-2 layer (T=65536, d_model=1024, d_ff=4096, E=16, GELU,
+bf16, Zipf(1.2) expert load).  The same run also times every other workload (tiny fp32,
+Switch top-1, noisy top-4, GShard top-2) with the same step and reports them under
+`per_config`.  Under torchrun every rank runs an independent replica on its own GPU (the
+layer forward has no exchange step on one device), the step time is the max over ranks,
+and the value is the tokens of all ranks per second.
 
 Timing: W untimed warm-up steps; then K steps, each preceded (outside its events) by a
 write and read-back of a 256 MB buffer that flushes the 126 MB L2; CUDA events on the
@@ -15,14 +17,16 @@ launching stream bracket each step and each step call.  The dominant kernel is t
 tcgen05 grouped GEMM (two launches per step: up- and down-projection); its roofline uses
 the algorithmic bytes/FLOPs of those two launches over the event time of the expert-FFN
 call, and its DRAM traffic per launch comes from the committed ncu summary while the
-kernel sources match it.  Also reported: the same step captured into a CUDA graph and
-replayed (`graph`), and the end-to-end throughput through MoELayer.forward with every
-step's inputs copied in from pinned host memory and its output copied out, consecutive
-steps pipelined over H2D / compute / D2H streams (`e2e`, with the serial per-step
-latency beside it).
+kernel sources match it.  Also reported for the headline workload: the same step
+captured into a CUDA graph and replayed (`graph`), and the end-to-end throughput through
+MoELayer.forward with every step's inputs copied in from pinned host memory and its
+output copied out, consecutive steps pipelined over H2D / compute / D2H streams (`e2e`,
+with the serial per-step latency beside it).
 
---impl reference times the CPU oracle on this machine's host cores instead (a bounded
-sample of the same workload per step) and prints the same JSON line with impl=reference.
+The CPU oracle (NumPy fp64) is timed on a fixed sample per workload: each oracle step
+routes and dispatches all T tokens (so capacity is the workload's own) and runs the
+expert FFN and combine for S fixed tokens (every (T/S)-th); its rate counts those S
+tokens.  `cpu_baseline` and `--impl reference` run exactly this step.
 """
 from __future__ import annotations
 
@@ -183,14 +187,23 @@ def algorithmic(w: workloads.Workload, n_kept: int, counts_kept, fused=False):
 
 # ------------------------------------------------------------------------ CPU oracle arm
 
-def oracle_sample(w, inp, n_tokens):
-    """The oracle's forward over a contiguous sample of n_tokens tokens (routing and
-    capacity computed over that sample).  Returns seconds."""
+# Tokens whose expert FFN and combine each oracle step evaluates (every (T/S)-th token);
+# routing and dispatch always cover all T tokens.  Sized so that one step takes about one
+# to four seconds on a 16-core host.
+ORACLE_SAMPLE = {"tiny": 512, "switch": 128, "noisy": 32, "gshard": 32, "zipf": 32}
+
+
+def oracle_rows(w):
+    S = min(w.T, ORACLE_SAMPLE.get(w.name, 64))
+    return [i * w.T // S for i in range(S)]
+
+
+def oracle_step(w, inp, rows):
+    """One oracle step: route and dispatch all T tokens, expert FFN and combine for
+    ``rows``.  Returns seconds of wall time."""
     from oracle import moe_oracle as orc
-    sub = {k: (v[:n_tokens] if k in ("x", "noise") else v) for k, v in inp.items()}
-    ws = w.scaled(T=n_tokens)
     t0 = time.perf_counter()
-    orc.moe_forward(sub, ws)
+    orc.moe_forward_rows(inp, w, rows)
     return time.perf_counter() - t0
 
 
@@ -204,21 +217,26 @@ def cpu_cores():
     return n, blas
 
 
-def sample_size(w, inp, seconds):
-    """Tokens of the workload the oracle forwards in about `seconds` (>= 16)."""
-    n0 = min(w.T, 256)
-    dt = oracle_sample(w, inp, n0)
-    return int(max(16, min(w.T, n0 * seconds / max(dt, 1e-4))))
-
-
-def cpu_baseline(w, inp, budget_s=15.0):
-    """Time the oracle as it stands on a token sample sized to about budget_s."""
-    n = sample_size(w, inp, budget_s)
-    dt = oracle_sample(w, inp, n)
+def sample_text(w, rows):
     cores, blas = cpu_cores()
-    return {"value": n / dt, "unit": "tokens/s", "cores": blas, "kind": "oracle",
-            "sample": "%d of the workload's %d tokens, one forward pass (NumPy fp64; %d host "
-                      "cores visible, %d BLAS threads)" % (n, w.T, cores, blas)}
+    return ("each step: routing and capacity dispatch of all %d tokens, expert FFN and combine "
+            "for %d fixed tokens (every %d-th); the rate counts those %d tokens (NumPy fp64; "
+            "%d host cores visible, %d BLAS threads)" % (w.T, len(rows), w.T // len(rows),
+                                                         len(rows), cores, blas))
+
+
+def cpu_baseline(w, inp, budget_s=6.0):
+    """The oracle as it stands, timed on its fixed sample: one untimed step, then steps
+    until about budget_s seconds have been timed (at least two)."""
+    rows = oracle_rows(w)
+    oracle_step(w, inp, rows)
+    times = []
+    while len(times) < 2 or sum(times) < budget_s:
+        times.append(oracle_step(w, inp, rows))
+    _, blas = cpu_cores()
+    mean = sum(times) / len(times)
+    return {"value": len(rows) / mean, "unit": "tokens/s", "cores": blas, "kind": "oracle",
+            "ms_per_step": mean * 1e3, "steps": len(times), "sample": sample_text(w, rows)}
 
 
 def run_reference(args, w):
@@ -226,23 +244,21 @@ def run_reference(args, w):
     if rank != 0:
         return
     inp = workloads.make_inputs(w)
-    per_step = max(0.05, 120.0 / (args.steps + args.warmup))
-    n = sample_size(w, inp, per_step)
+    rows = oracle_rows(w)
     for _ in range(args.warmup):
-        oracle_sample(w, inp, n)
-    times = [oracle_sample(w, inp, n) for _ in range(args.steps)]
-    per_tok = sum(times) / (len(times) * n)
-    value = 1.0 / per_tok
-    cores, blas = cpu_cores()
+        oracle_step(w, inp, rows)
+    times = [oracle_step(w, inp, rows) for _ in range(args.steps)]
+    mean = sum(times) / len(times)
+    value = len(rows) / mean
+    _, blas = cpu_cores()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": per_tok * w.T * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": mean * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_json(w),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas, "kind": "oracle",
-                         "sample": "each step: %d of the workload's %d tokens, one forward pass "
-                                   "(ms_per_step scaled to all tokens)" % (n, w.T)},
+                         "sample": sample_text(w, rows)},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -250,10 +266,11 @@ def run_reference(args, w):
 
 
 def config_json(w):
-    c = {"workload": "%s: T=%d d_model=%d d_ff=%d E=%d k=%d gating=%s%s cf=%s act=%s %s" % (
+    c = {"workload": "%s: T=%d d_model=%d d_ff=%d E=%d k=%d gating=%s%s cf=%s act=%s %s%s" % (
         w.name, w.T, w.d_model, w.d_ff, w.E, w.k, w.gating,
         "" if w.gating == "noisy_topk" else ("(renorm)" if w.renorm else "(full-softmax gate)"),
-        w.capacity_factor, w.act, w.dtype),
+        w.capacity_factor, w.act, w.dtype,
+        "" if w.zipf_s is None else " zipf_s=%s" % w.zipf_s),
         "T": w.T, "d_model": w.d_model, "d_ff": w.d_ff, "E": w.E, "k": w.k,
         "capacity_factor": w.capacity_factor, "hidden_f16": w.hidden_f16,
         "l2": "flushed before every timed step (256 MB written, then read back, outside the events)",
@@ -263,130 +280,169 @@ def config_json(w):
 
 # ------------------------------------------------------------------------------ GPU arm
 
-def run_gpu(args, w):
-    import torch.distributed as dist
-    import sparsely_gated_mixture_moe_b200 as moe
+class LayerBench:
+    """Device inputs, outputs and workspace of one workload, and its timed step."""
 
-    rank, local_rank, world = dist_env()
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    if world > 1:
-        dist.init_process_group("nccl", device_id=dev,
-                                timeout=__import__("datetime").timedelta(seconds=120))
+    def __init__(self, moe, w, dev):
+        self.moe, self.w, self.dev = moe, w, dev
+        self.inp = workloads.make_inputs(w)
+        d = {k: v.to(dev) for k, v in self.inp.items()}
+        self.cfg = moe.make_config(w.T, w.d_model, w.d_ff, w.E, w.k, gating=w.gating,
+                                   renorm=w.renorm, capacity_factor=w.capacity_factor, act=w.act,
+                                   dtype=w.dtype, hidden_f16=w.hidden_f16)
+        self.d = moe.prepare_weights(self.cfg, d)  # fp16 w2 for fp16 hidden (exact re-encoding)
+        T, k, E, dm, f = w.T, w.k, w.E, w.d_model, w.d_ff
+        self.o = o = dict(
+            idx=torch.empty(T, k, dtype=torch.int32, device=dev),
+            gate=torch.empty(T, k, dtype=torch.float32, device=dev),
+            near=torch.empty(T, dtype=torch.uint8, device=dev),
+            counts=torch.empty(E, dtype=torch.int32, device=dev),
+            offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+            perm_src=torch.empty(T * k, dtype=torch.int32, device=dev),
+            slot_pos=torch.empty(T * k, dtype=torch.int32, device=dev),
+            x_perm=torch.empty(T * k, dm, dtype=w.torch_dtype, device=dev),
+            h=torch.empty(T * k, f, dtype=torch.float16 if w.hidden_f16 else w.torch_dtype,
+                          device=dev),
+            y_perm=torch.empty(T * k, dm, dtype=torch.float32, device=dev),
+            y=torch.empty(T, dm, dtype=torch.float32, device=dev))
+        self.noisy = w.gating == "noisy_topk"
+        o["importance"] = torch.empty(E, dtype=torch.float32, device=dev) if self.noisy else None
+        o["load"] = torch.empty(E, dtype=torch.float32, device=dev) if self.noisy and k < E else None
+        self.ws = moe.workspace(self.cfg, dev)
+        self.fused = moe.fused_combine(self.cfg)
+        self.stream = torch.cuda.current_stream(dev)
+        self.launches = 0
 
-    inp = workloads.make_inputs(w)
-    d = {k: v.to(dev) for k, v in inp.items()}
-    cfg = moe.make_config(w.T, w.d_model, w.d_ff, w.E, w.k, gating=w.gating, renorm=w.renorm,
-                          capacity_factor=w.capacity_factor, act=w.act, dtype=w.dtype,
-                          hidden_f16=w.hidden_f16)
-    d = moe.prepare_weights(cfg, d)     # fp16 w2 for fp16 hidden activations (exact re-encoding)
-    T, k, E, dm, f = w.T, w.k, w.E, w.d_model, w.d_ff
-    o = dict(
-        idx=torch.empty(T, k, dtype=torch.int32, device=dev),
-        gate=torch.empty(T, k, dtype=torch.float32, device=dev),
-        near=torch.empty(T, dtype=torch.uint8, device=dev),
-        counts=torch.empty(E, dtype=torch.int32, device=dev),
-        offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
-        perm_src=torch.empty(T * k, dtype=torch.int32, device=dev),
-        slot_pos=torch.empty(T * k, dtype=torch.int32, device=dev),
-        x_perm=torch.empty(T * k, dm, dtype=w.torch_dtype, device=dev),
-        h=torch.empty(T * k, f, dtype=torch.float16 if w.hidden_f16 else w.torch_dtype, device=dev),
-        y_perm=torch.empty(T * k, dm, dtype=torch.float32, device=dev),
-        y=torch.empty(T, dm, dtype=torch.float32, device=dev))
-    noisy = w.gating == "noisy_topk"
-    o["importance"] = torch.empty(E, dtype=torch.float32, device=dev) if noisy else None
-    o["load"] = torch.empty(E, dtype=torch.float32, device=dev) if noisy and k < E else None
-    ws = moe.workspace(cfg, dev)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-
-    def flush_l2(i):
-        # write 256 MB (evicts everything), then read it back so the step starts from a cold
-        # L2 holding clean lines: the write-back of the flush's own dirty lines is not
-        # charged to the first kernel of the step
-        flush.fill_(float(i))
-        flush.sum()
-    stream = torch.cuda.current_stream(dev)
-
-    launches = [0]
-    fused = moe.fused_combine(cfg)
-
-    def step(evs=None):
+    def step(self, evs=None):
+        """Route, permute, expert FFN, combine; events (if given) between the calls."""
+        moe, d, o, cfg, st = self.moe, self.d, self.o, self.cfg, self.stream
         n = 0
         if evs:
-            evs[0].record(stream)
-        moe.moe_route(cfg, d["x"], d["w_gate"], o["idx"], o["gate"], ws, w_noise=d.get("w_noise"),
+            evs[0].record(st)
+        moe.moe_route(cfg, d["x"], d["w_gate"], o["idx"], o["gate"], self.ws, w_noise=d.get("w_noise"),
                       noise=d.get("noise"), logit_bias=d.get("logit_bias"),
                       importance=o["importance"], load=o["load"], near_tie=o["near"])
         n += moe.last_launch_count()
         if evs:
-            evs[1].record(stream)
+            evs[1].record(st)
         moe.moe_permute(cfg, o["idx"], d["x"], o["counts"], o["offsets"], o["perm_src"],
-                        o["slot_pos"], o["x_perm"], ws)
+                        o["slot_pos"], o["x_perm"], self.ws)
         n += moe.last_launch_count()
         if evs:
-            evs[2].record(stream)
-        if fused:
+            evs[2].record(st)
+        if self.fused:
             # top-1: the down-projection writes gate * row straight into y
             moe.moe_expert_ffn_combine(cfg, o["x_perm"], o["offsets"], o["perm_src"], o["slot_pos"],
-                                       o["gate"], d["w1"], d["w2"], o["h"], o["y"], ws)
+                                       o["gate"], d["w1"], d["w2"], o["h"], o["y"], self.ws)
             n += moe.last_launch_count()
             if evs:
-                evs[3].record(stream)
+                evs[3].record(st)
         else:
             moe.moe_expert_ffn(cfg, o["x_perm"], o["offsets"], d["w1"], d["w2"], o["h"],
-                               o["y_perm"], ws)
+                               o["y_perm"], self.ws)
             n += moe.last_launch_count()
             if evs:
-                evs[3].record(stream)
-            moe.moe_combine(cfg, o["y_perm"], o["slot_pos"], o["gate"], o["y"], ws)
+                evs[3].record(st)
+            moe.moe_combine(cfg, o["y_perm"], o["slot_pos"], o["gate"], o["y"], self.ws)
             n += moe.last_launch_count()
         if evs:
-            evs[4].record(stream)
-        launches[0] += n
+            evs[4].record(st)
+        self.launches += n
 
-    for _ in range(args.warmup):
-        flush_l2(1)
-        step()
+
+class L2Flusher:
+    def __init__(self, dev):
+        self.buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def __call__(self, i):
+        # write 256 MB (evicts everything), then read it back so the step starts from a cold
+        # L2 holding clean lines: the write-back of the flush's own dirty lines is not
+        # charged to the first kernel of the step
+        self.buf.fill_(float(i))
+        self.buf.sum()
+
+
+def timed_steps(lb, flush, steps, warmup, world, dev, clock_gpu):
+    """W warm-up steps, then `steps` timed steps (L2 flushed before each).  Returns the
+    per-step phase times [steps, 4] (ms: route, permute, FFN, combine), the clock
+    summary, kernels launched in the timed region, and the kept-row counts."""
+    import torch.distributed as dist
+    moe = lb.moe
+    for _ in range(warmup):
+        flush(1)
+        lb.step()
     torch.cuda.synchronize(dev)
-    err = moe.moe_get_error(ws)
+    err = moe.moe_get_error(lb.ws)
     if err:
-        raise RuntimeError("device error word %d after warm-up" % err)
-    offs = o["offsets"].cpu().tolist()
-    kept = [offs[e + 1] - offs[e] for e in range(E)]
-    n_kept = offs[-1]
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    launches[0] = 0
+        raise RuntimeError("%s: device error word %d after warm-up" % (lb.w.name, err))
+    offs = lb.o["offsets"].cpu().tolist()
+    kept = [offs[e + 1] - offs[e] for e in range(lb.w.E)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    lb.launches = 0
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    with ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0) as clk:
-        for i in range(args.steps):
-            flush_l2(i)
-            step(evs[i])
+    with ClockSampler(clock_gpu) as clk:
+        for i in range(steps):
+            flush(i)
+            lb.step(evs[i])
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    timed_launches = launches[0]
     per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)]
-                    for i in range(args.steps)])  # ms: route, permute, ffn, combine
-    step_ms = float(np.mean(per.sum(axis=1)))
-    step_ms_max = max_over_ranks(step_ms, dev)
-    err = moe.moe_get_error(ws)
+                    for i in range(steps)])
+    err = moe.moe_get_error(lb.ws)
     if err:
-        raise RuntimeError("device error word %d after the timed steps" % err)
+        raise RuntimeError("%s: device error word %d after the timed steps" % (lb.w.name, err))
+    return per, clk.summary(), lb.launches, kept
 
-    # ---- the same step replayed from a CUDA graph (informational): no host work and no
-    # phase events between the kernels, so every launch edge is programmatic.  Every rank
-    # takes the same collective step whether or not its capture worked.
-    graph_err, g_local, n_graph = None, float("inf"), max(3, min(args.steps, 200))
+
+def summarize(w, per, kept, fused, step_ms_max, world, peaks):
+    """Throughput, per-step GB/s with fractions of the HBM peak, and the grouped GEMM's
+    roofline against the measured HBM copy and bf16 burst / sustained peaks."""
+    n_kept = int(sum(kept))
+    alg = algorithmic(w, n_kept, kept, fused)
+    ms = per.mean(axis=0)
+    ffn_s = ms[2] * 1e-3
+    tflops = alg["ffn_flops"] / ffn_s / 1e12
+    gbs = alg["ffn_bytes"] / ffn_s / 1e9
+    ai = alg["ffn_flops"] / alg["ffn_bytes"]
+    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    bound = "hbm" if ai < ridge else "tensor"
+    hbm = peaks["hbm_gbs"]
+    step_gbs = {"route": alg["route_bytes"] / (ms[0] * 1e-3) / 1e9,
+                "permute": alg["permute_bytes"] / (ms[1] * 1e-3) / 1e9,
+                "combine": None if fused else alg["combine_bytes"] / (ms[3] * 1e-3) / 1e9}
+    return {
+        "value": w.T * world / (step_ms_max * 1e-3), "unit": "tokens/s",
+        "ms_per_step": step_ms_max,
+        "steps_ms": {"route": float(ms[0]), "permute": float(ms[1]), "expert_ffn": float(ms[2]),
+                     "combine": "fused into expert_ffn" if fused else float(ms[3])},
+        "step_gbs": step_gbs,
+        "step_hbm_frac": {kk: (None if v is None else v / hbm) for kk, v in step_gbs.items()},
+        "expert_gemm": {"tflops": tflops, "frac_of_bf16_burst": tflops / peaks["bf16_tflops"],
+                        "frac_of_bf16_sustained": tflops / peaks["bf16_tflops_sustained"],
+                        "gbs": gbs, "frac_of_hbm": gbs / hbm, "arith_intensity": ai,
+                        "bound": bound,
+                        "roofline_frac": gbs / hbm if bound == "hbm"
+                        else tflops / peaks["bf16_tflops_sustained"],
+                        "compute": "tcgen05 bf16" if w.dtype == "bf16" else "fp32 SIMT FMA"},
+        "kept_rows": n_kept,
+        "_alg": alg,
+    }
+
+
+def graph_replay(lb, flush, steps, dev, stream):
+    """The same step captured once into a CUDA graph and replayed (L2 flushed before each
+    replay); returns (mean ms, None) or (inf, reason)."""
+    moe = lb.moe
     try:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, capture_error_mode="thread_local"):
-            step()
+            lb.step()
         g_ms = []
-        for i in range(n_graph + 3):
-            flush_l2(i)
+        for i in range(steps + 3):
+            flush(i)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             graph.replay()
@@ -395,28 +451,26 @@ def run_gpu(args, w):
             if i >= 3:
                 g_ms.append(a.elapsed_time(b))
         del graph
-        if moe.moe_get_error(ws):
+        if moe.moe_get_error(lb.ws):
             raise RuntimeError("device error word set after the graph replays")
-        g_local = float(np.mean(g_ms))
+        return float(np.mean(g_ms)), None
     except RuntimeError as ex:
-        graph_err = str(ex).splitlines()[0][:200]
-    g_mean = max_over_ranks(g_local, dev)
-    if graph_err is not None or not np.isfinite(g_mean):
-        graph_info = {"unavailable": graph_err or "capture failed on another rank"}
-    else:
-        graph_info = {"value": T * world / (g_mean * 1e-3), "unit": "tokens/s", "ms_per_step": g_mean,
-                      "steps": n_graph, "note": "one step (route, permute, expert FFN, combine) "
-                      "captured once and replayed; L2 flushed before each replay"}
+        return float("inf"), str(ex).splitlines()[0][:200]
 
-    # ---- end to end through the public layer call, host buffers in pinned memory.
-    # Every step copies its x (and noise) in from pinned host memory and its y out.  The
-    # headline figure pipelines consecutive steps the way a caller streaming batches
-    # would: H2D on one stream, the forward on the compute stream, D2H on a third, two
-    # sets of device buffers, so that step i's D2H and step i+1's H2D (the two PCIe
-    # directions) overlap the forwards.  The serial latency of one step (copy in,
-    # forward, copy out, nothing overlapped) is reported beside it.
+
+def end_to_end(lb, flush, steps, world, dev, stream):
+    """End to end through the public layer call, host buffers in pinned memory.  Every
+    step copies its x (and noise) in from pinned host memory and its y out.  The headline
+    figure pipelines consecutive steps the way a caller streaming batches would: H2D on
+    one stream, the forward on the compute stream, D2H on a third, two sets of device
+    buffers, so that step i's D2H and step i+1's H2D (the two PCIe directions) overlap
+    the forwards.  The serial latency of one step (copy in, forward, copy out, nothing
+    overlapped) is reported beside it."""
+    import torch.distributed as dist
+    moe, w, d, inp, noisy = lb.moe, lb.w, lb.d, lb.inp, lb.noisy
+    T, dm = w.T, w.d_model
     wl = {kk: v for kk, v in d.items() if kk not in ("x", "noise")}
-    layers = [moe.MoELayer(cfg, wl, device=dev) for _ in range(2)]
+    layers = [moe.MoELayer(lb.cfg, wl, device=dev) for _ in range(2)]
     x_host = inp["x"].pin_memory()
     noise_host = inp["noise"].pin_memory() if noisy else None
     y_host = [torch.empty(T, dm, dtype=torch.float32).pin_memory() for _ in range(2)]
@@ -456,15 +510,14 @@ def run_gpu(args, w):
                 y_host[b].copy_(layers[b].y, non_blocking=True)
                 ev_out[b].record(s_out)
 
-    for _ in range(max(3, args.warmup // 4)):
+    for _ in range(3):
         serial_step()
     pipelined(4)
     torch.cuda.synchronize(dev)
-    # serial latency per step (L2 flushed before each)
-    lat_steps = max(3, min(args.steps, 100))
+    lat_steps = max(3, min(steps, 50))
     lat_ms = []
     for i in range(lat_steps):
-        flush_l2(i)
+        flush(i)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         serial_step()
@@ -474,8 +527,7 @@ def run_gpu(args, w):
     lat_mean = max_over_ranks(float(np.mean(lat_ms)), dev)
     if not torch.equal(y_host[0], layers[0].y.cpu()):
         raise RuntimeError("end-to-end output mismatch between host copy and device result")
-    # pipelined throughput: all streams joined on both sides of the timed steps
-    e2e_steps = max(4, min(args.steps, 200))
+    e2e_steps = max(4, min(steps, 100))
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
@@ -492,62 +544,109 @@ def run_gpu(args, w):
     last = (e2e_steps - 1) % 2
     if not torch.equal(y_host[last], layers[last].y.cpu()):
         raise RuntimeError("pipelined end-to-end output mismatch between host copy and device result")
+    return {"value": T * world / (e2e_mean * 1e-3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_mean,
+            "serial_latency_ms_per_step": lat_mean,
+            "call": "MoELayer.forward (moe_forward); x/noise copied in from pinned host memory and "
+                    "y copied out every step; consecutive steps pipelined on three streams "
+                    "(H2D / forward / D2H, two buffer sets); no L2 flush between pipelined "
+                    "steps (each step's x arrives by H2D)"}
 
+
+def run_gpu(args, w):
+    import torch.distributed as dist
+    import sparsely_gated_mixture_moe_b200 as moe
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    clock_gpu = local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0
     peaks, peak_src = load_peaks()
-    alg = algorithmic(w, n_kept, kept, fused)
-    ffn_ms = float(np.mean(per[:, 2]))
-    gemm_launch_s = ffn_ms * 1e-3 / 2.0
-    ffn_tflops = alg["ffn_flops"] / (ffn_ms * 1e-3) / 1e12
-    ffn_gbs = alg["ffn_bytes"] / (ffn_ms * 1e-3) / 1e9
-    ai = alg["ffn_flops"] / alg["ffn_bytes"]
-    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    traffic = recorded_traffic(w.name)
-    if ai < ridge:
-        roof = {"bound": "hbm", "achieved": ffn_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": ffn_gbs / peaks["hbm_gbs"]}
+    flush = L2Flusher(dev)
+    stream = torch.cuda.current_stream(dev)
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+
+    # ---- the headline workload
+    lb = LayerBench(moe, w, dev)
+    per, clocks, timed_launches, kept = timed_steps(lb, flush, args.steps, args.warmup, world,
+                                                   dev, clock_gpu)
+    step_ms_max = max_over_ranks(float(np.mean(per.sum(axis=1))), dev)
+    main = summarize(w, per, kept, lb.fused, step_ms_max, world, peaks)
+    alg = main.pop("_alg")
+
+    n_graph = max(3, min(args.steps, 200))
+    g_local, graph_err = graph_replay(lb, flush, n_graph, dev, stream)
+    g_mean = max_over_ranks(g_local, dev)
+    if graph_err is not None or not np.isfinite(g_mean):
+        graph_info = {"unavailable": graph_err or "capture failed on another rank"}
     else:
-        roof = {"bound": "tensor", "achieved": ffn_tflops, "peak": peaks["bf16_tflops_sustained"],
-                "unit": "TFLOP/s", "frac": ffn_tflops / peaks["bf16_tflops_sustained"]}
+        graph_info = {"value": w.T * world / (g_mean * 1e-3), "unit": "tokens/s",
+                      "ms_per_step": g_mean, "steps": n_graph,
+                      "note": "one step (route, permute, expert FFN, combine) captured once and "
+                              "replayed; L2 flushed before each replay"}
+    e2e = end_to_end(lb, flush, args.steps, world, dev, stream)
+
+    eg = main["expert_gemm"]
+    ffn_ms = main["steps_ms"]["expert_ffn"]
+    traffic = recorded_traffic(w.name)
+    if eg["bound"] == "hbm":
+        roof = {"bound": "hbm", "achieved": eg["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": eg["frac_of_hbm"]}
+    else:
+        roof = {"bound": "tensor", "achieved": eg["tflops"], "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": eg["frac_of_bf16_sustained"]}
     roof.update({"traffic": traffic,
                  "kernel": "grouped_gemm_tc_kernel (2 launches/step%s)" % (
                      "; the down-projection writes gate * row into y and zeroes dropped "
-                     "tokens' rows" if fused else ""),
+                     "tokens' rows" if lb.fused else ""),
                  "algorithmic_per_launch": {"flops": alg["ffn_flops"] / 2,
                                             "bytes": alg["ffn_bytes"] / 2},
-                 "launch_ms": gemm_launch_s * 1e3, "peak_source": "%s (MEASURED_PEAKS.json)" % peak_src
-                 if peak_src == "measured" else "fallback"})
-
-    value = T * world / (step_ms_max * 1e-3)
+                 "launch_ms": ffn_ms / 2.0,
+                 "peak_source": ("%s (MEASURED_PEAKS.json; %s)" % (
+                     peak_src, "bf16 sustained: the kernel runs inside multi-kernel steps"
+                     if roof["bound"] == "tensor" else "HBM copy")) if peak_src == "measured"
+                 else "fallback"})
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC, "value": main["value"], "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms_max,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded; random-init weights)", "config": config_json(w),
         "roofline": roof,
-        "expert_gemm": {"tflops": ffn_tflops, "frac_of_bf16_peak": ffn_tflops / peaks["bf16_tflops"],
-                        "gbs": ffn_gbs, "frac_of_hbm": ffn_gbs / peaks["hbm_gbs"],
-                        "arith_intensity": ai},
-        "steps_ms": {"route": float(np.mean(per[:, 0])), "permute": float(np.mean(per[:, 1])),
-                     "expert_ffn": ffn_ms,
-                     "combine": "fused into expert_ffn" if fused else float(np.mean(per[:, 3]))},
-        "step_gbs": {"route": alg["route_bytes"] / (np.mean(per[:, 0]) * 1e-3) / 1e9,
-                     "permute": alg["permute_bytes"] / (np.mean(per[:, 1]) * 1e-3) / 1e9,
-                     "combine": None if fused else
-                     alg["combine_bytes"] / (np.mean(per[:, 3]) * 1e-3) / 1e9},
-        "kept_rows": n_kept,
-        "e2e": {"value": T * world / (e2e_mean * 1e-3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_mean,
-                "serial_latency_ms_per_step": lat_mean,
-                "call": "MoELayer.forward (moe_forward); x/noise copied in from pinned host memory and "
-                        "y copied out every step; consecutive steps pipelined on three streams "
-                        "(H2D / forward / D2H, two buffer sets); no L2 flush between pipelined "
-                        "steps (each step's x arrives by H2D; the weights exceed L2)"},
-        "graph": graph_info,
-        "gpu_launches": timed_launches,
-        "clocks": clk.summary(),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, inp)
+    line.update({kk: v for kk, v in main.items() if kk not in ("value", "unit", "ms_per_step")})
+    line.update({"e2e": e2e, "graph": graph_info, "gpu_launches": timed_launches, "clocks": clocks})
+    inp_main = lb.inp
+    del lb
+    torch.cuda.empty_cache()
+
+    # ---- every other workload: the same timed step, fewer extras
+    per_config = {}
+    if not args.no_per_config:
+        pc_steps = max(3, min(args.steps, 50))
+        for name in workloads.ORDER:
+            if name == w.name:
+                continue
+            wk = workloads.WORKLOADS[name]
+            lbk = LayerBench(moe, wk, dev)
+            perk, clk, nl, keptk = timed_steps(lbk, flush, pc_steps, args.warmup, world, dev,
+                                               clock_gpu)
+            smax = max_over_ranks(float(np.mean(perk.sum(axis=1))), dev)
+            r = summarize(wk, perk, keptk, lbk.fused, smax, world, peaks)
+            r.pop("_alg")
+            r.update({"steps": pc_steps, "gpu_launches": nl, "clocks": clk,
+                      "config": config_json(wk)})
+            if want_cpu:
+                r["cpu_baseline"] = cpu_baseline(wk, lbk.inp)
+            per_config[name] = r
+            del lbk
+            torch.cuda.empty_cache()
+        line["per_config"] = per_config
+    if want_cpu:
+        line["cpu_baseline"] = cpu_baseline(w, inp_main, budget_s=12.0)
+    line["peaks"] = dict(peaks, source=peak_src)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -558,11 +657,13 @@ def run_gpu(args, w):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="switch", choices=list(workloads.WORKLOADS))
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="zipf", choices=list(workloads.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the headline workload")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -247,9 +247,11 @@ moe_status moe_bf16_to_f16(const void* src, void* dst, int64_t n, int32_t* n_ine
  *  Sizes: 256 + ceil(T*k / 256) * E * 4 must not exceed MOE_NOALLOC_SCRATCH_BYTES (for
  *  E = 128 that is T*k up to 524,032); larger problems return MOE_ERR_UNSUPPORTED and
  *  queue nothing.
- *  Set-up: the first call on a device, with that device current, looks up the array's
- *  device address (cudaGetSymbolAddress) and caches it; make that first call before any
- *  stream capture.
+ *  Set-up: the first call in a CUDA context (in practice, the first call on a device, made
+ *  with that device current) looks up the array's device address there
+ *  (cudaGetSymbolAddress) and caches it under the context's unique id, so a context that
+ *  replaces an earlier one (after cudaDeviceReset) gets a fresh lookup; make that first
+ *  call before any stream capture.
  *  Sharing: every call uses the same array, which keeps the previous call's contents;
  *  each call clears the counter that must start at zero (cudaMemsetAsync on `stream`) and
  *  rewrites everything else it reads.  Calls whose work overlaps on the GPU (other

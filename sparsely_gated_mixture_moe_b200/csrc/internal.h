@@ -23,18 +23,25 @@ struct LaunchCtx {
   int* launches;  // host counter
 };
 
-// Raises a kernel's dynamic shared-memory limit to at least `bytes` on the current device,
-// calling cudaFuncSetAttribute only the first time a larger limit is needed there (the
-// attribute outlives the call; repeating it on every launch only costs host time).
+// Unique id of the CUDA context current on this thread (cuCtxGetId), initialising the
+// device's primary context first if need be.  Ids are never reused within a process, so
+// state cached per context (a looked-up symbol address, a raised kernel attribute) is
+// never taken for a context that replaced it, e.g. after cudaDeviceReset.
+cudaError_t current_context_id(unsigned long long* id);
+
+// Raises a kernel's dynamic shared-memory limit to at least `bytes` in the current
+// context, calling cudaFuncSetAttribute only the first time a larger limit is needed
+// there (the attribute outlives the call; repeating it on every launch only costs host
+// time).
 template <typename... KArgs>
 cudaError_t ensure_smem_limit(void (*kernel)(KArgs...), int bytes) {
   static std::mutex mu;
-  static std::map<std::pair<int, const void*>, int> limit;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static std::map<std::pair<unsigned long long, const void*>, int> limit;
+  unsigned long long ctx = 0;
+  cudaError_t e = current_context_id(&ctx);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(mu);
-  const auto key = std::make_pair(dev, reinterpret_cast<const void*>(kernel));
+  const auto key = std::make_pair(ctx, reinterpret_cast<const void*>(kernel));
   const auto it = limit.find(key);
   if (it != limit.end() && it->second >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);

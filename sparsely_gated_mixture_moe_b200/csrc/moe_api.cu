@@ -1,6 +1,9 @@
 // C ABI of libmoe (declared in include/moe.h): host-side argument validation, the
 // workspace layout, and the launch sequence of each step and of the fused forward.
+#include <cudaTypedefs.h>
 #include <string.h>
+
+#include <mutex>
 
 #include "internal.h"
 #include "moe.h"
@@ -251,6 +254,35 @@ moe_status empty_batch(const moe_config* cfg, int32_t* counts, int32_t* offsets,
 }
 
 }  // namespace
+
+cudaError_t current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return cudaErrorNotSupported;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  if (ctx == nullptr) {
+    // no context yet on this thread: cudaSetDevice makes the device's primary context
+    // current (initialising it), as every later runtime call would
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaSetDevice(dev);
+    if (e != cudaSuccess) return e;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorDeviceUninitialized;
+  }
+  return get_id(ctx, id) == CUDA_SUCCESS ? cudaSuccess : cudaErrorDeviceUninitialized;
+}
 
 moe_status check_config_host(const moe_config* cfg) { return check_config(cfg); }
 int64_t capacity_host(const moe_config* cfg) { return capacity_of(cfg); }

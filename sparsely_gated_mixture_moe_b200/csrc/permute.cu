@@ -18,6 +18,7 @@
 //   gather      x_perm[s] = x[perm_src[s] / k] for every kept row s < offsets[E]: one warp
 //               per row, 16-byte vectors, a grid of several blocks per SM so that enough
 //               loads are in flight to stream at HBM rate
+#include <map>
 #include <mutex>
 
 #include "common.cuh"
@@ -519,23 +520,27 @@ namespace moe {
 static __device__ __align__(256) int32_t g_permute_scratch[MOE_NOALLOC_SCRATCH_BYTES / 4];
 
 namespace {
-constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+std::map<unsigned long long, void*> g_scratch_addr;  // context id -> device address
 
-// Device address of g_permute_scratch on the current device.  In host code the name
-// g_permute_scratch is only a host-side stand-in, so the address is looked up once per
-// device, with that device current, and cached.
-cudaError_t scratch_address(int dev, void** out) {
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+// Device address of g_permute_scratch in the current context.  In host code the name
+// g_permute_scratch is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress, once per context (the context current on this thread, i.e. the
+// current device's), and cached under the context's unique id: a context that replaces
+// an earlier one (after cudaDeviceReset, say) gets its own lookup.
+cudaError_t scratch_address(void** out) {
+  unsigned long long ctx = 0;
+  cudaError_t e = current_context_id(&ctx);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  auto it = g_scratch_addr.find(ctx);
+  if (it == g_scratch_addr.end()) {
     void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_permute_scratch);
+    e = cudaGetSymbolAddress(&p, g_permute_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
+    it = g_scratch_addr.emplace(ctx, p).first;
   }
-  *out = g_scratch_addr[dev];
+  *out = it->second;
   return cudaSuccess;
 }
 }  // namespace
@@ -571,7 +576,7 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
   void* scratch = nullptr;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&c.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      scratch_address(dev, &scratch) != cudaSuccess)
+      scratch_address(&scratch) != cudaSuccess)
     return MOE_ERR_CUDA;
   c.stream = s;
   c.err = nullptr;  // no error word: out-of-range expert indices are dropped unreported

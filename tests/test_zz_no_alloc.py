@@ -77,9 +77,56 @@ def test_noalloc_permute_matches_workspace_permute(name):
         assert torch.equal(got["x_perm"][:n_kept], ref["x_perm"][:n_kept])
 
 
-def test_noalloc_rejects_sizes_beyond_its_scratch():
-    # ceil(T*k/2048) * E * 4 bytes > 1 MiB: refused on the host, nothing queued
-    cfg = moe.make_config(1 << 23, 64, 64, 256, 1)
-    d = torch.zeros(16, dtype=torch.int32, device="cuda")
-    p = ctypes.c_void_p(d.data_ptr())
-    assert moe.lib.moe_permute_noalloc(ctypes.byref(cfg), p, p, p, p, p, p, p, None) == 2
+def _random_choices(T, k, E, seed):
+    gen = torch.Generator().manual_seed(seed)
+    return torch.randint(0, E, (T, k), generator=gen, dtype=torch.int32)
+
+
+def test_noalloc_size_limit_boundary():
+    """The scratch holds 256 bytes of counters and one int32 per (256-assignment chunk,
+    expert): with E = 128 and k = 1 that allows T = 524,032 (2047 chunks) and refuses
+    T = 524,033 (2048 chunks, 256 + 2048 * 512 bytes > 1 MiB) on the host, queueing
+    nothing.  The largest accepted size runs and equals moe_permute bit for bit."""
+    E, d = 128, 64
+    too_big = moe.make_config(524_033, d, 64, E, 1)
+    z = torch.zeros(16, dtype=torch.int32, device="cuda")
+    p = ctypes.c_void_p(z.data_ptr())
+    assert moe.lib.moe_permute_noalloc(ctypes.byref(too_big), p, p, p, p, p, p, p, None) == 2
+
+    w = Workload("lim", T=524_032, d_model=d, d_ff=64, E=E, k=1)
+    cfg = _cfg(w)
+    x = workloads.make_x(w).cuda()
+    idx = _random_choices(w.T, 1, E, 11).cuda()
+    ref, got = _outputs(w), _outputs(w)
+    ws = moe.workspace(cfg)
+    moe.moe_permute(cfg, idx, x, ref["counts"], ref["offsets"], ref["perm_src"], ref["slot_pos"],
+                    ref["x_perm"], ws)
+    assert moe.moe_get_error(ws) == 0
+    _noalloc(cfg, idx, x, got)
+    torch.cuda.synchronize()
+    for key in ("counts", "offsets", "perm_src", "slot_pos", "x_perm"):
+        assert torch.equal(got[key], ref[key]), key
+
+
+def test_noalloc_out_of_range_expert_is_dropped():
+    """Without a device error word, an expert index outside [0, E) is dropped silently:
+    its slot is -1, and counts and offsets tally only the valid entries."""
+    w = Workload("oor", T=300, d_model=64, d_ff=64, E=8, k=2, dtype="f32")
+    cfg = _cfg(w)
+    x = workloads.make_x(w).cuda()
+    idx = _random_choices(w.T, w.k, w.E, 5)
+    bad = [(3, 0, -1), (10, 1, 8), (77, 0, 8), (299, 1, -1), (150, 0, 1000)]
+    for t, j, v in bad:
+        idx[t, j] = v
+    got = _outputs(w)
+    _noalloc(cfg, idx.cuda(), x, got)
+    torch.cuda.synchronize()
+    flat = idx.view(-1)
+    valid = (flat >= 0) & (flat < w.E)
+    tally = torch.bincount(flat[valid].long(), minlength=w.E)
+    assert got["counts"].cpu().tolist() == tally.tolist()
+    assert got["offsets"].cpu().tolist() == [0] + torch.cumsum(tally, 0).tolist()
+    sp = got["slot_pos"].cpu()
+    for t, j, _ in bad:
+        assert int(sp[t * w.k + j]) == -1
+    assert bool((sp[valid] >= 0).all())
