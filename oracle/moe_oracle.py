@@ -30,6 +30,10 @@ Readings where the pages are silent or garbled:
     per expert the C assignments of lowest flattened index t*k + j are kept; a dropped
     assignment contributes zero and gates are not renormalised after a drop.
   * Experts are E_i(x) = W2_i act(W1_i x) with no biases; GELU is the exact erf form.
+  * Hierarchical MoE (one sentence on the page, "MoE-H" in the setups table): two levels
+    of the page's top-k gate without noise, a primary gate over groups and a secondary
+    gate over each chosen group's experts; an assignment's gate is the product of the
+    two levels' gates, and the layer sums over both levels' chosen entries.
 
 parity pins: every function below is pinned by tests/test_oracle_pins.py against hand
 derivations, library routines (torch.nn.functional, scipy.stats) or brute force.
@@ -192,6 +196,72 @@ def load(P):
     return np.sum(_f64(P), axis=0)
 
 
+# ------------------------------------------------------------ hierarchical gating
+
+
+def hierarchical_gates(l, groups, k_primary, k_group):
+    """Two-level gating of a hierarchical MoE [SGMoE "Schlüsselbegriffe": a primary gating
+    network routes each input to secondary MoE groups; Setups Table 2: "MoE-H" with 4 or
+    2 chosen per level].
+
+    l [T, a + a*b] holds the clean logits of the primary gate over the a groups (columns
+    0 .. a-1), then group i's secondary logits over its b experts (columns a + i*b ..
+    a + i*b + b - 1).  Each level is the page's top-k gate without noise:
+      G_p(x)   = Softmax(KeepTopK(primary logits, k_primary))        over the a groups
+      G_i(x)   = Softmax(KeepTopK(group i's logits, k_group))        over its b experts
+      y        = sum_i G_p(x)_i sum_j G_i(x)_j E_{i,j}(x)
+    so a token has k_primary * k_group assignments; expert (i, j) has the flat index
+    i*b + j and the gate G_p(x)_i * G_i(x)_j.  Chosen groups are listed by descending
+    primary score, and within a group the chosen experts by descending secondary score
+    (ties to the lowest index at both levels, decided on fp32 scores as top_k does).
+
+    Returns (idx [T, k_primary*k_group] int64, gates [T, k_primary*k_group], gap [T]):
+    gap is the smallest k-th vs (k+1)-th gap among the primary scores and the chosen
+    groups' secondary scores (a near tie at either level where it is <= 1e-4)."""
+    l = _f64(l)
+    T = l.shape[0]
+    a = int(groups)
+    b = (l.shape[1] - a) // a
+    if l.shape[1] != a + a * b or not (1 <= k_primary <= a and 1 <= k_group <= b):
+        raise ValueError("bad hierarchical gating shape")
+    prim = l[:, :a]
+    sec = l[:, a:].reshape(T, a, b)
+    chosen = top_k(prim, k_primary)                  # [T, k_primary]
+    g_prim = gate_values(prim, chosen, True)         # G_p at the chosen groups
+    gap = topk_gap(prim, k_primary)
+    k = k_primary * k_group
+    idx = np.zeros((T, k), np.int64)
+    gates = np.zeros((T, k))
+    rows = np.arange(T)
+    for q in range(k_primary):
+        g = chosen[:, q]
+        s = sec[rows, g, :]                          # [T, b]: the chosen group's logits
+        j = top_k(s, k_group)
+        idx[:, q * k_group:(q + 1) * k_group] = g[:, None] * b + j
+        gates[:, q * k_group:(q + 1) * k_group] = g_prim[:, q:q + 1] * gate_values(s, j, True)
+        gap = np.minimum(gap, topk_gap(s, k_group))
+    return idx, gates, gap
+
+
+def hierarchical_dense_gates(l, groups, k_primary, k_group):
+    """G(x) of the hierarchical layer as a dense [T, a*b] matrix, by its definition: the
+    dense primary gate Softmax(KeepTopK(., k_primary)) over the groups times each
+    group's dense secondary gate Softmax(KeepTopK(., k_group)), evaluated for every group
+    (unchosen groups get primary weight 0)."""
+    l = _f64(l)
+    T = l.shape[0]
+    a = int(groups)
+    b = (l.shape[1] - a) // a
+    prim = l[:, :a]
+    Gp = softmax(keep_top_k(prim, top_k(prim, k_primary)))       # [T, a]
+    G = np.zeros((T, a * b))
+    for i in range(a):
+        s = l[:, a + i * b:a + (i + 1) * b]
+        Gi = softmax(keep_top_k(s, top_k(s, k_group)))            # [T, b]
+        G[:, i * b:(i + 1) * b] = Gp[:, i:i + 1] * Gi
+    return G
+
+
 # ------------------------------------------------------------------ capacity, dispatch
 
 
@@ -299,6 +369,11 @@ def route(inp, w):
     x = inp["x"]
     bias = inp.get("logit_bias")
     out = {}
+    if w.gating == "hierarchical":
+        scores = router_logits(x, inp["w_gate"], bias)
+        idx, gates, gap = hierarchical_gates(scores, w.groups, w.k_primary, w.k // w.k_primary)
+        out.update(scores=scores, idx=idx, gates=gates, gap=gap)
+        return out
     if w.gating == "noisy_topk":
         l, s, H = noisy_logits(x, inp["w_gate"], inp["w_noise"], inp["noise"], bias)
         scores = H
@@ -341,7 +416,17 @@ def moe_forward_dense(inp, w):
     T = r["idx"].shape[0]
     C = capacity(w.capacity_factor, T, w.k, w.E)
     _, _, _, slot_pos = dispatch(r["idx"], w.E, C)
-    G = dense_gates(T, w.E, r["idx"], r["gates"], slot_pos)
+    if w.gating == "hierarchical":
+        # the two-level definition, dense; then dropped assignments get 0
+        G = hierarchical_dense_gates(r["scores"], w.groups, w.k_primary, w.k // w.k_primary)
+        keep = np.ones((T, w.E))
+        sp = slot_pos.reshape(T, w.k)
+        for j in range(w.k):
+            drop = sp[:, j] < 0
+            keep[np.nonzero(drop)[0], r["idx"][drop, j]] = 0.0
+        G = G * keep
+    else:
+        G = dense_gates(T, w.E, r["idx"], r["gates"], slot_pos)
     x = _f64(inp["x"])
     y = np.zeros((T, x.shape[1]))
     for e in range(w.E):

@@ -328,6 +328,98 @@ def test_importance_sums_to_T_and_gates_sum_to_one():
     assert r["load"].shape == (8,) and np.all(r["load"] >= 0) and np.all(r["load"] <= T)
 
 
+# ------------------------------------------------------------- hierarchical gating
+
+
+@pytest.mark.parametrize("case", _gold("hierarchical_hand.json")["cases"])
+def test_hierarchical_gating_hand_cases(case):
+    """Two-level Softmax(KeepTopK) on hand-worked logits (ties at both levels)."""
+    l = np.log(np.array([case["q"]], np.float64))
+    idx, gates, _ = orc.hierarchical_gates(l, case["a"], case["k_primary"], case["k_group"])
+    assert idx[0].tolist() == case["idx"]
+    assert np.allclose(gates[0], [n / d for n, d in case["gates"]], rtol=1e-14, atol=0)
+
+
+def _hier_brute(row, a, k1, k2):
+    """Pure-Python loops: sort groups, then each chosen group's experts, by (-score,
+    index); shares from math.exp over the kept entries of each level."""
+    b = (len(row) - a) // a
+    prim = [row[i] for i in range(a)]
+    groups = sorted(range(a), key=lambda i: (-float(np.float32(prim[i])), i))[:k1]
+    zp = sum(math.exp(prim[i] - prim[groups[0]]) for i in groups)
+    idx, gates = [], []
+    for gi in groups:
+        sec = [row[a + gi * b + j] for j in range(b)]
+        chosen = sorted(range(b), key=lambda j: (-float(np.float32(sec[j])), j))[:k2]
+        zs = sum(math.exp(sec[j] - sec[chosen[0]]) for j in chosen)
+        for j in chosen:
+            idx.append(gi * b + j)
+            gates.append(math.exp(prim[gi] - prim[groups[0]]) / zp *
+                         math.exp(sec[j] - sec[chosen[0]]) / zs)
+    return idx, gates
+
+
+@pytest.mark.parametrize("a,b,k1,k2", [(4, 3, 2, 2), (3, 5, 1, 3), (5, 2, 3, 1), (2, 6, 2, 4)])
+def test_hierarchical_gating_brute_force(a, b, k1, k2):
+    g = np.random.default_rng(20 + a * b)
+    # coarse values make ties at both levels frequent
+    l = np.round(g.standard_normal((60, a + a * b)) * 2) / 2
+    idx, gates, _ = orc.hierarchical_gates(l, a, k1, k2)
+    for t in range(l.shape[0]):
+        bi, bg = _hier_brute(l[t], a, k1, k2)
+        assert idx[t].tolist() == bi
+        assert np.allclose(gates[t], bg, rtol=1e-13, atol=0)
+    assert np.allclose(gates.sum(1), 1.0, rtol=0, atol=1e-14)
+
+
+def test_hierarchical_one_group_is_flat_topk():
+    """One group: the primary gate is 1 and the layer is flat top-k over its experts
+    (torch.topk, then torch.softmax over the kept logits)."""
+    g = np.random.default_rng(30)
+    l = g.standard_normal((40, 1 + 9))
+    idx, gates, _ = orc.hierarchical_gates(l, 1, 1, 3)
+    v, i = torch.topk(torch.from_numpy(l[:, 1:]), 3)
+    assert idx.tolist() == i.tolist()
+    assert np.allclose(gates, torch.softmax(v, -1).numpy(), rtol=1e-13)
+
+
+def test_hierarchical_single_expert_groups_is_flat_topk_over_groups():
+    """Groups of one expert: the secondary gate is 1 and the layer is flat top-k over the
+    primary logits."""
+    g = np.random.default_rng(31)
+    a = 7
+    l = np.concatenate([g.standard_normal((40, a)), g.standard_normal((40, a))], axis=1)
+    idx, gates, _ = orc.hierarchical_gates(l, a, 3, 1)
+    v, i = torch.topk(torch.from_numpy(l[:, :a]), 3)
+    assert idx.tolist() == i.tolist()
+    assert np.allclose(gates, torch.softmax(v, -1).numpy(), rtol=1e-13)
+
+
+def _hier_inputs(T, d, f, a, b, seed):
+    inp = _tiny_inputs(T, d, f, a * b, seed)
+    g = np.random.default_rng(seed + 1000)
+    inp["w_gate"] = g.standard_normal((a + a * b, d)) / math.sqrt(d)
+    return inp
+
+
+@pytest.mark.parametrize("cf", [None, 0.5])
+def test_hierarchical_sparse_equals_dense_definition(cf):
+    """y = sum_i G_p(x)_i sum_j G_i(x)_j E_ij(x) evaluated densely (every group's
+    secondary gate) equals the sparse dispatch path, also with capacity drops."""
+    a, b = 3, 4
+    inp = _hier_inputs(48, 10, 14, a, b, 40)
+    w = workloads.Workload("h", T=48, d_model=10, d_ff=14, E=a * b, k=4, gating="hierarchical",
+                           groups=a, k_primary=2, capacity_factor=cf, act="gelu", dtype="f32")
+    sparse = orc.moe_forward(inp, w)
+    dense = orc.moe_forward_dense(inp, w)
+    assert np.allclose(sparse["y"], dense, rtol=0, atol=1e-12)
+    if cf is not None:
+        assert int(sparse["offsets"][-1]) < 48 * 4   # some assignments were dropped
+    rows = [0, 7, 47]
+    y_rows, _ = orc.moe_forward_rows(inp, w, rows)
+    assert np.allclose(y_rows, sparse["y"][rows], rtol=0, atol=1e-12)
+
+
 def test_oracle_and_library_share_no_code():
     """The oracle never imports the CUDA library's package, and the package never
     imports the oracle."""

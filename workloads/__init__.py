@@ -12,7 +12,8 @@ Distributions (fan_in is the contraction length of the product the tensor enters
   x ~ N(0, 1)                        [T, d_model]
   w_gate, w_noise ~ N(0, 1/d_model)  [E, d_model]  (the gating matrices W_g, W_noise of
                                        "Noisy Top-K Gating", stored transposed: one row
-                                       per expert, so each row is contiguous along d_model)
+                                       per expert, so each row is contiguous along d_model;
+                                       [groups + E, d_model] for hierarchical gating)
   w1 ~ N(0, 1/d_model)               [E, d_ff, d_model]   up-projection, K-major
   w2 ~ N(0, 1/d_ff)                  [E, d_model, d_ff]   down-projection, K-major
   noise ~ N(0, 1) fp32               [T, E]  the StandardNormal() draws of noisy gating,
@@ -49,6 +50,10 @@ class Workload:
             under the softmax over all experts (Switch top-1 rule).
     capacity_factor: None = no limit; else C = ceil(cf * T * k / E) per expert.
     zipf_s: None, or the Zipf exponent of the per-expert logit bias.
+    groups, k_primary: hierarchical gating ("hierarchical"): E experts in `groups` groups
+            of E / groups; the primary gate keeps k_primary groups and each chosen group's
+            gate keeps k / k_primary of its experts.  w_gate then has groups + E rows: the
+            primary gating rows, then each group's secondary gating rows.
     hidden_f16: store the expert hidden activations in fp16 (11 significant bits)
             instead of bf16 (8), with W2 re-encoded to fp16 for the second product.  The
             Switch workload needs it to keep the layer output within max|err|/RMS <= 2e-2:
@@ -69,6 +74,8 @@ class Workload:
     dtype: str = "bf16"
     zipf_s: Optional[float] = None
     hidden_f16: bool = False
+    groups: Optional[int] = None
+    k_primary: int = 1
     seed: int = 0
 
     def scaled(self, **kw) -> "Workload":
@@ -135,7 +142,8 @@ def make_inputs(w: Workload, beta: Optional[float] = None) -> Dict[str, torch.Te
     d, f, E, T = w.d_model, w.d_ff, w.E, w.T
     out: Dict[str, torch.Tensor] = {}
     out["x"] = _normal((T, d), "x", w.seed, 1.0).to(dt)
-    out["w_gate"] = _normal((E, d), "w_gate", w.seed, 1.0 / math.sqrt(d)).to(dt)
+    n_gate = E + (w.groups if w.gating == "hierarchical" else 0)
+    out["w_gate"] = _normal((n_gate, d), "w_gate", w.seed, 1.0 / math.sqrt(d)).to(dt)
     if w.gating == "noisy_topk":
         out["w_noise"] = _normal((E, d), "w_noise", w.seed, 1.0 / math.sqrt(d)).to(dt)
         out["noise"] = _normal((T, E), "noise", w.seed, 1.0)
