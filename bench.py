@@ -164,22 +164,24 @@ def algorithmic(w: workloads.Workload, n_kept: int, counts_kept, fused=False):
     """Algorithmic FLOPs and bytes of each step (kept assignments only, no padding).
 
     FFN FLOPs 4*N*d*f (two products).  FFN bytes: the weights of the experts that got
-    rows, x_perm (dtype) read, y_perm (fp32) written.  Route bytes: x, the gating
-    weights, noise, and the chosen indices and gates.  Permute: x rows read, x_perm
-    rows written, indices.  Combine: y_perm rows read, gates and slots, y written.
-    fused (k = 1, FFN and combine as one step): the FFN writes every row of y (fp32) and
-    reads each kept row's source index and gate; no combine bytes."""
+    rows, the kept assignments' token rows (dtype, gathered from x by the up-projection)
+    and their source indices read, y_perm (fp32) written.  Route bytes: x, the gating
+    weights, noise, and the chosen indices and gates.  Permute (index arrays only): the
+    chosen experts read, slot_pos and perm_src written, counts and offsets.  Combine:
+    y_perm rows read, gates and slots, y written.  fused (k = 1, FFN and combine as one
+    step): the FFN writes every row of y (fp32) and reads each kept row's source index
+    and gate; no combine bytes."""
     es = 2 if w.dtype == "bf16" else 4
     T, d, f, E, k = w.T, w.d_model, w.d_ff, w.E, w.k
     active = int(sum(1 for c in counts_kept if c > 0))
     ffn_flops = 4.0 * n_kept * d * f
-    ffn_bytes = active * 2.0 * d * f * es + n_kept * d * es + n_kept * d * 4.0
+    ffn_bytes = active * 2.0 * d * f * es + n_kept * (d * es + 4.0) + n_kept * d * 4.0
     noisy = w.gating == "noisy_topk"
     route_bytes = T * d * es + E * d * es * (2 if noisy else 1) + (T * E * 4 if noisy else 0) + T * k * 8
-    permute_bytes = n_kept * d * es * 2 + T * k * 4 * 3
+    permute_bytes = T * k * 4 * 3 + E * 8.0
     combine_bytes = n_kept * d * 4.0 + T * k * 8 + T * d * 4.0
     if fused:
-        ffn_bytes = active * 2.0 * d * f * es + n_kept * d * es + T * d * 4.0 + n_kept * 8.0 + T * 4.0
+        ffn_bytes = active * 2.0 * d * f * es + n_kept * (d * es + 4.0) + T * d * 4.0 + n_kept * 8.0 + T * 4.0
         combine_bytes = 0.0
     return {"ffn_flops": ffn_flops, "ffn_bytes": ffn_bytes, "route_bytes": route_bytes,
             "permute_bytes": permute_bytes, "combine_bytes": combine_bytes}
@@ -300,7 +302,6 @@ class LayerBench:
             offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
             perm_src=torch.empty(T * k, dtype=torch.int32, device=dev),
             slot_pos=torch.empty(T * k, dtype=torch.int32, device=dev),
-            x_perm=torch.empty(T * k, dm, dtype=w.torch_dtype, device=dev),
             h=torch.empty(T * k, f, dtype=torch.float16 if w.hidden_f16 else w.torch_dtype,
                           device=dev),
             y_perm=torch.empty(T * k, dm, dtype=torch.float32, device=dev),
@@ -325,21 +326,23 @@ class LayerBench:
         n += moe.last_launch_count()
         if evs:
             evs[1].record(st)
-        moe.moe_permute(cfg, o["idx"], d["x"], o["counts"], o["offsets"], o["perm_src"],
-                        o["slot_pos"], o["x_perm"], self.ws)
+        # index arrays only: the up-projection gathers the token rows from x itself
+        moe.moe_permute(cfg, o["idx"], None, o["counts"], o["offsets"], o["perm_src"],
+                        o["slot_pos"], None, self.ws)
         n += moe.last_launch_count()
         if evs:
             evs[2].record(st)
         if self.fused:
             # top-1: the down-projection writes gate * row straight into y
-            moe.moe_expert_ffn_combine(cfg, o["x_perm"], o["offsets"], o["perm_src"], o["slot_pos"],
-                                       o["gate"], d["w1"], d["w2"], o["h"], o["y"], self.ws)
+            moe.moe_expert_ffn_combine_gather(cfg, d["x"], o["offsets"], o["perm_src"],
+                                              o["slot_pos"], o["gate"], d["w1"], d["w2"], o["h"],
+                                              o["y"], self.ws)
             n += moe.last_launch_count()
             if evs:
                 evs[3].record(st)
         else:
-            moe.moe_expert_ffn(cfg, o["x_perm"], o["offsets"], d["w1"], d["w2"], o["h"],
-                               o["y_perm"], self.ws)
+            moe.moe_expert_ffn_gather(cfg, d["x"], o["perm_src"], o["offsets"], d["w1"], d["w2"],
+                                      o["h"], o["y_perm"], self.ws)
             n += moe.last_launch_count()
             if evs:
                 evs[3].record(st)

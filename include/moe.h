@@ -44,7 +44,9 @@
  *
  * Supported shapes: bf16 needs d_model and d_ff multiples of 64 and E <= 256; fp32
  * needs d_model and d_ff multiples of 4; all need 1 <= k <= min(E, 8), d_model % 8 == 0
- * and T*k < 2^31.  Outside these the call returns MOE_ERR_UNSUPPORTED.
+ * and T*k < 2^31.  Hierarchical gating also needs groups + E <= 256 (bf16) or <= 1024
+ * (fp32) and at most 4 kept per level.  Outside these the call returns
+ * MOE_ERR_UNSUPPORTED.
  */
 #ifndef MOE_H_
 #define MOE_H_
@@ -87,8 +89,22 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
  * MOE_GATE_NOISY_TOPK: H = x.W_g (+ logit_bias) + noise * Softplus(x.W_noise), the k
  *   largest of H are chosen and gates = Softmax(KeepTopK(H, k)) (Shazeer et al.,
  *   "Noisy Top-K Gating"; renorm is ignored).  `noise` holds the StandardNormal() draws.
+ * MOE_GATE_HIERARCHICAL: a two-level gate (Shazeer et al., "Schlüsselbegriffe":
+ *   hierarchical MoE, a primary gating network routing to secondary MoE groups; "MoE-H"
+ *   in the setups table of the "moe paper models" page).  The E experts form
+ *   cfg->groups groups of b = E / groups; w_gate holds groups + E rows: the primary
+ *   gating rows, then group i's b secondary rows.  The primary gate Softmax(KeepTopK(.,
+ *   k_primary)) keeps k_primary groups; each kept group's gate Softmax(KeepTopK(.,
+ *   k / k_primary)) keeps k / k_primary of its experts; expert j of group i is expert
+ *   i*b + j and its gate is the product of the two levels' gates.  Chosen groups are
+ *   listed largest primary score first, each followed by its chosen experts, largest
+ *   first.  No noise; renorm and logit_bias are ignored.
  * Ties go to the lowest expert index; chosen experts are listed largest score first. */
-typedef enum { MOE_GATE_SOFTMAX_TOPK = 0, MOE_GATE_NOISY_TOPK = 1 } moe_gating;
+typedef enum {
+  MOE_GATE_SOFTMAX_TOPK = 0,
+  MOE_GATE_NOISY_TOPK = 1,
+  MOE_GATE_HIERARCHICAL = 2
+} moe_gating;
 
 /* Expert activation: ReLU, or GELU in its erf form 0.5 z (1 + erf(z / sqrt 2)) (not the
  * tanh approximation).  The bf16 tensor-core path evaluates erf by Abramowitz & Stegun
@@ -112,6 +128,9 @@ typedef struct {
                              both operands of one tensor-core product share a type; a bf16
                              w2 converts to fp16 exactly wherever |w| >= 2^-17 (see
                              moe_bf16_to_f16).  Needs |h| < 65504. */
+  int32_t groups;         /* MOE_GATE_HIERARCHICAL: expert groups (divides E); else ignored */
+  int32_t k_primary;      /* MOE_GATE_HIERARCHICAL: groups kept per token (divides k, and
+                             k / k_primary <= E / groups); else ignored */
 } moe_config;
 
 /* Human-readable name of a status code (static string). */
@@ -127,7 +146,7 @@ int64_t moe_capacity(const moe_config* cfg);
 size_t moe_workspace_size(const moe_config* cfg);
 
 /* Bytes of workspace moe_forward needs: the step workspace plus the intermediates
- * (offsets, slot_pos, perm_src, x_perm, h, y_perm) it keeps there. */
+ * (offsets, slot_pos, perm_src, h, y_perm) it keeps there. */
 size_t moe_forward_workspace_size(const moe_config* cfg);
 
 /* Router product and gate [Shazeer et al., "Noisy Top-K Gating"; Switch Transformer,
@@ -160,7 +179,9 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_gate,
  *  perm_src [T*k] int32 out: perm_src[s] = assignment a held by permuted row s
  *           (entries at s >= offsets[E] are left untouched)
  *  slot_pos [T*k] int32 out: permuted row of assignment a, or -1 if dropped
- *  x_perm   [T*k, d_model] dtype out: x_perm[s] = x[perm_src[s] / k]
+ *  x_perm   [T*k, d_model] dtype out: x_perm[s] = x[perm_src[s] / k]; or NULL, and then
+ *           x may be NULL too: only the index arrays are written and no row is copied
+ *           (the expert FFN gathers the rows itself: moe_expert_ffn_gather)
  * Within an expert rows keep ascending a; the first C are kept (C = moe_capacity). */
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* x,
                        int32_t* counts, int32_t* offsets, int32_t* perm_src,
@@ -181,6 +202,20 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
 moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
                           const void* w1, const void* w2, void* h, void* y_perm, void* ws,
                           moe_stream_t stream);
+
+/* moe_expert_ffn with the permuted rows gathered from the token rows instead of read
+ * from x_perm [Switch Transformer, switch_routing: dispatch is a gather of each expert's
+ * tokens]: permuted row s is x[perm_src[s] / k], fetched by the up-projection's tensor
+ * memory accelerator (TMA) straight into the tensor cores' operand tiles, so x_perm is
+ * never written or read back.  Results are bit-identical to moe_permute (with x_perm)
+ * followed by moe_expert_ffn.
+ *  x        [T, d_model] dtype in (the token rows)
+ *  perm_src [T*k] int32 in, as written by moe_permute (entries s < offsets[E] are read;
+ *           a value outside [0, T*k) reads zeros for that row's operand)
+ *  offsets, w1, w2, h, y_perm, ws: as moe_expert_ffn. */
+moe_status moe_expert_ffn_gather(const moe_config* cfg, const void* x, const int32_t* perm_src,
+                                 const int32_t* offsets, const void* w1, const void* w2, void* h,
+                                 void* y_perm, void* ws, moe_stream_t stream);
 
 /* Gate-weighted combine [Shazeer et al., "Methode": y = sum_i G(x)_i E_i(x)]:
  *   y[t] = sum_j topk_gate[t, j] * y_perm[slot_pos[t*k + j]]   (dropped slots add 0)
@@ -207,8 +242,19 @@ moe_status moe_expert_ffn_combine(const moe_config* cfg, const void* x_perm,
                                   const void* w1, const void* w2, void* h, void* y, void* ws,
                                   moe_stream_t stream);
 
-/* The whole layer forward on one stream: moe_route, moe_permute, moe_expert_ffn,
- * moe_combine (moe_expert_ffn_combine in their place when k = 1 and dtype is bf16).  Inputs as in the step calls; y [T, d_model] fp32 out.  topk_idx,
+/* moe_expert_ffn_combine with the permuted rows gathered from the token rows x (as
+ * moe_expert_ffn_gather does) instead of read from x_perm; k = 1 and bf16 only.
+ *  x [T, d_model] bf16 in; the other arguments as moe_expert_ffn_combine.  y is
+ *  bit-identical to moe_expert_ffn_combine's on x_perm. */
+moe_status moe_expert_ffn_combine_gather(const moe_config* cfg, const void* x,
+                                         const int32_t* offsets, const int32_t* perm_src,
+                                         const int32_t* slot_pos, const float* topk_gate,
+                                         const void* w1, const void* w2, void* h, void* y,
+                                         void* ws, moe_stream_t stream);
+
+/* The whole layer forward on one stream: moe_route, moe_permute (index arrays only),
+ * moe_expert_ffn_gather, moe_combine (moe_expert_ffn_combine_gather in place of the last
+ * two when k = 1 and dtype is bf16).  Inputs as in the step calls; y [T, d_model] fp32 out.  topk_idx,
  * topk_gate (both [T, k]) and counts ([E]) are outputs the caller must provide;
  * importance, load and near_tie may be NULL.  The intermediates live in `ws`
  * (moe_forward_workspace_size bytes). */
@@ -217,6 +263,60 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_gate,
                        const void* w1, const void* w2, void* y, int32_t* topk_idx,
                        float* topk_gate, int32_t* counts, float* importance, float* load,
                        uint8_t* near_tie, void* ws, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- training
+ * The backward pass of the layer for
+ *   L = sum(dy * y) + w_importance * CV(Importance(X))^2 + w_load * CV(Load(X))^2
+ * [Shazeer et al., "Load-Balancing-Losses": the auxiliary losses are weights times the
+ * squared coefficient of variation of Importance and Load; "Fragen": the top-k choice
+ * is taken before the softmax, so the chosen experts' gates keep continuous derivatives
+ * and gradients reach the gating network].  Which experts are chosen or dropped passes no
+ * gradient; the noise draws are inputs; CV uses the population standard deviation;
+ * kth_excluding passes its gradient to the entry of H it picks.  bf16 layers with the
+ * softmax or noisy gate only (others return MOE_ERR_UNSUPPORTED).  */
+
+/* Bytes of the forward state moe_forward_train writes and moe_backward reads (the kept
+ * rows, permutation, expert pre-activations, hidden activations and expert outputs of
+ * one batch); 0 for an unsupported cfg.  The layout is internal to the library. */
+size_t moe_train_state_size(const moe_config* cfg);
+
+/* Bytes of workspace moe_backward needs (the step workspace, whose device error word it
+ * shares, plus its own intermediates). */
+size_t moe_backward_workspace_size(const moe_config* cfg);
+
+/* moe_forward that also keeps what the backward pass needs in `state` (a device buffer of
+ * moe_train_state_size bytes, 16-byte aligned).  Same arguments and outputs as
+ * moe_forward; y is the same function of the inputs.  Pass importance (and load, for
+ * noisy gating) when the backward will weight their losses. */
+moe_status moe_forward_train(const moe_config* cfg, const void* x, const void* w_gate,
+                             const void* w_noise, const float* noise, const float* logit_bias,
+                             const void* w1, const void* w2, void* y, int32_t* topk_idx,
+                             float* topk_gate, int32_t* counts, float* importance, float* load,
+                             uint8_t* near_tie, void* state, void* ws, moe_stream_t stream);
+
+/* Gradients of L with respect to the layer's inputs and parameters.
+ *  x, w_gate, w_noise, noise, logit_bias, w1, w2: the inputs of the forward call
+ *  topk_idx, topk_gate, importance, load: its outputs; state: its saved state
+ *  dy          [T, d_model] fp32: dL/dy of the layer output
+ *  w_importance, w_load: loss weights (0 drops a term; w_load needs noisy gating, k < E)
+ *  dx          [T, d_model] fp32 out
+ *  dw_gate     [E, d_model] fp32 out; dw_noise [E, d_model] fp32 out (noisy gating)
+ *  dlogit_bias [E] fp32 out or NULL
+ *  dw1         [E, d_ff, d_model] fp32 out; dw2 [E, d_model, d_ff] fp32 out
+ *  dgates      [T, k] fp32 out: dL/d of each chosen gate from the layer output (0 where
+ *              the assignment was dropped)
+ *  losses      [2] fp32 out or NULL: w_importance CV^2 and w_load CV^2
+ *  ws          moe_backward_workspace_size bytes
+ * The expert products run on the tensor cores in bf16 with fp32 accumulation (the
+ * upstream gradient of each expert row is rounded to bf16, or fp16 with hidden_f16);
+ * the router's gradients are fp32. */
+moe_status moe_backward(const moe_config* cfg, const void* x, const void* w_gate,
+                        const void* w_noise, const float* noise, const float* logit_bias,
+                        const void* w1, const void* w2, const int32_t* topk_idx,
+                        const float* topk_gate, const float* importance, const float* load,
+                        const void* state, const float* dy, float w_importance, float w_load,
+                        float* dx, float* dw_gate, float* dw_noise, float* dlogit_bias, float* dw1,
+                        float* dw2, float* dgates, float* losses, void* ws, moe_stream_t stream);
 
 /* Synchronises `stream`, then reads the device error word in `ws` into *device_error
  * (may be NULL) and clears it.  Returns MOE_OK if no bit was set, MOE_ERR_DEVICE if

@@ -39,12 +39,19 @@ def _load():
         "moe_expert_ffn": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
         "moe_combine": (ctypes.c_int, [C, P, P, P, P, P, P]),
         "moe_expert_ffn_combine": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P]),
+        "moe_expert_ffn_gather": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P]),
+        "moe_expert_ffn_combine_gather": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P]),
         "moe_forward": (ctypes.c_int, [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]),
         "moe_get_error": (ctypes.c_int, [P, P, ctypes.POINTER(ctypes.c_int32)]),
         "moe_last_launch_count": (ctypes.c_int32, []),
         "moe_bf16_to_f16": (ctypes.c_int, [P, P, ctypes.c_int64, P, P]),
         "moe_permute_noalloc": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
         "moe_erf_check": (ctypes.c_int, [P, P, P, ctypes.c_int64, P]),
+        "moe_train_state_size": (ctypes.c_size_t, [C]),
+        "moe_backward_workspace_size": (ctypes.c_size_t, [C]),
+        "moe_forward_train": (ctypes.c_int, [C] + [P] * 17),
+        "moe_backward": (ctypes.c_int, [C] + [P] * 14 + [ctypes.c_float, ctypes.c_float] +
+                         [P] * 10),
         "moe_wait_timeout_check": (ctypes.c_int, [P, P]),
     }
     for name, (res, args) in sig.items():
@@ -112,6 +119,7 @@ def moe_route(cfg, x, w_gate, topk_idx, topk_gate, ws, w_noise=None, noise=None,
 
 
 def moe_permute(cfg, topk_idx, x, counts, offsets, perm_src, slot_pos, x_perm, ws, stream=None):
+    """x_perm (and x) may be None: only the index arrays are written."""
     _check(lib.moe_permute(ctypes.byref(cfg), _ptr(topk_idx, "topk_idx"), _ptr(x, "x"),
                            _ptr(counts, "counts"), _ptr(offsets, "offsets"),
                            _ptr(perm_src, "perm_src"), _ptr(slot_pos, "slot_pos"),
@@ -135,6 +143,24 @@ def moe_expert_ffn(cfg, x_perm, offsets, w1, w2, h, y_perm, ws, stream=None):
                               _ptr(w1, "w1"), _ptr(w2, "w2"), _ptr(h, "h"),
                               _ptr(y_perm, "y_perm"), _ptr(ws, "ws"), _stream(stream)),
            "moe_expert_ffn")
+
+
+def moe_expert_ffn_gather(cfg, x, perm_src, offsets, w1, w2, h, y_perm, ws, stream=None):
+    """moe_expert_ffn with permuted row s gathered from x[perm_src[s] // k] by the kernel."""
+    _check(lib.moe_expert_ffn_gather(ctypes.byref(cfg), _ptr(x, "x"), _ptr(perm_src, "perm_src"),
+                                     _ptr(offsets, "offsets"), _ptr(w1, "w1"), _ptr(w2, "w2"),
+                                     _ptr(h, "h"), _ptr(y_perm, "y_perm"), _ptr(ws, "ws"),
+                                     _stream(stream)), "moe_expert_ffn_gather")
+
+
+def moe_expert_ffn_combine_gather(cfg, x, offsets, perm_src, slot_pos, topk_gate, w1, w2, h, y,
+                                  ws, stream=None):
+    """moe_expert_ffn_combine with the permuted rows gathered from x (k = 1, bf16)."""
+    _check(lib.moe_expert_ffn_combine_gather(
+        ctypes.byref(cfg), _ptr(x, "x"), _ptr(offsets, "offsets"), _ptr(perm_src, "perm_src"),
+        _ptr(slot_pos, "slot_pos"), _ptr(topk_gate, "topk_gate"), _ptr(w1, "w1"), _ptr(w2, "w2"),
+        _ptr(h, "h"), _ptr(y, "y"), _ptr(ws, "ws"), _stream(stream)),
+        "moe_expert_ffn_combine_gather")
 
 
 def moe_combine(cfg, y_perm, slot_pos, topk_gate, y, ws, stream=None):
@@ -169,6 +195,52 @@ def moe_forward(cfg, x, w_gate, w1, w2, y, topk_idx, topk_gate, counts, ws, w_no
                            _ptr(counts, "counts"), _ptr(importance, "importance"),
                            _ptr(load, "load"), _ptr(near_tie, "near_tie"), _ptr(ws, "ws"),
                            _stream(stream)), "moe_forward")
+
+
+def train_state(cfg, device="cuda") -> torch.Tensor:
+    """A device buffer for the forward state moe_forward_train keeps for moe_backward."""
+    n = int(lib.moe_train_state_size(ctypes.byref(cfg)))
+    if n == 0:
+        raise MoEError(2, "config unsupported by the training path")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def backward_workspace(cfg, device="cuda") -> torch.Tensor:
+    """A zero-filled device workspace for moe_backward (its error word included)."""
+    n = int(lib.moe_backward_workspace_size(ctypes.byref(cfg)))
+    if n == 0:
+        raise MoEError(2, "config unsupported by the training path")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def moe_forward_train(cfg, x, w_gate, w1, w2, y, topk_idx, topk_gate, counts, state, ws,
+                      w_noise=None, noise=None, logit_bias=None, importance=None, load=None,
+                      near_tie=None, stream=None):
+    _check(lib.moe_forward_train(ctypes.byref(cfg), _ptr(x, "x"), _ptr(w_gate, "w_gate"),
+                                 _ptr(w_noise, "w_noise"), _ptr(noise, "noise"),
+                                 _ptr(logit_bias, "logit_bias"), _ptr(w1, "w1"), _ptr(w2, "w2"),
+                                 _ptr(y, "y"), _ptr(topk_idx, "topk_idx"),
+                                 _ptr(topk_gate, "topk_gate"), _ptr(counts, "counts"),
+                                 _ptr(importance, "importance"), _ptr(load, "load"),
+                                 _ptr(near_tie, "near_tie"), _ptr(state, "state"), _ptr(ws, "ws"),
+                                 _stream(stream)), "moe_forward_train")
+
+
+def moe_backward(cfg, x, w_gate, w1, w2, topk_idx, topk_gate, state, dy, dx, dw_gate, dw1, dw2,
+                 dgates, ws, w_noise=None, noise=None, logit_bias=None, importance=None,
+                 load=None, w_importance=0.0, w_load=0.0, dw_noise=None, dlogit_bias=None,
+                 losses=None, stream=None):
+    _check(lib.moe_backward(ctypes.byref(cfg), _ptr(x, "x"), _ptr(w_gate, "w_gate"),
+                            _ptr(w_noise, "w_noise"), _ptr(noise, "noise"),
+                            _ptr(logit_bias, "logit_bias"), _ptr(w1, "w1"), _ptr(w2, "w2"),
+                            _ptr(topk_idx, "topk_idx"), _ptr(topk_gate, "topk_gate"),
+                            _ptr(importance, "importance"), _ptr(load, "load"),
+                            _ptr(state, "state"), _ptr(dy, "dy"), float(w_importance),
+                            float(w_load), _ptr(dx, "dx"), _ptr(dw_gate, "dw_gate"),
+                            _ptr(dw_noise, "dw_noise"), _ptr(dlogit_bias, "dlogit_bias"),
+                            _ptr(dw1, "dw1"), _ptr(dw2, "dw2"), _ptr(dgates, "dgates"),
+                            _ptr(losses, "losses"), _ptr(ws, "ws"), _stream(stream)),
+           "moe_backward")
 
 
 def moe_get_error(ws: torch.Tensor, stream=None) -> int:
@@ -240,4 +312,6 @@ __all__ = ["ACT", "DTYPE", "GATING", "MoEConfig", "MoEError", "MoELayer", "STATU
            "make_config", "moe_capacity", "moe_combine", "moe_expert_ffn", "moe_forward",
            "moe_forward_workspace_size", "moe_get_error", "moe_permute", "moe_route",
            "moe_workspace_size", "workspace", "last_launch_count", "moe_bf16_to_f16",
-           "prepare_weights", "moe_permute_noalloc", "moe_expert_ffn_combine", "fused_combine"]
+           "prepare_weights", "moe_permute_noalloc", "moe_expert_ffn_combine", "fused_combine",
+           "moe_expert_ffn_gather", "moe_expert_ffn_combine_gather", "train_state",
+           "backward_workspace", "moe_forward_train", "moe_backward"]

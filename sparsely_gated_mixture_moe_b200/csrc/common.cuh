@@ -111,6 +111,21 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Four rows of a 2-D tensor, each one box of [1 row x box-width columns] at column x,
+// gathered into consecutive rows of this CTA's shared memory (TMA tile::gather4); rows
+// r0..r3 may be any rows of the tensor, in any order.  The tensor map's box is one row
+// high.  With 128-byte swizzling the rows land where a tiled load of rows (dst / 128)
+// mod 8 ... of a 1024-byte-aligned tile would put them, so a 4-row group at a 512-byte
+// offset of such a tile fits the tile's layout.  No multicast.
+__device__ __forceinline__ void tma_gather4_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                               int x, int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+
 // ----------------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t holder_smem, uint32_t ncols) {
@@ -176,6 +191,28 @@ __device__ __forceinline__ uint64_t sdesc_k128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor of an MN-major operand tile written by TMA with 128-byte
+// swizzling (the operand's M or N index is the contiguous one, as for a row-major [K, N]
+// weight read as B = W^T): the tile is a run of chunks of 64 MN-elements, each chunk
+// [K rows x 128 B] from one TMA box, K rows 128 B apart, 8-row groups 1024 B apart
+// (stride offset), chunks `chunk_bytes` apart (leading offset).  Advancing K by 16 rows
+// adds 2048 bytes to the start address.
+__device__ __forceinline__ uint64_t sdesc_mn128(uint32_t saddr, uint32_t chunk_bytes) {
+  uint64_t d = static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((chunk_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+// idesc_f32acc with the major order of each operand: bit 15 set when A is M-major, bit 16
+// when B is N-major.
+__host__ __device__ constexpr uint32_t idesc_f32acc_major(int M, int N, uint32_t ab_fmt, bool a_mn,
+                                                          bool b_mn) {
+  return idesc_f32acc(M, N, ab_fmt) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u);
+}
+
 // Each thread of the warp reads 32 consecutive fp32 columns of its own TMEM lane
 // (the warp's lane quarter is fixed by its warp index modulo 4).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -209,6 +246,94 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------- CTA pairs (clusters of two CTAs)
+//
+// The two CTAs of a cluster share one tensor-core product of M = 256 rows
+// (tcgen05 cta_group::2): each holds half of A (its 128 rows) and half of B in its own
+// shared memory and gets its 128 rows of D in its own TMEM.  Every tcgen05 instruction of
+// a kernel that does this uses cta_group::2.
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address in the shared::cluster window of the object at shared::cta address `addr` in the
+// cluster's CTA of rank `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// Barrier over all threads of both CTAs of the cluster (release / acquire).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+
+// Arrive on an mbarrier given by its shared::cluster address (possibly the peer CTA's).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+               : "memory");
+}
+
+// As tma_load_2d, into this CTA's shared memory, with completion signalled on `bar`, a
+// shared::cluster address that may be the peer CTA's mbarrier.  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+// As tma_gather4_2d, with completion signalled on a shared::cluster mbarrier address that
+// may be the peer CTA's.  No multicast.
+__device__ __forceinline__ void tma_gather4_2d_pair(uint32_t dst, const CUtensorMap* map,
+                                                    uint32_t bar, int x, int r0, int r1, int r2,
+                                                    int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+
+// TMEM allocation shared by the pair: a warp of the same index in each CTA runs it.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t holder_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(holder_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+// Arrive once on the mbarrier at shared::cluster address `bar` (this CTA's or the peer's)
+// when every tcgen05 operation this thread issued so far is done.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+// D[tmem] (+)= A * B^T over the pair: M = 256 (128 rows of A and D in each CTA), B split
+// by N between the CTAs; the descriptors name the same shared-memory offsets in both.
+__device__ __forceinline__ void tc_mma_pair_f16kind(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                    uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 // --------------------------------------------------------------------- utilities

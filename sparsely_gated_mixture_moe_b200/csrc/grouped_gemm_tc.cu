@@ -32,6 +32,7 @@
 // kErrTimeout, drains this CTA's in-flight copies and MMAs and frees TMEM.
 #include <cudaTypedefs.h>
 
+#include <map>
 #include <mutex>
 
 #include "common.cuh"
@@ -76,6 +77,10 @@ struct Args {
   const int32_t* perm_src;  // OUT_COMBINE: assignment of each permuted row (= token, k = 1)
   const float* gate;        // OUT_COMBINE: gate of each assignment
   const int32_t* slot_pos;  // OUT_COMBINE: permuted row of each token, < 0 when dropped
+  const int32_t* gather_src;  // non-null: A row s is row gather_src[s] / gather_k of the
+  int gather_k;               // A tensor (the token rows x), gathered by the TMA itself
+  void* pre;                  // OUT_BF16 / OUT_F16 with an activation: also store the
+                              // pre-activation there (same type and layout as out), or null
   int* err;
 };
 
@@ -83,7 +88,9 @@ struct Tile {
   int e, mt, nt, row0, valid;
 };
 
-__device__ __forceinline__ Tile decode_tile(int L, const int* tp, const Args& a) {
+// Tile L of the (expert, m-tile, n-tile) list, m-tiles of bm rows: row0 is the tile's
+// first permuted row, valid its rows that belong to the expert (>= 1).
+__device__ __forceinline__ Tile decode_tile(int L, const int* tp, const Args& a, int bm) {
   // expert: the largest e with tp[e] * n_tiles <= L
   int lo = 0, hi = a.E - 1;
   while (lo < hi) {
@@ -96,8 +103,8 @@ __device__ __forceinline__ Tile decode_tile(int L, const int* tp, const Args& a)
   t.mt = local / a.n_tiles;
   t.nt = local - t.mt * a.n_tiles;
   const int r0 = __ldg(a.offsets + lo), r1 = __ldg(a.offsets + lo + 1);
-  t.row0 = r0 + t.mt * BM;
-  t.valid = min(BM, r1 - t.row0);
+  t.row0 = r0 + t.mt * bm;
+  t.valid = min(bm, r1 - t.row0);
   return t;
 }
 
@@ -130,6 +137,17 @@ __device__ __forceinline__ void epilogue_rows(const Args& a, uint32_t tbase, int
                              __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
     } else {
       uint32_t pk[16];
+      if (a.pre != nullptr) {  // the pre-activation, for the backward pass
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float z0 = __uint_as_float(v[2 * j]), z1 = __uint_as_float(v[2 * j + 1]);
+          pk[j] = MODE == OUT_F16 ? pack_f16x2(z0, z1) : pack_bf16x2(z0, z1);
+        }
+        uint4* pdst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.pre) + oidx + c);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          pdst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+      }
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const float x0 = epi_act<ACT>(__uint_as_float(v[2 * j]));
@@ -144,6 +162,15 @@ __device__ __forceinline__ void epilogue_rows(const Args& a, uint32_t tbase, int
   }
 }
 
+// PAIR = false: one CTA per SM, 128-row tiles, tcgen05 cta_group::1.
+// PAIR = true: clusters of two CTAs on the two SMs of a pair share 256-row tiles
+// (tcgen05 cta_group::2, M = 256): CTA rank r loads rows [row0 + 128 r, +128) of A and
+// rows [n0 + r bn/2, +bn/2) of the B tile into its own shared memory, with the copies of
+// both CTAs completing on the rank-0 CTA's full barrier; one thread of rank 0 issues the
+// MMAs and commits their completion to both CTAs' barriers; each CTA's epilogue reads its
+// own 128 TMEM lanes and both arrive on rank 0's accumulator-empty barrier.  Each SM then
+// streams half of the B tile per k-block instead of all of it.
+template <bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmB, const Args a) {
@@ -165,6 +192,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   int* tp = scratch + 40;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  constexpr int TBM = PAIR ? 2 * BM : BM;  // rows of one tile (of the pair)
+  const int first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int stride = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -173,7 +204,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
-      mbar_init(tempty0 + 8 * b, EPI_WARPS);
+      mbar_init(tempty0 + 8 * b, PAIR ? 2 * EPI_WARPS : EPI_WARPS);
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -184,40 +215,120 @@ __global__ void __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_holder), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   grid_dep_wait();  // offsets and A come from the previous kernels on the stream
   grid_dep_launch();
-  const bool ok = block_tile_prefix(a.offsets, a.E, a.rows_cap, BM, tp, scratch);
-  if (!ok && threadIdx.x == 0) set_error(a.err, kErrOffsets);
+  const bool ok = block_tile_prefix(a.offsets, a.E, a.rows_cap, TBM, tp, scratch);
+  if (!ok && threadIdx.x == 0 && rank == 0) set_error(a.err, kErrOffsets);
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int total = ok ? tp[a.E] * a.n_tiles : 0;
   const int kblocks = a.K / BK;
-  const uint32_t b_bytes = static_cast<uint32_t>(a.bn) * BK * 2;
+  const int b_rows = PAIR ? a.bn / 2 : a.bn;  // rows of the B tile this CTA loads
+  const uint32_t b_bytes = static_cast<uint32_t>(b_rows) * BK * 2;
+  const uint32_t stage_tx = (PAIR ? 2u : 1u) * (A_BYTES + b_bytes);  // bytes per full phase
+  // the full barrier every copy of a stage completes on: rank 0's in a pair
+  auto full_bar = [&](int stage) -> uint32_t {
+    return PAIR ? mapa_shared(full0 + 8 * stage, 0) : full0 + 8 * stage;
+  };
 
-  if (warp == 0) {
+  if (warp == 0 && a.gather_src != nullptr) {
+    // ------------------------------------------------- TMA producer, gathered A rows
+    // The A operand of permuted row s is token row gather_src[s] / gather_k of x: lane l
+    // fetches rows 4l .. 4l+3 of this CTA's 128 rows with one tile::gather4 per k-block
+    // (the same 512 bytes a tiled load of the permuted rows would place there).  Rows
+    // past the expert's end repeat its last row; they only feed masked output rows.
+    int stage = 0;
+    uint32_t phase = 0, armed = 0, armed_par = 0;
+    bool aborted = false;
+    int cur_row0 = -1;
+    int g0 = 0, g1 = 0, g2 = 0, g3 = 0;
+    for (int L = first; L < total && !aborted; L += stride) {
+      const Tile t = decode_tile(L, tp, a, TBM);
+      if (t.row0 != cur_row0) {  // n-tiles of one m-tile are consecutive: gather once
+        cur_row0 = t.row0;
+        const int last = t.valid - 1;
+        const int r = static_cast<int>(rank) * BM + 4 * lane;
+        g0 = __ldg(a.gather_src + t.row0 + min(r + 0, last)) / a.gather_k;
+        g1 = __ldg(a.gather_src + t.row0 + min(r + 1, last)) / a.gather_k;
+        g2 = __ldg(a.gather_src + t.row0 + min(r + 2, last)) / a.gather_k;
+        g3 = __ldg(a.gather_src + t.row0 + min(r + 3, last)) / a.gather_k;
+      }
+      const int brow = t.e * a.N + t.nt * a.bn + static_cast<int>(rank) * b_rows;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        int okw = 1;
+        if (lane == 0) okw = mbar_wait(empty0 + 8 * stage, phase ^ 1, s_abort) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, okw, 0)) {
+          aborted = true;
+          break;
+        }
+        uint8_t* st = ring + stage * STAGE_BYTES;
+        const uint32_t fb = full_bar(stage);
+        if (lane == 0 && rank == 0) mbar_arrive_expect_tx(full0 + 8 * stage, stage_tx);
+        __syncwarp();
+        if constexpr (PAIR) {
+          tma_gather4_2d_pair(smem_u32(st) + 512u * lane, &tmA, fb, kb * BK, g0, g1, g2, g3);
+          if (lane == 0) tma_load_2d_pair(smem_u32(st + A_BYTES), &tmB, fb, kb * BK, brow);
+        } else {
+          tma_gather4_2d(smem_u32(st) + 512u * lane, &tmA, fb, kb * BK, g0, g1, g2, g3);
+          if (lane == 0) tma_load_2d(smem_u32(st + A_BYTES), &tmB, fb, kb * BK, brow);
+        }
+        armed |= 1u << stage;
+        armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (aborted && lane == 0) {
+      set_error(a.err, kErrTimeout);
+      *s_abort = 1;
+      // let every copy this warp started land before the CTA releases its smem (a pair's
+      // second CTA cannot watch rank 0's barrier: it waits out a fixed drain time)
+      if (rank == 0) {
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s)) mbar_wait(full0 + 8 * s, (armed_par >> s) & 1, nullptr, kDrainLimitNs);
+      } else {
+        const unsigned long long t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < kDrainLimitNs / 4) __nanosleep(1000);
+      }
+    }
+  } else if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_par = 0;
       bool aborted = false;
-      for (int L = blockIdx.x; L < total && !aborted; L += gridDim.x) {
-        const Tile t = decode_tile(L, tp, a);
-        const int brow = t.e * a.N + t.nt * a.bn;
+      for (int L = first; L < total && !aborted; L += stride) {
+        const Tile t = decode_tile(L, tp, a, TBM);
+        const int brow = t.e * a.N + t.nt * a.bn + static_cast<int>(rank) * b_rows;
+        const int arow = t.row0 + static_cast<int>(rank) * BM;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, s_abort)) {
             aborted = true;
             break;
           }
           uint8_t* st = ring + stage * STAGE_BYTES;
-          const uint32_t fb = full0 + 8 * stage;
-          mbar_arrive_expect_tx(fb, A_BYTES + b_bytes);
-          tma_load_2d(smem_u32(st), &tmA, fb, kb * BK, t.row0);
-          tma_load_2d(smem_u32(st + A_BYTES), &tmB, fb, kb * BK, brow);
+          const uint32_t fb = full_bar(stage);
+          if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * stage, stage_tx);
+          if constexpr (PAIR) {
+            tma_load_2d_pair(smem_u32(st), &tmA, fb, kb * BK, arow);
+            tma_load_2d_pair(smem_u32(st + A_BYTES), &tmB, fb, kb * BK, brow);
+          } else {
+            tma_load_2d(smem_u32(st), &tmA, fb, kb * BK, arow);
+            tma_load_2d(smem_u32(st + A_BYTES), &tmB, fb, kb * BK, brow);
+          }
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -230,18 +341,23 @@ __global__ void __launch_bounds__(THREADS, 1)
         set_error(a.err, kErrTimeout);
         *s_abort = 1;
         // let every copy this thread started land before the CTA releases its smem
-        for (int s = 0; s < STAGES; ++s)
-          if (armed & (1u << s)) mbar_wait(full0 + 8 * s, (armed_par >> s) & 1, nullptr, kDrainLimitNs);
+        if (rank == 0) {
+          for (int s = 0; s < STAGES; ++s)
+            if (armed & (1u << s)) mbar_wait(full0 + 8 * s, (armed_par >> s) & 1, nullptr, kDrainLimitNs);
+        } else {
+          const unsigned long long t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < kDrainLimitNs / 4) __nanosleep(1000);
+        }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       // ------------------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_f32acc(BM, a.bn, a.ab_f16 ? kFmtF16 : kFmtBF16);
+      const uint32_t idesc = idesc_f32acc(TBM, a.bn, a.ab_f16 ? kFmtF16 : kFmtBF16);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool aborted = false;
-      for (int L = blockIdx.x; L < total && !aborted; L += gridDim.x) {
+      for (int L = first; L < total && !aborted; L += stride) {
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1, s_abort)) {
           aborted = true;
           break;
@@ -257,24 +373,41 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t a0 = smem_u32(ring + stage * STAGE_BYTES);
           const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            tc_mma_f16kind(d_tmem, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32), idesc,
-                           (kb | kk) != 0 ? 1u : 0u);
-          tc_commit(empty0 + 8 * stage);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            if constexpr (PAIR)
+              tc_mma_pair_f16kind(d_tmem, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32), idesc,
+                                  (kb | kk) != 0 ? 1u : 0u);
+            else
+              tc_mma_f16kind(d_tmem, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32), idesc,
+                             (kb | kk) != 0 ? 1u : 0u);
+          }
+          if constexpr (PAIR) {  // both CTAs' stages are free once these MMAs are done
+            tc_commit_pair(mapa_shared(empty0 + 8 * stage, 0));
+            tc_commit_pair(mapa_shared(empty0 + 8 * stage, 1));
+          } else {
+            tc_commit(empty0 + 8 * stage);
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (aborted) break;
-        tc_commit(tfull0 + 8 * acc);
+        if constexpr (PAIR) {
+          tc_commit_pair(mapa_shared(tfull0 + 8 * acc, 0));
+          tc_commit_pair(mapa_shared(tfull0 + 8 * acc, 1));
+        } else {
+          tc_commit(tfull0 + 8 * acc);
+        }
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1;
       }
       if (aborted) {
         set_error(a.err, kErrTimeout);
         *s_abort = 1;
-        tc_commit(drain);  // wait for the MMAs already issued before TMEM is freed
+        // wait for the MMAs already issued before TMEM is freed
+        if constexpr (PAIR) tc_commit_pair(mapa_shared(drain, 0));
+        else tc_commit(drain);
         mbar_wait(drain, 0, nullptr, kDrainLimitNs);
       }
     }
@@ -287,9 +420,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       // y = 0 for tokens whose only assignment was dropped (no tile writes them); done
       // while the first tile's operands stream in
       const int ew = warp - 2;
-      const int64_t stride = static_cast<int64_t>(gridDim.x) * EPI_WARPS * 32;
+      const int64_t gstride = static_cast<int64_t>(gridDim.x) * EPI_WARPS * 32;
       for (int64_t b = (static_cast<int64_t>(blockIdx.x) * EPI_WARPS + ew) * 32; b < a.rows_cap;
-           b += stride) {
+           b += gstride) {
         const bool drop = b + lane < a.rows_cap && __ldg(a.slot_pos + b + lane) < 0;
         uint32_t m = __ballot_sync(0xffffffffu, drop);
         while (m) {
@@ -300,10 +433,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
+    const uint32_t tempty_peer0 = PAIR ? mapa_shared(tempty0, 0) : tempty0;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x) {
-      const Tile t = decode_tile(L, tp, a);
+    for (int L = first; L < total; L += stride) {
+      const Tile t = decode_tile(L, tp, a, TBM);
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, s_abort)) {
         if (lane == 0) set_error(a.err, kErrTimeout);
         *s_abort = 1;
@@ -311,8 +445,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_after();
       const int r = q * 32 + lane;
-      bool row_ok = r < t.valid;
-      int64_t orow = t.row0 + r;
+      const int crow = static_cast<int>(rank) * BM + r;  // row within the (pair's) tile
+      bool row_ok = crow < t.valid;
+      int64_t orow = t.row0 + crow;
       float scale = 1.0f;
       if (a.out_mode == OUT_COMBINE && row_ok) {
         // k = 1: the permuted row's assignment is its token; y[t] = g_t * (h W2^T)[row]
@@ -340,16 +475,26 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(tempty_peer0 + 8 * acc);
+        else mbar_arrive(tempty0 + 8 * acc);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
   }
 
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
+  // a pair's CTAs leave together: rank 0's MMAs read the other CTA's shared memory and
+  // the other CTA's epilogue arrives on rank 0's barriers
+  if constexpr (PAIR) cluster_sync_all();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == 1) {
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
+  }
 }
 
 }  // namespace gg
@@ -392,14 +537,62 @@ static int pick_bn(int N) {
   return 64;
 }
 
+// Experts with at least this many rows on average (T*k / E, counted before capacity
+// drops) run on CTA pairs (256-row tiles, cta_group::2); fewer rows per expert would
+// leave most of each 256-row tile empty.
+constexpr int64_t kPairMinRowsPerExpert = 256;
+
+// Clusters of two CTAs of grouped_gemm_tc_kernel<true> that fit on the device at once (a
+// persistent grid larger than that would serialise), looked up once per context.
+static int max_active_pairs(const LaunchCtx& c) {
+  static std::mutex mu;
+  static std::map<unsigned long long, int> cache;
+  unsigned long long ctx = 0;
+  if (current_context_id(&ctx) != cudaSuccess) return c.num_sms / 2;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(ctx);
+  if (it != cache.end()) return it->second;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (c.num_sms / 2));
+  cfg.blockDim = dim3(gg::THREADS);
+  cfg.dynamicSmemBytes = gg::SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gg::grouped_gemm_tc_kernel<true>, &cfg) != cudaSuccess ||
+      n <= 0)
+    n = c.num_sms / 2;
+  if (n > c.num_sms / 2) n = c.num_sms / 2;
+  cache[ctx] = n;
+  return n;
+}
+
+// A: the permuted rows [rows_cap, K], or with gather_src the token rows [a_rows, K] that
+// permuted row s reads at row gather_src[s] / gather_k.
 static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void* B, int E, int N,
                               int ab_f16, void* out, int out_mode, const int32_t* offsets, int act,
                               const LaunchCtx& c, const int32_t* perm_src = nullptr,
-                              const float* gate = nullptr, const int32_t* slot_pos = nullptr) {
+                              const float* gate = nullptr, const int32_t* slot_pos = nullptr,
+                              const int32_t* gather_src = nullptr, int gather_k = 1,
+                              int64_t a_rows = 0, void* pre = nullptr) {
   const int bn = pick_bn(N);
+  const bool pair = rows_cap >= kPairMinRowsPerExpert * E;
   CUtensorMap tmA, tmB;
-  if (!make_tmap_2b(&tmA, A, static_cast<uint64_t>(rows_cap), K, gg::BM, ab_f16)) return cudaErrorInvalidValue;
-  if (!make_tmap_2b(&tmB, B, static_cast<uint64_t>(E) * N, K, bn, ab_f16)) return cudaErrorInvalidValue;
+  if (gather_src != nullptr) {
+    // one-row boxes for tile::gather4
+    if (a_rows <= 0 || !make_tmap_2b(&tmA, A, static_cast<uint64_t>(a_rows), K, 1, ab_f16))
+      return cudaErrorInvalidValue;
+  } else if (!make_tmap_2b(&tmA, A, static_cast<uint64_t>(rows_cap), K, gg::BM, ab_f16)) {
+    return cudaErrorInvalidValue;
+  }
+  // a pair's CTA loads half of each B tile
+  if (!make_tmap_2b(&tmB, B, static_cast<uint64_t>(E) * N, K, pair ? bn / 2 : bn, ab_f16))
+    return cudaErrorInvalidValue;
   gg::Args a;
   a.offsets = offsets;
   a.E = E;
@@ -415,15 +608,40 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
   a.perm_src = perm_src;
   a.gate = gate;
   a.slot_pos = slot_pos;
+  a.gather_src = gather_src;
+  a.gather_k = gather_k;
+  a.pre = pre;
   a.err = c.err;
-  // upper bound of the tile count: sum_e ceil(n_e / BM) <= rows_cap / BM + E
-  const int64_t max_tiles = (rows_cap / gg::BM + E) * static_cast<int64_t>(a.n_tiles);
+  // upper bound of the tile count: sum_e ceil(n_e / bm) <= rows_cap / bm + E
+  const int tbm = pair ? 2 * gg::BM : gg::BM;
+  const int64_t max_tiles = (rows_cap / tbm + E) * static_cast<int64_t>(a.n_tiles);
+  if (pair) {
+    cudaError_t e = ensure_smem_limit(gg::grouped_gemm_tc_kernel<true>, gg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    const int64_t pairs_cap = max_active_pairs(c);
+    const int pairs = static_cast<int>(max_tiles < pairs_cap ? max_tiles : pairs_cap);
+    if (pairs <= 0) return cudaSuccess;
+    return launch_kernel_pairs(gg::grouped_gemm_tc_kernel<true>, dim3(2 * pairs), dim3(gg::THREADS),
+                               gg::SMEM_BYTES, c, tmA, tmB, a);
+  }
   const int grid = static_cast<int>(max_tiles < c.num_sms ? max_tiles : c.num_sms);
   if (grid <= 0) return cudaSuccess;
-  cudaError_t e = ensure_smem_limit(gg::grouped_gemm_tc_kernel, gg::SMEM_BYTES);
+  cudaError_t e = ensure_smem_limit(gg::grouped_gemm_tc_kernel<false>, gg::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  return launch_kernel(gg::grouped_gemm_tc_kernel, dim3(grid), dim3(gg::THREADS), gg::SMEM_BYTES, c,
-                       tmA, tmB, a);
+  return launch_kernel(gg::grouped_gemm_tc_kernel<false>, dim3(grid), dim3(gg::THREADS),
+                       gg::SMEM_BYTES, c, tmA, tmB, a);
+}
+
+// The up-projection h = act(A . W1^T): A is x_perm, or the token rows x gathered by the
+// TMA through gather_src (no x_perm).
+static cudaError_t launch_up(const FfnProblem& p, const LaunchCtx& c) {
+  const int hf = p.hidden_f16 ? 1 : 0;
+  const int mode = hf ? gg::OUT_F16 : gg::OUT_BF16;
+  if (p.gather_src != nullptr)
+    return launch_one(p.x, p.rows_cap, p.d, p.w1, p.E, p.f, 0, p.h, mode, p.offsets, p.act, c,
+                      nullptr, nullptr, nullptr, p.gather_src, p.k, p.x_rows, p.u);
+  return launch_one(p.x_perm, p.rows_cap, p.d, p.w1, p.E, p.f, 0, p.h, mode, p.offsets, p.act, c,
+                    nullptr, nullptr, nullptr, nullptr, 1, 0, p.u);
 }
 
 cudaError_t launch_ffn_combine_bf16(const FfnProblem& p, const int32_t* perm_src,
@@ -431,8 +649,7 @@ cudaError_t launch_ffn_combine_bf16(const FfnProblem& p, const int32_t* perm_src
                                     const LaunchCtx& c) {
   if (p.E > gg::MAX_GROUPS) return cudaErrorInvalidValue;
   const int hf = p.hidden_f16 ? 1 : 0;
-  cudaError_t e = launch_one(p.x_perm, p.rows_cap, p.d, p.w1, p.E, p.f, 0, p.h, hf ? gg::OUT_F16 : gg::OUT_BF16,
-                 p.offsets, p.act, c);
+  cudaError_t e = launch_up(p, c);
   if (e != cudaSuccess) return e;
   return launch_one(p.h, p.rows_cap, p.f, p.w2, p.E, p.d, hf, y, gg::OUT_COMBINE, p.offsets, 0, c,
                     perm_src, gate, slot_pos);
@@ -441,8 +658,7 @@ cudaError_t launch_ffn_combine_bf16(const FfnProblem& p, const int32_t* perm_src
 cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c) {
   if (p.E > gg::MAX_GROUPS) return cudaErrorInvalidValue;
   const int hf = p.hidden_f16 ? 1 : 0;
-  cudaError_t e = launch_one(p.x_perm, p.rows_cap, p.d, p.w1, p.E, p.f, 0, p.h,
-                             hf ? gg::OUT_F16 : gg::OUT_BF16, p.offsets, p.act, c);
+  cudaError_t e = launch_up(p, c);
   if (e != cudaSuccess) return e;
   return launch_one(p.h, p.rows_cap, p.f, p.w2, p.E, p.d, hf, p.y_perm, gg::OUT_F32, p.offsets, 0, c);
 }

@@ -72,11 +72,36 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
   return e;
 }
 
+// As launch_kernel, for a kernel whose CTAs run in clusters of two (grid.x even): the two
+// CTAs of a cluster are co-scheduled on a pair of SMs and share a tensor-core product.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel_pairs(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                const LaunchCtx& c, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = c.stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  ++*c.launches;
+  return e;
+}
+
 // ---- route -----------------------------------------------------------------------
 struct RouteProblem {
   int64_t T;
   int d, E, k;
   int noisy, renorm;
+  int hier = 0, groups = 0, k_primary = 0;  // hierarchical gating: w_gate has groups + E rows
   const void* x;
   const void* w_gate;
   const void* w_noise;
@@ -88,7 +113,7 @@ struct RouteProblem {
   float* importance;  // may be null
   float* load;        // may be null
   float* partials;    // workspace: [route_blocks][2][E]
-  float* logits_ws;   // fp32 path only: [T][E]
+  float* logits_ws;   // fp32 path only: [T][E] ([T][groups + E] for hierarchical gating)
   float* nz_ws;       // fp32 path only: [T][E]
 };
 int route_blocks(int64_t T);
@@ -123,7 +148,12 @@ struct FfnProblem {
   int64_t rows_cap;  // T*k
   int d, f, E, act;  // act: 1 ReLU, 2 GELU
   int hidden_f16;    // bf16 path: h stored in fp16 and w2 given in fp16
-  const void* x_perm;
+  const void* x_perm;  // permuted rows, or null when gather_src is given
+  const void* x = nullptr;              // token rows [x_rows, d] (gather mode)
+  const int32_t* gather_src = nullptr;  // permuted row s reads x[gather_src[s] / k]
+  int64_t x_rows = 0;
+  int k = 1;
+  void* u = nullptr;                    // bf16 path: also store the pre-activations [rows, f]
   const int32_t* offsets;
   const void* w1;
   const void* w2;
@@ -138,11 +168,13 @@ cudaError_t launch_ffn_combine_bf16(const FfnProblem& p, const int32_t* perm_src
                                     const int32_t* slot_pos, const float* gate, float* y,
                                     const LaunchCtx& c);
 
-// fp32 SIMT grouped product out[r, n] = act(sum_k A[r, k] B_g[n, k]) for the rows r of
-// each group g (offsets, or a single group of `rows` rows when offsets is null).
+// fp32 SIMT grouped product out[r, n] = act(sum_k A'[r, k] B_g[n, k]) for the rows r of
+// each group g (offsets, or a single group of `rows` rows when offsets is null), where
+// A'[r] = A[a_idx[r] / a_div] when a_idx is given, else A[r].
 cudaError_t launch_sgemm_grouped(const float* A, const float* B, float* out,
                                  const int32_t* offsets, int groups, int64_t rows_cap, int N,
-                                 int K, int act, const LaunchCtx& c);
+                                 int K, int act, const LaunchCtx& c,
+                                 const int32_t* a_idx = nullptr, int a_div = 1);
 
 // ---- combine ---------------------------------------------------------------------
 struct CombineProblem {
@@ -154,6 +186,59 @@ struct CombineProblem {
   void* y;
 };
 cudaError_t launch_combine(const CombineProblem& p, const LaunchCtx& c);
+
+// ---- backward --------------------------------------------------------------------
+// Everything moe_backward launches; the buffers come from the training state and the
+// backward workspace (see moe_api.cu for their layout).
+struct BackwardProblem {
+  int64_t T;
+  int d, f, E, k, act;  // act: 1 ReLU, 2 GELU
+  int noisy, renorm, hidden_f16;
+  float w_importance, w_load;
+  // forward inputs and saved forward state
+  const void* x;
+  const void* w_gate;
+  const void* w_noise;
+  const float* noise;
+  const float* bias;
+  const void* w1;
+  const void* w2;
+  const int32_t* topk_idx;
+  const float* topk_gate;
+  const float* importance;
+  const float* load;
+  const int32_t* offsets;
+  const int32_t* slot_pos;
+  const void* x_perm;
+  const void* u;
+  const void* h;
+  const float* y_perm;
+  const float* dy;
+  // outputs
+  float* dx;
+  float* dw_gate;
+  float* dw_noise;
+  float* dbias;
+  float* dw1;
+  float* dw2;
+  float* dgate;
+  float* losses;  // [2] or null: w_importance CV^2 and w_load CV^2
+  // workspace
+  int32_t* poff;
+  void* d_o;      // [T*k + 64 E, d] 16-bit
+  void* du;       // [T*k + 64 E, f] bf16
+  float* dx_perm; // [T*k, d]
+  float* logits;  // [T, E]
+  float* zlog;    // [T, E]
+  float* dl;      // [T, E]
+  float* dz;      // [T, E]
+  float* dimp;    // [E]
+  float* dload;   // [E]
+  float* part;    // split-contraction partial sums
+  int64_t part_cap;
+};
+int64_t backward_padded_rows(int64_t rows_cap, int E);
+cudaError_t launch_backward(const BackwardProblem& p, const LaunchCtx& c);
 
 // ---- weight preparation ----------------------------------------------------------
 cudaError_t launch_bf16_to_f16(const void* src, void* dst, int64_t n, int32_t* n_inexact,

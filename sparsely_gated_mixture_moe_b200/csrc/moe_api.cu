@@ -27,7 +27,17 @@ moe_status check_config(const moe_config* c) {
   if (c == nullptr) return MOE_ERR_INVALID_ARG;
   if (c->T < 0 || c->d_model <= 0 || c->d_ff <= 0 || c->E <= 0 || c->k <= 0 || c->k > c->E)
     return MOE_ERR_INVALID_ARG;
-  if (c->gating != MOE_GATE_SOFTMAX_TOPK && c->gating != MOE_GATE_NOISY_TOPK) return MOE_ERR_INVALID_ARG;
+  if (c->gating != MOE_GATE_SOFTMAX_TOPK && c->gating != MOE_GATE_NOISY_TOPK &&
+      c->gating != MOE_GATE_HIERARCHICAL)
+    return MOE_ERR_INVALID_ARG;
+  if (c->gating == MOE_GATE_HIERARCHICAL) {
+    if (c->groups <= 0 || c->E % c->groups != 0 || c->k_primary <= 0 ||
+        c->k_primary > c->groups || c->k % c->k_primary != 0 ||
+        c->k / c->k_primary > c->E / c->groups)
+      return MOE_ERR_INVALID_ARG;
+    if (c->k_primary > 4 || c->k / c->k_primary > 4) return MOE_ERR_UNSUPPORTED;
+    if (c->groups + c->E > (c->dtype == MOE_BF16 ? 256 : 1024)) return MOE_ERR_UNSUPPORTED;
+  }
   if (c->act != MOE_ACT_RELU && c->act != MOE_ACT_GELU) return MOE_ERR_INVALID_ARG;
   if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (!(c->capacity_factor == c->capacity_factor)) return MOE_ERR_INVALID_ARG;  // NaN
@@ -46,7 +56,7 @@ moe_status check_config(const moe_config* c) {
 
 struct Layout {
   size_t err, blk, partials, logits, nz, steps;                  // step workspace
-  size_t offsets, slot_pos, perm_src, x_perm, h, y_perm, forward;  // + forward intermediates
+  size_t offsets, slot_pos, perm_src, h, y_perm, forward;  // + forward intermediates
 };
 
 Layout layout(const moe_config* c) {
@@ -62,7 +72,8 @@ Layout layout(const moe_config* c) {
   L.logits = o;
   L.nz = o;
   if (c->dtype == MOE_F32) {
-    o = align_up(o + static_cast<size_t>(c->T) * c->E * 4);
+    const size_t cols = c->E + (c->gating == MOE_GATE_HIERARCHICAL ? c->groups : 0);
+    o = align_up(o + static_cast<size_t>(c->T) * cols * 4);
     L.nz = o;
     if (c->gating == MOE_GATE_NOISY_TOPK) o = align_up(o + static_cast<size_t>(c->T) * c->E * 4);
   }
@@ -73,14 +84,88 @@ Layout layout(const moe_config* c) {
   o = align_up(o + static_cast<size_t>(n) * 4);
   L.perm_src = o;
   o = align_up(o + static_cast<size_t>(n) * 4);
-  L.x_perm = o;
-  o = align_up(o + static_cast<size_t>(n) * c->d_model * esize(c));
   L.h = o;
   o = align_up(o + static_cast<size_t>(n) * c->d_ff * esize(c));
   L.y_perm = o;
   o = align_up(o + static_cast<size_t>(n) * c->d_model * 4);
   L.forward = o;
   return L;
+}
+
+// The forward state moe_forward_train keeps for moe_backward.
+struct TrainLayout {
+  size_t offsets, slot_pos, perm_src, x_perm, u, h, y_perm, total;
+};
+
+TrainLayout train_layout(const moe_config* c) {
+  TrainLayout L;
+  const int64_t n = c->T * c->k;
+  size_t o = 0;
+  L.offsets = o;
+  o = align_up(o + static_cast<size_t>(c->E + 1) * 4);
+  L.slot_pos = o;
+  o = align_up(o + static_cast<size_t>(n) * 4);
+  L.perm_src = o;
+  o = align_up(o + static_cast<size_t>(n) * 4);
+  L.x_perm = o;
+  o = align_up(o + static_cast<size_t>(n) * c->d_model * 2);
+  L.u = o;
+  o = align_up(o + static_cast<size_t>(n) * c->d_ff * 2);
+  L.h = o;
+  o = align_up(o + static_cast<size_t>(n) * c->d_ff * 2);
+  L.y_perm = o;
+  o = align_up(o + static_cast<size_t>(n) * c->d_model * 4);
+  L.total = o;
+  return L;
+}
+
+// moe_backward's workspace: the step workspace (error word first), then its buffers.
+struct BackwardLayout {
+  size_t poff, d_o, du, dx_perm, logits, zlog, dl, dz, dimp, dload, part, total;
+  int64_t part_cap;
+};
+
+BackwardLayout backward_layout(const moe_config* c, size_t steps) {
+  BackwardLayout L;
+  const int64_t n = c->T * c->k;
+  const int64_t prows = backward_padded_rows(n, c->E);
+  const size_t TE = static_cast<size_t>(c->T) * c->E;
+  size_t o = steps;
+  L.poff = o;
+  o = align_up(o + static_cast<size_t>(c->E + 1) * 4);
+  L.d_o = o;
+  o = align_up(o + static_cast<size_t>(prows) * c->d_model * 2);
+  L.du = o;
+  o = align_up(o + static_cast<size_t>(prows) * c->d_ff * 2);
+  L.dx_perm = o;
+  o = align_up(o + static_cast<size_t>(n) * c->d_model * 4);
+  L.logits = o;
+  o = align_up(o + TE * 4);
+  L.zlog = o;
+  o = align_up(o + TE * 4);
+  L.dl = o;
+  o = align_up(o + TE * 4);
+  L.dz = o;
+  o = align_up(o + TE * 4);
+  L.dimp = o;
+  o = align_up(o + static_cast<size_t>(c->E) * 4);
+  L.dload = o;
+  o = align_up(o + static_cast<size_t>(c->E) * 4);
+  L.part = o;
+  const int64_t a = 64LL * c->E * c->d_model, b = 4LL * c->T * c->E;
+  L.part_cap = a > b ? a : b;
+  o = align_up(o + static_cast<size_t>(L.part_cap) * 4);
+  L.total = o;
+  return L;
+}
+
+// Configurations the training forward and the backward support: bf16 layers with the
+// softmax or noisy gate.
+moe_status check_train_config(const moe_config* c) {
+  moe_status st = check_config(c);
+  if (st != MOE_OK) return st;
+  if (c->dtype != MOE_BF16 || c->gating == MOE_GATE_HIERARCHICAL) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
 }
 
 int64_t capacity_of(const moe_config* c) {
@@ -135,11 +220,14 @@ moe_status do_route(const moe_config* cfg, const Layout& L, const void* x, const
   p.k = cfg->k;
   p.noisy = cfg->gating == MOE_GATE_NOISY_TOPK;
   p.renorm = cfg->renorm != 0;
+  p.hier = cfg->gating == MOE_GATE_HIERARCHICAL;
+  p.groups = p.hier ? cfg->groups : 0;
+  p.k_primary = p.hier ? cfg->k_primary : 0;
+  p.bias = p.hier ? nullptr : logit_bias;
   p.x = x;
   p.w_gate = w_gate;
   p.w_noise = w_noise;
   p.noise = noise;
-  p.bias = logit_bias;
   p.topk_idx = topk_idx;
   p.topk_gate = topk_gate;
   p.near_tie = near_tie;
@@ -154,12 +242,14 @@ moe_status do_route(const moe_config* cfg, const Layout& L, const void* x, const
 
 moe_status check_route_args(const moe_config* cfg, const void* x, const void* w_gate,
                             const void* w_noise, const float* noise, const int32_t* topk_idx,
-                            const float* topk_gate, const float* load, const void* ws) {
+                            const float* topk_gate, const float* importance, const float* load,
+                            const void* ws) {
   if (!x || !w_gate || !topk_idx || !topk_gate || !ws) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_gate) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
   const bool noisy = cfg->gating == MOE_GATE_NOISY_TOPK;
   if (noisy && (!w_noise || !noise || !aligned16(w_noise))) return MOE_ERR_INVALID_ARG;
   if (load && !(noisy && cfg->k < cfg->E)) return MOE_ERR_INVALID_ARG;
+  if (cfg->gating == MOE_GATE_HIERARCHICAL && importance) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -186,9 +276,17 @@ moe_status do_permute(const moe_config* cfg, const Layout& L, const int32_t* top
   return launch_permute(p, ctx.lc) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// x_perm: the permuted rows; or, with gather_src, x is the token rows and permuted row s
+// reads x[gather_src[s] / k].
 moe_status do_ffn(const moe_config* cfg, const void* x_perm, const int32_t* offsets, const void* w1,
-                  const void* w2, void* h, void* y_perm, Ctx& ctx) {
+                  const void* w2, void* h, void* y_perm, Ctx& ctx, const void* x = nullptr,
+                  const int32_t* gather_src = nullptr, void* u = nullptr) {
   FfnProblem p;
+  p.u = u;
+  p.x = x;
+  p.gather_src = gather_src;
+  p.x_rows = cfg->T;
+  p.k = cfg->k;
   p.rows_cap = cfg->T * cfg->k;
   p.d = cfg->d_model;
   p.f = cfg->d_ff;
@@ -220,8 +318,13 @@ moe_status do_combine(const moe_config* cfg, const void* y_perm, const int32_t* 
 
 moe_status do_ffn_combine(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
                           const int32_t* perm_src, const int32_t* slot_pos, const float* gate,
-                          const void* w1, const void* w2, void* h, void* y, Ctx& ctx) {
+                          const void* w1, const void* w2, void* h, void* y, Ctx& ctx,
+                          const void* x = nullptr, bool gather = false) {
   FfnProblem p;
+  p.x = x;
+  p.gather_src = gather ? perm_src : nullptr;
+  p.x_rows = cfg->T;
+  p.k = cfg->k;
   p.rows_cap = cfg->T;  // k = 1
   p.d = cfg->d_model;
   p.f = cfg->d_ff;
@@ -327,7 +430,8 @@ moe_status moe_route(const moe_config* cfg, const void* x, const void* w_gate, c
   moe_status st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return empty_batch(cfg, nullptr, nullptr, importance, load, stream);
-  st = check_route_args(cfg, x, w_gate, w_noise, noise, topk_idx, topk_gate, load, ws);
+  st = check_route_args(cfg, x, w_gate, w_noise, noise, topk_idx, topk_gate, importance, load,
+                          ws);
   if (st != MOE_OK) return st;
   Ctx ctx(ws, stream);
   if (!ctx.ok) return MOE_ERR_CUDA;
@@ -343,8 +447,8 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
   if (st != MOE_OK) return st;
   if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
   if (cfg->T == 0) return empty_batch(cfg, counts, offsets, nullptr, nullptr, stream);
-  if (!topk_idx || !x || !perm_src || !slot_pos || !x_perm || !ws) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(x_perm) || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (!topk_idx || !perm_src || !slot_pos || !ws || (x_perm && !x)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(ws) || (x_perm && (!aligned16(x) || !aligned16(x_perm)))) return MOE_ERR_INVALID_ARG;
   Ctx ctx(ws, stream);
   if (!ctx.ok) return MOE_ERR_CUDA;
   st = do_permute(cfg, layout(cfg), topk_idx, x, counts, offsets, perm_src, slot_pos, x_perm, ws, ctx);
@@ -367,6 +471,25 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32
   Ctx ctx(ws, stream);
   if (!ctx.ok) return MOE_ERR_CUDA;
   st = do_ffn(cfg, x_perm, offsets, w1, w2, h, y_perm, ctx);
+  return st == MOE_OK ? ctx.finish(cudaSuccess) : st;
+}
+
+moe_status moe_expert_ffn_gather(const moe_config* cfg, const void* x, const int32_t* perm_src,
+                                 const int32_t* offsets, const void* w1, const void* w2, void* h,
+                                 void* y_perm, void* ws, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) {
+    g_last_launches = 0;
+    return MOE_OK;
+  }
+  if (!x || !perm_src || !offsets || !w1 || !w2 || !h || !y_perm || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w1) || !aligned16(w2) || !aligned16(h) || !aligned16(y_perm) ||
+      !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  Ctx ctx(ws, stream);
+  if (!ctx.ok) return MOE_ERR_CUDA;
+  st = do_ffn(cfg, nullptr, offsets, w1, w2, h, y_perm, ctx, x, perm_src);
   return st == MOE_OK ? ctx.finish(cudaSuccess) : st;
 }
 
@@ -409,6 +532,30 @@ moe_status moe_expert_ffn_combine(const moe_config* cfg, const void* x_perm,
   return st == MOE_OK ? ctx.finish(cudaSuccess) : st;
 }
 
+moe_status moe_expert_ffn_combine_gather(const moe_config* cfg, const void* x,
+                                         const int32_t* offsets, const int32_t* perm_src,
+                                         const int32_t* slot_pos, const float* topk_gate,
+                                         const void* w1, const void* w2, void* h, void* y,
+                                         void* ws, moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!fused_combine(cfg)) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T == 0) {
+    g_last_launches = 0;
+    return MOE_OK;
+  }
+  if (!x || !offsets || !perm_src || !slot_pos || !topk_gate || !w1 || !w2 || !h || !y || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w1) || !aligned16(w2) || !aligned16(h) || !aligned16(y) ||
+      !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  Ctx ctx(ws, stream);
+  if (!ctx.ok) return MOE_ERR_CUDA;
+  st = do_ffn_combine(cfg, nullptr, offsets, perm_src, slot_pos, topk_gate, w1, w2, h, y, ctx, x,
+                      true);
+  return st == MOE_OK ? ctx.finish(cudaSuccess) : st;
+}
+
 moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_gate, const void* w_noise,
                        const float* noise, const float* logit_bias, const void* w1, const void* w2,
                        void* y, int32_t* topk_idx, float* topk_gate, int32_t* counts,
@@ -418,7 +565,8 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_gate,
   if (st != MOE_OK) return st;
   if (!counts) return MOE_ERR_INVALID_ARG;
   if (cfg->T == 0) return empty_batch(cfg, counts, nullptr, importance, load, stream);
-  st = check_route_args(cfg, x, w_gate, w_noise, noise, topk_idx, topk_gate, load, ws);
+  st = check_route_args(cfg, x, w_gate, w_noise, noise, topk_idx, topk_gate, importance, load,
+                          ws);
   if (st != MOE_OK) return st;
   if (!w1 || !w2 || !y) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w1) || !aligned16(w2) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
@@ -429,24 +577,159 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_gate,
   int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
   int32_t* slot_pos = reinterpret_cast<int32_t*>(w + L.slot_pos);
   int32_t* perm_src = reinterpret_cast<int32_t*>(w + L.perm_src);
-  void* x_perm = w + L.x_perm;
   void* h = w + L.h;
   void* y_perm = w + L.y_perm;
   st = do_route(cfg, L, x, w_gate, w_noise, noise, logit_bias, topk_idx, topk_gate, importance, load,
                 near_tie, ws, ctx);
   if (st != MOE_OK) return st;
-  st = do_permute(cfg, L, topk_idx, x, counts, offsets, perm_src, slot_pos, x_perm, ws, ctx);
+  // index arrays only: the up-projection gathers the token rows from x itself
+  st = do_permute(cfg, L, topk_idx, x, counts, offsets, perm_src, slot_pos, nullptr, ws, ctx);
   if (st != MOE_OK) return st;
   if (fused_combine(cfg)) {
-    st = do_ffn_combine(cfg, x_perm, offsets, perm_src, slot_pos, topk_gate, w1, w2, h, y, ctx);
+    st = do_ffn_combine(cfg, nullptr, offsets, perm_src, slot_pos, topk_gate, w1, w2, h, y, ctx, x,
+                        true);
     if (st != MOE_OK) return st;
     return ctx.finish(cudaSuccess);
   }
-  st = do_ffn(cfg, x_perm, offsets, w1, w2, h, y_perm, ctx);
+  st = do_ffn(cfg, nullptr, offsets, w1, w2, h, y_perm, ctx, x, perm_src);
   if (st != MOE_OK) return st;
   st = do_combine(cfg, y_perm, slot_pos, topk_gate, y, ctx);
   if (st != MOE_OK) return st;
   return ctx.finish(cudaSuccess);
+}
+
+size_t moe_train_state_size(const moe_config* cfg) {
+  if (check_train_config(cfg) != MOE_OK) return 0;
+  return train_layout(cfg).total;
+}
+
+size_t moe_backward_workspace_size(const moe_config* cfg) {
+  if (check_train_config(cfg) != MOE_OK) return 0;
+  return backward_layout(cfg, layout(cfg).steps).total;
+}
+
+moe_status moe_forward_train(const moe_config* cfg, const void* x, const void* w_gate,
+                             const void* w_noise, const float* noise, const float* logit_bias,
+                             const void* w1, const void* w2, void* y, int32_t* topk_idx,
+                             float* topk_gate, int32_t* counts, float* importance, float* load,
+                             uint8_t* near_tie, void* state, void* ws, moe_stream_t stream) {
+  moe_status st = check_train_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts || !state) return MOE_ERR_INVALID_ARG;
+  if (cfg->T == 0) return empty_batch(cfg, counts, nullptr, importance, load, stream);
+  st = check_route_args(cfg, x, w_gate, w_noise, noise, topk_idx, topk_gate, importance, load, ws);
+  if (st != MOE_OK) return st;
+  if (!w1 || !w2 || !y || !aligned16(w1) || !aligned16(w2) || !aligned16(y) || !aligned16(state))
+    return MOE_ERR_INVALID_ARG;
+  Ctx ctx(ws, stream);
+  if (!ctx.ok) return MOE_ERR_CUDA;
+  const Layout L = layout(cfg);
+  const TrainLayout S = train_layout(cfg);
+  uint8_t* sb = static_cast<uint8_t*>(state);
+  int32_t* offsets = reinterpret_cast<int32_t*>(sb + S.offsets);
+  int32_t* slot_pos = reinterpret_cast<int32_t*>(sb + S.slot_pos);
+  int32_t* perm_src = reinterpret_cast<int32_t*>(sb + S.perm_src);
+  void* x_perm = sb + S.x_perm;
+  void* u = sb + S.u;
+  void* h = sb + S.h;
+  void* y_perm = sb + S.y_perm;
+  st = do_route(cfg, L, x, w_gate, w_noise, noise, logit_bias, topk_idx, topk_gate, importance, load,
+                near_tie, ws, ctx);
+  if (st != MOE_OK) return st;
+  st = do_permute(cfg, L, topk_idx, x, counts, offsets, perm_src, slot_pos, x_perm, ws, ctx);
+  if (st != MOE_OK) return st;
+  st = do_ffn(cfg, x_perm, offsets, w1, w2, h, y_perm, ctx, nullptr, nullptr, u);
+  if (st != MOE_OK) return st;
+  st = do_combine(cfg, y_perm, slot_pos, topk_gate, y, ctx);
+  if (st != MOE_OK) return st;
+  return ctx.finish(cudaSuccess);
+}
+
+moe_status moe_backward(const moe_config* cfg, const void* x, const void* w_gate,
+                        const void* w_noise, const float* noise, const float* logit_bias,
+                        const void* w1, const void* w2, const int32_t* topk_idx,
+                        const float* topk_gate, const float* importance, const float* load,
+                        const void* state, const float* dy, float w_importance, float w_load,
+                        float* dx, float* dw_gate, float* dw_noise, float* dlogit_bias, float* dw1,
+                        float* dw2, float* dgates, float* losses, void* ws, moe_stream_t stream) {
+  moe_status st = check_train_config(cfg);
+  if (st != MOE_OK) return st;
+  const bool noisy = cfg->gating == MOE_GATE_NOISY_TOPK;
+  if (!(w_importance == w_importance) || !(w_load == w_load)) return MOE_ERR_INVALID_ARG;
+  if (w_importance != 0.0f && !importance) return MOE_ERR_INVALID_ARG;
+  if (w_load != 0.0f && !(noisy && load && cfg->k < cfg->E)) return MOE_ERR_INVALID_ARG;
+  if (!x || !w_gate || !w1 || !w2 || !topk_idx || !topk_gate || !state || !dy || !dx || !dw_gate ||
+      !dw1 || !dw2 || !dgates || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if (noisy && (!w_noise || !noise || !dw_noise)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate) || !aligned16(w1) || !aligned16(w2) || !aligned16(state) ||
+      !aligned16(dy) || !aligned16(dx) || !aligned16(dw1) || !aligned16(dw2) || !aligned16(ws) ||
+      (noisy && !aligned16(w_noise)))
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->T == 0) {
+    g_last_launches = 0;
+    return MOE_OK;
+  }
+  Ctx ctx(ws, stream);
+  if (!ctx.ok) return MOE_ERR_CUDA;
+  const Layout L = layout(cfg);
+  const TrainLayout S = train_layout(cfg);
+  const BackwardLayout B = backward_layout(cfg, L.steps);
+  const uint8_t* sb = static_cast<const uint8_t*>(state);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  BackwardProblem p;
+  p.T = cfg->T;
+  p.d = cfg->d_model;
+  p.f = cfg->d_ff;
+  p.E = cfg->E;
+  p.k = cfg->k;
+  p.act = cfg->act == MOE_ACT_GELU ? 2 : 1;
+  p.noisy = noisy;
+  p.renorm = cfg->renorm != 0;
+  p.hidden_f16 = cfg->hidden_f16;
+  p.w_importance = w_importance;
+  p.w_load = w_load;
+  p.x = x;
+  p.w_gate = w_gate;
+  p.w_noise = w_noise;
+  p.noise = noise;
+  p.bias = logit_bias;
+  p.w1 = w1;
+  p.w2 = w2;
+  p.topk_idx = topk_idx;
+  p.topk_gate = topk_gate;
+  p.importance = importance;
+  p.load = load;
+  p.offsets = reinterpret_cast<const int32_t*>(sb + S.offsets);
+  p.slot_pos = reinterpret_cast<const int32_t*>(sb + S.slot_pos);
+  p.x_perm = sb + S.x_perm;
+  p.u = sb + S.u;
+  p.h = sb + S.h;
+  p.y_perm = reinterpret_cast<const float*>(sb + S.y_perm);
+  p.dy = dy;
+  p.dx = dx;
+  p.dw_gate = dw_gate;
+  p.dw_noise = dw_noise;
+  p.dbias = dlogit_bias;
+  p.dw1 = dw1;
+  p.dw2 = dw2;
+  p.dgate = dgates;
+  p.losses = losses;
+  p.poff = reinterpret_cast<int32_t*>(w + B.poff);
+  p.d_o = w + B.d_o;
+  p.du = w + B.du;
+  p.dx_perm = reinterpret_cast<float*>(w + B.dx_perm);
+  p.logits = reinterpret_cast<float*>(w + B.logits);
+  p.zlog = reinterpret_cast<float*>(w + B.zlog);
+  p.dl = reinterpret_cast<float*>(w + B.dl);
+  p.dz = reinterpret_cast<float*>(w + B.dz);
+  p.dimp = reinterpret_cast<float*>(w + B.dimp);
+  p.dload = reinterpret_cast<float*>(w + B.dload);
+  p.part = reinterpret_cast<float*>(w + B.part);
+  p.part_cap = B.part_cap;
+  if (losses && cudaMemsetAsync(losses, 0, 2 * sizeof(float), ctx.lc.stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return ctx.finish(launch_backward(p, ctx.lc));
 }
 
 moe_status moe_get_error(void* ws, moe_stream_t stream, int32_t* device_error) {

@@ -18,6 +18,8 @@
 //   gather      x_perm[s] = x[perm_src[s] / k] for every kept row s < offsets[E]: one warp
 //               per row, 16-byte vectors, a grid of several blocks per SM so that enough
 //               loads are in flight to stream at HBM rate
+// With x_perm null only the index arrays are written (no row copy): the expert FFN then
+// gathers the token rows itself (moe_expert_ffn_gather).
 #include <map>
 #include <mutex>
 
@@ -374,8 +376,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     }
     __syncthreads();
     // the chunk's kept rows, in assignment order; warp w takes assignments w, w + 32, ...
+    // (nothing to copy when only the index arrays are asked for)
     const int nv = row_bytes >> 4;
-    for (int i = warp; i < cn; i += 2 * pf::WARPS) {
+    for (int i = warp; x_perm != nullptr && i < cn; i += 2 * pf::WARPS) {
       const int i2 = i + pf::WARPS;
       const int sl1 = s_slot[i];
       const int sl2 = i2 < cn ? s_slot[i2] : -1;
@@ -495,7 +498,7 @@ cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c) {
   e = launch_kernel(perm_scatter_kernel, dim3(static_cast<unsigned>(nblk)), dim3(pm::THREADS),
                     wsmem, c, p.topk_idx, p.n, p.E, p.C, static_cast<const int32_t*>(p.blk),
                     static_cast<const int32_t*>(p.offsets), p.perm_src, p.slot_pos);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || p.x_perm == nullptr) return e;
   // enough warps for every row when the grid allows, capped at 16 blocks per SM
   int64_t gblocks = (p.n + kGatherWarps - 1) / kGatherWarps;
   const int64_t cap = static_cast<int64_t>(c.num_sms) * 16;
@@ -563,8 +566,9 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
     set_last_launch_count(0);
     return MOE_OK;
   }
-  if (!topk_idx || !x || !perm_src || !slot_pos || !x_perm) return MOE_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(x_perm) & 15u))
+  if (!topk_idx || !perm_src || !slot_pos || (x_perm && !x)) return MOE_ERR_INVALID_ARG;
+  if (x_perm && ((reinterpret_cast<uintptr_t>(x) & 15u) ||
+                 (reinterpret_cast<uintptr_t>(x_perm) & 15u)))
     return MOE_ERR_INVALID_ARG;
   const int64_t n = cfg->T * cfg->k;
   // the scratch holds a 256-byte counter block, then one int32 per (chunk, expert)

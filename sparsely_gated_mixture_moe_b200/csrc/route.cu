@@ -43,6 +43,7 @@ int route_blocks(int64_t T) { return static_cast<int>((T + 63) / 64); }
 struct GateArgs {
   int64_t T;
   int E, k, noisy, renorm;
+  int groups, k_primary;  // hierarchical gating (groups > 0): E experts in groups of E/groups
   const float* noise;
   const float* bias;
   int32_t* topk_idx;
@@ -428,6 +429,105 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
   sync();  // qsum and the lists are reused by the next tile
 }
 
+// The hierarchical gate for one tile of 128 tokens, by 128 threads (one token row each;
+// the thread in lane l of the warp reading TMEM lane quarter q owns row 32*q + l).  The
+// score columns are the primary gate's over the A = g.groups groups, then group i's
+// secondary scores over its B = E / A experts at A + i*B.  `fetch(c, l, z)` fills
+// l[0..15] with the scores of columns c .. c+15 (c a multiple of 16).
+//   pass 1  top-(k_primary+1) of the primary scores (TopList, ties to the lower group)
+//   pass 2  every secondary column once, in ascending order; a column of one of this
+//           token's chosen groups enters that group's top-(k_group+1) list
+//   gates   Softmax(KeepTopK) at each level, multiplied; expert j of group i is i*B + j
+// Everything stays in registers: no shared memory and no barrier.
+template <int KP, int KG, class Fetch>
+__device__ __forceinline__ void gate_tile_hier(const Fetch& fetch, int q, int lane, int64_t tile,
+                                               const GateArgs& g) {
+  const int row = q * 32 + lane;
+  const int64_t t = tile * 128 + row;
+  const bool valid = t < g.T;
+  const int A = g.groups, NG = g.groups + g.E, B = g.E / g.groups;
+  const int k1 = g.k_primary, k2 = g.k / g.k_primary;
+  TopList<KP> prim;
+  prim.init();
+#pragma unroll 1
+  for (int cs = 0; cs < A; cs += 16) {
+    float l[16], z[16];
+    fetch(cs, l, z);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (cs + j < A) prim.push(l[j], cs + j);
+  }
+  int chosen[KP];
+#pragma unroll
+  for (int q2 = 0; q2 < KP; ++q2) chosen[q2] = (q2 < k1) ? prim.i[q2] : -1;
+  TopList<KG> sec[KP];
+#pragma unroll
+  for (int q2 = 0; q2 < KP; ++q2) sec[q2].init();
+  // (grp, e): group and expert-in-group of column c, advanced column by column
+  int grp = 0, e = 0;
+#pragma unroll 1
+  for (int cs = (A / 16) * 16; cs < NG; cs += 16) {
+    float l[16], z[16];
+    fetch(cs, l, z);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int c = cs + j;
+      if (c >= A && c < NG) {
+#pragma unroll
+        for (int q2 = 0; q2 < KP; ++q2)
+          if (chosen[q2] == grp) sec[q2].push(l[j], e);
+        if (++e == B) {
+          e = 0;
+          ++grp;
+        }
+      }
+    }
+  }
+  // primary gates over the kept groups, and the primary k-th vs (k+1)-th gap
+  float gp[KP];
+  float den = 0.0f;
+#pragma unroll
+  for (int q2 = 0; q2 < KP; ++q2) {
+    gp[q2] = (q2 < k1) ? expf(prim.v[q2] - prim.v[0]) : 0.0f;
+    den += gp[q2];
+  }
+  float kth = INFINITY, kth1 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j <= KP; ++j) {
+    if (j < k1) kth = fminf(kth, prim.v[j]);
+    else kth1 = fmaxf(kth1, prim.v[j]);
+  }
+  float gap = (k1 < A) ? kth - kth1 : INFINITY;
+#pragma unroll
+  for (int q2 = 0; q2 < KP; ++q2) {
+    if (q2 >= k1) continue;
+    const float share = gp[q2] / den;
+    float gs[KG];
+    float ds = 0.0f;
+#pragma unroll
+    for (int j = 0; j < KG; ++j) {
+      gs[j] = (j < k2) ? expf(sec[q2].v[j] - sec[q2].v[0]) : 0.0f;
+      ds += gs[j];
+    }
+    float sk = INFINITY, sk1 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j <= KG; ++j) {
+      if (j < k2) sk = fminf(sk, sec[q2].v[j]);
+      else sk1 = fmaxf(sk1, sec[q2].v[j]);
+    }
+    if (k2 < B) gap = fminf(gap, sk - sk1);
+    if (valid) {
+#pragma unroll
+      for (int j = 0; j < KG; ++j)
+        if (j < k2) {
+          g.topk_idx[t * g.k + q2 * k2 + j] = chosen[q2] * B + sec[q2].i[j];
+          g.topk_gate[t * g.k + q2 * k2 + j] = share * (gs[j] / ds);
+        }
+    }
+  }
+  if (valid && g.near_tie) g.near_tie[t] = (gap <= 1e-4f) ? 1 : 0;
+}
+
 // ------------------------------------------------------------------ bf16 router
 //
 // Persistent and warp-specialised.  Warp 0 streams the x tile and the gating weights of
@@ -465,7 +565,9 @@ __device__ __forceinline__ void gate_bar_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
-template <int KM, int G = rt::groups_for(KM)>
+// HKG > 0: hierarchical gating with KM the primary and HKG the secondary list bucket
+// (one column group of gate warps).
+template <int KM, int HKG = 0, int G = (HKG > 0 ? 1 : rt::groups_for(KM))>
 __global__ void __launch_bounds__(64 + 128 * G)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     const __grid_constant__ CUtensorMap tmG,
@@ -654,7 +756,11 @@ __global__ void __launch_bounds__(64 + 128 * G)
             z[j] = 0.0f;
           }
         };
-        gate_tile<KM, G, 16>(fetch, sync, q, grp, gtid, L, a.half != 0, a.g, gsm);
+        if constexpr (HKG > 0) {
+          gate_tile_hier<KM, HKG>(fetch, q, lane, L, a.g);
+        } else {
+          gate_tile<KM, G, 16>(fetch, sync, q, grp, gtid, L, a.half != 0, a.g, gsm);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -701,6 +807,28 @@ __global__ void __launch_bounds__(128, 1)
                        static_cast<int64_t>(blockIdx.x), false, g, gsmem);
 }
 
+// Hierarchical gate on the fp32 logits [T, groups + E] of the workspace: 128 threads,
+// one token row each.
+template <int KP, int KG>
+__global__ void __launch_bounds__(128, 1)
+    gate_f32_hier_kernel(const float* __restrict__ logits, GateArgs g) {
+  grid_dep_wait();
+  grid_dep_launch();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kRouteBM + threadIdx.x;
+  const bool valid = t < g.T;
+  const int NG = g.groups + g.E;
+  auto fetch = [&](int c, float (&l)[16], float (&z)[16]) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const bool in = valid && (c + j < NG);
+      l[j] = in ? logits[t * NG + c + j] : 0.0f;
+      z[j] = 0.0f;
+    }
+  };
+  gate_tile_hier<KP, KG>(fetch, static_cast<int>(threadIdx.x) >> 5,
+                         static_cast<int>(threadIdx.x) & 31, static_cast<int64_t>(blockIdx.x), g);
+}
+
 __global__ void finalize_importance_load_kernel(const float* __restrict__ partials, int nblocks,
                                                 int E, float* importance, float* load) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
@@ -725,6 +853,8 @@ static GateArgs gate_args(const RouteProblem& p) {
   g.k = p.k;
   g.noisy = p.noisy;
   g.renorm = p.renorm;
+  g.groups = p.hier ? p.groups : 0;
+  g.k_primary = p.hier ? p.k_primary : 0;
   g.noise = p.noise;
   g.bias = p.bias;
   g.topk_idx = p.topk_idx;
@@ -742,31 +872,46 @@ static cudaError_t launch_finalize(const RouteProblem& p, int nblocks, const Lau
                        static_cast<const float*>(p.partials), nblocks, p.E, p.importance, p.load);
 }
 
-template <int KM>
+template <int KM, int HKG = 0>
 static cudaError_t launch_route_tc(const CUtensorMap& tmX, const CUtensorMap& tmG,
                                    const CUtensorMap& tmN, const RouteTcArgs& a, int smem,
                                    int grid, const LaunchCtx& c) {
-  cudaError_t e = ensure_smem_limit(route_tc_kernel<KM>, smem);
+  cudaError_t e = ensure_smem_limit(route_tc_kernel<KM, HKG>, smem);
   if (e != cudaSuccess) return e;
-  return launch_kernel(route_tc_kernel<KM>, dim3(grid), dim3(64 + 128 * rt::groups_for(KM)), smem,
-                       c, tmX, tmG, tmN, a);
+  const int G = HKG > 0 ? 1 : rt::groups_for(KM);
+  return launch_kernel(route_tc_kernel<KM, HKG>, dim3(grid), dim3(64 + 128 * G), smem, c, tmX, tmG,
+                       tmN, a);
+}
+
+// hierarchical: list buckets of the primary (KP) and secondary (KG) levels, 1, 2 or 4
+template <int KP>
+static cudaError_t launch_route_tc_hier(int kg, const CUtensorMap& tmX, const CUtensorMap& tmG,
+                                        const RouteTcArgs& a, int smem, int grid,
+                                        const LaunchCtx& c) {
+  switch (kg) {
+    case 1: return launch_route_tc<KP, 1>(tmX, tmG, tmG, a, smem, grid, c);
+    case 2: return launch_route_tc<KP, 2>(tmX, tmG, tmG, a, smem, grid, c);
+    default: return launch_route_tc<KP, 4>(tmX, tmG, tmG, a, smem, grid, c);
+  }
 }
 
 cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   RouteTcArgs a;
   a.g = gate_args(p);
-  a.e_pad = (p.E + 15) / 16 * 16;
+  const int n_scores = p.hier ? p.E + p.groups : p.E;  // score columns (rows of w_gate)
+  a.e_pad = (n_scores + 15) / 16 * 16;
   a.acc_cols = 32;
   while (a.acc_cols < a.e_pad) a.acc_cols <<= 1;
   a.kblocks = p.d / rt::BK;
   a.nb = p.noisy ? 2 : 1;
   a.nbuf = 2 * a.nb * a.acc_cols <= 512 ? 2 : 1;
-  // half tiles when 128-token tiles would fill at most half of the SMs
+  // half tiles when 128-token tiles would fill at most half of the SMs (not for the
+  // hierarchical gate, whose one thread per token reads every score column)
   const int full_tiles = static_cast<int>((p.T + kRouteBM - 1) / kRouteBM);
-  a.half = 2 * full_tiles <= c.num_sms ? 1 : 0;
+  a.half = (!p.hier && 2 * full_tiles <= c.num_sms) ? 1 : 0;
   a.ntiles = a.half ? static_cast<int>((p.T + 63) / 64) : full_tiles;
-  const int km = k_bucket(p.k);
-  const int scratch = gate_smem_bytes(km, rt::groups_for(km), p.E);
+  const int km = p.hier ? k_bucket(p.k_primary) : k_bucket(p.k);
+  const int scratch = gate_smem_bytes(km, p.hier ? 1 : rt::groups_for(km), p.E);
   const int stage_bytes = rt::A_BYTES + a.nb * a.e_pad * rt::BK * 2;
   // the ring takes what the gate scratch and the barriers leave of 227 KB
   const int bar_bytes = 8 * (2 * 8 + 5) + 16;
@@ -782,7 +927,8 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   CUtensorMap tmX, tmG, tmN;
   if (!make_tmap_bf16(&tmX, p.x, static_cast<uint64_t>(p.T), p.d, a.half ? 64 : kRouteBM))
     return cudaErrorInvalidValue;
-  if (!make_tmap_bf16(&tmG, p.w_gate, static_cast<uint64_t>(p.E), p.d, a.e_pad)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16(&tmG, p.w_gate, static_cast<uint64_t>(n_scores), p.d, a.e_pad))
+    return cudaErrorInvalidValue;
   if (p.noisy) {
     if (!make_tmap_bf16(&tmN, p.w_noise, static_cast<uint64_t>(p.E), p.d, a.e_pad)) return cudaErrorInvalidValue;
   } else {
@@ -790,6 +936,15 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   }
   const int grid = a.ntiles < c.num_sms ? a.ntiles : c.num_sms;
   cudaError_t e;
+  if (p.hier) {
+    const int kg = k_bucket(p.k / p.k_primary);
+    switch (km) {
+      case 1: e = launch_route_tc_hier<1>(kg, tmX, tmG, a, smem, grid, c); break;
+      case 2: e = launch_route_tc_hier<2>(kg, tmX, tmG, a, smem, grid, c); break;
+      default: e = launch_route_tc_hier<4>(kg, tmX, tmG, a, smem, grid, c); break;
+    }
+    return e;
+  }
   switch (km) {
     case 1: e = launch_route_tc<1>(tmX, tmG, tmN, a, smem, grid, c); break;
     case 2: e = launch_route_tc<2>(tmX, tmG, tmN, a, smem, grid, c); break;
@@ -813,10 +968,32 @@ static cudaError_t launch_gate_f32(const RouteProblem& p, const GateArgs& g, int
                        static_cast<const float*>(p.noisy ? p.nz_ws : nullptr), g);
 }
 
+template <int KP>
+static cudaError_t launch_gate_f32_hier(int kg, const RouteProblem& p, const GateArgs& g,
+                                        int nblocks, const LaunchCtx& c) {
+  const float* lg = p.logits_ws;
+  switch (kg) {
+    case 1: return launch_kernel(gate_f32_hier_kernel<KP, 1>, dim3(nblocks), dim3(128), 0, c, lg, g);
+    case 2: return launch_kernel(gate_f32_hier_kernel<KP, 2>, dim3(nblocks), dim3(128), 0, c, lg, g);
+    default: return launch_kernel(gate_f32_hier_kernel<KP, 4>, dim3(nblocks), dim3(128), 0, c, lg, g);
+  }
+}
+
 cudaError_t launch_route_f32(const RouteProblem& p, const LaunchCtx& c) {
+  const int n_scores = p.hier ? p.E + p.groups : p.E;
   cudaError_t e = launch_sgemm_grouped(static_cast<const float*>(p.x), static_cast<const float*>(p.w_gate),
-                                       p.logits_ws, nullptr, 1, p.T, p.E, p.d, 0, c);
+                                       p.logits_ws, nullptr, 1, p.T, n_scores, p.d, 0, c);
   if (e != cudaSuccess) return e;
+  if (p.hier) {
+    const GateArgs g = gate_args(p);
+    const int nblocks = static_cast<int>((p.T + kRouteBM - 1) / kRouteBM);
+    const int kg = k_bucket(p.k / p.k_primary);
+    switch (k_bucket(p.k_primary)) {
+      case 1: return launch_gate_f32_hier<1>(kg, p, g, nblocks, c);
+      case 2: return launch_gate_f32_hier<2>(kg, p, g, nblocks, c);
+      default: return launch_gate_f32_hier<4>(kg, p, g, nblocks, c);
+    }
+  }
   if (p.noisy) {
     e = launch_sgemm_grouped(static_cast<const float*>(p.x), static_cast<const float*>(p.w_noise),
                              p.nz_ws, nullptr, 1, p.T, p.E, p.d, 0, c);

@@ -41,7 +41,7 @@ def f64(t: torch.Tensor) -> np.ndarray:
 def config_of(w: workloads.Workload) -> moe.MoEConfig:
     return moe.make_config(w.T, w.d_model, w.d_ff, w.E, w.k, gating=w.gating, renorm=w.renorm,
                            capacity_factor=w.capacity_factor, act=w.act, dtype=w.dtype,
-                           hidden_f16=w.hidden_f16)
+                           hidden_f16=w.hidden_f16, groups=w.groups, k_primary=w.k_primary)
 
 
 def hidden_dtype(w):
@@ -80,7 +80,8 @@ def run_steps(w, dev, cfg=None):
         "y": torch.full((T, d), float("nan"), dtype=torch.float32, device=cu),
     }
     noisy = w.gating == "noisy_topk"
-    o["importance"] = torch.full((E,), float("nan"), device=cu)
+    hier = w.gating == "hierarchical"
+    o["importance"] = None if hier else torch.full((E,), float("nan"), device=cu)
     o["load"] = torch.full((E,), float("nan"), device=cu) if noisy and k < E else None
     ws = moe.workspace(cfg, cu)
     moe.moe_route(cfg, dev["x"], dev["w_gate"], o["topk_idx"], o["topk_gate"], ws,
@@ -97,10 +98,46 @@ def run_steps(w, dev, cfg=None):
         h2 = torch.zeros_like(o["h"])
         moe.moe_expert_ffn_combine(cfg, o["x_perm"], o["offsets"], o["perm_src"], o["slot_pos"],
                                    o["topk_gate"], dev["w1"], dev["w2"], h2, o["y_fused"], ws)
+    # the same permutation with index arrays only, and the expert FFN gathering its rows
+    # from x by perm_src (no x_perm): must give the same bits
+    n = max(T * k, 1)
+    gth = {"counts": torch.full((E,), -7, dtype=torch.int32, device=cu),
+           "offsets": torch.full((E + 1,), -7, dtype=torch.int32, device=cu),
+           "perm_src": torch.full((n,), -7, dtype=torch.int32, device=cu),
+           "slot_pos": torch.full((n,), -7, dtype=torch.int32, device=cu),
+           "h": torch.zeros(n, f, dtype=hidden_dtype(w), device=cu),
+           "y_perm": torch.zeros(n, d, dtype=torch.float32, device=cu)}
+    moe.moe_permute(cfg, o["topk_idx"], None, gth["counts"], gth["offsets"], gth["perm_src"],
+                    gth["slot_pos"], None, ws)
+    moe.moe_expert_ffn_gather(cfg, dev["x"], gth["perm_src"], gth["offsets"], dev["w1"], dev["w2"],
+                              gth["h"], gth["y_perm"], ws)
+    if moe.fused_combine(cfg):
+        gth["y_fused"] = torch.full((T, d), float("nan"), dtype=torch.float32, device=cu)
+        h3 = torch.zeros_like(o["h"])
+        moe.moe_expert_ffn_combine_gather(cfg, dev["x"], gth["offsets"], gth["perm_src"],
+                                          gth["slot_pos"], o["topk_gate"], dev["w1"], dev["w2"], h3,
+                                          gth["y_fused"], ws)
     err = moe.moe_get_error(ws)
     out = {kk: (v.cpu() if v is not None else None) for kk, v in o.items()}
+    out["gather"] = {kk: v.cpu() for kk, v in gth.items()}
     out["device_error"] = err
     return out
+
+
+def check_gather_path(w, g, report):
+    """The index-only permutation and the FFN that gathers its rows from x equal the
+    x_perm path bit for bit (the same rows reach the same tensor-core tiles)."""
+    gp = g["gather"]
+    n = int(g["offsets"][-1]) if w.T else 0
+    for key in ("counts", "offsets"):
+        assert torch.equal(gp[key], g[key]), key
+    assert torch.equal(gp["slot_pos"][: w.T * w.k], g["slot_pos"][: w.T * w.k])
+    assert torch.equal(gp["perm_src"][:n], g["perm_src"][:n])
+    assert torch.equal(gp["h"][:n], g["h"][:n]), "h differs between the gather and x_perm paths"
+    assert torch.equal(gp["y_perm"][:n], g["y_perm"][:n]), "y_perm differs"
+    if "y_fused" in gp:
+        assert torch.equal(gp["y_fused"], g["y_fused"]), "fused y differs"
+    report["gather_path"] = "equal"
 
 
 def run_forward(w, dev, cfg=None):
@@ -136,7 +173,63 @@ def reconcile_choice(w, r, idx_gpu):
     return idx, int(near.sum()), int(differ.sum())
 
 
+def hier_gates_for(w, scores, idx):
+    """The oracle's two-level gates for a given hierarchical choice idx [T, k] (e.g. the
+    GPU's at a near tie): orc.gate_values at the primary level over the chosen groups,
+    then within each chosen group over its chosen experts, multiplied."""
+    a, k1 = w.groups, w.k_primary
+    k2 = w.k // k1
+    b = w.E // a
+    T = idx.shape[0]
+    prim = scores[:, :a]
+    groups = idx[:, ::k2] // b                       # [T, k1]
+    gp = orc.gate_values(prim, groups, True)
+    out = np.zeros((T, w.k))
+    rows = np.arange(T)
+    for q in range(k1):
+        g_ = groups[:, q]
+        sec = np.stack([scores[t, a + g_[t] * b:a + (g_[t] + 1) * b] for t in range(T)])
+        j = idx[:, q * k2:(q + 1) * k2] - g_[:, None] * b
+        out[:, q * k2:(q + 1) * k2] = gp[:, q:q + 1] * orc.gate_values(sec, j, True)
+    return out
+
+
+def check_route_hier(w, inp, g, report):
+    """Hierarchical gating: the GPU's choice equals the oracle's on every token whose gap
+    at both levels exceeds the near-tie margin; elsewhere it must be a valid two-level
+    choice (whole groups of k / k_primary distinct experts, distinct groups), which the
+    later steps then follow.  Gates within GATE_ATOL of the oracle's for the choice."""
+    r = orc.route(inp, w)
+    idx_g = g["topk_idx"].long().numpy()
+    assert idx_g.min() >= 0 and idx_g.max() < w.E
+    near = r["gap"] <= NEAR_TIE
+    differ = ~np.all(idx_g == r["idx"], axis=1)
+    bad = differ & ~near
+    assert not bad.any(), "expert choice differs on %d non-near-tie tokens, e.g. %s" % (
+        int(bad.sum()), np.nonzero(bad)[0][:5])
+    k2 = w.k // w.k_primary
+    b = w.E // w.groups
+    grp = idx_g // b
+    for q in range(w.k_primary):   # each chosen group's block lies in one group
+        blk = grp[:, q * k2:(q + 1) * k2]
+        assert np.all(blk == blk[:, :1])
+    assert all(len(set(v)) == w.k_primary for v in grp[:, ::k2].tolist())
+    assert all(len(set(v)) == w.k for v in idx_g.tolist())
+    idx = r["idx"].copy()
+    idx[differ] = idx_g[differ]
+    gates_o = hier_gates_for(w, r["scores"], idx)
+    gerr = float(np.max(np.abs(g["topk_gate"].double().numpy() - gates_o))) if w.T else 0.0
+    assert gerr <= GATE_ATOL, gerr
+    nt = g["near_tie"].numpy().astype(bool)
+    assert not np.any(nt & (r["gap"] > 2 * NEAR_TIE))
+    assert not np.any(~nt & (r["gap"] < 0.5 * NEAR_TIE))
+    report.update(near_ties=int(near.sum()), choice_differs=int(differ.sum()), gate_abs_err=gerr)
+    return idx, gates_o
+
+
 def check_route(w, inp, g, report):
+    if w.gating == "hierarchical":
+        return check_route_hier(w, inp, g, report)
     r = orc.route(inp, w)
     idx_g = g["topk_idx"].long().numpy()
     assert idx_g.min() >= 0 and idx_g.max() < w.E

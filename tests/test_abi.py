@@ -30,11 +30,13 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_config_struct_layout():
-    # int64 T, six int32, float, three int32 -> 48 bytes with 8-byte alignment
-    assert ctypes.sizeof(moe.MoEConfig) == 48
+    # int64 T, six int32, float, five int32 -> 56 bytes with 8-byte alignment
+    assert ctypes.sizeof(moe.MoEConfig) == 56
     assert moe.MoEConfig.capacity_factor.offset == 32
     assert moe.MoEConfig.dtype.offset == 40
     assert moe.MoEConfig.hidden_f16.offset == 44
+    assert moe.MoEConfig.groups.offset == 48
+    assert moe.MoEConfig.k_primary.offset == 52
 
 
 def test_status_strings():
@@ -93,6 +95,12 @@ def test_route_validation():
     bad = _cfg()
     bad.hidden_f16 = 2
     assert _route(bad) == 1
+    # hierarchical gating: groups divide E, k_primary divides k, per-level limits
+    assert _route(_cfg(gating="hierarchical", E=16, k=4, groups=3, k_primary=2)) == 1
+    assert _route(_cfg(gating="hierarchical", E=16, k=4, groups=4, k_primary=3)) == 1
+    assert _route(_cfg(gating="hierarchical", E=16, k=4, groups=8, k_primary=1)) == 1  # 4 > b=2
+    assert _route(_cfg(gating="hierarchical", E=16, k=8, groups=2, k_primary=1)) == 2  # 8 per group
+    assert _route(_cfg(gating="hierarchical", E=256, k=4, groups=16, k_primary=2)) == 2  # 272 rows
     assert moe.lib.moe_route(None, FAKE, FAKE, None, None, None, FAKE, FAKE, None, None, None,
                              FAKE, None) == 1
 
@@ -125,9 +133,9 @@ def test_workspace_sizes():
     assert moe.moe_workspace_size(c) > 0
     assert moe.moe_forward_workspace_size(c) > moe.moe_workspace_size(c)
     assert moe.moe_workspace_size(_cfg(d_model=96)) == 0
-    # the forward workspace holds x_perm, h and y_perm of T*k rows
+    # the forward workspace holds h (bf16) and y_perm (fp32) of T*k rows
     big = _cfg(T=16384, d_model=768, d_ff=3072, E=128, k=1)
-    assert moe.moe_forward_workspace_size(big) >= 16384 * (768 + 3072 + 768) * 2
+    assert moe.moe_forward_workspace_size(big) >= 16384 * (3072 * 2 + 768 * 4)
 
 
 def test_python_binding_rejects_cpu_tensors():

@@ -51,6 +51,20 @@ SMALL = {
     # noisy gating with capacity drops (Importance still sums the gates before the drop)
     "noisy_capacity": Workload("nzc", T=900, d_model=128, d_ff=128, E=16, k=2,
                                gating="noisy_topk", capacity_factor=0.5),
+    # hierarchical (two-level) gating: 8 groups of 16 keeping 2 x 2; one kept group of
+    # 16 groups with capacity drops; 1 x 3 in fp32; 2 x 4 and 4 x 2 (the longest lists
+    # per level, k = 8)
+    "hier_8x16_k2x2": Workload("h1", T=1500, d_model=128, d_ff=128, E=128, k=4,
+                               gating="hierarchical", groups=8, k_primary=2, act="gelu"),
+    "hier_16x4_k1x1_cap": Workload("h2", T=1000, d_model=64, d_ff=128, E=64, k=1,
+                                   gating="hierarchical", groups=16, k_primary=1,
+                                   capacity_factor=1.0),
+    "hier_f32_3x4_k1x3": Workload("h3", T=300, d_model=64, d_ff=64, E=12, k=3,
+                                  gating="hierarchical", groups=3, k_primary=1, dtype="f32"),
+    "hier_4x16_k2x4": Workload("h4", T=700, d_model=128, d_ff=64, E=64, k=8,
+                               gating="hierarchical", groups=4, k_primary=2, act="relu"),
+    "hier_8x8_k4x2": Workload("h5", T=700, d_model=128, d_ff=64, E=64, k=8,
+                              gating="hierarchical", groups=8, k_primary=4, act="relu"),
 }
 
 
@@ -67,6 +81,7 @@ def test_steps_and_forward_small(name):
     H.check_ffn(w, inp, g, n, rep)
     H.check_combine(w, g, rep)
     H.check_end_to_end(w, inp, g, idx, gates, rep)
+    H.check_gather_path(w, g, rep)
     f = H.run_forward(w, dev)
     assert f["device_error"] == 0
     # the fused call runs the same kernels: identical results
@@ -152,6 +167,10 @@ FULL["k8_full_tiles_T12000"] = Workload("k8f", T=12_000, d_model=256, d_ff=256, 
 # just past the half-tile threshold (75 tiles of 128 > 148 / 2): 128-token tiles with a
 # ragged last tile
 FULL["noisy_full_tiles_ragged_T9473"] = W["noisy"].scaled(T=9_473)
+# hierarchical MoE at the noisy workload's size: 8 groups of 16 experts, 2 groups and 2
+# experts per group kept ("MoE-H" keeps 2 per level)
+FULL["hierarchical_T8192"] = Workload("hier", T=8192, d_model=512, d_ff=1024, E=128, k=4,
+                                      gating="hierarchical", groups=8, k_primary=2, act="relu")
 
 
 # workloads whose every expert row and every token the fp64 oracle checks at full size
@@ -204,6 +223,7 @@ def test_full_size_sampled(name):
                       | {0, w.T - 1})
         H.check_combine(w, g, rep, rows=toks)
         H.check_end_to_end(w, inp, g, idx, gates, rep, rows=toks)
+    H.check_gather_path(w, g, rep)
     f = H.run_forward(w, dev)
     assert f["device_error"] == 0
     assert torch.equal(f["y"], g["y"])
@@ -268,6 +288,11 @@ def test_permute_launch_path(name, launches):
     assert moe.last_launch_count() == launches
     assert moe.moe_get_error(ws) == 0
     assert o["counts"].tolist() == torch.bincount(idx.view(-1).long(), minlength=w.E).tolist()
+    # index arrays only: the three-kernel path leaves out its row-copy kernel
+    moe.moe_permute(cfg, idx, None, o["counts"], o["offsets"], o["perm_src"], o["slot_pos"],
+                    None, ws)
+    assert moe.last_launch_count() == min(launches, 2)
+    assert moe.moe_get_error(ws) == 0
 
 
 def test_forward_replays_from_a_cuda_graph():
