@@ -164,24 +164,23 @@ def algorithmic(w: workloads.Workload, n_kept: int, counts_kept, fused=False):
     """Algorithmic FLOPs and bytes of each step (kept assignments only, no padding).
 
     FFN FLOPs 4*N*d*f (two products).  FFN bytes: the weights of the experts that got
-    rows, the kept assignments' token rows (dtype, gathered from x by the up-projection)
-    and their source indices read, y_perm (fp32) written.  Route bytes: x, the gating
-    weights, noise, and the chosen indices and gates.  Permute (index arrays only): the
-    chosen experts read, slot_pos and perm_src written, counts and offsets.  Combine:
-    y_perm rows read, gates and slots, y written.  fused (k = 1, FFN and combine as one
-    step): the FFN writes every row of y (fp32) and reads each kept row's source index
-    and gate; no combine bytes."""
+    rows, x_perm (dtype) read, y_perm (fp32) written.  Route bytes: x, the gating
+    weights, noise, and the chosen indices and gates.  Permute: the chosen experts read,
+    slot_pos and perm_src written, counts and offsets, and the kept token rows read from
+    x and written to x_perm.  Combine: y_perm rows read, gates and slots, y written.
+    fused (k = 1, FFN and combine as one step): the FFN writes every row of y (fp32) and
+    reads each kept row's source index and gate; no combine bytes."""
     es = 2 if w.dtype == "bf16" else 4
     T, d, f, E, k = w.T, w.d_model, w.d_ff, w.E, w.k
     active = int(sum(1 for c in counts_kept if c > 0))
     ffn_flops = 4.0 * n_kept * d * f
-    ffn_bytes = active * 2.0 * d * f * es + n_kept * (d * es + 4.0) + n_kept * d * 4.0
+    ffn_bytes = active * 2.0 * d * f * es + n_kept * d * es + n_kept * d * 4.0
     noisy = w.gating == "noisy_topk"
     route_bytes = T * d * es + E * d * es * (2 if noisy else 1) + (T * E * 4 if noisy else 0) + T * k * 8
-    permute_bytes = T * k * 4 * 3 + E * 8.0
+    permute_bytes = T * k * 4 * 3 + E * 8.0 + n_kept * d * es * 2
     combine_bytes = n_kept * d * 4.0 + T * k * 8 + T * d * 4.0
     if fused:
-        ffn_bytes = active * 2.0 * d * f * es + n_kept * (d * es + 4.0) + T * d * 4.0 + n_kept * 8.0 + T * 4.0
+        ffn_bytes = active * 2.0 * d * f * es + n_kept * d * es + T * d * 4.0 + n_kept * 8.0 + T * 4.0
         combine_bytes = 0.0
     return {"ffn_flops": ffn_flops, "ffn_bytes": ffn_bytes, "route_bytes": route_bytes,
             "permute_bytes": permute_bytes, "combine_bytes": combine_bytes}
@@ -192,7 +191,8 @@ def algorithmic(w: workloads.Workload, n_kept: int, counts_kept, fused=False):
 # Tokens whose expert FFN and combine each oracle step evaluates (every (T/S)-th token);
 # routing and dispatch always cover all T tokens.  Sized so that one step takes about one
 # to four seconds on a 16-core host.
-ORACLE_SAMPLE = {"tiny": 512, "switch": 128, "noisy": 32, "gshard": 32, "zipf": 32}
+ORACLE_SAMPLE = {"tiny": 512, "switch": 128, "noisy": 32, "gshard": 32, "zipf": 32,
+                 "hierarchical": 32}
 
 
 def oracle_rows(w):
@@ -268,9 +268,11 @@ def run_reference(args, w):
 
 
 def config_json(w):
+    gate = {"noisy_topk": "", "hierarchical": "(%d groups, %d x %d kept)" % (
+        w.groups or 0, w.k_primary, w.k // max(w.k_primary, 1))}.get(
+        w.gating, "(renorm)" if w.renorm else "(full-softmax gate)")
     c = {"workload": "%s: T=%d d_model=%d d_ff=%d E=%d k=%d gating=%s%s cf=%s act=%s %s%s" % (
-        w.name, w.T, w.d_model, w.d_ff, w.E, w.k, w.gating,
-        "" if w.gating == "noisy_topk" else ("(renorm)" if w.renorm else "(full-softmax gate)"),
+        w.name, w.T, w.d_model, w.d_ff, w.E, w.k, w.gating, gate,
         w.capacity_factor, w.act, w.dtype,
         "" if w.zipf_s is None else " zipf_s=%s" % w.zipf_s),
         "T": w.T, "d_model": w.d_model, "d_ff": w.d_ff, "E": w.E, "k": w.k,
@@ -291,7 +293,8 @@ class LayerBench:
         d = {k: v.to(dev) for k, v in self.inp.items()}
         self.cfg = moe.make_config(w.T, w.d_model, w.d_ff, w.E, w.k, gating=w.gating,
                                    renorm=w.renorm, capacity_factor=w.capacity_factor, act=w.act,
-                                   dtype=w.dtype, hidden_f16=w.hidden_f16)
+                                   dtype=w.dtype, hidden_f16=w.hidden_f16, groups=w.groups,
+                                   k_primary=w.k_primary)
         self.d = moe.prepare_weights(self.cfg, d)  # fp16 w2 for fp16 hidden (exact re-encoding)
         T, k, E, dm, f = w.T, w.k, w.E, w.d_model, w.d_ff
         self.o = o = dict(
@@ -302,6 +305,7 @@ class LayerBench:
             offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
             perm_src=torch.empty(T * k, dtype=torch.int32, device=dev),
             slot_pos=torch.empty(T * k, dtype=torch.int32, device=dev),
+            x_perm=torch.empty(T * k, dm, dtype=w.torch_dtype, device=dev),
             h=torch.empty(T * k, f, dtype=torch.float16 if w.hidden_f16 else w.torch_dtype,
                           device=dev),
             y_perm=torch.empty(T * k, dm, dtype=torch.float32, device=dev),
@@ -326,23 +330,22 @@ class LayerBench:
         n += moe.last_launch_count()
         if evs:
             evs[1].record(st)
-        # index arrays only: the up-projection gathers the token rows from x itself
-        moe.moe_permute(cfg, o["idx"], None, o["counts"], o["offsets"], o["perm_src"],
-                        o["slot_pos"], None, self.ws)
+        moe.moe_permute(cfg, o["idx"], d["x"], o["counts"], o["offsets"], o["perm_src"],
+                        o["slot_pos"], o["x_perm"], self.ws)
         n += moe.last_launch_count()
         if evs:
             evs[2].record(st)
         if self.fused:
             # top-1: the down-projection writes gate * row straight into y
-            moe.moe_expert_ffn_combine_gather(cfg, d["x"], o["offsets"], o["perm_src"],
-                                              o["slot_pos"], o["gate"], d["w1"], d["w2"], o["h"],
-                                              o["y"], self.ws)
+            moe.moe_expert_ffn_combine(cfg, o["x_perm"], o["offsets"], o["perm_src"],
+                                       o["slot_pos"], o["gate"], d["w1"], d["w2"], o["h"], o["y"],
+                                       self.ws)
             n += moe.last_launch_count()
             if evs:
                 evs[3].record(st)
         else:
-            moe.moe_expert_ffn_gather(cfg, d["x"], o["perm_src"], o["offsets"], d["w1"], d["w2"],
-                                      o["h"], o["y_perm"], self.ws)
+            moe.moe_expert_ffn(cfg, o["x_perm"], o["offsets"], d["w1"], d["w2"], o["h"],
+                               o["y_perm"], self.ws)
             n += moe.last_launch_count()
             if evs:
                 evs[3].record(st)
@@ -667,10 +670,15 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="time only the headline workload")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="run the workload with this many tokens instead of its own T (small "
+                         "cases for profiler captures; not a benchmark figure)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = workloads.WORKLOADS[args.workload]
+    if args.tokens is not None:
+        w = w.scaled(T=args.tokens)
     if args.impl == "reference":
         run_reference(args, w)
     else:

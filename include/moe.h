@@ -146,7 +146,7 @@ int64_t moe_capacity(const moe_config* cfg);
 size_t moe_workspace_size(const moe_config* cfg);
 
 /* Bytes of workspace moe_forward needs: the step workspace plus the intermediates
- * (offsets, slot_pos, perm_src, h, y_perm) it keeps there. */
+ * (offsets, slot_pos, perm_src, x_perm, h, y_perm) it keeps there. */
 size_t moe_forward_workspace_size(const moe_config* cfg);
 
 /* Router product and gate [Shazeer et al., "Noisy Top-K Gating"; Switch Transformer,
@@ -252,9 +252,9 @@ moe_status moe_expert_ffn_combine_gather(const moe_config* cfg, const void* x,
                                          const void* w1, const void* w2, void* h, void* y,
                                          void* ws, moe_stream_t stream);
 
-/* The whole layer forward on one stream: moe_route, moe_permute (index arrays only),
- * moe_expert_ffn_gather, moe_combine (moe_expert_ffn_combine_gather in place of the last
- * two when k = 1 and dtype is bf16).  Inputs as in the step calls; y [T, d_model] fp32 out.  topk_idx,
+/* The whole layer forward on one stream: moe_route, moe_permute, moe_expert_ffn,
+ * moe_combine (moe_expert_ffn_combine in place of the last two when k = 1 and dtype is
+ * bf16).  Inputs as in the step calls; y [T, d_model] fp32 out.  topk_idx,
  * topk_gate (both [T, k]) and counts ([E]) are outputs the caller must provide;
  * importance, load and near_tie may be NULL.  The intermediates live in `ws`
  * (moe_forward_workspace_size bytes). */

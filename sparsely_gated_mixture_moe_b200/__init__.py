@@ -50,7 +50,7 @@ def _load():
         "moe_train_state_size": (ctypes.c_size_t, [C]),
         "moe_backward_workspace_size": (ctypes.c_size_t, [C]),
         "moe_forward_train": (ctypes.c_int, [C] + [P] * 17),
-        "moe_backward": (ctypes.c_int, [C] + [P] * 14 + [ctypes.c_float, ctypes.c_float] +
+        "moe_backward": (ctypes.c_int, [C] + [P] * 13 + [ctypes.c_float, ctypes.c_float] +
                          [P] * 10),
         "moe_wait_timeout_check": (ctypes.c_int, [P, P]),
     }

@@ -56,7 +56,7 @@ moe_status check_config(const moe_config* c) {
 
 struct Layout {
   size_t err, blk, partials, logits, nz, steps;                  // step workspace
-  size_t offsets, slot_pos, perm_src, h, y_perm, forward;  // + forward intermediates
+  size_t offsets, slot_pos, perm_src, x_perm, h, y_perm, forward;  // + forward intermediates
 };
 
 Layout layout(const moe_config* c) {
@@ -84,6 +84,8 @@ Layout layout(const moe_config* c) {
   o = align_up(o + static_cast<size_t>(n) * 4);
   L.perm_src = o;
   o = align_up(o + static_cast<size_t>(n) * 4);
+  L.x_perm = o;
+  o = align_up(o + static_cast<size_t>(n) * c->d_model * esize(c));
   L.h = o;
   o = align_up(o + static_cast<size_t>(n) * c->d_ff * esize(c));
   L.y_perm = o;
@@ -577,21 +579,22 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_gate,
   int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
   int32_t* slot_pos = reinterpret_cast<int32_t*>(w + L.slot_pos);
   int32_t* perm_src = reinterpret_cast<int32_t*>(w + L.perm_src);
+  void* x_perm = w + L.x_perm;
   void* h = w + L.h;
   void* y_perm = w + L.y_perm;
   st = do_route(cfg, L, x, w_gate, w_noise, noise, logit_bias, topk_idx, topk_gate, importance, load,
                 near_tie, ws, ctx);
   if (st != MOE_OK) return st;
-  // index arrays only: the up-projection gathers the token rows from x itself
-  st = do_permute(cfg, L, topk_idx, x, counts, offsets, perm_src, slot_pos, nullptr, ws, ctx);
+  // the kept rows are copied into x_perm once and read by tiled TMA loads: measured
+  // faster than gathering them inside the up-projection (tile::gather4)
+  st = do_permute(cfg, L, topk_idx, x, counts, offsets, perm_src, slot_pos, x_perm, ws, ctx);
   if (st != MOE_OK) return st;
   if (fused_combine(cfg)) {
-    st = do_ffn_combine(cfg, nullptr, offsets, perm_src, slot_pos, topk_gate, w1, w2, h, y, ctx, x,
-                        true);
+    st = do_ffn_combine(cfg, x_perm, offsets, perm_src, slot_pos, topk_gate, w1, w2, h, y, ctx);
     if (st != MOE_OK) return st;
     return ctx.finish(cudaSuccess);
   }
-  st = do_ffn(cfg, nullptr, offsets, w1, w2, h, y_perm, ctx, x, perm_src);
+  st = do_ffn(cfg, x_perm, offsets, w1, w2, h, y_perm, ctx);
   if (st != MOE_OK) return st;
   st = do_combine(cfg, y_perm, slot_pos, topk_gate, y, ctx);
   if (st != MOE_OK) return st;

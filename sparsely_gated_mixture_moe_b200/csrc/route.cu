@@ -558,8 +558,20 @@ struct RouteTcArgs {
   int ntiles;     // ceil(T / 128), or ceil(T / 64) with half tiles
   int gate_off;   // byte offset of the gate scratch in shared memory
   int bar_off;    // byte offset of the barriers
+  const uint8_t* x;  // token rows, for L2 prefetches of each tile's contiguous rows
+  int row_bytes;     // bytes of one token row of x
   int* err;
 };
+
+// Prefetches into L2 the contiguous rows of x (and of the noise) of token tile L.
+__device__ __forceinline__ void prefetch_route_tile(const RouteTcArgs& a, int L) {
+  if (L >= a.ntiles) return;
+  const int ntok = a.half ? 64 : 128;
+  const int64_t t0 = static_cast<int64_t>(L) * ntok;
+  const int64_t n = min(static_cast<int64_t>(ntok), a.g.T - t0);
+  l2_prefetch_range(a.x + t0 * a.row_bytes, static_cast<uint64_t>(n) * a.row_bytes);
+  if (a.g.noisy) l2_prefetch_range(a.g.noise + t0 * a.g.E, static_cast<uint64_t>(n) * a.g.E * 4);
+}
 
 __device__ __forceinline__ void gate_bar_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
@@ -627,7 +639,9 @@ __global__ void __launch_bounds__(64 + 128 * G)
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_par = 0;
       bool aborted = false;
+      prefetch_route_tile(a, blockIdx.x);
       for (int L = blockIdx.x; L < a.ntiles && !aborted; L += gridDim.x) {
+        prefetch_route_tile(a, L + gridDim.x);  // the next tile's rows, one tile ahead
         for (int kb = 0; kb < a.kblocks; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, s_abort)) {
             aborted = true;
@@ -921,6 +935,8 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   a.stages = stages;
   a.gate_off = stages * stage_bytes;
   a.bar_off = a.gate_off + (scratch + 127) / 128 * 128;
+  a.x = static_cast<const uint8_t*>(p.x);
+  a.row_bytes = p.d * 2;
   a.err = c.err;
   const int smem = 1024 + a.bar_off + 8 * (2 * stages + 5) + 16;
 

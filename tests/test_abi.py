@@ -133,9 +133,9 @@ def test_workspace_sizes():
     assert moe.moe_workspace_size(c) > 0
     assert moe.moe_forward_workspace_size(c) > moe.moe_workspace_size(c)
     assert moe.moe_workspace_size(_cfg(d_model=96)) == 0
-    # the forward workspace holds h (bf16) and y_perm (fp32) of T*k rows
+    # the forward workspace holds x_perm, h (bf16) and y_perm (fp32) of T*k rows
     big = _cfg(T=16384, d_model=768, d_ff=3072, E=128, k=1)
-    assert moe.moe_forward_workspace_size(big) >= 16384 * (3072 * 2 + 768 * 4)
+    assert moe.moe_forward_workspace_size(big) >= 16384 * (768 * 2 + 3072 * 2 + 768 * 4)
 
 
 def test_python_binding_rejects_cpu_tensors():

@@ -75,8 +75,8 @@ def test_algorithmic_counts_switch():
     a = bench.algorithmic(w, 16384, kept)
     assert a["ffn_flops"] == 4.0 * 16384 * 768 * 3072
     weights = 128 * 2 * 768 * 3072 * 2
-    assert a["ffn_bytes"] == weights + 16384 * (768 * 2 + 4) + 16384 * 768 * 4
-    assert a["permute_bytes"] == 16384 * 12 + 128 * 8
+    assert a["ffn_bytes"] == weights + 16384 * 768 * 2 + 16384 * 768 * 4
+    assert a["permute_bytes"] == 16384 * 12 + 128 * 8 + 16384 * 768 * 2 * 2
     assert a["route_bytes"] == 16384 * 768 * 2 + 128 * 768 * 2 + 16384 * 8
 
 

@@ -13,9 +13,14 @@ from oracle import moe_oracle as orc
 
 def test_five_workloads_shapes():
     W = workloads.WORKLOADS
-    assert [W[n].T for n in workloads.ORDER] == [512, 16384, 8192, 32768, 65536]
-    assert [W[n].k for n in workloads.ORDER] == [2, 1, 4, 2, 2]
-    assert [W[n].E for n in workloads.ORDER] == [8, 128, 256, 64, 16]
+    five = ["tiny", "switch", "noisy", "gshard", "zipf"]
+    assert workloads.ORDER[:5] == five
+    assert [W[n].T for n in five] == [512, 16384, 8192, 32768, 65536]
+    assert [W[n].k for n in five] == [2, 1, 4, 2, 2]
+    assert [W[n].E for n in five] == [8, 128, 256, 64, 16]
+    h = W["hierarchical"]
+    assert (h.groups, h.k_primary, h.E, h.k) == (8, 2, 128, 4)
+    assert workloads.make_inputs(h.scaled(T=4, d_ff=64))["w_gate"].shape == (8 + 128, 512)
     assert orc.capacity(W["switch"].capacity_factor, 16384, 1, 128) == 160
     assert orc.capacity(W["gshard"].capacity_factor, 32768, 2, 64) == 2048
 

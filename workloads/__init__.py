@@ -107,8 +107,13 @@ WORKLOADS: Dict[str, Workload] = {
     "zipf": Workload("zipf", T=65536, d_model=1024, d_ff=4096, E=16, k=2,
                      gating="softmax_topk", renorm=True, capacity_factor=None,
                      act="gelu", dtype="bf16", zipf_s=1.2),
+    # a two-level (hierarchical) layer at the noisy workload's size: 8 groups of 16
+    # experts, 2 groups and 2 experts in each kept ("MoE-H" keeps 2 per level)
+    "hierarchical": Workload("hierarchical", T=8192, d_model=512, d_ff=1024, E=128, k=4,
+                             gating="hierarchical", groups=8, k_primary=2, act="relu",
+                             dtype="bf16"),
 }
-ORDER = ["tiny", "switch", "noisy", "gshard", "zipf"]
+ORDER = ["tiny", "switch", "noisy", "gshard", "zipf", "hierarchical"]
 
 
 def zipf_beta() -> float:
