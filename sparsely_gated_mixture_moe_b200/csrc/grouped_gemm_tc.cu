@@ -53,6 +53,11 @@ constexpr int MAX_GROUPS = 1024;
 constexpr int TMEM_COLS = 512;              // two accumulators of up to 256 columns
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES_MAX;
 constexpr int RING_BYTES = STAGES * STAGE_BYTES;  // 192 KB
+// CTA pairs load half of each B box, so the same ring holds 6 stages of 32 KB
+constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_STAGE_BYTES = A_BYTES + B_BYTES_MAX / 2;
+static_assert(PAIR_STAGES * PAIR_STAGE_BYTES <= RING_BYTES, "pair ring fits the ring");
+static_assert(2 * PAIR_STAGES + 5 <= 28, "barriers fit their 256 bytes with the flags");
 constexpr int SMEM_BYTES = 1024 /*align slack*/ + RING_BYTES + 256 /*barriers, flags*/ +
                            4 * (MAX_GROUPS + 1 + 40);
 
@@ -179,16 +184,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  // stage s: A tile at ring + s * STAGE_BYTES, then the B tile
+  // stage s: A tile at ring + s * SB, then the B tile
+  constexpr int NST = PAIR ? PAIR_STAGES : STAGES;        // stages of the ring
+  constexpr int SB = PAIR ? PAIR_STAGE_BYTES : STAGE_BYTES;  // bytes of one stage
   uint8_t* ring = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RING_BYTES);
-  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+  // bars: full[NST], empty[NST], tfull[2], tempty[2], drain
   const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = smem_u32(bars + STAGES);
-  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
-  const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
-  const uint32_t drain = smem_u32(bars + 2 * STAGES + 4);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  const uint32_t empty0 = smem_u32(bars + NST);
+  const uint32_t tfull0 = smem_u32(bars + 2 * NST);
+  const uint32_t tempty0 = smem_u32(bars + 2 * NST + 2);
+  const uint32_t drain = smem_u32(bars + 2 * NST + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * NST + 5);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* scratch = reinterpret_cast<int*>(smem + RING_BYTES + 256);
   int* tp = scratch + 40;
@@ -200,7 +207,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int stride = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
@@ -277,7 +284,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           aborted = true;
           break;
         }
-        uint8_t* st = ring + stage * STAGE_BYTES;
+        uint8_t* st = ring + stage * SB;
         const uint32_t fb = full_bar(stage);
         if (lane == 0 && rank == 0) mbar_arrive_expect_tx(full0 + 8 * stage, stage_tx);
         __syncwarp();
@@ -290,7 +297,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         armed |= 1u << stage;
         armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-        if (++stage == STAGES) {
+        if (++stage == NST) {
           stage = 0;
           phase ^= 1;
         }
@@ -302,7 +309,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // let every copy this warp started land before the CTA releases its smem (a pair's
       // second CTA cannot watch rank 0's barrier: it waits out a fixed drain time)
       if (rank == 0) {
-        for (int s = 0; s < STAGES; ++s)
+        for (int s = 0; s < NST; ++s)
           if (armed & (1u << s)) mbar_wait(full0 + 8 * s, (armed_par >> s) & 1, nullptr, kDrainLimitNs);
       } else {
         const unsigned long long t0 = globaltimer_ns();
@@ -331,7 +338,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             aborted = true;
             break;
           }
-          uint8_t* st = ring + stage * STAGE_BYTES;
+          uint8_t* st = ring + stage * SB;
           const uint32_t fb = full_bar(stage);
           if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * stage, stage_tx);
           if constexpr (PAIR) {
@@ -343,7 +350,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1;
           }
@@ -354,7 +361,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         *s_abort = 1;
         // let every copy this thread started land before the CTA releases its smem
         if (rank == 0) {
-          for (int s = 0; s < STAGES; ++s)
+          for (int s = 0; s < NST; ++s)
             if (armed & (1u << s)) mbar_wait(full0 + 8 * s, (armed_par >> s) & 1, nullptr, kDrainLimitNs);
         } else {
           const unsigned long long t0 = globaltimer_ns();
@@ -382,7 +389,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(ring + stage * STAGE_BYTES);
+          const uint32_t a0 = smem_u32(ring + stage * SB);
           const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
@@ -399,7 +406,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           } else {
             tc_commit(empty0 + 8 * stage);
           }
-          if (++stage == STAGES) {
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1;
           }

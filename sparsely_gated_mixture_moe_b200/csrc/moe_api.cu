@@ -55,7 +55,7 @@ moe_status check_config(const moe_config* c) {
 }
 
 struct Layout {
-  size_t err, blk, partials, logits, nz, steps;                  // step workspace
+  size_t err, blk, partials, logits, nz, lw, sw, kw, steps;      // step workspace
   size_t offsets, slot_pos, perm_src, x_perm, h, y_perm, forward;  // + forward intermediates
 };
 
@@ -76,6 +76,15 @@ Layout layout(const moe_config* c) {
     o = align_up(o + static_cast<size_t>(c->T) * cols * 4);
     L.nz = o;
     if (c->gating == MOE_GATE_NOISY_TOPK) o = align_up(o + static_cast<size_t>(c->T) * c->E * 4);
+  }
+  L.lw = L.sw = L.kw = o;
+  if (c->dtype == MOE_BF16 && c->gating == MOE_GATE_NOISY_TOPK) {
+    // the per-token values the Importance/Load sums are formed from
+    o = align_up(o + static_cast<size_t>(c->T) * c->E * 4);
+    L.sw = o;
+    o = align_up(o + static_cast<size_t>(c->T) * c->E * 4);
+    L.kw = o;
+    o = align_up(o + static_cast<size_t>(c->T) * 2 * 4);
   }
   L.steps = o;
   L.offsets = o;
@@ -238,6 +247,11 @@ moe_status do_route(const moe_config* cfg, const Layout& L, const void* x, const
   p.partials = reinterpret_cast<float*>(w + L.partials);
   p.logits_ws = reinterpret_cast<float*>(w + L.logits);
   p.nz_ws = reinterpret_cast<float*>(w + L.nz);
+  if (cfg->dtype == MOE_BF16 && cfg->gating == MOE_GATE_NOISY_TOPK) {
+    p.lw = reinterpret_cast<float*>(w + L.lw);
+    p.sw = reinterpret_cast<float*>(w + L.sw);
+    p.kw = reinterpret_cast<float*>(w + L.kw);
+  }
   cudaError_t e = cfg->dtype == MOE_BF16 ? launch_route_bf16(p, ctx.lc) : launch_route_f32(p, ctx.lc);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

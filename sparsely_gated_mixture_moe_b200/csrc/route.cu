@@ -50,6 +50,13 @@ struct GateArgs {
   float* topk_gate;
   uint8_t* near_tie;
   float* partials;  // [gridDim.x][2][E] or null
+  // noisy gating with Importance/Load asked for, on the tensor-core path: the gate writes
+  // each token's clean logits (bias added) and Softplus(x.W_noise) [T, E] and its k-th and
+  // (k+1)-th noisy scores [T, 2] here instead of forming the sums itself
+  // (importance_load_kernel does, over the whole grid); null otherwise
+  float* lw;
+  float* sw;
+  float* kw;
 };
 
 // Softplus(z) = max(z, 0) + log(1 + e^-|z|), with the fast exponential and logarithm:
@@ -230,7 +237,14 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
         float sv = -INFINITY;
         if (e < E) {
           sv = l[jj] + sbias[e];
-          if (noisy) sv += nz[j] * softplus_f(z[jj]);
+          if (noisy) {
+            const float sp = softplus_f(z[jj]);
+            if (g.lw != nullptr && valid) {
+              g.lw[t * E + e] = sv;
+              g.sw[t * E + e] = sp;
+            }
+            sv = __fmaf_rn(nz[j], sp, sv);  // H; recomputed bit for bit by the Load sums
+          }
         }
         sc[jj] = sv;
       }
@@ -343,9 +357,13 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
     }
     fkth[row * 2 + 0] = kth;
     fkth[row * 2 + 1] = kth1;
+    if (g.kw != nullptr && valid) {
+      g.kw[t * 2 + 0] = kth;
+      g.kw[t * 2 + 1] = kth1;
+    }
   }
-  if (g.partials == nullptr) {  // uniform across the gate threads
-    sync();                     // the lists are reused by the next tile
+  if (g.partials == nullptr || g.lw != nullptr) {  // uniform across the gate threads
+    sync();                                        // the lists are reused by the next tile
     return;
   }
   sync();
@@ -383,7 +401,7 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
                 // recomputed exactly as in pass 1, so H >= kth means "among the top k"
                 const float li = l[jj] + sbias[e];
                 const float sp = softplus_f(z[jj]);
-                const float H = li + nz[j] * sp;
+                const float H = __fmaf_rn(nz[j], sp, li);
                 const float ex = (H >= kth) ? kth1 : kth;  // kth_excluding(H, k, e)
                 // Phi((l_e - kth_excluding) / Softplus(z_e))
                 pl[jj] = 0.5f + 0.5f * erf_as7126(__fdividef(li - ex, sp) * 0.70710678118654752f);
@@ -843,6 +861,56 @@ __global__ void __launch_bounds__(128, 1)
                          static_cast<int>(threadIdx.x) & 31, static_cast<int64_t>(blockIdx.x), g);
 }
 
+// Importance and Load partial sums of noisy gating from the gate's per-token values:
+// block (cb, chunk) covers experts 32*cb .. 32*cb+31 (one per lane) and a run of tokens;
+// its 8 warps take every 8th token of the run.  For token t and expert e:
+//   Importance term: the gate of e if e is one of t's chosen experts, else 0
+//   Load term: P(t, e) = Phi((l_te - kth_excluding(H_t, k, e)) / Softplus(z_te)), with
+//   H_te = l_te + noise_te * Softplus(z_te) and kth_excluding = the (k+1)-th largest
+//   score when H_te >= the k-th largest, else the k-th largest.
+// The 8 warps' sums are added in warp order into partials[chunk][2][E], so the result
+// does not depend on scheduling.
+__global__ void __launch_bounds__(256)
+    importance_load_kernel(const float* __restrict__ lw, const float* __restrict__ sw,
+                           const float* __restrict__ kw, const float* __restrict__ noise,
+                           const int32_t* __restrict__ topk_idx,
+                           const float* __restrict__ topk_gate, int64_t T, int E, int k,
+                           int64_t chunk_tokens, int want_load, float* __restrict__ partials) {
+  __shared__ float s_imp[8][32], s_load[8][32];
+  grid_dep_wait();
+  grid_dep_launch();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 32 + lane;
+  const int64_t t_lo = static_cast<int64_t>(blockIdx.y) * chunk_tokens;
+  const int64_t t_hi = min(T, t_lo + chunk_tokens);
+  float si = 0.0f, sl = 0.0f;
+  for (int64_t t = t_lo + warp; t < t_hi; t += 8) {
+    float gi = 0.0f;
+    for (int j = 0; j < k; ++j)
+      if (__ldg(topk_idx + t * k + j) == e) gi = __ldg(topk_gate + t * k + j);
+    si += gi;
+    if (want_load && e < E) {
+      const float li = __ldg(lw + t * E + e), sp = __ldg(sw + t * E + e);
+      const float H = __fmaf_rn(__ldg(noise + t * E + e), sp, li);  // as the gate formed it
+      const float kth = __ldg(kw + t * 2), kth1 = __ldg(kw + t * 2 + 1);
+      const float ex = (H >= kth) ? kth1 : kth;
+      sl += 0.5f + 0.5f * erf_as7126(__fdividef(li - ex, sp) * 0.70710678118654752f);
+    }
+  }
+  s_imp[warp][lane] = si;
+  s_load[warp][lane] = sl;
+  __syncthreads();
+  if (warp == 0 && e < E) {
+    float a = 0.0f, b = 0.0f;
+    for (int w = 0; w < 8; ++w) {
+      a += s_imp[w][lane];
+      b += s_load[w][lane];
+    }
+    partials[(blockIdx.y * 2 + 0) * static_cast<int64_t>(E) + e] = a;
+    partials[(blockIdx.y * 2 + 1) * static_cast<int64_t>(E) + e] = b;
+  }
+}
+
 __global__ void finalize_importance_load_kernel(const float* __restrict__ partials, int nblocks,
                                                 int E, float* importance, float* load) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
@@ -875,6 +943,7 @@ static GateArgs gate_args(const RouteProblem& p) {
   g.topk_gate = p.topk_gate;
   g.near_tie = p.near_tie;
   g.partials = (p.importance || p.load) ? p.partials : nullptr;
+  g.lw = g.sw = g.kw = nullptr;
   return g;
 }
 
@@ -909,9 +978,39 @@ static cudaError_t launch_route_tc_hier(int kg, const CUtensorMap& tmX, const CU
   }
 }
 
+// Noisy gating on the tensor-core path with Importance or Load asked for: after the
+// router kernel, the sums over the whole grid (importance_load_kernel), then the fixed-
+// order total over the chunks.
+static cudaError_t launch_importance_load(const RouteProblem& p, const LaunchCtx& c) {
+  const int cb = (p.E + 31) / 32;
+  // about four blocks per SM, at most one chunk per 64 tokens (the partials' rows)
+  int64_t chunks = (4LL * c.num_sms + cb - 1) / cb;
+  const int64_t cap = route_blocks(p.T);
+  if (chunks > cap) chunks = cap;
+  if (chunks < 1) chunks = 1;
+  const int64_t per = (p.T + chunks - 1) / chunks;
+  chunks = (p.T + per - 1) / per;
+  cudaError_t e = launch_kernel(importance_load_kernel, dim3(cb, static_cast<unsigned>(chunks)),
+                                dim3(256), 0, c, static_cast<const float*>(p.lw),
+                                static_cast<const float*>(p.sw), static_cast<const float*>(p.kw),
+                                p.noise, static_cast<const int32_t*>(p.topk_idx),
+                                static_cast<const float*>(p.topk_gate), p.T, p.E, p.k, per,
+                                p.load != nullptr ? 1 : 0, p.partials);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(finalize_importance_load_kernel, dim3((p.E + 127) / 128), dim3(128), 0, c,
+                       static_cast<const float*>(p.partials), static_cast<int>(chunks), p.E,
+                       p.importance, p.load);
+}
+
 cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   RouteTcArgs a;
   a.g = gate_args(p);
+  const bool split = p.noisy && (p.importance || p.load) && p.lw != nullptr;
+  if (split) {
+    a.g.lw = p.lw;
+    a.g.sw = p.sw;
+    a.g.kw = p.kw;
+  }
   const int n_scores = p.hier ? p.E + p.groups : p.E;  // score columns (rows of w_gate)
   a.e_pad = (n_scores + 15) / 16 * 16;
   a.acc_cols = 32;
@@ -968,6 +1067,7 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
     default: e = launch_route_tc<8>(tmX, tmG, tmN, a, smem, grid, c); break;
   }
   if (e != cudaSuccess) return e;
+  if (split) return launch_importance_load(p, c);
   return launch_finalize(p, a.ntiles, c);
 }
 
