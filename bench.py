@@ -559,6 +559,80 @@ def end_to_end(lb, flush, steps, world, dev, stream):
                     "steps (each step's x arrives by H2D)"}
 
 
+def training_step(lb, flush, steps, world, dev, stream):
+    """The training step of the same layer: moe_forward_train, then moe_backward of
+    L = sum(dy * y) + 0.01 CV(Importance)^2 (+ 0.01 CV(Load)^2 for noisy gating), timed
+    with CUDA events (L2 flushed before each step).  Algorithmic FLOPs: the forward's two
+    expert products and the backward's four (dgrad and wgrad of each), 12 N d f."""
+    import torch.distributed as dist
+    moe, w, d = lb.moe, lb.w, lb.d
+    cfg = lb.cfg
+    T, k, E, dm, f = w.T, w.k, w.E, w.d_model, w.d_ff
+    if moe.lib.moe_train_state_size(__import__("ctypes").byref(cfg)) == 0:
+        return {"unavailable": "no backward pass for this configuration"}
+    noisy = lb.noisy
+    o = {"y": torch.empty(T, dm, device=dev), "idx": torch.empty(T, k, dtype=torch.int32, device=dev),
+         "gate": torch.empty(T, k, device=dev), "counts": torch.empty(E, dtype=torch.int32, device=dev),
+         "imp": torch.empty(E, device=dev), "load": torch.empty(E, device=dev) if noisy else None,
+         "dx": torch.empty(T, dm, device=dev), "dwg": torch.empty(E, dm, device=dev),
+         "dwn": torch.empty(E, dm, device=dev) if noisy else None,
+         "dbias": torch.empty(E, device=dev) if "logit_bias" in d else None,
+         "dw1": torch.empty(E, f, dm, device=dev), "dw2": torch.empty(E, dm, f, device=dev),
+         "dg": torch.empty(T, k, device=dev)}
+    g = torch.Generator().manual_seed(77)
+    dy = torch.randn(T, dm, generator=g).to(dev)
+    state = moe.train_state(cfg, dev)
+    ws = moe.backward_workspace(cfg, dev)
+    w_load = 0.01 if noisy else 0.0
+
+    def one(evs=None):
+        if evs:
+            evs[0].record(stream)
+        moe.moe_forward_train(cfg, d["x"], d["w_gate"], d["w1"], d["w2"], o["y"], o["idx"], o["gate"],
+                              o["counts"], state, ws, w_noise=d.get("w_noise"), noise=d.get("noise"),
+                              logit_bias=d.get("logit_bias"), importance=o["imp"], load=o["load"])
+        nf = moe.last_launch_count()
+        if evs:
+            evs[1].record(stream)
+        moe.moe_backward(cfg, d["x"], d["w_gate"], d["w1"], d["w2"], o["idx"], o["gate"], state, dy,
+                         o["dx"], o["dwg"], o["dw1"], o["dw2"], o["dg"], ws, w_noise=d.get("w_noise"),
+                         noise=d.get("noise"), logit_bias=d.get("logit_bias"), importance=o["imp"],
+                         load=o["load"], w_importance=0.01, w_load=w_load, dw_noise=o["dwn"],
+                         dlogit_bias=o["dbias"])
+        if evs:
+            evs[2].record(stream)
+        return nf + moe.last_launch_count()
+
+    for _ in range(3):
+        flush(1)
+        one()
+    torch.cuda.synchronize(dev)
+    if moe.moe_get_error(ws):
+        raise RuntimeError("device error word set in the training step")
+    n = max(3, min(steps, 20))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    if world > 1:
+        dist.barrier()
+    launches = 0
+    for i in range(n):
+        flush(i)
+        launches += one(evs[i])
+    torch.cuda.synchronize(dev)
+    fwd = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    bwd = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    fwd, bwd = max_over_ranks(fwd, dev), max_over_ranks(bwd, dev)
+    offs = lb.o["offsets"].cpu().tolist()
+    n_kept = offs[-1]
+    bwd_flops = 8.0 * n_kept * dm * f
+    return {"value": T * world / ((fwd + bwd) * 1e-3), "unit": "tokens/s",
+            "forward_train_ms": fwd, "backward_ms": bwd, "steps": n,
+            "backward_expert_tflops": bwd_flops / (bwd * 1e-3) / 1e12,
+            "gpu_launches_per_step": launches / n,
+            "loss": "sum(dy*y) + 0.01 CV(Importance)^2" + (" + 0.01 CV(Load)^2" if noisy else ""),
+            "note": "backward_expert_tflops counts the four expert products (8 N d f) over the "
+                    "whole backward call (router, gate and loss kernels included)"}
+
+
 def run_gpu(args, w):
     import torch.distributed as dist
     import sparsely_gated_mixture_moe_b200 as moe
@@ -594,6 +668,7 @@ def run_gpu(args, w):
                       "note": "one step (route, permute, expert FFN, combine) captured once and "
                               "replayed; L2 flushed before each replay"}
     e2e = end_to_end(lb, flush, args.steps, world, dev, stream)
+    train = training_step(lb, flush, args.steps, world, dev, stream) if not args.no_training else None
 
     eg = main["expert_gemm"]
     ffn_ms = main["steps_ms"]["expert_ffn"]
@@ -624,6 +699,8 @@ def run_gpu(args, w):
     }
     line.update({kk: v for kk, v in main.items() if kk not in ("value", "unit", "ms_per_step")})
     line.update({"e2e": e2e, "graph": graph_info, "gpu_launches": timed_launches, "clocks": clocks})
+    if train is not None:
+        line["training_step"] = train
     inp_main = lb.inp
     del lb
     torch.cuda.empty_cache()
@@ -670,6 +747,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="time only the headline workload")
+    ap.add_argument("--no-training", action="store_true",
+                    help="skip the training-step (forward + backward) figure")
     ap.add_argument("--tokens", type=int, default=None,
                     help="run the workload with this many tokens instead of its own T (small "
                          "cases for profiler captures; not a benchmark figure)")

@@ -111,22 +111,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Asks L2 to fetch `bytes` (a multiple of 16) of global memory from `src` (16-byte
-// aligned) ahead of the loads that will read it, in pieces of at most 64 KB: one long
-// sequential fetch instead of the 128-byte pieces of many rows that 2-D TMA boxes request
-// (the pieces of one row then arrive at different times and each reopens its DRAM page).
-__device__ __forceinline__ void l2_prefetch_range(const void* src, uint64_t bytes) {
-  const char* p = static_cast<const char*>(src);
-  while (bytes > 0) {
-    const uint32_t n = bytes > 65536 ? 65536u : static_cast<uint32_t>(bytes);
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
-                 "r"(n)
-                 : "memory");
-    p += n;
-    bytes -= n;
-  }
-}
-
 // Four rows of a 2-D tensor, each one box of [1 row x box-width columns] at column x,
 // gathered into consecutive rows of this CTA's shared memory (TMA tile::gather4); rows
 // r0..r3 may be any rows of the tensor, in any order.  The tensor map's box is one row

@@ -86,8 +86,6 @@ struct Args {
   int gather_k;               // A tensor (the token rows x), gathered by the TMA itself
   void* pre;                  // OUT_BF16 / OUT_F16 with an activation: also store the
                               // pre-activation there (same type and layout as out), or null
-  const uint8_t* a_ptr;       // the A rows (x_perm) and the weights, for L2 prefetches of
-  const uint8_t* b_ptr;       // each tile's contiguous rows (a_ptr null when gathering)
   int* err;
 };
 
@@ -274,9 +272,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         g3 = __ldg(a.gather_src + t.row0 + min(r + 3, last)) / a.gather_k;
       }
       const int brow = t.e * a.N + t.nt * a.bn + static_cast<int>(rank) * b_rows;
-      if (lane == 0)
-        l2_prefetch_range(a.b_ptr + static_cast<int64_t>(brow) * a.K * 2,
-                          static_cast<uint64_t>(b_rows) * a.K * 2);
       for (int kb = 0; kb < kblocks; ++kb) {
         int okw = 1;
         if (lane == 0) okw = mbar_wait(empty0 + 8 * stage, phase ^ 1, s_abort) ? 1 : 0;
@@ -326,13 +321,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         const Tile t = decode_tile(L, tp, a, TBM);
         const int brow = t.e * a.N + t.nt * a.bn + static_cast<int>(rank) * b_rows;
         const int arow = t.row0 + static_cast<int>(rank) * BM;
-        // this tile's weight rows and A rows are contiguous runs of memory: fetch them into
-        // L2 as such, ahead of the k-block boxes
-        l2_prefetch_range(a.b_ptr + static_cast<int64_t>(brow) * a.K * 2,
-                          static_cast<uint64_t>(b_rows) * a.K * 2);
-        if (arow < a.rows_cap)
-          l2_prefetch_range(a.a_ptr + static_cast<int64_t>(arow) * a.K * 2,
-                            static_cast<uint64_t>(min(static_cast<int64_t>(BM), a.rows_cap - arow)) * a.K * 2);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, s_abort)) {
             aborted = true;
@@ -630,8 +618,6 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
   a.gather_src = gather_src;
   a.gather_k = gather_k;
   a.pre = pre;
-  a.a_ptr = gather_src != nullptr ? nullptr : static_cast<const uint8_t*>(A);
-  a.b_ptr = static_cast<const uint8_t*>(B);
   a.err = c.err;
   // upper bound of the tile count: sum_e ceil(n_e / bm) <= rows_cap / bm + E
   const int tbm = pair ? 2 * gg::BM : gg::BM;

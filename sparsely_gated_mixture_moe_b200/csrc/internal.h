@@ -115,9 +115,10 @@ struct RouteProblem {
   float* partials;    // workspace: [route_blocks][2][E]
   float* logits_ws;   // fp32 path only: [T][E] ([T][groups + E] for hierarchical gating)
   float* nz_ws;       // fp32 path only: [T][E]
-  float* lw = nullptr;  // bf16 noisy path with Importance/Load: clean logits [T][E],
-  float* sw = nullptr;  // Softplus(x.W_noise) [T][E] and the k-th / (k+1)-th noisy
-  float* kw = nullptr;  // scores [T][2] of each token
+  float* lw = nullptr;  // bf16 noisy path with Importance/Load: clean logits, Softplus
+  float* sw = nullptr;  // (x.W_noise) and noisy scores H, each [E][T], and the k-th /
+  float* hw = nullptr;  // (k+1)-th noisy scores [2][T] of each token
+  float* kw = nullptr;
 };
 int route_blocks(int64_t T);
 cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c);

@@ -55,7 +55,7 @@ moe_status check_config(const moe_config* c) {
 }
 
 struct Layout {
-  size_t err, blk, partials, logits, nz, lw, sw, kw, steps;      // step workspace
+  size_t err, blk, partials, logits, nz, lw, sw, hw, kw, steps;  // step workspace
   size_t offsets, slot_pos, perm_src, x_perm, h, y_perm, forward;  // + forward intermediates
 };
 
@@ -77,11 +77,13 @@ Layout layout(const moe_config* c) {
     L.nz = o;
     if (c->gating == MOE_GATE_NOISY_TOPK) o = align_up(o + static_cast<size_t>(c->T) * c->E * 4);
   }
-  L.lw = L.sw = L.kw = o;
+  L.lw = L.sw = L.hw = L.kw = o;
   if (c->dtype == MOE_BF16 && c->gating == MOE_GATE_NOISY_TOPK) {
     // the per-token values the Importance/Load sums are formed from
     o = align_up(o + static_cast<size_t>(c->T) * c->E * 4);
     L.sw = o;
+    o = align_up(o + static_cast<size_t>(c->T) * c->E * 4);
+    L.hw = o;
     o = align_up(o + static_cast<size_t>(c->T) * c->E * 4);
     L.kw = o;
     o = align_up(o + static_cast<size_t>(c->T) * 2 * 4);
@@ -250,6 +252,7 @@ moe_status do_route(const moe_config* cfg, const Layout& L, const void* x, const
   if (cfg->dtype == MOE_BF16 && cfg->gating == MOE_GATE_NOISY_TOPK) {
     p.lw = reinterpret_cast<float*>(w + L.lw);
     p.sw = reinterpret_cast<float*>(w + L.sw);
+    p.hw = reinterpret_cast<float*>(w + L.hw);
     p.kw = reinterpret_cast<float*>(w + L.kw);
   }
   cudaError_t e = cfg->dtype == MOE_BF16 ? launch_route_bf16(p, ctx.lc) : launch_route_f32(p, ctx.lc);

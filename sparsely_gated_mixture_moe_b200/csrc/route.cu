@@ -51,11 +51,13 @@ struct GateArgs {
   uint8_t* near_tie;
   float* partials;  // [gridDim.x][2][E] or null
   // noisy gating with Importance/Load asked for, on the tensor-core path: the gate writes
-  // each token's clean logits (bias added) and Softplus(x.W_noise) [T, E] and its k-th and
-  // (k+1)-th noisy scores [T, 2] here instead of forming the sums itself
-  // (importance_load_kernel does, over the whole grid); null otherwise
+  // each token's clean logits (bias added), Softplus(x.W_noise) and noisy scores H, all
+  // [E, T] (expert-major, so a warp's 32 tokens store 128 contiguous bytes), and its k-th
+  // and (k+1)-th H [2, T] here instead of forming the sums itself (importance_load_kernel
+  // does, over the whole grid); null otherwise
   float* lw;
   float* sw;
+  float* hw;
   float* kw;
 };
 
@@ -239,11 +241,13 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
           sv = l[jj] + sbias[e];
           if (noisy) {
             const float sp = softplus_f(z[jj]);
+            const float li = sv;
+            sv = __fmaf_rn(nz[j], sp, sv);  // H
             if (g.lw != nullptr && valid) {
-              g.lw[t * E + e] = sv;
-              g.sw[t * E + e] = sp;
+              g.lw[e * g.T + t] = li;
+              g.sw[e * g.T + t] = sp;
+              g.hw[e * g.T + t] = sv;
             }
-            sv = __fmaf_rn(nz[j], sp, sv);  // H; recomputed bit for bit by the Load sums
           }
         }
         sc[jj] = sv;
@@ -358,8 +362,8 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
     fkth[row * 2 + 0] = kth;
     fkth[row * 2 + 1] = kth1;
     if (g.kw != nullptr && valid) {
-      g.kw[t * 2 + 0] = kth;
-      g.kw[t * 2 + 1] = kth1;
+      g.kw[t] = kth;
+      g.kw[g.T + t] = kth1;
     }
   }
   if (g.partials == nullptr || g.lw != nullptr) {  // uniform across the gate threads
@@ -576,20 +580,8 @@ struct RouteTcArgs {
   int ntiles;     // ceil(T / 128), or ceil(T / 64) with half tiles
   int gate_off;   // byte offset of the gate scratch in shared memory
   int bar_off;    // byte offset of the barriers
-  const uint8_t* x;  // token rows, for L2 prefetches of each tile's contiguous rows
-  int row_bytes;     // bytes of one token row of x
   int* err;
 };
-
-// Prefetches into L2 the contiguous rows of x (and of the noise) of token tile L.
-__device__ __forceinline__ void prefetch_route_tile(const RouteTcArgs& a, int L) {
-  if (L >= a.ntiles) return;
-  const int ntok = a.half ? 64 : 128;
-  const int64_t t0 = static_cast<int64_t>(L) * ntok;
-  const int64_t n = min(static_cast<int64_t>(ntok), a.g.T - t0);
-  l2_prefetch_range(a.x + t0 * a.row_bytes, static_cast<uint64_t>(n) * a.row_bytes);
-  if (a.g.noisy) l2_prefetch_range(a.g.noise + t0 * a.g.E, static_cast<uint64_t>(n) * a.g.E * 4);
-}
 
 __device__ __forceinline__ void gate_bar_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
@@ -657,9 +649,7 @@ __global__ void __launch_bounds__(64 + 128 * G)
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_par = 0;
       bool aborted = false;
-      prefetch_route_tile(a, blockIdx.x);
       for (int L = blockIdx.x; L < a.ntiles && !aborted; L += gridDim.x) {
-        prefetch_route_tile(a, L + gridDim.x);  // the next tile's rows, one tile ahead
         for (int kb = 0; kb < a.kblocks; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, s_abort)) {
             aborted = true;
@@ -862,52 +852,48 @@ __global__ void __launch_bounds__(128, 1)
 }
 
 // Importance and Load partial sums of noisy gating from the gate's per-token values:
-// block (cb, chunk) covers experts 32*cb .. 32*cb+31 (one per lane) and a run of tokens;
-// its 8 warps take every 8th token of the run.  For token t and expert e:
+// block (chunk, eb) covers a run of tokens and experts 8*eb .. 8*eb+7, one per warp; the
+// lanes take the run's tokens 32 at a time.  For token t and expert e:
 //   Importance term: the gate of e if e is one of t's chosen experts, else 0
-//   Load term: P(t, e) = Phi((l_te - kth_excluding(H_t, k, e)) / Softplus(z_te)), with
-//   H_te = l_te + noise_te * Softplus(z_te) and kth_excluding = the (k+1)-th largest
-//   score when H_te >= the k-th largest, else the k-th largest.
-// The 8 warps' sums are added in warp order into partials[chunk][2][E], so the result
-// does not depend on scheduling.
+//   Load term: P(t, e) = Phi((l_te - kth_excluding(H_t, k, e)) / Softplus(z_te)), where
+//   kth_excluding is the (k+1)-th largest score when H_te >= the k-th largest, else the
+//   k-th largest (H_te as the gate formed it, so H >= the k-th means "among the top k").
+// Each warp's lanes are summed in a fixed butterfly order into partials[chunk][2][E], so
+// the result does not depend on scheduling.
 __global__ void __launch_bounds__(256)
     importance_load_kernel(const float* __restrict__ lw, const float* __restrict__ sw,
-                           const float* __restrict__ kw, const float* __restrict__ noise,
+                           const float* __restrict__ hw, const float* __restrict__ kw,
                            const int32_t* __restrict__ topk_idx,
                            const float* __restrict__ topk_gate, int64_t T, int E, int k,
                            int64_t chunk_tokens, int want_load, float* __restrict__ partials) {
-  __shared__ float s_imp[8][32], s_load[8][32];
   grid_dep_wait();
   grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * 32 + lane;
-  const int64_t t_lo = static_cast<int64_t>(blockIdx.y) * chunk_tokens;
+  const int e = blockIdx.y * 8 + warp;
+  if (e >= E) return;
+  const int64_t t_lo = static_cast<int64_t>(blockIdx.x) * chunk_tokens;
   const int64_t t_hi = min(T, t_lo + chunk_tokens);
   float si = 0.0f, sl = 0.0f;
-  for (int64_t t = t_lo + warp; t < t_hi; t += 8) {
+  for (int64_t t = t_lo + lane; t < t_hi; t += 32) {
     float gi = 0.0f;
     for (int j = 0; j < k; ++j)
       if (__ldg(topk_idx + t * k + j) == e) gi = __ldg(topk_gate + t * k + j);
     si += gi;
-    if (want_load && e < E) {
-      const float li = __ldg(lw + t * E + e), sp = __ldg(sw + t * E + e);
-      const float H = __fmaf_rn(__ldg(noise + t * E + e), sp, li);  // as the gate formed it
-      const float kth = __ldg(kw + t * 2), kth1 = __ldg(kw + t * 2 + 1);
-      const float ex = (H >= kth) ? kth1 : kth;
+    if (want_load) {
+      const int64_t i = static_cast<int64_t>(e) * T + t;
+      const float li = __ldg(lw + i), sp = __ldg(sw + i), H = __ldg(hw + i);
+      const float ex = (H >= __ldg(kw + t)) ? __ldg(kw + T + t) : __ldg(kw + t);
       sl += 0.5f + 0.5f * erf_as7126(__fdividef(li - ex, sp) * 0.70710678118654752f);
     }
   }
-  s_imp[warp][lane] = si;
-  s_load[warp][lane] = sl;
-  __syncthreads();
-  if (warp == 0 && e < E) {
-    float a = 0.0f, b = 0.0f;
-    for (int w = 0; w < 8; ++w) {
-      a += s_imp[w][lane];
-      b += s_load[w][lane];
-    }
-    partials[(blockIdx.y * 2 + 0) * static_cast<int64_t>(E) + e] = a;
-    partials[(blockIdx.y * 2 + 1) * static_cast<int64_t>(E) + e] = b;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    si += __shfl_xor_sync(0xffffffffu, si, o);
+    sl += __shfl_xor_sync(0xffffffffu, sl, o);
+  }
+  if (lane == 0) {
+    partials[(blockIdx.x * 2 + 0) * static_cast<int64_t>(E) + e] = si;
+    partials[(blockIdx.x * 2 + 1) * static_cast<int64_t>(E) + e] = sl;
   }
 }
 
@@ -943,7 +929,7 @@ static GateArgs gate_args(const RouteProblem& p) {
   g.topk_gate = p.topk_gate;
   g.near_tie = p.near_tie;
   g.partials = (p.importance || p.load) ? p.partials : nullptr;
-  g.lw = g.sw = g.kw = nullptr;
+  g.lw = g.sw = g.hw = g.kw = nullptr;
   return g;
 }
 
@@ -982,18 +968,21 @@ static cudaError_t launch_route_tc_hier(int kg, const CUtensorMap& tmX, const CU
 // router kernel, the sums over the whole grid (importance_load_kernel), then the fixed-
 // order total over the chunks.
 static cudaError_t launch_importance_load(const RouteProblem& p, const LaunchCtx& c) {
-  const int cb = (p.E + 31) / 32;
-  // about four blocks per SM, at most one chunk per 64 tokens (the partials' rows)
-  int64_t chunks = (4LL * c.num_sms + cb - 1) / cb;
+  const int eb = (p.E + 7) / 8;
+  // about four blocks per SM; chunks of whole 32-token groups, at most one chunk per 64
+  // tokens (the partials' rows)
+  int64_t chunks = (4LL * c.num_sms + eb - 1) / eb;
   const int64_t cap = route_blocks(p.T);
   if (chunks > cap) chunks = cap;
   if (chunks < 1) chunks = 1;
-  const int64_t per = (p.T + chunks - 1) / chunks;
+  int64_t per = (p.T + chunks - 1) / chunks;
+  per = (per + 31) / 32 * 32;
   chunks = (p.T + per - 1) / per;
-  cudaError_t e = launch_kernel(importance_load_kernel, dim3(cb, static_cast<unsigned>(chunks)),
+  cudaError_t e = launch_kernel(importance_load_kernel, dim3(static_cast<unsigned>(chunks), eb),
                                 dim3(256), 0, c, static_cast<const float*>(p.lw),
-                                static_cast<const float*>(p.sw), static_cast<const float*>(p.kw),
-                                p.noise, static_cast<const int32_t*>(p.topk_idx),
+                                static_cast<const float*>(p.sw), static_cast<const float*>(p.hw),
+                                static_cast<const float*>(p.kw),
+                                static_cast<const int32_t*>(p.topk_idx),
                                 static_cast<const float*>(p.topk_gate), p.T, p.E, p.k, per,
                                 p.load != nullptr ? 1 : 0, p.partials);
   if (e != cudaSuccess) return e;
@@ -1009,6 +998,7 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   if (split) {
     a.g.lw = p.lw;
     a.g.sw = p.sw;
+    a.g.hw = p.hw;
     a.g.kw = p.kw;
   }
   const int n_scores = p.hier ? p.E + p.groups : p.E;  // score columns (rows of w_gate)
@@ -1034,8 +1024,6 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   a.stages = stages;
   a.gate_off = stages * stage_bytes;
   a.bar_off = a.gate_off + (scratch + 127) / 128 * 128;
-  a.x = static_cast<const uint8_t*>(p.x);
-  a.row_bytes = p.d * 2;
   a.err = c.err;
   const int smem = 1024 + a.bar_off + 8 * (2 * stages + 5) + 16;
 

@@ -4,8 +4,8 @@ moe_forward_train + moe_backward on seeded bf16 workloads against oracle/moe_bac
 (whose gradients are pinned to central finite differences of the forward oracle's loss).
 The reference recomputes the forward itself, so each case is chosen without near ties
 (every token's k-th vs (k+1)-th score gap above 1e-4, checked here): both sides then route
-every token alike.  Each gradient must be within max|err| / RMS <= 2e-2 of the reference,
-the layer-output tolerance of the bf16 path: the expert products take bf16 operands (the
+every token alike.  Each gradient must be within max|err| / RMS <= 2e-2 of the reference
+(the weight gradients expert by expert), the layer-output tolerance of the bf16 path: the expert products take bf16 operands (the
 upstream gradient of each expert row and the hidden activations are rounded to 16 bits)
 with fp32 accumulation; the router's gradients are fp32."""
 import numpy as np
@@ -105,7 +105,14 @@ def test_backward_matches_reference_gradients(name):
     if "logit_bias" in inp:
         pairs.append(("dbias", "dlogit_bias"))
     for got_key, ref_key in pairs:
-        e = H.rel_err(g[got_key].double().numpy(), ref[ref_key])
+        got, want = g[got_key].double().numpy(), ref[ref_key]
+        if got_key in ("dw1", "dw2"):
+            # each expert's weight gradient is its own parameter block: measured against
+            # its own RMS (with Zipf-skewed expert sizes one global RMS is set by the many
+            # small blocks and would stretch the hot expert's rounding error)
+            e = max(H.rel_err(got[i], want[i]) for i in range(w.E) if np.any(want[i] != 0))
+        else:
+            e = H.rel_err(got, want)
         rep[got_key] = e
         assert e <= TOL, (got_key, e)
     # the auxiliary loss values
