@@ -12,8 +12,11 @@ layer forward has no exchange step on one device), the step time is the max over
 and the value is the tokens of all ranks per second.
 
 Timing: W untimed warm-up steps; then K steps, each preceded (outside its events) by a
-write and read-back of a 256 MB buffer that flushes the 126 MB L2; CUDA events on the
-launching stream bracket each step and each step call.  The dominant kernel is the
+write and read-back of a 256 MB buffer that flushes the 126 MB L2 and by a ~0.2 ms
+GPU-side wait, during which the host queues the whole step, so that the step's kernels
+run back to back as they do in a CUDA-graph replay (the Python binding's launch latency
+is not part of the step); CUDA events on the launching stream bracket each step and each
+step call.  The dominant kernel is the
 tcgen05 grouped GEMM (two launches per step: up- and down-projection); its roofline uses
 the algorithmic bytes/FLOPs of those two launches over the event time of the expert-FFN
 call, and its DRAM traffic per launch comes from the committed ncu summary while the
@@ -356,6 +359,11 @@ class LayerBench:
         self.launches += n
 
 
+# GPU clock cycles of the wait queued before each timed step (~0.2 ms): longer than the
+# host needs to queue one step's calls
+HOST_AHEAD_CYCLES = 400_000
+
+
 class L2Flusher:
     def __init__(self, dev):
         self.buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -366,6 +374,9 @@ class L2Flusher:
         # charged to the first kernel of the step
         self.buf.fill_(float(i))
         self.buf.sum()
+        # then keep the GPU busy while the host queues the step, so that no host launch
+        # latency falls between the step's kernels
+        torch.cuda._sleep(HOST_AHEAD_CYCLES)
 
 
 def timed_steps(lb, flush, steps, warmup, world, dev, clock_gpu):

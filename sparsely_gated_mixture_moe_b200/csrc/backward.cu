@@ -317,12 +317,14 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_ld32(tbase + c, v);
           tmem_ld_wait();
           if (m >= a.M) continue;
-          float4* dst = reinterpret_cast<float4*>(dst_row + c);
+          if (!any) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            dst[j] = any ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                       __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < 32; ++j) v[j] = 0u;
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            st_global_v8(dst_row + c + 8 * j, v[8 * j], v[8 * j + 1], v[8 * j + 2], v[8 * j + 3],
+                         v[8 * j + 4], v[8 * j + 5], v[8 * j + 6], v[8 * j + 7]);
         }
       } else {
         const int p0 = __ldg(a.poff + t.e), p1 = __ldg(a.poff + t.e + 1);
@@ -357,18 +359,17 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
               for (int j = 0; j < 16; ++j) pk[j] = 0u;  // padding rows of du are zero
             }
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) +
-                                                  (p0 + static_cast<int64_t>(i)) * a.N + col0 + c);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            uint16_t* dst = static_cast<uint16_t*>(a.out) + (p0 + static_cast<int64_t>(i)) * a.N +
+                            col0 + c;
+            st_global_v8(dst, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+            st_global_v8(dst + 16, pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14], pk[15]);
           } else {  // DGRAD_UP: dx_perm at the unpadded row
             if (!kept) continue;
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + s * a.N + col0 + c);
+            float* dst = static_cast<float*>(a.out) + s * a.N + col0 + c;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                   __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+            for (int j = 0; j < 4; ++j)
+              st_global_v8(dst + 8 * j, v[8 * j], v[8 * j + 1], v[8 * j + 2], v[8 * j + 3],
+                           v[8 * j + 4], v[8 * j + 5], v[8 * j + 6], v[8 * j + 7]);
           }
         }
       }

@@ -338,6 +338,16 @@ __device__ __forceinline__ void tc_mma_pair_f16kind(uint32_t d_tmem, uint64_t ad
 
 // --------------------------------------------------------------------- utilities
 
+// One 32-byte store of 8 words (the address 32-byte aligned): a whole L2 sector per
+// thread, where two 16-byte stores would each write half of one.
+__device__ __forceinline__ void st_global_v8(void* p, uint32_t a0, uint32_t a1, uint32_t a2,
+                                             uint32_t a3, uint32_t a4, uint32_t a5, uint32_t a6,
+                                             uint32_t a7) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a0),
+               "r"(a1), "r"(a2), "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);

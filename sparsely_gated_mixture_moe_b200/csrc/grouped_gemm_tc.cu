@@ -131,15 +131,15 @@ __device__ __forceinline__ void epilogue_rows(const Args& a, uint32_t tbase, int
     tmem_ld_wait();
     if (!row_ok) continue;
     if (MODE == OUT_F32 || MODE == OUT_COMBINE) {
-      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + oidx + c);
+      float* dst = static_cast<float*>(a.out) + oidx + c;  // 128-byte aligned
       if (MODE == OUT_COMBINE) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(scale * __uint_as_float(v[j]));
       }
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                             __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+      for (int j = 0; j < 4; ++j)
+        st_global_v8(dst + 8 * j, v[8 * j], v[8 * j + 1], v[8 * j + 2], v[8 * j + 3], v[8 * j + 4],
+                     v[8 * j + 5], v[8 * j + 6], v[8 * j + 7]);
     } else {
       uint32_t pk[16];
       if (a.pre != nullptr) {  // the pre-activation, for the backward pass
@@ -148,10 +148,9 @@ __device__ __forceinline__ void epilogue_rows(const Args& a, uint32_t tbase, int
           const float z0 = __uint_as_float(v[2 * j]), z1 = __uint_as_float(v[2 * j + 1]);
           pk[j] = MODE == OUT_F16 ? pack_f16x2(z0, z1) : pack_bf16x2(z0, z1);
         }
-        uint4* pdst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.pre) + oidx + c);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          pdst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        uint16_t* pdst = static_cast<uint16_t*>(a.pre) + oidx + c;  // 64-byte aligned
+        st_global_v8(pdst, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+        st_global_v8(pdst + 16, pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14], pk[15]);
       }
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
@@ -159,10 +158,9 @@ __device__ __forceinline__ void epilogue_rows(const Args& a, uint32_t tbase, int
         const float x1 = epi_act<ACT>(__uint_as_float(v[2 * j + 1]));
         pk[j] = MODE == OUT_F16 ? pack_f16x2(x0, x1) : pack_bf16x2(x0, x1);
       }
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + oidx + c);
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+      uint16_t* dst = static_cast<uint16_t*>(a.out) + oidx + c;  // 64-byte aligned
+      st_global_v8(dst, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+      st_global_v8(dst + 16, pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14], pk[15]);
     }
   }
 }

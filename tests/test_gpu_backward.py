@@ -4,8 +4,10 @@ moe_forward_train + moe_backward on seeded bf16 workloads against oracle/moe_bac
 (whose gradients are pinned to central finite differences of the forward oracle's loss).
 The reference recomputes the forward itself, so each case is chosen without near ties
 (every token's k-th vs (k+1)-th score gap above 1e-4, checked here): both sides then route
-every token alike.  Each gradient must be within max|err| / RMS <= 2e-2 of the reference
-(the weight gradients expert by expert), the layer-output tolerance of the bf16 path: the expert products take bf16 operands (the
+every token alike.  dx, the router's and the gates' gradients must be within
+max|err| / RMS <= 2e-2 of the reference, the layer-output tolerance of the bf16 path; the
+expert weight gradients, expert by expert, within 4e-2 (see TOL_WEIGHT) and within 1e-2
+of the same arithmetic with the backward's 16-bit roundings applied explicitly: the expert products take bf16 operands (the
 upstream gradient of each expert row and the hidden activations are rounded to 16 bits)
 with fp32 accumulation; the router's gradients are fp32."""
 import numpy as np
@@ -22,6 +24,18 @@ from workloads import Workload
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-2
+# Expert weight gradients, per expert, against the fp64 reference.  Their operands are
+# rounded to 16 bits three times on the way (the pre-activation u, the expert rows'
+# upstream gradient d_o, and du = dh * act'(u)), each by up to 2^-9 relative; a weight
+# gradient entry sums those products over the expert's rows, and for an expert with few
+# rows (the Zipf case has experts of 8 and 14 rows) its max-to-RMS ratio stretches that
+# to 2.6e-2 (dW1) and 2.9e-2 (dW2) in the bit-exact simulation of those roundings.  The
+# GPU result is also checked against that simulation (bf16_expert_grads below), which it
+# matches up to accumulation order: fp32 sums on the GPU against fp64 in the simulation
+# move an intermediate across a rounding boundary now and then, and one such 16-bit ulp
+# (2^-8 relative) in one product of an expert with few rows is ~4e-3 of the entry's RMS.
+TOL_WEIGHT = 4e-2
+TOL_ROUNDING_SIM = 1e-2
 
 CASES = {
     # (workload, w_importance, w_load)
@@ -38,6 +52,46 @@ CASES = {
     "k4_E32_capacity": (Workload("bk", T=800, d_model=64, d_ff=128, E=32, k=4, act="gelu",
                                  capacity_factor=0.8, seed=1), 0.2, 0.0),
 }
+
+
+def _round16(a, f16):
+    t = torch.from_numpy(np.asarray(a, np.float64)).float()
+    return t.to(torch.float16 if f16 else torch.bfloat16).double().numpy()
+
+
+def bf16_expert_grads(w, inp, dy, idx, gates):
+    """dW1, dW2 from the oracle's routing and dispatch with the backward's 16-bit rounding
+    points applied explicitly: u (the stored pre-activation) and d_o = G dy rounded to
+    h's type (fp16 with hidden_f16, else bf16), du = (d_o . W2_e) * act'(u) rounded to
+    bf16, h = act(u) rounded to its stored type; products summed in fp64."""
+    import math
+    from scipy.special import erf
+    C = orc.capacity(w.capacity_factor, w.T, w.k, w.E)
+    _, off, perm_src, _ = orc.dispatch(idx, w.E, C)
+    x = inp["x"].double().numpy()
+    W1, W2 = inp["w1"].double().numpy(), inp["w2"].double().numpy()
+    if w.hidden_f16:
+        W2 = _round16(W2, True)
+    xp = x[perm_src // w.k]
+    g = gates.reshape(-1)[perm_src]
+    t = perm_src // w.k
+    dW1, dW2 = np.zeros_like(W1), np.zeros_like(W2)
+    for e in range(w.E):
+        a, b = int(off[e]), int(off[e + 1])
+        if b <= a:
+            continue
+        u = xp[a:b] @ W1[e].T
+        h = _round16(orc.ACTS[w.act](u), w.hidden_f16)
+        ub = _round16(u, w.hidden_f16)
+        d_o = _round16(g[a:b, None] * dy[t[a:b]], w.hidden_f16)
+        if w.act == "relu":
+            ag = (ub > 0).astype(np.float64)
+        else:
+            ag = 0.5 * (1 + erf(ub / math.sqrt(2))) + ub * np.exp(-0.5 * ub * ub) / math.sqrt(2 * math.pi)
+        du = _round16((d_o @ W2[e]) * ag, False)
+        dW2[e] = d_o.T @ h
+        dW1[e] = du.T @ xp[a:b]
+    return dW1, dW2
 
 
 def _dy(w):
@@ -104,17 +158,23 @@ def test_backward_matches_reference_gradients(name):
         pairs.append(("dw_noise", "dw_noise"))
     if "logit_bias" in inp:
         pairs.append(("dbias", "dlogit_bias"))
+    sim = dict(zip(("dw1", "dw2"), bf16_expert_grads(w, inp, dy.double().numpy(), r["idx"],
+                                                     r["gates"])))
     for got_key, ref_key in pairs:
         got, want = g[got_key].double().numpy(), ref[ref_key]
         if got_key in ("dw1", "dw2"):
-            # each expert's weight gradient is its own parameter block: measured against
-            # its own RMS (with Zipf-skewed expert sizes one global RMS is set by the many
-            # small blocks and would stretch the hot expert's rounding error)
-            e = max(H.rel_err(got[i], want[i]) for i in range(w.E) if np.any(want[i] != 0))
+            # each expert's weight gradient is its own parameter block, measured against its
+            # own RMS (one global RMS is set by the many small blocks of Zipf-skewed experts)
+            experts = [i for i in range(w.E) if np.any(want[i] != 0)]
+            e = max(H.rel_err(got[i], want[i]) for i in experts)
+            es = max(H.rel_err(got[i], sim[got_key][i]) for i in experts)
+            rep[got_key + "_vs_rounding_sim"] = es
+            assert es <= TOL_ROUNDING_SIM, (got_key, "rounding simulation", es)
+            assert e <= TOL_WEIGHT, (got_key, e)
         else:
             e = H.rel_err(got, want)
+            assert e <= TOL, (got_key, e)
         rep[got_key] = e
-        assert e <= TOL, (got_key, e)
     # the auxiliary loss values
     if w_imp:
         imp = orc.importance(orc.dense_gates(w.T, w.E, r["idx"], r["gates"]))
