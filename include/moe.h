@@ -381,6 +381,15 @@ moe_status moe_wait_timeout_check(void* ws, moe_stream_t stream);
 moe_status moe_erf_check(const float* x, float* fast, float* ref, int64_t n,
                          moe_stream_t stream);
 
+/* Self-check of the GELU epilogue of the up-projection: writes the epilogue's paired
+ * evaluation of GELU(z) = z Phi(z) (erf by Abramowitz & Stegun 7.1.26 on f32x2 pairs
+ * (z[2i], z[2i+1]); an odd last value is paired with itself) into fast[] and
+ * 0.5 z (1 + erff(z / sqrt 2)) into ref[], so a test can bound their difference.  All
+ * pointers device, n >= 0 values; MOE_ERR_INVALID_ARG for n < 0 or a null pointer
+ * with n > 0. */
+moe_status moe_gelu_check(const float* z, float* fast, float* ref, int64_t n,
+                          moe_stream_t stream);
+
 /* Number of kernels the most recent successful call on this host thread queued. */
 int32_t moe_last_launch_count(void);
 

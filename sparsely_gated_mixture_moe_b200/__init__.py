@@ -47,6 +47,7 @@ def _load():
         "moe_bf16_to_f16": (ctypes.c_int, [P, P, ctypes.c_int64, P, P]),
         "moe_permute_noalloc": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
         "moe_erf_check": (ctypes.c_int, [P, P, P, ctypes.c_int64, P]),
+        "moe_gelu_check": (ctypes.c_int, [P, P, P, ctypes.c_int64, P]),
         "moe_train_state_size": (ctypes.c_size_t, [C]),
         "moe_backward_workspace_size": (ctypes.c_size_t, [C]),
         "moe_forward_train": (ctypes.c_int, [C] + [P] * 17),

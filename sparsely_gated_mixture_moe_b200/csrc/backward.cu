@@ -128,11 +128,11 @@ __device__ __forceinline__ int bwd_kblocks(const Args& a, int e) {
   return a.K / BK;
 }
 
+// the derivative of the activation for ReLU (1) and identity (0); GELU pairs take
+// gelu_grad2_as7126
 __device__ __forceinline__ float act_grad(float u, int act) {
   if (act == 1) return u > 0.0f ? 1.0f : 0.0f;
-  // GELU'(u) = Phi(u) + u phi(u)
-  const float Phi = 0.5f * (1.0f + erf_as7126(u * 0.70710678118654752f));
-  return Phi + u * 0.3989422804014327f * __expf(-0.5f * u * u);
+  return 1.0f;
 }
 
 __device__ __forceinline__ float u16_to_float(uint16_t v, int f16) {
@@ -352,8 +352,14 @@ __global__ void __launch_bounds__(THREADS, 1)
               for (int j = 0; j < 16; ++j) {
                 const float u0 = u16_to_float(static_cast<uint16_t>(uw[j] & 0xFFFFu), a.u_f16);
                 const float u1 = u16_to_float(static_cast<uint16_t>(uw[j] >> 16), a.u_f16);
-                pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * act_grad(u0, a.act),
-                                    __uint_as_float(v[2 * j + 1]) * act_grad(u1, a.act));
+                float g0, g1;
+                if (a.act == 2) {
+                  gelu_grad2_as7126(u0, u1, g0, g1);
+                } else {
+                  g0 = act_grad(u0, a.act);
+                  g1 = act_grad(u1, a.act);
+                }
+                pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * g0, __uint_as_float(v[2 * j + 1]) * g1);
               }
             } else {
 #pragma unroll

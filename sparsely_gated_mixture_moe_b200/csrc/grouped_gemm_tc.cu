@@ -17,12 +17,14 @@
 //   warp 1      TMEM owner and MMA issuer: one thread issues tcgen05.mma (M=128, N=BN,
 //               K=16) into one of two TMEM accumulators (2 x 256 fp32 columns), and
 //               tcgen05.commit releases smem stages and hands finished accumulators on.
-//   warps 2-13  epilogue: tcgen05.ld of the accumulator (each warp reads its 32-lane
-//               quarter and every third 32-column chunk), activation, rounding to
+//   warps 2-17  epilogue: tcgen05.ld of the accumulator (each warp reads its 32-lane
+//               quarter and every fourth 32-column chunk), activation, rounding to
 //               bf16/fp16 (or fp32 as is), stores of the rows that belong to the expert
-//               (a ragged tail is masked).  Three warps per lane quarter keep a ragged
-//               tile, whose rows all sit in the first quarters, from serialising on few
-//               warps.
+//               (a ragged tail is masked).  Four warps per lane quarter split a 256-column
+//               accumulator evenly (two chunks each) and keep a ragged tile, whose rows
+//               all sit in the first quarters, from serialising on few warps; the GELU
+//               epilogue of the up-projection is latency-bound, and four warps per SM
+//               sub-partition measured 1.2% faster on the whole expert FFN than three.
 // Tiles are (expert, m-tile, n-tile) with n innermost: CTAs running at the same time share
 // the A rows of an m-tile through L2 while each streams a different weight tile (measured
 // 1.5-3.5% faster than m innermost on the five workloads).
@@ -44,7 +46,7 @@ namespace gg {
 constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int STAGES = 4;
-constexpr int EPI_WARPS = 12;  // 3 per TMEM lane quarter (more would cap registers below need)
+constexpr int EPI_WARPS = 16;  // 4 per TMEM lane quarter (96 registers a thread, no spills)
 constexpr int EPI_SUBS = EPI_WARPS / 4;
 constexpr int THREADS = 64 + EPI_WARPS * 32;
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
@@ -154,8 +156,13 @@ __device__ __forceinline__ void epilogue_rows(const Args& a, uint32_t tbase, int
       }
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const float x0 = epi_act<ACT>(__uint_as_float(v[2 * j]));
-        const float x1 = epi_act<ACT>(__uint_as_float(v[2 * j + 1]));
+        float x0, x1;
+        if (ACT == 2) {
+          gelu2_as7126(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1]), x0, x1);
+        } else {
+          x0 = epi_act<ACT>(__uint_as_float(v[2 * j]));
+          x1 = epi_act<ACT>(__uint_as_float(v[2 * j + 1]));
+        }
         pk[j] = MODE == OUT_F16 ? pack_f16x2(x0, x1) : pack_bf16x2(x0, x1);
       }
       uint16_t* dst = static_cast<uint16_t*>(a.out) + oidx + c;  // 64-byte aligned
@@ -419,7 +426,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;               // TMEM lane quarter this warp may read
-    const int sub = (warp - 2) >> 2;      // which 32-column chunks: sub*32 + 96*i
+    const int sub = (warp - 2) >> 2;      // which 32-column chunks: sub*32 + 128*i
     const int mode = a.out_mode * 3 + a.act;
     if (a.out_mode == OUT_COMBINE) {
       // y = 0 for tokens whose only assignment was dropped (no tile writes them); done
@@ -681,6 +688,25 @@ __global__ void erf_check_kernel(const float* __restrict__ x, float* __restrict_
     ref[i] = erff(x[i]);
   }
 }
+
+// the GELU epilogue's paired evaluation on (z[2i], z[2i+1]); an odd last value is paired
+// with itself
+__global__ void gelu_check_kernel(const float* __restrict__ z, float* __restrict__ fast,
+                                  float* __restrict__ ref, int64_t n) {
+  const int64_t pairs = (n + 1) / 2;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < pairs;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t j0 = 2 * i, j1 = 2 * i + 1 < n ? 2 * i + 1 : 2 * i;
+    float g0, g1;
+    gelu2_as7126(z[j0], z[j1], g0, g1);
+    fast[j0] = g0;
+    ref[j0] = gelu_exact(z[j0]);
+    if (j1 != j0) {
+      fast[j1] = g1;
+      ref[j1] = gelu_exact(z[j1]);
+    }
+  }
+}
 }  // namespace moe
 
 extern "C" moe_status moe_erf_check(const float* x, float* fast, float* ref, int64_t n,
@@ -691,6 +717,18 @@ extern "C" moe_status moe_erf_check(const float* x, float* fast, float* ref, int
   if (blocks > 4096) blocks = 4096;
   moe::erf_check_kernel<<<static_cast<unsigned>(blocks), 256, 0,
                           reinterpret_cast<cudaStream_t>(stream)>>>(x, fast, ref, n);
+  moe::set_last_launch_count(1);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" moe_status moe_gelu_check(const float* z, float* fast, float* ref, int64_t n,
+                                     moe_stream_t stream) {
+  if (n < 0 || (n > 0 && (!z || !fast || !ref))) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  int64_t blocks = ((n + 1) / 2 + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  moe::gelu_check_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                           reinterpret_cast<cudaStream_t>(stream)>>>(z, fast, ref, n);
   moe::set_last_launch_count(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

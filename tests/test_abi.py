@@ -22,6 +22,15 @@ def _declared_functions():
     return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", src)))
 
 
+def test_self_checks_validate_before_launching():
+    """The erf and GELU self-check entry points refuse a negative count or a null
+    pointer, and do nothing for n = 0 (no launch, so no GPU is needed here)."""
+    for fn in (moe.lib.moe_erf_check, moe.lib.moe_gelu_check):
+        assert fn(None, None, None, -1, None) == 1
+        assert fn(None, None, None, 4, None) == 1
+        assert fn(None, None, None, 0, None) == 0
+
+
 def test_library_exports_every_declared_symbol():
     names = _declared_functions()
     assert len(names) >= 11

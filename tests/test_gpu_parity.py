@@ -268,6 +268,26 @@ def test_fast_erf_matches_cuda_erff():
     assert fast[-4].item() == 1.0 and fast[-3].item() == -1.0
 
 
+def test_packed_gelu_matches_exact_gelu():
+    """The up-projection's GELU epilogue (A&S 7.1.26 erf evaluated on f32x2 pairs) stays
+    within 2e-7 |z| + 1e-6 of 0.5 z (1 + erff(z / sqrt 2)): the formula's 1.5e-7 on erf,
+    scaled by z / 2, plus a few fp32 roundings.  Its results are rounded to 16 bits
+    (half-ulp >= 2.4e-4 relative) before anything else reads them."""
+    import ctypes
+    import sparsely_gated_mixture_moe_b200 as moe
+    z = torch.cat([torch.linspace(-12, 12, 2_000_001), torch.tensor(
+        [0.0, -0.0, 1e-30, -1e-30, 3.0e4, -3.0e4, 1e-3])]).cuda()  # odd count: last pairs with itself
+    fast, ref = torch.empty_like(z), torch.empty_like(z)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    assert moe.lib.moe_gelu_check(p(z), p(fast), p(ref), z.numel(), None) == 0
+    torch.cuda.synchronize()
+    bound = 2e-7 * z.abs() + 1e-6
+    d = (fast - ref).abs()
+    assert bool((d <= bound).all()), float((d - bound).max())
+    assert fast[-3].item() == 3.0e4 and fast[-2].item() == 0.0
+    assert moe.lib.moe_gelu_check(p(z), p(fast), p(ref), -1, None) != 0
+
+
 @pytest.mark.parametrize("name,launches", [("switch", 1), ("three_kernel_permute_T200k", 3)])
 def test_permute_launch_path(name, launches):
     """moe_permute runs as one launch (grid barriers between its phases) when every block
