@@ -277,7 +277,10 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_gate,
 
 /* Bytes of the forward state moe_forward_train writes and moe_backward reads (the kept
  * rows, permutation, expert pre-activations, hidden activations and expert outputs of
- * one batch); 0 for an unsupported cfg.  The layout is internal to the library. */
+ * one batch, and the router's scores as the gate computed them: clean logits, and for
+ * noisy gating Softplus(x.W_noise), the noisy scores and each token's k-th and (k+1)-th
+ * of them, so that the backward differentiates exactly the forward's choice); 0 for an
+ * unsupported cfg.  The layout is internal to the library. */
 size_t moe_train_state_size(const moe_config* cfg);
 
 /* Bytes of workspace moe_backward needs (the step workspace, whose device error word it
@@ -309,7 +312,8 @@ moe_status moe_forward_train(const moe_config* cfg, const void* x, const void* w
  *  ws          moe_backward_workspace_size bytes
  * The expert products run on the tensor cores in bf16 with fp32 accumulation (the
  * upstream gradient of each expert row is rounded to bf16, or fp16 with hidden_f16);
- * the router's gradients are fp32. */
+ * the router's gradients are fp32, from the scores kept in `state` (the router is not
+ * recomputed), with every sum over tokens taken in a fixed order. */
 moe_status moe_backward(const moe_config* cfg, const void* x, const void* w_gate,
                         const void* w_noise, const float* noise, const float* logit_bias,
                         const void* w1, const void* w2, const int32_t* topk_idx,

@@ -517,257 +517,315 @@ __global__ void cv2_grad_kernel(const float* __restrict__ v, int n, float w, flo
 }
 
 // Softplus(z) as the router computes it, and its derivative sigmoid(z).
-__device__ __forceinline__ float bwd_softplus(float z) {
-  return fmaxf(z, 0.0f) + log1pf(__expf(-fabsf(z)));
-}
-__device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + __expf(-z)); }
-
-// Gate backward, one thread per token, over the E score columns of its row.
+// Gate backward, one thread per token over its E score columns.  Every [E, T] array is
+// read and written at e * T + t, so a warp's 32 tokens touch 128 contiguous bytes.
 //   dgate [T, k]: gradient of L with respect to each chosen gate (from combine_bwd)
 //   dimp [E] (or null): the Importance loss gradient, added to every chosen gate's
-//   logits [T, E]: the clean logits x.W_g (+ bias); zlog [T, E]: x.W_noise (noisy)
-//   dload [E] (or null): the Load loss gradient
-// Writes dl [T, E] (gradient of the clean logits) and, for noisy gating, dz [T, E]
-// (gradient of x.W_noise).  The gates of the forward pass are topk_gate (the chosen
-// experts' Softmax(KeepTopK) values, or for the Switch gate the full-softmax values).
+//   lg [E, T]: the forward's clean logits x.W_g (+ bias)
+//   noisy gating: sw [E, T] Softplus(x.W_noise) and hw [E, T] the noisy scores H, both as
+//   the forward computed them, the noise [T, E], and dload [E] (or null): the Load loss
+//   gradient
+// Writes dl [E, T] (gradient of the clean logits) and, for noisy gating, dz [E, T]
+// (gradient of x.W_noise).  topk_gate holds the forward's gates: the chosen experts'
+// Softmax(KeepTopK) values, or for the Switch gate their full-softmax values.
 __global__ void __launch_bounds__(128)
     gate_bwd_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_gate,
                     const float* __restrict__ dgate, const float* __restrict__ dimp,
-                    const float* __restrict__ logits, const float* __restrict__ zlog,
-                    const float* __restrict__ noise, const float* __restrict__ dload,
-                    float* __restrict__ dl, float* __restrict__ dz, int64_t T, int E, int k,
-                    int noisy, int renorm) {
+                    const float* __restrict__ lg, const float* __restrict__ sw,
+                    const float* __restrict__ hw, const float* __restrict__ noise,
+                    const float* __restrict__ dload, float* __restrict__ dl, float* __restrict__ dz,
+                    int64_t T, int E, int k, int noisy, int renorm) {
   const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   grid_dep_wait();
   grid_dep_launch();
   if (t >= T) return;
-  const float* lrow = logits + t * E;
-  float* dlr = dl + t * E;
-  float* dzr = noisy ? dz + t * E : nullptr;
-  for (int e = 0; e < E; ++e) dlr[e] = 0.0f;
-  // chosen gates and their gradients
+  // the chosen experts (k <= 8), their gates G_j and gradients dg_j; S = sum_j G_j dg_j
+  int ci[8];
+  float cg[8], cd[8];
   float S = 0.0f;
-  for (int j = 0; j < k; ++j) {
-    const int e = topk_idx[t * k + j];
-    const float dg = dgate[t * k + j] + (dimp ? dimp[e] : 0.0f);
-    S += topk_gate[t * k + j] * dg;
-  }
-  const bool full = !noisy && !renorm;
-  if (full) {
-    // Switch gate: p = softmax over all logits; d score_e = p_e (dp_e - S), dp nonzero
-    // only at the chosen experts
-    float m = -INFINITY;
-    for (int e = 0; e < E; ++e) m = fmaxf(m, lrow[e]);
-    float z = 0.0f;
-    for (int e = 0; e < E; ++e) z += expf(lrow[e] - m);
-    for (int e = 0; e < E; ++e) dlr[e] = -(expf(lrow[e] - m) / z) * S;
-    for (int j = 0; j < k; ++j) {
-      const int e = topk_idx[t * k + j];
-      const float dg = dgate[t * k + j] + (dimp ? dimp[e] : 0.0f);
-      dlr[e] += topk_gate[t * k + j] * dg;
-    }
-  } else {
-    // Softmax(KeepTopK): d score_i = G_i (dg_i - S) at the chosen experts
-    for (int j = 0; j < k; ++j) {
-      const int e = topk_idx[t * k + j];
-      const float dg = dgate[t * k + j] + (dimp ? dimp[e] : 0.0f);
-      dlr[e] = topk_gate[t * k + j] * (dg - S);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    ci[j] = -1;
+    cg[j] = cd[j] = 0.0f;
+    if (j < k) {
+      ci[j] = topk_idx[t * k + j];
+      cg[j] = topk_gate[t * k + j];
+      cd[j] = dgate[t * k + j] + (dimp ? dimp[ci[j]] : 0.0f);
+      S += cg[j] * cd[j];
     }
   }
-  if (!noisy) return;
-  // noisy gating: the scores are H = l + n * Softplus(z); dlr holds dH so far
-  const float* zrow = zlog + t * E;
+  // Softmax(KeepTopK): d score_e = G_e (dg_e - S) at the chosen experts, 0 elsewhere
+  auto keep_part = [&](int e) {
+    float v = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (ci[j] == e) v = cg[j] * (cd[j] - S);
+    return v;
+  };
+  if (!noisy) {
+    if (renorm) {
+      for (int e = 0; e < E; ++e) dl[e * T + t] = keep_part(e);
+    } else {
+      // Switch gate: p = softmax over all logits; d score_e = p_e (dp_e - S) with dp
+      // nonzero only at the chosen experts, where p_e = G_e
+      float m = -INFINITY;
+      for (int e = 0; e < E; ++e) m = fmaxf(m, lg[e * T + t]);
+      float z = 0.0f;
+      for (int e = 0; e < E; ++e) z += expf(lg[e * T + t] - m);
+      for (int e = 0; e < E; ++e) {
+        float v = -(expf(lg[e * T + t] - m) / z) * S;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (ci[j] == e) v += cg[j] * cd[j];
+        dl[e * T + t] = v;
+      }
+    }
+    return;
+  }
+  // noisy gating: the scores are H = l + n Softplus(z), so far d score = dH; Softplus'(z)
+  // = sigmoid(z) = 1 - exp(-Softplus(z))
   const float* nrow = noise + t * E;
-  if (dload != nullptr) {
-    // kth_excluding(H, k, i) is the (k+1)-th largest H when H_i is among the k largest
-    // (H_i >= the k-th largest value), else the k-th largest, ranked by (-H, index):
-    // one pass keeps the k+1 largest (k <= 8) in ascending expert order, so an equal
-    // later value never displaces an earlier one
-    float tv[9];
-    int ti[9];
-    for (int j = 0; j <= k; ++j) {
-      tv[j] = -INFINITY;
-      ti[j] = 0;
-    }
+  if (dload == nullptr) {
     for (int e = 0; e < E; ++e) {
-      float cv = lrow[e] + nrow[e] * bwd_softplus(zrow[e]);
-      int ci = e;
-      for (int j = 0; j <= k; ++j) {
-        if (cv > tv[j]) {
-          const float sv = tv[j];
-          const int si = ti[j];
-          tv[j] = cv;
-          ti[j] = ci;
-          cv = sv;
-          ci = si;
-        }
+      const float dH = keep_part(e);
+      dl[e * T + t] = dH;
+      dz[e * T + t] = dH * nrow[e] * -expm1f(-sw[e * T + t]);
+    }
+    return;
+  }
+  // kth_excluding(H, k, i) is the (k+1)-th largest H when H_i is among the k largest
+  // (H_i >= the k-th largest value), else the k-th largest, ranked by (-H, index): one
+  // pass keeps the k+1 largest (k <= 8) in ascending expert order, so an equal later value
+  // never displaces an earlier one
+  float tv[9];
+  int ti[9];
+#pragma unroll
+  for (int j = 0; j < 9; ++j) {
+    tv[j] = -INFINITY;
+    ti[j] = 0;
+  }
+  for (int e = 0; e < E; ++e) {
+    float cv = hw[e * T + t];
+    int cix = e;
+#pragma unroll
+    for (int j = 0; j < 9; ++j) {
+      if (j <= k && cv > tv[j]) {
+        const float sv = tv[j];
+        const int si = ti[j];
+        tv[j] = cv;
+        ti[j] = cix;
+        cv = sv;
+        cix = si;
       }
     }
-    const float hk = tv[k - 1], hk1 = tv[k];
-    const int pk = ti[k - 1], pk1 = ti[k];
-    // P(x, e) = Phi(zeta), zeta = (l_e - kth_excluding) / Softplus(z_e): its gradient goes
-    // to l_e, to Softplus(z_e), and to H at the entry kth_excluding picked; the dH part
-    // is gathered first, since any entry may receive it
-    for (int e = 0; e < E; ++e) {
-      const float sp = bwd_softplus(zrow[e]);
-      const float He = lrow[e] + nrow[e] * sp;
-      const bool top = He >= hk;
-      const float zeta = (lrow[e] - (top ? hk1 : hk)) / sp;
-      const float g = dload[e] * 0.3989422804014327f * expf(-0.5f * zeta * zeta);
-      dlr[top ? pk1 : pk] += -g / sp;   // dH at the picked entry
-      dzr[e] = -g * zeta / sp;          // d Softplus(z_e), times sigmoid(z_e) below
+  }
+  float hk = tv[0], hk1 = tv[1];
+  int pk = ti[0], pk1 = ti[1];
+#pragma unroll
+  for (int j = 1; j < 9; ++j)
+    if (j == k) {
+      hk = tv[j - 1];
+      pk = ti[j - 1];
+      hk1 = tv[j];
+      pk1 = ti[j];
     }
-    for (int e = 0; e < E; ++e) {
-      const float sp = bwd_softplus(zrow[e]);
-      const float He = lrow[e] + nrow[e] * sp;
-      const bool top = He >= hk;
-      const float zeta = (lrow[e] - (top ? hk1 : hk)) / sp;
-      const float g = dload[e] * 0.3989422804014327f * expf(-0.5f * zeta * zeta);
-      const float dH = dlr[e];
-      dzr[e] = (dH * nrow[e] + dzr[e]) * sigmoidf_(zrow[e]);
-      dlr[e] = dH + g / sp;
-    }
-  } else {
-    for (int e = 0; e < E; ++e) dzr[e] = dlr[e] * nrow[e] * sigmoidf_(zrow[e]);
+  // P(x, e) = Phi(zeta), zeta = (l_e - kth_excluding) / Softplus(z_e): its gradient goes to
+  // l_e, to Softplus(z_e), and to H at the entry kth_excluding picked (pk or pk1), whose
+  // totals are gathered first
+  float to_pk = 0.0f, to_pk1 = 0.0f;
+  for (int e = 0; e < E; ++e) {
+    const float sp = sw[e * T + t];
+    const bool top = hw[e * T + t] >= hk;
+    const float zeta = (lg[e * T + t] - (top ? hk1 : hk)) / sp;
+    const float g = dload[e] * 0.3989422804014327f * expf(-0.5f * zeta * zeta);
+    if (top) to_pk1 -= g / sp;
+    else to_pk -= g / sp;
+  }
+  for (int e = 0; e < E; ++e) {
+    const float sp = sw[e * T + t];
+    const bool top = hw[e * T + t] >= hk;
+    const float zeta = (lg[e * T + t] - (top ? hk1 : hk)) / sp;
+    const float g = dload[e] * 0.3989422804014327f * expf(-0.5f * zeta * zeta);
+    const float dH = keep_part(e) + (e == pk ? to_pk : 0.0f) + (e == pk1 ? to_pk1 : 0.0f);
+    dz[e * T + t] = (dH * nrow[e] - g * zeta / sp) * -expm1f(-sp);
+    dl[e * T + t] = dH + g / sp;
   }
 }
 
-// ---------------------------------------------------- strided SIMT products (router)
+// ------------------------------------------------------------- router products
 //
-// C(m, n) (+)= sum_k A(m, k) B(n, k) with arbitrary element strides, fp32 accumulation;
-// A and B bf16 or fp32.  blockIdx.z splits the contraction into `splits` runs whose
-// partial results go to C + z * M * N (contiguous [M, N]) when splits > 1, to be summed
-// in order by sum_partials_kernel.
-namespace sr {
-constexpr int BM = 64, BN = 64, BK = 16, THREADS = 256;
+// The router's gradients from dl (and dz) [R, T] (R = E, or 2E with dz below dl):
+//   dx[t, n]  += sum_r A[r, t] B[r, n],  B = W_g (rows r < E) and W_noise (rows E..2E-1)
+//   dW[r, n]   = sum_t A[r, t] x[t, n]   (dW_g, dW_noise)
+//   dbias[e]   = sum_t dl[e, t]
+// SIMT fp32 arithmetic on coalesced tiles: every operand row is read along its contiguous
+// dimension.
+
+namespace rx {
+constexpr int TT = 32, TN = 256, TR = 32, THREADS = 256;
 }
 
-template <typename TA, typename TB>
-__device__ __forceinline__ float ldf(const TA* p, int64_t i);
-template <>
-__device__ __forceinline__ float ldf<float, float>(const float* p, int64_t i) { return __ldg(p + i); }
-template <>
-__device__ __forceinline__ float ldf<__nv_bfloat16, __nv_bfloat16>(const __nv_bfloat16* p, int64_t i) {
-  return __bfloat162float(p[i]);
+// dx += A^T B over a 32-token x 256-column tile per block, r in chunks of 32; each thread
+// holds 8 tokens x 4 columns.
+__global__ void __launch_bounds__(rx::THREADS)
+    router_dx_kernel(const float* __restrict__ A, const __nv_bfloat16* __restrict__ B0,
+                     const __nv_bfloat16* __restrict__ B1, int E, int R, int64_t T, int d,
+                     float* __restrict__ dx) {
+  __shared__ __align__(16) float sA[rx::TR][rx::TT];
+  __shared__ __align__(16) __nv_bfloat16 sB[rx::TR][rx::TN];
+  const int tid = threadIdx.x, tx = tid & 63, ty = tid >> 6;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * rx::TT;
+  const int n0 = blockIdx.y * rx::TN;
+  grid_dep_wait();
+  grid_dep_launch();
+  float acc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
+  for (int r0 = 0; r0 < R; r0 += rx::TR) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // A tile: 32 rows x 32 tokens, along the tokens
+      const int idx = tid + i * rx::THREADS, r = idx >> 5, tt = idx & 31;
+      sA[r][tt] = (r0 + r < R && t0 + tt < T) ? __ldg(A + (r0 + r) * T + t0 + tt) : 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // B tile: 32 rows x 256 columns, 8 columns per load
+      const int idx = tid + i * rx::THREADS, r = idx >> 5, c8 = (idx & 31) * 8;
+      const int row = r0 + r, col = n0 + c8;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (row < R && col < d) {
+        const __nv_bfloat16* src = row < E ? B0 + static_cast<int64_t>(row) * d
+                                           : B1 + static_cast<int64_t>(row - E) * d;
+        v = __ldg(reinterpret_cast<const uint4*>(src + col));
+      }
+      *reinterpret_cast<uint4*>(&sB[r][c8]) = v;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int r = 0; r < rx::TR; ++r) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&sA[r][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&sA[r][ty * 8 + 4]);
+      const uint2 bb = *reinterpret_cast<const uint2*>(&sB[r][tx * 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float b[4] = {__uint_as_float(bb.x << 16), __uint_as_float(bb.x & 0xFFFF0000u),
+                          __uint_as_float(bb.y << 16), __uint_as_float(bb.y & 0xFFFF0000u)};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  const int n = n0 + tx * 4;
+  if (n >= d) return;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t t = t0 + ty * 8 + i;
+    if (t >= T) break;
+    float4* p = reinterpret_cast<float4*>(dx + t * d + n);
+    float4 v = *p;
+    v.x += acc[i][0];
+    v.y += acc[i][1];
+    v.z += acc[i][2];
+    v.w += acc[i][3];
+    *p = v;
+  }
 }
 
-template <typename TA, typename TB>
-__global__ void __launch_bounds__(sr::THREADS)
-    sgemm_strided_kernel(const TA* __restrict__ A, int64_t sam, int64_t sak, const TB* __restrict__ B,
-                         int64_t sbn, int64_t sbk, float* __restrict__ C, int64_t scm, int64_t scn,
-                         int M, int N, int64_t K, int64_t kchunk, int accumulate) {
-  __shared__ float As[sr::BK][sr::BM + 4];
-  __shared__ float Bs[sr::BK][sr::BN + 4];
+namespace rw {
+constexpr int TT = 64, TN = 256, THREADS = 128;
+}
+
+// part[z][r][n] = sum over the tokens of chunk z of A[r, t] x[t, n] for the block's RG rows
+// of A (from blockIdx.y * RG) and 256 columns (two per thread); the chunk's tokens pass
+// through shared memory 64 at a time, A transposed there so that a token's RG values are
+// read as float4s.
+template <int RG>
+__global__ void __launch_bounds__(rw::THREADS)
+    router_wgrad_kernel(const float* __restrict__ A, int R, int64_t T,
+                        const __nv_bfloat16* __restrict__ x, int d, int64_t tchunk,
+                        float* __restrict__ part) {
+  __shared__ __align__(16) float sA[rw::TT][RG + 4];
   const int tid = threadIdx.x;
+  const int n = blockIdx.x * rw::TN + 2 * tid;
+  const int r0 = blockIdx.y * RG;
+  const int64_t lo = static_cast<int64_t>(blockIdx.z) * tchunk;
+  const int64_t hi = min(T, lo + tchunk);
   grid_dep_wait();
   grid_dep_launch();
-  const int m0 = blockIdx.x * sr::BM, n0 = blockIdx.y * sr::BN;
-  const int64_t k_lo = blockIdx.z * kchunk;
-  const int64_t k_hi = min(K, k_lo + kchunk);
-  const int tx = tid & 15, ty = tid >> 4;
-  float acc[4][4] = {};
-  for (int64_t k0 = k_lo; k0 < k_hi; k0 += sr::BK) {
+  float acc0[RG], acc1[RG];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int idx = tid + i * sr::THREADS;
-      const int r = idx & 63, kk = idx >> 6;   // 64 rows x 16 k
-      const int64_t kc = k0 + kk;
-      As[kk][r] = (m0 + r < M && kc < k_hi) ? ldf<TA, TA>(A, (m0 + r) * sam + kc * sak) : 0.0f;
-      Bs[kk][r] = (n0 + r < N && kc < k_hi) ? ldf<TB, TB>(B, (n0 + r) * sbn + kc * sbk) : 0.0f;
+  for (int r = 0; r < RG; ++r) acc0[r] = acc1[r] = 0.0f;
+  const bool col_ok = n < d;
+  for (int64_t t0 = lo; t0 < hi; t0 += rw::TT) {
+    for (int idx = tid; idx < RG * rw::TT; idx += rw::THREADS) {
+      const int r = idx / rw::TT, tt = idx % rw::TT;
+      sA[tt][r] = (r0 + r < R && t0 + tt < hi) ? __ldg(A + (r0 + r) * T + t0 + tt) : 0.0f;
     }
     __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < sr::BK; ++kk) {
-      float av[4], bv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        av[i] = As[kk][ty * 4 + i];
-        bv[i] = Bs[kk][tx * 4 + i];
+    const int nt = static_cast<int>(min(static_cast<int64_t>(rw::TT), hi - t0));
+#pragma unroll 4
+    for (int tt = 0; tt < nt; ++tt) {
+      float x0 = 0.0f, x1 = 0.0f;
+      if (col_ok) {
+        const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(x + (t0 + tt) * d + n));
+        x0 = __uint_as_float(v << 16);
+        x1 = __uint_as_float(v & 0xFFFF0000u);
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+      for (int r = 0; r < RG; r += 4) {
+        const float4 a = *reinterpret_cast<const float4*>(&sA[tt][r]);
+        acc0[r] = fmaf(a.x, x0, acc0[r]);
+        acc1[r] = fmaf(a.x, x1, acc1[r]);
+        acc0[r + 1] = fmaf(a.y, x0, acc0[r + 1]);
+        acc1[r + 1] = fmaf(a.y, x1, acc1[r + 1]);
+        acc0[r + 2] = fmaf(a.z, x0, acc0[r + 2]);
+        acc1[r + 2] = fmaf(a.z, x1, acc1[r + 2]);
+        acc0[r + 3] = fmaf(a.w, x0, acc0[r + 3]);
+        acc1[r + 3] = fmaf(a.w, x1, acc1[r + 3]);
+      }
     }
     __syncthreads();
   }
-  const bool partial = gridDim.z > 1;
+  if (!col_ok) return;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + ty * 4 + i;
-    if (m >= M) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx * 4 + j;
-      if (n >= N) continue;
-      if (partial) {
-        C[(static_cast<int64_t>(blockIdx.z) * M + m) * N + n] = acc[i][j];
-      } else {
-        float* c = C + m * scm + n * scn;
-        *c = accumulate ? *c + acc[i][j] : acc[i][j];
-      }
-    }
-  }
+  for (int r = 0; r < RG; ++r)
+    if (r0 + r < R)
+      *reinterpret_cast<float2*>(part + (static_cast<int64_t>(blockIdx.z) * R + r0 + r) * d + n) =
+          make_float2(acc0[r], acc1[r]);
 }
 
-// out(m, n) (+)= sum_z part[z][m][n], z in order.
-__global__ void sum_partials_kernel(const float* __restrict__ part, int splits, int M, int N,
-                                    float* __restrict__ C, int64_t scm, int64_t scn, int accumulate) {
+// dW_g[r, n] (r < E) and dW_noise[r - E, n] (r >= E) = sum_z part[z][r][n], z in order.
+__global__ void sum_router_wgrad_kernel(const float* __restrict__ part, int chunks, int E, int R,
+                                        int d, float* __restrict__ dwg, float* __restrict__ dwn) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   grid_dep_wait();
   grid_dep_launch();
-  if (i >= static_cast<int64_t>(M) * N) return;
+  if (i >= static_cast<int64_t>(R) * d) return;
   float s = 0.0f;
-  for (int z = 0; z < splits; ++z) s += part[static_cast<int64_t>(z) * M * N + i];
-  const int64_t m = i / N, n = i - m * N;
-  float* c = C + m * scm + n * scn;
-  *c = accumulate ? *c + s : s;
+  for (int z = 0; z < chunks; ++z) s += part[static_cast<int64_t>(z) * R * d + i];
+  const int64_t r = i / d;
+  if (r < E) dwg[i] = s;
+  else dwn[i - static_cast<int64_t>(E) * d] = s;
 }
 
-// Column sums of a row-major [T, E] fp32 matrix in token order: out[e] = sum_t v[t, e].
-__global__ void colsum_kernel(const float* __restrict__ v, int64_t T, int E, float* __restrict__ out) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+// out[e] = sum_t A[e, t] for a row-major [E, T] matrix: one block per row, each thread a
+// fixed strided subset in order, then a fixed tree over the block.
+__global__ void __launch_bounds__(256)
+    rowsum_kernel(const float* __restrict__ A, int64_t T, float* __restrict__ out) {
+  const float* row = A + static_cast<int64_t>(blockIdx.x) * T;
   grid_dep_wait();
   grid_dep_launch();
-  if (e >= E) return;
   float s = 0.0f;
-  for (int64_t t = 0; t < T; ++t) s += v[t * E + e];
-  out[e] = s;
-}
-
-// Adds a per-column bias to a row-major [T, E] matrix.
-__global__ void add_bias_kernel(float* __restrict__ v, int64_t T, int E, const float* __restrict__ b) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  grid_dep_wait();
-  grid_dep_launch();
-  if (i < T * E) v[i] += b[i % E];
+  for (int64_t t = threadIdx.x; t < T; t += 256) s += __ldg(row + t);
+  s = block_sum_fixed<256>(s);
+  if (threadIdx.x == 0) out[blockIdx.x] = s;
 }
 
 // ------------------------------------------------------------------ host side
 
 namespace {
-
-template <typename TA, typename TB>
-cudaError_t sgemm_strided(const TA* A, int64_t sam, int64_t sak, const TB* B, int64_t sbn, int64_t sbk,
-                          float* C, int64_t scm, int64_t scn, int M, int N, int64_t K, int accumulate,
-                          float* part, int64_t part_cap, const LaunchCtx& c) {
-  if (M <= 0 || N <= 0) return cudaSuccess;
-  const int gm = (M + sr::BM - 1) / sr::BM, gn = (N + sr::BN - 1) / sr::BN;
-  // split the contraction when the output has few tiles, so that the grid fills the GPU
-  int splits = 1;
-  while (static_cast<int64_t>(gm) * gn * splits < 2 * c.num_sms && K / (splits * 2) >= 256 &&
-         static_cast<int64_t>(splits * 2) * M * N <= part_cap)
-    splits *= 2;
-  int64_t kchunk = (K + splits - 1) / splits;
-  kchunk = (kchunk + sr::BK - 1) / sr::BK * sr::BK;
-  cudaError_t e = launch_kernel(sgemm_strided_kernel<TA, TB>, dim3(gm, gn, splits), dim3(sr::THREADS), 0,
-                                c, A, sam, sak, B, sbn, sbk, splits > 1 ? part : C, scm, scn, M, N, K,
-                                kchunk, accumulate);
-  if (e != cudaSuccess || splits == 1) return e;
-  const int64_t n = static_cast<int64_t>(M) * N;
-  return launch_kernel(sum_partials_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0,
-                       c, static_cast<const float*>(part), splits, M, N, C, scm, scn, accumulate);
-}
 
 int pick_bn_bwd(int N) {
   if (N % 256 == 0) return 256;
@@ -878,50 +936,53 @@ cudaError_t launch_backward(const BackwardProblem& p, const LaunchCtx& c) {
                       p.losses, 1);
     if (e != cudaSuccess) return e;
   }
-  // ---- router: recompute the logits (and x.W_noise), gate backward, parameter grads
+  // ---- router: gate backward from the forward's scores, then the parameter gradients
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(p.x);
   const __nv_bfloat16* wg = static_cast<const __nv_bfloat16*>(p.w_gate);
   const __nv_bfloat16* wn = static_cast<const __nv_bfloat16*>(p.w_noise);
-  e = sgemm_strided(x, d, 1, wg, d, 1, p.logits, E, 1, static_cast<int>(p.T), E, d, 0, p.part,
-                    p.part_cap, c);
-  if (e != cudaSuccess) return e;
-  if (p.bias) {
-    const int64_t m = p.T * E;
-    e = launch_kernel(add_bias_kernel, dim3(static_cast<unsigned>((m + 255) / 256)), dim3(256), 0, c,
-                      p.logits, p.T, E, p.bias);
-    if (e != cudaSuccess) return e;
-  }
-  if (p.noisy) {
-    e = sgemm_strided(x, d, 1, wn, d, 1, p.zlog, E, 1, static_cast<int>(p.T), E, d, 0, p.part,
-                      p.part_cap, c);
-    if (e != cudaSuccess) return e;
-  }
   e = launch_kernel(gate_bwd_kernel, dim3(static_cast<unsigned>((p.T + 127) / 128)), dim3(128), 0, c,
                     p.topk_idx, p.topk_gate, static_cast<const float*>(p.dgate),
-                    static_cast<const float*>(p.w_importance != 0.0f ? p.dimp : nullptr),
-                    static_cast<const float*>(p.logits), static_cast<const float*>(p.zlog), p.noise,
-                    static_cast<const float*>(p.w_load != 0.0f ? p.dload : nullptr), p.dl, p.dz, p.T,
-                    E, p.k, p.noisy, p.renorm);
+                    static_cast<const float*>(p.w_importance != 0.0f ? p.dimp : nullptr), p.lg, p.sw,
+                    p.hw, p.noise, static_cast<const float*>(p.w_load != 0.0f ? p.dload : nullptr),
+                    p.dl, p.dz, p.T, E, p.k, p.noisy, p.renorm);
   if (e != cudaSuccess) return e;
-  // dx += dl . W_g: A = dl [T, E], B(n, e) = W_g[e, n]
-  e = sgemm_strided(static_cast<const float*>(p.dl), E, 1, wg, 1, d, p.dx, d, 1, static_cast<int>(p.T),
-                    d, E, 1, p.part, p.part_cap, c);
+  // A = dl (and dz below it): R rows of [T]
+  const int R = p.noisy ? 2 * E : E;
+  const float* A = p.dl;
+  // dx += A^T [W_g; W_noise]
+  e = launch_kernel(router_dx_kernel,
+                    dim3(static_cast<unsigned>((p.T + rx::TT - 1) / rx::TT), (d + rx::TN - 1) / rx::TN),
+                    dim3(rx::THREADS), 0, c, A, wg, wn, E, R, p.T, d, p.dx);
   if (e != cudaSuccess) return e;
-  // dW_g[e, :] = sum_t dl[t, e] x[t, :]
-  e = sgemm_strided(static_cast<const float*>(p.dl), 1, E, x, 1, d, p.dw_gate, d, 1, E, d, p.T, 0,
-                    p.part, p.part_cap, c);
-  if (e != cudaSuccess) return e;
-  if (p.dbias) {
-    e = launch_kernel(colsum_kernel, dim3((E + 127) / 128), dim3(128), 0, c,
-                      static_cast<const float*>(p.dl), p.T, E, p.dbias);
+  // [dW_g; dW_noise] = A x, as partial sums over token chunks summed in chunk order
+  {
+    const int rg = R <= 8 ? 8 : R <= 16 ? 16 : 32;
+    const int gx = (d + rw::TN - 1) / rw::TN, gy = (R + rg - 1) / rg;
+    int64_t chunks = (2LL * c.num_sms + gx * gy - 1) / (gx * gy);
+    const int64_t by_cap = p.part_cap / (static_cast<int64_t>(R) * d);
+    const int64_t by_t = (p.T + rw::TT - 1) / rw::TT;
+    if (chunks > by_cap) chunks = by_cap;
+    if (chunks > by_t) chunks = by_t;
+    if (chunks < 1) chunks = 1;
+    int64_t tchunk = (p.T + chunks - 1) / chunks;
+    tchunk = (tchunk + rw::TT - 1) / rw::TT * rw::TT;
+    chunks = (p.T + tchunk - 1) / tchunk;
+    const dim3 grid(gx, gy, static_cast<unsigned>(chunks));
+    switch (rg) {
+      case 8: e = launch_kernel(router_wgrad_kernel<8>, grid, dim3(rw::THREADS), 0, c, A, R, p.T, x, d, tchunk, p.part); break;
+      case 16: e = launch_kernel(router_wgrad_kernel<16>, grid, dim3(rw::THREADS), 0, c, A, R, p.T, x, d, tchunk, p.part); break;
+      default: e = launch_kernel(router_wgrad_kernel<32>, grid, dim3(rw::THREADS), 0, c, A, R, p.T, x, d, tchunk, p.part); break;
+    }
+    if (e != cudaSuccess) return e;
+    const int64_t nout = static_cast<int64_t>(R) * d;
+    e = launch_kernel(sum_router_wgrad_kernel, dim3(static_cast<unsigned>((nout + 255) / 256)), dim3(256), 0,
+                      c, static_cast<const float*>(p.part), static_cast<int>(chunks), E, R, d, p.dw_gate,
+                      p.dw_noise);
     if (e != cudaSuccess) return e;
   }
-  if (p.noisy) {
-    e = sgemm_strided(static_cast<const float*>(p.dz), E, 1, wn, 1, d, p.dx, d, 1, static_cast<int>(p.T),
-                      d, E, 1, p.part, p.part_cap, c);
-    if (e != cudaSuccess) return e;
-    e = sgemm_strided(static_cast<const float*>(p.dz), 1, E, x, 1, d, p.dw_noise, d, 1, E, d, p.T, 0,
-                      p.part, p.part_cap, c);
+  if (p.dbias) {
+    e = launch_kernel(rowsum_kernel, dim3(E), dim3(256), 0, c, static_cast<const float*>(p.dl), p.T,
+                      p.dbias);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -358,6 +358,24 @@ __device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Sum of one value per thread over a block of NT threads (a multiple of 32) in a fixed
+// order: a butterfly within each warp, then the warps' sums in warp order by thread 0.
+// The result is returned to thread 0 only.  Every thread of the block must call it.
+template <int NT>
+__device__ __forceinline__ float block_sum_fixed(float v) {
+  __shared__ float warp_sums[NT / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float s = 0.0f;
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) s += warp_sums[w];
+  }
+  return s;
+}
+
 // erf by Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26:
 // erf(x) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-x^2), t = 1 / (1 + p x),
 // x >= 0, |error| <= 1.5e-7 (odd extension for x < 0).  About a third of the

@@ -115,10 +115,11 @@ struct RouteProblem {
   float* partials;    // workspace: [route_blocks][2][E]
   float* logits_ws;   // fp32 path only: [T][E] ([T][groups + E] for hierarchical gating)
   float* nz_ws;       // fp32 path only: [T][E]
-  float* lw = nullptr;  // bf16 noisy path with Importance/Load: clean logits, Softplus
+  float* lw = nullptr;  // bf16 path: clean logits (+ bias), and for noisy gating Softplus
   float* sw = nullptr;  // (x.W_noise) and noisy scores H, each [E][T], and the k-th /
-  float* hw = nullptr;  // (k+1)-th noisy scores [2][T] of each token
-  float* kw = nullptr;
+  float* hw = nullptr;  // (k+1)-th noisy scores [2][T] of each token; written for noisy
+  float* kw = nullptr;  // gating with Importance/Load, or always with store_scores
+  bool store_scores = false;  // the training forward keeps them for the backward
 };
 int route_blocks(int64_t T);
 cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c);
@@ -232,10 +233,13 @@ struct BackwardProblem {
   void* d_o;      // [T*k + 64 E, d] 16-bit
   void* du;       // [T*k + 64 E, f] bf16
   float* dx_perm; // [T*k, d]
-  float* logits;  // [T, E]
-  float* zlog;    // [T, E]
-  float* dl;      // [T, E]
-  float* dz;      // [T, E]
+  // the router's scores kept by the training forward, [E, T]: clean logits (+ bias),
+  // and for noisy gating Softplus(x.W_noise) and the noisy scores H
+  const float* lg;
+  const float* sw;
+  const float* hw;
+  float* dl;      // [E, T]; for noisy gating dz [E, T] follows it (dz = dl + E T)
+  float* dz;
   float* dimp;    // [E]
   float* dload;   // [E]
   float* part;    // split-contraction partial sums

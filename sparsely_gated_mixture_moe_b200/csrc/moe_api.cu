@@ -106,8 +106,11 @@ Layout layout(const moe_config* c) {
 }
 
 // The forward state moe_forward_train keeps for moe_backward.
+// The router's scores are kept expert-major ([E, T]) as the gate wrote them: clean
+// logits (+ bias) in lg, and for noisy gating Softplus(x.W_noise) in sw, the noisy scores
+// H in hw and the k-th / (k+1)-th H of each token [2, T] in kw.
 struct TrainLayout {
-  size_t offsets, slot_pos, perm_src, x_perm, u, h, y_perm, total;
+  size_t offsets, slot_pos, perm_src, x_perm, u, h, y_perm, lg, sw, hw, kw, total;
 };
 
 TrainLayout train_layout(const moe_config* c) {
@@ -128,13 +131,24 @@ TrainLayout train_layout(const moe_config* c) {
   o = align_up(o + static_cast<size_t>(n) * c->d_ff * 2);
   L.y_perm = o;
   o = align_up(o + static_cast<size_t>(n) * c->d_model * 4);
+  const size_t TE = static_cast<size_t>(c->T) * c->E;
+  L.lg = o;
+  o = align_up(o + TE * 4);
+  L.sw = L.hw = L.kw = o;
+  if (c->gating == MOE_GATE_NOISY_TOPK) {
+    o = align_up(o + TE * 4);
+    L.hw = o;
+    o = align_up(o + TE * 4);
+    L.kw = o;
+    o = align_up(o + static_cast<size_t>(c->T) * 2 * 4);
+  }
   L.total = o;
   return L;
 }
 
 // moe_backward's workspace: the step workspace (error word first), then its buffers.
 struct BackwardLayout {
-  size_t poff, d_o, du, dx_perm, logits, zlog, dl, dz, dimp, dload, part, total;
+  size_t poff, d_o, du, dx_perm, dl, dimp, dload, part, total;  // dz follows dl
   int64_t part_cap;
 };
 
@@ -152,14 +166,8 @@ BackwardLayout backward_layout(const moe_config* c, size_t steps) {
   o = align_up(o + static_cast<size_t>(prows) * c->d_ff * 2);
   L.dx_perm = o;
   o = align_up(o + static_cast<size_t>(n) * c->d_model * 4);
-  L.logits = o;
-  o = align_up(o + TE * 4);
-  L.zlog = o;
-  o = align_up(o + TE * 4);
-  L.dl = o;
-  o = align_up(o + TE * 4);
-  L.dz = o;
-  o = align_up(o + TE * 4);
+  L.dl = o;  // [E, T], for noisy gating followed by dz [E, T]
+  o = align_up(o + TE * 4 * (c->gating == MOE_GATE_NOISY_TOPK ? 2 : 1));
   L.dimp = o;
   o = align_up(o + static_cast<size_t>(c->E) * 4);
   L.dload = o;
@@ -221,10 +229,12 @@ struct Ctx {
   }
 };
 
+// keep (training only, or null): the train state's base; the gate then writes the
+// router's scores into its lg / sw / hw / kw buffers for the backward.
 moe_status do_route(const moe_config* cfg, const Layout& L, const void* x, const void* w_gate,
                     const void* w_noise, const float* noise, const float* logit_bias,
                     int32_t* topk_idx, float* topk_gate, float* importance, float* load,
-                    uint8_t* near_tie, void* ws, Ctx& ctx) {
+                    uint8_t* near_tie, void* ws, Ctx& ctx, uint8_t* keep = nullptr) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   RouteProblem p;
   p.T = cfg->T;
@@ -249,7 +259,14 @@ moe_status do_route(const moe_config* cfg, const Layout& L, const void* x, const
   p.partials = reinterpret_cast<float*>(w + L.partials);
   p.logits_ws = reinterpret_cast<float*>(w + L.logits);
   p.nz_ws = reinterpret_cast<float*>(w + L.nz);
-  if (cfg->dtype == MOE_BF16 && cfg->gating == MOE_GATE_NOISY_TOPK) {
+  if (keep != nullptr) {
+    const TrainLayout S = train_layout(cfg);
+    p.lw = reinterpret_cast<float*>(keep + S.lg);
+    p.sw = reinterpret_cast<float*>(keep + S.sw);
+    p.hw = reinterpret_cast<float*>(keep + S.hw);
+    p.kw = reinterpret_cast<float*>(keep + S.kw);
+    p.store_scores = true;
+  } else if (cfg->dtype == MOE_BF16 && cfg->gating == MOE_GATE_NOISY_TOPK) {
     p.lw = reinterpret_cast<float*>(w + L.lw);
     p.sw = reinterpret_cast<float*>(w + L.sw);
     p.hw = reinterpret_cast<float*>(w + L.hw);
@@ -654,7 +671,7 @@ moe_status moe_forward_train(const moe_config* cfg, const void* x, const void* w
   void* h = sb + S.h;
   void* y_perm = sb + S.y_perm;
   st = do_route(cfg, L, x, w_gate, w_noise, noise, logit_bias, topk_idx, topk_gate, importance, load,
-                near_tie, ws, ctx);
+                near_tie, ws, ctx, sb);
   if (st != MOE_OK) return st;
   st = do_permute(cfg, L, topk_idx, x, counts, offsets, perm_src, slot_pos, x_perm, ws, ctx);
   if (st != MOE_OK) return st;
@@ -739,10 +756,11 @@ moe_status moe_backward(const moe_config* cfg, const void* x, const void* w_gate
   p.d_o = w + B.d_o;
   p.du = w + B.du;
   p.dx_perm = reinterpret_cast<float*>(w + B.dx_perm);
-  p.logits = reinterpret_cast<float*>(w + B.logits);
-  p.zlog = reinterpret_cast<float*>(w + B.zlog);
+  p.lg = reinterpret_cast<const float*>(sb + S.lg);
+  p.sw = noisy ? reinterpret_cast<const float*>(sb + S.sw) : nullptr;
+  p.hw = noisy ? reinterpret_cast<const float*>(sb + S.hw) : nullptr;
   p.dl = reinterpret_cast<float*>(w + B.dl);
-  p.dz = reinterpret_cast<float*>(w + B.dz);
+  p.dz = noisy ? p.dl + cfg->T * cfg->E : nullptr;
   p.dimp = reinterpret_cast<float*>(w + B.dimp);
   p.dload = reinterpret_cast<float*>(w + B.dload);
   p.part = reinterpret_cast<float*>(w + B.part);

@@ -50,15 +50,18 @@ struct GateArgs {
   float* topk_gate;
   uint8_t* near_tie;
   float* partials;  // [gridDim.x][2][E] or null
-  // noisy gating with Importance/Load asked for, on the tensor-core path: the gate writes
-  // each token's clean logits (bias added), Softplus(x.W_noise) and noisy scores H, all
-  // [E, T] (expert-major, so a warp's 32 tokens store 128 contiguous bytes), and its k-th
-  // and (k+1)-th H [2, T] here instead of forming the sums itself (importance_load_kernel
-  // does, over the whole grid); null otherwise
+  // Scores kept for later kernels, all [E, T] (expert-major, so a warp's 32 tokens store
+  // 128 contiguous bytes), or null: each token's clean logits (bias added) in lw and, for
+  // noisy gating, Softplus(x.W_noise) in sw, the noisy scores H in hw and the k-th and
+  // (k+1)-th H [2, T] in kw.  Written for noisy gating with Importance/Load asked for on
+  // the tensor-core path (split = 1: the gate leaves the sums to importance_load_kernel,
+  // which forms them over the whole grid) and for the training forward (the backward
+  // reads them instead of recomputing the router).
   float* lw;
   float* sw;
   float* hw;
   float* kw;
+  int split;
 };
 
 // Softplus(z) = max(z, 0) + log(1 + e^-|z|), with the fast exponential and logarithm:
@@ -248,6 +251,8 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
               g.sw[e * g.T + t] = sp;
               g.hw[e * g.T + t] = sv;
             }
+          } else if (g.lw != nullptr && valid) {
+            g.lw[e * g.T + t] = sv;
           }
         }
         sc[jj] = sv;
@@ -366,7 +371,7 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
       g.kw[g.T + t] = kth1;
     }
   }
-  if (g.partials == nullptr || g.lw != nullptr) {  // uniform across the gate threads
+  if (g.partials == nullptr || g.split) {  // uniform across the gate threads
     sync();                                        // the lists are reused by the next tile
     return;
   }
@@ -897,19 +902,23 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-__global__ void finalize_importance_load_kernel(const float* __restrict__ partials, int nblocks,
-                                                int E, float* importance, float* load) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+// Importance[e] (blockIdx.y = 0) and Load[e] (blockIdx.y = 1) from the per-block
+// partials [nblocks][2][E]: one block per expert and quantity, each thread a fixed strided
+// subset of the partials in order, then a fixed tree over the block, so the sum is the
+// same on every run.
+__global__ void __launch_bounds__(256)
+    finalize_importance_load_kernel(const float* __restrict__ partials, int nblocks, int E,
+                                    float* importance, float* load) {
+  const int e = blockIdx.x, which = blockIdx.y;
   grid_dep_wait();
   grid_dep_launch();
-  if (e >= E) return;
-  float si = 0.0f, sl = 0.0f;
-  for (int b = 0; b < nblocks; ++b) {
-    si += partials[(static_cast<int64_t>(b) * 2 + 0) * E + e];
-    sl += partials[(static_cast<int64_t>(b) * 2 + 1) * E + e];
-  }
-  if (importance) importance[e] = si;
-  if (load) load[e] = sl;
+  float* out = which == 0 ? importance : load;
+  if (out == nullptr) return;  // uniform over the block
+  float s = 0.0f;
+  for (int b = threadIdx.x; b < nblocks; b += 256)
+    s += partials[(static_cast<int64_t>(b) * 2 + which) * E + e];
+  s = block_sum_fixed<256>(s);
+  if (threadIdx.x == 0) out[e] = s;
 }
 
 // ------------------------------------------------------------------ launchers
@@ -930,6 +939,7 @@ static GateArgs gate_args(const RouteProblem& p) {
   g.near_tie = p.near_tie;
   g.partials = (p.importance || p.load) ? p.partials : nullptr;
   g.lw = g.sw = g.hw = g.kw = nullptr;
+  g.split = 0;
   return g;
 }
 
@@ -937,7 +947,7 @@ static int k_bucket(int k) { return k <= 1 ? 1 : k <= 2 ? 2 : k <= 4 ? 4 : 8; }
 
 static cudaError_t launch_finalize(const RouteProblem& p, int nblocks, const LaunchCtx& c) {
   if (!(p.importance || p.load)) return cudaSuccess;
-  return launch_kernel(finalize_importance_load_kernel, dim3((p.E + 127) / 128), dim3(128), 0, c,
+  return launch_kernel(finalize_importance_load_kernel, dim3(p.E, 2), dim3(256), 0, c,
                        static_cast<const float*>(p.partials), nblocks, p.E, p.importance, p.load);
 }
 
@@ -986,7 +996,7 @@ static cudaError_t launch_importance_load(const RouteProblem& p, const LaunchCtx
                                 static_cast<const float*>(p.topk_gate), p.T, p.E, p.k, per,
                                 p.load != nullptr ? 1 : 0, p.partials);
   if (e != cudaSuccess) return e;
-  return launch_kernel(finalize_importance_load_kernel, dim3((p.E + 127) / 128), dim3(128), 0, c,
+  return launch_kernel(finalize_importance_load_kernel, dim3(p.E, 2), dim3(256), 0, c,
                        static_cast<const float*>(p.partials), static_cast<int>(chunks), p.E,
                        p.importance, p.load);
 }
@@ -995,12 +1005,15 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   RouteTcArgs a;
   a.g = gate_args(p);
   const bool split = p.noisy && (p.importance || p.load) && p.lw != nullptr;
-  if (split) {
+  if (split || p.store_scores) {
     a.g.lw = p.lw;
-    a.g.sw = p.sw;
-    a.g.hw = p.hw;
-    a.g.kw = p.kw;
+    if (p.noisy) {
+      a.g.sw = p.sw;
+      a.g.hw = p.hw;
+      a.g.kw = p.kw;
+    }
   }
+  a.g.split = split ? 1 : 0;
   const int n_scores = p.hier ? p.E + p.groups : p.E;  // score columns (rows of w_gate)
   a.e_pad = (n_scores + 15) / 16 * 16;
   a.acc_cols = 32;
