@@ -163,6 +163,12 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def y_bf16_of(w: workloads.Workload) -> bool:
+    """The benchmark's layer output type: bf16 for a bf16 layer (each row's fp32 sum
+    rounded once), fp32 for an fp32 layer."""
+    return w.dtype == "bf16"
+
+
 def algorithmic(w: workloads.Workload, n_kept: int, counts_kept, fused=False):
     """Algorithmic FLOPs and bytes of each step (kept assignments only, no padding).
 
@@ -170,10 +176,12 @@ def algorithmic(w: workloads.Workload, n_kept: int, counts_kept, fused=False):
     rows, x_perm (dtype) read, y_perm (fp32) written.  Route bytes: x, the gating
     weights, noise, and the chosen indices and gates.  Permute: the chosen experts read,
     slot_pos and perm_src written, counts and offsets, and the kept token rows read from
-    x and written to x_perm.  Combine: y_perm rows read, gates and slots, y written.
-    fused (k = 1, FFN and combine as one step): the FFN writes every row of y (fp32) and
-    reads each kept row's source index and gate; no combine bytes."""
+    x and written to x_perm.  Combine: y_perm rows read, gates and slots, y written (in
+    the output type of y_bf16_of).  fused (k = 1, FFN and combine as one step): the FFN
+    writes every row of y and reads each kept row's source index and gate; no combine
+    bytes."""
     es = 2 if w.dtype == "bf16" else 4
+    ys = 2 if y_bf16_of(w) else 4
     T, d, f, E, k = w.T, w.d_model, w.d_ff, w.E, w.k
     active = int(sum(1 for c in counts_kept if c > 0))
     ffn_flops = 4.0 * n_kept * d * f
@@ -181,9 +189,9 @@ def algorithmic(w: workloads.Workload, n_kept: int, counts_kept, fused=False):
     noisy = w.gating == "noisy_topk"
     route_bytes = T * d * es + E * d * es * (2 if noisy else 1) + (T * E * 4 if noisy else 0) + T * k * 8
     permute_bytes = T * k * 4 * 3 + E * 8.0 + n_kept * d * es * 2
-    combine_bytes = n_kept * d * 4.0 + T * k * 8 + T * d * 4.0
+    combine_bytes = n_kept * d * 4.0 + T * k * 8 + T * d * float(ys)
     if fused:
-        ffn_bytes = active * 2.0 * d * f * es + n_kept * d * es + T * d * 4.0 + n_kept * 8.0 + T * 4.0
+        ffn_bytes = active * 2.0 * d * f * es + n_kept * d * es + T * d * float(ys) + n_kept * 8.0 + T * 4.0
         combine_bytes = 0.0
     return {"ffn_flops": ffn_flops, "ffn_bytes": ffn_bytes, "route_bytes": route_bytes,
             "permute_bytes": permute_bytes, "combine_bytes": combine_bytes}
@@ -280,6 +288,7 @@ def config_json(w):
         "" if w.zipf_s is None else " zipf_s=%s" % w.zipf_s),
         "T": w.T, "d_model": w.d_model, "d_ff": w.d_ff, "E": w.E, "k": w.k,
         "capacity_factor": w.capacity_factor, "hidden_f16": w.hidden_f16,
+        "y": "bf16 (fp32 sums rounded once)" if y_bf16_of(w) else "fp32",
         "l2": "flushed before every timed step (256 MB written, then read back, outside the events)",
         "parallelism": "replicas"}
     return c
@@ -297,7 +306,8 @@ class LayerBench:
         self.cfg = moe.make_config(w.T, w.d_model, w.d_ff, w.E, w.k, gating=w.gating,
                                    renorm=w.renorm, capacity_factor=w.capacity_factor, act=w.act,
                                    dtype=w.dtype, hidden_f16=w.hidden_f16, groups=w.groups,
-                                   k_primary=w.k_primary)
+                                   k_primary=w.k_primary, y_bf16=y_bf16_of(w))
+        self.ydt = torch.bfloat16 if y_bf16_of(w) else torch.float32
         self.d = moe.prepare_weights(self.cfg, d)  # fp16 w2 for fp16 hidden (exact re-encoding)
         T, k, E, dm, f = w.T, w.k, w.E, w.d_model, w.d_ff
         self.o = o = dict(
@@ -312,7 +322,7 @@ class LayerBench:
             h=torch.empty(T * k, f, dtype=torch.float16 if w.hidden_f16 else w.torch_dtype,
                           device=dev),
             y_perm=torch.empty(T * k, dm, dtype=torch.float32, device=dev),
-            y=torch.empty(T, dm, dtype=torch.float32, device=dev))
+            y=torch.empty(T, dm, dtype=self.ydt, device=dev))
         self.noisy = w.gating == "noisy_topk"
         o["importance"] = torch.empty(E, dtype=torch.float32, device=dev) if self.noisy else None
         o["load"] = torch.empty(E, dtype=torch.float32, device=dev) if self.noisy and k < E else None
@@ -490,11 +500,11 @@ def end_to_end(lb, flush, steps, world, dev, stream):
     layers = [moe.MoELayer(lb.cfg, wl, device=dev) for _ in range(2)]
     x_host = inp["x"].pin_memory()
     noise_host = inp["noise"].pin_memory() if noisy else None
-    y_host = [torch.empty(T, dm, dtype=torch.float32).pin_memory() for _ in range(2)]
+    y_host = [torch.empty(T, dm, dtype=lb.ydt).pin_memory() for _ in range(2)]
     x_dev = [torch.empty_like(d["x"]) for _ in range(2)]
     noise_dev = [torch.empty_like(d["noise"]) if noisy else None for _ in range(2)]
     h2d = x_host.numel() * x_host.element_size() + (noise_host.numel() * 4 if noisy else 0)
-    d2h = y_host[0].numel() * 4
+    d2h = y_host[0].numel() * y_host[0].element_size()
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_c = [torch.cuda.Event() for _ in range(2)]
@@ -582,7 +592,8 @@ def training_step(lb, flush, steps, world, dev, stream):
     if moe.lib.moe_train_state_size(__import__("ctypes").byref(cfg)) == 0:
         return {"unavailable": "no backward pass for this configuration"}
     noisy = lb.noisy
-    o = {"y": torch.empty(T, dm, device=dev), "idx": torch.empty(T, k, dtype=torch.int32, device=dev),
+    o = {"y": torch.empty(T, dm, dtype=lb.ydt, device=dev),
+         "idx": torch.empty(T, k, dtype=torch.int32, device=dev),
          "gate": torch.empty(T, k, device=dev), "counts": torch.empty(E, dtype=torch.int32, device=dev),
          "imp": torch.empty(E, device=dev), "load": torch.empty(E, device=dev) if noisy else None,
          "dx": torch.empty(T, dm, device=dev), "dwg": torch.empty(E, dm, device=dev),

@@ -31,9 +31,10 @@
  *    per output feature, contiguous along the contraction): the pages write x.W_g with
  *    W_g as [d_model, E]; w_gate here is its transpose [E, d_model].
  *  - Index tensors are int32.  Assignment a = t*k + j is token t's j-th choice.
- *  - x, the weights, x_perm and h are in cfg->dtype; the expert outputs y_perm, the
- *    layer output y, gates, noise, logit_bias, importance and load are always fp32 (the
- *    products accumulate in fp32 and are not rounded to bf16 on the way out).
+ *  - x, the weights, x_perm and h are in cfg->dtype; the expert outputs y_perm, gates,
+ *    noise, logit_bias, importance and load are always fp32 (the products accumulate in
+ *    fp32 and are not rounded to bf16 on the way out); the layer output y is fp32, or
+ *    bf16 with cfg->y_bf16 (the fp32 sum of its row rounded once).
  *  - T == 0 is valid: nothing is launched, the per-expert outputs that are given
  *    (counts, offsets, importance, load) are zero-filled on `stream`, and per-token
  *    pointers may be NULL.
@@ -131,6 +132,9 @@ typedef struct {
   int32_t groups;         /* MOE_GATE_HIERARCHICAL: expert groups (divides E); else ignored */
   int32_t k_primary;      /* MOE_GATE_HIERARCHICAL: groups kept per token (divides k, and
                              k / k_primary <= E / groups); else ignored */
+  int32_t y_bf16;         /* bf16 only, 0 or 1: 1 writes the layer output y in bf16, each
+                             row's fp32 sum rounded once to nearest even (y_perm stays
+                             fp32); 0 writes y in fp32 */
 } moe_config;
 
 /* Human-readable name of a status code (static string). */
@@ -220,7 +224,8 @@ moe_status moe_expert_ffn_gather(const moe_config* cfg, const void* x, const int
 /* Gate-weighted combine [Shazeer et al., "Methode": y = sum_i G(x)_i E_i(x)]:
  *   y[t] = sum_j topk_gate[t, j] * y_perm[slot_pos[t*k + j]]   (dropped slots add 0)
  *  y_perm [T*k, d_model] fp32, slot_pos [T*k] int32, topk_gate [T, k] fp32 in
- *  y      [T, d_model] fp32 out; accumulated in the order j = 0 .. k-1. */
+ *  y      [T, d_model] fp32 out (bf16 with cfg->y_bf16); accumulated in fp32 in the order
+ *         j = 0 .. k-1, then stored. */
 moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* slot_pos,
                        const float* topk_gate, void* y, void* ws, moe_stream_t stream);
 
@@ -232,7 +237,8 @@ moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t*
  * for k = 1), so y_perm never exists.  Same arithmetic as the two steps: y is bit-equal
  * to moe_expert_ffn + moe_combine on the same inputs.
  *  x_perm, offsets, w1, w2, h as moe_expert_ffn;  perm_src, slot_pos as written by
- *  moe_permute;  topk_gate [T, 1] fp32 in;  y [T, d_model] fp32 out (every row written).
+ *  moe_permute;  topk_gate [T, 1] fp32 in;  y [T, d_model] fp32 out, bf16 with
+ *  cfg->y_bf16 (every row written).
  * The rows of dropped tokens (slot_pos[t] < 0) are zeroed by the down-projection's
  * epilogue threads before its first tile; a perm_src entry outside [0, T) sets
  * MOE_DEVERR_SLOT.  * Returns MOE_ERR_UNSUPPORTED when k != 1 or dtype is not bf16. */
@@ -254,7 +260,7 @@ moe_status moe_expert_ffn_combine_gather(const moe_config* cfg, const void* x,
 
 /* The whole layer forward on one stream: moe_route, moe_permute, moe_expert_ffn,
  * moe_combine (moe_expert_ffn_combine in place of the last two when k = 1 and dtype is
- * bf16).  Inputs as in the step calls; y [T, d_model] fp32 out.  topk_idx,
+ * bf16).  Inputs as in the step calls; y [T, d_model] fp32 (bf16 with cfg->y_bf16) out.  topk_idx,
  * topk_gate (both [T, k]) and counts ([E]) are outputs the caller must provide;
  * importance, load and near_tie may be NULL.  The intermediates live in `ws`
  * (moe_forward_workspace_size bytes). */

@@ -283,14 +283,15 @@ class MoELayer:
 
     weights: dict with w_gate [E,d], w1 [E,f,d], w2 [E,d,f] (and w_noise [E,d] for noisy
     gating, logit_bias [E] fp32 if used), CUDA tensors in the config's dtype.  The layer
-    output y [T, d] is fp32.
+    output y [T, d] is fp32, or bf16 when the config asks for it (y_bf16).
     """
 
     def __init__(self, cfg: MoEConfig, weights: dict, device="cuda"):
         self.cfg = cfg
         self.w = prepare_weights(cfg, weights)
         T, k, E, d = cfg.T, cfg.k, cfg.E, cfg.d_model
-        self.y = torch.empty(T, d, dtype=torch.float32, device=device)
+        self.y = torch.empty(T, d, dtype=torch.bfloat16 if cfg.y_bf16 else torch.float32,
+                             device=device)
         self.topk_idx = torch.empty(T, k, dtype=torch.int32, device=device)
         self.topk_gate = torch.empty(T, k, dtype=torch.float32, device=device)
         self.counts = torch.empty(E, dtype=torch.int32, device=device)

@@ -32,17 +32,20 @@ class MoEConfig(ctypes.Structure):
         ("hidden_f16", ctypes.c_int32),
         ("groups", ctypes.c_int32),
         ("k_primary", ctypes.c_int32),
+        ("y_bf16", ctypes.c_int32),
     ]
 
 
 def make_config(T, d_model, d_ff, E, k, gating="softmax_topk", renorm=True,
                 capacity_factor=None, act="relu", dtype="bf16", hidden_f16=False, groups=None,
-                k_primary=1) -> MoEConfig:
+                k_primary=1, y_bf16=False) -> MoEConfig:
     """Build a MoEConfig from plain values (capacity_factor None = no limit; groups and
-    k_primary only for hierarchical gating)."""
+    k_primary only for hierarchical gating; y_bf16: the layer output in bf16, bf16 layers
+    only)."""
     return MoEConfig(T=T, d_model=d_model, d_ff=d_ff, E=E, k=k, gating=GATING[gating],
                      renorm=1 if renorm else 0,
                      capacity_factor=0.0 if capacity_factor is None else float(capacity_factor),
                      act=ACT[act], dtype=DTYPE[dtype], hidden_f16=1 if hidden_f16 else 0,
                      groups=0 if groups is None else int(groups),
-                     k_primary=int(k_primary) if gating == "hierarchical" else 0)
+                     k_primary=int(k_primary) if gating == "hierarchical" else 0,
+                     y_bf16=1 if y_bf16 else 0)

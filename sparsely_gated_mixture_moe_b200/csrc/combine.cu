@@ -2,14 +2,17 @@
 //
 // The layer output of Shazeer et al. ("Methode"): y = sum_i G(x)_i E_i(x), with only the
 // k chosen experts contributing and a dropped assignment (slot_pos = -1) adding nothing.
-// y_perm and y are fp32 for both layer dtypes (the expert outputs leave the tensor cores
-// as fp32 accumulators).  One warp per token; each lane handles 16-byte vectors of the
-// row, gathers the k expert rows and accumulates in fp32 in the order j = 0 .. k-1.
+// y_perm is fp32 for both layer dtypes (the expert outputs leave the tensor cores as fp32
+// accumulators); y is fp32, or bf16 when asked for (each fp32 sum rounded once).  One
+// warp per token; each lane handles 4-value vectors of the row, gathers the k expert rows
+// and accumulates in fp32 in the order j = 0 .. k-1.
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
 
+// Four consecutive values of a row: loads from fp32, stores to fp32 (16 bytes) or bf16
+// (8 bytes, round to nearest even).
 template <typename T>
 struct Vec;
 template <>
@@ -23,13 +26,20 @@ struct Vec<float> {
     *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
   }
 };
+template <>
+struct Vec<__nv_bfloat16> {
+  __device__ static void store(void* p, const float (&v)[4]) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+  }
+};
 constexpr int kCombineWarps = 8;
 
-template <typename T>
+template <typename OUT>
 __global__ void __launch_bounds__(kCombineWarps * 32)
-    combine_kernel(const T* __restrict__ y_perm, const int32_t* __restrict__ slot_pos,
-                   const float* __restrict__ gate, T* __restrict__ y, int64_t T_, int k, int d,
+    combine_kernel(const float* __restrict__ y_perm, const int32_t* __restrict__ slot_pos,
+                   const float* __restrict__ gate, OUT* __restrict__ y, int64_t T_, int k, int d,
                    int* err) {
+  using T = float;
   constexpr int V = Vec<T>::N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kCombineWarps + warp;
@@ -76,7 +86,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) Vec<T>::store(y + t * d + (v + u * 32) * V, acc[u]);
+    for (int u = 0; u < 4; ++u) Vec<OUT>::store(y + t * d + (v + u * 32) * V, acc[u]);
   }
   for (; v < nv; v += 32) {
     float acc[V];
@@ -91,13 +101,18 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
         for (int i = 0; i < V; ++i) acc[i] = fmaf(g[j], r[i], acc[i]);
       }
     }
-    Vec<T>::store(y + t * d + v * V, acc);
+    Vec<OUT>::store(y + t * d + v * V, acc);
   }
 }
 
 cudaError_t launch_combine(const CombineProblem& p, const LaunchCtx& c) {
   const int64_t blocks = (p.T + kCombineWarps - 1) / kCombineWarps;
   if (blocks == 0) return cudaSuccess;
+  if (p.y_bf16)
+    return launch_kernel(combine_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(blocks)),
+                         dim3(kCombineWarps * 32), 0, c, static_cast<const float*>(p.y_perm),
+                         p.slot_pos, p.gate, static_cast<__nv_bfloat16*>(p.y), p.T, p.k, p.d,
+                         c.err);
   return launch_kernel(combine_kernel<float>, dim3(static_cast<unsigned>(blocks)),
                        dim3(kCombineWarps * 32), 0, c, static_cast<const float*>(p.y_perm),
                        p.slot_pos, p.gate, static_cast<float*>(p.y), p.T, p.k, p.d, c.err);

@@ -68,6 +68,7 @@ constexpr int OUT_BF16 = 0;  // act, bf16
 constexpr int OUT_F16 = 1;   // act, fp16
 constexpr int OUT_F32 = 2;   // fp32
 constexpr int OUT_COMBINE = 3;  // fp32 times the gate, into the token's row of y (k = 1)
+constexpr int OUT_COMBINE_BF16 = 4;  // as OUT_COMBINE, y in bf16 (the scaled fp32 rounded)
 
 struct Args {
   const int32_t* offsets;
@@ -81,9 +82,9 @@ struct Args {
   int act;       // 0 none, 1 ReLU, 2 GELU
   int out_mode;  // OUT_*
   int ab_f16;    // operand type of A and B: 1 fp16, 0 bf16
-  const int32_t* perm_src;  // OUT_COMBINE: assignment of each permuted row (= token, k = 1)
-  const float* gate;        // OUT_COMBINE: gate of each assignment
-  const int32_t* slot_pos;  // OUT_COMBINE: permuted row of each token, < 0 when dropped
+  const int32_t* perm_src;  // OUT_COMBINE*: assignment of each permuted row (= token, k = 1)
+  const float* gate;        // OUT_COMBINE*: gate of each assignment
+  const int32_t* slot_pos;  // OUT_COMBINE*: permuted row of each token, < 0 when dropped
   const int32_t* gather_src;  // non-null: A row s is row gather_src[s] / gather_k of the
   int gather_k;               // A tensor (the token rows x), gathered by the TMA itself
   void* pre;                  // OUT_BF16 / OUT_F16 with an activation: also store the
@@ -132,7 +133,15 @@ __device__ __forceinline__ void epilogue_rows(const Args& a, uint32_t tbase, int
     tmem_ld32(tbase + c, v);
     tmem_ld_wait();
     if (!row_ok) continue;
-    if (MODE == OUT_F32 || MODE == OUT_COMBINE) {
+    if (MODE == OUT_COMBINE_BF16) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        pk[j] = pack_bf16x2(scale * __uint_as_float(v[2 * j]), scale * __uint_as_float(v[2 * j + 1]));
+      uint16_t* dst = static_cast<uint16_t*>(a.out) + oidx + c;  // 64-byte aligned
+      st_global_v8(dst, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+      st_global_v8(dst + 16, pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14], pk[15]);
+    } else if (MODE == OUT_F32 || MODE == OUT_COMBINE) {
       float* dst = static_cast<float*>(a.out) + oidx + c;  // 128-byte aligned
       if (MODE == OUT_COMBINE) {
 #pragma unroll
@@ -428,9 +437,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int q = warp & 3;               // TMEM lane quarter this warp may read
     const int sub = (warp - 2) >> 2;      // which 32-column chunks: sub*32 + 128*i
     const int mode = a.out_mode * 3 + a.act;
-    if (a.out_mode == OUT_COMBINE) {
+    const bool combine = a.out_mode == OUT_COMBINE || a.out_mode == OUT_COMBINE_BF16;
+    if (combine) {
       // y = 0 for tokens whose only assignment was dropped (no tile writes them); done
       // while the first tile's operands stream in
+      const int row_vec = a.out_mode == OUT_COMBINE ? a.N / 4 : a.N / 8;  // 16-byte vectors
       const int ew = warp - 2;
       const int64_t gstride = static_cast<int64_t>(gridDim.x) * EPI_WARPS * 32;
       for (int64_t b = (static_cast<int64_t>(blockIdx.x) * EPI_WARPS + ew) * 32; b < a.rows_cap;
@@ -440,8 +451,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         while (m) {
           const int j = __ffs(m) - 1;
           m &= m - 1;
-          float4* row = reinterpret_cast<float4*>(static_cast<float*>(a.out) + (b + j) * a.N);
-          for (int v = lane; v < a.N / 4; v += 32) row[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+          float4* row = reinterpret_cast<float4*>(static_cast<uint8_t*>(a.out) + (b + j) * row_vec * 16);
+          for (int v = lane; v < row_vec; v += 32) row[v] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
     }
@@ -461,7 +472,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool row_ok = crow < t.valid;
       int64_t orow = t.row0 + crow;
       float scale = 1.0f;
-      if (a.out_mode == OUT_COMBINE && row_ok) {
+      if (combine && row_ok) {
         // k = 1: the permuted row's assignment is its token; y[t] = g_t * (h W2^T)[row]
         const int asg = __ldg(a.perm_src + orow);
         if (asg < 0 || asg >= a.rows_cap) {
@@ -482,6 +493,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           case OUT_F16 * 3 + 1: epilogue_rows<OUT_F16, 1>(a, tbase, oidx, sub, row_ok, scale); break;
           case OUT_F16 * 3 + 2: epilogue_rows<OUT_F16, 2>(a, tbase, oidx, sub, row_ok, scale); break;
           case OUT_COMBINE * 3 + 0: epilogue_rows<OUT_COMBINE, 0>(a, tbase, oidx, sub, row_ok, scale); break;
+          case OUT_COMBINE_BF16 * 3 + 0: epilogue_rows<OUT_COMBINE_BF16, 0>(a, tbase, oidx, sub, row_ok, scale); break;
           default: epilogue_rows<OUT_F32, 0>(a, tbase, oidx, sub, row_ok, scale); break;
         }
       }
@@ -657,14 +669,15 @@ static cudaError_t launch_up(const FfnProblem& p, const LaunchCtx& c) {
 }
 
 cudaError_t launch_ffn_combine_bf16(const FfnProblem& p, const int32_t* perm_src,
-                                    const int32_t* slot_pos, const float* gate, float* y,
+                                    const int32_t* slot_pos, const float* gate, void* y,
                                     const LaunchCtx& c) {
   if (p.E > gg::MAX_GROUPS) return cudaErrorInvalidValue;
   const int hf = p.hidden_f16 ? 1 : 0;
   cudaError_t e = launch_up(p, c);
   if (e != cudaSuccess) return e;
-  return launch_one(p.h, p.rows_cap, p.f, p.w2, p.E, p.d, hf, y, gg::OUT_COMBINE, p.offsets, 0, c,
-                    perm_src, gate, slot_pos);
+  return launch_one(p.h, p.rows_cap, p.f, p.w2, p.E, p.d, hf, y,
+                    p.y_bf16 ? gg::OUT_COMBINE_BF16 : gg::OUT_COMBINE, p.offsets, 0, c, perm_src,
+                    gate, slot_pos);
 }
 
 cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c) {

@@ -164,13 +164,15 @@ struct FfnProblem {
   const void* w2;
   void* h;
   void* y_perm;
+  int y_bf16 = 0;  // fused combine (k = 1): y in bf16
 };
 cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c);
 cudaError_t launch_ffn_f32(const FfnProblem& p, const LaunchCtx& c);
 // k = 1, bf16: expert FFN whose down-projection writes y[t] = gate[t] * row directly (its
-// epilogue also zeroes the rows of dropped tokens) instead of y_perm.
+// epilogue also zeroes the rows of dropped tokens) instead of y_perm; y in fp32, or bf16
+// with p.y_bf16.
 cudaError_t launch_ffn_combine_bf16(const FfnProblem& p, const int32_t* perm_src,
-                                    const int32_t* slot_pos, const float* gate, float* y,
+                                    const int32_t* slot_pos, const float* gate, void* y,
                                     const LaunchCtx& c);
 
 // fp32 SIMT grouped product out[r, n] = act(sum_k A'[r, k] B_g[n, k]) for the rows r of
@@ -189,6 +191,7 @@ struct CombineProblem {
   const int32_t* slot_pos;
   const float* gate;
   void* y;
+  int y_bf16 = 0;  // y in bf16 (each fp32 sum rounded once), else fp32
 };
 cudaError_t launch_combine(const CombineProblem& p, const LaunchCtx& c);
 

@@ -42,6 +42,8 @@ moe_status check_config(const moe_config* c) {
   if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (!(c->capacity_factor == c->capacity_factor)) return MOE_ERR_INVALID_ARG;  // NaN
   if (c->hidden_f16 != 0 && c->hidden_f16 != 1) return MOE_ERR_INVALID_ARG;
+  if (c->y_bf16 != 0 && c->y_bf16 != 1) return MOE_ERR_INVALID_ARG;
+  if (c->y_bf16 != 0 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (c->k > 8) return MOE_ERR_UNSUPPORTED;
   if (c->T * static_cast<int64_t>(c->k) >= (int64_t{1} << 31)) return MOE_ERR_UNSUPPORTED;
   if (c->T * static_cast<int64_t>(c->E) >= (int64_t{1} << 31)) return MOE_ERR_UNSUPPORTED;
@@ -349,6 +351,7 @@ moe_status do_combine(const moe_config* cfg, const void* y_perm, const int32_t* 
   p.slot_pos = slot_pos;
   p.gate = gate;
   p.y = y;
+  p.y_bf16 = cfg->y_bf16;
   return launch_combine(p, ctx.lc) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -373,7 +376,8 @@ moe_status do_ffn_combine(const moe_config* cfg, const void* x_perm, const int32
   p.w2 = w2;
   p.h = h;
   p.y_perm = nullptr;
-  cudaError_t e = launch_ffn_combine_bf16(p, perm_src, slot_pos, gate, static_cast<float*>(y), ctx.lc);
+  p.y_bf16 = cfg->y_bf16;
+  cudaError_t e = launch_ffn_combine_bf16(p, perm_src, slot_pos, gate, y, ctx.lc);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

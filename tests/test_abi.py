@@ -39,13 +39,14 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_config_struct_layout():
-    # int64 T, six int32, float, five int32 -> 56 bytes with 8-byte alignment
-    assert ctypes.sizeof(moe.MoEConfig) == 56
+    # int64 T, six int32, float, six int32 -> 60 bytes, 64 with 8-byte alignment
+    assert ctypes.sizeof(moe.MoEConfig) == 64
     assert moe.MoEConfig.capacity_factor.offset == 32
     assert moe.MoEConfig.dtype.offset == 40
     assert moe.MoEConfig.hidden_f16.offset == 44
     assert moe.MoEConfig.groups.offset == 48
     assert moe.MoEConfig.k_primary.offset == 52
+    assert moe.MoEConfig.y_bf16.offset == 56
 
 
 def test_status_strings():
@@ -97,6 +98,10 @@ def test_route_validation():
     assert _route(bad) == 1
     bad = _cfg()
     bad.act = 5
+    assert _route(bad) == 1
+    assert _route(_cfg(y_bf16=True, dtype="f32")) == 1      # bf16 output of an fp32 layer
+    bad = _cfg()
+    bad.y_bf16 = 2
     assert _route(bad) == 1
     bad = _cfg()
     bad.T = -1

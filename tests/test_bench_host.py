@@ -78,6 +78,12 @@ def test_algorithmic_counts_switch():
     assert a["ffn_bytes"] == weights + 16384 * 768 * 2 + 16384 * 768 * 4
     assert a["permute_bytes"] == 16384 * 12 + 128 * 8 + 16384 * 768 * 2 * 2
     assert a["route_bytes"] == 16384 * 768 * 2 + 128 * 768 * 2 + 16384 * 8
+    # a bf16 layer's output y is bf16 in the benchmark: 2 bytes per value written
+    assert bench.y_bf16_of(w) and not bench.y_bf16_of(workloads.WORKLOADS["tiny"])
+    assert a["combine_bytes"] == 16384 * 768 * 4 + 16384 * 8 + 16384 * 768 * 2
+    f = bench.algorithmic(w, 16384, kept, fused=True)
+    assert f["combine_bytes"] == 0.0
+    assert f["ffn_bytes"] == weights + 16384 * 768 * 2 + 16384 * 768 * 2 + 16384 * 8 + 16384 * 4
 
 
 def test_reference_arm_json_line():

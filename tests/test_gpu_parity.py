@@ -315,6 +315,45 @@ def test_permute_launch_path(name, launches):
     assert moe.moe_get_error(ws) == 0
 
 
+Y_BF16 = {
+    # k = 2 through the combine kernel, several tiles with a ragged tail
+    "combine_k2": Workload("yk2", T=1000, d_model=256, d_ff=512, E=8, k=2, act="gelu"),
+    # k = 1 through the fused down-projection epilogue, with dropped tokens (zero rows)
+    "fused_k1_drops": Workload("yk1", T=1500, d_model=256, d_ff=512, E=8, k=1, renorm=False,
+                               capacity_factor=0.9, act="gelu"),
+    "noisy_k4": W["noisy"].scaled(T=700),
+    "zipf_full": W["zipf"],
+    "switch_full": W["switch"],
+}
+
+
+@pytest.mark.parametrize("name", list(Y_BF16))
+def test_bf16_output_is_the_rounded_fp32_output(name):
+    """With y_bf16 the layer output is the fp32 output rounded once to bf16 (nearest even),
+    bit for bit: on the combine kernel (k >= 2) and on the fused down-projection epilogue
+    (k = 1), whose dropped tokens' rows are zero.  So it inherits the fp32 output's parity
+    with the oracle, plus one bf16 rounding (<= 2^-9 relative)."""
+    import sparsely_gated_mixture_moe_b200 as moe
+    w = Y_BF16[name]
+    dev = H.to_device(workloads.make_inputs(w))
+    weights = {kk: v for kk, v in dev.items() if kk not in ("x", "noise")}
+    cfg32 = H.config_of(w)
+    cfg16 = H.config_of(w)
+    cfg16.y_bf16 = 1
+    l32 = moe.MoELayer(cfg32, weights)
+    y32 = l32.forward(dev["x"], noise=dev.get("noise")).clone()
+    del l32
+    l16 = moe.MoELayer(cfg16, weights)
+    y16 = l16.forward(dev["x"], noise=dev.get("noise"))
+    torch.cuda.synchronize()
+    assert y16.dtype == torch.bfloat16
+    assert moe.moe_get_error(l16.ws) == 0
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+    if name == "fused_k1_drops":  # some expert overflows its capacity: zero rows exist
+        assert int(l16.counts.max()) > moe.moe_capacity(cfg16)
+        assert bool((y16.float().abs().sum(1) == 0).any())
+
+
 def test_forward_replays_from_a_cuda_graph():
     """moe_forward captured into a CUDA graph (its kernels and their programmatic launch
     edges) and replayed gives the eager result bit for bit, also after the input changes
