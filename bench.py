@@ -163,10 +163,18 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# The layer output y is fp32 in every benchmark figure: the workloads' bar (max|err| /
+# RMS <= 2e-2 for bf16 layers) leaves no room for a bf16 rounding of y (on the Switch
+# workload that rounding alone exceeds it).  --y-bf16 times the bf16-output option of
+# the library instead (for callers that round y to bf16 anyway); such a line is labelled
+# in its config and is not a figure for these workloads.
+Y_BF16 = False
+
+
 def y_bf16_of(w: workloads.Workload) -> bool:
-    """The benchmark's layer output type: bf16 for a bf16 layer (each row's fp32 sum
-    rounded once), fp32 for an fp32 layer."""
-    return w.dtype == "bf16"
+    """Whether the benchmark runs the layer with a bf16 output y (bf16 layers under
+    --y-bf16 only)."""
+    return Y_BF16 and w.dtype == "bf16"
 
 
 def algorithmic(w: workloads.Workload, n_kept: int, counts_kept, fused=False):
@@ -771,10 +779,15 @@ def main(argv=None):
                     help="time only the headline workload")
     ap.add_argument("--no-training", action="store_true",
                     help="skip the training-step (forward + backward) figure")
+    ap.add_argument("--y-bf16", action="store_true",
+                    help="layer output y in bf16 for bf16 layers (outside these workloads' "
+                         "error bar; not a benchmark figure)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="run the workload with this many tokens instead of its own T (small "
                          "cases for profiler captures; not a benchmark figure)")
     args = ap.parse_args(argv)
+    global Y_BF16
+    Y_BF16 = bool(args.y_bf16)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = workloads.WORKLOADS[args.workload]

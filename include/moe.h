@@ -134,7 +134,9 @@ typedef struct {
                              k / k_primary <= E / groups); else ignored */
   int32_t y_bf16;         /* bf16 only, 0 or 1: 1 writes the layer output y in bf16, each
                              row's fp32 sum rounded once to nearest even (y_perm stays
-                             fp32); 0 writes y in fp32 */
+                             fp32; the rounding adds up to 2^-9 relative per value, which
+                             a max|err|/RMS bar of 2e-2 does not absorb when a few outputs
+                             are many times the RMS); 0 writes y in fp32 */
 } moe_config;
 
 /* Human-readable name of a status code (static string). */

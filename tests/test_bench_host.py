@@ -78,12 +78,19 @@ def test_algorithmic_counts_switch():
     assert a["ffn_bytes"] == weights + 16384 * 768 * 2 + 16384 * 768 * 4
     assert a["permute_bytes"] == 16384 * 12 + 128 * 8 + 16384 * 768 * 2 * 2
     assert a["route_bytes"] == 16384 * 768 * 2 + 128 * 768 * 2 + 16384 * 8
-    # a bf16 layer's output y is bf16 in the benchmark: 2 bytes per value written
-    assert bench.y_bf16_of(w) and not bench.y_bf16_of(workloads.WORKLOADS["tiny"])
-    assert a["combine_bytes"] == 16384 * 768 * 4 + 16384 * 8 + 16384 * 768 * 2
+    # y is fp32 in the benchmark figures (4 bytes per value written) unless --y-bf16
+    assert not bench.y_bf16_of(w)
+    assert a["combine_bytes"] == 16384 * 768 * 4 + 16384 * 8 + 16384 * 768 * 4
     f = bench.algorithmic(w, 16384, kept, fused=True)
     assert f["combine_bytes"] == 0.0
-    assert f["ffn_bytes"] == weights + 16384 * 768 * 2 + 16384 * 768 * 2 + 16384 * 8 + 16384 * 4
+    assert f["ffn_bytes"] == weights + 16384 * 768 * 2 + 16384 * 768 * 4 + 16384 * 8 + 16384 * 4
+    bench.Y_BF16 = True
+    try:
+        assert bench.y_bf16_of(w) and not bench.y_bf16_of(workloads.WORKLOADS["tiny"])
+        b16 = bench.algorithmic(w, 16384, kept)
+        assert b16["combine_bytes"] == 16384 * 768 * 4 + 16384 * 8 + 16384 * 768 * 2
+    finally:
+        bench.Y_BF16 = False
 
 
 def test_reference_arm_json_line():
