@@ -339,16 +339,21 @@ class LayerBench:
         self.stream = torch.cuda.current_stream(dev)
         self.launches = 0
 
+    def route(self):
+        moe, d, o = self.moe, self.d, self.o
+        moe.moe_route(self.cfg, d["x"], d["w_gate"], o["idx"], o["gate"], self.ws,
+                      w_noise=d.get("w_noise"), noise=d.get("noise"),
+                      logit_bias=d.get("logit_bias"), importance=o["importance"], load=o["load"],
+                      near_tie=o["near"])
+        return moe.last_launch_count()
+
     def step(self, evs=None):
         """Route, permute, expert FFN, combine; events (if given) between the calls."""
         moe, d, o, cfg, st = self.moe, self.d, self.o, self.cfg, self.stream
         n = 0
         if evs:
             evs[0].record(st)
-        moe.moe_route(cfg, d["x"], d["w_gate"], o["idx"], o["gate"], self.ws, w_noise=d.get("w_noise"),
-                      noise=d.get("noise"), logit_bias=d.get("logit_bias"),
-                      importance=o["importance"], load=o["load"], near_tie=o["near"])
-        n += moe.last_launch_count()
+        n += self.route()
         if evs:
             evs[1].record(st)
         moe.moe_permute(cfg, o["idx"], d["x"], o["counts"], o["offsets"], o["perm_src"],
@@ -698,6 +703,7 @@ def run_gpu(args, w):
                       "note": "one step (route, permute, expert FFN, combine) captured once and "
                               "replayed; L2 flushed before each replay"}
     e2e = end_to_end(lb, flush, args.steps, world, dev, stream)
+    floor = launch_floor(lb, flush, dev, stream)
     train = training_step(lb, flush, args.steps, world, dev, stream) if not args.no_training else None
 
     eg = main["expert_gemm"]
@@ -728,7 +734,8 @@ def run_gpu(args, w):
         "roofline": roof,
     }
     line.update({kk: v for kk, v in main.items() if kk not in ("value", "unit", "ms_per_step")})
-    line.update({"e2e": e2e, "graph": graph_info, "gpu_launches": timed_launches, "clocks": clocks})
+    line.update({"e2e": e2e, "graph": graph_info, "gpu_launches": timed_launches, "clocks": clocks,
+                 "launch_floor": floor})
     if train is not None:
         line["training_step"] = train
     inp_main = lb.inp
@@ -765,6 +772,39 @@ def run_gpu(args, w):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def launch_floor(lb, flush, dev, stream, reps=20):
+    """What one launch costs on its own in the step breakdown: event-to-event time of a
+    trivial kernel (a one-value fill) with the host ahead of the GPU, and of the router
+    alone, against the router's time per launch when 20 run back to back (their launch
+    latencies then overlap the previous kernels).  Medians over `reps`, L2 flushed first."""
+    small = torch.zeros(1, device=dev)
+
+    def timed(fn):
+        ts = []
+        for i in range(reps + 3):
+            flush(i)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            if i >= 3:
+                ts.append(a.elapsed_time(b) * 1e3)
+        return float(np.median(ts))
+
+    trivial = timed(lambda: small.fill_(1.0))
+    route = timed(lb.route)
+
+    def twenty():
+        for _ in range(20):
+            lb.route()
+
+    b2b = timed(twenty) / 20.0
+    return {"trivial_kernel_us": trivial, "route_us": route, "route_back_to_back_us": b2b,
+            "note": "event-to-event times with the host ahead of the GPU; a single launch "
+                    "measures at least trivial_kernel_us here, whatever its bytes"}
 
 
 def main(argv=None):
