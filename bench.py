@@ -781,10 +781,12 @@ def launch_floor(lb, flush, dev, stream, reps=20):
     latencies then overlap the previous kernels).  Medians over `reps`, L2 flushed first."""
     small = torch.zeros(1, device=dev)
 
-    def timed(fn):
+    def timed(fn, pre=None):
         ts = []
         for i in range(reps + 3):
             flush(i)
+            if pre is not None:
+                pre()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             fn()
@@ -801,7 +803,9 @@ def launch_floor(lb, flush, dev, stream, reps=20):
         for _ in range(20):
             lb.route()
 
-    b2b = timed(twenty) / 20.0
+    # a longer GPU-side wait before the first event, so that the host has queued all
+    # twenty calls (about 25 us of host time each) before the GPU reaches them
+    b2b = timed(twenty, pre=lambda: torch.cuda._sleep(4 * HOST_AHEAD_CYCLES)) / 20.0
     return {"trivial_kernel_us": trivial, "route_us": route, "route_back_to_back_us": b2b,
             "note": "event-to-event times with the host ahead of the GPU; a single launch "
                     "measures at least trivial_kernel_us here, whatever its bytes"}

@@ -858,13 +858,17 @@ __global__ void __launch_bounds__(128, 1)
 
 // Importance and Load partial sums of noisy gating from the gate's per-token values:
 // block (chunk, eb) covers a run of tokens and experts 8*eb .. 8*eb+7, one per warp; the
-// lanes take the run's tokens 32 at a time.  For token t and expert e:
+// lanes take the run's tokens 32 at a time, four such groups per step with every load of
+// the step issued before any arithmetic (the kernel is bound by load latency, not bytes).
+// For token t and expert e:
 //   Importance term: the gate of e if e is one of t's chosen experts, else 0
 //   Load term: P(t, e) = Phi((l_te - kth_excluding(H_t, k, e)) / Softplus(z_te)), where
 //   kth_excluding is the (k+1)-th largest score when H_te >= the k-th largest, else the
 //   k-th largest (H_te as the gate formed it, so H >= the k-th means "among the top k").
-// Each warp's lanes are summed in a fixed butterfly order into partials[chunk][2][E], so
-// the result does not depend on scheduling.
+// Each lane adds its tokens in increasing order and the warp's lanes are then summed in
+// a fixed butterfly order into partials[chunk][2][E], so the result does not depend on
+// scheduling.
+constexpr int kIlGroups = 4;  // 32-token groups per lane step
 __global__ void __launch_bounds__(256)
     importance_load_kernel(const float* __restrict__ lw, const float* __restrict__ sw,
                            const float* __restrict__ hw, const float* __restrict__ kw,
@@ -879,16 +883,34 @@ __global__ void __launch_bounds__(256)
   const int64_t t_lo = static_cast<int64_t>(blockIdx.x) * chunk_tokens;
   const int64_t t_hi = min(T, t_lo + chunk_tokens);
   float si = 0.0f, sl = 0.0f;
-  for (int64_t t = t_lo + lane; t < t_hi; t += 32) {
-    float gi = 0.0f;
-    for (int j = 0; j < k; ++j)
-      if (__ldg(topk_idx + t * k + j) == e) gi = __ldg(topk_gate + t * k + j);
-    si += gi;
-    if (want_load) {
-      const int64_t i = static_cast<int64_t>(e) * T + t;
-      const float li = __ldg(lw + i), sp = __ldg(sw + i), H = __ldg(hw + i);
-      const float ex = (H >= __ldg(kw + t)) ? __ldg(kw + T + t) : __ldg(kw + t);
-      sl += 0.5f + 0.5f * erf_as7126(__fdividef(li - ex, sp) * 0.70710678118654752f);
+  for (int64_t t0 = t_lo + lane; t0 < t_hi; t0 += 32 * kIlGroups) {
+    float gi[kIlGroups], li[kIlGroups], sp[kIlGroups], H[kIlGroups], k0[kIlGroups], k1[kIlGroups];
+#pragma unroll
+    for (int u = 0; u < kIlGroups; ++u) {
+      const int64_t t = t0 + 32 * u;
+      gi[u] = 0.0f;
+      li[u] = sp[u] = H[u] = k0[u] = k1[u] = 0.0f;
+      if (t < t_hi) {
+        for (int j = 0; j < k; ++j)
+          if (__ldg(topk_idx + t * k + j) == e) gi[u] = __ldg(topk_gate + t * k + j);
+        if (want_load) {
+          const int64_t i = static_cast<int64_t>(e) * T + t;
+          li[u] = __ldg(lw + i);
+          sp[u] = __ldg(sw + i);
+          H[u] = __ldg(hw + i);
+          k0[u] = __ldg(kw + t);
+          k1[u] = __ldg(kw + T + t);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kIlGroups; ++u) {
+      if (t0 + 32 * u >= t_hi) break;
+      si += gi[u];
+      if (want_load) {
+        const float ex = (H[u] >= k0[u]) ? k1[u] : k0[u];
+        sl += 0.5f + 0.5f * erf_as7126(__fdividef(li[u] - ex, sp[u]) * 0.70710678118654752f);
+      }
     }
   }
 #pragma unroll
@@ -979,14 +1001,17 @@ static cudaError_t launch_route_tc_hier(int kg, const CUtensorMap& tmX, const CU
 // order total over the chunks.
 static cudaError_t launch_importance_load(const RouteProblem& p, const LaunchCtx& c) {
   const int eb = (p.E + 7) / 8;
-  // about four blocks per SM; chunks of whole 32-token groups, at most one chunk per 64
-  // tokens (the partials' rows)
-  int64_t chunks = (4LL * c.num_sms + eb - 1) / eb;
+  // one lane step per chunk where the grid stays within about eight blocks per SM (a
+  // 128-token chunk: each lane's four tokens), longer chunks of whole 128-token steps
+  // beyond; at most one chunk per 64 tokens (the partials' rows)
+  int64_t chunks = (p.T + 32 * kIlGroups - 1) / (32 * kIlGroups);
+  const int64_t most = (8LL * c.num_sms + eb - 1) / eb;
+  if (chunks > most) chunks = most;
   const int64_t cap = route_blocks(p.T);
   if (chunks > cap) chunks = cap;
   if (chunks < 1) chunks = 1;
   int64_t per = (p.T + chunks - 1) / chunks;
-  per = (per + 31) / 32 * 32;
+  per = (per + 32 * kIlGroups - 1) / (32 * kIlGroups) * (32 * kIlGroups);
   chunks = (p.T + per - 1) / per;
   cudaError_t e = launch_kernel(importance_load_kernel, dim3(static_cast<unsigned>(chunks), eb),
                                 dim3(256), 0, c, static_cast<const float*>(p.lw),
