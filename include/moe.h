@@ -209,6 +209,26 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32
                           const void* w1, const void* w2, void* h, void* y_perm, void* ws,
                           moe_stream_t stream);
 
+/* The expert FFN over row groups that share weight blocks: group g (0 <= g < groups) is
+ * rows [offsets[g], offsets[g+1]) of x_rows and runs expert g mod E of w1/w2 (E =
+ * cfg->E weight blocks).  With the rows that R source ranks sent to this rank's E
+ * experts laid out source by source, each source's rows by expert (groups = R E), this is
+ * the expert computation of an expert-parallel layer [Shazeer et al., "Kombinierte Daten-
+ * und Modellparallelität": each device holds some experts and receives, from every
+ * device, the tokens routed to them].  Arithmetic as moe_expert_ffn (bf16 only).
+ *  x_rows   [rows_cap, d_model] bf16 in;  offsets [groups+1] int32 in, non-decreasing in
+ *           [0, rows_cap] (else MOE_DEVERR_OFFSETS and no output)
+ *  w1 [E, d_ff, d_model], w2 [E, d_model, d_ff] (fp16 with cfg->hidden_f16)
+ *  h        [rows_cap, d_ff] out;  y_rows [rows_cap, d_model] fp32 out (rows below
+ *           offsets[groups] written)
+ *  ws       at least moe_workspace_size(cfg) bytes (its device error word is used)
+ * cfg->T and cfg->k are not used.  groups <= 1024 and rows_cap < 2^31 (else
+ * MOE_ERR_UNSUPPORTED); rows_cap == 0 launches nothing. */
+moe_status moe_expert_ffn_grouped(const moe_config* cfg, const void* x_rows, int64_t rows_cap,
+                                  const int32_t* offsets, int32_t groups, const void* w1,
+                                  const void* w2, void* h, void* y_rows, void* ws,
+                                  moe_stream_t stream);
+
 /* moe_expert_ffn with the permuted rows gathered from the token rows instead of read
  * from x_perm [Switch Transformer, switch_routing: dispatch is a gather of each expert's
  * tokens]: permuted row s is x[perm_src[s] / k], fetched by the up-projection's tensor

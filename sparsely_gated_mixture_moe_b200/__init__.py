@@ -16,7 +16,7 @@ from typing import Optional
 
 import torch
 
-from .config import (ACT, DTYPE, GATING, MoEConfig, MoEError, STATUS, make_config)
+from .config import (ACT, DEVERR, DTYPE, GATING, MoEConfig, MoEError, STATUS, make_config)
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 
@@ -48,6 +48,8 @@ def _load():
         "moe_permute_noalloc": (ctypes.c_int, [C, P, P, P, P, P, P, P, P]),
         "moe_erf_check": (ctypes.c_int, [P, P, P, ctypes.c_int64, P]),
         "moe_gelu_check": (ctypes.c_int, [P, P, P, ctypes.c_int64, P]),
+        "moe_expert_ffn_grouped": (ctypes.c_int, [C, P, ctypes.c_int64, P, ctypes.c_int32, P, P, P, P,
+                                                  P, P]),
         "moe_train_state_size": (ctypes.c_size_t, [C]),
         "moe_backward_workspace_size": (ctypes.c_size_t, [C]),
         "moe_forward_train": (ctypes.c_int, [C] + [P] * 17),
@@ -144,6 +146,17 @@ def moe_expert_ffn(cfg, x_perm, offsets, w1, w2, h, y_perm, ws, stream=None):
                               _ptr(w1, "w1"), _ptr(w2, "w2"), _ptr(h, "h"),
                               _ptr(y_perm, "y_perm"), _ptr(ws, "ws"), _stream(stream)),
            "moe_expert_ffn")
+
+
+def moe_expert_ffn_grouped(cfg, x_rows, offsets, groups, w1, w2, h, y_rows, ws, stream=None):
+    """moe_expert_ffn over `groups` row groups, group g running expert g % cfg.E (the rows
+    an expert-parallel rank receives, source by source); x_rows' first dimension is the
+    row capacity."""
+    _check(lib.moe_expert_ffn_grouped(ctypes.byref(cfg), _ptr(x_rows, "x_rows"),
+                                      int(x_rows.shape[0]), _ptr(offsets, "offsets"), int(groups),
+                                      _ptr(w1, "w1"), _ptr(w2, "w2"), _ptr(h, "h"),
+                                      _ptr(y_rows, "y_rows"), _ptr(ws, "ws"), _stream(stream)),
+           "moe_expert_ffn_grouped")
 
 
 def moe_expert_ffn_gather(cfg, x, perm_src, offsets, w1, w2, h, y_perm, ws, stream=None):
@@ -310,10 +323,11 @@ class MoELayer:
         return self.y
 
 
-__all__ = ["ACT", "DTYPE", "GATING", "MoEConfig", "MoEError", "MoELayer", "STATUS", "lib",
+__all__ = ["ACT", "DEVERR", "DTYPE", "GATING", "MoEConfig", "MoEError", "MoELayer", "STATUS", "lib",
            "make_config", "moe_capacity", "moe_combine", "moe_expert_ffn", "moe_forward",
            "moe_forward_workspace_size", "moe_get_error", "moe_permute", "moe_route",
            "moe_workspace_size", "workspace", "last_launch_count", "moe_bf16_to_f16",
+           "moe_expert_ffn_grouped",
            "prepare_weights", "moe_permute_noalloc", "moe_expert_ffn_combine", "fused_combine",
            "moe_expert_ffn_gather", "moe_expert_ffn_combine_gather", "train_state",
            "backward_workspace", "moe_forward_train", "moe_backward"]

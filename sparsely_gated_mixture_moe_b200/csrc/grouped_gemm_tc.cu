@@ -89,6 +89,8 @@ struct Args {
   int gather_k;               // A tensor (the token rows x), gathered by the TMA itself
   void* pre;                  // OUT_BF16 / OUT_F16 with an activation: also store the
                               // pre-activation there (same type and layout as out), or null
+  int w_mod;                  // row group g multiplies weight block g % w_mod (w_mod >= E:
+                              // group g uses block g)
   int* err;
 };
 
@@ -285,7 +287,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         g2 = __ldg(a.gather_src + t.row0 + min(r + 2, last)) / a.gather_k;
         g3 = __ldg(a.gather_src + t.row0 + min(r + 3, last)) / a.gather_k;
       }
-      const int brow = t.e * a.N + t.nt * a.bn + static_cast<int>(rank) * b_rows;
+      const int brow = (t.e % a.w_mod) * a.N + t.nt * a.bn + static_cast<int>(rank) * b_rows;
       for (int kb = 0; kb < kblocks; ++kb) {
         int okw = 1;
         if (lane == 0) okw = mbar_wait(empty0 + 8 * stage, phase ^ 1, s_abort) ? 1 : 0;
@@ -333,7 +335,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool aborted = false;
       for (int L = first; L < total && !aborted; L += stride) {
         const Tile t = decode_tile(L, tp, a, TBM);
-        const int brow = t.e * a.N + t.nt * a.bn + static_cast<int>(rank) * b_rows;
+        const int brow = (t.e % a.w_mod) * a.N + t.nt * a.bn + static_cast<int>(rank) * b_rows;
         const int arow = t.row0 + static_cast<int>(rank) * BM;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, s_abort)) {
@@ -603,8 +605,9 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
                               const LaunchCtx& c, const int32_t* perm_src = nullptr,
                               const float* gate = nullptr, const int32_t* slot_pos = nullptr,
                               const int32_t* gather_src = nullptr, int gather_k = 1,
-                              int64_t a_rows = 0, void* pre = nullptr) {
+                              int64_t a_rows = 0, void* pre = nullptr, int w_count = 0) {
   const int bn = pick_bn(N);
+  const int wb = w_count > 0 ? w_count : E;  // weight blocks of B
   const bool pair = rows_cap >= kPairMinRowsPerExpert * E;
   CUtensorMap tmA, tmB;
   if (gather_src != nullptr) {
@@ -615,7 +618,7 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
     return cudaErrorInvalidValue;
   }
   // a pair's CTA loads half of each B tile
-  if (!make_tmap_2b(&tmB, B, static_cast<uint64_t>(E) * N, K, pair ? bn / 2 : bn, ab_f16))
+  if (!make_tmap_2b(&tmB, B, static_cast<uint64_t>(wb) * N, K, pair ? bn / 2 : bn, ab_f16))
     return cudaErrorInvalidValue;
   gg::Args a;
   a.offsets = offsets;
@@ -635,6 +638,7 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
   a.gather_src = gather_src;
   a.gather_k = gather_k;
   a.pre = pre;
+  a.w_mod = wb;
   a.err = c.err;
   // upper bound of the tile count: sum_e ceil(n_e / bm) <= rows_cap / bm + E
   const int tbm = pair ? 2 * gg::BM : gg::BM;
@@ -663,9 +667,9 @@ static cudaError_t launch_up(const FfnProblem& p, const LaunchCtx& c) {
   const int mode = hf ? gg::OUT_F16 : gg::OUT_BF16;
   if (p.gather_src != nullptr)
     return launch_one(p.x, p.rows_cap, p.d, p.w1, p.E, p.f, 0, p.h, mode, p.offsets, p.act, c,
-                      nullptr, nullptr, nullptr, p.gather_src, p.k, p.x_rows, p.u);
+                      nullptr, nullptr, nullptr, p.gather_src, p.k, p.x_rows, p.u, p.w_count);
   return launch_one(p.x_perm, p.rows_cap, p.d, p.w1, p.E, p.f, 0, p.h, mode, p.offsets, p.act, c,
-                    nullptr, nullptr, nullptr, nullptr, 1, 0, p.u);
+                    nullptr, nullptr, nullptr, nullptr, 1, 0, p.u, p.w_count);
 }
 
 cudaError_t launch_ffn_combine_bf16(const FfnProblem& p, const int32_t* perm_src,
@@ -685,7 +689,8 @@ cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c) {
   const int hf = p.hidden_f16 ? 1 : 0;
   cudaError_t e = launch_up(p, c);
   if (e != cudaSuccess) return e;
-  return launch_one(p.h, p.rows_cap, p.f, p.w2, p.E, p.d, hf, p.y_perm, gg::OUT_F32, p.offsets, 0, c);
+  return launch_one(p.h, p.rows_cap, p.f, p.w2, p.E, p.d, hf, p.y_perm, gg::OUT_F32, p.offsets, 0, c,
+                    nullptr, nullptr, nullptr, nullptr, 1, 0, nullptr, p.w_count);
 }
 
 }  // namespace moe

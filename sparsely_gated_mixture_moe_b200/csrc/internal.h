@@ -165,6 +165,7 @@ struct FfnProblem {
   void* h;
   void* y_perm;
   int y_bf16 = 0;  // fused combine (k = 1): y in bf16
+  int w_count = 0;  // > 0: E row groups over w_count weight blocks, group g using g % w_count
 };
 cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c);
 cudaError_t launch_ffn_f32(const FfnProblem& p, const LaunchCtx& c);

@@ -514,6 +514,44 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const int32
   return st == MOE_OK ? ctx.finish(cudaSuccess) : st;
 }
 
+moe_status moe_expert_ffn_grouped(const moe_config* cfg, const void* x_rows, int64_t rows_cap,
+                                  const int32_t* offsets, int32_t groups, const void* w1,
+                                  const void* w2, void* h, void* y_rows, void* ws,
+                                  moe_stream_t stream) {
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (rows_cap < 0 || groups <= 0) return MOE_ERR_INVALID_ARG;
+  if (groups > 1024 || rows_cap >= (int64_t{1} << 31)) return MOE_ERR_UNSUPPORTED;
+  if (rows_cap == 0) {
+    g_last_launches = 0;
+    return MOE_OK;
+  }
+  if (!x_rows || !offsets || !w1 || !w2 || !h || !y_rows || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_rows) || !aligned16(w1) || !aligned16(w2) || !aligned16(h) ||
+      !aligned16(y_rows) || !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  Ctx ctx(ws, stream);
+  if (!ctx.ok) return MOE_ERR_CUDA;
+  FfnProblem p;
+  p.x_rows = rows_cap;
+  p.rows_cap = rows_cap;
+  p.d = cfg->d_model;
+  p.f = cfg->d_ff;
+  p.E = groups;
+  p.w_count = cfg->E;
+  p.act = cfg->act == MOE_ACT_GELU ? 2 : 1;
+  p.hidden_f16 = cfg->hidden_f16;
+  p.x_perm = x_rows;
+  p.offsets = offsets;
+  p.w1 = w1;
+  p.w2 = w2;
+  p.h = h;
+  p.y_perm = y_rows;
+  const cudaError_t e = launch_ffn_bf16(p, ctx.lc);
+  return ctx.finish(e);
+}
+
 moe_status moe_expert_ffn_gather(const moe_config* cfg, const void* x, const int32_t* perm_src,
                                  const int32_t* offsets, const void* w1, const void* w2, void* h,
                                  void* y_perm, void* ws, moe_stream_t stream) {

@@ -31,6 +31,21 @@ def test_self_checks_validate_before_launching():
         assert fn(None, None, None, 0, None) == 0
 
 
+def test_grouped_ffn_validates_before_launching():
+    """moe_expert_ffn_grouped: fp32 layers are unsupported, groups must be positive and at
+    most 1024, and zero rows launch nothing (no GPU needed for any of these)."""
+    c = moe.make_config(64, 128, 128, 2, 1, dtype="bf16")
+    c32 = moe.make_config(64, 128, 128, 2, 1, dtype="f32")
+    f = moe.lib.moe_expert_ffn_grouped
+    assert f(ctypes.byref(c32), FAKE, 64, FAKE, 4, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 2
+    assert f(ctypes.byref(c), FAKE, 64, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f(ctypes.byref(c), FAKE, 64, FAKE, 1025, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 2
+    assert f(ctypes.byref(c), FAKE, -1, FAKE, 4, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f(ctypes.byref(c), FAKE, 0, None, 4, None, None, None, None, None, None) == 0
+    assert f(ctypes.byref(c), None, 64, FAKE, 4, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f(ctypes.byref(c), FAKE_ODD, 64, FAKE, 4, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+
+
 def test_library_exports_every_declared_symbol():
     names = _declared_functions()
     assert len(names) >= 11
