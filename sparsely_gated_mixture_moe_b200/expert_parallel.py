@@ -8,22 +8,23 @@ receives, from every device, the examples routed to them].
 One rank's forward pass:
   1. moe_route and moe_permute on its T tokens (all E experts; capacity per rank, each
      rank's batch being one group for the capacity rule);
-  2. the kept rows, already ordered by expert and so by the rank that holds the expert
-     (rank r holds experts [r E/R, (r+1) E/R)), go out with one all-to-all; a first
-     all-to-all of the per-expert row counts tells every rank what it receives;
-  3. moe_expert_ffn_grouped runs the received rows, source by source, each source's rows
-     expert by expert (group g = source * E/R + local expert, weights g mod E/R);
-  4. the expert outputs return with the reverse all-to-all into the sender's permuted
-     order, and moe_combine forms y from them as on one device.
+  2. the kept rows are already ordered by expert, and so by the rank that holds the
+     expert (rank r holds experts [r E/R, (r+1) E/R)); an all-to-all of the per-expert row
+     counts tells every rank what it receives, then every (source, expert) run of rows
+     travels as its own point-to-point message straight to its place in the receiver's
+     expert-major layout (expert by expert, each expert's rows source by source);
+  3. moe_expert_ffn_grouped runs the received rows with one group per local expert, so a
+     rank's expert step is the single-device expert FFN on the rows it holds;
+  4. every (source, expert) run of outputs returns the same way to the slot its rows came
+     from, and moe_combine forms y from them as on one device.
 
-The exchange helpers here are plain torch.distributed collectives on tensors of any
-device (NCCL between GPUs); the compute steps are libmoe's kernels.  This is the NCCL
-form of the exchange: the rows cross the links in two collective calls around the expert
-products rather than inside them.
+The exchange helpers here are plain torch.distributed collectives and point-to-point
+operations on tensors of any device (NCCL between GPUs); the compute steps are libmoe's
+kernels.  This is the NCCL form of the exchange: the rows cross the links in messages
+around the expert products rather than inside them.
 """
 from __future__ import annotations
 
-import ctypes
 from dataclasses import dataclass
 from typing import List, Optional
 
@@ -41,61 +42,114 @@ def local_expert_range(E: int, world: int, rank: int):
 
 @dataclass
 class ExchangePlan:
-    send_splits: List[int]     # rows this rank sends to each rank
-    recv_splits: List[int]     # rows this rank receives from each rank
-    recv_counts: torch.Tensor  # [world, E_local]: rows from source s for local expert e
-    group_offsets: torch.Tensor  # [world * E_local + 1] int32: row groups, source-major
+    send_counts: List[List[int]]  # [world][E_local]: rows sent to rank d for its expert e
+    recv_counts: List[List[int]]  # [world][E_local]: rows received from s for expert e
+    send_pos: List[List[int]]     # first row of each sent run in the sender's kept rows
+    recv_pos: List[List[int]]     # first row of each received run (expert-major layout)
+    expert_offsets: torch.Tensor  # [E_local + 1] int32: each local expert's received rows
 
     @property
     def rows_out(self) -> int:
-        return int(sum(self.send_splits))
+        return int(sum(sum(r) for r in self.send_counts))
 
     @property
     def rows_in(self) -> int:
-        return int(sum(self.recv_splits))
+        return int(sum(sum(r) for r in self.recv_counts))
+
+
+def _staged(t: torch.Tensor, group) -> bool:
+    """Device tensors go through host memory when the group's backend cannot move them
+    itself (gloo); NCCL moves them directly."""
+    return t.is_cuda and dist.is_initialized() and dist.get_backend(group) != "nccl"
 
 
 def exchange_plan(kept_per_expert: torch.Tensor, world: int, group=None) -> ExchangePlan:
     """Exchange the per-expert kept-row counts [E] (int, on the collective's device) and
-    derive the row splits of both all-to-alls and the receiver's group offsets.  The
-    split lists are read back to the host (the collectives take them as lists)."""
+    lay out both directions: each (rank, local expert) run's place in the sender's kept
+    rows (expert order) and in the receiver's expert-major layout.  The counts are read
+    back to the host once (the messages' sizes)."""
     E = int(kept_per_expert.numel())
     if E % world != 0:
         raise ValueError("E = %d experts do not split evenly over %d ranks" % (E, world))
-    send = kept_per_expert.to(torch.int64).reshape(world, E // world).contiguous()
-    recv = torch.empty_like(send)
+    El = E // world
+    send = kept_per_expert.to(torch.int64).reshape(world, El).contiguous()
     if world == 1:
-        recv.copy_(send)
+        recv = send.clone()
     else:
+        if _staged(send, group):
+            send = send.cpu()
+        recv = torch.empty_like(send)
         dist.all_to_all_single(recv, send, group=group)
-    send_splits = [int(v) for v in send.sum(dim=1).tolist()]
-    recv_splits = [int(v) for v in recv.sum(dim=1).tolist()]
-    offsets = torch.zeros(recv.numel() + 1, dtype=torch.int64, device=recv.device)
-    torch.cumsum(recv.reshape(-1), dim=0, out=offsets[1:])
-    return ExchangePlan(send_splits, recv_splits, recv, offsets.to(torch.int32))
+    sc = [[int(v) for v in row] for row in send.tolist()]
+    rc = [[int(v) for v in row] for row in recv.tolist()]
+    send_pos, p = [], 0
+    for d in range(world):
+        send_pos.append([])
+        for e in range(El):
+            send_pos[d].append(p)
+            p += sc[d][e]
+    recv_pos = [[0] * El for _ in range(world)]
+    eoff, p = [0], 0
+    for e in range(El):
+        for s_ in range(world):
+            recv_pos[s_][e] = p
+            p += rc[s_][e]
+        eoff.append(p)
+    offsets = torch.tensor(eoff, dtype=torch.int32, device=kept_per_expert.device)
+    return ExchangePlan(sc, rc, send_pos, recv_pos, offsets)
+
+
+def _exchange(src: torch.Tensor, dst: torch.Tensor, out_pos, out_counts, in_pos, in_counts,
+              group=None):
+    """Send run (d, e) = src[out_pos[d][e] : + out_counts[d][e]] to rank d and receive run
+    (s, e) into dst[in_pos[s][e] : + in_counts[s][e]], for every rank and local expert in
+    the same order on both sides; this rank's own runs are copied."""
+    world = len(out_counts)
+    rank = dist.get_rank(group) if world > 1 else 0
+    staged = world > 1 and _staged(src, group)
+    ops, landings = [], []
+    for peer in range(world):
+        for e in range(len(out_counts[peer])):
+            n_out, n_in = out_counts[peer][e], in_counts[peer][e]
+            if peer == rank:
+                if n_out:
+                    a, b = out_pos[peer][e], in_pos[peer][e]
+                    dst[b:b + n_out].copy_(src[a:a + n_out])
+                continue
+            if n_out:
+                a = out_pos[peer][e]
+                run = src[a:a + n_out]
+                run = run.cpu() if staged else run.contiguous()
+                ops.append(dist.P2POp(dist.isend, run, peer, group))
+            if n_in:
+                b = in_pos[peer][e]
+                if staged:
+                    buf = torch.empty((n_in,) + tuple(dst.shape[1:]), dtype=dst.dtype)
+                    landings.append((buf, b))
+                    ops.append(dist.P2POp(dist.irecv, buf, peer, group))
+                else:
+                    ops.append(dist.P2POp(dist.irecv, dst[b:b + n_in], peer, group))
+    if ops:
+        for req in dist.batch_isend_irecv(ops):
+            req.wait()
+    for buf, b in landings:
+        dst[b:b + buf.shape[0]].copy_(buf)
 
 
 def dispatch_rows(rows: torch.Tensor, plan: ExchangePlan, out: torch.Tensor, group=None):
-    """All-to-all of the kept rows [rows_out, d] (in expert order) into out[:rows_in]."""
-    dst = out[: plan.rows_in]
-    if len(plan.send_splits) == 1:
-        dst.copy_(rows[: plan.rows_out])
-    else:
-        dist.all_to_all_single(dst, rows[: plan.rows_out].contiguous(), plan.recv_splits,
-                               plan.send_splits, group=group)
-    return dst
+    """The kept rows [rows_out, d] (expert order) to the ranks holding their experts, into
+    out[:rows_in] in expert-major order."""
+    _exchange(rows, out, plan.send_pos, plan.send_counts, plan.recv_pos, plan.recv_counts,
+              group)
+    return out[: plan.rows_in]
 
 
 def return_rows(rows: torch.Tensor, plan: ExchangePlan, out: torch.Tensor, group=None):
-    """The reverse all-to-all: rows [rows_in, d] computed here go back to their senders,
-    into out[:rows_out] in the sender's original (expert) order."""
-    dst = out[: plan.rows_out]
-    if len(plan.send_splits) == 1:
-        dst.copy_(rows[: plan.rows_in])
-    else:
-        dist.all_to_all_single(dst, rows[: plan.rows_in].contiguous(), plan.send_splits,
-                               plan.recv_splits, group=group)
-    return dst
+    """The expert outputs [rows_in, d] back to their senders, into out[:rows_out] at the
+    places the rows left from."""
+    _exchange(rows, out, plan.recv_pos, plan.recv_counts, plan.send_pos, plan.send_counts,
+              group)
+    return out[: plan.rows_out]
 
 
 class ExpertParallelMoE:
@@ -155,9 +209,8 @@ class ExpertParallelMoE:
         self.plan = plan = exchange_plan(kept, self.world, self.group)
         recv = dispatch_rows(self.x_perm, plan, self.x_recv, self.group)
         del recv  # the grouped FFN reads x_recv by its row capacity
-        groups = self.world * self.E_local
-        moe.moe_expert_ffn_grouped(self.cfg_local, self.x_recv, plan.group_offsets, groups,
-                                   w["w1"], w["w2"], self.h, self.y_recv, self.ws)
+        moe.moe_expert_ffn_grouped(self.cfg_local, self.x_recv, plan.expert_offsets,
+                                   self.E_local, w["w1"], w["w2"], self.h, self.y_recv, self.ws)
         return_rows(self.y_recv, plan, self.y_back, self.group)
         moe.moe_combine(cfg, self.y_back, self.slot_pos, self.gate, self.y, self.ws)
         return self.y

@@ -1,10 +1,11 @@
 """Expert parallelism's exchange, on CPU with two gloo ranks (no GPU).
 
 Each rank routes its own batch with the oracle, sends its kept rows with the library's
-exchange helpers (`exchange_plan`, `dispatch_rows`, `return_rows`), runs the experts it
-holds on the rows it received with the oracle's expert function (group g = source * E/R
-+ local expert, weights g mod E/R, exactly the grouping moe_expert_ffn_grouped gets),
-sends the outputs back and combines them.  The result must equal the oracle's
+exchange helpers (`exchange_plan`, `dispatch_rows`, `return_rows`: one message per
+(rank, expert) run, landing expert-major), runs the experts it holds on the rows it
+received with the oracle's expert function (one group per local expert, as
+ExpertParallelMoE hands them to moe_expert_ffn_grouped), sends the outputs back and
+combines them.  The result must equal the oracle's
 single-device layer on the same rank's batch: every row reached the right expert and
 came back to the right slot.  The compute here is the oracle's; the kernels' side of the
 same grouping is tested on the GPU (tests/test_gpu_expert_parallel.py)."""
@@ -67,20 +68,20 @@ def _worker(rank, world, port, name, q):
         # what every rank sends to every other, gathered, so the plan can be checked
         all_kept = [torch.zeros_like(kept) for _ in range(world)]
         dist.all_gather(all_kept, kept)
-        want_recv = torch.stack([a.reshape(world, El)[rank] for a in all_kept])
-        assert torch.equal(plan.recv_counts, want_recv)
-        assert plan.send_splits == [int(v) for v in kept.reshape(world, El).sum(1)]
+        want_recv = [[int(v) for v in a.reshape(world, El)[rank]] for a in all_kept]
+        assert plan.recv_counts == want_recv
+        assert plan.send_counts == [[int(v) for v in row] for row in kept.reshape(world, El)]
         recv_buf = torch.zeros(world * T * k, w.d_model, dtype=torch.float64)
         recv = ep.dispatch_rows(x_perm, plan, recv_buf)
-        off = plan.group_offsets.numpy()
+        off = plan.expert_offsets.numpy()
         assert off[-1] == plan.rows_in == recv.shape[0]
         y_recv = torch.zeros(world * T * k, w.d_model, dtype=torch.float64)
         w1, w2 = inp["w1"], inp["w2"]
-        for g in range(world * El):
-            a, b = int(off[g]), int(off[g + 1])
+        for e in range(El):
+            a, b = int(off[e]), int(off[e + 1])
             if b > a:
-                e = e0 + g % El
-                y_recv[a:b] = torch.from_numpy(orc.expert(recv[a:b].numpy(), w1[e], w2[e], w.act)[1])
+                y_recv[a:b] = torch.from_numpy(orc.expert(recv[a:b].numpy(), w1[e0 + e], w2[e0 + e],
+                                                          w.act)[1])
         back = torch.zeros(int(offsets[-1]), w.d_model, dtype=torch.float64)
         ep.return_rows(y_recv, plan, back)
         y = orc.combine(back.numpy(), slot_pos, r["gates"], T, k)
@@ -117,5 +118,9 @@ def test_local_expert_range_and_plan_single_rank():
         ep.local_expert_range(6, 4, 0)
     kept = torch.tensor([3, 0, 5, 2])
     plan = ep.exchange_plan(kept, 1)
-    assert plan.send_splits == [10] and plan.recv_splits == [10]
-    assert plan.group_offsets.tolist() == [0, 3, 3, 8, 10]
+    assert plan.send_counts == [[3, 0, 5, 2]] and plan.recv_counts == [[3, 0, 5, 2]]
+    assert plan.send_pos == [[0, 3, 3, 8]] and plan.recv_pos == [[0, 3, 3, 8]]
+    assert plan.expert_offsets.tolist() == [0, 3, 3, 8, 10]
+    rows = torch.arange(10.0).reshape(10, 1)
+    out = torch.zeros(10, 1)
+    assert torch.equal(ep.dispatch_rows(rows, plan, out), rows)

@@ -8,8 +8,10 @@ and the tensor-core accumulation order over K does not depend on which other row
 the tile, so the grouped result must equal, row for row and bit for bit, moe_expert_ffn
 on the same rows regrouped expert by expert; sampled rows are also checked against the
 fp64 oracle.  ExpertParallelMoE on a single rank (no exchange) must give MoELayer's
-output bit for bit.  The multi-rank exchange itself is tested on CPU with gloo
-(tests/test_expert_parallel.py)."""
+output bit for bit, and so must each of two ranks run as two processes on this GPU,
+each holding half of the experts, exchanging their runs of rows through gloo (staged
+through host memory; every wait is on the host, no kernel waits for another process).
+The exchange alone is also tested on CPU (tests/test_expert_parallel.py)."""
 import numpy as np
 import pytest
 import torch
@@ -135,3 +137,61 @@ def test_expert_parallel_single_rank_equals_layer(name):
     assert moe.moe_get_error(epl.ws) == 0
     assert epl.world == 1 and epl.plan.rows_in == epl.plan.rows_out
     assert torch.equal(y, y_ref)
+
+
+EP_TWO_RANKS = {
+    "k2_gelu": Workload("ept2", T=1200, d_model=256, d_ff=512, E=8, k=2, act="gelu"),
+    "k1_capacity": Workload("ept1", T=1600, d_model=256, d_ff=512, E=16, k=1, renorm=False,
+                            capacity_factor=1.0, act="gelu"),
+    "noisy_k4": workloads.WORKLOADS["noisy"].scaled(T=700),
+}
+
+
+def _ep_rank(rank, world, port, name, q):
+    try:
+        import torch.distributed as dist
+        import sparsely_gated_mixture_moe_b200 as moe
+        from sparsely_gated_mixture_moe_b200.expert_parallel import (ExpertParallelMoE,
+                                                                     local_expert_range)
+        from tests.test_expert_parallel import _rank_inputs
+        torch.cuda.set_device(0)
+        dist.init_process_group("gloo", init_method="tcp://127.0.0.1:%d" % port, rank=rank,
+                                world_size=world)
+        w = EP_TWO_RANKS[name]
+        dev = H.to_device(_rank_inputs(w, rank))
+        full = {kk: v for kk, v in dev.items() if kk not in ("x", "noise")}
+        e0, e1 = local_expert_range(w.E, world, rank)
+        mine = dict(full, w1=full["w1"][e0:e1].contiguous(), w2=full["w2"][e0:e1].contiguous())
+        epl = ExpertParallelMoE(H.config_of(w), mine)
+        y = epl.forward(dev["x"], noise=dev.get("noise")).clone()
+        err = moe.moe_get_error(epl.ws)
+        layer = moe.MoELayer(H.config_of(w), full)
+        y_ref = layer.forward(dev["x"], noise=dev.get("noise"))
+        torch.cuda.synchronize()
+        sent_away = sum(sum(r) for i, r in enumerate(epl.plan.send_counts) if i != rank)
+        q.put((rank, err, bool(torch.equal(y, y_ref)), sent_away, None))
+        dist.barrier()
+        dist.destroy_process_group()
+    except Exception as exc:  # report to the parent instead of hanging it
+        q.put((rank, None, None, None, repr(exc)))
+
+
+@pytest.mark.parametrize("name", list(EP_TWO_RANKS))
+def test_expert_parallel_two_ranks_on_one_gpu(name):
+    import torch.multiprocessing as mp
+    from tests.test_expert_parallel import _free_port
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ep_rank, args=(r, world, port, name, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=300) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+    for rank, err, equal, sent_away, exc in results:
+        assert exc is None, (rank, exc)
+        assert err == 0, (rank, err)
+        assert sent_away > 0, rank   # rows really crossed to the other rank
+        assert equal, rank
