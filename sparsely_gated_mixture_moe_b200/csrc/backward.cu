@@ -51,6 +51,12 @@ constexpr int MAX_GROUPS = 1024;
 constexpr int TMEM_COLS = 512;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES_MAX;
 constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+// CTA pairs (cta_group::2, 256-row tiles): each CTA holds its 128 rows of A and half of
+// the B columns, so a stage is 32 KB and six of them fill the same ring
+constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_STAGE_BYTES = A_BYTES + B_BYTES_MAX / 2;
+static_assert(PAIR_STAGES * PAIR_STAGE_BYTES <= RING_BYTES, "pair ring fits the ring");
+static_assert(2 * PAIR_STAGES + 5 <= 28, "barriers fit their 256 bytes with the flags");
 constexpr int SMEM_BYTES = 1024 + RING_BYTES + 256 + 4 * (MAX_GROUPS + 1 + 40);
 
 enum Mode { DGRAD_DOWN = 0, DGRAD_UP = 1, WGRAD = 2 };
@@ -73,9 +79,10 @@ struct Args {
   int* err;
 };
 
-// DGRAD: m-tiles of 128 padded rows per expert; WGRAD: m_tiles per expert.  tp[e] = tiles
-// before expert e (times n_tiles later).  Checks poff.  Every thread must call it.
-__device__ bool bwd_tile_prefix(const Args& a, int* tp, int* scratch) {
+// DGRAD: m-tiles of tbm (128, or 256 for a pair) padded rows per expert; WGRAD: m_tiles
+// per expert.  tp[e] = tiles before expert e (times n_tiles later).  Checks poff.  Every
+// thread must call it.
+__device__ bool bwd_tile_prefix(const Args& a, int* tp, int* scratch, int tbm) {
   if (threadIdx.x == 0) {
     tp[0] = 0;
     scratch[33] = 0;
@@ -93,7 +100,7 @@ __device__ bool bwd_tile_prefix(const Args& a, int* tp, int* scratch) {
         if (p0 < 0 || p1 < p0 || (p1 - p0) % 64 != 0 || p1 > a.rows_cap + 64LL * a.E)
           scratch[33] = 1;
         else
-          v = (p1 - p0 + BM - 1) / BM;
+          v = (p1 - p0 + tbm - 1) / tbm;
       }
     }
     int tot;
@@ -140,34 +147,48 @@ __device__ __forceinline__ float u16_to_float(uint16_t v, int f16) {
   return __bfloat162float(__ushort_as_bfloat16(v));
 }
 
+// PAIR = false: one CTA per SM, 128-row tiles (tcgen05 cta_group::1).
+// PAIR = true: clusters of two CTAs share 256-row tiles (cta_group::2, M = 256): rank r
+// loads rows [128 r, +128) of the tile's A (dgrad: padded expert rows; wgrad: weight
+// rows, as two 64-column MN-major chunks) and B chunks [r bn/128, (r+1) bn/128) of the
+// tile's bn columns, all completing on rank 0's full barrier; one thread of rank 0 issues
+// the MMAs and commits to both CTAs' barriers; each CTA's epilogue reads its own 128 TMEM
+// lanes and arrives on rank 0's accumulator-empty barrier.
+template <bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const Args a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  constexpr int NST = PAIR ? PAIR_STAGES : STAGES;
+  constexpr int SB = PAIR ? PAIR_STAGE_BYTES : STAGE_BYTES;
+  constexpr int TBM = PAIR ? 2 * BM : BM;
   uint8_t* ring = smem;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RING_BYTES);
   const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = smem_u32(bars + STAGES);
-  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
-  const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
-  const uint32_t drain = smem_u32(bars + 2 * STAGES + 4);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  const uint32_t empty0 = smem_u32(bars + NST);
+  const uint32_t tfull0 = smem_u32(bars + 2 * NST);
+  const uint32_t tempty0 = smem_u32(bars + 2 * NST + 2);
+  const uint32_t drain = smem_u32(bars + 2 * NST + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * NST + 5);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* scratch = reinterpret_cast<int*>(smem + RING_BYTES + 256);
   int* tp = scratch + 40;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool wgrad = a.mode == WGRAD;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int stride = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
-      mbar_init(tempty0 + 8 * b, EPI_WARPS);
+      mbar_init(tempty0 + 8 * b, PAIR ? 2 * EPI_WARPS : EPI_WARPS);
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -178,21 +199,37 @@ __global__ void __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(tmem_holder), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   grid_dep_wait();
   grid_dep_launch();
-  const bool ok = bwd_tile_prefix(a, tp, scratch);
-  if (!ok && threadIdx.x == 0) set_error(a.err, kErrOffsets);
+  const bool ok = bwd_tile_prefix(a, tp, scratch, TBM);
+  if (!ok && threadIdx.x == 0 && rank == 0) set_error(a.err, kErrOffsets);
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int total = ok ? tp[a.E] * a.n_tiles : 0;
-  const int b_chunks = a.bn / 64;
+  const int b_chunks = (PAIR ? a.bn / 2 : a.bn) / 64;  // B chunks this CTA loads
+  const int b_chunk0 = static_cast<int>(rank) * b_chunks;
   const uint32_t b_bytes = static_cast<uint32_t>(b_chunks) * CHUNK;
   const uint32_t a_bytes = wgrad ? 2u * CHUNK : static_cast<uint32_t>(A_BYTES);
+  const uint32_t stage_tx = (PAIR ? 2u : 1u) * (a_bytes + b_bytes);  // bytes per full phase
+  // the full barrier every copy of a stage completes on: rank 0's in a pair
+  auto full_bar = [&](int stage) -> uint32_t {
+    return PAIR ? mapa_shared(full0 + 8 * stage, 0) : full0 + 8 * stage;
+  };
+  auto load = [&](uint32_t dst, const CUtensorMap* m, uint32_t fb, int c0, int c1) {
+    if constexpr (PAIR) tma_load_2d_pair(dst, m, fb, c0, c1);
+    else tma_load_2d(dst, m, fb, c0, c1);
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -200,36 +237,36 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_par = 0;
       bool aborted = false;
-      for (int L = blockIdx.x; L < total && !aborted; L += gridDim.x) {
+      for (int L = first; L < total && !aborted; L += stride) {
         const BTile t = bwd_decode(L, tp, a);
         const int kblocks = bwd_kblocks(a, t.e);
         const int p0 = __ldg(a.poff + t.e), r0 = __ldg(a.offsets + t.e);
+        const int m0 = t.mt * TBM + static_cast<int>(rank) * BM;  // this CTA's first row
+        const int n0 = t.nt * a.bn + 64 * b_chunk0;                // this CTA's first column
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, s_abort)) {
             aborted = true;
             break;
           }
-          const uint32_t st = smem_u32(ring + stage * STAGE_BYTES);
-          const uint32_t fb = full0 + 8 * stage;
-          mbar_arrive_expect_tx(fb, a_bytes + b_bytes);
+          const uint32_t st = smem_u32(ring + stage * SB);
+          const uint32_t fb = full_bar(stage);
+          if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * stage, stage_tx);
           if (wgrad) {
-            // A: the padded rows p0 + 64 kb .. (contraction) x columns mt*128 .. (M)
-            for (int c = 0; c < 2; ++c)
-              tma_load_2d(st + c * CHUNK, &tmA, fb, t.mt * BM + 64 * c, p0 + kb * BK);
-            // B: the unpadded rows r0 + 64 kb .. x columns nt*bn .. (N)
+            // A: the padded rows p0 + 64 kb .. (contraction) x columns m0 .. (M)
+            for (int c = 0; c < 2; ++c) load(st + c * CHUNK, &tmA, fb, m0 + 64 * c, p0 + kb * BK);
+            // B: the unpadded rows r0 + 64 kb .. x columns n0 .. (N)
             for (int c = 0; c < b_chunks; ++c)
-              tma_load_2d(st + A_BYTES + c * CHUNK, &tmB, fb, t.nt * a.bn + 64 * c, r0 + kb * BK);
+              load(st + A_BYTES + c * CHUNK, &tmB, fb, n0 + 64 * c, r0 + kb * BK);
           } else {
             // A: 128 padded rows, 64 contraction columns (K-major)
-            tma_load_2d(st, &tmA, fb, kb * BK, p0 + t.mt * BM);
-            // B: weight rows e*K + 64 kb .. (contraction) x columns nt*bn .. (N-major)
+            load(st, &tmA, fb, kb * BK, p0 + m0);
+            // B: weight rows e*K + 64 kb .. (contraction) x columns n0 .. (N-major)
             for (int c = 0; c < b_chunks; ++c)
-              tma_load_2d(st + A_BYTES + c * CHUNK, &tmB, fb, t.nt * a.bn + 64 * c,
-                          t.e * a.K + kb * BK);
+              load(st + A_BYTES + c * CHUNK, &tmB, fb, n0 + 64 * c, t.e * a.K + kb * BK);
           }
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1;
           }
@@ -238,18 +275,25 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (aborted) {
         set_error(a.err, kErrTimeout);
         *s_abort = 1;
-        for (int s = 0; s < STAGES; ++s)
-          if (armed & (1u << s)) mbar_wait(full0 + 8 * s, (armed_par >> s) & 1, nullptr, kDrainLimitNs);
+        // let every copy this thread started land before the CTA releases its smem (a
+        // pair's second CTA cannot watch rank 0's barrier: it waits out a fixed drain time)
+        if (rank == 0) {
+          for (int s = 0; s < NST; ++s)
+            if (armed & (1u << s)) mbar_wait(full0 + 8 * s, (armed_par >> s) & 1, nullptr, kDrainLimitNs);
+        } else {
+          const unsigned long long t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < kDrainLimitNs / 4) __nanosleep(1000);
+        }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       // ------------------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_f32acc_major(BM, a.bn, a.ab_f16 ? kFmtF16 : kFmtBF16, wgrad, true);
+      const uint32_t idesc = idesc_f32acc_major(TBM, a.bn, a.ab_f16 ? kFmtF16 : kFmtBF16, wgrad, true);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool aborted = false;
-      for (int L = blockIdx.x; L < total && !aborted; L += gridDim.x) {
+      for (int L = first; L < total && !aborted; L += stride) {
         const BTile t = bwd_decode(L, tp, a);
         const int kblocks = bwd_kblocks(a, t.e);
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1, s_abort)) {
@@ -264,29 +308,46 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(ring + stage * STAGE_BYTES);
+          const uint32_t a0 = smem_u32(ring + stage * SB);
           const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = wgrad ? sdesc_mn128(a0 + kk * 2048, CHUNK) : sdesc_k128(a0 + kk * 32);
-            tc_mma_f16kind(d_tmem, ad, sdesc_mn128(b0 + kk * 2048, CHUNK), idesc,
-                           (kb | kk) != 0 ? 1u : 0u);
+            if constexpr (PAIR)
+              tc_mma_pair_f16kind(d_tmem, ad, sdesc_mn128(b0 + kk * 2048, CHUNK), idesc,
+                                  (kb | kk) != 0 ? 1u : 0u);
+            else
+              tc_mma_f16kind(d_tmem, ad, sdesc_mn128(b0 + kk * 2048, CHUNK), idesc,
+                             (kb | kk) != 0 ? 1u : 0u);
           }
-          tc_commit(empty0 + 8 * stage);
-          if (++stage == STAGES) {
+          if constexpr (PAIR) {  // both CTAs' stages are free once these MMAs are done
+            tc_commit_pair(mapa_shared(empty0 + 8 * stage, 0));
+            tc_commit_pair(mapa_shared(empty0 + 8 * stage, 1));
+          } else {
+            tc_commit(empty0 + 8 * stage);
+          }
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (aborted) break;
-        tc_commit(tfull0 + 8 * acc);  // also with no k-block: the epilogue writes zeros
+        // also with no k-block: the epilogue writes zeros
+        if constexpr (PAIR) {
+          tc_commit_pair(mapa_shared(tfull0 + 8 * acc, 0));
+          tc_commit_pair(mapa_shared(tfull0 + 8 * acc, 1));
+        } else {
+          tc_commit(tfull0 + 8 * acc);
+        }
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1;
       }
       if (aborted) {
         set_error(a.err, kErrTimeout);
         *s_abort = 1;
-        tc_commit(drain);
+        // wait for the MMAs already issued before TMEM is freed
+        if constexpr (PAIR) tc_commit_pair(mapa_shared(drain, 0));
+        else tc_commit(drain);
         mbar_wait(drain, 0, nullptr, kDrainLimitNs);
       }
     }
@@ -294,9 +355,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;
     const int sub = (warp - 2) >> 2;
+    const uint32_t tempty_peer0 = PAIR ? mapa_shared(tempty0, 0) : tempty0;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x) {
+    for (int L = first; L < total; L += stride) {
       const BTile t = bwd_decode(L, tp, a);
       if (!mbar_wait(tfull0 + 8 * acc, acc_phase, s_abort)) {
         if (lane == 0) set_error(a.err, kErrTimeout);
@@ -308,7 +370,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * 256;
       const int col0 = t.nt * a.bn;
       if (wgrad) {
-        const int m = t.mt * BM + r;
+        const int m = t.mt * TBM + static_cast<int>(rank) * BM + r;
         const bool any = bwd_kblocks(a, t.e) > 0;
         float* dst_row = static_cast<float*>(a.out) +
                          (static_cast<int64_t>(t.e) * a.M + m) * a.N + col0;
@@ -329,7 +391,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       } else {
         const int p0 = __ldg(a.poff + t.e), p1 = __ldg(a.poff + t.e + 1);
         const int r0 = __ldg(a.offsets + t.e), r1 = __ldg(a.offsets + t.e + 1);
-        const int i = t.mt * BM + r;         // row within the expert's padded run
+        const int i = t.mt * TBM + static_cast<int>(rank) * BM + r;  // row in the padded run
         const bool kept = i < r1 - r0;
         const bool pad = !kept && i < p1 - p0;
         const int64_t s = r0 + i;            // unpadded row of a kept one
@@ -381,7 +443,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(tempty_peer0 + 8 * acc);
+        else mbar_arrive(tempty0 + 8 * acc);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
@@ -390,8 +455,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
+  // a pair's CTAs leave together: rank 0's MMAs read the other CTA's shared memory and
+  // the other CTA's epilogue arrives on rank 0's barriers
+  if constexpr (PAIR) cluster_sync_all();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == 1) {
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
+  }
 }
 
 }  // namespace bw
@@ -839,14 +910,66 @@ bool tmap16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int bo
                       static_cast<uint32_t>(box_rows), f16);
 }
 
-cudaError_t launch_bwd_gemm(const bw::Args& a, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                            int64_t max_tiles, const LaunchCtx& c) {
+// Clusters of two CTAs of bwd_gemm_kernel<true> that fit on the device at once, looked up
+// once per context.
+int bwd_max_active_pairs(const LaunchCtx& c) {
+  static std::mutex mu;
+  static std::map<unsigned long long, int> cache;
+  unsigned long long ctx = 0;
+  if (current_context_id(&ctx) != cudaSuccess) return c.num_sms / 2;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(ctx);
+  if (it != cache.end()) return it->second;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (c.num_sms / 2));
+  cfg.blockDim = dim3(bw::THREADS);
+  cfg.dynamicSmemBytes = bw::SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, bw::bwd_gemm_kernel<true>, &cfg) != cudaSuccess || n <= 0)
+    n = c.num_sms / 2;
+  if (n > c.num_sms / 2) n = c.num_sms / 2;
+  cache[ctx] = n;
+  return n;
+}
+
+// Experts with at least this many rows on average (T*k / E) run their products on CTA
+// pairs (256-row tiles), as the forward pass does.
+constexpr int64_t kBwdPairMinRowsPerExpert = 256;
+
+// One product: pairs when the experts are large enough, B's bn columns split into whole
+// 64-column chunks per CTA, and (weight gradients) the M rows into 256-row tiles.  Sets
+// a.m_tiles for the weight gradients.  prows: rows of the padded layout.
+cudaError_t launch_bwd_gemm(bw::Args a, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                            int64_t prows, const LaunchCtx& c) {
+  const bool wg = a.mode == bw::WGRAD;
+  const bool pair = a.bn >= 128 && a.rows_cap >= kBwdPairMinRowsPerExpert * a.E &&
+                    (!wg || a.M % (2 * bw::BM) == 0);
+  const int tbm = pair ? 2 * bw::BM : bw::BM;
+  if (wg) a.m_tiles = (a.M + tbm - 1) / tbm;
+  const int64_t max_tiles = wg ? static_cast<int64_t>(a.E) * a.m_tiles * a.n_tiles
+                               : (prows / tbm + a.E) * static_cast<int64_t>(a.n_tiles);
+  if (pair) {
+    cudaError_t e = ensure_smem_limit(bw::bwd_gemm_kernel<true>, bw::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    const int64_t cap = bwd_max_active_pairs(c);
+    const int pairs = static_cast<int>(max_tiles < cap ? max_tiles : cap);
+    if (pairs <= 0) return cudaSuccess;
+    return launch_kernel_pairs(bw::bwd_gemm_kernel<true>, dim3(2 * pairs), dim3(bw::THREADS),
+                               bw::SMEM_BYTES, c, tmA, tmB, a);
+  }
   const int grid = static_cast<int>(max_tiles < c.num_sms ? max_tiles : c.num_sms);
   if (grid <= 0) return cudaSuccess;
-  cudaError_t e = ensure_smem_limit(bw::bwd_gemm_kernel, bw::SMEM_BYTES);
+  cudaError_t e = ensure_smem_limit(bw::bwd_gemm_kernel<false>, bw::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  return launch_kernel(bw::bwd_gemm_kernel, dim3(grid), dim3(bw::THREADS), bw::SMEM_BYTES, c, tmA,
-                       tmB, a);
+  return launch_kernel(bw::bwd_gemm_kernel<false>, dim3(grid), dim3(bw::THREADS), bw::SMEM_BYTES,
+                       c, tmA, tmB, a);
 }
 
 }  // namespace
@@ -884,18 +1007,18 @@ cudaError_t launch_backward(const BackwardProblem& p, const LaunchCtx& c) {
     if (!tmap16(&tA, p.d_o, prows, d, bw::BM, w2f16) ||
         !tmap16(&tB, p.w2, static_cast<int64_t>(E) * d, f, 64, w2f16))
       return cudaErrorInvalidValue;
-    e = launch_bwd_gemm(a, tA, tB, (prows / bw::BM + E) * static_cast<int64_t>(a.n_tiles), c);
+    e = launch_bwd_gemm(a, tA, tB, prows, c);
     if (e != cudaSuccess) return e;
   }
   {  // dW2_e = d_o_e^T . h_e: M = d, N = f, contraction over the expert's rows
     bw::Args a = {};
     a.mode = bw::WGRAD; a.E = E; a.offsets = p.offsets; a.poff = p.poff;
-    a.M = d; a.N = f; a.bn = pick_bn_bwd(f); a.n_tiles = f / a.bn; a.m_tiles = (d + bw::BM - 1) / bw::BM;
+    a.M = d; a.N = f; a.bn = pick_bn_bwd(f); a.n_tiles = f / a.bn;
     a.rows_cap = n; a.out = p.dw2; a.ab_f16 = w2f16; a.err = c.err;
     CUtensorMap tA, tB;
     if (!tmap16(&tA, p.d_o, prows, d, 64, w2f16) || !tmap16(&tB, p.h, n, f, 64, w2f16))
       return cudaErrorInvalidValue;
-    e = launch_bwd_gemm(a, tA, tB, static_cast<int64_t>(E) * a.m_tiles * a.n_tiles, c);
+    e = launch_bwd_gemm(a, tA, tB, prows, c);
     if (e != cudaSuccess) return e;
   }
   {  // dx_perm = du . W1_e: M = padded rows, N = d, K = f; W1 [E, f, d] as [E*f, d]
@@ -907,18 +1030,18 @@ cudaError_t launch_backward(const BackwardProblem& p, const LaunchCtx& c) {
     if (!tmap16(&tA, p.du, prows, f, bw::BM, 0) ||
         !tmap16(&tB, p.w1, static_cast<int64_t>(E) * f, d, 64, 0))
       return cudaErrorInvalidValue;
-    e = launch_bwd_gemm(a, tA, tB, (prows / bw::BM + E) * static_cast<int64_t>(a.n_tiles), c);
+    e = launch_bwd_gemm(a, tA, tB, prows, c);
     if (e != cudaSuccess) return e;
   }
   {  // dW1_e = du_e^T . x_perm_e: M = f, N = d
     bw::Args a = {};
     a.mode = bw::WGRAD; a.E = E; a.offsets = p.offsets; a.poff = p.poff;
-    a.M = f; a.N = d; a.bn = pick_bn_bwd(d); a.n_tiles = d / a.bn; a.m_tiles = (f + bw::BM - 1) / bw::BM;
+    a.M = f; a.N = d; a.bn = pick_bn_bwd(d); a.n_tiles = d / a.bn;
     a.rows_cap = n; a.out = p.dw1; a.ab_f16 = 0; a.err = c.err;
     CUtensorMap tA, tB;
     if (!tmap16(&tA, p.du, prows, f, 64, 0) || !tmap16(&tB, p.x_perm, n, d, 64, 0))
       return cudaErrorInvalidValue;
-    e = launch_bwd_gemm(a, tA, tB, static_cast<int64_t>(E) * a.m_tiles * a.n_tiles, c);
+    e = launch_bwd_gemm(a, tA, tB, prows, c);
     if (e != cudaSuccess) return e;
   }
   e = launch_kernel(unpermute_kernel, dim3(static_cast<unsigned>((p.T + 7) / 8)), dim3(256), 0, c,

@@ -51,6 +51,16 @@ CASES = {
                                                                seed=1), 0.0, 0.0),
     "k4_E32_capacity": (Workload("bk", T=800, d_model=64, d_ff=128, E=32, k=4, act="gelu",
                                  capacity_factor=0.8, seed=1), 0.2, 0.0),
+    # experts averaging >= 256 rows: the four expert products run on CTA pairs (256-row
+    # tiles), with the skewed experts' ragged and small runs, and with fp16 hidden
+    # activations and capacity drops
+    "pairs_k2_gelu": (Workload("bp", T=2048, d_model=256, d_ff=512, E=4, k=2, act="gelu",
+                               seed=1), 0.1, 0.0),
+    "pairs_zipf_bias": (workloads.WORKLOADS["zipf"].scaled(T=4096, d_model=256, d_ff=512,
+                                                           seed=1), 0.0, 0.0),
+    "pairs_switch_f16_capacity": (Workload("bpf", T=4096, d_model=256, d_ff=512, E=8, k=1,
+                                           renorm=False, capacity_factor=1.0, act="gelu",
+                                           hidden_f16=True, seed=5), 0.0, 0.0),
 }
 
 
