@@ -656,8 +656,9 @@ def training_step(lb, flush, steps, world, dev, stream):
     fwd = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     bwd = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
     fwd, bwd = max_over_ranks(fwd, dev), max_over_ranks(bwd, dev)
-    offs = lb.o["offsets"].cpu().tolist()
-    n_kept = offs[-1]
+    # kept rows of the training forward: each expert's assignments up to the capacity
+    C = moe.moe_capacity(cfg)
+    n_kept = sum(min(c, C) if C >= 0 else c for c in o["counts"].cpu().tolist())
     bwd_flops = 8.0 * n_kept * dm * f
     return {"value": T * world / ((fwd + bwd) * 1e-3), "unit": "tokens/s",
             "forward_train_ms": fwd, "backward_ms": bwd, "steps": n,
@@ -686,6 +687,15 @@ def run_gpu(args, w):
 
     # ---- the headline workload
     lb = LayerBench(moe, w, dev)
+    if args.training_only:
+        # the training step alone (for profiler captures of the backward pass)
+        train = training_step(lb, flush, args.steps, world, dev, stream)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"training_step": train, "config": config_json(w)}), flush=True)
+        return
     per, clocks, timed_launches, kept = timed_steps(lb, flush, args.steps, args.warmup, world,
                                                    dev, clock_gpu)
     step_ms_max = max_over_ranks(float(np.mean(per.sum(axis=1))), dev)
@@ -823,6 +833,9 @@ def main(argv=None):
                     help="time only the headline workload")
     ap.add_argument("--no-training", action="store_true",
                     help="skip the training-step (forward + backward) figure")
+    ap.add_argument("--training-only", action="store_true",
+                    help="time only the training step (forward keeping its state, then the "
+                         "backward); for profiler captures")
     ap.add_argument("--y-bf16", action="store_true",
                     help="layer output y in bf16 for bf16 layers (outside these workloads' "
                          "error bar; not a benchmark figure)")
