@@ -91,6 +91,60 @@ def test_steps_and_forward_small(name):
     print(name, rep)
 
 
+def _random_cases(n=16, seed=2024):
+    """Seeded random small layers: dtype, expert count (1 to 256), k (up to 8, <= E),
+    gating, capacity, activation, widths and token counts drawn independently, so that
+    shapes no hand-written case names still meet the oracle.  A Switch-style top-1 gate
+    (renorm off) stores h in fp16, as the Switch workload does (its gates vary too much for
+    one bf16 rounding of h within the bar)."""
+    rng = np.random.default_rng(seed)
+    cases = {}
+    for i in range(n):
+        dtype = "f32" if i % 5 == 4 else "bf16"
+        E = int(rng.choice([1, 2, 3, 5, 8, 13, 16, 32, 64, 100, 256]))
+        k = int(rng.integers(1, min(E, 8) + 1))
+        gating = "noisy_topk" if rng.random() < 0.3 else "softmax_topk"
+        renorm = True if (gating == "noisy_topk" or k > 1) else bool(rng.random() < 0.5)
+        if dtype == "bf16":
+            d = int(rng.choice([64, 128, 192, 256, 512]))
+            f = int(rng.choice([64, 128, 192, 320, 512, 1024]))
+        else:
+            d = int(rng.choice([8, 24, 64, 96]))
+            f = int(rng.choice([4, 12, 64, 100]))
+        T = int(rng.integers(1, 2500))
+        cf = None if rng.random() < 0.5 else float(rng.choice([0.5, 0.8, 1.0, 1.25, 2.0]))
+        act = "gelu" if rng.random() < 0.5 else "relu"
+        hidden_f16 = dtype == "bf16" and (not renorm or rng.random() < 0.3)
+        name = "rand%02d_%s_T%d_E%d_k%d_%s" % (i, dtype, T, E, k, gating.split("_")[0])
+        cases[name] = Workload("r%02d" % i, T=T, d_model=d, d_ff=f, E=E, k=k, gating=gating,
+                               renorm=renorm, capacity_factor=cf, act=act, dtype=dtype,
+                               hidden_f16=hidden_f16, seed=100 + i)
+    return cases
+
+
+RANDOM = _random_cases()
+
+
+@pytest.mark.parametrize("name", list(RANDOM))
+def test_steps_and_forward_random_shapes(name):
+    w = RANDOM[name]
+    inp = workloads.make_inputs(w)
+    dev = H.to_device(inp)
+    g = H.run_steps(w, dev)
+    assert g["device_error"] == 0
+    rep = {}
+    idx, gates = H.check_route(w, inp, g, rep)
+    n = H.check_permute(w, inp, g, rep)
+    H.check_ffn(w, inp, g, n, rep)
+    H.check_combine(w, g, rep)
+    H.check_end_to_end(w, inp, g, idx, gates, rep)
+    H.check_gather_path(w, g, rep)
+    f = H.run_forward(w, dev)
+    assert f["device_error"] == 0
+    assert torch.equal(f["y"], g["y"])
+    print(name, rep)
+
+
 def test_empty_batch():
     w = Workload("t0", T=0, d_model=64, d_ff=64, E=4, k=2, gating="noisy_topk")
     inp = workloads.make_inputs(w)
