@@ -62,6 +62,21 @@ CASES = {
                                            renorm=False, capacity_factor=1.0, act="gelu",
                                            hidden_f16=True, seed=5), 0.0, 0.0),
 }
+# shapes drawn at random once (seeded), each with the first seed whose routing has no near
+# ties: k = E, top-1 with capacity and fp16 hidden activations, small and odd widths,
+# and noisy gating with both losses
+for _i, (_T, _d, _f, _E, _k, _g, _rn, _cf, _act, _hf, _seed, _wi, _wl) in enumerate([
+        (1565, 256, 64, 2, 2, "softmax_topk", True, None, "gelu", False, 1, 0.1, 0.0),
+        (1330, 64, 320, 4, 1, "softmax_topk", False, 1.5, "gelu", True, 1, 0.5, 0.0),
+        (1291, 256, 64, 6, 3, "softmax_topk", True, None, "relu", True, 1, 0.1, 0.0),
+        (265, 128, 192, 6, 2, "softmax_topk", True, None, "relu", True, 1, 0.5, 0.0),
+        (831, 128, 128, 16, 4, "softmax_topk", True, 1.5, "gelu", False, 1, 0.5, 0.0),
+        (900, 128, 128, 8, 2, "noisy_topk", True, None, "relu", False, 1, 0.3, 0.4),
+        (1500, 64, 192, 4, 2, "noisy_topk", True, 1.25, "gelu", False, 1, 0.2, 0.2),
+        (400, 192, 64, 16, 3, "noisy_topk", True, None, "gelu", False, 1, 0.0, 0.5)]):
+    CASES["random%d_T%d_E%d_k%d_%s" % (_i, _T, _E, _k, _g.split("_")[0])] = (
+        Workload("rb%d" % _i, T=_T, d_model=_d, d_ff=_f, E=_E, k=_k, gating=_g, renorm=_rn,
+                 capacity_factor=_cf, act=_act, hidden_f16=_hf, seed=_seed), _wi, _wl)
 
 
 def _round16(a, f16):
