@@ -564,9 +564,11 @@ static int pick_bn(int N) {
 }
 
 // Experts with at least this many rows on average (T*k / E, counted before capacity
-// drops) run on CTA pairs (256-row tiles, cta_group::2); fewer rows per expert would
-// leave most of each 256-row tile empty.
-constexpr int64_t kPairMinRowsPerExpert = 256;
+// drops) run on CTA pairs (256-row tiles, cta_group::2).  Near 256 rows a good share of
+// the experts spill into a second, mostly empty 256-row tile (the two-level workload's
+// experts hold 195-331 rows: its expert FFN took 116.7 us on pairs, 111.6 us on 128-row
+// tiles); from 512 on that share is small.
+constexpr int64_t kPairMinRowsPerExpert = 512;
 
 // Clusters of two CTAs of grouped_gemm_tc_kernel<true> that fit on the device at once (a
 // persistent grid larger than that would serialise), looked up once per context.
