@@ -555,6 +555,111 @@ __device__ __forceinline__ void gate_tile_hier(const Fetch& fetch, int q, int la
   if (valid && g.near_tie) g.near_tie[t] = (gap <= 1e-4f) ? 1 : 0;
 }
 
+// The hierarchical gate of the tensor-core router, spread over column groups: the same
+// token rows and score columns as gate_tile_hier, with the thread in lane l of gate warp
+// w owning row r = 32*q + l of column group grp = w / 4 (with half tiles, 64 tokens in
+// both halves of the MMA operand: row 32*(q & 1) + l of column group 2*grp + q / 2, as
+// in gate_tile).  Every thread scores the primary columns of its token; column group cg
+// then forms the secondary list of each group i = cg, cg + CG, ... over that group's
+// columns in ascending order (a fresh list per group, so no thread walks the groups it
+// does not own) and, where its token kept group i, writes that group's assignments.
+// Results equal gate_tile_hier's: the same lists, gates and gaps, formed by the same
+// operations.  The per-token minimum gap over the kept groups meets in shared memory.
+template <int KP, int KG, int G, class Fetch, class Sync>
+__device__ __forceinline__ void gate_tile_hier_cg(const Fetch& fetch, const Sync& sync, int q,
+                                                  int grp, int lane, int64_t tile, bool half,
+                                                  const GateArgs& g, uint8_t* smem) {
+  const int ntok = half ? 64 : 128;
+  const int row = half ? (q & 1) * 32 + lane : q * 32 + lane;
+  const int CG = half ? 2 * G : G;
+  const int cgrp = half ? grp * 2 + (q >> 1) : grp;
+  const int64_t t = tile * ntok + row;
+  const bool valid = t < g.T;
+  const int A = g.groups, B = g.E / g.groups;
+  const int k1 = g.k_primary, k2 = g.k / g.k_primary;
+  TopList<KP> prim;
+  prim.init();
+#pragma unroll 1
+  for (int cs = 0; cs < A; cs += 16) {
+    float l[16], z[16];
+    fetch(cs, l, z);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (cs + j < A) prim.push(l[j], cs + j);
+  }
+  float gp[KP];
+  float den = 0.0f;
+#pragma unroll
+  for (int q2 = 0; q2 < KP; ++q2) {
+    gp[q2] = (q2 < k1) ? expf(prim.v[q2] - prim.v[0]) : 0.0f;
+    den += gp[q2];
+  }
+  float gmin = INFINITY;  // smallest secondary gap over the kept groups this thread owns
+#pragma unroll 1
+  for (int i = cgrp; i < A; i += CG) {
+    TopList<KG> cur;
+    cur.init();
+    const int c0 = A + i * B, c1 = c0 + B;
+#pragma unroll 1
+    for (int cs = c0 & ~15; cs < c1; cs += 16) {
+      float l[16], z[16];
+      fetch(cs, l, z);
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (cs + j >= c0 && cs + j < c1) cur.push(l[j], cs + j - c0);
+    }
+    // the rank of group i among this token's kept groups, if it kept it
+    int slot = -1;
+    float share = 0.0f;
+#pragma unroll
+    for (int q2 = 0; q2 < KP; ++q2)
+      if (q2 < k1 && prim.i[q2] == i) {
+        slot = q2;
+        share = gp[q2] / den;
+      }
+    if (slot >= 0) {
+      float gs[KG];
+      float ds = 0.0f;
+#pragma unroll
+      for (int j = 0; j < KG; ++j) {
+        gs[j] = (j < k2) ? expf(cur.v[j] - cur.v[0]) : 0.0f;
+        ds += gs[j];
+      }
+      float sk = INFINITY, sk1 = -INFINITY;
+#pragma unroll
+      for (int j = 0; j <= KG; ++j) {
+        if (j < k2) sk = fminf(sk, cur.v[j]);
+        else sk1 = fmaxf(sk1, cur.v[j]);
+      }
+      if (k2 < B) gmin = fminf(gmin, sk - sk1);
+      if (valid) {
+#pragma unroll
+        for (int j = 0; j < KG; ++j)
+          if (j < k2) {
+            g.topk_idx[t * g.k + slot * k2 + j] = i * B + cur.i[j];
+            g.topk_gate[t * g.k + slot * k2 + j] = share * (gs[j] / ds);
+          }
+      }
+    }
+  }
+  if (g.near_tie != nullptr) {  // uniform across the gate threads
+    float* hg = reinterpret_cast<float*>(smem);  // [CG][ntok]
+    hg[cgrp * ntok + row] = gmin;
+    sync();
+    if (cgrp == 0 && valid) {
+      float kth = INFINITY, kth1 = -INFINITY;
+#pragma unroll
+      for (int j = 0; j <= KP; ++j) {
+        if (j < k1) kth = fminf(kth, prim.v[j]);
+        else kth1 = fmaxf(kth1, prim.v[j]);
+      }
+      float gap = (k1 < A) ? kth - kth1 : INFINITY;
+      for (int c2 = 0; c2 < CG; ++c2) gap = fminf(gap, hg[c2 * ntok + row]);
+      g.near_tie[t] = (gap <= 1e-4f) ? 1 : 0;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ bf16 router
 //
 // Persistent and warp-specialised.  Warp 0 streams the x tile and the gating weights of
@@ -592,9 +697,8 @@ __device__ __forceinline__ void gate_bar_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
-// HKG > 0: hierarchical gating with KM the primary and HKG the secondary list bucket
-// (one column group of gate warps).
-template <int KM, int HKG = 0, int G = (HKG > 0 ? 1 : rt::groups_for(KM))>
+// HKG > 0: hierarchical gating with KM the primary and HKG the secondary list bucket.
+template <int KM, int HKG = 0, int G = rt::groups_for(KM)>
 __global__ void __launch_bounds__(64 + 128 * G)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     const __grid_constant__ CUtensorMap tmG,
@@ -784,7 +888,7 @@ __global__ void __launch_bounds__(64 + 128 * G)
           }
         };
         if constexpr (HKG > 0) {
-          gate_tile_hier<KM, HKG>(fetch, q, lane, L, a.g);
+          gate_tile_hier_cg<KM, HKG, G>(fetch, sync, q, grp, lane, L, a.half != 0, a.g, gsm);
         } else {
           gate_tile<KM, G, 16>(fetch, sync, q, grp, gtid, L, a.half != 0, a.g, gsm);
         }
@@ -979,7 +1083,7 @@ static cudaError_t launch_route_tc(const CUtensorMap& tmX, const CUtensorMap& tm
                                    int grid, const LaunchCtx& c) {
   cudaError_t e = ensure_smem_limit(route_tc_kernel<KM, HKG>, smem);
   if (e != cudaSuccess) return e;
-  const int G = HKG > 0 ? 1 : rt::groups_for(KM);
+  const int G = rt::groups_for(KM);
   return launch_kernel(route_tc_kernel<KM, HKG>, dim3(grid), dim3(64 + 128 * G), smem, c, tmX, tmG,
                        tmN, a);
 }
@@ -1046,13 +1150,12 @@ cudaError_t launch_route_bf16(const RouteProblem& p, const LaunchCtx& c) {
   a.kblocks = p.d / rt::BK;
   a.nb = p.noisy ? 2 : 1;
   a.nbuf = 2 * a.nb * a.acc_cols <= 512 ? 2 : 1;
-  // half tiles when 128-token tiles would fill at most half of the SMs (not for the
-  // hierarchical gate, whose one thread per token reads every score column)
+  // half tiles when 128-token tiles would fill at most half of the SMs
   const int full_tiles = static_cast<int>((p.T + kRouteBM - 1) / kRouteBM);
-  a.half = (!p.hier && 2 * full_tiles <= c.num_sms) ? 1 : 0;
+  a.half = (2 * full_tiles <= c.num_sms) ? 1 : 0;
   a.ntiles = a.half ? static_cast<int>((p.T + 63) / 64) : full_tiles;
   const int km = p.hier ? k_bucket(p.k_primary) : k_bucket(p.k);
-  const int scratch = gate_smem_bytes(km, p.hier ? 1 : rt::groups_for(km), p.E);
+  const int scratch = gate_smem_bytes(km, rt::groups_for(km), p.E);
   const int stage_bytes = rt::A_BYTES + a.nb * a.e_pad * rt::BK * 2;
   // the ring takes what the gate scratch and the barriers leave of 227 KB
   const int bar_bytes = 8 * (2 * 8 + 5) + 16;

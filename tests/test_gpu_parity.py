@@ -65,6 +65,19 @@ SMALL = {
                                gating="hierarchical", groups=4, k_primary=2, act="relu"),
     "hier_8x8_k4x2": Workload("h5", T=700, d_model=128, d_ff=64, E=64, k=8,
                               gating="hierarchical", groups=8, k_primary=4, act="relu"),
+    # the router's gate splits the groups over its column groups: 32 primary columns (two
+    # 16-column slices) with four groups to a slice; two groups of 64 (each over four
+    # slices, most column groups idle); groups of 12 straddling slices with three of five
+    # kept; 128-token tiles (more than 74 of them) instead of 64-token ones
+    "hier_32x4_k2x1": Workload("h6", T=1000, d_model=128, d_ff=64, E=128, k=2,
+                               gating="hierarchical", groups=32, k_primary=2, act="relu"),
+    "hier_2x64_k1x4": Workload("h7", T=333, d_model=64, d_ff=64, E=128, k=4,
+                               gating="hierarchical", groups=2, k_primary=1, act="gelu"),
+    "hier_5x12_k3x1": Workload("h8", T=517, d_model=64, d_ff=64, E=60, k=3,
+                               gating="hierarchical", groups=5, k_primary=3, act="relu"),
+    "hier_full_tiles_T10000": Workload("h9", T=10000, d_model=128, d_ff=64, E=64, k=4,
+                                       gating="hierarchical", groups=8, k_primary=2,
+                                       act="relu"),
 }
 
 
