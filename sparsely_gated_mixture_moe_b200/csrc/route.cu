@@ -108,21 +108,54 @@ struct TopList {
     v[0] = first ? cv : v[0];
     i[0] = first ? ci : i[0];
   }
-  // keeps the first k+1 slots (k <= KM); equal scores rank by expert index
-  __device__ __forceinline__ void insert(float cv, int ci, int k) {
+};
+
+// Merges the list (ov, oi), over experts disjoint from t's, into t: afterwards t holds
+// the KM+1 highest-ranked pairs of both.  A pair's place in the union is its place in
+// its own list plus the number of pairs of the other list ranked above it; the
+// (KM+1)^2 comparisons are independent of one another, unlike insertion one pair at a
+// time.  Empty slots (-inf, 0x7fffffff) rank below every expert's score and never above
+// one another, so they only fill the places the experts leave.
+template <int KM>
+__device__ __forceinline__ void merge_top(TopList<KM>& t, const float (&ov)[KM + 1],
+                                          const int (&oi)[KM + 1]) {
+  int ra[KM + 1], rb[KM + 1];
+#pragma unroll
+  for (int p = 0; p <= KM; ++p) {
+    ra[p] = p;
+    rb[p] = p;
+  }
+#pragma unroll
+  for (int p = 0; p <= KM; ++p)
 #pragma unroll
     for (int q = 0; q <= KM; ++q) {
-      if (q <= k && (cv > v[q] || (cv == v[q] && ci < i[q]))) {
-        const float tv = v[q];
-        const int ti = i[q];
-        v[q] = cv;
-        i[q] = ci;
-        cv = tv;
-        ci = ti;
-      }
+      const bool above = ov[q] > t.v[p] || (ov[q] == t.v[p] && oi[q] < t.i[p]);
+      ra[p] += above ? 1 : 0;
+      rb[q] += above ? 0 : 1;
+    }
+  float nv[KM + 1];
+  int ni[KM + 1];
+#pragma unroll
+  for (int r = 0; r <= KM; ++r) {
+    nv[r] = -INFINITY;
+    ni[r] = 0x7fffffff;
+#pragma unroll
+    for (int p = 0; p <= KM; ++p) {
+      nv[r] = (ra[p] == r) ? t.v[p] : nv[r];
+      ni[r] = (ra[p] == r) ? t.i[p] : ni[r];
+    }
+#pragma unroll
+    for (int q = 0; q <= KM; ++q) {
+      nv[r] = (rb[q] == r) ? ov[q] : nv[r];
+      ni[r] = (rb[q] == r) ? oi[q] : ni[r];
     }
   }
-};
+#pragma unroll
+  for (int r = 0; r <= KM; ++r) {
+    t.v[r] = nv[r];
+    t.i[r] = ni[r];
+  }
+}
 
 // Shared-memory bytes gate_tile needs for 128*G gate threads.
 __host__ __device__ constexpr int gate_smem_bytes(int KM, int G, int E) {
@@ -183,8 +216,9 @@ __device__ __forceinline__ int colsum8_column(int lane) {
 // loads.  `sync()` is a barrier over the 128*G gate threads.  Each W-column slice is
 // scored from registers: its maximum updates the running softmax (one rescale per
 // slice), and a group of 8 scores enters the top list by branch-free insertion unless
-// no lane of the warp has one above its current (k+1)-th score.  The logit bias has been loaded into shared memory
-// (load_bias_smem) by the caller.
+// no lane of the warp has one above its current (k+1)-th score.  The column groups'
+// partial lists then merge pairwise in log2(column groups) rounds (merge_top).  The
+// logit bias has been loaded into shared memory (load_bias_smem) by the caller.
 template <int KM, int G, int W, class Fetch, class Sync>
 __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, int q, int grp,
                                           int gtid, int64_t tile, bool half, const GateArgs& g,
@@ -312,21 +346,42 @@ __device__ __forceinline__ void gate_tile(const Fetch& fetch, const Sync& sync, 
   ps[cgrp * ntok + row] = ssum;
   sync();
 
-  // ---- merge the G partial results of each token (group 0) and write the outputs
-  if (cgrp == 0) {
+  // ---- merge the CG partial results of each token pairwise (column group c takes in
+  // c + s for s = CG/2, CG/4, ..., 1), then group 0 writes the outputs
 #pragma unroll 1
-    for (int g2 = 1; g2 < CG; ++g2) {
+  for (int s = CG >> 1; s >= 1; s >>= 1) {
+    if (cgrp < s) {
+      const int o = (cgrp + s) * ntok + row;
+      float ov[KM + 1];
+      int oi[KM + 1];
 #pragma unroll
-      for (int s2 = 0; s2 <= KM; ++s2)
-        if (s2 <= k)
-          top.insert(pv[(g2 * ntok + row) * (KM + 1) + s2], pi[(g2 * ntok + row) * (KM + 1) + s2], k);
-      const float m2 = pm[g2 * ntok + row], s2v = ps[g2 * ntok + row];
-      if (m2 != -INFINITY) {
-        const float nm = fmaxf(m, m2);
-        ssum = (m == -INFINITY ? 0.0f : ssum * expf(m - nm)) + s2v * expf(m2 - nm);
-        m = nm;
+      for (int s2 = 0; s2 <= KM; ++s2) {
+        ov[s2] = pv[o * (KM + 1) + s2];
+        oi[s2] = pi[o * (KM + 1) + s2];
+      }
+      merge_top<KM>(top, ov, oi);
+      if (full_softmax) {
+        const float m2 = pm[o], s2v = ps[o];
+        if (m2 != -INFINITY) {
+          const float nm = fmaxf(m, m2);
+          ssum = (m == -INFINITY ? 0.0f : ssum * expf(m - nm)) + s2v * expf(m2 - nm);
+          m = nm;
+        }
+      }
+      if (s > 1) {
+        const int own = cgrp * ntok + row;
+#pragma unroll
+        for (int s2 = 0; s2 <= KM; ++s2) {
+          pv[own * (KM + 1) + s2] = top.v[s2];
+          pi[own * (KM + 1) + s2] = top.i[s2];
+        }
+        pm[own] = m;
+        ps[own] = ssum;
       }
     }
+    if (s > 1) sync();
+  }
+  if (cgrp == 0) {
     float gate[KM];
     if (full_softmax) {
 #pragma unroll
