@@ -1015,71 +1015,94 @@ __global__ void __launch_bounds__(128, 1)
                          static_cast<int>(threadIdx.x) & 31, static_cast<int64_t>(blockIdx.x), g);
 }
 
-// Importance and Load partial sums of noisy gating from the gate's per-token values:
-// block (chunk, eb) covers a run of tokens and experts 8*eb .. 8*eb+7, one per warp; the
-// lanes take the run's tokens 32 at a time, four such groups per step with every load of
-// the step issued before any arithmetic (the kernel is bound by load latency, not bytes).
+// Importance and Load partial sums of noisy gating from the gate's per-token values.
+// Block (chunk, slice) covers a run of tokens and 8*R experts; warp w of the block takes
+// experts slice*8R + w*R .. +R-1 and its lanes the run's tokens 32 at a time, each lane
+// reading its token's chosen experts, gates and k-th / (k+1)-th scores once and then the
+// warp's R experts' values (a warp reads 128 contiguous bytes per expert and quantity).
 // For token t and expert e:
 //   Importance term: the gate of e if e is one of t's chosen experts, else 0
 //   Load term: P(t, e) = Phi((l_te - kth_excluding(H_t, k, e)) / Softplus(z_te)), where
 //   kth_excluding is the (k+1)-th largest score when H_te >= the k-th largest, else the
 //   k-th largest (H_te as the gate formed it, so H >= the k-th means "among the top k").
-// Each lane adds its tokens in increasing order and the warp's lanes are then summed in
-// a fixed butterfly order into partials[chunk][2][E], so the result does not depend on
-// scheduling.
-constexpr int kIlGroups = 4;  // 32-token groups per lane step
+// Each lane adds its tokens in increasing order, then the lanes of each expert column are
+// summed in a fixed butterfly order into partials[chunk][2][E], so the result does not
+// depend on scheduling.
+template <int R>
 __global__ void __launch_bounds__(256)
     importance_load_kernel(const float* __restrict__ lw, const float* __restrict__ sw,
                            const float* __restrict__ hw, const float* __restrict__ kw,
                            const int32_t* __restrict__ topk_idx,
                            const float* __restrict__ topk_gate, int64_t T, int E, int k,
                            int64_t chunk_tokens, int want_load, float* __restrict__ partials) {
+  static_assert(R % 8 == 0, "experts per warp: whole 8-column reduce steps");
   grid_dep_wait();
   grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.y * 8 + warp;
-  if (e >= E) return;
+  const int e0 = (blockIdx.y * 8 + warp) * R;
+  if (e0 >= E) return;  // the whole warp
   const int64_t t_lo = static_cast<int64_t>(blockIdx.x) * chunk_tokens;
   const int64_t t_hi = min(T, t_lo + chunk_tokens);
-  float si = 0.0f, sl = 0.0f;
-  for (int64_t t0 = t_lo + lane; t0 < t_hi; t0 += 32 * kIlGroups) {
-    float gi[kIlGroups], li[kIlGroups], sp[kIlGroups], H[kIlGroups], k0[kIlGroups], k1[kIlGroups];
+  float si[R], sl[R];
 #pragma unroll
-    for (int u = 0; u < kIlGroups; ++u) {
-      const int64_t t = t0 + 32 * u;
-      gi[u] = 0.0f;
-      li[u] = sp[u] = H[u] = k0[u] = k1[u] = 0.0f;
-      if (t < t_hi) {
-        for (int j = 0; j < k; ++j)
-          if (__ldg(topk_idx + t * k + j) == e) gi[u] = __ldg(topk_gate + t * k + j);
-        if (want_load) {
-          const int64_t i = static_cast<int64_t>(e) * T + t;
-          li[u] = __ldg(lw + i);
-          sp[u] = __ldg(sw + i);
-          H[u] = __ldg(hw + i);
-          k0[u] = __ldg(kw + t);
-          k1[u] = __ldg(kw + T + t);
-        }
-      }
+  for (int r = 0; r < R; ++r) si[r] = sl[r] = 0.0f;
+  for (int64_t tb = t_lo; tb < t_hi; tb += 32) {
+    const int64_t t = tb + lane;
+    const bool tv = t < t_hi;
+    int id[8];
+    float gv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const bool in = tv && j < k;
+      id[j] = in ? __ldg(topk_idx + t * k + j) : -1;
+      gv[j] = in ? __ldg(topk_gate + t * k + j) : 0.0f;
     }
 #pragma unroll
-    for (int u = 0; u < kIlGroups; ++u) {
-      if (t0 + 32 * u >= t_hi) break;
-      si += gi[u];
-      if (want_load) {
-        const float ex = (H[u] >= k0[u]) ? k1[u] : k0[u];
-        sl += 0.5f + 0.5f * erf_as7126(__fdividef(li[u] - ex, sp[u]) * 0.70710678118654752f);
+    for (int r = 0; r < R; ++r) {
+      const int e = e0 + r;
+      float gi = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) gi = (id[j] == e) ? gv[j] : gi;
+      si[r] += gi;
+    }
+    if (want_load) {  // uniform over the grid
+      // every load of the group first (a lane past the run or an expert past E reads an
+      // in-range element and discards it), then the arithmetic: the kernel is bound by
+      // load latency, not by bytes
+      const int64_t tt = tv ? t : t_hi - 1;
+      const float k0 = __ldg(kw + tt), k1 = __ldg(kw + T + tt);
+      float li[R], sp[R], H[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int64_t i = static_cast<int64_t>(min(e0 + r, E - 1)) * T + tt;
+        li[r] = __ldg(lw + i);
+        sp[r] = __ldg(sw + i);
+        H[r] = __ldg(hw + i);
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float ex = (H[r] >= k0) ? k1 : k0;
+        const float pl = 0.5f + 0.5f * erf_as7126(__fdividef(li[r] - ex, sp[r]) * 0.70710678118654752f);
+        sl[r] += (tv && e0 + r < E) ? pl : 0.0f;
       }
     }
   }
+  // column sums over the lanes, 8 experts at a time
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    si += __shfl_xor_sync(0xffffffffu, si, o);
-    sl += __shfl_xor_sync(0xffffffffu, sl, o);
-  }
-  if (lane == 0) {
-    partials[(blockIdx.x * 2 + 0) * static_cast<int64_t>(E) + e] = si;
-    partials[(blockIdx.x * 2 + 1) * static_cast<int64_t>(E) + e] = sl;
+  for (int g8 = 0; g8 < R / 8; ++g8) {
+    float a8[8], b8[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      a8[j] = si[8 * g8 + j];
+      b8[j] = sl[8 * g8 + j];
+    }
+    const float ci = warp_colsum8(a8, lane);
+    const float cl = warp_colsum8(b8, lane);
+    const int e = e0 + 8 * g8 + colsum8_column(lane);
+    if (lane < 8 && e < E) {
+      partials[(blockIdx.x * 2 + 0) * static_cast<int64_t>(E) + e] = ci;
+      partials[(blockIdx.x * 2 + 1) * static_cast<int64_t>(E) + e] = cl;
+    }
   }
 }
 
@@ -1158,27 +1181,33 @@ static cudaError_t launch_route_tc_hier(int kg, const CUtensorMap& tmX, const CU
 // Noisy gating on the tensor-core path with Importance or Load asked for: after the
 // router kernel, the sums over the whole grid (importance_load_kernel), then the fixed-
 // order total over the chunks.
+template <int R>
+static cudaError_t launch_importance_load_r(const RouteProblem& p, int64_t chunks, int64_t per,
+                                           const LaunchCtx& c) {
+  const int slices = (p.E + 8 * R - 1) / (8 * R);
+  return launch_kernel(importance_load_kernel<R>, dim3(static_cast<unsigned>(chunks), slices),
+                       dim3(256), 0, c, static_cast<const float*>(p.lw),
+                       static_cast<const float*>(p.sw), static_cast<const float*>(p.hw),
+                       static_cast<const float*>(p.kw), static_cast<const int32_t*>(p.topk_idx),
+                       static_cast<const float*>(p.topk_gate), p.T, p.E, p.k, per,
+                       p.load != nullptr ? 1 : 0, p.partials);
+}
+
 static cudaError_t launch_importance_load(const RouteProblem& p, const LaunchCtx& c) {
-  const int eb = (p.E + 7) / 8;
-  // one lane step per chunk where the grid stays within about eight blocks per SM (a
-  // 128-token chunk: each lane's four tokens), longer chunks of whole 128-token steps
-  // beyond; at most one chunk per 64 tokens (the partials' rows)
-  int64_t chunks = (p.T + 32 * kIlGroups - 1) / (32 * kIlGroups);
-  const int64_t most = (8LL * c.num_sms + eb - 1) / eb;
-  if (chunks > most) chunks = most;
+  // experts per warp: a block's eight warps cover up to 8R experts
+  const int R = p.E <= 64 ? 8 : 16;
+  const int slices = (p.E + 8 * R - 1) / (8 * R);
+  // token runs of whole 32-token groups, about two blocks per SM, at most one run per
+  // 64 tokens (the partials' rows)
+  int64_t chunks = (2LL * c.num_sms + slices - 1) / slices;
   const int64_t cap = route_blocks(p.T);
   if (chunks > cap) chunks = cap;
   if (chunks < 1) chunks = 1;
   int64_t per = (p.T + chunks - 1) / chunks;
-  per = (per + 32 * kIlGroups - 1) / (32 * kIlGroups) * (32 * kIlGroups);
+  per = per < 32 ? 32 : (per + 31) / 32 * 32;
   chunks = (p.T + per - 1) / per;
-  cudaError_t e = launch_kernel(importance_load_kernel, dim3(static_cast<unsigned>(chunks), eb),
-                                dim3(256), 0, c, static_cast<const float*>(p.lw),
-                                static_cast<const float*>(p.sw), static_cast<const float*>(p.hw),
-                                static_cast<const float*>(p.kw),
-                                static_cast<const int32_t*>(p.topk_idx),
-                                static_cast<const float*>(p.topk_gate), p.T, p.E, p.k, per,
-                                p.load != nullptr ? 1 : 0, p.partials);
+  cudaError_t e = R == 8 ? launch_importance_load_r<8>(p, chunks, per, c)
+                         : launch_importance_load_r<16>(p, chunks, per, c);
   if (e != cudaSuccess) return e;
   return launch_kernel(finalize_importance_load_kernel, dim3(p.E, 2), dim3(256), 0, c,
                        static_cast<const float*>(p.partials), static_cast<int>(chunks), p.E,
