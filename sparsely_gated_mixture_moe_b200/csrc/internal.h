@@ -144,7 +144,7 @@ struct PermuteProblem {
                     // path (null: always use the three-kernel path)
 };
 int64_t permute_blocks(int64_t n);
-int64_t permute_count_chunks(int64_t n);
+int64_t permute_count_ints(int64_t n, int E);
 cudaError_t launch_permute(const PermuteProblem& p, const LaunchCtx& c);
 cudaError_t launch_wait_timeout_check(int32_t* sync, int* err, const LaunchCtx& c);
 

@@ -68,7 +68,7 @@ Layout layout(const moe_config* c) {
   L.err = o;
   o = align_up(o + 16);
   L.blk = o;
-  o = align_up(o + static_cast<size_t>(permute_count_chunks(n)) * c->E * 4);
+  o = align_up(o + static_cast<size_t>(permute_count_ints(n, c->E)) * 4);
   L.partials = o;
   o = align_up(o + static_cast<size_t>(route_blocks(c->T)) * 2 * c->E * 4);
   L.logits = o;

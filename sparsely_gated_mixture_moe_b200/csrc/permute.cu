@@ -34,10 +34,14 @@ static_assert(kPermChunk == THREADS, "one assignment per thread per chunk");
 }  // namespace pm
 
 int64_t permute_blocks(int64_t n) { return (n + kPermChunk - 1) / kPermChunk; }
-// Chunks of the per-chunk count array the workspace must hold: the three-kernel path uses
-// ceil(n / 256) chunks of 256 assignments, the one-launch path at most ceil(n / 128),
-// padded to a multiple of 4.
-int64_t permute_count_chunks(int64_t n) { return (n + 127) / 128 + 3; }
+// Ints of the per-chunk count array the workspace must hold: the three-kernel path uses
+// ceil(n / 256) chunks of 256 assignments by E experts, the one-launch path at most
+// ceil(n / 128) chunks by E rounded up to a multiple of 4.
+int64_t permute_count_ints(int64_t n, int E) {
+  const int64_t three = permute_blocks(n) * E;
+  const int64_t fused = (n + 127) / 128 * ((E + 3) & ~3);
+  return three > fused ? three : fused;
+}
 
 // Shared memory of perm_count_scan_kernel: hist[E] and, for the scan, seg[2][256] and
 // kept[E] ints.
@@ -202,12 +206,13 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
 // assignments, one per block of 1024 threads; all blocks are resident at once (the grid
 // never exceeds what the occupancy query says fits).
 //   phase 1  the block ranks its chunk stably (warp match + per-warp prefix, kept in
-//            registers and shared memory) and writes its per-expert counts to blk[e][c]
-//            (rows padded to a multiple of 4 chunks, the padding zeroed by block 0, so
-//            that phase 2 reads them as 16-byte vectors)
+//            registers and shared memory) and writes its per-expert counts to row c of
+//            blk [nchunks][Ep] (Ep = E rounded up to a multiple of 4, the padding zeroed,
+//            so that phase 2 reads the rows as 16-byte vectors)
 //   barrier
-//   phase 2  the block sums column e of blk below its chunk (its rank base) and over all
-//            chunks (the expert's count), scans min(count, C) into offsets (block 0
+//   phase 2  the block sums column e of blk over the rows below its chunk (its rank base)
+//            and over all rows (the expert's count), reading whole rows (a warp reads
+//            512 contiguous bytes), scans min(count, C) into offsets (block 0
 //            writes counts and offsets), writes slot_pos and perm_src for its chunk, and
 //            copies its kept rows x[a / k] -> x_perm[slot] (16-byte vectors, two rows
 //            per warp in flight).  Every block redoes the small column sums itself, so
@@ -220,7 +225,8 @@ constexpr int WARPS = THREADS / 32;
 }  // namespace pf
 
 static size_t fused_smem(int E) {
-  return (static_cast<size_t>(pf::WARPS) * E + 3 * static_cast<size_t>(E) + 3 * pf::THREADS + 64) * 4;
+  return (8 * pf::THREADS + static_cast<size_t>(pf::WARPS) * E + 3 * static_cast<size_t>(E) +
+          pf::THREADS + 64) * 4;
 }
 
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
@@ -258,14 +264,13 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                       int32_t* __restrict__ offsets, int32_t* __restrict__ perm_src,
                       int32_t* __restrict__ slot_pos, const uint8_t* __restrict__ x,
                       uint8_t* __restrict__ x_perm, int row_bytes, int32_t* sync, int* err) {
-  extern __shared__ int fsm[];
-  int* wbase = fsm;                     // [WARPS][E]: per-warp rank bases
+  extern __shared__ __align__(16) int fsm[];
+  int4* red = reinterpret_cast<int4*>(fsm);  // [2][THREADS]: column-sum partials
+  int* wbase = fsm + 8 * pf::THREADS;   // [WARPS][E]: per-warp rank bases
   int* s_pre = wbase + pf::WARPS * E;   // [E]: rank base of this chunk
   int* s_tot = s_pre + E;               // [E]: assignments per expert
   int* s_off = s_tot + E;               // [E]: offsets
-  int* segp = s_off + E;                // [THREADS]
-  int* segt = segp + pf::THREADS;       // [THREADS]
-  int* s_slot = segt + pf::THREADS;     // [THREADS]: slot of each assignment of the chunk
+  int* s_slot = s_off + E;              // [THREADS]: slot of each assignment of the chunk
   int* scratch = s_slot + pf::THREADS;  // [64]
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -296,53 +301,79 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     if (e >= 0 && (peers & lt_mask) == 0) wbase[warp * E + e] = __popc(peers);
   }
   __syncthreads();
-  const int ncs = (nchunks + 3) & ~3;  // padded row length of blk
-  for (int xe = tid; xe < E; xe += pf::THREADS) {
+  const int Ep = (E + 3) & ~3;  // row length of blk
+  for (int xe = tid; xe < Ep; xe += pf::THREADS) {
     int run = 0;
-    for (int w = 0; w < nw; ++w) {
-      const int v = wbase[w * E + xe];
-      wbase[w * E + xe] = run;
-      run += v;
-    }
-    blk[static_cast<int64_t>(xe) * ncs + c] = run;
-    if (c == 0)
-      for (int b = nchunks; b < ncs; ++b) blk[static_cast<int64_t>(xe) * ncs + b] = 0;
+    if (xe < E)
+      for (int w = 0; w < nw; ++w) {
+        const int v = wbase[w * E + xe];
+        wbase[w * E + xe] = run;
+        run += v;
+      }
+    blk[static_cast<int64_t>(c) * Ep + xe] = run;
   }
   const bool ok = grid_barrier(sync, nchunks, err, &s_abort);
 
   // ---- phase 2: rank bases, counts, offsets; slot_pos, perm_src and rows of this chunk
   if (ok) {
-    int tpe = 1;  // threads per expert, each summing a run of 4-chunk vectors
-    while (tpe * 2 * E <= pf::THREADS) tpe *= 2;
-    const int epr = pf::THREADS / tpe;  // experts per round
-    const int nq = ncs >> 2;
-    const int len = (nq + tpe - 1) / tpe;
-    for (int e0 = 0; e0 < E; e0 += epr) {
-      const int el = tid % epr, part = tid / epr, xe = e0 + el;
-      int pre = 0, tot = 0;
-      if (xe < E) {
-        const int q0 = part * len, q1 = min(nq, q0 + len);
-        const int4* col = reinterpret_cast<const int4*>(blk + static_cast<int64_t>(xe) * ncs);
+    // thread (row group rg, column quad q) sums rows rg, rg + RG, ... of its four columns;
+    // then the first row group adds up the RG partials (integer sums: any order is exact)
+    const int NQ = Ep >> 2;
+    const int4* rows = reinterpret_cast<const int4*>(blk);
+    for (int qb = 0; qb < NQ; qb += pf::THREADS) {
+      const int nqb = min(NQ - qb, pf::THREADS);
+      const int RG = pf::THREADS / nqb;
+      const int q = qb + tid % nqb, rg = tid / nqb;
+      int4 pre = make_int4(0, 0, 0, 0), tot = make_int4(0, 0, 0, 0);
+      if (rg < RG) {
 #pragma unroll 4
-        for (int qi = q0; qi < q1; ++qi) {
-          const int4 v = __ldcg(col + qi);
-          const int b = 4 * qi;
-          tot += v.x + v.y + v.z + v.w;
-          pre += (b < c ? v.x : 0) + (b + 1 < c ? v.y : 0) + (b + 2 < c ? v.z : 0) +
-                 (b + 3 < c ? v.w : 0);
+        for (int r = rg; r < nchunks; r += RG) {
+          const int4 v = __ldcg(rows + static_cast<int64_t>(r) * NQ + q);
+          tot.x += v.x;
+          tot.y += v.y;
+          tot.z += v.z;
+          tot.w += v.w;
+          if (r < c) {
+            pre.x += v.x;
+            pre.y += v.y;
+            pre.z += v.z;
+            pre.w += v.w;
+          }
         }
       }
-      segp[tid] = pre;
-      segt[tid] = tot;
+      red[tid] = pre;
+      red[pf::THREADS + tid] = tot;
       __syncthreads();
-      if (part == 0 && xe < E) {
-        int P = 0, S = 0;
-        for (int q = 0; q < tpe; ++q) {
-          P += segp[q * epr + el];
-          S += segt[q * epr + el];
+      if (tid < nqb) {
+        int4 P = make_int4(0, 0, 0, 0), S = make_int4(0, 0, 0, 0);
+        for (int g = 0; g < RG; ++g) {
+          const int4 a = red[g * nqb + tid], b = red[pf::THREADS + g * nqb + tid];
+          P.x += a.x;
+          P.y += a.y;
+          P.z += a.z;
+          P.w += a.w;
+          S.x += b.x;
+          S.y += b.y;
+          S.z += b.z;
+          S.w += b.w;
         }
-        s_pre[xe] = P;
-        s_tot[xe] = S;
+        const int e4 = 4 * (qb + tid);
+        if (e4 < E) {
+          s_pre[e4] = P.x;
+          s_tot[e4] = S.x;
+        }
+        if (e4 + 1 < E) {
+          s_pre[e4 + 1] = P.y;
+          s_tot[e4 + 1] = S.y;
+        }
+        if (e4 + 2 < E) {
+          s_pre[e4 + 2] = P.z;
+          s_tot[e4 + 2] = S.z;
+        }
+        if (e4 + 3 < E) {
+          s_pre[e4 + 3] = P.w;
+          s_tot[e4 + 3] = S.w;
+        }
       }
       __syncthreads();
     }
