@@ -185,8 +185,9 @@ def algorithmic(w: workloads.Workload, n_kept: int, counts_kept, fused=False):
     weights, noise, and the chosen indices and gates.  Permute: the chosen experts read,
     slot_pos and perm_src written, counts and offsets, and the kept token rows read from
     x and written to x_perm.  Combine: y_perm rows read, gates and slots, y written (in
-    the output type of y_bf16_of).  fused (k = 1, FFN and combine as one step): the FFN
-    writes every row of y and reads each kept row's source index and gate; no combine
+    the output type of y_bf16_of).  fused (FFN and combine as one step): the FFN writes
+    every row of y and reads each kept row's source index and gate; for k = 2 it also adds
+    each kept row into its token's row of y (the up-projection zeroes y); no combine
     bytes."""
     es = 2 if w.dtype == "bf16" else 4
     ys = 2 if y_bf16_of(w) else 4
@@ -199,7 +200,8 @@ def algorithmic(w: workloads.Workload, n_kept: int, counts_kept, fused=False):
     permute_bytes = T * k * 4 * 3 + E * 8.0 + n_kept * d * es * 2
     combine_bytes = n_kept * d * 4.0 + T * k * 8 + T * d * float(ys)
     if fused:
-        ffn_bytes = active * 2.0 * d * f * es + n_kept * d * es + T * d * float(ys) + n_kept * 8.0 + T * 4.0
+        ffn_bytes = active * 2.0 * d * f * es + n_kept * d * es + T * d * float(ys) + n_kept * 8.0
+        ffn_bytes += n_kept * d * 4.0 if k == 2 else T * 4.0
         combine_bytes = 0.0
     return {"ffn_flops": ffn_flops, "ffn_bytes": ffn_bytes, "route_bytes": route_bytes,
             "permute_bytes": permute_bytes, "combine_bytes": combine_bytes}
@@ -335,7 +337,8 @@ class LayerBench:
         o["importance"] = torch.empty(E, dtype=torch.float32, device=dev) if self.noisy else None
         o["load"] = torch.empty(E, dtype=torch.float32, device=dev) if self.noisy and k < E else None
         self.ws = moe.workspace(self.cfg, dev)
-        self.fused = moe.fused_combine(self.cfg)
+        # FFN and combine as one call where moe_forward takes it (top-1)
+        self.fused = moe.fused_combine(self.cfg) and self.cfg.k == 1
         self.stream = torch.cuda.current_stream(dev)
         self.launches = 0
 

@@ -75,7 +75,7 @@ enum {
   MOE_DEVERR_EXPERT_INDEX = 1, /* a topk_idx entry outside [0, E): treated as dropped */
   MOE_DEVERR_OFFSETS = 2,      /* offsets not non-decreasing in [0, T*k]: FFN skipped */
   MOE_DEVERR_SLOT = 4,         /* a slot_pos entry outside [-1, T*k), or a perm_src entry
-                                  outside [0, T) in moe_expert_ffn_combine: treated as
+                                  outside [0, T*k) in moe_expert_ffn_combine: treated as
                                   dropped (that row is not written) */
   MOE_DEVERR_TIMEOUT = 8       /* a bounded wait inside a pipelined kernel expired */
 };
@@ -251,19 +251,26 @@ moe_status moe_expert_ffn_gather(const moe_config* cfg, const void* x, const int
 moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* slot_pos,
                        const float* topk_gate, void* y, void* ws, moe_stream_t stream);
 
-/* moe_expert_ffn followed by moe_combine as one step, for k = 1 and bf16 only [Switch
- * Transformer, switch_routing: with one expert per token the combine is a scaled copy]:
- *   y[t] = topk_gate[t] * (act(x[t] . W1_e^T) . W2_e^T)  for a token kept by expert e,
- *   y[t] = 0                                            for a token that was dropped.
- * The down-projection writes each fp32 row straight into y at its token (perm_src[s] = t
- * for k = 1), so y_perm never exists.  Same arithmetic as the two steps: y is bit-equal
- * to moe_expert_ffn + moe_combine on the same inputs.
+/* moe_expert_ffn followed by moe_combine as one step, in bf16 for k = 1, and for k = 2
+ * with an fp32 y [Switch Transformer, switch_routing: with one expert per token the
+ * combine is a scaled copy; Shazeer et al., "Methode": y = sum_i G(x)_i E_i(x)]:
+ *   y[t] = sum over t's kept assignments a of topk_gate[a] * (act(x[t] . W1_e^T) . W2_e^T)
+ *   (y[t] = 0 for a token all of whose assignments were dropped).
+ * The down-projection puts each gate-weighted fp32 row straight into y at its token
+ * (token = perm_src[s] / k), so y_perm never exists.  k = 1: a store; the rows of dropped
+ * tokens are zeroed by the down-projection's epilogue threads before its first tile.
+ * k = 2: the up-projection's epilogue threads zero y (a 16 KB chunk per CTA and tile) and
+ * the down-projection adds each rounded product into the row in memory; the two adds of a
+ * token commute, so y does not depend on their order.  For k = 1 y is bit-equal to
+ * moe_expert_ffn + moe_combine on the same inputs; for k = 2 it differs from it by at most
+ * the rounding of one product (moe_combine folds the second product into a fused
+ * multiply-add).
  *  x_perm, offsets, w1, w2, h as moe_expert_ffn;  perm_src, slot_pos as written by
- *  moe_permute;  topk_gate [T, 1] fp32 in;  y [T, d_model] fp32 out, bf16 with
- *  cfg->y_bf16 (every row written).
- * The rows of dropped tokens (slot_pos[t] < 0) are zeroed by the down-projection's
- * epilogue threads before its first tile; a perm_src entry outside [0, T) sets
- * MOE_DEVERR_SLOT.  * Returns MOE_ERR_UNSUPPORTED when k != 1 or dtype is not bf16. */
+ *  moe_permute;  topk_gate [T, k] fp32 in;  y [T, d_model] fp32 out, bf16 with
+ *  cfg->y_bf16 for k = 1 (every row written).
+ * A perm_src entry outside [0, T*k) sets MOE_DEVERR_SLOT (that row is not written).
+ * Returns MOE_ERR_UNSUPPORTED unless dtype is bf16 and k == 1, or k == 2 without
+ * cfg->y_bf16. */
 moe_status moe_expert_ffn_combine(const moe_config* cfg, const void* x_perm,
                                   const int32_t* offsets, const int32_t* perm_src,
                                   const int32_t* slot_pos, const float* topk_gate,
@@ -271,7 +278,7 @@ moe_status moe_expert_ffn_combine(const moe_config* cfg, const void* x_perm,
                                   moe_stream_t stream);
 
 /* moe_expert_ffn_combine with the permuted rows gathered from the token rows x (as
- * moe_expert_ffn_gather does) instead of read from x_perm; k = 1 and bf16 only.
+ * moe_expert_ffn_gather does) instead of read from x_perm; the same k and dtype rules.
  *  x [T, d_model] bf16 in; the other arguments as moe_expert_ffn_combine.  y is
  *  bit-identical to moe_expert_ffn_combine's on x_perm. */
 moe_status moe_expert_ffn_combine_gather(const moe_config* cfg, const void* x,
@@ -282,7 +289,7 @@ moe_status moe_expert_ffn_combine_gather(const moe_config* cfg, const void* x,
 
 /* The whole layer forward on one stream: moe_route, moe_permute, moe_expert_ffn,
  * moe_combine (moe_expert_ffn_combine in place of the last two when k = 1 and dtype is
- * bf16).  Inputs as in the step calls; y [T, d_model] fp32 (bf16 with cfg->y_bf16) out.  topk_idx,
+ * bf16; for k = 2 its fused form is not faster, so the two steps run).  Inputs as in the step calls; y [T, d_model] fp32 (bf16 with cfg->y_bf16) out.  topk_idx,
  * topk_gate (both [T, k]) and counts ([E]) are outputs the caller must provide;
  * importance, load and near_tie may be NULL.  The intermediates live in `ws`
  * (moe_forward_workspace_size bytes). */

@@ -169,7 +169,7 @@ def moe_expert_ffn_gather(cfg, x, perm_src, offsets, w1, w2, h, y_perm, ws, stre
 
 def moe_expert_ffn_combine_gather(cfg, x, offsets, perm_src, slot_pos, topk_gate, w1, w2, h, y,
                                   ws, stream=None):
-    """moe_expert_ffn_combine with the permuted rows gathered from x (k = 1, bf16)."""
+    """moe_expert_ffn_combine with the permuted rows gathered from x."""
     _check(lib.moe_expert_ffn_combine_gather(
         ctypes.byref(cfg), _ptr(x, "x"), _ptr(offsets, "offsets"), _ptr(perm_src, "perm_src"),
         _ptr(slot_pos, "slot_pos"), _ptr(topk_gate, "topk_gate"), _ptr(w1, "w1"), _ptr(w2, "w2"),
@@ -185,8 +185,9 @@ def moe_combine(cfg, y_perm, slot_pos, topk_gate, y, ws, stream=None):
 
 def moe_expert_ffn_combine(cfg, x_perm, offsets, perm_src, slot_pos, topk_gate, w1, w2, h, y,
                            ws, stream=None):
-    """moe_expert_ffn + moe_combine as one step (k = 1, bf16): the down-projection writes
-    gate * row straight into y at its token."""
+    """moe_expert_ffn + moe_combine as one step (bf16; k = 1, or k = 2 with an fp32 y): the
+    down-projection puts gate * row straight into y at its token (a store for k = 1, an
+    in-memory add onto the row the up-projection zeroed for k = 2)."""
     _check(lib.moe_expert_ffn_combine(ctypes.byref(cfg), _ptr(x_perm, "x_perm"),
                                       _ptr(offsets, "offsets"), _ptr(perm_src, "perm_src"),
                                       _ptr(slot_pos, "slot_pos"), _ptr(topk_gate, "topk_gate"),
@@ -195,8 +196,9 @@ def moe_expert_ffn_combine(cfg, x_perm, offsets, perm_src, slot_pos, topk_gate, 
 
 
 def fused_combine(cfg) -> bool:
-    """Whether moe_expert_ffn_combine applies (top-1 routing in bf16)."""
-    return cfg.k == 1 and cfg.dtype == DTYPE["bf16"]
+    """Whether moe_expert_ffn_combine applies: bf16 with top-1 routing, or top-2 with an
+    fp32 layer output."""
+    return cfg.dtype == DTYPE["bf16"] and (cfg.k == 1 or (cfg.k == 2 and not cfg.y_bf16))
 
 
 def moe_forward(cfg, x, w_gate, w1, w2, y, topk_idx, topk_gate, counts, ws, w_noise=None,

@@ -69,6 +69,10 @@ constexpr int OUT_F16 = 1;   // act, fp16
 constexpr int OUT_F32 = 2;   // fp32
 constexpr int OUT_COMBINE = 3;  // fp32 times the gate, into the token's row of y (k = 1)
 constexpr int OUT_COMBINE_BF16 = 4;  // as OUT_COMBINE, y in bf16 (the scaled fp32 rounded)
+constexpr int OUT_COMBINE_ADD = 5;   // fp32 times the gate, added in memory into the token's
+                                     // row of y (k = 2; y zeroed by the up-projection)
+// 16-byte vectors of a zeroing chunk: two per epilogue thread
+constexpr int ZERO_CHUNK_VECS = EPI_WARPS * 32 * 2;
 
 struct Args {
   const int32_t* offsets;
@@ -82,7 +86,8 @@ struct Args {
   int act;       // 0 none, 1 ReLU, 2 GELU
   int out_mode;  // OUT_*
   int ab_f16;    // operand type of A and B: 1 fp16, 0 bf16
-  const int32_t* perm_src;  // OUT_COMBINE*: assignment of each permuted row (= token, k = 1)
+  const int32_t* perm_src;  // OUT_COMBINE*: assignment t*comb_k + j of each permuted row
+  int comb_k;               // OUT_COMBINE*: assignments per token
   const float* gate;        // OUT_COMBINE*: gate of each assignment
   const int32_t* slot_pos;  // OUT_COMBINE*: permuted row of each token, < 0 when dropped
   const int32_t* gather_src;  // non-null: A row s is row gather_src[s] / gather_k of the
@@ -91,6 +96,8 @@ struct Args {
                               // pre-activation there (same type and layout as out), or null
   int w_mod;                  // row group g multiplies weight block g % w_mod (w_mod >= E:
                               // group g uses block g)
+  float4* zero_out;           // non-null: the epilogue threads also zero zero_out[0, zero_vecs)
+  int64_t zero_vecs;          // (16-byte vectors), one chunk per CTA and tile
   int* err;
 };
 
@@ -143,6 +150,18 @@ __device__ __forceinline__ void epilogue_rows(const Args& a, uint32_t tbase, int
       uint16_t* dst = static_cast<uint16_t*>(a.out) + oidx + c;  // 64-byte aligned
       st_global_v8(dst, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
       st_global_v8(dst + 16, pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14], pk[15]);
+    } else if (MODE == OUT_COMBINE_ADD) {
+      // the token's other assignment adds its row too: the two in-memory adds onto the
+      // zeroed row commute, so y does not depend on which lands first
+      float* dst = static_cast<float*>(a.out) + oidx + c;  // 128-byte aligned
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4 * j),
+                     "f"(__fmul_rn(scale, __uint_as_float(v[4 * j]))),
+                     "f"(__fmul_rn(scale, __uint_as_float(v[4 * j + 1]))),
+                     "f"(__fmul_rn(scale, __uint_as_float(v[4 * j + 2]))),
+                     "f"(__fmul_rn(scale, __uint_as_float(v[4 * j + 3])))
+                     : "memory");
     } else if (MODE == OUT_F32 || MODE == OUT_COMBINE) {
       float* dst = static_cast<float*>(a.out) + oidx + c;  // 128-byte aligned
       if (MODE == OUT_COMBINE) {
@@ -439,8 +458,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int q = warp & 3;               // TMEM lane quarter this warp may read
     const int sub = (warp - 2) >> 2;      // which 32-column chunks: sub*32 + 128*i
     const int mode = a.out_mode * 3 + a.act;
-    const bool combine = a.out_mode == OUT_COMBINE || a.out_mode == OUT_COMBINE_BF16;
-    if (combine) {
+    const bool combine = a.out_mode == OUT_COMBINE || a.out_mode == OUT_COMBINE_BF16 ||
+                         a.out_mode == OUT_COMBINE_ADD;
+    // zeroing of zero_out: chunk blockIdx.x + i * gridDim.x after this CTA's i-th tile,
+    // the chunks left after its last tile at the end
+    int64_t zc = blockIdx.x;
+    const int64_t zchunks = a.zero_out != nullptr
+                                ? (a.zero_vecs + ZERO_CHUNK_VECS - 1) / ZERO_CHUNK_VECS : 0;
+    auto zero_chunk = [&]() {
+      const int64_t v0 = zc * ZERO_CHUNK_VECS + (warp - 2) * 64 + lane * 2;
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        if (v0 + u < a.zero_vecs) a.zero_out[v0 + u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      zc += gridDim.x;
+    };
+    if (a.out_mode == OUT_COMBINE || a.out_mode == OUT_COMBINE_BF16) {
       // y = 0 for tokens whose only assignment was dropped (no tile writes them); done
       // while the first tile's operands stream in
       const int row_vec = a.out_mode == OUT_COMBINE ? a.N / 4 : a.N / 8;  // 16-byte vectors
@@ -475,14 +507,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       int64_t orow = t.row0 + crow;
       float scale = 1.0f;
       if (combine && row_ok) {
-        // k = 1: the permuted row's assignment is its token; y[t] = g_t * (h W2^T)[row]
+        // the permuted row's assignment a = t*comb_k + j: y[t] gets g_a * (h W2^T)[row]
         const int asg = __ldg(a.perm_src + orow);
         if (asg < 0 || asg >= a.rows_cap) {
           set_error(a.err, kErrSlot);  // not a permutation written by the permute step
           row_ok = false;
         } else {
           scale = __ldg(a.gate + asg);
-          orow = asg;
+          orow = asg / a.comb_k;
         }
       }
       const int64_t oidx = orow * a.N + t.nt * a.bn;
@@ -496,6 +528,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           case OUT_F16 * 3 + 2: epilogue_rows<OUT_F16, 2>(a, tbase, oidx, sub, row_ok, scale); break;
           case OUT_COMBINE * 3 + 0: epilogue_rows<OUT_COMBINE, 0>(a, tbase, oidx, sub, row_ok, scale); break;
           case OUT_COMBINE_BF16 * 3 + 0: epilogue_rows<OUT_COMBINE_BF16, 0>(a, tbase, oidx, sub, row_ok, scale); break;
+          case OUT_COMBINE_ADD * 3 + 0: epilogue_rows<OUT_COMBINE_ADD, 0>(a, tbase, oidx, sub, row_ok, scale); break;
           default: epilogue_rows<OUT_F32, 0>(a, tbase, oidx, sub, row_ok, scale); break;
         }
       }
@@ -507,7 +540,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
+      if (zc < zchunks) zero_chunk();
     }
+    while (zc < zchunks) zero_chunk();
   }
 
   __syncwarp();
@@ -607,7 +642,8 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
                               const LaunchCtx& c, const int32_t* perm_src = nullptr,
                               const float* gate = nullptr, const int32_t* slot_pos = nullptr,
                               const int32_t* gather_src = nullptr, int gather_k = 1,
-                              int64_t a_rows = 0, void* pre = nullptr, int w_count = 0) {
+                              int64_t a_rows = 0, void* pre = nullptr, int w_count = 0,
+                              int comb_k = 1, void* zero_out = nullptr, int64_t zero_bytes = 0) {
   const int bn = pick_bn(N);
   const int wb = w_count > 0 ? w_count : E;  // weight blocks of B
   const bool pair = rows_cap >= kPairMinRowsPerExpert * E;
@@ -641,6 +677,9 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
   a.gather_k = gather_k;
   a.pre = pre;
   a.w_mod = wb;
+  a.comb_k = comb_k;
+  a.zero_out = static_cast<float4*>(zero_out);
+  a.zero_vecs = zero_out != nullptr ? zero_bytes / 16 : 0;
   a.err = c.err;
   // upper bound of the tile count: sum_e ceil(n_e / bm) <= rows_cap / bm + E
   const int tbm = pair ? 2 * gg::BM : gg::BM;
@@ -664,14 +703,18 @@ static cudaError_t launch_one(const void* A, int64_t rows_cap, int K, const void
 
 // The up-projection h = act(A . W1^T): A is x_perm, or the token rows x gathered by the
 // TMA through gather_src (no x_perm).
-static cudaError_t launch_up(const FfnProblem& p, const LaunchCtx& c) {
+// zero_out / zero_bytes: a buffer (16-byte multiple) the epilogue threads also zero.
+static cudaError_t launch_up(const FfnProblem& p, const LaunchCtx& c, void* zero_out = nullptr,
+                             int64_t zero_bytes = 0) {
   const int hf = p.hidden_f16 ? 1 : 0;
   const int mode = hf ? gg::OUT_F16 : gg::OUT_BF16;
   if (p.gather_src != nullptr)
     return launch_one(p.x, p.rows_cap, p.d, p.w1, p.E, p.f, 0, p.h, mode, p.offsets, p.act, c,
-                      nullptr, nullptr, nullptr, p.gather_src, p.k, p.x_rows, p.u, p.w_count);
+                      nullptr, nullptr, nullptr, p.gather_src, p.k, p.x_rows, p.u, p.w_count, 1,
+                      zero_out, zero_bytes);
   return launch_one(p.x_perm, p.rows_cap, p.d, p.w1, p.E, p.f, 0, p.h, mode, p.offsets, p.act, c,
-                    nullptr, nullptr, nullptr, nullptr, 1, 0, p.u, p.w_count);
+                    nullptr, nullptr, nullptr, nullptr, 1, 0, p.u, p.w_count, 1, zero_out,
+                    zero_bytes);
 }
 
 cudaError_t launch_ffn_combine_bf16(const FfnProblem& p, const int32_t* perm_src,
@@ -679,6 +722,17 @@ cudaError_t launch_ffn_combine_bf16(const FfnProblem& p, const int32_t* perm_src
                                     const LaunchCtx& c) {
   if (p.E > gg::MAX_GROUPS) return cudaErrorInvalidValue;
   const int hf = p.hidden_f16 ? 1 : 0;
+  if (p.k == 2) {
+    // y = 0 by the up-projection's epilogue threads (one 16 KB chunk per CTA and tile, in
+    // time with the tensor-core work), then each kept row added into its token's row
+    if (p.y_bf16) return cudaErrorInvalidValue;
+    const int64_t y_bytes = p.rows_cap / 2 * p.d * 4;
+    cudaError_t e = launch_up(p, c, y, y_bytes);
+    if (e != cudaSuccess) return e;
+    return launch_one(p.h, p.rows_cap, p.f, p.w2, p.E, p.d, hf, y, gg::OUT_COMBINE_ADD, p.offsets,
+                      0, c, perm_src, gate, slot_pos, nullptr, 1, 0, nullptr, 0, 2);
+  }
+  if (p.k != 1) return cudaErrorInvalidValue;
   cudaError_t e = launch_up(p, c);
   if (e != cudaSuccess) return e;
   return launch_one(p.h, p.rows_cap, p.f, p.w2, p.E, p.d, hf, y,

@@ -169,9 +169,10 @@ struct FfnProblem {
 };
 cudaError_t launch_ffn_bf16(const FfnProblem& p, const LaunchCtx& c);
 cudaError_t launch_ffn_f32(const FfnProblem& p, const LaunchCtx& c);
-// k = 1, bf16: expert FFN whose down-projection writes y[t] = gate[t] * row directly (its
-// epilogue also zeroes the rows of dropped tokens) instead of y_perm; y in fp32, or bf16
-// with p.y_bf16.
+// bf16 expert FFN whose down-projection forms y itself instead of y_perm.  k = 1: it
+// writes y[t] = gate[t] * row (its epilogue also zeroes the rows of dropped tokens); y in
+// fp32, or bf16 with p.y_bf16.  k = 2 (fp32 y): the up-projection's epilogue threads zero
+// y and the down-projection adds gate * row into its token's row in memory.
 cudaError_t launch_ffn_combine_bf16(const FfnProblem& p, const int32_t* perm_src,
                                     const int32_t* slot_pos, const float* gate, void* y,
                                     const LaunchCtx& c);

@@ -364,7 +364,7 @@ moe_status do_ffn_combine(const moe_config* cfg, const void* x_perm, const int32
   p.gather_src = gather ? perm_src : nullptr;
   p.x_rows = cfg->T;
   p.k = cfg->k;
-  p.rows_cap = cfg->T;  // k = 1
+  p.rows_cap = cfg->T * cfg->k;
   p.d = cfg->d_model;
   p.f = cfg->d_ff;
   p.E = cfg->E;
@@ -381,7 +381,11 @@ moe_status do_ffn_combine(const moe_config* cfg, const void* x_perm, const int32
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-bool fused_combine(const moe_config* cfg) { return cfg->k == 1 && cfg->dtype == MOE_BF16; }
+// FFN and combine as one step: bf16 with k = 1 (the combine is a scaled store), or k = 2
+// with an fp32 y (two in-memory adds per row, which commute)
+bool fused_combine(const moe_config* cfg) {
+  return cfg->dtype == MOE_BF16 && (cfg->k == 1 || (cfg->k == 2 && !cfg->y_bf16));
+}
 
 // T == 0: nothing to route; zero the per-expert outputs that are defined anyway.
 moe_status empty_batch(const moe_config* cfg, int32_t* counts, int32_t* offsets, float* importance,
@@ -665,7 +669,9 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_gate,
   // faster than gathering them inside the up-projection (tile::gather4)
   st = do_permute(cfg, L, topk_idx, x, counts, offsets, perm_src, slot_pos, x_perm, ws, ctx);
   if (st != MOE_OK) return st;
-  if (fused_combine(cfg)) {
+  // k = 1: the down-projection stores y itself.  k = 2 takes the two steps: its fused form
+  // (in-memory adds onto a zeroed y) measured no faster on zipf and 3% slower on gshard
+  if (cfg->k == 1 && fused_combine(cfg)) {
     st = do_ffn_combine(cfg, x_perm, offsets, perm_src, slot_pos, topk_gate, w1, w2, h, y, ctx);
     if (st != MOE_OK) return st;
     return ctx.finish(cudaSuccess);

@@ -332,9 +332,24 @@ def check_combine(w, g, report, rows=None):
     assert e <= TOL["f32"], e
     report["combine_err"] = e
     if "y_fused" in g:
-        # one fp32 product g * row on both paths (k = 1): equal value for value
-        assert torch.equal(g["y_fused"], g["y"]), float((g["y_fused"] - g["y"]).abs().max())
-        report["fused_combine"] = "equal"
+        if w.k == 1:
+            # one fp32 product g * row on both paths: equal value for value
+            assert torch.equal(g["y_fused"], g["y"]), float((g["y_fused"] - g["y"]).abs().max())
+            report["fused_combine"] = "equal"
+        else:
+            # k = 2: the fused path adds the two rounded products (in-memory adds, which
+            # commute); moe_combine folds the second product into its add (one FMA), so the
+            # two differ by at most the rounding of that product
+            yf, yc = g["y_fused"].double(), g["y"].double()
+            assert torch.isfinite(yf).all()
+            T_, k_ = w.T, w.k
+            sp = g["slot_pos"].long().view(T_, k_)
+            kept = (sp >= 0).double().unsqueeze(-1)
+            yp = g["y_perm"].double()[sp.clamp(min=0)]                     # [T, k, d]
+            mag = (g["topk_gate"].double().abs().view(T_, k_, 1) * yp.abs() * kept).sum(1)
+            bound = 2.0 ** -22 * mag            # two roundings of size <= 2^-24 |term| each
+            assert bool(((yf - yc).abs() <= bound).all()), float((yf - yc).abs().max())
+            report["fused_combine"] = "within one rounding"
 
 
 def oracle_layer_rows(w, inp, idx, gates, rows):

@@ -143,11 +143,16 @@ def test_other_steps_validation():
     assert moe.lib.moe_expert_ffn(c, P, P, P, P, FAKE_ODD, P, P, None) == 1
     assert moe.lib.moe_combine(c, P, None, P, P, P, None) == 1
     assert moe.lib.moe_combine(c, P, P, P, FAKE_ODD, P, None) == 1
-    # the fused FFN + combine step: k = 1 and bf16 only, then the usual argument checks
+    # the fused FFN + combine step: bf16 with k = 1, or k = 2 with an fp32 y; then the
+    # usual argument checks
     c1 = ctypes.byref(_cfg(k=1))
-    assert moe.lib.moe_expert_ffn_combine(c, P, P, P, P, P, P, P, P, P, P, None) == 2
-    assert moe.lib.moe_expert_ffn_combine(ctypes.byref(_cfg(k=1, dtype="f32")), P, P, P, P, P, P,
-                                          P, P, P, P, None) == 2
+    for bad in (_cfg(k=3), _cfg(k=2, y_bf16=True), _cfg(k=1, dtype="f32"), _cfg(k=2, dtype="f32")):
+        assert moe.lib.moe_expert_ffn_combine(ctypes.byref(bad), P, P, P, P, P, P, P, P, P, P,
+                                              None) == 2
+        assert moe.lib.moe_expert_ffn_combine_gather(ctypes.byref(bad), P, P, P, P, P, P, P, P, P,
+                                                     P, None) == 2
+    assert moe.fused_combine(_cfg(k=1)) and moe.fused_combine(_cfg(k=2))
+    assert not moe.fused_combine(_cfg(k=2, y_bf16=True)) and not moe.fused_combine(_cfg(k=4))
     assert moe.lib.moe_expert_ffn_combine(c1, P, P, None, P, P, P, P, P, P, P, None) == 1
     assert moe.lib.moe_expert_ffn_combine(c1, P, P, P, P, P, P, P, P, FAKE_ODD, P, None) == 1
     assert moe.lib.moe_forward(c, P, P, None, None, None, P, P, None, P, P, P, None, None, None,

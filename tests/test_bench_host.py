@@ -84,6 +84,13 @@ def test_algorithmic_counts_switch():
     f = bench.algorithmic(w, 16384, kept, fused=True)
     assert f["combine_bytes"] == 0.0
     assert f["ffn_bytes"] == weights + 16384 * 768 * 2 + 16384 * 768 * 4 + 16384 * 8 + 16384 * 4
+    # k = 2 fused: y zeroed (written once) and every kept row added into it
+    z = workloads.WORKLOADS["zipf"]
+    zk = [8192] * 16
+    fz = bench.algorithmic(z, 131072, zk, fused=True)
+    assert fz["combine_bytes"] == 0.0
+    assert fz["ffn_bytes"] == (16 * 2 * 1024 * 4096 * 2 + 131072 * 1024 * 2 + 65536 * 1024 * 4
+                               + 131072 * 8 + 131072 * 1024 * 4)
     bench.Y_BF16 = True
     try:
         assert bench.y_bf16_of(w) and not bench.y_bf16_of(workloads.WORKLOADS["tiny"])
