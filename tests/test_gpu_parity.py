@@ -421,6 +421,71 @@ def test_bf16_output_is_the_rounded_fp32_output(name):
         assert bool((y16.float().abs().sum(1) == 0).any())
 
 
+FUSED_K2 = {
+    # y (32 MB) in 2048 zeroing chunks against ~256 up-projection pair tiles: most chunks
+    # are zeroed after a CTA's last tile
+    "zero_tail_T8192": Workload("fk2", T=8192, d_model=1024, d_ff=1024, E=8, k=2, act="gelu"),
+    # capacity drops: tokens with one or no kept assignment (rows that only the zeroing
+    # writes), 128-row tiles
+    "drops_T6000": Workload("fk2c", T=6000, d_model=512, d_ff=512, E=32, k=2, act="relu",
+                            capacity_factor=0.6),
+    "zipf_full": W["zipf"],
+}
+
+
+@pytest.mark.parametrize("name", list(FUSED_K2))
+def test_fused_top2_combine_covers_every_row(name):
+    """moe_expert_ffn_combine with k = 2 into a y filled with NaN: the up-projection must
+    zero every row and the down-projection add each kept row into its token, so y is
+    finite everywhere, zero exactly for the tokens with no kept assignment, within one
+    rounding of the second product of moe_expert_ffn + moe_combine, and the same bits on
+    a second run (the two in-memory adds of a token commute)."""
+    import sparsely_gated_mixture_moe_b200 as moe
+    w = FUSED_K2[name]
+    dev = H.to_device(workloads.make_inputs(w))
+    cfg = H.config_of(w)
+    assert moe.fused_combine(cfg)
+    T, k, E, d, f = w.T, w.k, w.E, w.d_model, w.d_ff
+    cu = "cuda"
+    o = {"idx": torch.empty(T, k, dtype=torch.int32, device=cu),
+         "gate": torch.empty(T, k, device=cu),
+         "counts": torch.empty(E, dtype=torch.int32, device=cu),
+         "offsets": torch.empty(E + 1, dtype=torch.int32, device=cu),
+         "perm_src": torch.empty(T * k, dtype=torch.int32, device=cu),
+         "slot_pos": torch.empty(T * k, dtype=torch.int32, device=cu),
+         "x_perm": torch.empty(T * k, d, dtype=torch.bfloat16, device=cu),
+         "h": torch.empty(T * k, f, dtype=torch.bfloat16, device=cu),
+         "y_perm": torch.empty(T * k, d, device=cu), "y": torch.empty(T, d, device=cu)}
+    ws = moe.workspace(cfg)
+    moe.moe_route(cfg, dev["x"], dev["w_gate"], o["idx"], o["gate"], ws,
+                  logit_bias=dev.get("logit_bias"))
+    moe.moe_permute(cfg, o["idx"], dev["x"], o["counts"], o["offsets"], o["perm_src"],
+                    o["slot_pos"], o["x_perm"], ws)
+    moe.moe_expert_ffn(cfg, o["x_perm"], o["offsets"], dev["w1"], dev["w2"], o["h"], o["y_perm"], ws)
+    moe.moe_combine(cfg, o["y_perm"], o["slot_pos"], o["gate"], o["y"], ws)
+    ys = []
+    for _ in range(2):
+        yf = torch.full((T, d), float("nan"), device=cu)
+        moe.moe_expert_ffn_combine(cfg, o["x_perm"], o["offsets"], o["perm_src"], o["slot_pos"],
+                                   o["gate"], dev["w1"], dev["w2"], o["h"], yf, ws)
+        assert moe.last_launch_count() == 2
+        ys.append(yf)
+    torch.cuda.synchronize()
+    assert moe.moe_get_error(ws) == 0
+    assert torch.equal(ys[0], ys[1])
+    yf, yc = ys[0].double(), o["y"].double()
+    assert bool(torch.isfinite(yf).all())
+    sp = o["slot_pos"].long().view(T, k)
+    kept = (sp >= 0)
+    none_kept = ~kept.any(1)
+    if w.capacity_factor is not None:
+        assert bool(none_kept.any()) and bool((kept.sum(1) == 1).any())
+    assert bool((yf[none_kept] == 0).all())
+    yp = o["y_perm"].double()[sp.clamp(min=0)]
+    mag = (o["gate"].double().abs().view(T, k, 1) * yp.abs() * kept.double().unsqueeze(-1)).sum(1)
+    assert bool(((yf - yc).abs() <= 2.0 ** -22 * mag).all()), float((yf - yc).abs().max())
+
+
 def test_forward_replays_from_a_cuda_graph():
     """moe_forward captured into a CUDA graph (its kernels and their programmatic launch
     edges) and replayed gives the eager result bit for bit, also after the input changes
