@@ -444,8 +444,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if constexpr (PAIR) mbar_arrive_cluster(tempty_peer0 + 8 * acc);
-        else mbar_arrive(tempty0 + 8 * acc);
+        // relaxed: the accumulator's TMEM reads are complete (tcgen05.wait::ld) and the
+        // MMA thread reads none of this warp's global stores
+        if constexpr (PAIR) mbar_arrive_cluster_relaxed(tempty_peer0 + 8 * acc);
+        else mbar_arrive_relaxed(tempty0 + 8 * acc);
       }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;

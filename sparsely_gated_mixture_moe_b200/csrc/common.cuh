@@ -276,6 +276,18 @@ __device__ __forceinline__ void cluster_sync_all() {
 }
 
 // Arrive on an mbarrier given by its shared::cluster address (possibly the peer CTA's).
+// Arrivals that order nothing before them (relaxed), for a barrier whose waiter needs only
+// the arrival: an accumulator handed back to the MMA thread after tcgen05.wait::ld (the
+// TMEM reads have completed; nothing the waiter does reads the epilogue's global
+// stores).  A release arrival would hold the warp until its earlier global stores are
+// performed.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint32_t bar) {
+  asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+               : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
                : "memory");
